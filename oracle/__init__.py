@@ -1,0 +1,252 @@
+"""The oracle: a plain fp64 CPU implementation of the quantized-state decode path.
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg
+of ``bench.py`` may import this package. The product library
+(``quantized_linear_attention_stq_b200``) never imports, loads or calls it, and the two share
+no code: the arithmetic lives in ``stq_oracle.c`` (plain C99, fp64, no FMA contraction); this
+module only builds that file with gcc and marshals numpy arrays through ctypes.
+
+Every function follows the pages it cites in ``stq_oracle.c``:
+  "K1 論文詳解" (k1-news.pages.dev/paper/2026-10-09), sections 方法 / 實驗結果, and
+  "线性注意力状态量化难题" (aitest123.com/news/n1kj09), sections 直接量化为什么会翻车 / 时间维度 /
+  空间维度 / 工程落地.
+Parity of the accuracy claims (perplexity, benchmark scores, generation lengths) is unpinned:
+those need the models and evaluation suites, which this library does not have.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "stq_oracle.c")
+_HDR = os.path.join(_HERE, "stq_oracle.h")
+_OUT_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_OUT_DIR, "libstq_oracle.so")
+
+OK, EINVAL, ENONFINITE = 0, 1, 4
+GATE_SCALAR, GATE_CHANNEL, GATE_CHANNEL_DECAY_FIRST = 0, 1, 2
+TIE_DELTA = 1e-3
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``stq_oracle.c`` into ``_build/libstq_oracle.so`` (gcc, -O2, no FMA contraction)."""
+    os.makedirs(_OUT_DIR, exist_ok=True)
+    stale = (not os.path.exists(_LIB_PATH)
+             or os.path.getmtime(_LIB_PATH) < max(os.path.getmtime(_SRC), os.path.getmtime(_HDR)))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-std=c99", "-O2", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+               "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = build()
+            L = ctypes.CDLL(path)
+            P = ctypes.c_void_p
+            i32, f64, sz = ctypes.c_int, ctypes.c_double, ctypes.c_size_t
+            L.orc_qmax.argtypes, L.orc_qmax.restype = [i32], i32
+            L.orc_round_half_even.argtypes, L.orc_round_half_even.restype = [f64], f64
+            for name in ("orc_codes_bytes", "orc_scale_offset", "orc_block_bytes"):
+                getattr(L, name).argtypes = [i32, i32, i32]
+                getattr(L, name).restype = sz
+            L.orc_pack.argtypes, L.orc_pack.restype = [i32, sz, P, P], None
+            L.orc_unpack.argtypes, L.orc_unpack.restype = [i32, sz, P, P], None
+            L.orc_half_to_double.argtypes, L.orc_half_to_double.restype = [ctypes.c_uint16], f64
+            L.orc_double_to_half.argtypes, L.orc_double_to_half.restype = [f64], ctypes.c_uint16
+            L.orc_quantize.argtypes = [i32, i32, i32, P, P, P, P, P, f64]
+            L.orc_quantize.restype = i32
+            L.orc_dequantize.argtypes, L.orc_dequantize.restype = [i32, i32, i32, P, P], i32
+            L.orc_update.argtypes = [i32, i32, i32, P, P, P, P, f64, P, P]
+            L.orc_update.restype = None
+            L.orc_decode_step.argtypes = [i32, i32, i32, i32, P, P, P, P, f64, P, P, P, P, P, P, f64]
+            L.orc_decode_step.restype = i32
+            L.orc_prefill_seq.argtypes = [i32, i32, i32, i32, P, i32, i32, P, P, P, P, P, P, P, P, P, f64]
+            L.orc_prefill_seq.restype = i32
+            L.orc_chunk_wy.argtypes = [i32, i32, i32, P, P, P, P, P, P, P, P]
+            L.orc_chunk_wy.restype = i32
+            _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+# ----------------------------------------------------------------------------------------------
+# Elementary pieces
+# ----------------------------------------------------------------------------------------------
+
+def qmax(bits: int) -> int:
+    return lib().orc_qmax(bits)
+
+
+def round_half_even(y: float) -> float:
+    return lib().orc_round_half_even(float(y))
+
+
+def codes_bytes(bits: int, dk: int, dv: int) -> int:
+    return lib().orc_codes_bytes(bits, dk, dv)
+
+
+def scale_offset(bits: int, dk: int, dv: int) -> int:
+    return lib().orc_scale_offset(bits, dk, dv)
+
+
+def block_bytes(bits: int, dk: int, dv: int) -> int:
+    return lib().orc_block_bytes(bits, dk, dv)
+
+
+def pack(bits: int, u) -> np.ndarray:
+    u = np.ascontiguousarray(np.asarray(u, dtype=np.int32).ravel())
+    out = np.zeros((bits * u.size + 7) // 8, dtype=np.uint8)
+    lib().orc_pack(bits, u.size, _p(u), _p(out))
+    return out
+
+
+def unpack(bits: int, n: int, data) -> np.ndarray:
+    data = np.ascontiguousarray(np.asarray(data, dtype=np.uint8))
+    assert data.size * 8 >= bits * n
+    u = np.zeros(n, dtype=np.int32)
+    lib().orc_unpack(bits, n, _p(data), _p(u))
+    return u
+
+
+def half_to_double(h: int) -> float:
+    return lib().orc_half_to_double(int(h))
+
+
+def double_to_half(x: float) -> int:
+    return lib().orc_double_to_half(float(x))
+
+
+# ----------------------------------------------------------------------------------------------
+# One head block
+# ----------------------------------------------------------------------------------------------
+
+def quantize(bits: int, S, w=None, delta: float = TIE_DELTA):
+    """Quantize an fp64 state into a fresh head block. Returns (block, x, tie, status)."""
+    S = _f64(S)
+    dk, dv = S.shape
+    w = _f64(np.ones(dk) if w is None else w)
+    block = np.zeros(block_bytes(bits, dk, dv), dtype=np.uint8)
+    x = np.zeros((dk, dv))
+    tie = np.zeros((dk, dv), dtype=np.uint8)
+    st = lib().orc_quantize(bits, dk, dv, _p(S), _p(w), _p(block), _p(x), _p(tie), float(delta))
+    return block, x, tie.astype(bool), st
+
+
+def dequantize(bits: int, dk: int, dv: int, block) -> np.ndarray:
+    block = np.ascontiguousarray(np.asarray(block, dtype=np.uint8))
+    assert block.size >= block_bytes(bits, dk, dv)
+    S = np.zeros((dk, dv))
+    st = lib().orc_dequantize(bits, dk, dv, _p(block), _p(S))
+    assert st == OK
+    return S
+
+
+def codes(bits: int, dk: int, dv: int, block) -> np.ndarray:
+    """Signed integer codes Q (dk x dv) of a quantized head block."""
+    u = unpack(bits, dk * dv, np.asarray(block, dtype=np.uint8)[: codes_bytes(bits, dk, dv)])
+    return (u - (1 << (bits - 1))).reshape(dk, dv)
+
+
+def scales(bits: int, dk: int, dv: int, block):
+    """(r, c) fp32 scales of a quantized head block."""
+    off = scale_offset(bits, dk, dv)
+    raw = np.asarray(block, dtype=np.uint8)
+    r = raw[off: off + 4 * dk].view(np.float32).copy()
+    c = raw[off + 4 * dk: off + 4 * dk + 4 * dv].view(np.float32).copy()
+    return r, c
+
+
+def pivot_values(dk: int, dv: int, block) -> np.ndarray:
+    return np.asarray(block, dtype=np.uint8)[: 2 * dk * dv].view(np.uint16).reshape(dk, dv).copy()
+
+
+def update(gate: int, S, q, k, v, beta: float, alpha):
+    """Unquantized fp64 gated-delta-rule update (returns S', o); no rounding of any kind."""
+    S = _f64(S).copy()
+    dk, dv = S.shape
+    o = np.zeros(dv)
+    a = _f64(np.atleast_1d(alpha))
+    lib().orc_update(dk, dv, gate, _p(S), _p(_f64(q)), _p(_f64(k)), _p(_f64(v)), float(beta), _p(a), _p(o))
+    return S, o
+
+
+def decode_step(bits: int, gate: int, block, q, k, v, beta: float, alpha, w,
+                dk: int, dv: int, delta: float = TIE_DELTA):
+    """One decode step on a copy of ``block``.
+
+    Returns dict(block, o (fp32), S_new (fp64, before requantization), x, tie, status)."""
+    blk = np.ascontiguousarray(np.asarray(block, dtype=np.uint8)).copy()
+    o = np.zeros(dv, dtype=np.float32)
+    S_new = np.zeros((dk, dv))
+    x = np.zeros((dk, dv))
+    tie = np.zeros((dk, dv), dtype=np.uint8)
+    a = _f64(np.atleast_1d(alpha))
+    wv = _f64(np.ones(dk) if w is None else w)
+    st = lib().orc_decode_step(bits, dk, dv, gate, _p(blk), _p(_f64(q)), _p(_f64(k)), _p(_f64(v)),
+                               float(beta), _p(a), _p(wv), _p(o), _p(S_new), _p(x), _p(tie),
+                               float(delta))
+    return dict(block=blk, o=o, S_new=S_new, x=x, tie=tie.astype(bool), status=st)
+
+
+def prefill_seq(bits: int, gate: int, block, q, k, v, beta, alpha, w, chunk: int,
+                dk: int, dv: int, delta: float = TIE_DELTA):
+    """Sequential chunked prefill on a copy of ``block`` (q,k: [T][dk], v: [T][dv])."""
+    blk = np.ascontiguousarray(np.asarray(block, dtype=np.uint8)).copy()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T = q.shape[0]
+    o = np.zeros((T, dv), dtype=np.float32)
+    x = np.zeros((dk, dv))
+    tie = np.zeros((dk, dv), dtype=np.uint8)
+    st = lib().orc_prefill_seq(bits, dk, dv, gate, _p(blk), T, chunk, _p(q), _p(k), _p(v),
+                               _p(_f64(beta)), _p(_f64(alpha)), _p(_f64(w)), _p(o), _p(x), _p(tie),
+                               float(delta))
+    return dict(block=blk, o=o, x=x, tie=tie.astype(bool), status=st)
+
+
+def chunk_wy(S0, q, k, v, beta, alpha):
+    """fp64 WY/UT evaluation of one chunk (scalar gate, no quantization) -> (S_end, O)."""
+    S0 = _f64(S0)
+    dk, dv = S0.shape
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    C = q.shape[0]
+    S_end = np.zeros((dk, dv))
+    O = np.zeros((C, dv))
+    st = lib().orc_chunk_wy(dk, dv, C, _p(S0), _p(q), _p(k), _p(v), _p(_f64(beta)), _p(_f64(alpha)),
+                            _p(S_end), _p(O))
+    assert st == OK
+    return S_end, O
+
+
+# ----------------------------------------------------------------------------------------------
+# Request blocks (a request's head blocks back to back, padded to 128 bytes)
+# ----------------------------------------------------------------------------------------------
+
+def request_layout(head_bits, dk: int, dv: int):
+    """Per-head byte offsets inside one request block, and the request block size."""
+    offs, pos = [], 0
+    for b in head_bits:
+        offs.append(pos)
+        pos += block_bytes(int(b), dk, dv)
+    total = (pos + 127) // 128 * 128
+    return np.array(offs, dtype=np.int64), total

@@ -1,0 +1,534 @@
+"""Pins of the oracle against facts fixed outside the oracle itself (CPU only).
+
+Each group checks the oracle against one of: a hand derivation from a layout or format
+definition, a library routine that implements the same special case (numpy's LSB-first bit
+packing, numpy's IEEE float16 conversion, numpy's round-half-to-even ``rint``, a numpy matrix
+product), a closed form, an invariant, or brute force on tiny heads. The groups are chosen so
+that a dropped term, a wrong sign, a wrong index or a transposed operand anywhere in the oracle
+fails at least one of them.
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+BITS = (4, 6, 8)
+
+
+# ----------------------------------------------------------------------------------------------
+# Packing: code (i,j) at bit offset b*(i*dv+j) of a little-endian bitstream, offset-binary
+# ----------------------------------------------------------------------------------------------
+
+def test_pack_hand_derived_bytes(orc):
+    # 4-bit: two codes per byte, the first in the low nibble.
+    assert list(orc.pack(4, [1, 2, 3, 4, 15, 0, 10, 5])) == [0x21, 0x43, 0x0F, 0x5A]
+    # 6-bit: four codes fill three bytes; 1 + 2*64 + 3*4096 + 4*262144 = 0x103081.
+    assert list(orc.pack(6, [1, 2, 3, 4])) == [0x81, 0x30, 0x10]
+    # 63 + 63*4096 = 0x03F03F.
+    assert list(orc.pack(6, [63, 0, 63, 0])) == [0x3F, 0xF0, 0x03]
+    # 8-bit: one code per byte.
+    assert list(orc.pack(8, [1, 255, 128])) == [0x01, 0xFF, 0x80]
+    # A 6-bit code straddling a byte boundary: code 1 occupies bits 6..11.
+    assert list(orc.pack(6, [0, 63])) == [0xC0, 0x0F]
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("n", [16, 256, 300])
+def test_pack_matches_numpy_lsb_first_bitstream(orc, bits, n):
+    rng = np.random.default_rng(bits * 1000 + n)
+    u = rng.integers(0, 1 << bits, size=n)
+    # Expand every code into its bits, least significant first, and let numpy pack them.
+    stream = ((u[:, None] >> np.arange(bits)[None, :]) & 1).astype(np.uint8).ravel()
+    ref = np.packbits(stream, bitorder="little")
+    assert np.array_equal(orc.pack(bits, u), ref)
+    assert np.array_equal(orc.unpack(bits, n, ref), u)
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("d", [4, 16])
+def test_pack_every_value_every_position(orc, bits, d):
+    n = d * d
+    rng = np.random.default_rng(7 + bits + d)
+    base = rng.integers(0, 1 << bits, size=n)
+    packed_base = orc.pack(bits, base)
+    positions = range(n) if d == 4 else rng.choice(n, size=24, replace=False)
+    for p in positions:
+        for val in range(1 << bits):
+            u = base.copy()
+            u[p] = val
+            pk = orc.pack(bits, u)
+            back = orc.unpack(bits, n, pk)
+            assert np.array_equal(back, u)
+            # Only the bits of position p may differ from the base stream.
+            diff = np.unpackbits(pk ^ packed_base, bitorder="little")
+            changed = np.nonzero(diff)[0]
+            assert np.all((changed >= bits * p) & (changed < bits * (p + 1)))
+
+
+def test_block_sizes_from_layout_definition(orc):
+    # codes bytes, padded to 16, + 4*dk + 4*dv scale bytes, padded to 128.
+    assert orc.block_bytes(4, 128, 128) == 8192 + 1024          # 9216
+    assert orc.block_bytes(6, 128, 128) == 12288 + 1024         # 13312
+    assert orc.block_bytes(8, 128, 128) == 16384 + 1024         # 17408
+    assert orc.block_bytes(16, 128, 128) == 32768
+    # 6-bit 16x16: 1536 bits = 192 bytes (16-aligned), + 128 scale bytes = 320 -> 384.
+    assert orc.block_bytes(6, 16, 16) == 384
+    # 4-bit 5x5: 100 bits -> 13 bytes -> 16, + 40 scale bytes = 56 -> 128.
+    assert orc.block_bytes(4, 5, 5) == 128
+
+
+# ----------------------------------------------------------------------------------------------
+# IEEE binary16 (pivot heads)
+# ----------------------------------------------------------------------------------------------
+
+def test_half_decode_all_patterns_match_numpy(orc):
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = pats.view(np.float16).astype(np.float64)
+    got = np.array([orc.half_to_double(int(h)) for h in pats])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def test_half_encode_matches_numpy(orc):
+    rng = np.random.default_rng(3)
+    vals = [0.0, -0.0, 65504.0, 65519.99, 65520.0, 70000.0, 1e-8, 2.0 ** -24, 2.0 ** -25,
+            3 * 2.0 ** -26, 2.0 ** -14, 2.0 ** -14 - 2.0 ** -25, np.inf, -np.inf]
+    # exact ties between neighbouring halves, in the normal and the subnormal range
+    for e in range(-14, 15):
+        for m in (0, 1, 2, 3, 1022, 1023):
+            lo = (1024 + m) * 2.0 ** (e - 10)
+            vals.append(lo + 2.0 ** (e - 11))
+            vals.append(-(lo + 2.0 ** (e - 11)))
+    for m in range(0, 1024, 37):
+        vals.append((m + 0.5) * 2.0 ** -24)
+    vals += list(rng.standard_normal(2000) * 10.0 ** rng.uniform(-8, 5, 2000))
+    for x in vals:
+        ref = int(np.array([x], dtype=np.float64).astype(np.float16).view(np.uint16)[0])
+        assert orc.double_to_half(x) == ref, x
+
+
+def test_round_half_even_matches_numpy_rint(orc):
+    ys = [n + 0.5 for n in range(-300, 300)] + list(np.random.default_rng(1).uniform(-200, 200, 3000))
+    ys += [0.49999999999999994, -0.49999999999999994, 2.5000000000000004]
+    for y in ys:
+        assert orc.round_half_even(y) == np.rint(y), y
+
+
+# ----------------------------------------------------------------------------------------------
+# Quantizer
+# ----------------------------------------------------------------------------------------------
+
+TIE_CASES = {
+    # circulant base rows whose squares sum to 5 * 4^-e, each containing +-qmax once:
+    # 49+20.25+6.25+2.25+2.25 = 80; 961+306.25+12.25+.25+.25 = 1280; 16129+4290.25+56.25+2.25+2.25 = 20480
+    4: ([7, 4.5, 2.5, 1.5, 1.5], -2),
+    6: ([31, 17.5, 3.5, 0.5, 0.5], -4),
+    8: ([127, 65.5, 7.5, 1.5, 1.5], -6),
+}
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_quantizer_exact_planted_ties(orc, bits):
+    """S = 2^e X diag(C) with X a signed circulant of half-integers: every fitted scale and
+    every real code is exact, so each half-integer is an exact rounding tie."""
+    g, e = TIE_CASES[bits]
+    d = 5
+    X = np.array([[g[(i - j) % d] for j in range(d)] for i in range(d)], dtype=np.float64)
+    X *= np.where(np.random.default_rng(bits).random((d, d)) < 0.5, -1.0, 1.0)
+    C = np.array([1.0, 0.75, 3.0, 0.125, 1.5])
+    S = X * C[None, :] * 2.0 ** e
+    for w in (np.full(d, 3.0), np.full(d, 0.25)):
+        block, x, tie, st = orc.quantize(bits, S, w)
+        assert st == orc.OK
+        r, c = orc.scales(bits, d, d, block)
+        assert np.array_equal(x, X)
+        assert np.array_equal(r, np.full(d, 2.0 ** e, dtype=np.float32))
+        assert np.array_equal(c, C.astype(np.float32))
+        Q = orc.codes(bits, d, d, block)
+        assert np.array_equal(Q, np.rint(X).astype(int))  # numpy rint rounds half to even
+        assert np.array_equal(tie, X != np.round(X + 0.25))  # ties exactly at the half-integers
+        assert tie.sum() == 20
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("d", [16, 128])
+def test_quantizer_sign_pattern_gives_full_scale(orc, bits, d):
+    """S = diag(a) Sigma diag(b), Sigma in {+-1}: every code is +-qmax with Sigma's sign."""
+    rng = np.random.default_rng(d + bits)
+    a = np.exp(rng.normal(0, 0.8, d))
+    b = np.exp(rng.normal(0, 0.8, d))
+    sig = np.where(rng.random((d, d)) < 0.5, -1.0, 1.0)
+    w = np.exp(rng.normal(0, 1, d))
+    block, x, tie, st = orc.quantize(bits, a[:, None] * sig * b[None, :], w)
+    assert st == orc.OK
+    Q = orc.codes(bits, d, d, block)
+    assert np.array_equal(Q, orc.qmax(bits) * sig.astype(int))
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("d", [4, 16, 128])
+def test_quantizer_integer_circulant_round_trip(orc, bits, d):
+    """S = rho * circ(g) * diag(c) with integer g, max|g| = qmax and equal w: codes are g exactly
+    and dequantization reproduces S to a few fp32 ulps."""
+    rng = np.random.default_rng(100 + d + bits)
+    qm = orc.qmax(bits)
+    g = rng.integers(-qm, qm + 1, size=d)
+    g[rng.integers(d)] = qm * (1 if rng.random() < 0.5 else -1)
+    G = np.array([[g[(j - i) % d] for j in range(d)] for i in range(d)])
+    cvec = np.exp(rng.normal(0, 1.0, d))
+    rho = 0.37
+    S = rho * G * cvec[None, :]
+    block, x, tie, st = orc.quantize(bits, S, np.full(d, 2.5))
+    assert st == orc.OK
+    assert np.array_equal(orc.codes(bits, d, d, block), G)
+    Sd = orc.dequantize(bits, d, d, block)
+    nz = S != 0
+    assert np.max(np.abs(Sd[nz] - S[nz]) / np.abs(S[nz])) < 4 * 2.0 ** -23
+
+
+def _outlier_state(rng, d, row_ratio=10.3, col_ratio=19.4):
+    a = np.exp(rng.normal(0, 0.8, d))
+    b = np.exp(rng.normal(0, 0.8, d))
+    a[np.argmax(a)] = row_ratio * np.median(a)
+    b[np.argmax(b)] = col_ratio * np.median(b)
+    return a[:, None] * rng.standard_normal((d, d)) * b[None, :]
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_quantizer_closed_form_bounds(orc, bits):
+    rng = np.random.default_rng(bits)
+    dk, dv = 128, 96
+    S = _outlier_state(rng, 128)[:, :dv]
+    w = np.exp(rng.normal(0, 1, dk))
+    block, x, tie, st = orc.quantize(bits, S, w)
+    assert st == orc.OK
+    Q = orc.codes(bits, dk, dv, block)
+    r, c = orc.scales(bits, dk, dv, block)
+    step = r.astype(np.float64)[:, None] * c.astype(np.float64)[None, :]
+    # reconstruction error at most half a step (plus fp64 slack)
+    assert np.all(np.abs(S - step * Q) <= 0.5 * step * (1 + 1e-9))
+    # every row reaches full scale
+    assert np.all(np.abs(Q).max(axis=1) == orc.qmax(bits))
+    # the column scale is the impact-weighted RMS: c_j^2 * sum(w) == sum_i w_i S_ij^2
+    lhs = c.astype(np.float64) ** 2 * w.sum()
+    rhs = (w[:, None] * S ** 2).sum(axis=0)
+    assert np.max(np.abs(lhs - rhs) / rhs) < 2.5e-7
+    # the row scale is the largest column-normalised magnitude over qmax
+    t = np.abs(S / c.astype(np.float64)[None, :]).max(axis=1) / orc.qmax(bits)
+    assert np.max(np.abs(r - t) / t) < 1e-7
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_quantizer_weight_roles(orc, bits):
+    """Weight concentrated on one key row: the column scale becomes that row's magnitude (catches
+    a row/column index swap or a missing square); scaling all weights by 4 changes nothing."""
+    rng = np.random.default_rng(11)
+    dk, dv = 12, 20
+    S = rng.standard_normal((dk, dv))
+    m = 5
+    w = np.full(dk, 1e-12)
+    w[m] = 1.0
+    block, _, _, st = orc.quantize(bits, S, w)
+    _, c = orc.scales(bits, dk, dv, block)
+    assert np.allclose(c, np.abs(S[m]), rtol=1e-5)
+    w2 = np.exp(rng.normal(0, 1, dk))
+    b1, _, _, _ = orc.quantize(bits, S, w2)
+    b2, _, _, _ = orc.quantize(bits, S, 4.0 * w2)
+    assert np.array_equal(b1, b2)
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_quantizer_zero_rows_and_columns(orc, bits):
+    rng = np.random.default_rng(5)
+    S = rng.standard_normal((8, 8))
+    S[3, :] = 0.0
+    S[:, 6] = 0.0
+    block, _, _, st = orc.quantize(bits, S, np.ones(8))
+    assert st == orc.OK
+    r, c = orc.scales(bits, 8, 8, block)
+    Q = orc.codes(bits, 8, 8, block)
+    assert r[3] == 1.0 and c[6] == 1.0
+    assert np.all(Q[3] == 0) and np.all(Q[:, 6] == 0)
+    blk0, _, _, st0 = orc.quantize(bits, np.zeros((4, 4)), np.ones(4))
+    assert st0 == orc.OK and np.all(orc.codes(bits, 4, 4, blk0) == 0)
+    assert np.all(np.concatenate(orc.scales(bits, 4, 4, blk0)) == 1.0)
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_quantizer_brute_force_4x4(orc, bits):
+    """On 4x4 heads every code is the argmin over all integers in [-qmax, qmax] of the distance
+    to the real code, ties to the even integer."""
+    qm = orc.qmax(bits)
+    cands = np.arange(-qm, qm + 1)
+    rng = np.random.default_rng(bits + 40)
+    for trial in range(200):
+        S = rng.standard_normal((4, 4)) * np.exp(rng.normal(0, 1, (4, 1)))
+        block, x, tie, st = orc.quantize(bits, S, np.exp(rng.normal(0, 1, 4)))
+        Q = orc.codes(bits, 4, 4, block)
+        for i, j in itertools.product(range(4), range(4)):
+            dist = np.abs(x[i, j] - cands)
+            best = cands[dist == dist.min()]
+            want = best[0] if best.size == 1 else best[best % 2 == 0][0]
+            assert Q[i, j] == want
+
+
+def test_quantizer_pivot_is_numpy_float16(orc):
+    rng = np.random.default_rng(9)
+    S = rng.standard_normal((16, 24)) * 300.0
+    block, _, _, st = orc.quantize(16, S)
+    assert st == orc.OK
+    assert np.array_equal(orc.pivot_values(16, 24, block), S.astype(np.float16).view(np.uint16))
+    S[2, 3] = 1e6  # overflows fp16
+    _, _, _, st = orc.quantize(16, S)
+    assert st == orc.ENONFINITE
+
+
+def test_quantizer_rejects_bad_weights(orc):
+    S = np.ones((4, 4))
+    for w in ([1, 1, 0, 1], [1, -1, 1, 1], [1, np.nan, 1, 1], [np.inf, 1, 1, 1]):
+        assert orc.quantize(6, S, np.array(w, dtype=float))[3] == orc.EINVAL
+
+
+# ----------------------------------------------------------------------------------------------
+# Decode step: gated delta rule update and readout
+# ----------------------------------------------------------------------------------------------
+
+def _random_block(orc, bits, dk, dv, seed):
+    rng = np.random.default_rng(seed)
+    S = rng.standard_normal((dk, dv)) * np.exp(rng.normal(0, 0.8, (dk, 1)))
+    w = np.exp(rng.normal(0, 1, dk))
+    block, _, _, st = orc.quantize(bits, S, w)
+    assert st == orc.OK
+    return block, w
+
+
+@pytest.mark.parametrize("bits", BITS + (16,))
+@pytest.mark.parametrize("shape", [(16, 16), (8, 12)])
+@pytest.mark.parametrize("gate", [0, 1, 2])
+def test_unit_key_write(orc, bits, shape, gate):
+    """alpha=1, beta=1, k = e_m: row m of the updated state is v exactly, the other rows are the
+    dequantized state exactly, and a query q = e_m reads back v."""
+    dk, dv = shape
+    block, w = _random_block(orc, bits, dk, dv, 1)
+    S = orc.dequantize(bits, dk, dv, block)
+    rng = np.random.default_rng(2)
+    v = rng.standard_normal(dv)
+    m = 3
+    k = np.zeros(dk)
+    k[m] = 1.0
+    alpha = 1.0 if gate == 0 else np.ones(dk)
+    res = orc.decode_step(bits, gate, block, k, k, v, 1.0, alpha, w, dk, dv)
+    Sn = res["S_new"]
+    assert np.array_equal(Sn[m], v)
+    others = np.arange(dk) != m
+    assert np.array_equal(Sn[others], S[others])
+    assert np.array_equal(res["o"], v.astype(np.float32))
+
+
+@pytest.mark.parametrize("bits", (4, 8))
+def test_unit_key_write_general_direction(orc, bits):
+    """For any unit k with alpha=1, beta=1: S'^T k = v."""
+    dk = dv = 32
+    block, w = _random_block(orc, bits, dk, dv, 3)
+    rng = np.random.default_rng(4)
+    k = rng.standard_normal(dk)
+    k /= np.linalg.norm(k)
+    v = rng.standard_normal(dv)
+    res = orc.decode_step(bits, 0, block, k, k, v, 1.0, 1.0, w, dk, dv)
+    assert np.allclose(res["S_new"].T @ k, v, atol=1e-12, rtol=0)
+    assert np.allclose(res["o"], v, atol=1e-6, rtol=1e-6)
+
+
+@pytest.mark.parametrize("gate", [0, 1, 2])
+def test_beta_zero_is_pure_decay(orc, gate):
+    dk, dv = 16, 24
+    block, w = _random_block(orc, 6, dk, dv, 5)
+    S = orc.dequantize(6, dk, dv, block)
+    rng = np.random.default_rng(6)
+    q, k, v = rng.standard_normal(dk), rng.standard_normal(dk), rng.standard_normal(dv)
+    alpha = 0.9 if gate == 0 else np.exp(-1.0 / rng.uniform(1, 100, dk))
+    res = orc.decode_step(6, gate, block, q, k, v, 0.0, alpha, w, dk, dv)
+    a = np.atleast_1d(alpha)[:, None] if gate else alpha
+    assert np.array_equal(res["S_new"], a * S)
+
+
+def test_readout_is_transposed_state_times_query(orc):
+    """alpha=1, beta=0: o = deq(S)^T q, checked against numpy's matrix product, d_k != d_v."""
+    dk, dv = 24, 40
+    block, w = _random_block(orc, 8, dk, dv, 7)
+    S = orc.dequantize(8, dk, dv, block)
+    rng = np.random.default_rng(8)
+    q, k, v = rng.standard_normal(dk), rng.standard_normal(dk), rng.standard_normal(dv)
+    res = orc.decode_step(8, 0, block, q, k, v, 0.0, 1.0, w, dk, dv)
+    ref = (S.T @ q).astype(np.float32)
+    assert np.allclose(res["o"], ref, rtol=1e-6, atol=1e-6 * np.abs(ref).max())
+
+
+def test_update_is_non_expansive_plus_write(orc):
+    rng = np.random.default_rng(10)
+    dk = dv = 32
+    for t in range(50):
+        S = rng.standard_normal((dk, dv))
+        k = rng.standard_normal(dk)
+        k /= np.linalg.norm(k)
+        v = rng.standard_normal(dv)
+        beta, alpha = rng.uniform(0, 1), rng.uniform(0.2, 1)
+        Sn, _ = orc.update(0, S, k, k, v, beta, alpha)
+        assert np.linalg.norm(Sn) <= np.linalg.norm(S) + beta * np.linalg.norm(v) + 1e-12
+
+
+@pytest.mark.parametrize("bits", (4, 16))
+def test_channel_gate_with_equal_entries_is_scalar_gate(orc, bits):
+    dk, dv = 16, 16
+    block, w = _random_block(orc, bits, dk, dv, 12)
+    rng = np.random.default_rng(13)
+    q, k, v = rng.standard_normal(dk), rng.standard_normal(dk), rng.standard_normal(dv)
+    a = 0.875
+    r0 = orc.decode_step(bits, 0, block, q, k, v, 0.6, a, w, dk, dv)
+    r1 = orc.decode_step(bits, 1, block, q, k, v, 0.6, np.full(dk, a), w, dk, dv)
+    assert np.array_equal(r0["S_new"], r1["S_new"])
+    assert np.array_equal(r0["block"], r1["block"])
+    # decay-first with equal entries: alpha*(S - beta k u) == alpha S - beta k (alpha u)
+    r2 = orc.decode_step(bits, 2, block, q, k, v, 0.6, np.full(dk, a), w, dk, dv)
+    assert np.allclose(r2["S_new"], r0["S_new"], rtol=1e-13, atol=1e-13)
+
+
+def test_channel_gate_orders_differ_in_general(orc):
+    dk = dv = 16
+    block, w = _random_block(orc, 6, dk, dv, 14)
+    rng = np.random.default_rng(15)
+    q, k, v = rng.standard_normal(dk), rng.standard_normal(dk), rng.standard_normal(dv)
+    alpha = np.exp(-1.0 / rng.uniform(1, 50, dk))
+    r1 = orc.decode_step(6, 1, block, q, k, v, 0.7, alpha, w, dk, dv)
+    r2 = orc.decode_step(6, 2, block, q, k, v, 0.7, alpha, w, dk, dv)
+    assert not np.allclose(r1["S_new"], r2["S_new"])
+
+
+def test_fp16_pivot_tracks_unquantized_recurrence(orc):
+    """A pivot head (fp16 storage) follows the unquantized fp64 recurrence over 64 steps of the
+    d=16 test workload (h = 256): every single step stores each element within half an fp16
+    quantum of the exact update of the stored state, and over the trajectory the relative error
+    is at most 1e-3 (RMS over the 64 readouts, and mean of the per-step state errors; the
+    per-step drift is a random walk of fp16 roundings and reaches ~1.2e-3 at single steps)."""
+    rng = np.random.default_rng(0)
+    d = 16
+    a = np.exp(rng.normal(0, 0.8, d))
+    b = np.exp(rng.normal(0, 0.8, d))
+    S0 = a[:, None] * rng.standard_normal((d, d)) * b[None, :]
+    w = np.exp(rng.normal(0, 1, d))
+    alpha = np.exp(-1.0 / 256)
+    block, _, _, _ = orc.quantize(16, S0)
+    Sref = orc.dequantize(16, d, d, block)
+    O, Oref, s_err = [], [], []
+    for t in range(64):
+        q = rng.standard_normal(d)
+        q /= np.linalg.norm(q)
+        k = rng.standard_normal(d)
+        k /= np.linalg.norm(k)
+        v = rng.standard_normal(d)
+        beta = 1.0 / (1.0 + np.exp(-rng.standard_normal()))
+        Sprev = orc.dequantize(16, d, d, block)
+        res = orc.decode_step(16, 0, block, q, k, v, beta, alpha, w, d, d)
+        block = res["block"]
+        Sd = orc.dequantize(16, d, d, block)
+        # single step: exact update of the stored state, then one fp16 rounding
+        exact = alpha * (Sprev - beta * np.outer(k, k @ Sprev)) + beta * np.outer(k, v)
+        quantum = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(exact), 2.0 ** -14))) - 10)
+        assert np.all(np.abs(Sd - exact) <= 0.5 * quantum * (1 + 1e-9))
+        Sref = alpha * (Sref - beta * np.outer(k, k @ Sref)) + beta * np.outer(k, v)
+        O.append(res["o"])
+        Oref.append(Sref.T @ q)
+        s_err.append(np.linalg.norm(Sd - Sref) / np.linalg.norm(Sref))
+    O, Oref = np.array(O, dtype=np.float64), np.array(Oref)
+    assert np.linalg.norm(O - Oref) <= 1e-3 * np.linalg.norm(Oref)
+    assert np.mean(s_err) <= 1e-3
+    assert np.max(s_err) <= 2e-3
+
+
+def test_decode_flags(orc):
+    block, w = _random_block(orc, 6, 8, 8, 16)
+    z = np.zeros(8)
+    bad = w.copy()
+    bad[0] = 0.0
+    assert orc.decode_step(6, 0, block, z, z, z, 0.5, 0.9, bad, 8, 8)["status"] == orc.EINVAL
+    v = np.full(8, np.inf)
+    assert orc.decode_step(6, 0, block, z, np.ones(8), v, 0.5, 0.9, w, 8, 8)["status"] == orc.ENONFINITE
+
+
+# ----------------------------------------------------------------------------------------------
+# Chunked prefill
+# ----------------------------------------------------------------------------------------------
+
+def _chunk_inputs(rng, C, dk, dv):
+    q = rng.standard_normal((C, dk))
+    k = rng.standard_normal((C, dk))
+    q /= np.linalg.norm(q, axis=1, keepdims=True)
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    v = rng.standard_normal((C, dv))
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal(C)))
+    alpha = np.exp(-1.0 / rng.uniform(1, 400, C))
+    return q, k, v, beta, alpha
+
+
+@pytest.mark.parametrize("C,dk,dv", [(1, 16, 16), (7, 16, 16), (64, 16, 24), (64, 64, 64)])
+def test_wy_form_matches_token_recurrence(orc, C, dk, dv):
+    rng = np.random.default_rng(C + dk)
+    S0 = rng.standard_normal((dk, dv))
+    q, k, v, beta, alpha = _chunk_inputs(rng, C, dk, dv)
+    S_end, O = orc.chunk_wy(S0, q, k, v, beta, alpha)
+    S = S0.copy()
+    Oseq = np.zeros((C, dv))
+    for t in range(C):
+        S, Oseq[t] = orc.update(0, S, q[t], k[t], v[t], beta[t], alpha[t])
+    assert np.max(np.abs(S_end - S)) <= 1e-10 * np.max(np.abs(S))
+    assert np.max(np.abs(O - Oseq)) <= 1e-10 * np.max(np.abs(Oseq))
+
+
+def test_wy_pure_decay(orc):
+    rng = np.random.default_rng(21)
+    C, d = 64, 16
+    S0 = rng.standard_normal((d, d))
+    q, k, v, _, _ = _chunk_inputs(rng, C, d, d)
+    a = 0.97
+    S_end, _ = orc.chunk_wy(S0, q, k, v, np.zeros(C), np.full(C, a))
+    assert np.allclose(S_end, a ** C * S0, rtol=1e-12, atol=0)
+
+
+@pytest.mark.parametrize("bits", BITS + (16,))
+def test_prefill_chunk_of_one_is_decode(orc, bits):
+    dk, dv, T = 16, 16, 9
+    block, w = _random_block(orc, bits, dk, dv, 22)
+    rng = np.random.default_rng(23)
+    q, k, v, beta, alpha = _chunk_inputs(rng, T, dk, dv)
+    res = orc.prefill_seq(bits, 0, block, q, k, v, beta, alpha, w, 1, dk, dv)
+    blk = block.copy()
+    for t in range(T):
+        r = orc.decode_step(bits, 0, blk, q[t], k[t], v[t], beta[t], alpha[t], w, dk, dv)
+        blk = r["block"]
+        assert np.array_equal(res["o"][t], r["o"])
+    assert np.array_equal(res["block"], blk)
+
+
+def test_prefill_multi_chunk_equals_single_chunk_calls(orc):
+    dk, dv, T, C = 16, 16, 150, 64
+    block, w = _random_block(orc, 6, dk, dv, 24)
+    rng = np.random.default_rng(25)
+    q, k, v, beta, alpha = _chunk_inputs(rng, T, dk, dv)
+    full = orc.prefill_seq(6, 0, block, q, k, v, beta, alpha, w, C, dk, dv)
+    blk = block.copy()
+    outs = []
+    for c0 in range(0, T, C):
+        sl = slice(c0, min(c0 + C, T))
+        r = orc.prefill_seq(6, 0, blk, q[sl], k[sl], v[sl], beta[sl], alpha[sl], w, C, dk, dv)
+        blk = r["block"]
+        outs.append(r["o"])
+    assert np.array_equal(full["block"], blk)
+    assert np.array_equal(full["o"], np.concatenate(outs))
+
+
+def test_prefill_empty_call_is_identity(orc):
+    block, w = _random_block(orc, 4, 16, 16, 26)
+    e = np.zeros((0, 16))
+    res = orc.prefill_seq(4, 0, block, e, e, e, np.zeros(0), np.zeros(0), w, 64, 16, 16)
+    assert np.array_equal(res["block"], block)
