@@ -1,0 +1,442 @@
+#!/usr/bin/env python3
+"""Benchmark of the quantized-state decode step on B200.
+
+One step = one decode token for every head of every request of the workload: a single
+stq_decode_step over 2304 heads x 70 requests (48 layers x 48 heads of 128 x 128 states, mixed
+4/6/8-bit codes with 1.4% FP16 pivot heads), reading and writing the packed state in place.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+Under torchrun (N > 1) every rank runs its own 70 requests on its own GPU (weak scaling; the
+(request, head) tiles are independent, so no data-path collective exists); the timed region is
+bracketed by a barrier and a device synchronize, and the reported time is the max over ranks.
+Rank 0 prints one JSON line. `--impl reference` times the CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized-state head-steps/sec and achieved HBM GB/s (% roofline) at batch 70"
+DEFAULT_WORKLOAD = "full2304_b70_mixed"
+TOKENS_CYCLED = 8
+FALLBACK_HBM_GBS = 6650.0
+DECODE_SOURCES = ("quantized_linear_attention_stq_b200/csrc/decode_d128.cu",
+                  "quantized_linear_attention_stq_b200/csrc/stq_internal.cuh")
+TRAFFIC_FILE = "profiles/decode_d128_full2304_b70.md"
+
+
+# ------------------------------------------------------------------------------------------------
+# distributed plumbing (host logic; covered by gloo tests on CPU)
+# ------------------------------------------------------------------------------------------------
+
+def dist_env():
+    """(rank, world, local_rank) from the torchrun environment (1 process if absent)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def request_offset(rank: int, batch: int) -> int:
+    """First request index of a rank: every rank owns its own `batch` requests."""
+    return rank * batch
+
+
+def reduce_max(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.barrier(device_ids=[device.index] if device is not None and device.type == "cuda" else None)
+
+
+# ------------------------------------------------------------------------------------------------
+# small helpers
+# ------------------------------------------------------------------------------------------------
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "of measured"
+    return FALLBACK_HBM_GBS, "of fallback"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in DECODE_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
+    path = os.path.join(ROOT, TRAFFIC_FILE)
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "kernel_source_sha256")):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256") != decode_source_hash():
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling around the timed region."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self, t0: float, t1: float):
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        inside = [r for r in rows if t0 - 0.15 <= r[0] <= t1 + 0.15]
+        used = inside or sorted(rows, key=lambda r: min(abs(r[0] - t0), abs(r[0] - t1)))[:3]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in used for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in used), "sm_max_mhz": max(r[2] for r in used),
+                "reasons": reasons, "samples": len(used), "samples_inside_timed_region": len(inside)}
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle timing (the reported CPU baseline and the reference arm)
+# ------------------------------------------------------------------------------------------------
+
+def _oracle_worker(args):
+    """Runs in a spawned process: decode `reps` passes over a list of tiles with the oracle."""
+    tiles, reps = args
+    sys.path.insert(0, ROOT)
+    import oracle as orc
+
+    orc.lib()
+    blocks = [t["block"] for t in tiles]
+    t0 = time.perf_counter()
+    n = 0
+    for _ in range(reps):
+        for i, t in enumerate(tiles):
+            res = orc.decode_step(t["bits"], 0, blocks[i], t["q"], t["k"], t["v"], t["beta"], t["alpha"], t["w"],
+                                  128, 128)
+            blocks[i] = res["block"]
+            n += 1
+    return n, time.perf_counter() - t0
+
+
+def oracle_sample_tiles(workload_name: str, n_tiles: int, seed_offset: int = 0):
+    """A bounded sample of the workload's tiles (same width mix and input distributions)."""
+    import numpy as np
+    import oracle as orc
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl = wlm.WORKLOADS[workload_name]
+    bits_all = wlm.head_bits(wl)
+    rng = np.random.default_rng(1234 + seed_offset)
+    heads = rng.choice(len(bits_all), size=n_tiles, replace=False)
+    # make sure every width of the workload appears
+    for b in sorted(set(bits_all)):
+        if not any(bits_all[h] == b for h in heads):
+            heads[rng.integers(n_tiles)] = bits_all.index(b)
+    small = wlm.scaled(wl, batch=1, heads=len(heads), outliers=wl.outliers)
+    S0 = wlm.initial_state(small, 0).double().numpy()
+    w_all = wlm.impact_weights(wl).double().numpy()
+    inp = wlm.decode_inputs(small, 0)
+    alpha = wlm.gate_values(wl).double().numpy()
+    tiles = []
+    for i, h in enumerate(heads):
+        b = int(bits_all[h])
+        blk, _, _, _ = orc.quantize(b, S0[i], w_all[h])
+        tiles.append(dict(bits=b, block=blk, w=w_all[h], q=inp["q"][0, i].double().numpy(),
+                          k=inp["k"][0, i].double().numpy(), v=inp["v"][0, i].double().numpy(),
+                          beta=float(inp["beta"][0, i]), alpha=float(alpha[h])))
+    return tiles
+
+
+def time_oracle(workload_name: str, workers: int, tiles_per_worker: int, reps: int):
+    """Run the oracle on `workers` spawned processes; returns (head-steps/s, cores, sample text)."""
+    import multiprocessing as mp
+
+    samples = [oracle_sample_tiles(workload_name, tiles_per_worker, seed_offset=k) for k in range(workers)]
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(workers) as pool:
+        pool.map(_oracle_worker, [(s[:1], 1) for s in samples])  # warm the workers (load + build)
+        t0 = time.perf_counter()
+        res = pool.map(_oracle_worker, [(s, reps) for s in samples])
+        wall = time.perf_counter() - t0
+    n = sum(r[0] for r in res)
+    widths = sorted({t["bits"] for s in samples for t in s})
+    sample = (f"{n} head-steps: {workers} processes x {tiles_per_worker} sampled 128x128 tiles of "
+              f"{workload_name} (widths {widths}) x {reps} decode steps; fp64 C oracle")
+    return n / wall, workers, sample
+
+
+def oracle_workers():
+    return max(1, min(os.cpu_count() or 1, 32))
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import quantized_linear_attention_stq_b200 as stq
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    wl = wlm.WORKLOADS[args.workload]
+    B, H, d = wl.batch, wl.heads, wl.d
+    bits = wlm.head_bits(wl)
+    lay = stq.Layout(bits, d, gate=wl.gate, in_dtype=wl.in_dtype)
+    pool = lay.alloc_pool(B, dev)
+    slots = torch.arange(B, dtype=torch.int32, device=dev)
+    w = wlm.impact_weights(wl, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    r0 = request_offset(rank, B)
+    chunk = 10
+    for b0 in range(0, B, chunk):
+        nb = min(chunk, B - b0)
+        S0 = torch.stack([wlm.initial_state(wl, r0 + b0 + i, dev) for i in range(nb)])
+        stq.init_state(lay, pool, slots[b0:b0 + nb].clone(), S0, w, status=status)
+        del S0
+    # realised outlier ratios of the initial states (first request, first 64 heads)
+    S0s = wlm.initial_state(wl, r0, dev)[:64].double()
+    row_rms = S0s.pow(2).mean(dim=2).sqrt()
+    col_rms = S0s.pow(2).mean(dim=1).sqrt()
+    row_ratio = float((row_rms.max(dim=1).values / row_rms.median(dim=1).values).median())
+    col_ratio = float((col_rms.max(dim=1).values / col_rms.median(dim=1).values).median())
+    del S0s
+    toks = [wlm.decode_inputs(wl, 1000 * rank + t, dev) for t in range(TOKENS_CYCLED)]
+    o = torch.empty(B, H, d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+
+    def step(t):
+        x = toks[t % TOKENS_CYCLED]
+        stq.decode_step(lay, pool, slots, x["q"], x["k"], x["v"], x["beta"], x["alpha"], w, o, status=status,
+                        stream=stream)
+
+    for t in range(args.warmup):
+        step(t)
+    torch.cuda.synchronize(dev)
+    if status.item() != 0:
+        raise RuntimeError(f"device status after warm-up: {stq.status_flags(status)}")
+
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    ev[0].record(stream)
+    for t in range(args.steps):
+        step(args.warmup + t)
+        ev[t + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    barrier(dev)
+    time.sleep(0.3)
+    clocks.stop()
+    total_ms = ev[0].elapsed_time(ev[-1])
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms_max = reduce_max(total_ms, dev)
+    if status.item() != 0:
+        raise RuntimeError(f"device status after timing: {stq.status_flags(status)}")
+
+    # end to end through the public API with host buffers: H2D inputs, step, D2H readout
+    e2e_steps = max(1, min(args.steps, 50))
+    host_in = [{n: x.cpu().pin_memory() for n, x in toks[t].items()} for t in range(min(TOKENS_CYCLED, e2e_steps))]
+    dev_in = {n: torch.empty_like(x) for n, x in toks[0].items()}
+    host_o = torch.empty(B, H, d, dtype=torch.float32).pin_memory()
+    h2d_bytes = sum(x.numel() * x.element_size() for x in host_in[0].values())
+    d2h_bytes = host_o.numel() * host_o.element_size()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for t in range(e2e_steps):
+        src = host_in[t % len(host_in)]
+        for n in dev_in:
+            dev_in[n].copy_(src[n], non_blocking=True)
+        stq.decode_step(lay, pool, slots, dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"], dev_in["alpha"], w,
+                        o, status=status, stream=stream)
+        host_o.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
+
+    # figures
+    state_bytes = 2 * sum(lay.head_bytes(h) for h in range(H)) * B  # read + write, one launch
+    io_bytes = B * H * (3 * d * (2 if wl.in_dtype == torch.bfloat16 else 4) + 4 * d + 8)
+    launches_per_step = math.ceil(B / 1024) * math.ceil(H / 3072)
+    avg_launch_s = total_ms / 1e3 / (args.steps * launches_per_step)
+    achieved = state_bytes / launches_per_step / avg_launch_s / 1e9
+    peak, peak_kind = measured_peaks()
+    step_s = total_ms_max / 1e3 / args.steps
+    head_steps = B * H * world
+    result = {
+        "metric": METRIC,
+        "value": head_steps / step_s,
+        "unit": "head-steps/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "batch_per_gpu": B, "heads": H, "d_k": d, "d_v": d,
+                   "widths": {str(b): bits.count(b) for b in sorted(set(bits))}, "in_dtype": str(wl.in_dtype),
+                   "gate": "scalar" if wl.gate == 0 else "channel", "tokens_cycled": TOKENS_CYCLED,
+                   "l2": "no flush: the 2.0 GB state pool read+written per step exceeds the 126 MB L2",
+                   "parallelism": f"dp{world} (independent requests per GPU)",
+                   "s0_row_max_to_median": round(row_ratio, 2), "s0_col_max_to_median": round(col_ratio, 2)},
+        "tokens_per_s": B * world / step_s,
+        "state_gbs": state_bytes / step_s / 1e9,
+        "state_plus_io_gbs": (state_bytes + io_bytes * launches_per_step) / step_s / 1e9,
+        "step_ms_median": statistics.median(per_step),
+        "step_ms_min": min(per_step),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": peak_kind, "traffic": profiled_traffic(),
+                     "bytes_per_launch": state_bytes / launches_per_step,
+                     "kernel": "decode_d128_kernel", "kernel_source_sha256": decode_source_hash()},
+        "e2e": {"value": head_steps / (e2e_ms / 1e3 / e2e_steps), "unit": "head-steps/s",
+                "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes, "steps": e2e_steps},
+        "gpu_launches": args.steps * launches_per_step,
+        "clocks": clocks.summary(t_wall0, t_wall1),
+        "gpu": torch.cuda.get_device_name(dev),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, sample = time_oracle(args.workload, oracle_workers(), 16, 20)
+        result["cpu_baseline"] = {"value": rate, "unit": "head-steps/s", "cores": cores, "kind": "oracle",
+                                  "sample": sample}
+    elif rank == 0:
+        result["cpu_baseline"] = None
+    if world > 1:
+        dist.barrier(device_ids=[dev.index])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    workers = oracle_workers()
+    # one step = one sampled tile per worker; all steps run back to back inside the workers
+    rate, cores, sample = time_oracle(args.workload, workers, 1, max(1, args.steps))
+    result = {
+        "metric": METRIC,
+        "impl": "reference",
+        "value": rate,
+        "unit": "head-steps/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": workers / rate * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "note": "CPU oracle on the host cores; bounded sample per step"},
+        "cpu_baseline": {"value": rate, "unit": "head-steps/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": rate, "unit": "head-steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(result), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,172 @@
+/*
+ * stq.h -- C ABI of the quantized linear-attention state library (B200, sm_100a).
+ *
+ * What it computes. Linear-attention models with the gated delta rule keep one fixed-size
+ * recurrent state per request and head ("线性注意力状态量化难题" (aitest123.com/news/n1kj09),
+ * introduction); serving many requests makes that state pool the memory bottleneck ("K1 論文詳解"
+ * (k1-news.pages.dev/paper/2026-10-09), section 背景). Each decode step reads the previous
+ * state, updates it, requantizes it and stores it back (aitest123 page, section
+ * 直接量化为什么会翻车). The state of a head is kept as low-bit integer codes with one scale per
+ * key row and one per value column whose product sets the step (k1 page, section 方法;
+ * aitest123 page, section 空间维度); widths come per head from a few discrete candidates and the
+ * highest-risk heads stay FP16 (k1 page, section 方法; aitest123 page, section 时间维度). The
+ * pages print no formula; this library fixes them as follows (d_k x d_v state S per head):
+ *
+ *   dequantize   S_ij = r_i c_j Q_ij,  Q_ij in [-qmax, qmax], qmax = 2^(b-1) - 1, b in {4,6,8}
+ *   update       u = k^T S;  S' = alpha (S - beta k u^T) + beta k v^T
+ *   readout      o = S'^T q               (after the update, before requantization)
+ *   column scale c'_j = sqrt( sum_i w_i S'_ij^2 / sum_i w_i )   (w: per-head key-row impact)
+ *   row scale    r'_i = max_j |S'_ij / c'_j| / qmax
+ *   requantize   Q'_ij = round_half_even(S'_ij / (r'_i c'_j)); a zero scale is replaced by 1
+ * Scales are stored as fp32 and codes are computed from the stored scales; a pivot head (b = 16)
+ * stores S' as fp16 (round to nearest even) and has no scales. With the channel gate alpha is a
+ * vector over key rows: STQ_GATE_CHANNEL substitutes it literally,
+ * S'_ij = alpha_i (S_ij - beta k_i u_j) + beta k_i v_j; STQ_GATE_CHANNEL_DECAY_FIRST decays first,
+ * u = k^T diag(alpha) S, S'_ij = alpha_i S_ij - beta k_i u_j + beta k_i v_j.
+ *
+ * Byte layout of the pool. A request block is the concatenation of its head blocks (in head
+ * order) padded to 128 bytes; request `slot` starts at pool + slot * bytes_per_request. A quantized
+ * head block holds the codes as a little-endian bitstream (code (i,j) at bit b*(i*d_v + j), bit k
+ * of the stream = bit k%8 of byte k/8, stored offset-binary Q + 2^(b-1)), zero padding to 16 bytes,
+ * r[d_k] fp32, c[d_v] fp32, zero padding to 128 bytes. A pivot head block is S as fp16 row-major,
+ * padded to 128 bytes. The pool is its own checkpoint: its bytes plus the layout descriptor.
+ *
+ * Conventions for every call below.
+ *   - All pointers named "device" point to memory of the current CUDA device; the caller owns and
+ *     allocates every buffer. The library allocates no device memory and never synchronizes.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). All work is
+ *     enqueued on it; results are ready when the stream reaches that point.
+ *   - Arguments are checked before anything is enqueued; a failed check returns
+ *     STQ_ERR_INVALID_ARG / STQ_ERR_UNSUPPORTED and enqueues nothing. A failed launch returns
+ *     STQ_ERR_CUDA.
+ *   - Conditions found on the device are OR-ed into *dev_status (a device int32 the caller zeroes;
+ *     may be NULL) as the bit (1 << code): STQ_ERR_NONFINITE when an updated state, scale or output
+ *     is not finite (or a pivot overflows fp16; the tile's bytes are then unspecified),
+ *     STQ_ERR_BOUNDS when a slot is outside [0, pool_slots) (that tile is skipped),
+ *     STQ_ERR_TIMEOUT when a bounded wait for a staged copy gave up (the call's remaining tiles
+ *     are skipped). Kernels never trap.
+ *   - Slots within one call must be distinct. Calls on different streams must not touch the same
+ *     slots concurrently.
+ *   - Supported on the device: d_k == d_v == d in {16, 32, 64, 128}; widths {4, 6, 8, 16};
+ *     q/k/v in fp32 or bf16. The prefill path supports d == 128 and the scalar gate.
+ */
+#ifndef STQ_H
+#define STQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define STQ_ABI_VERSION 1
+
+typedef enum {
+    STQ_OK = 0,
+    STQ_ERR_INVALID_ARG = 1,
+    STQ_ERR_UNSUPPORTED = 2,
+    STQ_ERR_CUDA = 3,
+    STQ_ERR_NONFINITE = 4,
+    STQ_ERR_TIMEOUT = 5,
+    STQ_ERR_BOUNDS = 6
+} stq_status;
+
+typedef enum { STQ_F32 = 0, STQ_BF16 = 1 } stq_dtype;
+
+typedef enum {
+    STQ_GATE_SCALAR = 0,             /* alpha [B][H]        */
+    STQ_GATE_CHANNEL = 1,            /* alpha [B][H][d_k]   */
+    STQ_GATE_CHANNEL_DECAY_FIRST = 2 /* alpha [B][H][d_k]   */
+} stq_gate;
+
+/* Static description of one model's state: fixed across requests and steps. */
+typedef struct {
+    int32_t num_heads;         /* H >= 1 (all layers' heads of one request, in pool order)   */
+    int32_t d_k;               /* key dimension (rows of a head's state)                     */
+    int32_t d_v;               /* value dimension (columns)                                  */
+    const uint8_t *head_bits;  /* host [H]: 4, 6, 8, or 16 (FP16 pivot head); copied         */
+    int32_t gate;              /* stq_gate                                                   */
+    int32_t in_dtype;          /* stq_dtype of q, k, v                                       */
+} stq_layout_desc;
+
+typedef struct stq_layout stq_layout; /* opaque, host-only, immutable after creation */
+
+/* Version of this ABI (STQ_ABI_VERSION of the built library). */
+int32_t stq_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *stq_status_string(int32_t status);
+
+/* Build a layout from `desc` (host only; no CUDA call). Returns STQ_ERR_INVALID_ARG for NULL
+ * pointers or non-positive sizes, STQ_ERR_UNSUPPORTED for widths other than {4,6,8,16} or
+ * shapes the device path does not support. On success *out owns a new layout, released with
+ * stq_layout_destroy. The layout may be shared between threads. */
+stq_status stq_layout_create(const stq_layout_desc *desc, stq_layout **out);
+void stq_layout_destroy(stq_layout *layout);
+
+/* Bytes of one request block (a multiple of 128), and the byte offset / size / width of head h
+ * inside it (0 for an invalid head). */
+size_t stq_layout_bytes_per_request(const stq_layout *layout);
+size_t stq_layout_head_offset(const stq_layout *layout, int32_t head);
+size_t stq_layout_head_bytes(const stq_layout *layout, int32_t head);
+int32_t stq_layout_head_bits(const stq_layout *layout, int32_t head);
+
+/* Quantize given fp32 states into the pool: the column / row scale fit and requantization above
+ * applied to S0 (or the fp16 conversion for pivot heads).
+ *   pool        device, >= pool_slots * bytes_per_request bytes, 128-byte aligned
+ *   slots       device int32 [B], the pool slot of each request
+ *   S0          device fp32 [B][H][d_k][d_v], row-major
+ *   w           device fp32 [H][d_k], impact weights, finite and > 0
+ * B == 0 is a no-op. */
+stq_status stq_init_state(const stq_layout *layout, void *pool, int32_t pool_slots,
+                          const int32_t *slots, int32_t B, const float *S0, const float *w,
+                          int32_t *dev_status, void *stream);
+
+/* One decode step, in place, for heads [head_begin, head_begin + head_count) of B requests:
+ * dequantize, update, read out, refit the scales, requantize, store. Per-head arrays below are
+ * indexed by (request b, head h - head_begin), i.e. they hold only the heads of this call:
+ *   q, k        device [B][head_count][d_k] of in_dtype, 16-byte aligned
+ *   v           device [B][head_count][d_v] of in_dtype, 16-byte aligned
+ *   beta        device fp32 [B][head_count]
+ *   alpha       device fp32 [B][head_count] (scalar gate) or [B][head_count][d_k], 16-byte aligned
+ *   w           device fp32 [head_count][d_k], finite and > 0, 16-byte aligned
+ *   o           device fp32 [B][head_count][d_v], written
+ * B == 0 or head_count == 0 is a no-op. */
+stq_status stq_decode_step(const stq_layout *layout, void *pool, int32_t pool_slots,
+                           const int32_t *slots, int32_t B, int32_t head_begin, int32_t head_count,
+                           const void *q, const void *k, const void *v, const float *beta,
+                           const float *alpha, const float *w, float *o, int32_t *dev_status,
+                           void *stream);
+
+/* Workspace bytes stq_prefill_chunk needs for B requests and T tokens in chunks of `chunk`. */
+size_t stq_prefill_workspace_bytes(const stq_layout *layout, int32_t B, int32_t T, int32_t chunk);
+
+/* Chunked prefill of T tokens for all H heads of B requests, in place. Tokens are cut into
+ * chunks [0,chunk), [chunk,2chunk), ... of this call (the last may be short); inside a chunk
+ * the state is carried unquantized, o_t = S_t^T q_t is emitted for every token, and the state is
+ * requantized into the pool at the end of every chunk. chunk == 1 is the decode step token by
+ * token.
+ *   q, k        device [B][H][T][d_k] of in_dtype;  v device [B][H][T][d_v] of in_dtype
+ *   beta, alpha device fp32 [B][H][T] (scalar gate)
+ *   w           device fp32 [H][d_k]
+ *   o           device fp32 [B][H][T][d_v], written
+ *   workspace   device scratch of >= stq_prefill_workspace_bytes(...) bytes, 256-byte aligned
+ * T == 0 or B == 0 is a no-op. */
+stq_status stq_prefill_chunk(const stq_layout *layout, void *pool, int32_t pool_slots,
+                             const int32_t *slots, int32_t B, int32_t T, int32_t chunk,
+                             const void *q, const void *k, const void *v, const float *beta,
+                             const float *alpha, const float *w, float *o, void *workspace,
+                             size_t workspace_bytes, int32_t *dev_status, void *stream);
+
+/* Dequantize the pool into fp32: S_out[b][h][i][j] = fp32(r_i c_j) * Q_ij (the fp16 value for a
+ * pivot head).  S_out device fp32 [B][H][d_k][d_v]. */
+stq_status stq_dequantize(const stq_layout *layout, const void *pool, int32_t pool_slots,
+                          const int32_t *slots, int32_t B, float *S_out, int32_t *dev_status,
+                          void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STQ_H */

@@ -1,0 +1,354 @@
+// generic_kernels.cu -- one CTA per (request, head) tile, the state staged in shared memory as
+// fp32 and every step written out directly: initial quantization, dequantization, and the decode
+// step for the small head sizes (d < 128). The tuned d = 128 decode lives in decode_d128.cu.
+//
+// Method (formulas in include/stq.h): per-step read -> gated delta rule update -> readout ->
+// requantize -> store ("线性注意力状态量化难题" (aitest123.com/news/n1kj09), section
+// 直接量化为什么会翻车); key-row x value-column scales with the impact-weighted column fit
+// (same page, section 空间维度; "K1 論文詳解" (k1-news.pages.dev/paper/2026-10-09), section 方法);
+// FP16 pivot heads (k1 page, section 方法).
+#include "stq_internal.cuh"
+
+namespace stq {
+namespace {
+
+constexpr int kThreads = 256;
+
+struct TileRef {
+    bool ok;
+    int b, head, bits;
+    uint8_t *block;
+};
+
+__device__ __forceinline__ TileRef tile_ref(const TileParams &p, int b, int pos)
+{
+    TileRef t;
+    const TileEntry e = p.table[pos];
+    t.b = b;
+    t.head = entry_head(e);
+    t.bits = entry_bits(e);
+    const int slot = p.slots[b];
+    t.ok = slot >= 0 && slot < p.pool_slots;
+    t.block = t.ok ? p.pool + (uint64_t)slot * p.req_bytes + e.off : nullptr;
+    return t;
+}
+
+// Code n (offset-binary) of a b-bit little-endian bitstream. Reads at most two bytes; the byte
+// after the last code is inside the block (scales follow the codes).
+__device__ __forceinline__ int read_code(const uint8_t *codes, int bits, int n)
+{
+    const uint32_t bit = (uint32_t)bits * (uint32_t)n;
+    const uint32_t lo = codes[bit >> 3];
+    const uint32_t hi = codes[(bit >> 3) + 1];
+    return (int)(((lo | (hi << 8)) >> (bit & 7)) & ((1u << bits) - 1u));
+}
+
+// Dequantize a tile from global memory into S (row stride ld): S_ij = fp32(r_i c_j) * Q_ij.
+__device__ void dequant_to_smem(const uint8_t *block, int bits, int dk, int dv, float *S, int ld)
+{
+    const int n = dk * dv;
+    if (bits == 16) {
+        const __half *h = reinterpret_cast<const __half *>(block);
+        for (int e = threadIdx.x; e < n; e += blockDim.x) S[(e / dv) * ld + e % dv] = __half2float(h[e]);
+        return;
+    }
+    const float *r = reinterpret_cast<const float *>(block + scale_offset(bits, dk, dv));
+    const float *c = r + dk;
+    const int off = 1 << (bits - 1);
+    for (int e = threadIdx.x; e < n; e += blockDim.x) {
+        const int i = e / dv, j = e % dv;
+        const float rc = r[i] * c[j];
+        S[i * ld + j] = rc * (float)(read_code(block, bits, e) - off);
+    }
+}
+
+// Fit scales to the fp32 state in S and write codes + scales into `block` (or fp16 values for a
+// pivot head). `wv` holds the impact weights of the head in shared memory. Needs a CTA-wide
+// barrier before (S complete) and provides one after.
+__device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, int dk, int dv,
+                                   uint8_t *block, float *cs, float *rs, int32_t *status)
+{
+    const int n = dk * dv;
+    if (bits == 16) {
+        __half *h = reinterpret_cast<__half *>(block);
+        bool bad = false;
+        for (int e = threadIdx.x; e < n; e += blockDim.x) {
+            const float x = S[(e / dv) * ld + e % dv];
+            bad |= !(fabsf(x) < 65520.0f);  // overflows fp16 (or is NaN)
+            h[e] = __float2half_rn(x);
+        }
+        if (__syncthreads_or(bad) && threadIdx.x == 0) flag(status, kFlagNonfinite);
+        return;
+    }
+    const float qmax = (float)((1 << (bits - 1)) - 1);
+    // column scales: impact-weighted RMS over the key rows
+    for (int j = threadIdx.x; j < dv; j += blockDim.x) {
+        float W = 0.f, E = 0.f;
+        for (int i = 0; i < dk; ++i) {
+            const float x = S[i * ld + j];
+            W += wv[i];
+            E += wv[i] * x * x;
+        }
+        float c = sqrtf(E / W);
+        if (c == 0.f) c = 1.f;
+        cs[j] = c;
+    }
+    __syncthreads();
+    // row scales: largest column-normalised magnitude over qmax
+    for (int i = threadIdx.x; i < dk; i += blockDim.x) {
+        float m = 0.f;
+        for (int j = 0; j < dv; ++j) m = fmaxf(m, fabsf(S[i * ld + j] / cs[j]));
+        float r = m / qmax;
+        if (r == 0.f) r = 1.f;
+        rs[i] = r;
+    }
+    __syncthreads();
+    bool bad = false;
+    float *rg = reinterpret_cast<float *>(block + scale_offset(bits, dk, dv));
+    for (int i = threadIdx.x; i < dk; i += blockDim.x) {
+        rg[i] = rs[i];
+        bad |= !isfinite(rs[i]) || rs[i] == 0.f;
+    }
+    for (int j = threadIdx.x; j < dv; j += blockDim.x) {
+        rg[dk + j] = cs[j];
+        bad |= !isfinite(cs[j]);
+    }
+    // codes, packed by groups of whole bytes: 2 codes/byte (4-bit), 4 codes/3 bytes (6-bit),
+    // 1 code/byte (8-bit)
+    const int cpg = bits == 4 ? 2 : (bits == 6 ? 4 : 1);
+    const int bpg = bits == 6 ? 3 : 1;
+    const int off = 1 << (bits - 1);
+    for (int g = threadIdx.x; g < n / cpg; g += blockDim.x) {
+        uint32_t word = 0;
+        for (int t = 0; t < cpg; ++t) {
+            const int e = g * cpg + t;
+            const int i = e / dv, j = e % dv;
+            float x = (S[i * ld + j] / cs[j]) / rs[i];
+            x = fminf(fmaxf(rintf(x), -qmax), qmax);  // rintf rounds half to even
+            if (!isfinite(x)) x = 0.f;
+            word |= (uint32_t)((int)x + off) << (bits * t);
+        }
+        for (int t = 0; t < bpg; ++t) block[g * bpg + t] = (uint8_t)(word >> (8 * t));
+    }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) flag(status, kFlagNonfinite);
+}
+
+// ------------------------------------------------------------------------------------------
+// Initial quantization: S0 fp32 [B][H][dk][dv] -> pool
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads) init_kernel(const __grid_constant__ TileParams p)
+{
+    extern __shared__ __align__(16) float sm[];
+    const int b = blockIdx.x, pos = blockIdx.y;
+    const TileRef t = tile_ref(p, b, pos);
+    if (!t.ok) {
+        if (threadIdx.x == 0) flag(p.status, kFlagBounds);
+        return;
+    }
+    const int dk = p.dk, dv = p.dv, ld = dv + 1;
+    float *S = sm;
+    float *wv = S + dk * ld;
+    float *cs = wv + dk;
+    float *rs = cs + dv;
+    const float *src = p.S0 + ((uint64_t)b * p.head_count + t.head) * dk * dv;
+    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) S[(e / dv) * ld + e % dv] = src[e];
+    for (int i = threadIdx.x; i < dk; i += blockDim.x) wv[i] = p.w[(uint64_t)t.head * dk + i];
+    __syncthreads();
+    quantize_from_smem(S, ld, wv, t.bits, dk, dv, t.block, cs, rs, p.status);
+}
+
+// ------------------------------------------------------------------------------------------
+// Dequantization: pool -> S_out fp32 [B][H][dk][dv]
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads) dequant_kernel(const __grid_constant__ TileParams p)
+{
+    const int b = blockIdx.x, pos = blockIdx.y;
+    const TileRef t = tile_ref(p, b, pos);
+    if (!t.ok) {
+        if (threadIdx.x == 0) flag(p.status, kFlagBounds);
+        return;
+    }
+    const int dk = p.dk, dv = p.dv;
+    float *dst = p.S_out + ((uint64_t)b * p.head_count + t.head) * dk * dv;
+    dequant_to_smem(t.block, t.bits, dk, dv, dst, dv);  // writes straight to global, row stride dv
+}
+
+// ------------------------------------------------------------------------------------------
+// Decode step, plain form
+// ------------------------------------------------------------------------------------------
+template <int IN_BF16>
+__global__ void __launch_bounds__(kThreads) decode_generic_kernel(const __grid_constant__ TileParams p)
+{
+    extern __shared__ __align__(16) float sm[];
+    const int b = blockIdx.x, pos = blockIdx.y;
+    const TileRef t = tile_ref(p, b, pos);
+    if (!t.ok) {
+        if (threadIdx.x == 0) flag(p.status, kFlagBounds);
+        return;
+    }
+    const int dk = p.dk, dv = p.dv, ld = dv + 1;
+    float *S = sm;
+    float *kv = S + dk * ld;
+    float *qv = kv + dk;
+    float *av = qv + dk;
+    float *wv = av + dk;
+    float *vv = wv + dk;
+    float *uv = vv + dv;
+    float *cs = uv + dv;
+    float *rs = cs + dv;
+    const uint64_t tile = (uint64_t)b * p.head_count + t.head;
+    const bool channel = p.gate != 0;
+    for (int i = threadIdx.x; i < dk; i += blockDim.x) {
+        kv[i] = load_in<IN_BF16>(p.k, tile * dk + i);
+        qv[i] = load_in<IN_BF16>(p.q, tile * dk + i);
+        av[i] = channel ? p.alpha[tile * dk + i] : p.alpha[tile];
+        wv[i] = p.w[(uint64_t)t.head * dk + i];
+    }
+    for (int j = threadIdx.x; j < dv; j += blockDim.x) vv[j] = load_in<IN_BF16>(p.v, tile * dv + j);
+    dequant_to_smem(t.block, t.bits, dk, dv, S, ld);
+    __syncthreads();
+    const float beta = p.beta[tile];
+    const bool decay_first = p.gate == 2;
+    // u = k^T S   (decay-first: k^T diag(alpha) S)
+    for (int j = threadIdx.x; j < dv; j += blockDim.x) {
+        float acc = 0.f;
+        for (int i = 0; i < dk; ++i) acc += kv[i] * (decay_first ? av[i] : 1.f) * S[i * ld + j];
+        uv[j] = acc;
+    }
+    __syncthreads();
+    // S' = alpha (S - beta k u^T) + beta k v^T   (decay-first: alpha S - beta k u^T + beta k v^T)
+    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
+        const int i = e / dv, j = e % dv;
+        const float s = S[i * ld + j];
+        S[i * ld + j] = decay_first ? av[i] * s - beta * kv[i] * uv[j] + beta * kv[i] * vv[j]
+                                    : av[i] * (s - beta * kv[i] * uv[j]) + beta * kv[i] * vv[j];
+    }
+    __syncthreads();
+    // o = S'^T q
+    bool bad = false;
+    for (int j = threadIdx.x; j < dv; j += blockDim.x) {
+        float acc = 0.f;
+        for (int i = 0; i < dk; ++i) acc += qv[i] * S[i * ld + j];
+        p.o[tile * dv + j] = acc;
+        bad |= !isfinite(acc);
+    }
+    if (bad) flag(p.status, kFlagNonfinite);
+    quantize_from_smem(S, ld, wv, t.bits, dk, dv, t.block, cs, rs, p.status);
+}
+
+// ------------------------------------------------------------------------------------------
+// Chunked prefill, sequential form: the state is carried unquantized in shared memory through a
+// chunk (token-by-token gated delta rule, o_t = S_t^T q_t per token) and requantized into the
+// pool at the end of every chunk; the next chunk starts from the dequantized state.
+// ------------------------------------------------------------------------------------------
+template <int IN_BF16>
+__global__ void __launch_bounds__(kThreads) prefill_seq_kernel(const __grid_constant__ TileParams p, int T, int chunk)
+{
+    extern __shared__ __align__(16) float sm[];
+    const int b = blockIdx.x, pos = blockIdx.y;
+    const TileRef t = tile_ref(p, b, pos);
+    if (!t.ok) {
+        if (threadIdx.x == 0) flag(p.status, kFlagBounds);
+        return;
+    }
+    const int dk = p.dk, dv = p.dv, ld = dv + 1;
+    float *S = sm;
+    float *kv = S + dk * ld;
+    float *qv = kv + dk;
+    float *av = qv + dk;
+    float *wv = av + dk;
+    float *vv = wv + dk;
+    float *uv = vv + dv;
+    float *cs = uv + dv;
+    float *rs = cs + dv;
+    const uint64_t tile = (uint64_t)b * p.head_count + t.head;
+    const bool channel = p.gate != 0, decay_first = p.gate == 2;
+    for (int i = threadIdx.x; i < dk; i += blockDim.x) wv[i] = p.w[(uint64_t)t.head * dk + i];
+    dequant_to_smem(t.block, t.bits, dk, dv, S, ld);
+    bool bad = false;
+    for (int tok = 0; tok < T; ++tok) {
+        const uint64_t row = tile * T + tok;
+        for (int i = threadIdx.x; i < dk; i += blockDim.x) {
+            kv[i] = load_in<IN_BF16>(p.k, row * dk + i);
+            qv[i] = load_in<IN_BF16>(p.q, row * dk + i);
+            av[i] = channel ? p.alpha[row * dk + i] : p.alpha[row];
+        }
+        for (int j = threadIdx.x; j < dv; j += blockDim.x) vv[j] = load_in<IN_BF16>(p.v, row * dv + j);
+        __syncthreads();
+        const float beta = p.beta[row];
+        for (int j = threadIdx.x; j < dv; j += blockDim.x) {
+            float acc = 0.f;
+            for (int i = 0; i < dk; ++i) acc += kv[i] * (decay_first ? av[i] : 1.f) * S[i * ld + j];
+            uv[j] = acc;
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
+            const int i = e / dv, j = e % dv;
+            const float s = S[i * ld + j];
+            S[i * ld + j] = decay_first ? av[i] * s - beta * kv[i] * uv[j] + beta * kv[i] * vv[j]
+                                        : av[i] * (s - beta * kv[i] * uv[j]) + beta * kv[i] * vv[j];
+        }
+        __syncthreads();
+        for (int j = threadIdx.x; j < dv; j += blockDim.x) {
+            float acc = 0.f;
+            for (int i = 0; i < dk; ++i) acc += qv[i] * S[i * ld + j];
+            p.o[row * dv + j] = acc;
+            bad |= !isfinite(acc);
+        }
+        if ((tok + 1) % chunk == 0 || tok == T - 1) {
+            __syncthreads();
+            quantize_from_smem(S, ld, wv, t.bits, dk, dv, t.block, cs, rs, p.status);
+            if (tok != T - 1) {
+                __syncthreads();
+                dequant_to_smem(t.block, t.bits, dk, dv, S, ld);
+            }
+        }
+        __syncthreads();
+    }
+    if (bad) flag(p.status, kFlagNonfinite);
+}
+
+size_t generic_smem_bytes(const TileParams &p)
+{
+    return sizeof(float) * ((size_t)p.dk * (p.dv + 1) + 5 * (size_t)p.dk + 4 * (size_t)p.dv + 64);
+}
+
+template <typename K>
+cudaError_t launch_tiles(K kernel, const TileParams &p, cudaStream_t s)
+{
+    const size_t smem = generic_smem_bytes(p);
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    dim3 grid((unsigned)p.B, (unsigned)p.npos);
+    kernel<<<grid, kThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_init_generic(const TileParams &p, cudaStream_t s) { return launch_tiles(init_kernel, p, s); }
+
+cudaError_t launch_dequant_generic(const TileParams &p, cudaStream_t s)
+{
+    dim3 grid((unsigned)p.B, (unsigned)p.npos);
+    dequant_kernel<<<grid, kThreads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_generic(const TileParams &p, int in_bf16, cudaStream_t s)
+{
+    return in_bf16 ? launch_tiles(decode_generic_kernel<1>, p, s) : launch_tiles(decode_generic_kernel<0>, p, s);
+}
+
+cudaError_t launch_prefill_seq(const TileParams &p, int in_bf16, int T, int chunk, cudaStream_t s)
+{
+    const size_t smem = generic_smem_bytes(p);
+    auto kernel = in_bf16 ? prefill_seq_kernel<1> : prefill_seq_kernel<0>;
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    dim3 grid((unsigned)p.B, (unsigned)p.npos);
+    kernel<<<grid, kThreads, smem, s>>>(p, T, chunk);
+    return cudaGetLastError();
+}
+
+}  // namespace stq

@@ -1,0 +1,290 @@
+// stq_host.cu -- host side of the C ABI declared in include/stq.h: layout objects, argument
+// checks, per-launch head tables and kernel dispatch. No device memory is allocated here and no
+// call synchronizes; every launch goes to the caller's stream.
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <memory>
+#include <new>
+#include <vector>
+
+#include "../../include/stq.h"
+#include "stq_internal.cuh"
+
+struct stq_layout {
+    int32_t H, dk, dv, gate, in_dtype;
+    std::vector<uint8_t> bits;
+    std::vector<uint64_t> offset;
+    std::vector<uint64_t> bytes;
+    uint64_t req_bytes;
+};
+
+namespace {
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Processing order of a launch: largest blocks first (FP16 pivots, then 8-, 6-, 4-bit), head
+// index order inside a width, so that round-robin CTAs see the same mix of tile sizes.
+std::vector<int> order_by_size(const stq_layout *L, int h0, int count)
+{
+    std::vector<int> ord(count);
+    for (int i = 0; i < count; ++i) ord[i] = h0 + i;
+    std::stable_sort(ord.begin(), ord.end(), [&](int a, int b) { return L->bits[a] > L->bits[b]; });
+    return ord;
+}
+
+// Fill the common fields of a TileParams for heads ord[first .. first+n) of a call.
+void fill_table(stq::TileParams &p, const stq_layout *L, const std::vector<int> &ord, int first, int n, int h0)
+{
+    p.npos = n;
+    for (int e = 0; e < n; ++e) {
+        const int h = ord[first + e];
+        p.table[e].off = (uint32_t)L->offset[h];
+        p.table[e].info = (uint32_t)(h - h0) | ((uint32_t)L->bits[h] << 16);
+    }
+}
+
+stq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? STQ_OK : STQ_ERR_CUDA; }
+
+// The parameter block is ~24 KB; keep it off the (small) thread stack.
+std::unique_ptr<stq::TileParams> new_params()
+{
+    std::unique_ptr<stq::TileParams> p(new (std::nothrow) stq::TileParams);
+    if (p) std::memset(p.get(), 0, sizeof(stq::TileParams));
+    return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t stq_abi_version(void) { return STQ_ABI_VERSION; }
+
+const char *stq_status_string(int32_t status)
+{
+    switch (status) {
+    case STQ_OK: return "ok";
+    case STQ_ERR_INVALID_ARG: return "invalid argument";
+    case STQ_ERR_UNSUPPORTED: return "unsupported shape, width or mode";
+    case STQ_ERR_CUDA: return "CUDA launch error";
+    case STQ_ERR_NONFINITE: return "non-finite state, scale or output";
+    case STQ_ERR_TIMEOUT: return "bounded wait timed out";
+    case STQ_ERR_BOUNDS: return "slot out of range";
+    default: return "unknown status";
+    }
+}
+
+stq_status stq_layout_create(const stq_layout_desc *desc, stq_layout **out)
+{
+    if (!desc || !out || !desc->head_bits) return STQ_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (desc->num_heads < 1 || desc->d_k < 1 || desc->d_v < 1) return STQ_ERR_INVALID_ARG;
+    if (desc->gate < STQ_GATE_SCALAR || desc->gate > STQ_GATE_CHANNEL_DECAY_FIRST) return STQ_ERR_INVALID_ARG;
+    if (desc->in_dtype != STQ_F32 && desc->in_dtype != STQ_BF16) return STQ_ERR_INVALID_ARG;
+    const int d = desc->d_k;
+    if (desc->d_v != d || !(d == 16 || d == 32 || d == 64 || d == 128)) return STQ_ERR_UNSUPPORTED;
+    if (desc->num_heads > 65535) return STQ_ERR_UNSUPPORTED;
+    std::unique_ptr<stq_layout> L(new (std::nothrow) stq_layout);
+    if (!L) return STQ_ERR_INVALID_ARG;
+    L->H = desc->num_heads;
+    L->dk = desc->d_k;
+    L->dv = desc->d_v;
+    L->gate = desc->gate;
+    L->in_dtype = desc->in_dtype;
+    uint64_t pos = 0;
+    for (int h = 0; h < L->H; ++h) {
+        const int b = desc->head_bits[h];
+        if (b != 4 && b != 6 && b != 8 && b != 16) return STQ_ERR_UNSUPPORTED;
+        L->bits.push_back((uint8_t)b);
+        L->offset.push_back(pos);
+        const uint64_t nb = stq::head_block_bytes(b, L->dk, L->dv);
+        L->bytes.push_back(nb);
+        pos += nb;
+    }
+    L->req_bytes = (pos + 127) / 128 * 128;
+    if (L->req_bytes > 0xFFFFFFFFull) return STQ_ERR_UNSUPPORTED;  // head offsets are 32-bit
+    *out = L.release();
+    return STQ_OK;
+}
+
+void stq_layout_destroy(stq_layout *layout) { delete layout; }
+
+size_t stq_layout_bytes_per_request(const stq_layout *L) { return L ? (size_t)L->req_bytes : 0; }
+
+size_t stq_layout_head_offset(const stq_layout *L, int32_t h)
+{
+    return (L && h >= 0 && h < L->H) ? (size_t)L->offset[h] : 0;
+}
+
+size_t stq_layout_head_bytes(const stq_layout *L, int32_t h)
+{
+    return (L && h >= 0 && h < L->H) ? (size_t)L->bytes[h] : 0;
+}
+
+int32_t stq_layout_head_bits(const stq_layout *L, int32_t h) { return (L && h >= 0 && h < L->H) ? L->bits[h] : 0; }
+
+stq_status stq_init_state(const stq_layout *L, void *pool, int32_t pool_slots, const int32_t *slots, int32_t B,
+                          const float *S0, const float *w, int32_t *dev_status, void *stream)
+{
+    if (!L || B < 0 || pool_slots < 0) return STQ_ERR_INVALID_ARG;
+    if (B == 0) return STQ_OK;
+    if (!pool || !slots || !S0 || !w || !aligned(pool, 128) || !aligned(S0, 4) || !aligned(w, 4))
+        return STQ_ERR_INVALID_ARG;
+    if (B > 2147483647 / L->H) return STQ_ERR_UNSUPPORTED;
+    auto p = new_params();
+    if (!p) return STQ_ERR_INVALID_ARG;
+    p->pool = static_cast<uint8_t *>(pool);
+    p->slots = slots;
+    p->status = dev_status;
+    p->req_bytes = L->req_bytes;
+    p->pool_slots = pool_slots;
+    p->B = B;
+    p->head_count = L->H;
+    p->dk = L->dk;
+    p->dv = L->dv;
+    p->gate = L->gate;
+    p->S0 = S0;
+    p->w = w;
+    const std::vector<int> ord = order_by_size(L, 0, L->H);
+    for (int first = 0; first < L->H; first += stq::kMaxTable) {
+        const int n = std::min(stq::kMaxTable, L->H - first);
+        fill_table(*p, L, ord, first, n, 0);
+        p->ntiles = B * n;
+        const stq_status st = from_cuda(stq::launch_init_generic(*p, (cudaStream_t)stream));
+        if (st != STQ_OK) return st;
+    }
+    return STQ_OK;
+}
+
+stq_status stq_dequantize(const stq_layout *L, const void *pool, int32_t pool_slots, const int32_t *slots, int32_t B,
+                          float *S_out, int32_t *dev_status, void *stream)
+{
+    if (!L || B < 0 || pool_slots < 0) return STQ_ERR_INVALID_ARG;
+    if (B == 0) return STQ_OK;
+    if (!pool || !slots || !S_out || !aligned(pool, 128) || !aligned(S_out, 4)) return STQ_ERR_INVALID_ARG;
+    auto p = new_params();
+    if (!p) return STQ_ERR_INVALID_ARG;
+    p->pool = static_cast<uint8_t *>(const_cast<void *>(pool));
+    p->slots = slots;
+    p->status = dev_status;
+    p->req_bytes = L->req_bytes;
+    p->pool_slots = pool_slots;
+    p->B = B;
+    p->head_count = L->H;
+    p->dk = L->dk;
+    p->dv = L->dv;
+    p->S_out = S_out;
+    const std::vector<int> ord = order_by_size(L, 0, L->H);
+    for (int first = 0; first < L->H; first += stq::kMaxTable) {
+        const int n = std::min(stq::kMaxTable, L->H - first);
+        fill_table(*p, L, ord, first, n, 0);
+        p->ntiles = B * n;
+        const stq_status st = from_cuda(stq::launch_dequant_generic(*p, (cudaStream_t)stream));
+        if (st != STQ_OK) return st;
+    }
+    return STQ_OK;
+}
+
+stq_status stq_decode_step(const stq_layout *L, void *pool, int32_t pool_slots, const int32_t *slots, int32_t B,
+                           int32_t head_begin, int32_t head_count, const void *q, const void *k, const void *v,
+                           const float *beta, const float *alpha, const float *w, float *o, int32_t *dev_status,
+                           void *stream)
+{
+    if (!L || B < 0 || pool_slots < 0 || head_begin < 0 || head_count < 0 || head_begin > L->H ||
+        head_count > L->H - head_begin)
+        return STQ_ERR_INVALID_ARG;
+    if (B == 0 || head_count == 0) return STQ_OK;
+    if (!pool || !slots || !q || !k || !v || !beta || !alpha || !w || !o) return STQ_ERR_INVALID_ARG;
+    if (!aligned(pool, 128) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(alpha, 16) ||
+        !aligned(w, 16) || !aligned(beta, 4) || !aligned(o, 16))
+        return STQ_ERR_INVALID_ARG;
+    if (B > 2147483647 / head_count) return STQ_ERR_UNSUPPORTED;
+    auto p = new_params();
+    if (!p) return STQ_ERR_INVALID_ARG;
+    p->pool = static_cast<uint8_t *>(pool);
+    p->status = dev_status;
+    p->req_bytes = L->req_bytes;
+    p->pool_slots = pool_slots;
+    p->head_count = head_count;
+    p->dk = L->dk;
+    p->dv = L->dv;
+    p->gate = L->gate;
+    p->w = w;
+    const int in_bf16 = L->in_dtype == STQ_BF16;
+    const bool tuned = L->dk == 128;
+    const int maxb = tuned ? stq::decode_d128_max_requests() : 65535;
+    const std::vector<int> ord = order_by_size(L, head_begin, head_count);
+    const size_t in_sz = in_bf16 ? 2 : 4;
+    const int na = L->gate == STQ_GATE_SCALAR ? 1 : L->dk;
+    for (int b0 = 0; b0 < B; b0 += maxb) {
+        const int nb = std::min(maxb, B - b0);
+        // requests [b0, b0+nb): shift every per-request array
+        const size_t rq = (size_t)b0 * head_count;
+        p->slots = slots + b0;
+        p->B = nb;
+        p->q = static_cast<const uint8_t *>(q) + rq * L->dk * in_sz;
+        p->k = static_cast<const uint8_t *>(k) + rq * L->dk * in_sz;
+        p->v = static_cast<const uint8_t *>(v) + rq * L->dv * in_sz;
+        p->beta = beta + rq;
+        p->alpha = alpha + rq * na;
+        p->o = o + rq * L->dv;
+        for (int first = 0; first < head_count; first += stq::kMaxTable) {
+            const int n = std::min(stq::kMaxTable, head_count - first);
+            fill_table(*p, L, ord, first, n, head_begin);
+            p->ntiles = nb * n;
+            const cudaError_t e = tuned ? stq::launch_decode_d128(*p, in_bf16, (cudaStream_t)stream)
+                                        : stq::launch_decode_generic(*p, in_bf16, (cudaStream_t)stream);
+            if (e != cudaSuccess) return STQ_ERR_CUDA;
+        }
+    }
+    return STQ_OK;
+}
+
+size_t stq_prefill_workspace_bytes(const stq_layout *L, int32_t B, int32_t T, int32_t chunk)
+{
+    if (!L || B < 0 || T < 0 || chunk < 1) return 0;
+    return 0;  // the sequential prefill carries its state in shared memory
+}
+
+stq_status stq_prefill_chunk(const stq_layout *L, void *pool, int32_t pool_slots, const int32_t *slots, int32_t B,
+                             int32_t T, int32_t chunk, const void *q, const void *k, const void *v, const float *beta,
+                             const float *alpha, const float *w, float *o, void *workspace, size_t workspace_bytes,
+                             int32_t *dev_status, void *stream)
+{
+    if (!L || B < 0 || T < 0 || chunk < 1 || pool_slots < 0) return STQ_ERR_INVALID_ARG;
+    if (B == 0 || T == 0) return STQ_OK;
+    if (!pool || !slots || !q || !k || !v || !beta || !alpha || !w || !o) return STQ_ERR_INVALID_ARG;
+    const size_t need = stq_prefill_workspace_bytes(L, B, T, chunk);
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256))) return STQ_ERR_INVALID_ARG;
+    if (B > 2147483647 / L->H) return STQ_ERR_UNSUPPORTED;
+    if (!aligned(pool, 128) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(w, 16) ||
+        !aligned(o, 16) || !aligned(beta, 4) || !aligned(alpha, 4))
+        return STQ_ERR_INVALID_ARG;
+    if (L->H > stq::kMaxTable) return STQ_ERR_UNSUPPORTED;
+    auto p = new_params();
+    if (!p) return STQ_ERR_INVALID_ARG;
+    p->pool = static_cast<uint8_t *>(pool);
+    p->slots = slots;
+    p->status = dev_status;
+    p->req_bytes = L->req_bytes;
+    p->pool_slots = pool_slots;
+    p->B = B;
+    p->head_count = L->H;
+    p->dk = L->dk;
+    p->dv = L->dv;
+    p->gate = L->gate;
+    p->q = q;
+    p->k = k;
+    p->v = v;
+    p->beta = beta;
+    p->alpha = alpha;
+    p->w = w;
+    p->o = o;
+    std::vector<int> ord(L->H);
+    for (int h = 0; h < L->H; ++h) ord[h] = h;
+    fill_table(*p, L, ord, 0, L->H, 0);
+    p->ntiles = B * L->H;
+    return from_cuda(stq::launch_prefill_seq(*p, L->in_dtype == STQ_BF16, T, chunk, (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,167 @@
+// stq_internal.cuh -- internal declarations shared by the host code and the kernels of the
+// quantized-state library (not part of the public ABI; see include/stq.h for the contract).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace stq {
+
+// ------------------------------------------------------------------------------------------
+// Status bits OR-ed into the caller's device status word: (1 << stq_status code).
+// ------------------------------------------------------------------------------------------
+constexpr int32_t kFlagNonfinite = 1 << 4;
+constexpr int32_t kFlagTimeout = 1 << 5;
+constexpr int32_t kFlagBounds = 1 << 6;
+
+// A bounded wait gives up after this many SM clock cycles (~2 s at 2 GHz).
+constexpr long long kWaitTimeoutCycles = 4000000000LL;
+
+// ------------------------------------------------------------------------------------------
+// Head-block layout (independent restatement of the byte layout in include/stq.h).
+// ------------------------------------------------------------------------------------------
+__host__ __device__ constexpr uint32_t round_up_u32(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+__host__ __device__ constexpr uint32_t codes_bytes(int bits, int dk, int dv)
+{
+    return (uint32_t)(((uint64_t)bits * dk * dv + 7) / 8);
+}
+__host__ __device__ constexpr uint32_t scale_offset(int bits, int dk, int dv)
+{
+    return round_up_u32(codes_bytes(bits, dk, dv), 16);
+}
+__host__ __device__ constexpr uint32_t head_block_bytes(int bits, int dk, int dv)
+{
+    return bits == 16 ? round_up_u32(2u * dk * dv, 128)
+                      : round_up_u32(scale_offset(bits, dk, dv) + 4u * dk + 4u * dv, 128);
+}
+
+// One entry of the per-launch head table, in processing order (largest blocks first).
+struct TileEntry {
+    uint32_t off;   // byte offset of the head block inside a request block
+    uint32_t info;  // bits 0..15: head index relative to the call's head_begin; 16..23: width
+};
+__host__ __device__ inline int entry_head(const TileEntry &e) { return (int)(e.info & 0xffffu); }
+__host__ __device__ inline int entry_bits(const TileEntry &e) { return (int)((e.info >> 16) & 0xffu); }
+
+// Head table capacity of one launch; larger head ranges are split into several launches.
+constexpr int kMaxTable = 3072;
+
+struct TileParams {
+    uint8_t *pool;
+    const int32_t *slots;
+    int32_t *status;
+    uint64_t req_bytes;
+    int32_t pool_slots;
+    int32_t B;           // requests of this launch
+    int32_t npos;        // heads of this launch (entries of the table)
+    int32_t ntiles;      // B * npos
+    int32_t head_count;  // heads of the call (row stride of the per-head input arrays)
+    int32_t dk, dv;
+    int32_t gate;
+    // decode / prefill inputs (indexed by request and call-relative head)
+    const void *q, *k, *v;
+    const float *beta, *alpha, *w;
+    float *o;
+    // init / dequantize
+    const float *S0;
+    float *S_out;
+    TileEntry table[kMaxTable];
+};
+
+// ------------------------------------------------------------------------------------------
+// Kernel launchers (host side; defined next to their kernels). Each returns a cudaError_t.
+// ------------------------------------------------------------------------------------------
+cudaError_t launch_init_generic(const TileParams &p, cudaStream_t s);
+cudaError_t launch_dequant_generic(const TileParams &p, cudaStream_t s);
+cudaError_t launch_decode_generic(const TileParams &p, int in_bf16, cudaStream_t s);
+cudaError_t launch_decode_d128(const TileParams &p, int in_bf16, cudaStream_t s);
+cudaError_t launch_prefill_seq(const TileParams &p, int in_bf16, int T, int chunk, cudaStream_t s);
+int decode_d128_max_requests();
+
+// ------------------------------------------------------------------------------------------
+// Device helpers
+// ------------------------------------------------------------------------------------------
+#ifdef __CUDACC__
+
+template <int IN_BF16>
+__device__ __forceinline__ float load_in(const void *base, size_t idx)
+{
+    if constexpr (IN_BF16)
+        return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base)[idx]);
+    else
+        return reinterpret_cast<const float *>(base)[idx];
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after kWaitTimeoutCycles. Returns false on
+// timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long start = clock64();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (clock64() - start > kWaitTimeoutCycles) return false;
+    }
+}
+
+// Bulk copy global -> this CTA's shared memory, completing `bytes` on the mbarrier.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void flag(int32_t *status, int32_t bits)
+{
+    if (status) atomicOr(status, bits);
+}
+
+#endif  // __CUDACC__
+
+}  // namespace stq

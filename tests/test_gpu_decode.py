@@ -1,0 +1,330 @@
+"""GPU parity of the decode step, init and dequantize against the CPU oracle (needs a B200).
+
+Teacher-forced protocol: the oracle's own trajectory is authoritative. Before each checked step
+the oracle's pre-step pool bytes are uploaded into the GPU pool, one GPU step runs through the C
+ABI, and the GPU's post-step bytes and readout are compared with the oracle's step from the same
+bytes and the same inputs (rules in tests/_parity.py).
+"""
+import numpy as np
+import pytest
+import torch
+
+from _parity import Tally, as_f64, compare_block, compare_o, oracle_pool, tile_bytes
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def stq():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for the gpu tests")
+    import quantized_linear_attention_stq_b200 as m
+
+    m.lib()  # fails loudly if libstq.so is missing
+    return m
+
+
+def _wl(name, **changes):
+    from quantized_linear_attention_stq_b200 import workloads as wl
+
+    return wl.scaled(wl.WORKLOADS[name], **changes)
+
+
+def _oracle_init(orc, wl_, bits, S0, w):
+    """Oracle init of every tile: S0 [B,H,d,d] and w [H,d] as torch CPU tensors."""
+    B, H, d = S0.shape[0], S0.shape[1], S0.shape[2]
+    blocks = []
+    for r in range(B):
+        row = []
+        for h in range(H):
+            blk, _, _, st = orc.quantize(bits[h], as_f64(S0[r, h]), as_f64(w[h]))
+            assert st == orc.OK
+            row.append(blk)
+        blocks.append(row)
+    return oracle_pool(orc, bits, d, blocks)
+
+
+def _decode_teacher_forced(stq, orc, wl_, bits, steps, head_begin=0, head_count=None, slots_perm=True, seed_tok=0):
+    """Run `steps` teacher-forced steps; returns the tally."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    B, H, d = wl_.batch, wl_.heads, wl_.d
+    hc = H - head_begin if head_count is None else head_count
+    lay = stq.Layout(bits, d, gate=wl_.gate, in_dtype=wl_.in_dtype)
+    w = wlm.impact_weights(wl_)
+    S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(B)])
+    opool = _oracle_init(orc, wl_, bits, S0, w)
+    nslots = B + 3
+    total = lay.bytes_per_request
+    # requests live at permuted slots of a larger pool (slot != request index)
+    slot_of = (np.random.default_rng(5).permutation(nslots)[:B] if slots_perm else np.arange(B)).astype(np.int32)
+    gpool = torch.zeros(nslots * total, dtype=torch.uint8, device=DEV)
+    slots = torch.from_numpy(slot_of).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    tally = Tally()
+    hs = slice(head_begin, head_begin + hc)
+    w_call = w[hs].contiguous()
+    for t in range(steps):
+        inp = wlm.decode_inputs(wl_, seed_tok + t)
+        inp_h = {n: x[:, hs].contiguous() for n, x in inp.items()}
+        # upload the oracle's pre-step state into the permuted slots
+        host = np.zeros(nslots * total, dtype=np.uint8)
+        for r in range(B):
+            host[slot_of[r] * total:(slot_of[r] + 1) * total] = opool[r * total:(r + 1) * total]
+        gpool.copy_(torch.from_numpy(host).to(DEV))
+        o = torch.zeros(B, hc, d, dtype=torch.float32, device=DEV)
+        g = {n: x.to(DEV) for n, x in inp_h.items()}
+        stq.decode_step(lay, gpool, slots, g["q"], g["k"], g["v"], g["beta"], g["alpha"], w_call.to(DEV), o,
+                        head_begin=head_begin, status=status)
+        torch.cuda.synchronize()
+        assert status.item() == 0, stq.status_flags(status)
+        gp = gpool.cpu().numpy()
+        og = o.cpu().numpy()
+        new_opool = opool.copy()
+        for r in range(B):
+            for h in range(H):
+                ref_blk = tile_bytes(orc, opool, bits, d, r, h)
+                got_blk = tile_bytes(orc, gp, bits, d, int(slot_of[r]), h)
+                if not (head_begin <= h < head_begin + hc):
+                    assert np.array_equal(got_blk, ref_blk), f"head {h} outside the call changed"
+                    continue
+                hr = h - head_begin
+                alpha = inp["alpha"][r, h].double().numpy()
+                res = orc.decode_step(bits[h], wl_.gate, ref_blk, as_f64(inp["q"][r, h]), as_f64(inp["k"][r, h]),
+                                      as_f64(inp["v"][r, h]), float(inp["beta"][r, h]), alpha, as_f64(w[h]), d, d)
+                assert res["status"] == orc.OK
+                compare_block(orc, bits[h], d, got_blk, res["block"], res["tie"], tally, f"step {t} req {r} head {h}")
+                compare_o(og[r, hr], res["o"], tally, f"o step {t} req {r} head {h}")
+                offs, _ = orc.request_layout(bits, d, d)
+                new_opool[r * total + offs[h]: r * total + offs[h] + res["block"].size] = res["block"]
+        opool = new_opool
+    tally.check_budget()
+    return tally
+
+
+def test_pr1_d16_sixty_four_steps(stq, orc):
+    """1 request x 1 head, d = 16, 6-bit, fp32 inputs, every one of the 64 steps."""
+    wl_ = _wl("pr1_d16_6bit")
+    t = _decode_teacher_forced(stq, orc, wl_, [6], 64)
+    assert t.codes == 64 * 256
+
+
+@pytest.mark.parametrize("bits", [4, 6, 8, 16])
+def test_layer_d128_uniform_width(stq, orc, bits):
+    """The 48-head layer workload (d = 128, bf16 inputs, scalar gate) at 5 requests x 12 heads."""
+    wl_ = _wl("layer48_b8_4bit", batch=5, heads=12, bits=bits)
+    _decode_teacher_forced(stq, orc, wl_, [bits] * 12, 4)
+
+
+def test_mixed_widths_with_pivots_ragged(stq, orc):
+    """Mixed 4/6/8/16 heads in one launch, 7 requests (ragged), fp32 inputs."""
+    wl_ = _wl("layer48_b8_4bit", batch=7, heads=9, bits=None, in_dtype=torch.float32)
+    bits = [4, 16, 6, 8, 4, 6, 16, 8, 4]
+    _decode_teacher_forced(stq, orc, wl_, bits, 3)
+
+
+@pytest.mark.parametrize("gate", [1, 2])
+def test_channel_gates(stq, orc, gate):
+    wl_ = _wl("channel32_b128_4bit", batch=3, heads=6, gate=gate)
+    _decode_teacher_forced(stq, orc, wl_, [4, 8, 6, 16, 4, 6], 3)
+
+
+@pytest.mark.parametrize("d", [32, 64])
+def test_small_heads(stq, orc, d):
+    wl_ = _wl("layer48_b8_4bit", batch=3, heads=5, d=d, in_dtype=torch.float32)
+    _decode_teacher_forced(stq, orc, wl_, [4, 6, 8, 16, 6], 3)
+
+
+def test_head_subset_leaves_other_heads_alone(stq, orc):
+    wl_ = _wl("layer48_b8_4bit", batch=3, heads=10, bits=None)
+    bits = [4, 6, 8, 16, 4, 6, 8, 16, 4, 6]
+    _decode_teacher_forced(stq, orc, wl_, bits, 2, head_begin=3, head_count=4)
+
+
+def test_many_requests_split_launches(stq, orc):
+    """More requests than one launch caches (1024): the host splits the call."""
+    wl_ = _wl("layer48_b8_4bit", batch=1030, heads=1, bits=4)
+    _decode_teacher_forced(stq, orc, wl_, [4], 1, slots_perm=False)
+
+
+# ------------------------------------------------------------------------------------------------
+# init and dequantize
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d", [16, 128])
+def test_init_matches_oracle(stq, orc, d):
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl_ = _wl("full2304_b70_mixed", batch=3, heads=8, d=d)
+    bits = [4, 6, 8, 16, 8, 6, 4, 16]
+    lay = stq.Layout(bits, d, in_dtype=torch.bfloat16)
+    w = wlm.impact_weights(wl_)
+    S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(3)])
+    ref = _oracle_init(orc, wl_, bits, S0, w)
+    pool = lay.alloc_pool(3)
+    slots = torch.arange(3, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stq.init_state(lay, pool, slots, S0.to(DEV), w.to(DEV), status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    gp = pool.cpu().numpy()
+    tally = Tally()
+    for r in range(3):
+        for h in range(8):
+            _, _, tie, _ = orc.quantize(bits[h], as_f64(S0[r, h]), as_f64(w[h]))
+            compare_block(orc, bits[h], d, tile_bytes(orc, gp, bits, d, r, h), tile_bytes(orc, ref, bits, d, r, h),
+                          tie, tally, f"init req {r} head {h}")
+    tally.check_budget()
+
+
+def test_dequantize_matches_oracle(stq, orc):
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl_ = _wl("full2304_b70_mixed", batch=2, heads=6)
+    bits = [4, 6, 8, 16, 4, 8]
+    lay = stq.Layout(bits, 128)
+    w = wlm.impact_weights(wl_)
+    S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(2)])
+    ref = _oracle_init(orc, wl_, bits, S0, w)
+    pool = torch.from_numpy(ref).to(DEV)
+    slots = torch.tensor([1, 0], dtype=torch.int32, device=DEV)
+    out = torch.zeros(2, 6, 128, 128, device=DEV)
+    stq.dequantize(lay, pool, slots, out)
+    got = out.cpu().double().numpy()
+    for r, slot in enumerate([1, 0]):
+        for h in range(6):
+            S = orc.dequantize(bits[h], 128, 128, tile_bytes(orc, ref, bits, 128, slot, h))
+            assert np.all(np.abs(got[r, h] - S) <= 2.0 ** -22 * np.abs(S))
+
+
+# ------------------------------------------------------------------------------------------------
+# edge cases and device status
+# ------------------------------------------------------------------------------------------------
+
+def test_zero_state_first_write(stq, orc):
+    """A zero state (scales 1, codes 0) takes a rank-1 write on its first step."""
+    lay = stq.Layout([6, 4], 128, in_dtype=torch.float32)
+    w = torch.ones(2, 128)
+    pool = lay.alloc_pool(1)
+    slots = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stq.init_state(lay, pool, slots, torch.zeros(1, 2, 128, 128, device=DEV), w.to(DEV))
+    ref0 = pool.cpu().numpy().copy()
+    rng = np.random.default_rng(0)
+    q, k, v = (torch.from_numpy(rng.standard_normal((1, 2, 128))).float() for _ in range(3))
+    beta = torch.full((1, 2), 0.5)
+    alpha = torch.full((1, 2), 0.9)
+    o = torch.zeros(1, 2, 128, device=DEV)
+    stq.decode_step(lay, pool, slots, q.to(DEV), k.to(DEV), v.to(DEV), beta.to(DEV), alpha.to(DEV), w.to(DEV), o)
+    gp = pool.cpu().numpy()
+    tally = Tally()
+    for h, b in enumerate([6, 4]):
+        blk = tile_bytes(orc, ref0, [6, 4], 128, 0, h)
+        assert not orc.codes(b, 128, 128, blk).any()
+        res = orc.decode_step(b, 0, blk, as_f64(q[0, h]), as_f64(k[0, h]), as_f64(v[0, h]), 0.5, 0.9,
+                              np.ones(128), 128, 128)
+        compare_block(orc, b, 128, tile_bytes(orc, gp, [6, 4], 128, 0, h), res["block"], res["tie"], tally)
+        compare_o(o[0, h].cpu().numpy(), res["o"], tally)
+
+
+def test_out_of_range_slot_is_flagged_and_skipped(stq):
+    lay = stq.Layout([4, 8], 128, in_dtype=torch.float32)
+    pool = lay.alloc_pool(2)
+    pool.fill_(7)
+    before = pool.clone()
+    slots = torch.tensor([5, -1], dtype=torch.int32, device=DEV)
+    B, H = 2, 2
+    z = torch.zeros(B, H, 128, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stq.decode_step(lay, pool, slots, z, z, z, torch.zeros(B, H, device=DEV), torch.ones(B, H, device=DEV),
+                    torch.ones(H, 128, device=DEV), torch.zeros(B, H, 128, device=DEV), status=status)
+    torch.cuda.synchronize()
+    assert status.item() & (1 << stq.api.STQ_ERR_BOUNDS)
+    assert torch.equal(pool, before)
+
+
+def test_nonfinite_input_is_flagged(stq, orc):
+    lay = stq.Layout([6, 16], 128, in_dtype=torch.float32)
+    pool = lay.alloc_pool(1)
+    slots = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stq.init_state(lay, pool, slots, torch.randn(1, 2, 128, 128, device=DEV), torch.ones(2, 128, device=DEV))
+    v = torch.full((1, 2, 128), float("inf"), device=DEV)
+    k = torch.nn.functional.normalize(torch.randn(1, 2, 128, device=DEV), dim=-1)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stq.decode_step(lay, pool, slots, k, k, v, torch.full((1, 2), 0.5, device=DEV), torch.full((1, 2), 0.9, device=DEV),
+                    torch.ones(2, 128, device=DEV), torch.zeros(1, 2, 128, device=DEV), status=status)
+    torch.cuda.synchronize()
+    assert status.item() & (1 << stq.api.STQ_ERR_NONFINITE)
+
+
+def test_empty_calls_are_noops(stq):
+    lay = stq.Layout([4], 128)
+    pool = lay.alloc_pool(1)
+    e = torch.zeros(0, 1, 128, dtype=torch.bfloat16, device=DEV)
+    stq.decode_step(lay, pool, torch.zeros(0, dtype=torch.int32, device=DEV), e, e, e,
+                    torch.zeros(0, 1, device=DEV), torch.zeros(0, 1, device=DEV), torch.ones(1, 128, device=DEV),
+                    torch.zeros(0, 1, 128, device=DEV))
+    torch.cuda.synchronize()
+    assert not pool.any()
+
+
+def test_step_is_deterministic(stq):
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl_ = _wl("full2304_b70_mixed", batch=9, heads=40)
+    bits = wlm.head_bits(wlm.WORKLOADS["full2304_b70_mixed"])[:40]
+    lay = stq.Layout(bits, 128)
+    w = wlm.impact_weights(wl_).to(DEV)
+    pool = lay.alloc_pool(9)
+    slots = torch.arange(9, dtype=torch.int32, device=DEV)
+    stq.init_state(lay, pool, slots, torch.stack([wlm.initial_state(wl_, r, DEV) for r in range(9)]), w)
+    inp = wlm.decode_inputs(wl_, 0, DEV)
+    outs = []
+    for _ in range(2):
+        p = pool.clone()
+        o = torch.zeros(9, 40, 128, device=DEV)
+        stq.decode_step(lay, p, slots, inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], w, o)
+        outs.append((p, o))
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+def test_free_running_error_statistics_match_oracle(stq, orc):
+    """Over 48 free-running steps, the GPU and oracle trajectories each drift from the unquantized
+    fp64 recurrence by the same amount (mean and p99 of the readout error within 10%)."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl_ = _wl("layer48_b8_4bit", batch=2, heads=4, bits=6, in_dtype=torch.float32)
+    bits = [6, 4, 8, 6]
+    B, H, d = 2, 4, 128
+    lay = stq.Layout(bits, d, in_dtype=torch.float32)
+    w = wlm.impact_weights(wl_)
+    S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(B)])
+    opool = _oracle_init(orc, wl_, bits, S0, w)
+    gpool = torch.from_numpy(opool.copy()).to(DEV)
+    slots = torch.arange(B, dtype=torch.int32, device=DEV)
+    Sref = {(r, h): orc.dequantize(bits[h], d, d, tile_bytes(orc, opool, bits, d, r, h)) for r in range(B) for h in range(H)}
+    err_g, err_o = [], []
+    total = lay.bytes_per_request
+    offs, _ = orc.request_layout(bits, d, d)
+    for t in range(48):
+        inp = wlm.decode_inputs(wl_, t)
+        o = torch.zeros(B, H, d, device=DEV)
+        stq.decode_step(lay, gpool, slots, *(inp[n].to(DEV) for n in ("q", "k", "v", "beta", "alpha")), w.to(DEV), o)
+        og = o.cpu().numpy()
+        for r in range(B):
+            for h in range(H):
+                a = float(inp["alpha"][r, h])
+                q, k, v = (as_f64(inp[n][r, h]) for n in ("q", "k", "v"))
+                Sn, oref = orc.update(0, Sref[(r, h)], q, k, v, float(inp["beta"][r, h]), a)
+                Sref[(r, h)] = Sn
+                blk = tile_bytes(orc, opool, bits, d, r, h)
+                res = orc.decode_step(bits[h], 0, blk, q, k, v, float(inp["beta"][r, h]), a, as_f64(w[h]), d, d)
+                opool[r * total + offs[h]: r * total + offs[h] + blk.size] = res["block"]
+                n = np.linalg.norm(oref)
+                err_o.append(np.linalg.norm(res["o"] - oref) / n)
+                err_g.append(np.linalg.norm(og[r, h] - oref) / n)
+    err_g, err_o = np.array(err_g), np.array(err_o)
+    assert abs(err_g.mean() / err_o.mean() - 1) < 0.10
+    assert abs(np.percentile(err_g, 99) / np.percentile(err_o, 99) - 1) < 0.10

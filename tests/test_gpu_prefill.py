@@ -1,0 +1,112 @@
+"""GPU parity of the chunked prefill against the oracle's sequential prefill (needs a B200).
+
+Teacher-forced per chunk: the oracle's pre-chunk pool is uploaded, one single-chunk GPU call runs,
+and the GPU's requantized state and every token's readout are compared with the oracle's chunk
+from the same bytes. A multi-chunk call must be bit-identical to the same chunks issued one call
+each.
+"""
+import numpy as np
+import pytest
+import torch
+
+from _parity import Tally, as_f64, compare_block, compare_o, oracle_pool, tile_bytes
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def stq():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for the gpu tests")
+    import quantized_linear_attention_stq_b200 as m
+
+    m.lib()
+    return m
+
+
+def _setup(orc, B, bits, d=128, dtype=torch.bfloat16):
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl_ = wlm.scaled(wlm.WORKLOADS["prefill16_b16_6bit"], batch=B, heads=len(bits), d=d, in_dtype=dtype)
+    w = wlm.impact_weights(wl_)
+    blocks = []
+    for r in range(B):
+        S0 = wlm.initial_state(wl_, r)
+        row = []
+        for h, b in enumerate(bits):
+            blk, _, _, st = orc.quantize(b, as_f64(S0[h]), as_f64(w[h]))
+            assert st == orc.OK
+            row.append(blk)
+        blocks.append(row)
+    return wl_, w, oracle_pool(orc, bits, d, blocks)
+
+
+def _oracle_chunk(orc, pool, bits, d, r, h, inp, t0, T, w, chunk):
+    blk = tile_bytes(orc, pool, bits, d, r, h)
+    sl = slice(t0, t0 + T)
+    return orc.prefill_seq(bits[h], 0, blk, as_f64(inp["q"][r, h, sl]), as_f64(inp["k"][r, h, sl]),
+                           as_f64(inp["v"][r, h, sl]), as_f64(inp["beta"][r, h, sl]), as_f64(inp["alpha"][r, h, sl]),
+                           as_f64(w[h]), chunk, d, d)
+
+
+@pytest.mark.parametrize("T", [64, 37, 1])
+def test_single_chunk_teacher_forced(stq, orc, T):
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    bits = [6, 4, 8, 16]
+    B, d = 3, 128
+    wl_, w, opool = _setup(orc, B, bits)
+    lay = stq.Layout(bits, d, in_dtype=torch.bfloat16)
+    inp = wlm.prefill_inputs(wl_, 0, T)
+    gpool = torch.from_numpy(opool.copy()).to(DEV)
+    slots = torch.arange(B, dtype=torch.int32, device=DEV)
+    o = torch.zeros(B, len(bits), T, d, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    ws_n = stq.prefill_workspace_bytes(lay, B, T, 64)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=DEV)
+    stq.prefill_chunk(lay, gpool, slots, *(inp[n].to(DEV) for n in ("q", "k", "v", "beta", "alpha")), w.to(DEV), o,
+                      chunk=64, workspace=ws, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    gp = gpool.cpu().numpy()
+    og = o.cpu().numpy()
+    tally = Tally()
+    for r in range(B):
+        for h in range(len(bits)):
+            res = _oracle_chunk(orc, opool, bits, d, r, h, inp, 0, T, w, 64)
+            assert res["status"] == orc.OK
+            compare_block(orc, bits[h], d, tile_bytes(orc, gp, bits, d, r, h), res["block"], res["tie"], tally,
+                          f"req {r} head {h}")
+            for t in range(T):
+                compare_o(og[r, h, t], res["o"][t], tally, f"token {t} req {r} head {h}")
+    tally.check_budget()
+
+
+def test_multi_chunk_equals_single_chunk_calls(stq, orc):
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    bits = [6, 8, 4]
+    B, d, T, C = 2, 128, 150, 64
+    wl_, w, opool = _setup(orc, B, bits)
+    lay = stq.Layout(bits, d, in_dtype=torch.bfloat16)
+    inp = {n: x.to(DEV) for n, x in wlm.prefill_inputs(wl_, 0, T).items()}
+    slots = torch.tensor([1, 0], dtype=torch.int32, device=DEV)
+    wd = w.to(DEV)
+    ws = torch.empty(max(stq.prefill_workspace_bytes(lay, B, T, C), 1), dtype=torch.uint8, device=DEV)
+    p_full = torch.from_numpy(opool.copy()).to(DEV)
+    o_full = torch.zeros(B, 3, T, d, device=DEV)
+    stq.prefill_chunk(lay, p_full, slots, inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], wd, o_full,
+                      chunk=C, workspace=ws)
+    p_seq = torch.from_numpy(opool.copy()).to(DEV)
+    outs = []
+    for c0 in range(0, T, C):
+        sl = slice(c0, min(c0 + C, T))
+        part = {n: x[:, :, sl].contiguous() for n, x in inp.items()}
+        o_part = torch.zeros(B, 3, sl.stop - sl.start, d, device=DEV)
+        stq.prefill_chunk(lay, p_seq, slots, part["q"], part["k"], part["v"], part["beta"], part["alpha"], wd, o_part,
+                          chunk=C, workspace=ws)
+        outs.append(o_part)
+    torch.cuda.synchronize()
+    assert torch.equal(p_full, p_seq)
+    assert torch.equal(o_full, torch.cat(outs, dim=2))
