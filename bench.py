@@ -255,6 +255,8 @@ def run_ours(args):
     dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(dev)
     wl = wlm.WORKLOADS[args.workload]
+    if args.batch:
+        wl = wlm.scaled(wl, batch=args.batch)
     B, H, d = wl.batch, wl.heads, wl.d
     bits = wlm.head_bits(wl)
     lay = stq.Layout(bits, d, gate=wl.gate, in_dtype=wl.in_dtype)
@@ -429,6 +431,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="requests per GPU (default: the workload's)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

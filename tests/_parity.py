@@ -6,7 +6,13 @@ The parity rule (codes, scales, readout):
     stay below 1e-4 of the codes checked;
   * stored fp32 scales within 2e-3 relative (expected: a few fp32 ulps);
   * readout o within 2e-3 of max|o| of the oracle's fp64 readout rounded to fp32;
-  * FP16 pivot values equal, or one fp16 quantum apart where the oracle flags a near-tie.
+  * FP16 pivot values are floating-point state, compared as such: every value within one fp16
+    quantum of the oracle's plus the fp32 evaluation error of the update, 2^-18 * M_ij, where
+    M_ij = |alpha| |S_ij| + beta |k_i| (|v_j| + |alpha| sum_l |k_l| |S_lj|) is the magnitude of
+    the terms that form S'_ij (an element born of cancellation has a tiny fp16 quantum but an
+    fp32 error set by those terms); and at most 1e-3 of the values not bit-identical (a wrong
+    rounding mode or a dropped term would move far more), per fp32 update carried (a prefill
+    chunk of T tokens carries T).
 Inputs always flow from the generator (or the oracle) to the GPU, never back into the oracle.
 """
 from __future__ import annotations
@@ -19,6 +25,7 @@ import torch
 CODE_TIE_BUDGET = 1e-4
 SCALE_RTOL = 2e-3
 O_TOL = 2e-3
+PIVOT_DIFF_BUDGET = 1e-3
 
 
 @dataclasses.dataclass
@@ -28,13 +35,14 @@ class Tally:
     max_scale_rel: float = 0.0
     max_o_rel: float = 0.0
     pivot_values: int = 0
-    pivot_flips: int = 0
+    pivot_diffs: int = 0
+    updates_per_check: int = 1   # fp32 updates a pivot state carried since the oracle's bytes
 
     def check_budget(self):
-        total = self.codes + self.pivot_values
-        flips = self.tie_flips + self.pivot_flips
-        assert total > 0
-        assert flips <= CODE_TIE_BUDGET * total, f"{flips} tie flips in {total} codes"
+        assert self.codes + self.pivot_values > 0
+        assert self.tie_flips <= CODE_TIE_BUDGET * self.codes, f"{self.tie_flips} tie flips in {self.codes} codes"
+        assert self.pivot_diffs <= PIVOT_DIFF_BUDGET * self.updates_per_check * self.pivot_values, \
+            f"{self.pivot_diffs} of {self.pivot_values} fp16 pivot values differ"
 
 
 def oracle_pool(orc, head_bits, d, blocks_per_request):
@@ -54,17 +62,34 @@ def tile_bytes(orc, pool, head_bits, d, slot, h):
     return np.asarray(pool[start: start + n])
 
 
-def compare_block(orc, bits, d, got, ref_block, ref_tie, tally: Tally, what=""):
+def update_magnitude(S, k, v, beta, alpha):
+    """M_ij of the pivot tolerance: magnitude of the terms of one update of S (fp64)."""
+    a = float(np.max(np.abs(alpha)))
+    S, k, v = np.abs(S), np.abs(np.asarray(k, dtype=np.float64)), np.abs(np.asarray(v, dtype=np.float64))
+    return a * S + beta * k[:, None] * (v[None, :] + a * (k @ S)[None, :])
+
+
+def fp16_quantum(x):
+    ax = np.maximum(np.abs(x), 2.0 ** -14)
+    return 2.0 ** (np.floor(np.log2(ax)) - 10)
+
+
+def compare_block(orc, bits, d, got, ref_block, ref_tie, tally: Tally, what="", err_scale=None):
     got = np.asarray(got, dtype=np.uint8)
     ref_block = np.asarray(ref_block, dtype=np.uint8)
     if bits == 16:
-        g = orc.pivot_values(d, d, got).astype(np.int32)
-        r = orc.pivot_values(d, d, ref_block).astype(np.int32)
-        diff = np.abs(g - r)
-        bad = (diff > 1) | ((diff == 1) & ~ref_tie)
-        assert not bad.any(), f"{what}: {int(bad.sum())} fp16 values differ off a tie"
-        tally.pivot_values += g.size
-        tally.pivot_flips += int((diff == 1).sum())
+        gb = orc.pivot_values(d, d, got)
+        rb = orc.pivot_values(d, d, ref_block)
+        gv = gb.view(np.float16).astype(np.float64)
+        rv = rb.view(np.float16).astype(np.float64)
+        tol = fp16_quantum(rv) + (0.0 if err_scale is None else 2.0 ** -18 * err_scale)
+        bad = ~(np.abs(gv - rv) <= tol)
+        if bad.any():
+            i, j = np.argwhere(bad)[0]
+            raise AssertionError(f"{what}: {int(bad.sum())} fp16 values outside tolerance, first at ({i},{j}): "
+                                 f"gpu {gv[i, j]!r} oracle {rv[i, j]!r} tol {tol[i, j]!r}")
+        tally.pivot_values += gb.size
+        tally.pivot_diffs += int((gb != rb).sum())
         return
     Qg = orc.codes(bits, d, d, got)
     Qr = orc.codes(bits, d, d, ref_block)

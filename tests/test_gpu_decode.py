@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from _parity import Tally, as_f64, compare_block, compare_o, oracle_pool, tile_bytes
+from _parity import Tally, as_f64, compare_block, compare_o, oracle_pool, tile_bytes, update_magnitude
 
 pytestmark = pytest.mark.gpu
 
@@ -95,7 +95,12 @@ def _decode_teacher_forced(stq, orc, wl_, bits, steps, head_begin=0, head_count=
                 res = orc.decode_step(bits[h], wl_.gate, ref_blk, as_f64(inp["q"][r, h]), as_f64(inp["k"][r, h]),
                                       as_f64(inp["v"][r, h]), float(inp["beta"][r, h]), alpha, as_f64(w[h]), d, d)
                 assert res["status"] == orc.OK
-                compare_block(orc, bits[h], d, got_blk, res["block"], res["tie"], tally, f"step {t} req {r} head {h}")
+                M = None
+                if bits[h] == 16:
+                    M = update_magnitude(orc.dequantize(16, d, d, ref_blk), as_f64(inp["k"][r, h]),
+                                         as_f64(inp["v"][r, h]), float(inp["beta"][r, h]), alpha)
+                compare_block(orc, bits[h], d, got_blk, res["block"], res["tie"], tally, f"step {t} req {r} head {h}",
+                              err_scale=M)
                 compare_o(og[r, hr], res["o"], tally, f"o step {t} req {r} head {h}")
                 offs, _ = orc.request_layout(bits, d, d)
                 new_opool[r * total + offs[h]: r * total + offs[h] + res["block"].size] = res["block"]
