@@ -99,13 +99,13 @@ def profiled_traffic():
     vals = {}
     with open(path) as f:
         for line in f:
-            if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "kernel_source_sha256")):
+            if ":" in line and line.strip().startswith(("traffic_bytes_per_step", "kernel_source_sha256")):
                 k, v = line.split(":", 1)
                 vals[k.strip()] = v.strip().strip("`")
     if vals.get("kernel_source_sha256") != decode_source_hash():
         return None
     try:
-        return float(vals["traffic_bytes_per_launch"])
+        return float(vals["traffic_bytes_per_step"])
     except (KeyError, ValueError):
         return None
 
@@ -341,9 +341,11 @@ def run_ours(args):
     # figures
     state_bytes = 2 * sum(lay.head_bytes(h) for h in range(H)) * B  # read + write, one launch
     io_bytes = B * H * (3 * d * (2 if wl.in_dtype == torch.bfloat16 else 4) + 4 * d + 8)
-    launches_per_step = math.ceil(B / 1024) * math.ceil(H / 3072)
-    avg_launch_s = total_ms / 1e3 / (args.steps * launches_per_step)
-    achieved = state_bytes / launches_per_step / avg_launch_s / 1e9
+    # the d = 128 decode launches one kernel per width present (largest blocks first), for every
+    # group of up to 1024 requests; its launches of one step together move `state_bytes`
+    launches_per_step = math.ceil(B / 1024) * sum(math.ceil(bits.count(b) / 3072) for b in set(bits))
+    step_s_local = total_ms / 1e3 / args.steps
+    achieved = state_bytes / step_s_local / 1e9
     peak, peak_kind = measured_peaks()
     step_s = total_ms_max / 1e3 / args.steps
     head_steps = B * H * world
@@ -373,8 +375,9 @@ def run_ours(args):
         "step_ms_min": min(per_step),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_kind": peak_kind, "traffic": profiled_traffic(),
-                     "bytes_per_launch": state_bytes / launches_per_step,
-                     "kernel": "decode_d128_kernel", "kernel_source_sha256": decode_source_hash()},
+                     "bytes_per_step": state_bytes, "launches_per_step": launches_per_step,
+                     "kernel": "decode_d128_kernel<width> (one launch per width of the step)",
+                     "kernel_source_sha256": decode_source_hash()},
         "e2e": {"value": head_steps / (e2e_ms / 1e3 / e2e_steps), "unit": "head-steps/s",
                 "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes, "steps": e2e_steps},
         "gpu_launches": args.steps * launches_per_step,

@@ -11,21 +11,31 @@
 // (k1 page, section 方法; aitest123 page, section 工程落地).
 //
 // Design (B200):
-//  * Persistent CTAs of 256 threads, two per SM, walking tiles round-robin over a list sorted by
-//    block size (FP16 pivots first, then 8-, 6-, 4-bit), so all CTAs see the same width mix.
-//  * A thread-0 producer streams each upcoming tile (packed codes + scales, and the q, k, v, w
-//    rows) into a byte-addressed shared-memory ring with cp.async.bulk, one mbarrier per tile in
-//    flight; every wait is bounded and reports STQ_ERR_TIMEOUT instead of hanging.
-//  * Each thread owns an 8 x 8 sub-block (rows 16m + 2*warp + half, columns 8*lane16 .. +7) in
-//    64 fp32 registers, so the state is read from HBM once and written once per step.
+//  * One persistent kernel per width (FP16 pivots, 8-, 6-, 4-bit), launched largest first; CTAs of
+//    256 threads walk the width's tiles round-robin.
+//  * Thread 0 streams each upcoming tile into a shared-memory slot ring: the packed codes + scales
+//    and the k, q, v, w (and alpha) rows by cp.async.bulk, the per-tile scalars by 4-byte cp.async,
+//    all completing on the slot's mbarrier. Every wait is bounded and reports STQ_ERR_TIMEOUT.
+//  * Each thread owns an 8 x 8 sub-block (rows 16m + 2*warp + half, columns 8*lane16 .. +7) of
+//    the tile, kept in its own lane of Tensor Memory (64 columns) between the sweeps and moved
+//    through registers 16 values at a time (tcgen05.ld / tcgen05.st). With the tile out of the
+//    register file a thread needs <= 64 registers, so four CTAs (32 warps) share an SM and hide
+//    each other's barrier and latency stalls; the state is still read from HBM once and written
+//    once per step.
 //  * The algebra runs in column-normalised coordinates: with y_ij = sqrt(w_i) S'_ij / c_j,
 //      y_ij = rho_i Q_ij + kappa_i g_j   (rho = alpha sqrt(w) r, kappa = sqrt(w) k, g = h / c,
 //                                         h = beta (v - alpha u))
 //    so the update, the column energy, the row maximum and the rounding are 1-2 packed f32x2
-//    operations per element each. Codes are unpacked with a LOP3/PRMT into the mantissa of
-//    2^23 (exact; a per-column power-of-two factor sigma is folded back per column) and rounded
+//    operations per element each. Codes are unpacked with a LOP3/PRMT into the mantissa of 2^23
+//    (exact; odd columns carry a power-of-two factor sigma, folded back per column) and rounded
 //    back with one FFMA against 2^23 + 2^(b-1), which rounds half to even for free.
-//  * Column sums cross warps through shared memory; row maxima stay inside a warp.
+//  * Four CTA barriers per tile: column sums of k~Q and q~Q (B1), the update coefficients (B2),
+//    the column energies (B3) and the new column scales (B4). Column partials are first summed
+//    between the two half-warps by shuffles, then across warps through shared memory; row maxima
+//    stay inside a warp. The next tile's row factors are computed by warps 4-7 while warps 0-3
+//    finish the column scales.
+//  * Scale arithmetic (reciprocals, square roots) uses the SFU approximations (a few ulp): the
+//    codes are always computed from the scales this kernel stores.
 #include "stq_internal.cuh"
 
 namespace stq {
@@ -33,66 +43,114 @@ namespace {
 
 constexpr int D = 128;
 constexpr int NT = 256;
-constexpr int NBAR = 8;                // tiles in flight per CTA (mbarriers)
-constexpr uint32_t RING = 72 * 1024;   // bytes of the staging ring per CTA
-constexpr int MAXB = 1024;             // requests per launch whose slots are cached in smem
+constexpr int NSMAX = 4;               // slots (tiles in flight) per CTA
+constexpr int MAXB = 256;              // requests per launch whose slots are cached in smem
 constexpr uint32_t MAGIC = 0x4B000000u;  // bit pattern of 2^23
+constexpr uint32_t TMEM_COLS = 128;    // per CTA: 2 x 64 columns (warps 0-3 / 4-7) over 128 lanes
 
-struct __align__(16) SmemD128 {
-    uint8_t ring[RING];
-    float red[16 * 2 * D];   // column partials per (warp, half); later the row-max partials
-    float4 rowA[2][D];       // per tile parity: (k~, q~, rho, kappa)
-    float2 rowB[2][D];       // per tile parity: (sqrt w, mu)
+struct __align__(16) SmemFixed {
+    float red[2 * 8 * D];    // column partials (U/P per warp; E per warp), then row-max partials
+    float4 rowKQ[D];         // (k~, k~, q~, q~)
+    float4 rowRK[D];         // (rho, rho, kappa, kappa)
+    float2 rowMu[D];         // (mu, mu)  (literal channel gate)
+    float rowSw[2][D];       // per tile parity: sqrt(w)
     float colG1[D];
     float colG2[D];
     float colH[D];           // rank-1 part of the readout
     float colB[D];           // c_j / (sigma_j c'_j)
     float2 rowS[D];          // (s_i, s_i), s_i = 1 / (sqrt(w_i) r'_i)
     float rsum[2][4][4];     // per parity, per precompute warp: sum w, q.k, q.(alpha*k)
-    float scal[2][4];        // per parity: beta, alpha, skip
+    float scal[NSMAX][4];    // per slot: beta, alpha, skip
     int32_t slots[MAXB];
-    uint32_t tpos[NBAR];     // ring position / wrap count of each tile in flight (producer only)
-    uint32_t twrap[NBAR];
-    unsigned long long bars[NBAR];
+    unsigned long long bars[NSMAX];
+    float2 unpack_off;       // (-(2^23 + o), -(2^23 + o * SIG1)), o = 2^(b-1)
+    uint32_t tmem_base;
 };
 
 // ---------------------------------------------------------------------------------------------
 // Static per-width facts
 // ---------------------------------------------------------------------------------------------
-template <int BITS>
-struct Width {
-    static constexpr int RB = 16 * BITS;                       // code bytes of one 128-wide row
+template <int BITS, int GATE, int IN_BF16>
+struct Cfg {
+    static constexpr int RB = BITS == 16 ? 256 : 16 * BITS;    // bytes of one 128-wide row
     static constexpr uint32_t SOFF = scale_offset(BITS, D, D);  // byte offset of r[]
     static constexpr uint32_t BLK = head_block_bytes(BITS, D, D);
-    static constexpr float QMAX = (float)((1 << (BITS - 1)) - 1);
-    static constexpr float ROUND = 8388608.0f + (float)(1 << (BITS - 1));  // 2^23 + offset
-    // power-of-two factor of column c (= j mod 8) left by the unpacking
-    __device__ static constexpr float sigma(int c)
-    {
-        return BITS == 4 ? (float)(1 << (4 * (c & 3)))
-             : BITS == 6 ? (float)(1 << (6 * (c % 3)))
-                         : 1.0f;
-    }
+    static constexpr uint32_t ROW_IN = D * (IN_BF16 ? 2u : 4u);
+    static constexpr uint32_t K_OFF = BLK, Q_OFF = BLK + ROW_IN, V_OFF = BLK + 2 * ROW_IN;
+    static constexpr uint32_t W_OFF = BLK + 3 * ROW_IN, A_OFF = W_OFF + 4 * D;
+    static constexpr uint32_t LEN = A_OFF + (GATE != 0 ? 4u * D : 0u);  // a multiple of 256
+    // slots so that four CTAs fit an SM's 228 KB for the 4- and 6-bit kernels
+    static constexpr int NS = BITS == 4 ? 3 : 2;
+    static constexpr size_t SMEM = sizeof(SmemFixed) + (size_t)NS * LEN;
+    static constexpr float QMAX = BITS == 16 ? 0.f : (float)((1 << (BITS - 1)) - 1);
+    static constexpr float ROUND = 8388608.0f + (BITS == 16 ? 0.f : (float)(1 << (BITS - 1)));
+    // odd columns are unpacked scaled by SIG1 (even columns by 1)
+    static constexpr float SIG1 = BITS == 4 ? 16.f : BITS == 6 ? 64.f : 1.f;
 };
 
 __device__ __forceinline__ float f_of(uint32_t x) { return __uint_as_float(x); }
 __device__ __forceinline__ uint32_t u_of(float x) { return __float_as_uint(x); }
 
-// Unpack the 8 codes of one thread's row segment (in shared memory) into sigma_c * Q.
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float min3(float a, float b, float c)
+{
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ float fast_rcp(float x) { return __fdividef(1.0f, x); }
+
+// ---------------------------------------------------------------------------------------------
+// Tensor Memory: each thread keeps its 64 values in 64 consecutive columns of its own lane.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float2 (&v)[8])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+        "%13, %14, %15, %16};" ::"r"(taddr),
+        "f"(v[0].x), "f"(v[0].y), "f"(v[1].x), "f"(v[1].y), "f"(v[2].x), "f"(v[2].y), "f"(v[3].x), "f"(v[3].y),
+        "f"(v[4].x), "f"(v[4].y), "f"(v[5].x), "f"(v[5].y), "f"(v[6].x), "f"(v[6].y), "f"(v[7].x), "f"(v[7].y)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float2 (&v)[8])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15}, [%16];"
+        : "=f"(v[0].x), "=f"(v[0].y), "=f"(v[1].x), "=f"(v[1].y), "=f"(v[2].x), "=f"(v[2].y), "=f"(v[3].x),
+          "=f"(v[3].y), "=f"(v[4].x), "=f"(v[4].y), "=f"(v[5].x), "=f"(v[5].y), "=f"(v[6].x), "=f"(v[6].y),
+          "=f"(v[7].x), "=f"(v[7].y)
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Two adjacent codes at bits [0, BITS) and [BITS, 2*BITS) of s, as (2^23 + u0, 2^23 + u1 * 2^BITS).
 template <int BITS>
-__device__ __forceinline__ void unpack_row(const uint8_t *src, int cg, float2 (&Q)[4])
+__device__ __forceinline__ float2 code_pair(uint32_t s)
+{
+    constexpr uint32_t M = (1u << BITS) - 1u;
+    return make_float2(f_of((s & M) | MAGIC), f_of((s & (M << BITS)) | MAGIC));
+}
+
+// Unpack the 8 codes of one thread's row segment (in shared memory) into (Q, SIG1 * Q) pairs;
+// `off` = (-(2^23 + o), -(2^23 + o * SIG1)) with o = 2^(b-1). A pivot row holds 8 halves.
+template <int BITS>
+__device__ __forceinline__ void unpack_row(const uint8_t *src, int cg, float2 off, float2 *Q)
 {
     if constexpr (BITS == 4) {
         const uint32_t wd = *reinterpret_cast<const uint32_t *>(src);
-        const uint32_t hi = wd >> 16;
-        Q[0] = __fadd2_rn(make_float2(f_of((wd & 0x000Fu) | MAGIC), f_of((wd & 0x00F0u) | MAGIC)),
-                          make_float2(-(8388608.0f + 8.0f), -(8388608.0f + 128.0f)));
-        Q[1] = __fadd2_rn(make_float2(f_of((wd & 0x0F00u) | MAGIC), f_of((wd & 0xF000u) | MAGIC)),
-                          make_float2(-(8388608.0f + 2048.0f), -(8388608.0f + 32768.0f)));
-        Q[2] = __fadd2_rn(make_float2(f_of((hi & 0x000Fu) | MAGIC), f_of((hi & 0x00F0u) | MAGIC)),
-                          make_float2(-(8388608.0f + 8.0f), -(8388608.0f + 128.0f)));
-        Q[3] = __fadd2_rn(make_float2(f_of((hi & 0x0F00u) | MAGIC), f_of((hi & 0xF000u) | MAGIC)),
-                          make_float2(-(8388608.0f + 2048.0f), -(8388608.0f + 32768.0f)));
+        Q[0] = __fadd2_rn(code_pair<4>(wd), off);
+        Q[1] = __fadd2_rn(code_pair<4>(wd >> 8), off);
+        Q[2] = __fadd2_rn(code_pair<4>(wd >> 16), off);
+        Q[3] = __fadd2_rn(code_pair<4>(wd >> 24), off);
     } else if constexpr (BITS == 6) {
         uint32_t lo, hi;
         if ((cg & 1) == 0) {
@@ -103,47 +161,37 @@ __device__ __forceinline__ void unpack_row(const uint8_t *src, int cg, float2 (&
             lo = (uint32_t)(*reinterpret_cast<const uint16_t *>(src)) | (w1 << 16);
             hi = w1 >> 16;
         }
-        const uint32_t t = __funnelshift_r(lo, hi, 18);
-        const uint32_t t2 = hi >> 4;
-        Q[0] = __fadd2_rn(make_float2(f_of((lo & 0x3Fu) | MAGIC), f_of((lo & 0xFC0u) | MAGIC)),
-                          make_float2(-(8388608.0f + 32.0f), -(8388608.0f + 2048.0f)));
-        Q[1] = __fadd2_rn(make_float2(f_of((lo & 0x3F000u) | MAGIC), f_of((t & 0x3Fu) | MAGIC)),
-                          make_float2(-(8388608.0f + 131072.0f), -(8388608.0f + 32.0f)));
-        Q[2] = __fadd2_rn(make_float2(f_of((t & 0xFC0u) | MAGIC), f_of((t & 0x3F000u) | MAGIC)),
-                          make_float2(-(8388608.0f + 2048.0f), -(8388608.0f + 131072.0f)));
-        Q[3] = __fadd2_rn(make_float2(f_of((t2 & 0x3Fu) | MAGIC), f_of((t2 & 0xFC0u) | MAGIC)),
-                          make_float2(-(8388608.0f + 32.0f), -(8388608.0f + 2048.0f)));
-    } else {
+        Q[0] = __fadd2_rn(code_pair<6>(lo), off);
+        Q[1] = __fadd2_rn(code_pair<6>(lo >> 12), off);
+        Q[2] = __fadd2_rn(code_pair<6>(__funnelshift_r(lo, hi, 24)), off);
+        Q[3] = __fadd2_rn(code_pair<6>(hi >> 4), off);
+    } else if constexpr (BITS == 8) {
         const uint2 wd = *reinterpret_cast<const uint2 *>(src);
-        const float2 off = make_float2(-(8388608.0f + 128.0f), -(8388608.0f + 128.0f));
         Q[0] = __fadd2_rn(make_float2(f_of(__byte_perm(wd.x, MAGIC, 0x7650)), f_of(__byte_perm(wd.x, MAGIC, 0x7651))), off);
         Q[1] = __fadd2_rn(make_float2(f_of(__byte_perm(wd.x, MAGIC, 0x7652)), f_of(__byte_perm(wd.x, MAGIC, 0x7653))), off);
         Q[2] = __fadd2_rn(make_float2(f_of(__byte_perm(wd.y, MAGIC, 0x7650)), f_of(__byte_perm(wd.y, MAGIC, 0x7651))), off);
         Q[3] = __fadd2_rn(make_float2(f_of(__byte_perm(wd.y, MAGIC, 0x7652)), f_of(__byte_perm(wd.y, MAGIC, 0x7653))), off);
+    } else {
+        const uint4 raw = *reinterpret_cast<const uint4 *>(src);
+        Q[0] = __half22float2(*reinterpret_cast<const __half2 *>(&raw.x));
+        Q[1] = __half22float2(*reinterpret_cast<const __half2 *>(&raw.y));
+        Q[2] = __half22float2(*reinterpret_cast<const __half2 *>(&raw.z));
+        Q[3] = __half22float2(*reinterpret_cast<const __half2 *>(&raw.w));
     }
 }
 
 // Pack 8 rounded codes (bit patterns 2^23 + u, u < 2^b) and store them to the tile in HBM.
 template <int BITS>
-__device__ __forceinline__ void pack_store_row(uint8_t *dst, int cg, const float2 (&F)[4])
+__device__ __forceinline__ void pack_store_row(uint8_t *dst, int cg, const float2 *F)
 {
     const uint32_t f0 = u_of(F[0].x), f1 = u_of(F[0].y), f2 = u_of(F[1].x), f3 = u_of(F[1].y);
     const uint32_t f4 = u_of(F[2].x), f5 = u_of(F[2].y), f6 = u_of(F[3].x), f7 = u_of(F[3].y);
     if constexpr (BITS == 4) {
-        // sum_c F_c << 4c minus the same sum of the 2^23 patterns (mod 2^32) leaves the nibbles
-        constexpr uint32_t C = (uint32_t)(((uint64_t)MAGIC << 0) + ((uint64_t)MAGIC << 4) + ((uint64_t)MAGIC << 8) +
-                                          ((uint64_t)MAGIC << 12) + ((uint64_t)MAGIC << 16) + ((uint64_t)MAGIC << 20) +
-                                          ((uint64_t)MAGIC << 24) + ((uint64_t)MAGIC << 28));
-        uint32_t acc = f7;
-        acc = (acc << 4) + f6;
-        acc = (acc << 4) + f5;
-        acc = (acc << 4) + f4;
-        acc = (acc << 4) + f3;
-        acc = (acc << 4) + f2;
-        acc = (acc << 4) + f1;
-        acc = (acc << 4) + f0;
-        *reinterpret_cast<uint32_t *>(dst) = acc - C;
+        // pair nibbles by shift-add (garbage above bit 8 is dropped), then gather the low bytes
+        const uint32_t p0 = (f1 << 4) + f0, p1 = (f3 << 4) + f2, p2 = (f5 << 4) + f4, p3 = (f7 << 4) + f6;
+        *reinterpret_cast<uint32_t *>(dst) = __byte_perm(__byte_perm(p0, p1, 0x0040), __byte_perm(p2, p3, 0x0040), 0x5410);
     } else if constexpr (BITS == 6) {
+        // sum_c F_c << 6c minus the same sum of the 2^23 patterns (mod 2^32) leaves the codes
         constexpr uint32_t C = (uint32_t)(((uint64_t)MAGIC << 0) + ((uint64_t)MAGIC << 6) + ((uint64_t)MAGIC << 12) +
                                           ((uint64_t)MAGIC << 18) + ((uint64_t)MAGIC << 24) + ((uint64_t)MAGIC << 30));
         const uint32_t lo = f0 + (f1 << 6) + (f2 << 12) + (f3 << 18) + (f4 << 24) + (f5 << 30) - C;
@@ -166,124 +214,113 @@ __device__ __forceinline__ void pack_store_row(uint8_t *dst, int cg, const float
 
 __device__ __forceinline__ float4 f4_of(float2 a, float2 b) { return make_float4(a.x, a.y, b.x, b.y); }
 
-__host__ __device__ constexpr uint32_t tile_bytes(int bits, int in_bf16, int gate)
+__device__ __forceinline__ void load_pairs(const float *src, float2 (&out)[4])
 {
-    return head_block_bytes(bits, D, D) + 3u * D * (in_bf16 ? 2u : 4u) + 4u * D + (gate != 0 ? 4u * D : 0u);
+    const float4 a = *reinterpret_cast<const float4 *>(src);
+    const float4 b = *reinterpret_cast<const float4 *>(src + 4);
+    out[0] = make_float2(a.x, a.y);
+    out[1] = make_float2(a.z, a.w);
+    out[2] = make_float2(b.x, b.y);
+    out[3] = make_float2(b.z, b.w);
 }
 
-// Deterministic placement of the next tile in the ring: continue, or wrap to 0 if it does not fit.
-__device__ __forceinline__ void ring_place(uint32_t &head, uint32_t &wrap, uint32_t len, uint32_t &pos)
+// Sum of 8 per-warp partials with a short dependency chain.
+__device__ __forceinline__ float sum8(const float *src)
 {
-    if (head + len > RING) {
-        head = 0;
-        ++wrap;
-    }
-    pos = head;
-    head += len;
+    return ((src[0] + src[D]) + (src[2 * D] + src[3 * D])) + ((src[4 * D] + src[5 * D]) + (src[6 * D] + src[7 * D]));
 }
 
 struct TileId {
-    int b, hr, bits;
+    int b, hr;
     uint32_t off;
 };
 
-__device__ __forceinline__ TileId tile_id(const TileParams &p, int t)
+__device__ __forceinline__ TileId tile_id(const TileParams &p, int n)
 {
-    TileId id;
+    const int t = (int)blockIdx.x + n * (int)gridDim.x;
     const int pos = t / p.B;
+    TileId id;
     id.b = t - pos * p.B;
     const TileEntry e = p.table[pos];
     id.hr = entry_head(e);
-    id.bits = entry_bits(e);
     id.off = e.off;
     return id;
 }
 
-// Thread 0's producer state.
-template <int GATE, int IN_BF16>
-struct Producer {
-    int issued = 0;
-    uint32_t head = 0, wrap = 0;
-    float nbeta = 0.f, nalpha = 0.f, nskip = 0.f;
-
-    // Issue bulk copies for as many upcoming tiles as fit next to the live ones. Tiles before
-    // `oldest` are dead (their ring bytes are no longer read). A tile always fits an empty ring,
-    // so every tile is eventually issued.
-    __device__ void issue_more(const TileParams &p, SmemD128 &sm, int my_count, int oldest)
-    {
-        constexpr uint32_t ROW_IN = D * (IN_BF16 ? 2 : 4);
-        while (issued < my_count && issued - oldest < NBAR) {
-            const TileId id = tile_id(p, (int)blockIdx.x + issued * (int)gridDim.x);
-            const uint32_t len = tile_bytes(id.bits, IN_BF16, GATE);
-            uint32_t h = head, wr = wrap, pos;
-            ring_place(h, wr, len, pos);
-            if (issued > oldest) {
-                const uint32_t opos = sm.tpos[oldest % NBAR], owrap = sm.twrap[oldest % NBAR];
-                const bool fits = (wr == owrap) || (wr == owrap + 1 && pos + len <= opos);
-                if (!fits) break;
-            }
-            head = h;
-            wrap = wr;
-            sm.tpos[issued % NBAR] = pos;
-            sm.twrap[issued % NBAR] = wr;
-            const uint32_t bar = smem_u32(&sm.bars[issued % NBAR]);
-            const int slot = sm.slots[id.b];
-            if (slot < 0 || slot >= p.pool_slots) {
-                flag(p.status, kFlagBounds);
-                mbar_arrive(bar);
-            } else {
-                const uint32_t blk = head_block_bytes(id.bits, D, D);
-                const uint32_t dst = smem_u32(sm.ring + pos);
-                const size_t row = (size_t)id.b * p.head_count + id.hr;
-                mbar_arrive_expect_tx(bar, len);
-                bulk_g2s(dst, p.pool + (uint64_t)slot * p.req_bytes + id.off, blk, bar);
-                bulk_g2s(dst + blk, (const uint8_t *)p.k + row * ROW_IN, ROW_IN, bar);
-                bulk_g2s(dst + blk + ROW_IN, (const uint8_t *)p.q + row * ROW_IN, ROW_IN, bar);
-                bulk_g2s(dst + blk + 2 * ROW_IN, (const uint8_t *)p.v + row * ROW_IN, ROW_IN, bar);
-                bulk_g2s(dst + blk + 3 * ROW_IN, p.w + (size_t)id.hr * D, 4 * D, bar);
-                if (GATE != 0) bulk_g2s(dst + blk + 3 * ROW_IN + 4 * D, p.alpha + row * D, 4 * D, bar);
-            }
-            ++issued;
-        }
-    }
-
-    // Start loading the per-tile scalars of tile n (plain loads; consumed one sweep later).
-    __device__ void load_scalars(const TileParams &p, const SmemD128 &sm, int n, int my_count)
-    {
-        if (n >= my_count) return;
-        const TileId id = tile_id(p, (int)blockIdx.x + n * (int)gridDim.x);
-        const size_t row = (size_t)id.b * p.head_count + id.hr;
-        const int slot = sm.slots[id.b];
-        nskip = (slot < 0 || slot >= p.pool_slots) ? 1.f : 0.f;
-        nbeta = p.beta[row];
-        nalpha = GATE == 0 ? p.alpha[row] : 1.f;
-    }
-    __device__ void store_scalars(SmemD128 &sm, int parity)
-    {
-        sm.scal[parity][0] = nbeta;
-        sm.scal[parity][1] = nalpha;
-        sm.scal[parity][2] = nskip;
-    }
-};
-
-// Row factors of one tile (threads 0..127, row i = tid), and per-warp sums of w, q.k, q.(alpha k).
-template <int GATE, int IN_BF16>
-__device__ __forceinline__ void precompute_rows(SmemD128 &sm, const uint8_t *tile, int bits, int pb)
+template <int BITS, int GATE, int IN_BF16>
+__device__ __forceinline__ uint8_t *ring_slot(uint8_t *smem, int n)
 {
-    constexpr uint32_t ROW_IN = D * (IN_BF16 ? 2 : 4);
-    const int i = threadIdx.x;
-    const uint32_t blk = head_block_bytes(bits, D, D);
-    const uint8_t *rows = tile + blk;
-    const bool pivot = bits == 16;
-    const float r = pivot ? 1.f : reinterpret_cast<const float *>(tile + scale_offset(bits, D, D))[i];
-    const float k = load_in<IN_BF16>(rows, i);
-    const float q = load_in<IN_BF16>(rows + ROW_IN, i);
-    const float w = reinterpret_cast<const float *>(rows + 3 * ROW_IN)[i];
-    const float a = GATE == 0 ? sm.scal[pb][1] : reinterpret_cast<const float *>(rows + 3 * ROW_IN + 4 * D)[i];
+    return smem + sizeof(SmemFixed) + (size_t)(n % Cfg<BITS, GATE, IN_BF16>::NS) * Cfg<BITS, GATE, IN_BF16>::LEN;
+}
+
+// Thread 0: stream tile n into slot n % NS (codes + scales, rows by bulk copy; scalars by
+// 4-byte cp.async), completing on the slot's mbarrier (two arrivals: expect_tx + cp.async).
+template <int BITS, int GATE, int IN_BF16>
+__device__ __forceinline__ void issue_tile(const TileParams &p, SmemFixed &sm, uint8_t *smem, int n, int my_count)
+{
+    using C = Cfg<BITS, GATE, IN_BF16>;
+    if (n >= my_count) return;
+    const int slot_i = n % C::NS;
+    const TileId id = tile_id(p, n);
+    const uint32_t bar = smem_u32(&sm.bars[slot_i]);
+    const int slot = sm.slots[id.b];
+    if (slot < 0 || slot >= p.pool_slots) {
+        flag(p.status, kFlagBounds);
+        sm.scal[slot_i][2] = 1.f;
+        mbar_arrive(bar);
+        mbar_arrive(bar);
+        return;
+    }
+    sm.scal[slot_i][2] = 0.f;
+    const size_t row = (size_t)id.b * p.head_count + id.hr;
+    cp_async4(smem_u32(&sm.scal[slot_i][0]), p.beta + row);
+    if (GATE == 0) cp_async4(smem_u32(&sm.scal[slot_i][1]), p.alpha + row);
+    cp_async_arrive(bar);
+    const uint32_t dst = smem_u32(ring_slot<BITS, GATE, IN_BF16>(smem, n));
+    mbar_arrive_expect_tx(bar, C::LEN);
+    bulk_g2s(dst, p.pool + (uint64_t)slot * p.req_bytes + id.off, C::BLK, bar);
+    bulk_g2s(dst + C::K_OFF, (const uint8_t *)p.k + row * C::ROW_IN, C::ROW_IN, bar);
+    bulk_g2s(dst + C::Q_OFF, (const uint8_t *)p.q + row * C::ROW_IN, C::ROW_IN, bar);
+    bulk_g2s(dst + C::V_OFF, (const uint8_t *)p.v + row * C::ROW_IN, C::ROW_IN, bar);
+    bulk_g2s(dst + C::W_OFF, p.w + (size_t)id.hr * D, 4 * D, bar);
+    if (GATE != 0) bulk_g2s(dst + C::A_OFF, p.alpha + row * D, 4 * D, bar);
+}
+
+template <int BITS, int GATE, int IN_BF16>
+__device__ __forceinline__ bool wait_tile(SmemFixed &sm, int n)
+{
+    using C = Cfg<BITS, GATE, IN_BF16>;
+    return mbar_wait_bounded(smem_u32(&sm.bars[n % C::NS]), (uint32_t)((n / C::NS) & 1));
+}
+
+// Wait for tile n and compute its row factors: run by the 128 threads of warps 4-7 (row
+// i = tid - 128), with per-warp sums of w, q.k and q.(alpha k). Returns false on a timeout.
+template <int BITS, int GATE, int IN_BF16>
+__device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, int n, int my_count)
+{
+    using C = Cfg<BITS, GATE, IN_BF16>;
+    if (n >= my_count) return true;
+    // the verdict is made warp-uniform before any warp-wide shuffle below
+    if (!__all_sync(0xffffffffu, wait_tile<BITS, GATE, IN_BF16>(sm, n))) return false;
+    const int slot_i = n % C::NS;
+    if (sm.scal[slot_i][2] != 0.f) return true;  // skipped tile: nothing was loaded
+    const int pb = n & 1;
+    const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16>(smem, n);
+    const int i = threadIdx.x - D;
+    constexpr bool pivot = BITS == 16;
+    const float r = pivot ? 1.f : reinterpret_cast<const float *>(tile + C::SOFF)[i];
+    const float k = load_in<IN_BF16>(tile + C::K_OFF, i);
+    const float q = load_in<IN_BF16>(tile + C::Q_OFF, i);
+    const float w = reinterpret_cast<const float *>(tile + C::W_OFF)[i];
+    const float a = GATE == 0 ? sm.scal[slot_i][1] : reinterpret_cast<const float *>(tile + C::A_OFF)[i];
     const float sw = pivot ? 1.f : sqrtf(w);
     const float kt = (GATE == 2 ? k * a : k) * r;
-    sm.rowA[pb][i] = make_float4(kt, q * a * r, a * sw * r, sw * k);
-    sm.rowB[pb][i] = make_float2(sw, -sw * a * k);
+    const float qt = q * a * r;
+    const float rho = a * sw * r, kap = sw * k, mu = -sw * a * k;
+    sm.rowKQ[i] = make_float4(kt, kt, qt, qt);
+    sm.rowRK[i] = make_float4(rho, rho, kap, kap);
+    if (GATE == 1) sm.rowMu[i] = make_float2(mu, mu);
+    sm.rowSw[pb][i] = sw;
     float s0 = w, s1 = q * k, s2 = q * a * k;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -296,357 +333,366 @@ __device__ __forceinline__ void precompute_rows(SmemD128 &sm, const uint8_t *til
         sm.rsum[pb][i >> 5][1] = s1;
         sm.rsum[pb][i >> 5][2] = s2;
     }
+    return true;
 }
 
-// Column finals after the first sweep: threads 0..127 turn the column sums of k~ Q into g (and
-// the readout's rank-1 part); threads 128..255 return the column sums of q~ Q (un-scaled).
-template <int GATE, int IN_BF16>
-__device__ __forceinline__ float finals_a(SmemD128 &sm, const uint8_t *tile, int bits, int pb, float cj,
-                                          float inv_sig, float sig)
+__device__ __forceinline__ uint8_t *tile_global(const TileParams &p, const SmemFixed &sm, const TileId &id)
 {
-    constexpr uint32_t ROW_IN = D * (IN_BF16 ? 2 : 4);
-    const int tid = threadIdx.x;
-    const int j = tid & (D - 1);
-    if (tid < D) {
-        float U = 0.f;
+    return p.pool + (uint64_t)sm.slots[id.b] * p.req_bytes + id.off;
+}
+
+// One tile; returns false if the wait for the next tile timed out.
+template <int BITS, int GATE, int IN_BF16>
+__device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm, uint8_t *smem, int n, int my_count,
+                                             uint32_t tcol)
+{
+    using C = Cfg<BITS, GATE, IN_BF16>;
+    constexpr bool pivot = BITS == 16;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, cg = lane & 15, sub = lane >> 4;
+    const int slot_i = n % C::NS, pb = n & 1;
+    const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16>(smem, n);
+    const uint8_t *rowsrc = tile + (2 * warp + sub) * C::RB + cg * (pivot ? 16 : BITS);
+
+    // ---- Sweep A: unpack to TMEM, column sums of k~Q and q~Q -------------------------------
+    {
+        const float2 off = sm.unpack_off;
+        float2 accU[4], accP[4];
 #pragma unroll
-        for (int s = 0; s < 16; ++s) U += sm.red[s * 2 * D + j];
-        U *= inv_sig;
-        const float beta = sm.scal[pb][0], alpha = sm.scal[pb][1];
-        const float vj = load_in<IN_BF16>(tile + head_block_bytes(bits, D, D) + 2 * ROW_IN, j);
+        for (int pp = 0; pp < 4; ++pp) accU[pp] = accP[pp] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float2 ch[8];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int m = 2 * k + r;
+                unpack_row<BITS>(rowsrc + 16 * m * C::RB, cg, off, ch + 4 * r);
+                const float4 kq = sm.rowKQ[16 * m + 2 * warp + sub];
+                const float2 kk = make_float2(kq.x, kq.y), qq = make_float2(kq.z, kq.w);
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) {
+                    accU[pp] = __ffma2_rn(kk, ch[4 * r + pp], accU[pp]);
+                    accP[pp] = __ffma2_rn(qq, ch[4 * r + pp], accP[pp]);
+                }
+            }
+            tmem_st16(tcol + 16 * k, ch);
+        }
+        // halves 0/1 of a warp hold the same columns: half 0 keeps U, half 1 keeps P
+        float *red = sm.red + (sub * 8 + warp) * D + 8 * cg;
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+            const float2 send = sub ? accU[pp] : accP[pp];
+            const float2 keep = sub ? accP[pp] : accU[pp];
+            const float2 got = make_float2(__shfl_xor_sync(0xffffffffu, send.x, 16),
+                                           __shfl_xor_sync(0xffffffffu, send.y, 16));
+            accU[pp] = __fadd2_rn(keep, got);
+        }
+        *reinterpret_cast<float4 *>(red) = f4_of(accU[0], accU[1]);
+        *reinterpret_cast<float4 *>(red + 4) = f4_of(accU[2], accU[3]);
+    }
+    __syncthreads();  // B1: column partials complete
+
+    // ---- Column finals: warps 0-3 the update coefficients, warps 4-7 the readout sums ------
+    const int j = tid & (D - 1);
+    const float cj = pivot ? 1.f : reinterpret_cast<const float *>(tile + C::SOFF)[D + j];
+    const float sig = (j & 1) ? C::SIG1 : 1.f;
+    const float inv_sig = (j & 1) ? 1.f / C::SIG1 : 1.f;  // powers of two: exact
+    const float S = sum8(sm.red + (tid < D ? 0 : 8 * D) + j) * inv_sig;
+    if (tid < D) {
+        const float beta = sm.scal[slot_i][0], alpha = sm.scal[slot_i][1];
+        const float vj = load_in<IN_BF16>(tile + C::V_OFF, j);
         const float qk = sm.rsum[pb][0][1] + sm.rsum[pb][1][1] + sm.rsum[pb][2][1] + sm.rsum[pb][3][1];
-        const float u = cj * U;
+        const float u = cj * S;
+        const float rc = pivot ? 1.f : fast_rcp(cj);
         if (GATE == 1) {
             const float qak = sm.rsum[pb][0][2] + sm.rsum[pb][1][2] + sm.rsum[pb][2][2] + sm.rsum[pb][3][2];
-            sm.colG1[j] = sig * (beta * vj / cj);
-            sm.colG2[j] = sig * (beta * u / cj);
+            sm.colG1[j] = sig * (beta * vj) * rc;
+            sm.colG2[j] = sig * (beta * u) * rc;
             sm.colH[j] = qk * beta * vj - qak * beta * u;
         } else {
             const float h = GATE == 0 ? beta * (vj - alpha * u) : beta * (vj - u);
-            sm.colG1[j] = sig * (h / cj);
+            sm.colG1[j] = sig * h * rc;
             sm.colH[j] = qk * h;
         }
-        return 0.f;
     }
-    float P = 0.f;
-#pragma unroll
-    for (int s = 0; s < 16; ++s) P += sm.red[s * 2 * D + D + j];
-    return P * inv_sig;
-}
-
-// Sweep A (shared by quantized and pivot tiles): column sums of k~ Q and q~ Q from registers.
-__device__ __forceinline__ void sweep_a_sums(SmemD128 &sm, const float2 (&Q)[8][4], int pb, int warp, int sub, int cg)
-{
-    float2 accU[4], accP[4];
-#pragma unroll
-    for (int pp = 0; pp < 4; ++pp) accU[pp] = accP[pp] = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const int i = 16 * m + 2 * warp + sub;
-        const float4 ra = sm.rowA[pb][i];
-        const float2 kk = make_float2(ra.x, ra.x), qq = make_float2(ra.y, ra.y);
-#pragma unroll
-        for (int pp = 0; pp < 4; ++pp) {
-            accU[pp] = __ffma2_rn(kk, Q[m][pp], accU[pp]);
-            accP[pp] = __ffma2_rn(qq, Q[m][pp], accP[pp]);
-        }
-    }
-    float *red = sm.red + (2 * warp + sub) * 2 * D + 8 * cg;
-    *reinterpret_cast<float4 *>(red) = f4_of(accU[0], accU[1]);
-    *reinterpret_cast<float4 *>(red + 4) = f4_of(accU[2], accU[3]);
-    *reinterpret_cast<float4 *>(red + D) = f4_of(accP[0], accP[1]);
-    *reinterpret_cast<float4 *>(red + D + 4) = f4_of(accP[2], accP[3]);
-}
-
-// y = rho Q + kappa g1 (+ mu g2), in place in Q; optionally accumulating the column energy.
-template <int GATE, bool ENERGY>
-__device__ __forceinline__ void sweep_b_update(SmemD128 &sm, float2 (&Q)[8][4], int pb, int warp, int sub, int cg,
-                                               float2 (&accE)[4], bool &bad)
-{
-    float2 g1[4], g2[4];
-    {
-        const float4 a = *reinterpret_cast<const float4 *>(sm.colG1 + 8 * cg);
-        const float4 b = *reinterpret_cast<const float4 *>(sm.colG1 + 8 * cg + 4);
-        g1[0] = make_float2(a.x, a.y); g1[1] = make_float2(a.z, a.w);
-        g1[2] = make_float2(b.x, b.y); g1[3] = make_float2(b.z, b.w);
-    }
-    if (GATE == 1) {
-        const float4 a = *reinterpret_cast<const float4 *>(sm.colG2 + 8 * cg);
-        const float4 b = *reinterpret_cast<const float4 *>(sm.colG2 + 8 * cg + 4);
-        g2[0] = make_float2(a.x, a.y); g2[1] = make_float2(a.z, a.w);
-        g2[2] = make_float2(b.x, b.y); g2[3] = make_float2(b.z, b.w);
-    }
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const int i = 16 * m + 2 * warp + sub;
-        const float4 ra = sm.rowA[pb][i];
-        const float2 rho = make_float2(ra.z, ra.z), kap = make_float2(ra.w, ra.w);
-        float2 mu = make_float2(0.f, 0.f);
-        if (GATE == 1) {
-            const float mv = sm.rowB[pb][i].y;
-            mu = make_float2(mv, mv);
-        }
-#pragma unroll
-        for (int pp = 0; pp < 4; ++pp) {
-            float2 t = __fmul2_rn(kap, g1[pp]);
-            if (GATE == 1) t = __ffma2_rn(mu, g2[pp], t);
-            const float2 y = __ffma2_rn(rho, Q[m][pp], t);
-            Q[m][pp] = y;
-            if (ENERGY) accE[pp] = __ffma2_rn(y, y, accE[pp]);
-            else bad |= !(fabsf(y.x) < 65520.0f) || !(fabsf(y.y) < 65520.0f);
-        }
-    }
-}
-
-template <int BITS, int GATE, int IN_BF16>
-__device__ __forceinline__ void tile_quant(const TileParams &p, SmemD128 &sm, const uint8_t *tile,
-                                           uint8_t *gblock, float *orow, int pb, int n, int my_count,
-                                           Producer<GATE, IN_BF16> &prod)
-{
-    using Wd = Width<BITS>;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, cg = lane & 15, sub = lane >> 4;
-    float2 Q[8][4];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) unpack_row<BITS>(tile + (16 * m + 2 * warp + sub) * Wd::RB + cg * BITS, cg, Q[m]);
-    sweep_a_sums(sm, Q, pb, warp, sub, cg);
-    if (tid == 0) prod.store_scalars(sm, pb ^ 1);
-    __syncthreads();  // B1: column partials complete
-
-    const int j = tid & (D - 1);
-    const float cj = reinterpret_cast<const float *>(tile + Wd::SOFF)[D + j];
-    const float sig = Wd::sigma(j & 7);
-    const float inv_sig = 1.0f / sig;  // power of two: exact
-    const float Pj = finals_a<GATE, IN_BF16>(sm, tile, BITS, pb, cj, inv_sig, sig);
-    __syncthreads();  // B2: g, readout parts ready; this tile's ring bytes are no longer read
-    if (tid == 0) prod.issue_more(p, sm, my_count, n + 1);
-
+    __syncthreads();  // B2: coefficients ready; this tile's ring bytes are no longer read
+    if (tid == 0) issue_tile<BITS, GATE, IN_BF16>(p, sm, smem, n + C::NS, my_count);
+    const TileId id = tile_id(p, n);
+    uint8_t *gblock = tile_global(p, sm, id);
     if (tid >= D) {
-        const float o = cj * Pj + sm.colH[j];
-        orow[j] = o;
+        const float o = cj * S + sm.colH[j];
+        p.o[((size_t)id.b * p.head_count + id.hr) * D + j] = o;
         if (!isfinite(o)) flag(p.status, kFlagNonfinite);
     }
-    float2 accE[4];
-#pragma unroll
-    for (int pp = 0; pp < 4; ++pp) accE[pp] = make_float2(0.f, 0.f);
-    bool bad_unused = false;
-    sweep_b_update<GATE, true>(sm, Q, pb, warp, sub, cg, accE, bad_unused);
+
+    // ---- Sweep B: y = rho Q + kappa g1 (+ mu g2), column energy ---------------------------
+    tmem_wait_st();
     {
-        float *red = sm.red + (2 * warp + sub) * D + 8 * cg;
-        *reinterpret_cast<float4 *>(red) = f4_of(accE[0], accE[1]);
-        *reinterpret_cast<float4 *>(red + 4) = f4_of(accE[2], accE[3]);
+        float2 g1[4], g2[4], accE[4];
+        load_pairs(sm.colG1 + 8 * cg, g1);
+        if (GATE == 1) load_pairs(sm.colG2 + 8 * cg, g2);
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) accE[pp] = make_float2(0.f, 0.f);
+        bool bad = false;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float2 ch[8];
+            tmem_ld16(tcol + 16 * k, ch);
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int i = 16 * (2 * k + r) + 2 * warp + sub;
+                const float4 rk = sm.rowRK[i];
+                const float2 rho = make_float2(rk.x, rk.y), kap = make_float2(rk.z, rk.w);
+                float2 mu = make_float2(0.f, 0.f);
+                if (GATE == 1) mu = sm.rowMu[i];
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) {
+                    float2 t = __fmul2_rn(kap, g1[pp]);
+                    if (GATE == 1) t = __ffma2_rn(mu, g2[pp], t);
+                    const float2 y = __ffma2_rn(rho, ch[4 * r + pp], t);
+                    ch[4 * r + pp] = y;
+                    if (!pivot) accE[pp] = __ffma2_rn(y, y, accE[pp]);
+                    else bad |= !(fabsf(y.x) < 65520.0f) || !(fabsf(y.y) < 65520.0f);
+                }
+            }
+            if constexpr (pivot) {
+                // an FP16 pivot head stores S' directly
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    uint4 raw;
+                    __half2 h0 = __float22half2_rn(ch[4 * r]), h1 = __float22half2_rn(ch[4 * r + 1]);
+                    __half2 h2 = __float22half2_rn(ch[4 * r + 2]), h3 = __float22half2_rn(ch[4 * r + 3]);
+                    raw.x = *reinterpret_cast<uint32_t *>(&h0);
+                    raw.y = *reinterpret_cast<uint32_t *>(&h1);
+                    raw.z = *reinterpret_cast<uint32_t *>(&h2);
+                    raw.w = *reinterpret_cast<uint32_t *>(&h3);
+                    const int i = 16 * (2 * k + r) + 2 * warp + sub;
+                    *reinterpret_cast<uint4 *>(gblock + i * 256 + cg * 16) = raw;
+                }
+            } else {
+                tmem_st16(tcol + 16 * k, ch);
+            }
+        }
+        if (pivot) {
+            if (bad) flag(p.status, kFlagNonfinite);
+        } else {
+            // both halves of a warp add their partner's energies; half 0 publishes
+#pragma unroll
+            for (int pp = 0; pp < 4; ++pp)
+                accE[pp] = __fadd2_rn(accE[pp], make_float2(__shfl_xor_sync(0xffffffffu, accE[pp].x, 16),
+                                                            __shfl_xor_sync(0xffffffffu, accE[pp].y, 16)));
+            if (sub == 0) {
+                float *red = sm.red + warp * D + 8 * cg;
+                *reinterpret_cast<float4 *>(red) = f4_of(accE[0], accE[1]);
+                *reinterpret_cast<float4 *>(red + 4) = f4_of(accE[2], accE[3]);
+            }
+        }
     }
     __syncthreads();  // B3: column energies complete
 
+    // ---- Warps 0-3: new column scales. Warps 4-7: the next tile's row factors -------------
+    bool ok = true;
     if (tid < D) {
-        float E = 0.f;
-#pragma unroll
-        for (int s = 0; s < 16; ++s) E += sm.red[s * D + j];
-        const float W = sm.rsum[pb][0][0] + sm.rsum[pb][1][0] + sm.rsum[pb][2][0] + sm.rsum[pb][3][0];
-        float c = (cj * inv_sig) * sqrtf(E / W);
-        if (c == 0.f) c = 1.f;
-        reinterpret_cast<float *>(gblock + Wd::SOFF)[D + j] = c;
-        if (!isfinite(c)) flag(p.status, kFlagNonfinite);
-        sm.colB[j] = (cj * inv_sig) / c;
+        if (!pivot) {
+            const float E = sum8(sm.red + j);
+            const float W = sm.rsum[pb][0][0] + sm.rsum[pb][1][0] + sm.rsum[pb][2][0] + sm.rsum[pb][3][0];
+            const float x = E * fast_rcp(W);
+            float c = (cj * inv_sig) * (x * rsqrtf(x));
+            if (!(x > 0.f)) c = (x == 0.f) ? 1.f : c;  // zero column: scale 1 (a NaN stays NaN)
+            reinterpret_cast<float *>(gblock + C::SOFF)[D + j] = c;
+            if (!isfinite(c) || c == 0.f) flag(p.status, kFlagNonfinite);
+            sm.colB[j] = (cj * inv_sig) * fast_rcp(c);
+        }
+    } else {
+        ok = precompute_rows<BITS, GATE, IN_BF16>(sm, smem, n + 1, my_count);
     }
-    __syncthreads();  // B4: new column scales ready
+    if (__syncthreads_or(!ok)) return false;  // B4: new column scales (and next row factors) ready
+    if constexpr (pivot) return true;
 
-    // Sweep C: column-normalised values z and the per-row maxima of |z|.
-    float mx[8];
+    // ---- Sweep C: z = y * c_j / c'_j and the per-row maxima of |z| ---------------------------
+    tmem_wait_st();
+    float *rm = sm.red + (2 * warp + sub) * 128;  // row-max partials of this (warp, half)
     {
         float2 bb[4];
-        const float4 a = *reinterpret_cast<const float4 *>(sm.colB + 8 * cg);
-        const float4 b = *reinterpret_cast<const float4 *>(sm.colB + 8 * cg + 4);
-        bb[0] = make_float2(a.x, a.y); bb[1] = make_float2(a.z, a.w);
-        bb[2] = make_float2(b.x, b.y); bb[3] = make_float2(b.z, b.w);
+        load_pairs(sm.colB + 8 * cg, bb);
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            float v = 0.f;
+        for (int k = 0; k < 4; ++k) {
+            float2 ch[8];
+            tmem_ld16(tcol + 16 * k, ch);
 #pragma unroll
-            for (int pp = 0; pp < 4; ++pp) {
-                Q[m][pp] = __fmul2_rn(Q[m][pp], bb[pp]);
-                v = fmaxf(v, fmaxf(fabsf(Q[m][pp].x), fabsf(Q[m][pp].y)));
+            for (int r = 0; r < 2; ++r) {
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) ch[4 * r + pp] = __fmul2_rn(ch[4 * r + pp], bb[pp]);
+                const float2 *z = ch + 4 * r;
+                const float mx = fmaxf(max3(z[0].x, z[0].y, z[1].x), max3(z[1].y, z[2].x, max3(z[2].y, z[3].x, z[3].y)));
+                const float mn = fminf(min3(z[0].x, z[0].y, z[1].x), min3(z[1].y, z[2].x, min3(z[2].y, z[3].x, z[3].y)));
+                rm[(2 * k + r) * 16 + cg] = fmaxf(mx, -mn);
             }
-            mx[m] = v;
+            tmem_st16(tcol + 16 * k, ch);
         }
     }
-    float *rm = sm.red + (2 * warp + sub) * 128;
-    *reinterpret_cast<float4 *>(rm + 8 * cg) = make_float4(mx[0], mx[1], mx[2], mx[3]);
-    *reinterpret_cast<float4 *>(rm + 8 * cg + 4) = make_float4(mx[4], mx[5], mx[6], mx[7]);
     __syncwarp();
     {
         const int m = cg >> 1, half = cg & 1;
-        float v = 0.f;
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) v = fmaxf(v, rm[(half * 8 + c8) * 8 + m]);
+        const float4 a = *reinterpret_cast<const float4 *>(rm + m * 16 + half * 8);
+        const float4 b = *reinterpret_cast<const float4 *>(rm + m * 16 + half * 8 + 4);
+        float v = max3(max3(a.x, a.y, a.z), max3(a.w, b.x, b.y), fmaxf(b.z, b.w));
         v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
         const int i = 16 * m + 2 * warp + sub;
-        const float sw = sm.rowB[pb][i].x;
-        float r = v / (sw * Wd::QMAX);
+        const float sw = sm.rowSw[pb][i];
+        float r = v * fast_rcp(sw * C::QMAX);
         if (v == 0.f) r = 1.f;
-        const float s = 1.0f / (sw * r);
+        const float s = fast_rcp(sw * r);
         if (half == 0) {
             sm.rowS[i] = make_float2(s, s);
-            reinterpret_cast<float *>(gblock + Wd::SOFF)[i] = r;
+            reinterpret_cast<float *>(gblock + C::SOFF)[i] = r;
             if (!isfinite(r) || r == 0.f) flag(p.status, kFlagNonfinite);
         }
     }
     __syncwarp();
 
-    // Sweep D: x = z s rounded half to even by the 2^23 + offset FFMA, packed and stored in place.
-    const float2 rnd = make_float2(Wd::ROUND, Wd::ROUND);
+    // ---- Sweep D: x = z s rounded half to even by the 2^23 + offset FFMA, packed, stored ----
+    tmem_wait_st();
+    {
+        const float2 rnd = make_float2(C::ROUND, C::ROUND);
+        uint8_t *dstrow = gblock + (2 * warp + sub) * C::RB + cg * BITS;
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const int i = 16 * m + 2 * warp + sub;
-        const float2 s2 = sm.rowS[i];
-        float2 F[4];
+        for (int k = 0; k < 4; ++k) {
+            float2 ch[8];
+            tmem_ld16(tcol + 16 * k, ch);
 #pragma unroll
-        for (int pp = 0; pp < 4; ++pp) F[pp] = __ffma2_rn(Q[m][pp], s2, rnd);
-        pack_store_row<BITS>(gblock + i * Wd::RB + cg * BITS, cg, F);
+            for (int r = 0; r < 2; ++r) {
+                const int m = 2 * k + r;
+                const float2 s2 = sm.rowS[16 * m + 2 * warp + sub];
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) ch[4 * r + pp] = __ffma2_rn(ch[4 * r + pp], s2, rnd);
+                pack_store_row<BITS>(dstrow + 16 * m * C::RB, cg, ch + 4 * r);
+            }
+        }
     }
+    return true;
 }
 
-template <int GATE, int IN_BF16>
-__device__ __forceinline__ void tile_pivot(const TileParams &p, SmemD128 &sm, const uint8_t *tile,
-                                           uint8_t *gblock, float *orow, int pb, int n, int my_count,
-                                           Producer<GATE, IN_BF16> &prod)
+template <int BITS, int GATE, int IN_BF16>
+__global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constant__ TileParams p)
 {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, cg = lane & 15, sub = lane >> 4;
-    float2 Q[8][4];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const uint4 raw = *reinterpret_cast<const uint4 *>(tile + (16 * m + 2 * warp + sub) * 256 + cg * 16);
-        Q[m][0] = __half22float2(*reinterpret_cast<const __half2 *>(&raw.x));
-        Q[m][1] = __half22float2(*reinterpret_cast<const __half2 *>(&raw.y));
-        Q[m][2] = __half22float2(*reinterpret_cast<const __half2 *>(&raw.z));
-        Q[m][3] = __half22float2(*reinterpret_cast<const __half2 *>(&raw.w));
-    }
-    sweep_a_sums(sm, Q, pb, warp, sub, cg);
-    if (tid == 0) prod.store_scalars(sm, pb ^ 1);
-    __syncthreads();  // B1
-
-    const int j = tid & (D - 1);
-    const float Pj = finals_a<GATE, IN_BF16>(sm, tile, 16, pb, 1.f, 1.f, 1.f);
-    __syncthreads();  // B2: this tile's ring bytes are no longer read
-    if (tid == 0) prod.issue_more(p, sm, my_count, n + 1);
-    if (tid >= D) {
-        const float o = Pj + sm.colH[j];
-        orow[j] = o;
-        if (!isfinite(o)) flag(p.status, kFlagNonfinite);
-    }
-    float2 accE[4];
-    bool bad = false;
-    sweep_b_update<GATE, false>(sm, Q, pb, warp, sub, cg, accE, bad);
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        uint4 raw;
-        __half2 h0 = __float22half2_rn(Q[m][0]), h1 = __float22half2_rn(Q[m][1]);
-        __half2 h2 = __float22half2_rn(Q[m][2]), h3 = __float22half2_rn(Q[m][3]);
-        raw.x = *reinterpret_cast<uint32_t *>(&h0);
-        raw.y = *reinterpret_cast<uint32_t *>(&h1);
-        raw.z = *reinterpret_cast<uint32_t *>(&h2);
-        raw.w = *reinterpret_cast<uint32_t *>(&h3);
-        *reinterpret_cast<uint4 *>(gblock + (16 * m + 2 * warp + sub) * 256 + cg * 16) = raw;
-    }
-    if (bad) flag(p.status, kFlagNonfinite);
-}
-
-template <int GATE, int IN_BF16>
-__global__ void __launch_bounds__(NT, 2) decode_d128_kernel(const __grid_constant__ TileParams p)
-{
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    SmemD128 &sm = *reinterpret_cast<SmemD128 *>(smem_raw);
-    const int tid = threadIdx.x;
+    using C = Cfg<BITS, GATE, IN_BF16>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    SmemFixed &sm = *reinterpret_cast<SmemFixed *>(smem);
+    const int tid = threadIdx.x, warp = tid >> 5;
     const int G = (int)gridDim.x;
     const int my_count = (p.ntiles - (int)blockIdx.x + G - 1) / G;
 
     for (int b = tid; b < p.B; b += NT) sm.slots[b] = p.slots[b];
+    if (warp == 0) {  // Tensor Memory for this CTA's tile (released below on every path)
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
+    }
     if (tid == 0) {
-        for (int i = 0; i < NBAR; ++i) mbar_init(smem_u32(&sm.bars[i]), 1);
+        for (int i = 0; i < C::NS; ++i) mbar_init(smem_u32(&sm.bars[i]), 2);
         fence_mbar_init();
+        const float o = BITS == 16 ? 0.f : (float)(1 << (BITS - 1));
+        sm.unpack_off = make_float2(-(8388608.0f + o), -(8388608.0f + o * C::SIG1));
     }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    // this thread's 64 columns: lanes 32*(warp%4).., columns 0..63 (warps 0-3) or 64..127 (4-7)
+    const uint32_t tcol = sm.tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + (warp >= 4 ? 64u : 0u);
 
-    Producer<GATE, IN_BF16> prod;
-    if (tid == 0) {
-        prod.issue_more(p, sm, my_count, 0);
-        prod.load_scalars(p, sm, 0, my_count);
-        prod.store_scalars(sm, 0);
-    }
-    __syncthreads();
+    if (tid == 0)
+        for (int n = 0; n < C::NS; ++n) issue_tile<BITS, GATE, IN_BF16>(p, sm, smem, n, my_count);
+    bool ok = true;
+    if (tid >= D) ok = precompute_rows<BITS, GATE, IN_BF16>(sm, smem, 0, my_count);
+    bool failed = __syncthreads_or(!ok);
 
-    uint32_t c_head = 0, c_wrap = 0;
-    for (int n = 0; n < my_count; ++n) {
-        const TileId id = tile_id(p, (int)blockIdx.x + n * G);
-        uint32_t tpos;  // replays the producer's deterministic placement
-        ring_place(c_head, c_wrap, tile_bytes(id.bits, IN_BF16, GATE), tpos);
-        const uint8_t *tile = sm.ring + tpos;
-        const int pb = n & 1;
-        const bool skip = sm.scal[pb][2] != 0.f;
-        const bool ok = mbar_wait_bounded(smem_u32(&sm.bars[n % NBAR]), (uint32_t)((n / NBAR) & 1));
-        if (tid < D && !skip) precompute_rows<GATE, IN_BF16>(sm, tile, id.bits, pb);
-        if (__syncthreads_or(!ok)) {  // B0
-            if (tid == 0) {
-                flag(p.status, kFlagTimeout);
-                for (int m = n; m < prod.issued; ++m)  // let copies in flight land before exiting
-                    mbar_wait_bounded(smem_u32(&sm.bars[m % NBAR]), (uint32_t)((m / NBAR) & 1));
-            }
-            return;
-        }
-        if (tid == 0) prod.load_scalars(p, sm, n + 1, my_count);
-        if (skip) {
-            if (tid == 0) {
-                prod.store_scalars(sm, pb ^ 1);
-                prod.issue_more(p, sm, my_count, n + 1);
-            }
+    int n = 0;
+    for (; n < my_count && !failed; ++n) {
+        // every thread observes the tile's completion itself (already complete: warps 4-7 waited)
+        const bool got = wait_tile<BITS, GATE, IN_BF16>(sm, n);
+        if (sm.scal[n % C::NS][2] != 0.f) {  // out-of-range slot: nothing loaded, nothing to do
             __syncthreads();
+            if (tid == 0) issue_tile<BITS, GATE, IN_BF16>(p, sm, smem, n + C::NS, my_count);
+            ok = true;
+            if (tid >= D) ok = precompute_rows<BITS, GATE, IN_BF16>(sm, smem, n + 1, my_count);
+            failed = __syncthreads_or(!ok || !got);
             continue;
         }
-        const int slot = sm.slots[id.b];
-        uint8_t *gblock = p.pool + (uint64_t)slot * p.req_bytes + id.off;
-        float *orow = p.o + ((size_t)id.b * p.head_count + id.hr) * D;
-        switch (id.bits) {
-        case 4: tile_quant<4, GATE, IN_BF16>(p, sm, tile, gblock, orow, pb, n, my_count, prod); break;
-        case 6: tile_quant<6, GATE, IN_BF16>(p, sm, tile, gblock, orow, pb, n, my_count, prod); break;
-        case 8: tile_quant<8, GATE, IN_BF16>(p, sm, tile, gblock, orow, pb, n, my_count, prod); break;
-        default: tile_pivot<GATE, IN_BF16>(p, sm, tile, gblock, orow, pb, n, my_count, prod); break;
-        }
+        failed = !process_tile<BITS, GATE, IN_BF16>(p, sm, smem, n, my_count, tcol);
+    }
+    if (failed && tid == 0) {
+        flag(p.status, kFlagTimeout);
+        // let every copy in flight land before the CTA's shared memory is released
+        const int last = (n + C::NS < my_count) ? n + C::NS : my_count;
+        for (int m = n; m < last; ++m) wait_tile<BITS, GATE, IN_BF16>(sm, m);
+    }
+    // release Tensor Memory once every thread's accesses have completed
+    tmem_wait_st();
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(sm.tmem_base), "r"(TMEM_COLS));
     }
 }
 
-template <int GATE, int IN_BF16>
+template <int BITS, int GATE, int IN_BF16>
 cudaError_t launch_t(const TileParams &p, cudaStream_t s)
 {
-    auto kernel = decode_d128_kernel<GATE, IN_BF16>;
-    const int smem = (int)sizeof(SmemD128);
+    using C = Cfg<BITS, GATE, IN_BF16>;
+    auto kernel = decode_d128_kernel<BITS, GATE, IN_BF16>;
+    const int smem = (int)C::SMEM;
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    int sms = 0, per_sm = 0;
+    int sms = 0, smem_sm = 0, regs_sm = 0;
     err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
     if (err != cudaSuccess) return err;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, NT, smem);
+    cudaFuncAttributes fa;
+    err = cudaFuncGetAttributes(&fa, kernel);
     if (err != cudaSuccess) return err;
+    // resident CTAs per SM, from shared memory (+1 KB reserved per CTA), registers and the SM's
+    // 512 Tensor Memory columns (TMEM_COLS per CTA); the runtime's occupancy query does not
+    // model Tensor Memory and reports 1 for kernels that allocate it
+    int per_sm = smem_sm / (smem + 1024);
+    const int by_regs = regs_sm / (NT * (fa.numRegs > 0 ? fa.numRegs : 64));
+    if (by_regs < per_sm) per_sm = by_regs;
+    if (per_sm > (int)(512 / TMEM_COLS)) per_sm = (int)(512 / TMEM_COLS);
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int grid = p.ntiles < sms * per_sm ? p.ntiles : sms * per_sm;
     kernel<<<grid, NT, smem, s>>>(p);
     return cudaGetLastError();
 }
 
+template <int BITS>
+cudaError_t launch_bits(const TileParams &p, int in_bf16, cudaStream_t s)
+{
+    switch (p.gate * 2 + (in_bf16 ? 1 : 0)) {
+    case 0: return launch_t<BITS, 0, 0>(p, s);
+    case 1: return launch_t<BITS, 0, 1>(p, s);
+    case 2: return launch_t<BITS, 1, 0>(p, s);
+    case 3: return launch_t<BITS, 1, 1>(p, s);
+    case 4: return launch_t<BITS, 2, 0>(p, s);
+    default: return launch_t<BITS, 2, 1>(p, s);
+    }
+}
+
 }  // namespace
 
 int decode_d128_max_requests() { return MAXB; }
 
-cudaError_t launch_decode_d128(const TileParams &p, int in_bf16, cudaStream_t s)
+// All entries of p.table have the width `bits`.
+cudaError_t launch_decode_d128(const TileParams &p, int bits, int in_bf16, cudaStream_t s)
 {
-    switch (p.gate * 2 + (in_bf16 ? 1 : 0)) {
-    case 0: return launch_t<0, 0>(p, s);
-    case 1: return launch_t<0, 1>(p, s);
-    case 2: return launch_t<1, 0>(p, s);
-    case 3: return launch_t<1, 1>(p, s);
-    case 4: return launch_t<2, 0>(p, s);
-    default: return launch_t<2, 1>(p, s);
+    switch (bits) {
+    case 4: return launch_bits<4>(p, in_bf16, s);
+    case 6: return launch_bits<6>(p, in_bf16, s);
+    case 8: return launch_bits<8>(p, in_bf16, s);
+    default: return launch_bits<16>(p, in_bf16, s);
     }
 }
 

@@ -228,13 +228,20 @@ stq_status stq_decode_step(const stq_layout *L, void *pool, int32_t pool_slots, 
         p->beta = beta + rq;
         p->alpha = alpha + rq * na;
         p->o = o + rq * L->dv;
-        for (int first = 0; first < head_count; first += stq::kMaxTable) {
-            const int n = std::min(stq::kMaxTable, head_count - first);
+        // the tuned kernel takes one width per launch (largest blocks first); the plain kernel any mix
+        for (int first = 0; first < head_count;) {
+            int n = std::min(stq::kMaxTable, head_count - first);
+            if (tuned) {
+                int same = 1;
+                while (same < n && L->bits[ord[first + same]] == L->bits[ord[first]]) ++same;
+                n = same;
+            }
             fill_table(*p, L, ord, first, n, head_begin);
             p->ntiles = nb * n;
-            const cudaError_t e = tuned ? stq::launch_decode_d128(*p, in_bf16, (cudaStream_t)stream)
+            const cudaError_t e = tuned ? stq::launch_decode_d128(*p, L->bits[ord[first]], in_bf16, (cudaStream_t)stream)
                                         : stq::launch_decode_generic(*p, in_bf16, (cudaStream_t)stream);
             if (e != cudaSuccess) return STQ_ERR_CUDA;
+            first += n;
         }
     }
     return STQ_OK;

@@ -78,7 +78,7 @@ struct TileParams {
 cudaError_t launch_init_generic(const TileParams &p, cudaStream_t s);
 cudaError_t launch_dequant_generic(const TileParams &p, cudaStream_t s);
 cudaError_t launch_decode_generic(const TileParams &p, int in_bf16, cudaStream_t s);
-cudaError_t launch_decode_d128(const TileParams &p, int in_bf16, cudaStream_t s);
+cudaError_t launch_decode_d128(const TileParams &p, int bits, int in_bf16, cudaStream_t s);  // one width per launch
 cudaError_t launch_prefill_seq(const TileParams &p, int in_bf16, int T, int chunk, cudaStream_t s);
 int decode_d128_max_requests();
 
@@ -146,6 +146,19 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
         if (mbar_try_wait(bar, parity)) return true;
         if (clock64() - start > kWaitTimeoutCycles) return false;
     }
+}
+
+// 4-byte asynchronous copy global -> shared (tracked with cp_async_arrive on an mbarrier).
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// The mbarrier receives one arrival when all of this thread's prior cp.async copies have landed
+// (no pending-count increment: the barrier's expected count includes this arrival).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
 // Bulk copy global -> this CTA's shared memory, completing `bytes` on the mbarrier.

@@ -333,3 +333,97 @@ def test_free_running_error_statistics_match_oracle(stq, orc):
     err_g, err_o = np.array(err_g), np.array(err_o)
     assert abs(err_g.mean() / err_o.mean() - 1) < 0.10
     assert abs(np.percentile(err_g, 99) / np.percentile(err_o, 99) - 1) < 0.10
+
+
+def test_partially_invalid_slots(stq, orc):
+    """Tiles of an out-of-range slot are skipped and flagged; the others of the same launch are
+    still computed correctly."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    bits = [4, 16, 8, 6]
+    wl_ = _wl("layer48_b8_4bit", batch=3, heads=4, bits=None)
+    lay = stq.Layout(bits, 128)
+    w = wlm.impact_weights(wl_)
+    S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(3)])
+    opool = _oracle_init(orc, wl_, bits, S0, w)
+    gpool = torch.from_numpy(opool.copy()).to(DEV)
+    slots = torch.tensor([2, 7, 0], dtype=torch.int32, device=DEV)  # request 1 has no valid slot
+    inp = wlm.decode_inputs(wl_, 3)
+    o = torch.zeros(3, 4, 128, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stq.decode_step(lay, gpool, slots, *(inp[n].to(DEV) for n in ("q", "k", "v", "beta", "alpha")), w.to(DEV), o,
+                    status=status)
+    torch.cuda.synchronize()
+    assert status.item() == (1 << stq.api.STQ_ERR_BOUNDS)
+    gp = gpool.cpu().numpy()
+    tally = Tally()
+    for r, slot in ((0, 2), (2, 0)):
+        for h in range(4):
+            pre = tile_bytes(orc, opool, bits, 128, slot, h)
+            res = orc.decode_step(bits[h], 0, pre, as_f64(inp["q"][r, h]), as_f64(inp["k"][r, h]),
+                                  as_f64(inp["v"][r, h]), float(inp["beta"][r, h]), float(inp["alpha"][r, h]),
+                                  as_f64(w[h]), 128, 128)
+            M = update_magnitude(orc.dequantize(16, 128, 128, pre), as_f64(inp["k"][r, h]), as_f64(inp["v"][r, h]),
+                                 float(inp["beta"][r, h]), float(inp["alpha"][r, h])) if bits[h] == 16 else None
+            compare_block(orc, bits[h], 128, tile_bytes(orc, gp, bits, 128, slot, h), res["block"], res["tie"],
+                          tally, err_scale=M)
+            compare_o(o[r, h].cpu().numpy(), res["o"], tally)
+    # slot 1 (not addressed by any request) is untouched
+    assert np.array_equal(gp[lay.bytes_per_request: 2 * lay.bytes_per_request],
+                          opool[lay.bytes_per_request: 2 * lay.bytes_per_request])
+
+
+def test_full_batch70_launch_sampled(stq, orc):
+    """The bench's launch (70 requests x 2304 mixed heads, ~545 tiles per CTA through the staging
+    ring) checked on 96 sampled tiles: their pre-step bytes come from the oracle, every other tile
+    is initialised on the GPU and only has to stay finite."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl_ = wlm.WORKLOADS["full2304_b70_mixed"]
+    B, H, d = wl_.batch, wl_.heads, wl_.d
+    bits = wlm.head_bits(wl_)
+    lay = stq.Layout(bits, d)
+    w = wlm.impact_weights(wl_, DEV)
+    pool = lay.alloc_pool(B)
+    slots = torch.arange(B, dtype=torch.int32, device=DEV)
+    rng = np.random.default_rng(42)
+    heads_by_width = {b: [h for h in range(H) if bits[h] == b] for b in (4, 6, 8, 16)}
+    sample = []
+    for b, hs in heads_by_width.items():
+        for h in rng.choice(hs, size=24, replace=False):
+            sample.append((int(rng.integers(B)), int(h)))
+    S0_sample = {}
+    for r0 in range(0, B, 10):
+        S0 = torch.stack([wlm.initial_state(wl_, r, DEV) for r in range(r0, min(r0 + 10, B))])
+        stq.init_state(lay, pool, slots[r0:r0 + S0.shape[0]].clone(), S0, w)
+        for (r, h) in sample:
+            if r0 <= r < r0 + S0.shape[0]:
+                S0_sample[(r, h)] = S0[r - r0, h].double().cpu().numpy()
+        del S0
+    wc = w.double().cpu().numpy()
+    offs, total = orc.request_layout(bits, d, d)
+    pre = {}
+    for (r, h) in sample:
+        blk, _, _, _ = orc.quantize(bits[h], S0_sample[(r, h)], wc[h])
+        pre[(r, h)] = blk
+        start = r * total + offs[h]
+        pool[start: start + blk.size] = torch.from_numpy(blk).to(DEV)
+    inp = wlm.decode_inputs(wl_, 0, DEV)
+    o = torch.zeros(B, H, d, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stq.decode_step(lay, pool, slots, inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], w, o, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0, stq.status_flags(status)
+    assert torch.isfinite(o).all()
+    tally = Tally()
+    for (r, h) in sample:
+        start = r * total + offs[h]
+        got = pool[start: start + pre[(r, h)].size].cpu().numpy()
+        args = [inp[n][r, h].double().cpu().numpy() for n in ("q", "k", "v")]
+        beta, alpha = float(inp["beta"][r, h]), float(inp["alpha"][r, h])
+        res = orc.decode_step(bits[h], 0, pre[(r, h)], *args, beta, alpha, wc[h], d, d)
+        M = update_magnitude(orc.dequantize(16, d, d, pre[(r, h)]), args[1], args[2], beta, alpha) \
+            if bits[h] == 16 else None
+        compare_block(orc, bits[h], d, got, res["block"], res["tie"], tally, f"req {r} head {h}", err_scale=M)
+        compare_o(o[r, h].cpu().numpy(), res["o"], tally, f"o req {r} head {h}")
+    tally.check_budget()
