@@ -12,16 +12,14 @@
 //
 // Design (B200):
 //  * One persistent kernel per width (FP16 pivots, 8-, 6-, 4-bit), launched largest first; CTAs of
-//    256 threads walk the width's tiles round-robin.
+//    128 threads (four per SM) walk the width's tiles round-robin.
 //  * Thread 0 streams each upcoming tile into a shared-memory slot ring: the packed codes + scales
 //    and the k, q, v, w (and alpha) rows by cp.async.bulk, the per-tile scalars by 4-byte cp.async,
 //    all completing on the slot's mbarrier. Every wait is bounded and reports STQ_ERR_TIMEOUT.
-//  * Each thread owns an 8 x 8 sub-block (rows 16m + 2*warp + half, columns 8*lane16 .. +7) of
-//    the tile, kept in its own lane of Tensor Memory (64 columns) between the sweeps and moved
-//    through registers 16 values at a time (tcgen05.ld / tcgen05.st). With the tile out of the
-//    register file a thread needs <= 64 registers, so four CTAs (32 warps) share an SM and hide
-//    each other's barrier and latency stalls; the state is still read from HBM once and written
-//    once per step.
+//  * Thread (warp w, lane l) owns a 16 x 8 sub-block of the tile: rows 8m + 2w + l/16 (m < 16),
+//    columns 8 (l%16) .. +7. Its 128 values live in its own lane of Tensor Memory (lane 32w + l,
+//    128 columns) between the sweeps and pass through registers 8 or 16 at a time (tcgen05.st /
+//    tcgen05.ld); the state is read from HBM once and written once per step.
 //  * The algebra runs in column-normalised coordinates: with y_ij = sqrt(w_i) S'_ij / c_j,
 //      y_ij = rho_i Q_ij + kappa_i g_j   (rho = alpha sqrt(w) r, kappa = sqrt(w) k, g = h / c,
 //                                         h = beta (v - alpha u))
@@ -30,10 +28,10 @@
 //    (exact; odd columns carry a power-of-two factor sigma, folded back per column) and rounded
 //    back with one FFMA against 2^23 + 2^(b-1), which rounds half to even for free.
 //  * Four CTA barriers per tile: column sums of k~Q and q~Q (B1), the update coefficients (B2),
-//    the column energies (B3) and the new column scales (B4). Column partials are first summed
-//    between the two half-warps by shuffles, then across warps through shared memory; row maxima
-//    stay inside a warp. The next tile's row factors are computed by warps 4-7 while warps 0-3
-//    finish the column scales.
+//    the column energies (B3) and the new column scales with the next tile's row factors (B4).
+//    Every thread takes one column (and one row) in each of these steps. Column partials are
+//    summed between the two half-warps by shuffles, then across the four warps through shared
+//    memory; row maxima stay inside a half-warp.
 //  * Scale arithmetic (reciprocals, square roots) uses the SFU approximations (a few ulp): the
 //    codes are always computed from the scales this kernel stores.
 #include "stq_internal.cuh"
@@ -42,29 +40,55 @@ namespace stq {
 namespace {
 
 constexpr int D = 128;
-constexpr int NT = 256;
+constexpr int NT = 128;                // threads per CTA: one tile at a time
 constexpr int NSMAX = 4;               // slots (tiles in flight) per CTA
 constexpr int MAXB = 256;              // requests per launch whose slots are cached in smem
 constexpr uint32_t MAGIC = 0x4B000000u;  // bit pattern of 2^23
-constexpr uint32_t TMEM_COLS = 128;    // per CTA: 2 x 64 columns (warps 0-3 / 4-7) over 128 lanes
+constexpr uint32_t TMEM_COLS = 128;    // per CTA: 128 lanes x 128 columns of fp32 = one tile
+// red[]: one region of RS floats per (warp, half) k = 2w + h. [0, 128): the half's column
+// partials (k~Q for h = 0, q~Q for h = 1); [128, 256) of the h = 0 region: the warp's column
+// energies; later the half's 16 row-max partial rows of RM floats. Only warp w writes its two
+// regions while other warps may be reading, so a warp never overwrites data still in use.
+constexpr int RM = 20;                 // row stride of the row-max partials (bank-conflict free)
+constexpr int RS = 336;                // region stride (= 16 mod 32 banks: the halves do not collide)
+
+// Thread 0's cursor over this CTA's tiles t = blockIdx.x + n * gridDim.x, kept as (table
+// position, request) = (t / B, t % B) and advanced without a division.
+struct Issuer {
+    int n, pos, b, qG, rG;
+};
+
+// Per tile, written by the issuing thread: where the tile lives and which input row it uses.
+struct SlotMeta {
+    unsigned long long gblock;  // address of the tile's head block in the pool
+    uint32_t orow;              // request * head_count + head: the row of q, k, v, beta, alpha, o
+    uint32_t skip;              // 1: out-of-range slot, nothing was loaded
+};
 
 struct __align__(16) SmemFixed {
-    float red[2 * 8 * D];    // column partials (U/P per warp; E per warp), then row-max partials
+    float red[8 * RS];
     float4 rowKQ[D];         // (k~, k~, q~, q~)
     float4 rowRK[D];         // (rho, rho, kappa, kappa)
-    float2 rowMu[D];         // (mu, mu)  (literal channel gate)
-    float rowSw[2][D];       // per tile parity: sqrt(w)
+    float rowRq[2][D];       // per tile parity: 1 / (sqrt(w_i) qmax)
+    float2 rowS[D];          // (s_i, s_i), s_i = 1 / (sqrt(w_i) r'_i) = qmax / max_j |z_ij|
     float colG1[D];
-    float colG2[D];
-    float colH[D];           // rank-1 part of the readout
-    float colB[D];           // c_j / (sigma_j c'_j)
-    float2 rowS[D];          // (s_i, s_i), s_i = 1 / (sqrt(w_i) r'_i)
-    float rsum[2][4][4];     // per parity, per precompute warp: sum w, q.k, q.(alpha*k)
-    float scal[NSMAX][4];    // per slot: beta, alpha, skip
+    float colB[D];           // c_j / (sigma_j c'_j) = 1 / sqrt(x_j)
+    float rsum[2][4][4];     // per parity, per warp: sum w, q.k, q.(alpha*k)
+    float scal[NSMAX][2];    // per slot: beta, alpha
+    SlotMeta meta[4];        // per tile n, at n % 4 (NS + 1 <= 4 tiles are live at a time)
+    Issuer iss;              // thread 0's tile cursor
     int32_t slots[MAXB];
     unsigned long long bars[NSMAX];
     float2 unpack_off;       // (-(2^23 + o), -(2^23 + o * SIG1)), o = 2^(b-1)
+    uint32_t magic;          // 0x4B000000, read at run time so the unpack keeps it in a register
+                             // and forms each value with one LOP3 ((s & mask) | magic)
     uint32_t tmem_base;
+};
+
+// Only the literal channel gate (gate 1) needs these; they follow SmemFixed when present.
+struct __align__(16) SmemChannel {
+    float2 rowMu[D];         // (mu, mu)
+    float colG2[D];
 };
 
 // ---------------------------------------------------------------------------------------------
@@ -79,9 +103,10 @@ struct Cfg {
     static constexpr uint32_t K_OFF = BLK, Q_OFF = BLK + ROW_IN, V_OFF = BLK + 2 * ROW_IN;
     static constexpr uint32_t W_OFF = BLK + 3 * ROW_IN, A_OFF = W_OFF + 4 * D;
     static constexpr uint32_t LEN = A_OFF + (GATE != 0 ? 4u * D : 0u);  // a multiple of 256
-    // slots so that four CTAs fit an SM's 228 KB for the 4- and 6-bit kernels
+    static constexpr uint32_t RING = (uint32_t)sizeof(SmemFixed) + (GATE == 1 ? (uint32_t)sizeof(SmemChannel) : 0u);
+    // slots so that four CTAs fit an SM's 228 KB where they can
     static constexpr int NS = BITS == 4 ? 3 : 2;
-    static constexpr size_t SMEM = sizeof(SmemFixed) + (size_t)NS * LEN;
+    static constexpr size_t SMEM = RING + (size_t)NS * LEN;
     static constexpr float QMAX = BITS == 16 ? 0.f : (float)((1 << (BITS - 1)) - 1);
     static constexpr float ROUND = 8388608.0f + (BITS == 16 ? 0.f : (float)(1 << (BITS - 1)));
     // odd columns are unpacked scaled by SIG1 (even columns by 1)
@@ -97,17 +122,13 @@ __device__ __forceinline__ float max3(float a, float b, float c)
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
 }
-__device__ __forceinline__ float min3(float a, float b, float c)
-{
-    float d;
-    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
 
 __device__ __forceinline__ float fast_rcp(float x) { return __fdividef(1.0f, x); }
 
 // ---------------------------------------------------------------------------------------------
-// Tensor Memory: each thread keeps its 64 values in 64 consecutive columns of its own lane.
+// Tensor Memory: each thread keeps its values in consecutive columns of its own lane. The loads
+// and stores carry no memory clobber (they touch only Tensor Memory), so shared-memory loads can
+// be scheduled across them; their ordering with each other is kept by the waits.
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float2 (&v)[8])
 {
@@ -115,10 +136,15 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float2 (&v)[8])
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
         "%13, %14, %15, %16};" ::"r"(taddr),
         "f"(v[0].x), "f"(v[0].y), "f"(v[1].x), "f"(v[1].y), "f"(v[2].x), "f"(v[2].y), "f"(v[3].x), "f"(v[3].y),
-        "f"(v[4].x), "f"(v[4].y), "f"(v[5].x), "f"(v[5].y), "f"(v[6].x), "f"(v[6].y), "f"(v[7].x), "f"(v[7].y)
-        : "memory");
+        "f"(v[4].x), "f"(v[4].y), "f"(v[5].x), "f"(v[5].y), "f"(v[6].x), "f"(v[6].y), "f"(v[7].x), "f"(v[7].y));
 }
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float2 (&v)[8])
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float2 (&v)[4])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "f"(v[0].x), "f"(v[0].y), "f"(v[1].x), "f"(v[1].y), "f"(v[2].x), "f"(v[2].y), "f"(v[3].x), "f"(v[3].y));
+}
+// Start loading 16 values; they may be read only after tmem_wait_ld on the same array.
+__device__ __forceinline__ void tmem_ld16_async(uint32_t taddr, float2 (&v)[8])
 {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
@@ -126,31 +152,40 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float2 (&v)[8])
         : "=f"(v[0].x), "=f"(v[0].y), "=f"(v[1].x), "=f"(v[1].y), "=f"(v[2].x), "=f"(v[2].y), "=f"(v[3].x),
           "=f"(v[3].y), "=f"(v[4].x), "=f"(v[4].y), "=f"(v[5].x), "=f"(v[5].y), "=f"(v[6].x), "=f"(v[6].y),
           "=f"(v[7].x), "=f"(v[7].y)
-        : "r"(taddr)
-        : "memory");
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        : "r"(taddr));
+}
+// Wait for this thread's outstanding Tensor Memory loads. The array is passed through as
+// read-write operands so that no use of it can be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld(float2 (&v)[8])
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+f"(v[0].x), "+f"(v[0].y), "+f"(v[1].x), "+f"(v[1].y), "+f"(v[2].x), "+f"(v[2].y), "+f"(v[3].x),
+                   "+f"(v[3].y), "+f"(v[4].x), "+f"(v[4].y), "+f"(v[5].x), "+f"(v[5].y), "+f"(v[6].x), "+f"(v[6].y),
+                   "+f"(v[7].x), "+f"(v[7].y)
+                 :
+                 : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Two adjacent codes at bits [0, BITS) and [BITS, 2*BITS) of s, as (2^23 + u0, 2^23 + u1 * 2^BITS).
 template <int BITS>
-__device__ __forceinline__ float2 code_pair(uint32_t s)
+__device__ __forceinline__ float2 code_pair(uint32_t s, uint32_t magic)
 {
     constexpr uint32_t M = (1u << BITS) - 1u;
-    return make_float2(f_of((s & M) | MAGIC), f_of((s & (M << BITS)) | MAGIC));
+    return make_float2(f_of((s & M) | magic), f_of((s & (M << BITS)) | magic));
 }
 
 // Unpack the 8 codes of one thread's row segment (in shared memory) into (Q, SIG1 * Q) pairs;
 // `off` = (-(2^23 + o), -(2^23 + o * SIG1)) with o = 2^(b-1). A pivot row holds 8 halves.
 template <int BITS>
-__device__ __forceinline__ void unpack_row(const uint8_t *src, int cg, float2 off, float2 *Q)
+__device__ __forceinline__ void unpack_row(const uint8_t *src, int cg, float2 off, uint32_t magic, float2 *Q)
 {
     if constexpr (BITS == 4) {
         const uint32_t wd = *reinterpret_cast<const uint32_t *>(src);
-        Q[0] = __fadd2_rn(code_pair<4>(wd), off);
-        Q[1] = __fadd2_rn(code_pair<4>(wd >> 8), off);
-        Q[2] = __fadd2_rn(code_pair<4>(wd >> 16), off);
-        Q[3] = __fadd2_rn(code_pair<4>(wd >> 24), off);
+        Q[0] = __fadd2_rn(code_pair<4>(wd, magic), off);
+        Q[1] = __fadd2_rn(code_pair<4>(wd >> 8, magic), off);
+        Q[2] = __fadd2_rn(code_pair<4>(wd >> 16, magic), off);
+        Q[3] = __fadd2_rn(code_pair<4>(wd >> 24, magic), off);
     } else if constexpr (BITS == 6) {
         uint32_t lo, hi;
         if ((cg & 1) == 0) {
@@ -161,16 +196,16 @@ __device__ __forceinline__ void unpack_row(const uint8_t *src, int cg, float2 of
             lo = (uint32_t)(*reinterpret_cast<const uint16_t *>(src)) | (w1 << 16);
             hi = w1 >> 16;
         }
-        Q[0] = __fadd2_rn(code_pair<6>(lo), off);
-        Q[1] = __fadd2_rn(code_pair<6>(lo >> 12), off);
-        Q[2] = __fadd2_rn(code_pair<6>(__funnelshift_r(lo, hi, 24)), off);
-        Q[3] = __fadd2_rn(code_pair<6>(hi >> 4), off);
+        Q[0] = __fadd2_rn(code_pair<6>(lo, magic), off);
+        Q[1] = __fadd2_rn(code_pair<6>(lo >> 12, magic), off);
+        Q[2] = __fadd2_rn(code_pair<6>(__funnelshift_r(lo, hi, 24), magic), off);
+        Q[3] = __fadd2_rn(code_pair<6>(hi >> 4, magic), off);
     } else if constexpr (BITS == 8) {
         const uint2 wd = *reinterpret_cast<const uint2 *>(src);
-        Q[0] = __fadd2_rn(make_float2(f_of(__byte_perm(wd.x, MAGIC, 0x7650)), f_of(__byte_perm(wd.x, MAGIC, 0x7651))), off);
-        Q[1] = __fadd2_rn(make_float2(f_of(__byte_perm(wd.x, MAGIC, 0x7652)), f_of(__byte_perm(wd.x, MAGIC, 0x7653))), off);
-        Q[2] = __fadd2_rn(make_float2(f_of(__byte_perm(wd.y, MAGIC, 0x7650)), f_of(__byte_perm(wd.y, MAGIC, 0x7651))), off);
-        Q[3] = __fadd2_rn(make_float2(f_of(__byte_perm(wd.y, MAGIC, 0x7652)), f_of(__byte_perm(wd.y, MAGIC, 0x7653))), off);
+        Q[0] = __fadd2_rn(make_float2(f_of(__byte_perm(wd.x, magic, 0x7650)), f_of(__byte_perm(wd.x, magic, 0x7651))), off);
+        Q[1] = __fadd2_rn(make_float2(f_of(__byte_perm(wd.x, magic, 0x7652)), f_of(__byte_perm(wd.x, magic, 0x7653))), off);
+        Q[2] = __fadd2_rn(make_float2(f_of(__byte_perm(wd.y, magic, 0x7650)), f_of(__byte_perm(wd.y, magic, 0x7651))), off);
+        Q[3] = __fadd2_rn(make_float2(f_of(__byte_perm(wd.y, magic, 0x7652)), f_of(__byte_perm(wd.y, magic, 0x7653))), off);
     } else {
         const uint4 raw = *reinterpret_cast<const uint4 *>(src);
         Q[0] = __half22float2(*reinterpret_cast<const __half2 *>(&raw.x));
@@ -224,109 +259,109 @@ __device__ __forceinline__ void load_pairs(const float *src, float2 (&out)[4])
     out[3] = make_float2(b.z, b.w);
 }
 
-// Sum of 8 per-warp partials with a short dependency chain.
-__device__ __forceinline__ float sum8(const float *src)
+// Sum of the 4 per-warp partials at `stride` floats apart.
+__device__ __forceinline__ float sum4(const float *src, int stride)
 {
-    return ((src[0] + src[D]) + (src[2 * D] + src[3 * D])) + ((src[4 * D] + src[5 * D]) + (src[6 * D] + src[7 * D]));
-}
-
-struct TileId {
-    int b, hr;
-    uint32_t off;
-};
-
-__device__ __forceinline__ TileId tile_id(const TileParams &p, int n)
-{
-    const int t = (int)blockIdx.x + n * (int)gridDim.x;
-    const int pos = t / p.B;
-    TileId id;
-    id.b = t - pos * p.B;
-    const TileEntry e = p.table[pos];
-    id.hr = entry_head(e);
-    id.off = e.off;
-    return id;
+    return (src[0] + src[stride]) + (src[2 * stride] + src[3 * stride]);
 }
 
 template <int BITS, int GATE, int IN_BF16>
-__device__ __forceinline__ uint8_t *ring_slot(uint8_t *smem, int n)
+__device__ __forceinline__ uint8_t *ring_slot(uint8_t *smem, int slot_i)
 {
-    return smem + sizeof(SmemFixed) + (size_t)(n % Cfg<BITS, GATE, IN_BF16>::NS) * Cfg<BITS, GATE, IN_BF16>::LEN;
+    return smem + Cfg<BITS, GATE, IN_BF16>::RING + (size_t)slot_i * Cfg<BITS, GATE, IN_BF16>::LEN;
 }
 
-// Thread 0: stream tile n into slot n % NS (codes + scales, rows by bulk copy; scalars by
-// 4-byte cp.async), completing on the slot's mbarrier (two arrivals: expect_tx + cp.async).
+__device__ __forceinline__ SmemChannel &channel(uint8_t *smem)
+{
+    return *reinterpret_cast<SmemChannel *>(smem + sizeof(SmemFixed));
+}
+
+// Thread 0: stream this CTA's next tile into ring slot n % NS (codes + scales and the input rows
+// by bulk copy, the per-tile scalars by 4-byte cp.async), completing on the slot's mbarrier (two
+// arrivals: expect_tx + cp.async), and record where the tile lives and which row it reads.
 template <int BITS, int GATE, int IN_BF16>
-__device__ __forceinline__ void issue_tile(const TileParams &p, SmemFixed &sm, uint8_t *smem, int n, int my_count)
+__device__ __forceinline__ void issue_next(const TileParams &p, SmemFixed &sm, uint8_t *smem, Issuer &it, int my_count)
 {
     using C = Cfg<BITS, GATE, IN_BF16>;
-    if (n >= my_count) return;
-    const int slot_i = n % C::NS;
-    const TileId id = tile_id(p, n);
+    if (it.n >= my_count) return;
+    const int n = it.n, slot_i = n % C::NS;
+    const TileEntry e = p.table[it.pos];
+    const int hr = entry_head(e), b = it.b;
+    ++it.n;
+    it.b += it.rG;
+    it.pos += it.qG;
+    if (it.b >= p.B) {
+        it.b -= p.B;
+        ++it.pos;
+    }
     const uint32_t bar = smem_u32(&sm.bars[slot_i]);
-    const int slot = sm.slots[id.b];
+    const uint32_t row = (uint32_t)b * (uint32_t)p.head_count + (uint32_t)hr;
+    SlotMeta &m = sm.meta[n & 3];
+    m.orow = row;
+    const int slot = sm.slots[b];
     if (slot < 0 || slot >= p.pool_slots) {
         flag(p.status, kFlagBounds);
-        sm.scal[slot_i][2] = 1.f;
+        m.skip = 1u;
+        m.gblock = 0ull;
         mbar_arrive(bar);
         mbar_arrive(bar);
         return;
     }
-    sm.scal[slot_i][2] = 0.f;
-    const size_t row = (size_t)id.b * p.head_count + id.hr;
+    const uint8_t *src = p.pool + (uint64_t)slot * p.req_bytes + e.off;
+    m.skip = 0u;
+    m.gblock = reinterpret_cast<unsigned long long>(src);
     cp_async4(smem_u32(&sm.scal[slot_i][0]), p.beta + row);
     if (GATE == 0) cp_async4(smem_u32(&sm.scal[slot_i][1]), p.alpha + row);
     cp_async_arrive(bar);
-    const uint32_t dst = smem_u32(ring_slot<BITS, GATE, IN_BF16>(smem, n));
+    const uint32_t dst = smem_u32(ring_slot<BITS, GATE, IN_BF16>(smem, slot_i));
     mbar_arrive_expect_tx(bar, C::LEN);
-    bulk_g2s(dst, p.pool + (uint64_t)slot * p.req_bytes + id.off, C::BLK, bar);
-    bulk_g2s(dst + C::K_OFF, (const uint8_t *)p.k + row * C::ROW_IN, C::ROW_IN, bar);
-    bulk_g2s(dst + C::Q_OFF, (const uint8_t *)p.q + row * C::ROW_IN, C::ROW_IN, bar);
-    bulk_g2s(dst + C::V_OFF, (const uint8_t *)p.v + row * C::ROW_IN, C::ROW_IN, bar);
-    bulk_g2s(dst + C::W_OFF, p.w + (size_t)id.hr * D, 4 * D, bar);
-    if (GATE != 0) bulk_g2s(dst + C::A_OFF, p.alpha + row * D, 4 * D, bar);
+    bulk_g2s(dst, src, C::BLK, bar);
+    bulk_g2s(dst + C::K_OFF, (const uint8_t *)p.k + (size_t)row * C::ROW_IN, C::ROW_IN, bar);
+    bulk_g2s(dst + C::Q_OFF, (const uint8_t *)p.q + (size_t)row * C::ROW_IN, C::ROW_IN, bar);
+    bulk_g2s(dst + C::V_OFF, (const uint8_t *)p.v + (size_t)row * C::ROW_IN, C::ROW_IN, bar);
+    bulk_g2s(dst + C::W_OFF, p.w + (size_t)hr * D, 4 * D, bar);
+    if (GATE != 0) bulk_g2s(dst + C::A_OFF, p.alpha + (size_t)row * D, 4 * D, bar);
 }
 
-template <int BITS, int GATE, int IN_BF16>
-__device__ __forceinline__ bool wait_tile(SmemFixed &sm, int n)
-{
-    using C = Cfg<BITS, GATE, IN_BF16>;
-    return mbar_wait_bounded(smem_u32(&sm.bars[n % C::NS]), (uint32_t)((n / C::NS) & 1));
-}
-
-// Wait for tile n and compute its row factors: run by the 128 threads of warps 4-7 (row
-// i = tid - 128), with per-warp sums of w, q.k and q.(alpha k). Returns false on a timeout.
+// Wait for tile n (ring slot n % NS) and compute its row factors, row i = threadIdx.x, with
+// per-warp sums of w, q.k and q.(alpha k). Returns false on a timeout.
 template <int BITS, int GATE, int IN_BF16>
 __device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, int n, int my_count)
 {
     using C = Cfg<BITS, GATE, IN_BF16>;
     if (n >= my_count) return true;
-    // the verdict is made warp-uniform before any warp-wide shuffle below
-    if (!__all_sync(0xffffffffu, wait_tile<BITS, GATE, IN_BF16>(sm, n))) return false;
     const int slot_i = n % C::NS;
-    if (sm.scal[slot_i][2] != 0.f) return true;  // skipped tile: nothing was loaded
+    const uint32_t phase = (uint32_t)(n / C::NS) & 1u;
+    // the verdict is made warp-uniform before any warp-wide shuffle below
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&sm.bars[slot_i]), phase))) return false;
+    if (sm.meta[n & 3].skip) return true;  // skipped tile: nothing was loaded
     const int pb = n & 1;
-    const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16>(smem, n);
-    const int i = threadIdx.x - D;
+    const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16>(smem, slot_i);
+    const int i = threadIdx.x;
     constexpr bool pivot = BITS == 16;
     const float r = pivot ? 1.f : reinterpret_cast<const float *>(tile + C::SOFF)[i];
     const float k = load_in<IN_BF16>(tile + C::K_OFF, i);
     const float q = load_in<IN_BF16>(tile + C::Q_OFF, i);
     const float w = reinterpret_cast<const float *>(tile + C::W_OFF)[i];
     const float a = GATE == 0 ? sm.scal[slot_i][1] : reinterpret_cast<const float *>(tile + C::A_OFF)[i];
-    const float sw = pivot ? 1.f : sqrtf(w);
+    // sqrt(w) for w > 0 (the weights are positive) from the SFU reciprocal square root
+    const float sw = pivot ? 1.f : w * rsqrtf(w);
     const float kt = (GATE == 2 ? k * a : k) * r;
     const float qt = q * a * r;
-    const float rho = a * sw * r, kap = sw * k, mu = -sw * a * k;
+    const float rho = a * sw * r, kap = sw * k;
     sm.rowKQ[i] = make_float4(kt, kt, qt, qt);
     sm.rowRK[i] = make_float4(rho, rho, kap, kap);
-    if (GATE == 1) sm.rowMu[i] = make_float2(mu, mu);
-    sm.rowSw[pb][i] = sw;
+    if (GATE == 1) {
+        const float mu = -sw * a * k;
+        channel(smem).rowMu[i] = make_float2(mu, mu);
+    }
+    if (!pivot) sm.rowRq[pb][i] = fast_rcp(sw * C::QMAX);
     float s0 = w, s1 = q * k, s2 = q * a * k;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         s0 += __shfl_xor_sync(0xffffffffu, s0, o);
         s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-        s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+        if (GATE == 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
     }
     if ((i & 31) == 0) {
         sm.rsum[pb][i >> 5][0] = s0;
@@ -336,12 +371,7 @@ __device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, in
     return true;
 }
 
-__device__ __forceinline__ uint8_t *tile_global(const TileParams &p, const SmemFixed &sm, const TileId &id)
-{
-    return p.pool + (uint64_t)sm.slots[id.b] * p.req_bytes + id.off;
-}
-
-// One tile; returns false if the wait for the next tile timed out.
+// Tile n (ring slot n % NS). Returns false if the wait for the next tile timed out.
 template <int BITS, int GATE, int IN_BF16>
 __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm, uint8_t *smem, int n, int my_count,
                                              uint32_t tcol)
@@ -349,35 +379,33 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
     using C = Cfg<BITS, GATE, IN_BF16>;
     constexpr bool pivot = BITS == 16;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, cg = lane & 15, sub = lane >> 4;
-    const int slot_i = n % C::NS, pb = n & 1;
-    const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16>(smem, n);
-    const uint8_t *rowsrc = tile + (2 * warp + sub) * C::RB + cg * (pivot ? 16 : BITS);
+    const int pb = n & 1, slot_i = n % C::NS;
+    const int rb = 2 * warp + sub;  // this thread's rows: rb + 8m, m < 16
+    const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16>(smem, slot_i);
+    // the tile's record (sm.meta[n & 3]) stays valid until the issue after the next tile's B2
 
     // ---- Sweep A: unpack to TMEM, column sums of k~Q and q~Q -------------------------------
     {
+        const uint8_t *rowsrc = tile + rb * C::RB + cg * (pivot ? 16 : BITS);
         const float2 off = sm.unpack_off;
+        const uint32_t magic = sm.magic;
         float2 accU[4], accP[4];
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp) accU[pp] = accP[pp] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            float2 ch[8];
+        for (int m = 0; m < 16; ++m) {
+            float2 ch[4];
+            unpack_row<BITS>(rowsrc + 8 * m * C::RB, cg, off, magic, ch);
+            const float4 kq = sm.rowKQ[8 * m + rb];
+            const float2 kk = make_float2(kq.x, kq.y), qq = make_float2(kq.z, kq.w);
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int m = 2 * k + r;
-                unpack_row<BITS>(rowsrc + 16 * m * C::RB, cg, off, ch + 4 * r);
-                const float4 kq = sm.rowKQ[16 * m + 2 * warp + sub];
-                const float2 kk = make_float2(kq.x, kq.y), qq = make_float2(kq.z, kq.w);
-#pragma unroll
-                for (int pp = 0; pp < 4; ++pp) {
-                    accU[pp] = __ffma2_rn(kk, ch[4 * r + pp], accU[pp]);
-                    accP[pp] = __ffma2_rn(qq, ch[4 * r + pp], accP[pp]);
-                }
+            for (int pp = 0; pp < 4; ++pp) {
+                accU[pp] = __ffma2_rn(kk, ch[pp], accU[pp]);
+                accP[pp] = __ffma2_rn(qq, ch[pp], accP[pp]);
             }
-            tmem_st16(tcol + 16 * k, ch);
+            tmem_st8(tcol + 8 * m, ch);
         }
         // halves 0/1 of a warp hold the same columns: half 0 keeps U, half 1 keeps P
-        float *red = sm.red + (sub * 8 + warp) * D + 8 * cg;
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp) {
             const float2 send = sub ? accU[pp] : accP[pp];
@@ -386,64 +414,67 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
                                            __shfl_xor_sync(0xffffffffu, send.y, 16));
             accU[pp] = __fadd2_rn(keep, got);
         }
-        *reinterpret_cast<float4 *>(red) = f4_of(accU[0], accU[1]);
-        *reinterpret_cast<float4 *>(red + 4) = f4_of(accU[2], accU[3]);
+        float *dst = sm.red + rb * RS + 8 * cg;
+        *reinterpret_cast<float4 *>(dst) = f4_of(accU[0], accU[1]);
+        *reinterpret_cast<float4 *>(dst + 4) = f4_of(accU[2], accU[3]);
     }
     __syncthreads();  // B1: column partials complete
 
-    // ---- Column finals: warps 0-3 the update coefficients, warps 4-7 the readout sums ------
-    const int j = tid & (D - 1);
+    // ---- Column finals (column j = tid): update coefficients and the readout ---------------
+    const int j = tid;
     const float cj = pivot ? 1.f : reinterpret_cast<const float *>(tile + C::SOFF)[D + j];
-    const float sig = (j & 1) ? C::SIG1 : 1.f;
     const float inv_sig = (j & 1) ? 1.f / C::SIG1 : 1.f;  // powers of two: exact
-    const float S = sum8(sm.red + (tid < D ? 0 : 8 * D) + j) * inv_sig;
-    if (tid < D) {
+    {
+        // k~Q partials in the half-0 regions (0, 2, 4, 6), q~Q partials in the half-1 regions
+        const float U = sum4(sm.red + j, 2 * RS) * inv_sig;
+        const float P = sum4(sm.red + RS + j, 2 * RS) * inv_sig;
+        const float sig = (j & 1) ? C::SIG1 : 1.f;
         const float beta = sm.scal[slot_i][0], alpha = sm.scal[slot_i][1];
         const float vj = load_in<IN_BF16>(tile + C::V_OFF, j);
         const float qk = sm.rsum[pb][0][1] + sm.rsum[pb][1][1] + sm.rsum[pb][2][1] + sm.rsum[pb][3][1];
-        const float u = cj * S;
+        const float u = cj * U;
         const float rc = pivot ? 1.f : fast_rcp(cj);
+        float o;
         if (GATE == 1) {
             const float qak = sm.rsum[pb][0][2] + sm.rsum[pb][1][2] + sm.rsum[pb][2][2] + sm.rsum[pb][3][2];
             sm.colG1[j] = sig * (beta * vj) * rc;
-            sm.colG2[j] = sig * (beta * u) * rc;
-            sm.colH[j] = qk * beta * vj - qak * beta * u;
+            channel(smem).colG2[j] = sig * (beta * u) * rc;
+            o = cj * P + (qk * beta * vj - qak * beta * u);
         } else {
             const float h = GATE == 0 ? beta * (vj - alpha * u) : beta * (vj - u);
             sm.colG1[j] = sig * h * rc;
-            sm.colH[j] = qk * h;
+            o = cj * P + qk * h;
         }
-    }
-    __syncthreads();  // B2: coefficients ready; this tile's ring bytes are no longer read
-    if (tid == 0) issue_tile<BITS, GATE, IN_BF16>(p, sm, smem, n + C::NS, my_count);
-    const TileId id = tile_id(p, n);
-    uint8_t *gblock = tile_global(p, sm, id);
-    if (tid >= D) {
-        const float o = cj * S + sm.colH[j];
-        p.o[((size_t)id.b * p.head_count + id.hr) * D + j] = o;
+        p.o[(size_t)sm.meta[n & 3].orow * D + j] = o;
         if (!isfinite(o)) flag(p.status, kFlagNonfinite);
     }
+    __syncthreads();  // B2: coefficients ready; this tile's ring bytes are no longer read
+    if (tid == 0) issue_next<BITS, GATE, IN_BF16>(p, sm, smem, sm.iss, my_count);
 
     // ---- Sweep B: y = rho Q + kappa g1 (+ mu g2), column energy ---------------------------
     tmem_wait_st();
     {
         float2 g1[4], g2[4], accE[4];
         load_pairs(sm.colG1 + 8 * cg, g1);
-        if (GATE == 1) load_pairs(sm.colG2 + 8 * cg, g2);
+        if (GATE == 1) load_pairs(channel(smem).colG2 + 8 * cg, g2);
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp) accE[pp] = make_float2(0.f, 0.f);
         bool bad = false;
+        float2 cha[8], chb[8];
+        tmem_ld16_async(tcol, cha);
+        tmem_wait_ld(cha);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            float2 ch[8];
-            tmem_ld16(tcol + 16 * k, ch);
+        for (int k = 0; k < 8; ++k) {
+            float2 (&ch)[8] = (k & 1) ? chb : cha;
+            float2 (&nx)[8] = (k & 1) ? cha : chb;
+            if (k + 1 < 8) tmem_ld16_async(tcol + 16 * (k + 1), nx);
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-                const int i = 16 * (2 * k + r) + 2 * warp + sub;
+                const int i = 8 * (2 * k + r) + rb;
                 const float4 rk = sm.rowRK[i];
                 const float2 rho = make_float2(rk.x, rk.y), kap = make_float2(rk.z, rk.w);
                 float2 mu = make_float2(0.f, 0.f);
-                if (GATE == 1) mu = sm.rowMu[i];
+                if (GATE == 1) mu = channel(smem).rowMu[i];
 #pragma unroll
                 for (int pp = 0; pp < 4; ++pp) {
                     float2 t = __fmul2_rn(kap, g1[pp]);
@@ -456,6 +487,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
             }
             if constexpr (pivot) {
                 // an FP16 pivot head stores S' directly
+                uint8_t *gblock = reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock);
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
                     uint4 raw;
@@ -465,12 +497,13 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
                     raw.y = *reinterpret_cast<uint32_t *>(&h1);
                     raw.z = *reinterpret_cast<uint32_t *>(&h2);
                     raw.w = *reinterpret_cast<uint32_t *>(&h3);
-                    const int i = 16 * (2 * k + r) + 2 * warp + sub;
+                    const int i = 8 * (2 * k + r) + rb;
                     *reinterpret_cast<uint4 *>(gblock + i * 256 + cg * 16) = raw;
                 }
             } else {
                 tmem_st16(tcol + 16 * k, ch);
             }
+            if (k + 1 < 8) tmem_wait_ld(nx);
         }
         if (pivot) {
             if (bad) flag(p.status, kFlagNonfinite);
@@ -481,72 +514,81 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
                 accE[pp] = __fadd2_rn(accE[pp], make_float2(__shfl_xor_sync(0xffffffffu, accE[pp].x, 16),
                                                             __shfl_xor_sync(0xffffffffu, accE[pp].y, 16)));
             if (sub == 0) {
-                float *red = sm.red + warp * D + 8 * cg;
-                *reinterpret_cast<float4 *>(red) = f4_of(accE[0], accE[1]);
-                *reinterpret_cast<float4 *>(red + 4) = f4_of(accE[2], accE[3]);
+                float *dst = sm.red + 2 * warp * RS + D + 8 * cg;
+                *reinterpret_cast<float4 *>(dst) = f4_of(accE[0], accE[1]);
+                *reinterpret_cast<float4 *>(dst + 4) = f4_of(accE[2], accE[3]);
             }
         }
     }
     __syncthreads();  // B3: column energies complete
 
-    // ---- Warps 0-3: new column scales. Warps 4-7: the next tile's row factors -------------
-    bool ok = true;
-    if (tid < D) {
-        if (!pivot) {
-            const float E = sum8(sm.red + j);
-            const float W = sm.rsum[pb][0][0] + sm.rsum[pb][1][0] + sm.rsum[pb][2][0] + sm.rsum[pb][3][0];
-            const float x = E * fast_rcp(W);
-            float c = (cj * inv_sig) * (x * rsqrtf(x));
-            if (!(x > 0.f)) c = (x == 0.f) ? 1.f : c;  // zero column: scale 1 (a NaN stays NaN)
-            reinterpret_cast<float *>(gblock + C::SOFF)[D + j] = c;
-            if (!isfinite(c) || c == 0.f) flag(p.status, kFlagNonfinite);
-            sm.colB[j] = (cj * inv_sig) * fast_rcp(c);
+    // ---- New column scale of column j, then the next tile's row factors -------------------
+    if (!pivot) {
+        // x = sum_i w_i S'_ij^2 / (sum_i w_i c_j^2) (times sigma_j^2), so c'_j = c_j sqrt(x) / sigma_j
+        // and the factor taking y to S'_ij / c'_j is 1 / sqrt(x)
+        const float E = sum4(sm.red + D + j, 2 * RS);
+        const float W = sm.rsum[pb][0][0] + sm.rsum[pb][1][0] + sm.rsum[pb][2][0] + sm.rsum[pb][3][0];
+        const float x = E * fast_rcp(W);
+        float b = rsqrtf(x);
+        float c = (cj * inv_sig) * (x * b);
+        if (x == 0.f) {  // zero column: scale 1 (a NaN stays NaN)
+            c = 1.f;
+            b = 0.f;
         }
-    } else {
-        ok = precompute_rows<BITS, GATE, IN_BF16>(sm, smem, n + 1, my_count);
+        reinterpret_cast<float *>(sm.meta[n & 3].gblock + C::SOFF)[D + j] = c;
+        if (!isfinite(c) || c == 0.f) flag(p.status, kFlagNonfinite);
+        sm.colB[j] = b;
     }
-    if (__syncthreads_or(!ok)) return false;  // B4: new column scales (and next row factors) ready
+    const bool ok = precompute_rows<BITS, GATE, IN_BF16>(sm, smem, n + 1, my_count);
+    if (__syncthreads_or(!ok)) return false;  // B4: new column scales and next row factors ready
     if constexpr (pivot) return true;
 
     // ---- Sweep C: z = y * c_j / c'_j and the per-row maxima of |z| ---------------------------
     tmem_wait_st();
-    float *rm = sm.red + (2 * warp + sub) * 128;  // row-max partials of this (warp, half)
     {
         float2 bb[4];
         load_pairs(sm.colB + 8 * cg, bb);
+        float *rm = sm.red + rb * RS + cg;
+        float2 cha[8], chb[8];
+        tmem_ld16_async(tcol, cha);
+        tmem_wait_ld(cha);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            float2 ch[8];
-            tmem_ld16(tcol + 16 * k, ch);
+        for (int k = 0; k < 8; ++k) {
+            float2 (&ch)[8] = (k & 1) ? chb : cha;
+            float2 (&nx)[8] = (k & 1) ? cha : chb;
+            if (k + 1 < 8) tmem_ld16_async(tcol + 16 * (k + 1), nx);
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
 #pragma unroll
                 for (int pp = 0; pp < 4; ++pp) ch[4 * r + pp] = __fmul2_rn(ch[4 * r + pp], bb[pp]);
                 const float2 *z = ch + 4 * r;
-                const float mx = fmaxf(max3(z[0].x, z[0].y, z[1].x), max3(z[1].y, z[2].x, max3(z[2].y, z[3].x, z[3].y)));
-                const float mn = fminf(min3(z[0].x, z[0].y, z[1].x), min3(z[1].y, z[2].x, min3(z[2].y, z[3].x, z[3].y)));
-                rm[(2 * k + r) * 16 + cg] = fmaxf(mx, -mn);
+                rm[(2 * k + r) * RM] = max3(max3(fabsf(z[0].x), fabsf(z[0].y), fabsf(z[1].x)),
+                                            max3(fabsf(z[1].y), fabsf(z[2].x), fabsf(z[2].y)),
+                                            fmaxf(fabsf(z[3].x), fabsf(z[3].y)));
             }
             tmem_st16(tcol + 16 * k, ch);
+            if (k + 1 < 8) tmem_wait_ld(nx);
         }
     }
     __syncwarp();
     {
-        const int m = cg >> 1, half = cg & 1;
-        const float4 a = *reinterpret_cast<const float4 *>(rm + m * 16 + half * 8);
-        const float4 b = *reinterpret_cast<const float4 *>(rm + m * 16 + half * 8 + 4);
-        float v = max3(max3(a.x, a.y, a.z), max3(a.w, b.x, b.y), fmaxf(b.z, b.w));
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
-        const int i = 16 * m + 2 * warp + sub;
-        const float sw = sm.rowSw[pb][i];
-        float r = v * fast_rcp(sw * C::QMAX);
-        if (v == 0.f) r = 1.f;
-        const float s = fast_rcp(sw * r);
-        if (half == 0) {
-            sm.rowS[i] = make_float2(s, s);
-            reinterpret_cast<float *>(gblock + C::SOFF)[i] = r;
-            if (!isfinite(r) || r == 0.f) flag(p.status, kFlagNonfinite);
+        // lane cg of this half finishes its row m = cg (i = 8 cg + rb) from the 16 partials
+        const float4 *src = reinterpret_cast<const float4 *>(sm.red + rb * RS + cg * RM);
+        const float4 a = src[0], b = src[1], c = src[2], d = src[3];
+        const float v = max3(max3(max3(a.x, a.y, a.z), max3(a.w, b.x, b.y), max3(b.z, b.w, c.x)),
+                             max3(c.y, c.z, c.w), max3(d.x, d.y, fmaxf(d.z, d.w)));
+        const int i = 8 * cg + rb;
+        // v = max_j |sqrt(w_i) S'_ij / c'_j|: r'_i = v / (sqrt(w_i) qmax), and the factor taking
+        // z to the code is 1 / (sqrt(w_i) r'_i) = qmax / v
+        float r = v * sm.rowRq[pb][i];
+        float s = C::QMAX * fast_rcp(v);
+        if (v == 0.f) {  // zero row: scale 1
+            r = 1.f;
+            s = 0.f;
         }
+        sm.rowS[i] = make_float2(s, s);
+        reinterpret_cast<float *>(sm.meta[n & 3].gblock + C::SOFF)[i] = r;
+        if (!isfinite(r) || r == 0.f) flag(p.status, kFlagNonfinite);
     }
     __syncwarp();
 
@@ -554,19 +596,24 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
     tmem_wait_st();
     {
         const float2 rnd = make_float2(C::ROUND, C::ROUND);
-        uint8_t *dstrow = gblock + (2 * warp + sub) * C::RB + cg * BITS;
+        uint8_t *dstrow = reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock) + rb * C::RB + cg * BITS;
+        float2 cha[8], chb[8];
+        tmem_ld16_async(tcol, cha);
+        tmem_wait_ld(cha);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            float2 ch[8];
-            tmem_ld16(tcol + 16 * k, ch);
+        for (int k = 0; k < 8; ++k) {
+            float2 (&ch)[8] = (k & 1) ? chb : cha;
+            float2 (&nx)[8] = (k & 1) ? cha : chb;
+            if (k + 1 < 8) tmem_ld16_async(tcol + 16 * (k + 1), nx);
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const int m = 2 * k + r;
-                const float2 s2 = sm.rowS[16 * m + 2 * warp + sub];
+                const float2 s2 = sm.rowS[8 * m + rb];
 #pragma unroll
                 for (int pp = 0; pp < 4; ++pp) ch[4 * r + pp] = __ffma2_rn(ch[4 * r + pp], s2, rnd);
-                pack_store_row<BITS>(dstrow + 16 * m * C::RB, cg, ch + 4 * r);
+                pack_store_row<BITS>(dstrow + 8 * m * C::RB, cg, ch + 4 * r);
             }
+            if (k + 1 < 8) tmem_wait_ld(nx);
         }
     }
     return true;
@@ -593,38 +640,43 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
         fence_mbar_init();
         const float o = BITS == 16 ? 0.f : (float)(1 << (BITS - 1));
         sm.unpack_off = make_float2(-(8388608.0f + o), -(8388608.0f + o * C::SIG1));
+        sm.magic = MAGIC;
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    // this thread's 64 columns: lanes 32*(warp%4).., columns 0..63 (warps 0-3) or 64..127 (4-7)
-    const uint32_t tcol = sm.tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + (warp >= 4 ? 64u : 0u);
+    // this thread's lane 32 * warp + lane, columns 0..127
+    const uint32_t tcol = sm.tmem_base + ((uint32_t)(32 * warp) << 16);
 
-    if (tid == 0)
-        for (int n = 0; n < C::NS; ++n) issue_tile<BITS, GATE, IN_BF16>(p, sm, smem, n, my_count);
-    bool ok = true;
-    if (tid >= D) ok = precompute_rows<BITS, GATE, IN_BF16>(sm, smem, 0, my_count);
-    bool failed = __syncthreads_or(!ok);
+    if (tid == 0) {
+        Issuer &it = sm.iss;
+        it.n = 0;
+        it.pos = (int)blockIdx.x / p.B;
+        it.b = (int)blockIdx.x - it.pos * p.B;
+        it.qG = G / p.B;
+        it.rG = G - it.qG * p.B;
+        for (int k = 0; k < C::NS; ++k) issue_next<BITS, GATE, IN_BF16>(p, sm, smem, it, my_count);
+    }
+    bool failed = __syncthreads_or(!precompute_rows<BITS, GATE, IN_BF16>(sm, smem, 0, my_count));
 
     int n = 0;
     for (; n < my_count && !failed; ++n) {
-        // every thread observes the tile's completion itself (already complete: warps 4-7 waited)
-        const bool got = wait_tile<BITS, GATE, IN_BF16>(sm, n);
-        if (sm.scal[n % C::NS][2] != 0.f) {  // out-of-range slot: nothing loaded, nothing to do
+        // every thread observes the tile's completion itself (already complete: all waited)
+        const bool got = mbar_wait_bounded(smem_u32(&sm.bars[n % C::NS]), (uint32_t)(n / C::NS) & 1u);
+        if (sm.meta[n & 3].skip) {  // out-of-range slot: nothing loaded, nothing to do
             __syncthreads();
-            if (tid == 0) issue_tile<BITS, GATE, IN_BF16>(p, sm, smem, n + C::NS, my_count);
-            ok = true;
-            if (tid >= D) ok = precompute_rows<BITS, GATE, IN_BF16>(sm, smem, n + 1, my_count);
+            if (tid == 0) issue_next<BITS, GATE, IN_BF16>(p, sm, smem, sm.iss, my_count);
+            const bool ok = precompute_rows<BITS, GATE, IN_BF16>(sm, smem, n + 1, my_count);
             failed = __syncthreads_or(!ok || !got);
-            continue;
+        } else {
+            failed = !process_tile<BITS, GATE, IN_BF16>(p, sm, smem, n, my_count, tcol);
         }
-        failed = !process_tile<BITS, GATE, IN_BF16>(p, sm, smem, n, my_count, tcol);
     }
     if (failed && tid == 0) {
         flag(p.status, kFlagTimeout);
-        // let every copy in flight land before the CTA's shared memory is released
-        const int last = (n + C::NS < my_count) ? n + C::NS : my_count;
-        for (int m = n; m < last; ++m) wait_tile<BITS, GATE, IN_BF16>(sm, m);
+        // let every copy in flight (tiles n .. iss.n - 1) land before the CTA's shared memory is released
+        for (int m = n; m < sm.iss.n; ++m)
+            mbar_wait_bounded(smem_u32(&sm.bars[m % C::NS]), (uint32_t)((m / C::NS) & 1));
     }
     // release Tensor Memory once every thread's accesses have completed
     tmem_wait_st();
