@@ -1,0 +1,795 @@
+// prefill_wy.cu -- chunked prefill of 128 x 128 quantized states in the WY / UT form, with the
+// dense contractions on the fifth-generation tensor cores (tcgen05, bf16 operands, fp32
+// accumulation in Tensor Memory).
+//
+// Method: the prompt is consumed in chunks; inside a chunk the state is carried unquantized and
+// at every chunk end it is refitted and requantized exactly like a decode step ("K1 論文詳解"
+// (k1-news.pages.dev/paper/2026-10-09), section 方法: chunked prefill writes the same quantized
+// state; "线性注意力状态量化难题" (aitest123.com/news/n1kj09), section 工程落地). The chunk algebra
+// is the standard UT transform of the gated delta rule S_t = a_t (S_{t-1} - b_t k_t k_t^T S_{t-1})
+// + b_t k_t v_t^T, o_t = S_t^T q_t. With gamma_t = prod_{s<=t} a_s (chunk-relative) and the chunk
+// start state S0 = diag(r) Q diag(c):
+//   L_ts = b_t (gamma_t / gamma_s) k_t.k_s            (s < t)      T = (I + L)^-1
+//   R'_t = b_t (v_t - gamma_t S0^T k_t)                             U = T R'
+//   P_ts = (gamma_t / gamma_s) q_t.k_s                 (s <= t)
+//   o_t  = gamma_t S0^T q_t + sum_s P_ts U_s
+//   S_C  = gamma_C S0 + K^T diag(gamma_C / gamma) U
+// Unrolling the per-token recurrence gives exactly these sums; inside a chunk nothing is rounded
+// to the state's codes.
+//
+// Design (B200, one persistent CTA of 256 threads per SM, 512 Tensor Memory columns):
+//  * bf16 inputs are exact bf16 MMA operands. fp32 quantities that enter a contraction (K r, Q r,
+//    T, R', U, decayed U) are split into three bf16 terms carrying all 24 significand bits; the
+//    products keep the terms whose order is at most 2^-24 of the result (P U, which only feeds the
+//    readout, uses two terms each). The codes themselves (|Q| <= 127) are exact in bf16.
+//  * Five MMA groups per chunk: D1 = [K;Q] K^T, D2 = [K r;Q r] Qcodes, DU = T R', DP = P U and
+//    D3 = K^T (decayed U); 64-row operands sit in rows 64..127 of an M = 128 instruction so that
+//    every accumulator row is its Tensor Memory lane.
+//  * The 64 x 64 unit lower-triangular inverse T is formed on the CUDA cores by 16 x 16 blocks.
+//  * K and Q of the next chunk stream in by cp.async while the current chunk finishes; the state
+//    stays on chip (codes as bf16 in the B-operand layout, scales in shared memory) between chunks
+//    and is packed to HBM once, after the last chunk.
+#include "stq_internal.cuh"
+#include "umma.cuh"
+
+namespace stq {
+namespace {
+
+using umma::sw128_chunk;
+
+constexpr int D = 128;
+constexpr int C = 64;   // chunk length
+constexpr int NT = 256;
+constexpr int LDL = 68; // row stride (floats) of the fp32 L and T work matrices
+
+// Shared-memory map (bytes from a 1024-aligned base).
+constexpr uint32_t XY_BYTES = 34816;           // one K/Q buffer (32 KB) or the L/T work area
+constexpr uint32_t OFF_XY0 = 0;
+constexpr uint32_t OFF_XY1 = XY_BYTES;
+constexpr uint32_t OFF_QC = 2 * XY_BYTES;      // 69632: codes, bf16, B operand (MN-major), 32 KB
+constexpr uint32_t OFF_BIG = OFF_QC + 32768;   // 102400: 96 KB of split operands
+constexpr uint32_t OFF_RT = OFF_BIG + 98304;   // 200704: T in three bf16 terms, 24 KB
+constexpr uint32_t OFF_SMALL = OFF_RT + 24576; // 225280
+// small area
+constexpr uint32_t S_BETA = 0;                 // [2][64] f32 (per buffer)
+constexpr uint32_t S_ALPHA = 512;              // [2][64] f32
+constexpr uint32_t S_LG = 1024;                // [64] f64: log alpha
+constexpr uint32_t S_G = 1536;                 // [64] f64: cumulative log decay
+constexpr uint32_t S_GAM = 2048;               // [64] f32: gamma_t
+constexpr uint32_t S_DC = 2304;                // [64] f32: gamma_C / gamma_t
+constexpr uint32_t S_R = 2560;                 // [128] f32 row scales
+constexpr uint32_t S_C = 3072;                 // [128] f32 column scales
+constexpr uint32_t S_W = 3584;                 // [128] f32 impact weights
+constexpr uint32_t S_BAR = 4096;               // 4 mbarriers
+constexpr uint32_t S_MISC = 4128;              // tmem base, W sum, gamma_C
+constexpr uint32_t SMALL_BYTES = 4224;
+constexpr uint32_t SMEM_BYTES = OFF_SMALL + SMALL_BYTES + 1024;  // + alignment slack
+
+// Within the K/Q buffer: [K d0..63 | Q d0..63 | K d64..127 | Q d64..127], 64 rows x 128 B each.
+constexpr uint32_t KQ_K0 = 0, KQ_Q0 = 8192, KQ_K1 = 16384, KQ_Q1 = 24576;
+// Within BIG: phase 1 = three 32 KB A tiles of D2; phase 2 = R' terms + P terms; phase 3 = U,
+// decayed-U and P terms.
+constexpr uint32_t BIG_R0 = 0, BIG_R1 = 16384, BIG_R2 = 32768;            // R' terms (MN-major)
+constexpr uint32_t BIG_P0 = 49152, BIG_P1 = 57344;                        // P terms (K-major)
+constexpr uint32_t BIG_U0 = 0, BIG_U1 = 16384;                            // U terms
+constexpr uint32_t BIG_Y0 = 32768, BIG_Y1 = 65536, BIG_Y2 = 81920;        // decayed U terms
+// requantization scratch in BIG (after the last MMA of the chunk has completed)
+constexpr uint32_t BIG_RED = 0;      // [4][128] f32 column-energy partials
+constexpr uint32_t BIG_RMAX = 2048;  // [2][128] f32 row-max partials
+// T-inverse scratch in the RT area (before the T terms are written)
+constexpr uint32_t RT_G = 0;         // [3][16][17] f32
+
+// Tensor Memory columns
+constexpr uint32_t TM_D1 = 0, TM_D3 = 0, TM_D2 = 128, TM_DU = 256, TM_DP = 384;
+
+struct PrefillArgs {
+    int T;       // tokens of this call
+};
+
+template <int BITS>
+struct PCfg {
+    static constexpr int QMAX = (1 << (BITS - 1)) - 1;
+    static constexpr int OFFS = 1 << (BITS - 1);
+    static constexpr uint32_t ROWB = 16u * BITS;               // packed bytes of one 128-code row
+    static constexpr uint32_t SOFF = scale_offset(BITS, D, D); // r[] then c[]
+};
+
+__device__ __forceinline__ float *smf(uint8_t *base, uint32_t off) { return reinterpret_cast<float *>(base + off); }
+__device__ __forceinline__ double *smd(uint8_t *base, uint32_t off) { return reinterpret_cast<double *>(base + off); }
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Start loading the K and Q rows of one chunk into a K/Q buffer (rows past the prompt are zero
+// filled), and its beta / alpha into ring `buf` of the small area (padding: beta 0, alpha 1).
+__device__ __forceinline__ void load_chunk_async(uint8_t *sm, uint32_t kq_off, int buf, const __nv_bfloat16 *kbase,
+                                                 const __nv_bfloat16 *qbase, const float *bbase, const float *abase,
+                                                 int Lc)
+{
+    const int tid = threadIdx.x;
+    // 2 tensors x 64 rows x 16 chunks of 16 B = 2048 copies, 8 per thread
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int e = tid + NT * k;
+        const int tensor = e >> 10, row = (e >> 4) & 63, ch = e & 15;
+        const __nv_bfloat16 *src = (tensor ? qbase : kbase) + (size_t)(row < Lc ? row : 0) * D + ch * 8;
+        const uint32_t box = (ch >> 3) ? (tensor ? KQ_Q1 : KQ_K1) : (tensor ? KQ_Q0 : KQ_K0);
+        const uint32_t dst = smem_u32(sm + kq_off + box + sw128_chunk(row, ch & 7));
+        cp_async16(dst, src, row < Lc ? 16u : 0u);
+    }
+    if (tid < C) {
+        float *bb = smf(sm, OFF_SMALL + S_BETA) + buf * C;
+        float *aa = smf(sm, OFF_SMALL + S_ALPHA) + buf * C;
+        if (tid < Lc) {
+            cp_async4(smem_u32(bb + tid), bbase + tid);
+            cp_async4(smem_u32(aa + tid), abase + tid);
+        } else {
+            bb[tid] = 0.f;
+            aa[tid] = 1.f;
+        }
+    }
+    cp_async_commit();
+}
+
+
+// ---------------------------------------------------------------------------------------------
+// State load / store (packed little-endian offset-binary bitstream, row-major)
+// ---------------------------------------------------------------------------------------------
+
+// Thread (row i, half h) unpacks codes i, 64h .. 64h+63 of the tile and writes them as bf16 into
+// the B-operand tile (contraction row i, atom column h).
+template <int BITS>
+__device__ __forceinline__ void load_codes_row(const uint8_t *gblock, uint8_t *qc, int i, int h)
+{
+    using P = PCfg<BITS>;
+    constexpr int NW = 2 * BITS;  // 32-bit words holding 64 codes
+    uint32_t wv[NW + 1];
+    const uint4 *src = reinterpret_cast<const uint4 *>(gblock + (size_t)i * P::ROWB + h * (P::ROWB / 2));
+#pragma unroll
+    for (int k = 0; k < NW / 4; ++k) {
+        const uint4 x = src[k];
+        wv[4 * k] = x.x;
+        wv[4 * k + 1] = x.y;
+        wv[4 * k + 2] = x.z;
+        wv[4 * k + 3] = x.w;
+    }
+    wv[NW] = 0u;
+#pragma unroll
+    for (int c8 = 0; c8 < 8; ++c8) {
+        uint32_t packed[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+            float f[2];
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+                const int col = 8 * c8 + e + z, bit = BITS * col, wi = bit >> 5, sh = bit & 31;
+                uint32_t u = wv[wi] >> sh;
+                if (sh + BITS > 32) u |= wv[wi + 1] << (32 - sh);
+                u &= (1u << BITS) - 1u;
+                f[z] = (float)((int)u - P::OFFS);
+            }
+            packed[e >> 1] = umma::pack_bf16(__float2bfloat16_rn(f[0]), __float2bfloat16_rn(f[1]));
+        }
+        *reinterpret_cast<uint4 *>(qc + h * 16384 + sw128_chunk(i, c8)) =
+            make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    }
+}
+
+// Pack 64 integer codes (values in [-qmax, qmax]) of row i, half h into the tile in HBM.
+template <int BITS>
+__device__ __forceinline__ void store_codes_row(uint8_t *gblock, int i, int h, const int (&q)[64])
+{
+    using P = PCfg<BITS>;
+    constexpr int NW = 2 * BITS;
+    uint32_t wv[NW];
+#pragma unroll
+    for (int k = 0; k < NW; ++k) wv[k] = 0u;
+#pragma unroll
+    for (int col = 0; col < 64; ++col) {
+        const uint32_t u = (uint32_t)(q[col] + P::OFFS);
+        const int bit = BITS * col, wi = bit >> 5, sh = bit & 31;
+        wv[wi] |= u << sh;
+        if (sh + BITS > 32) wv[wi + 1] |= u >> (32 - sh);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(gblock + (size_t)i * P::ROWB + h * (P::ROWB / 2));
+#pragma unroll
+    for (int k = 0; k < NW / 4; ++k) dst[k] = make_uint4(wv[4 * k], wv[4 * k + 1], wv[4 * k + 2], wv[4 * k + 3]);
+}
+
+// ---------------------------------------------------------------------------------------------
+// T = (I + L)^-1 for a strictly lower triangular 64 x 64 L (fp32, row stride LDL), by 16 x 16
+// blocks: the four diagonal blocks by forward substitution (one warp each), then the off-diagonal
+// blocks T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj in order of distance i - j. G: [3][16][17] scratch.
+// All 256 threads call it; it ends with a barrier.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void invert_unit_lower(const float *L, float *T, float *G)
+{
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (warp < 4 && lane < 16) {
+        const int b0 = 16 * warp, c = lane;
+        float x[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) x[t] = (t == c) ? 1.f : 0.f;
+#pragma unroll
+        for (int s = 0; s < 16; ++s) {
+            const float xs = x[s];
+#pragma unroll
+            for (int t = s + 1; t < 16; ++t) x[t] = fmaf(-L[(b0 + t) * LDL + b0 + s], xs, x[t]);
+        }
+#pragma unroll
+        for (int t = 0; t < 16; ++t) T[(b0 + t) * LDL + b0 + c] = x[t];
+    }
+    // zero the strictly upper blocks (never read by the products below, but T is an MMA operand)
+    for (int e = tid; e < 64 * 64; e += NT) {
+        const int t = e >> 6, s = e & 63;
+        if ((s >> 4) > (t >> 4)) T[t * LDL + s] = 0.f;
+    }
+    __syncthreads();
+    const int r = tid >> 4, c = tid & 15;
+#pragma unroll
+    for (int d = 1; d < 4; ++d) {
+        // G_ij = sum_{k=j}^{i-1} L_ik T_kj for the blocks at distance d
+        for (int j = 0; j + d < 4; ++j) {
+            const int i = j + d;
+            float acc = 0.f;
+            for (int k = j; k < i; ++k) {
+                const float *Lr = L + (16 * i + r) * LDL + 16 * k;
+                const float *Tc = T + (16 * k) * LDL + 16 * j + c;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) acc = fmaf(Lr[u], Tc[u * LDL], acc);
+            }
+            G[j * 272 + r * 17 + c] = acc;
+        }
+        __syncthreads();
+        for (int j = 0; j + d < 4; ++j) {
+            const int i = j + d;
+            const float *Tr = T + (16 * i + r) * LDL + 16 * i;
+            float acc = 0.f;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) acc = fmaf(Tr[u], G[j * 272 + u * 17 + c], acc);
+            T[(16 * i + r) * LDL + 16 * j + c] = -acc;
+        }
+        __syncthreads();
+    }
+}
+
+// Warp reduce-scatter of 64 per-lane values: afterwards lane l holds the warp sums of entries
+// 2l and 2l+1 in v[0], v[1].
+__device__ __forceinline__ void warp_reduce_scatter64(float (&v)[64])
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int step = 0; step < 5; ++step) {
+        const int o = 16 >> step, n = 64 >> step, hn = n >> 1;
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int k = 0; k < hn; ++k) {
+            const float keep = up ? v[k + hn] : v[k];
+            const float send = up ? v[k] : v[k + hn];
+            v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+}
+
+
+// Split helpers writing 8 consecutive values as one 16-byte chunk per term.
+__device__ __forceinline__ void store_split3(uint8_t *t0, uint8_t *t1, uint8_t *t2, uint32_t off, const float (&x)[8])
+{
+    uint32_t a[4], b[4], c[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        __nv_bfloat16 h0, m0, l0, h1, m1, l1;
+        umma::split3(x[2 * e], h0, m0, l0);
+        umma::split3(x[2 * e + 1], h1, m1, l1);
+        a[e] = umma::pack_bf16(h0, h1);
+        b[e] = umma::pack_bf16(m0, m1);
+        c[e] = umma::pack_bf16(l0, l1);
+    }
+    *reinterpret_cast<uint4 *>(t0 + off) = make_uint4(a[0], a[1], a[2], a[3]);
+    *reinterpret_cast<uint4 *>(t1 + off) = make_uint4(b[0], b[1], b[2], b[3]);
+    *reinterpret_cast<uint4 *>(t2 + off) = make_uint4(c[0], c[1], c[2], c[3]);
+}
+
+__device__ __forceinline__ void store_split2(uint8_t *t0, uint8_t *t1, uint32_t off, const float (&x)[8])
+{
+    uint32_t a[4], b[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * e]), h1 = __float2bfloat16_rn(x[2 * e + 1]);
+        const __nv_bfloat16 l0 = __float2bfloat16_rn(x[2 * e] - __bfloat162float(h0));
+        const __nv_bfloat16 l1 = __float2bfloat16_rn(x[2 * e + 1] - __bfloat162float(h1));
+        a[e] = umma::pack_bf16(h0, h1);
+        b[e] = umma::pack_bf16(l0, l1);
+    }
+    *reinterpret_cast<uint4 *>(t0 + off) = make_uint4(a[0], a[1], a[2], a[3]);
+    *reinterpret_cast<uint4 *>(t1 + off) = make_uint4(b[0], b[1], b[2], b[3]);
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(uint4 raw, float (&x)[8])
+{
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        x[2 * e] = __uint_as_float(w[e] << 16);
+        x[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+    }
+}
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int32_t *status)
+{
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+    if (!ok && (threadIdx.x & 31) == 0) flag(status, kFlagTimeout);
+    return ok;
+}
+
+
+// ---------------------------------------------------------------------------------------------
+// The kernel: persistent CTAs over (request, head) tiles of one code width; the chunks of a tile
+// run in order.
+// ---------------------------------------------------------------------------------------------
+template <int BITS>
+__global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant__ TileParams p, const int T_tok)
+{
+    using P = PCfg<BITS>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, ch = warp >> 2;
+    float *sR = smf(sm, OFF_SMALL + S_R), *sC = smf(sm, OFF_SMALL + S_C), *sW = smf(sm, OFF_SMALL + S_W);
+    double *sLG = smd(sm, OFF_SMALL + S_LG), *sG = smd(sm, OFF_SMALL + S_G);
+    float *sGam = smf(sm, OFF_SMALL + S_GAM), *sDC = smf(sm, OFF_SMALL + S_DC);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_SMALL + S_BAR);
+    uint32_t *misc = reinterpret_cast<uint32_t *>(sm + OFF_SMALL + S_MISC);  // [0] Tensor Memory base
+    float *miscf = reinterpret_cast<float *>(misc + 1);                     // [0] sum w, [1] gamma_C
+    uint8_t *big = sm + OFF_BIG;
+
+    if (warp == 0) umma::tmem_alloc(smem_u32(misc), 512);
+    if (tid == 0) {
+        for (int k = 0; k < 4; ++k) mbar_init(smem_u32(&bars[k]), 1);
+        fence_mbar_init();
+    }
+    umma::fence_before_sync();
+    __syncthreads();
+    umma::fence_after_sync();
+    const uint32_t tmem = misc[0];
+    const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);  // this warp's lane quarter
+    const int nch = (T_tok + C - 1) / C;
+    uint32_t parity = 0;
+    bool ok = true;
+
+    for (int n = blockIdx.x; n < p.ntiles && ok; n += gridDim.x) {
+        const int b = n % p.B, pos = n / p.B;
+        const TileEntry ent = p.table[pos];
+        const int head = entry_head(ent);
+        const int slot = p.slots[b];
+        if (slot < 0 || slot >= p.pool_slots) {
+            if (tid == 0) flag(p.status, kFlagBounds);
+            continue;
+        }
+        uint8_t *gblock = p.pool + (uint64_t)slot * p.req_bytes + ent.off;
+        const uint64_t trow = (uint64_t)b * (uint64_t)p.head_count + (uint64_t)head;
+        const __nv_bfloat16 *kg = reinterpret_cast<const __nv_bfloat16 *>(p.k) + trow * (uint64_t)T_tok * D;
+        const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(p.q) + trow * (uint64_t)T_tok * D;
+        const __nv_bfloat16 *vg = reinterpret_cast<const __nv_bfloat16 *>(p.v) + trow * (uint64_t)T_tok * D;
+        const float *bg = p.beta + trow * (uint64_t)T_tok, *ag = p.alpha + trow * (uint64_t)T_tok;
+        float *og = p.o + trow * (uint64_t)T_tok * D;
+
+        // ---- the tile's state onto the chip ----------------------------------------------
+        __syncthreads();  // the previous tile is completely done with shared memory
+        load_codes_row<BITS>(gblock, sm + OFF_QC, tid >> 1, tid & 1);
+        if (tid < D) {
+            const float *sc = reinterpret_cast<const float *>(gblock + P::SOFF);
+            sR[tid] = sc[tid];
+            sC[tid] = sc[D + tid];
+            sW[tid] = p.w[(size_t)head * D + tid];
+        }
+        load_chunk_async(sm, OFF_XY0, 0, kg, qg, bg, ag, T_tok < C ? T_tok : C);
+        __syncthreads();
+        if (warp == 0) {
+            float s = sW[lane] + sW[lane + 32] + sW[lane + 64] + sW[lane + 96];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            if (lane == 0) miscf[0] = s;
+        }
+
+        for (int c = 0; c < nch && ok; ++c, parity ^= 1u) {
+            const int t0 = c * C, Lc = (T_tok - t0) < C ? (T_tok - t0) : C;
+            const uint32_t kq = (c & 1) ? OFF_XY1 : OFF_XY0;  // this chunk's K / Q
+            const uint32_t lt = (c & 1) ? OFF_XY0 : OFF_XY1;  // L / T work, then the next chunk's K / Q
+            const int buf = c & 1;
+            const float *sBeta = smf(sm, OFF_SMALL + S_BETA) + buf * C;
+            const float *sAlpha = smf(sm, OFF_SMALL + S_ALPHA) + buf * C;
+            float *Lm = smf(sm, lt), *Tm = smf(sm, lt + 64 * LDL * 4);
+
+            // v rows for R' (lane quarters 0, 1: row t, columns 64 ch .. +63), in flight early
+            uint4 vraw[8];
+            if (q4 < 2) {
+                const int t = 32 * q4 + lane;
+                const uint4 *vs = reinterpret_cast<const uint4 *>(vg + (size_t)(t0 + (t < Lc ? t : 0)) * D + 64 * ch);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) vraw[k] = t < Lc ? vs[k] : make_uint4(0u, 0u, 0u, 0u);
+            }
+            cp_async_wait_all();
+            umma::fence_proxy_async();
+            umma::fence_before_sync();
+            __syncthreads();
+
+            // ---- D1 = [K;Q] K^T (M 128, N 64) ------------------------------------------
+            if (tid == 0) {
+                umma::fence_after_sync();
+                const uint32_t base = smem_u32(sm + kq);
+                const uint32_t id = umma::idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t o = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    umma::mma_bf16(tmem + TM_D1, umma::smem_desc(base + o, 16, 1024), umma::smem_desc(base + o, 16, 1024),
+                                   id, kk > 0);
+                }
+                umma::mma_commit(smem_u32(&bars[0]));
+            }
+            // ---- cumulative log decay of the chunk (fp64) ------------------------------
+            if (tid < C) {
+                double g = tid < Lc ? log((double)sAlpha[tid]) : 0.0;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const double y = __shfl_up_sync(0xffffffffu, g, o);
+                    if (lane >= o) g += y;
+                }
+                sLG[tid] = g;  // within-warp inclusive prefix
+            }
+            // ---- A operand of D2: three bf16 terms of [K r; Q r] ------------------------
+            {
+                const int m = tid >> 1, h = tid & 1, row = m & 63;
+                const uint8_t *xb = sm + kq + (m < 64 ? (h ? KQ_K1 : KQ_K0) : (h ? KQ_Q1 : KQ_Q0));
+                uint8_t *a0 = big + h * 16384, *a1 = a0 + 32768, *a2 = a0 + 65536;
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    float x[8];
+                    bf16x8_to_f32(*reinterpret_cast<const uint4 *>(xb + sw128_chunk(row, c8)), x);
+                    const float4 ra = *reinterpret_cast<const float4 *>(sR + 64 * h + 8 * c8);
+                    const float4 rb = *reinterpret_cast<const float4 *>(sR + 64 * h + 8 * c8 + 4);
+                    x[0] *= ra.x; x[1] *= ra.y; x[2] *= ra.z; x[3] *= ra.w;
+                    x[4] *= rb.x; x[5] *= rb.y; x[6] *= rb.z; x[7] *= rb.w;
+                    store_split3(a0, a1, a2, sw128_chunk(m, c8), x);
+                }
+            }
+            umma::fence_proxy_async();
+            __syncthreads();
+            if (tid == 0) {
+                const uint32_t abase = smem_u32(big), bbase = smem_u32(sm + OFF_QC);
+                const uint32_t id = umma::idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+                for (int term = 0; term < 3; ++term)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma::mma_bf16(tmem + TM_D2,
+                                       umma::smem_desc(abase + term * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                       umma::smem_desc(bbase + kk * 2048, 16384, 1024), id, (term | kk) != 0);
+                umma::mma_commit(smem_u32(&bars[1]));
+            }
+            // finish the prefix across the two warps, then the decay factors
+            if (tid < C) {
+                double g = sLG[tid];
+                if (tid >= 32) g += sLG[31];
+                sG[tid] = g;
+            }
+            __syncthreads();
+            if (tid < C) {
+                const double gl = sG[C - 1], g = sG[tid];
+                sGam[tid] = (float)exp(g);
+                sDC[tid] = (float)exp(gl - g);
+                if (tid == 0) miscf[1] = (float)exp(gl);
+            }
+
+            // ---- L (lane quarters 0, 1) and P (quarters 2, 3) from D1 ---------------------
+            ok = wait_bar(smem_u32(&bars[0]), parity, p.status);
+            if (!__syncthreads_and(ok)) break;
+            umma::fence_after_sync();
+            float pv[32];
+            {
+                float v[32];
+                umma::tmem_ld32(tl + TM_D1 + 32 * ch, v);
+                const int t = 32 * (q4 & 1) + lane;
+                const double gt = sG[t];
+                if (q4 < 2) {
+                    const float bt = sBeta[t];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const int s = 32 * ch + u;
+                        Lm[t * LDL + s] = s < t ? bt * expf((float)(gt - sG[s])) * v[u] : 0.f;
+                    }
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const int s = 32 * ch + u;
+                        pv[u] = s <= t ? expf((float)(gt - sG[s])) * v[u] : 0.f;
+                    }
+                }
+            }
+            __syncthreads();
+            invert_unit_lower(Lm, Tm, smf(sm, OFF_RT + RT_G));
+            // T in three bf16 terms (K-major, rows t, contraction s)
+            {
+                const int t = tid >> 2, part = tid & 3;
+                uint8_t *r0 = sm + OFF_RT, *r1 = r0 + 8192, *r2 = r0 + 16384;
+#pragma unroll
+                for (int hc = 0; hc < 2; ++hc) {
+                    const int c8 = 2 * part + hc;
+                    float x[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = Tm[t * LDL + 8 * c8 + e];
+                    store_split3(r0, r1, r2, sw128_chunk(t, c8), x);
+                }
+            }
+            __syncthreads();  // L / T are dead: the area takes the next chunk's K / Q
+            if (c + 1 < nch) {
+                const int t1 = t0 + C, L1 = (T_tok - t1) < C ? (T_tok - t1) : C;
+                load_chunk_async(sm, lt, buf ^ 1, kg + (size_t)t1 * D, qg + (size_t)t1 * D, bg + t1, ag + t1, L1);
+            }
+
+
+            // ---- R' (quarters 0, 1) and P terms (quarters 2, 3) once D2 is complete -------
+            ok = wait_bar(smem_u32(&bars[1]), parity, p.status);
+            if (!__syncthreads_and(ok)) break;
+            umma::fence_after_sync();
+            if (q4 < 2) {
+                const int t = 32 * q4 + lane;
+                const float bt = sBeta[t], gt = sGam[t];
+                uint8_t *r0 = big + BIG_R0 + ch * 8192, *r1 = big + BIG_R1 + ch * 8192, *r2 = big + BIG_R2 + ch * 8192;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v[32];
+                    umma::tmem_ld32(tl + TM_D2 + 64 * ch + 32 * hh, v);
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const int c8 = 4 * hh + c4;
+                        float vv[8], x[8];
+                        bf16x8_to_f32(vraw[c8], vv);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int j = 64 * ch + 8 * c8 + e;
+                            x[e] = bt * (vv[e] - gt * (sC[j] * v[8 * c4 + e]));
+                        }
+                        store_split3(r0, r1, r2, sw128_chunk(t, c8), x);
+                    }
+                }
+            } else {
+                const int t = 32 * (q4 - 2) + lane;
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    float x[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = pv[8 * c4 + e];
+                    store_split2(big + BIG_P0, big + BIG_P1, sw128_chunk(t, 4 * ch + c4), x);
+                }
+            }
+            umma::fence_proxy_async();
+            __syncthreads();
+            // ---- DU = T R' (rows 64..127 of an M 128 instruction) ---------------------------
+            if (tid == 0) {
+                const uint32_t ta = smem_u32(sm + OFF_RT) - 8192, rb = smem_u32(big);
+                const uint32_t id = umma::idesc_bf16(128, 128, 0, 1);
+                constexpr int A_T[6] = {0, 0, 1, 0, 1, 2}, B_T[6] = {0, 1, 0, 2, 1, 0};
+#pragma unroll
+                for (int cmb = 0; cmb < 6; ++cmb)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma::mma_bf16(tmem + TM_DU, umma::smem_desc(ta + A_T[cmb] * 8192 + kk * 32, 16, 1024),
+                                       umma::smem_desc(rb + B_T[cmb] * 16384 + kk * 2048, 8192, 1024), id,
+                                       (cmb | kk) != 0);
+                umma::mma_commit(smem_u32(&bars[2]));
+            }
+            ok = wait_bar(smem_u32(&bars[2]), parity, p.status);
+            if (!__syncthreads_and(ok)) break;
+            umma::fence_after_sync();
+            // ---- U terms and decayed-U terms (quarters 2, 3: row t = lane - 64) --------------
+            if (q4 >= 2) {
+                const int t = 32 * (q4 - 2) + lane;
+                const float dc = sDC[t];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v[32];
+                    umma::tmem_ld32(tl + TM_DU + 64 * ch + 32 * hh, v);
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const int c8 = 4 * hh + c4;
+                        const uint32_t off = ch * 8192 + sw128_chunk(t, c8);
+                        float x[8], y[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            x[e] = v[8 * c4 + e];
+                            y[e] = dc * x[e];
+                        }
+                        store_split2(big + BIG_U0, big + BIG_U1, off, x);
+                        store_split3(big + BIG_Y0, big + BIG_Y1, big + BIG_Y2, off, y);
+                    }
+                }
+            }
+            umma::fence_proxy_async();
+            umma::fence_before_sync();
+            __syncthreads();
+            // ---- DP = P U (rows 64..127) and D3 = K^T (decayed U) ----------------------------
+            if (tid == 0) {
+                umma::fence_after_sync();
+                const uint32_t bb = smem_u32(big);
+                const uint32_t id = umma::idesc_bf16(128, 128, 0, 1);
+                constexpr uint32_t PA[3] = {BIG_P0, BIG_P0, BIG_P1}, UB[3] = {BIG_U0, BIG_U1, BIG_U0};
+#pragma unroll
+                for (int cmb = 0; cmb < 3; ++cmb)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma::mma_bf16(tmem + TM_DP, umma::smem_desc(bb + PA[cmb] - 8192 + kk * 32, 16, 1024),
+                                       umma::smem_desc(bb + UB[cmb] + kk * 2048, 8192, 1024), id, (cmb | kk) != 0);
+                const uint32_t ka = smem_u32(sm + kq + KQ_K0);
+                const uint32_t id3 = umma::idesc_bf16(128, 128, 1, 1);
+                constexpr uint32_t YB[3] = {BIG_Y0, BIG_Y1, BIG_Y2};
+#pragma unroll
+                for (int y = 0; y < 3; ++y)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma::mma_bf16(tmem + TM_D3, umma::smem_desc(ka + kk * 2048, 16384, 1024),
+                                       umma::smem_desc(bb + YB[y] + kk * 2048, 8192, 1024), id3, (y | kk) != 0);
+                umma::mma_commit(smem_u32(&bars[3]));
+            }
+            ok = wait_bar(smem_u32(&bars[3]), parity, p.status);
+            if (!__syncthreads_and(ok)) break;
+            umma::fence_after_sync();
+
+            // ---- readout o_t = gamma_t S0^T q_t + (P U)_t (quarters 2, 3) -------------------
+            bool bad = false;
+            if (q4 >= 2) {
+                const int t = 32 * (q4 - 2) + lane;
+                const float gt = sGam[t];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float a[32], d[32];
+                    umma::tmem_ld32(tl + TM_D2 + 64 * ch + 32 * hh, a);
+                    umma::tmem_ld32(tl + TM_DP + 64 * ch + 32 * hh, d);
+                    if (t < Lc) {
+                        float4 *dst = reinterpret_cast<float4 *>(og + (size_t)(t0 + t) * D + 64 * ch + 32 * hh);
+#pragma unroll
+                        for (int u = 0; u < 32; u += 4) {
+                            float4 o4;
+                            const int j = 64 * ch + 32 * hh + u;
+                            o4.x = gt * (sC[j] * a[u]) + d[u];
+                            o4.y = gt * (sC[j + 1] * a[u + 1]) + d[u + 1];
+                            o4.z = gt * (sC[j + 2] * a[u + 2]) + d[u + 2];
+                            o4.w = gt * (sC[j + 3] * a[u + 3]) + d[u + 3];
+                            bad |= !isfinite(o4.x) || !isfinite(o4.y) || !isfinite(o4.z) || !isfinite(o4.w);
+                            dst[u >> 2] = o4;
+                        }
+                    }
+                }
+            }
+            // ---- chunk-end state S_C = gamma_C S0 + D3 (row i, columns 64 ch .. +63) --------
+            const int i = 32 * q4 + lane;
+            float S[64];
+            {
+                const float gC = miscf[1], ri = sR[i];
+                const uint8_t *qrow = sm + OFF_QC + ch * 16384;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v[32];
+                    umma::tmem_ld32(tl + TM_D3 + 64 * ch + 32 * hh, v);
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const int c8 = 4 * hh + c4;
+                        float qv[8];
+                        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(qrow + sw128_chunk(i, c8)), qv);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int j = 64 * ch + 8 * c8 + e;
+                            S[8 * c8 + e] = gC * ((ri * sC[j]) * qv[e]) + v[8 * c4 + e];
+                        }
+                    }
+                }
+            }
+            umma::fence_before_sync();
+            __syncthreads();  // every use of the chunk-start scales is done
+
+
+            // ---- requantize: column scales (impact-weighted RMS), row scales, codes -----------
+            {
+                float *red = smf(big, BIG_RED), *rmax = smf(big, BIG_RMAX);
+                const float wi = sW[i];
+                float e[64];
+#pragma unroll
+                for (int j = 0; j < 64; ++j) e[j] = wi * S[j] * S[j];
+                warp_reduce_scatter64(e);
+                *reinterpret_cast<float2 *>(red + q4 * D + 64 * ch + 2 * lane) = make_float2(e[0], e[1]);
+                __syncthreads();
+                if (tid < D) {
+                    const float E = (red[tid] + red[D + tid]) + (red[2 * D + tid] + red[3 * D + tid]);
+                    float cj = sqrtf(E / miscf[0]);
+                    if (cj == 0.f) cj = 1.f;
+                    bad |= !isfinite(cj);
+                    sC[tid] = cj;
+                    red[tid] = __frcp_rn(cj);  // this column's partials have been read
+                }
+                __syncthreads();
+                float m = 0.f;
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    S[j] = S[j] * red[64 * ch + j];
+                    m = fmaxf(m, fabsf(S[j]));
+                }
+                rmax[ch * D + i] = m;
+                __syncthreads();
+                m = fmaxf(rmax[i], rmax[D + i]);
+                float ri = m / (float)P::QMAX;
+                if (ri == 0.f) ri = 1.f;
+                bad |= !isfinite(ri);
+                const float rri = __frcp_rn(ri);
+                int qc[64];
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    float x = rintf(S[j] * rri);
+                    x = fminf(fmaxf(x, -(float)P::QMAX), (float)P::QMAX);
+                    qc[j] = (int)x;
+                }
+                // next chunk's B operand (row i, atom column ch) and scales
+                uint8_t *qrow = sm + OFF_QC + ch * 16384;
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; ++e2)
+                        w4[e2] = umma::pack_bf16(__float2bfloat16_rn((float)qc[8 * c8 + 2 * e2]),
+                                                 __float2bfloat16_rn((float)qc[8 * c8 + 2 * e2 + 1]));
+                    *reinterpret_cast<uint4 *>(qrow + sw128_chunk(i, c8)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+                if (ch == 0) sR[i] = ri;
+                if (c + 1 == nch) {  // the last chunk of the call: the state goes back to HBM
+                    store_codes_row<BITS>(gblock, i, ch, qc);
+                    float *gsc = reinterpret_cast<float *>(gblock + P::SOFF);
+                    if (ch == 0) gsc[i] = ri;
+                    if (tid < D) gsc[D + tid] = sC[tid];
+                }
+            }
+            if (bad) flag(p.status, kFlagNonfinite);
+            umma::fence_before_sync();
+            __syncthreads();
+        }
+    }
+    // release Tensor Memory once every thread's accesses have completed
+    umma::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        umma::fence_after_sync();
+        umma::tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int BITS>
+cudaError_t launch_w(const TileParams &p, int T, cudaStream_t s)
+{
+    auto kernel = prefill_wy_kernel<BITS>;
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    int dev = 0, sms = 0;
+    err = cudaGetDevice(&dev);
+    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+    const int grid = p.ntiles < sms ? p.ntiles : sms;
+    kernel<<<grid, NT, SMEM_BYTES, s>>>(p, T);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Chunked prefill of 128 x 128 tiles with bf16 inputs and the scalar gate; every entry of
+// p.table has width `bits` (4, 6 or 8).
+cudaError_t launch_prefill_wy(const TileParams &p, int bits, int T, cudaStream_t s)
+{
+    switch (bits) {
+    case 4: return launch_w<4>(p, T, s);
+    case 6: return launch_w<6>(p, T, s);
+    case 8: return launch_w<8>(p, T, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace stq

@@ -287,11 +287,30 @@ stq_status stq_prefill_chunk(const stq_layout *L, void *pool, int32_t pool_slots
     p->alpha = alpha;
     p->w = w;
     p->o = o;
-    std::vector<int> ord(L->H);
-    for (int h = 0; h < L->H; ++h) ord[h] = h;
-    fill_table(*p, L, ord, 0, L->H, 0);
-    p->ntiles = B * L->H;
-    return from_cuda(stq::launch_prefill_seq(*p, L->in_dtype == STQ_BF16, T, chunk, (cudaStream_t)stream));
+    // 128 x 128 heads with bf16 inputs, the scalar gate and 64-token chunks take the tensor-core
+    // WY path, one launch per code width; FP16 pivot heads and every other configuration take the
+    // sequential kernel.
+    const bool wy = L->dk == 128 && L->gate == STQ_GATE_SCALAR && L->in_dtype == STQ_BF16 && chunk == 64;
+    if (!wy) {
+        std::vector<int> ord(L->H);
+        for (int h = 0; h < L->H; ++h) ord[h] = h;
+        fill_table(*p, L, ord, 0, L->H, 0);
+        p->ntiles = B * L->H;
+        return from_cuda(stq::launch_prefill_seq(*p, L->in_dtype == STQ_BF16, T, chunk, (cudaStream_t)stream));
+    }
+    const std::vector<int> ord = order_by_size(L, 0, L->H);
+    for (int first = 0; first < L->H;) {
+        const int bits = L->bits[ord[first]];
+        int n = 0;
+        while (first + n < L->H && L->bits[ord[first + n]] == bits) ++n;
+        fill_table(*p, L, ord, first, n, 0);
+        p->ntiles = B * n;
+        const cudaError_t e = bits == 16 ? stq::launch_prefill_seq(*p, 1, T, chunk, (cudaStream_t)stream)
+                                         : stq::launch_prefill_wy(*p, bits, T, (cudaStream_t)stream);
+        if (e != cudaSuccess) return STQ_ERR_CUDA;
+        first += n;
+    }
+    return STQ_OK;
 }
 
 }  // extern "C"

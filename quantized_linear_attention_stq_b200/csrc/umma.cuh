@@ -1,0 +1,136 @@
+// umma.cuh -- fifth-generation tensor core (tcgen05) building blocks for sm_100a: shared-memory
+// matrix descriptors for 128-byte-swizzled bf16 tiles, the instruction descriptor of a
+// bf16 x bf16 -> fp32 MMA, MMA issue / commit, Tensor Memory allocation and loads.
+//
+// Tile layouts (all bf16, 128-byte swizzle; every swizzle atom of 8 rows x 128 B starts on a
+// 1024-byte boundary):
+//  * K-major operand (rows = M or N index, contraction index contiguous): a "box" holds 64
+//    contraction indices of R rows, row r at r * 128 B; the 16-byte chunk c of row r sits at chunk
+//    c ^ (r % 8). Boxes for contraction indices 64..127 follow at a fixed byte stride.
+//  * MN-major operand (rows = contraction index, M or N index contiguous): an "atom column" holds
+//    64 consecutive M/N indices of every contraction row, row k at k * 128 B, chunks swizzled the
+//    same way; the next 64 M/N indices follow at the descriptor's leading byte offset.
+#pragma once
+
+#include <cstdint>
+
+#include "stq_internal.cuh"
+
+namespace stq {
+namespace umma {
+
+#ifdef __CUDACC__
+
+// Byte offset of element (row, col) of a 64-wide bf16 swizzled box (col < 64), from the box base.
+__device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col)
+{
+    return row * 128u + ((((col >> 3) ^ (row & 7u)) & 7u) << 4) + (col & 7u) * 2u;
+}
+
+// Byte offset of the 16-byte chunk holding columns 8c .. 8c+7 of `row`.
+__device__ __forceinline__ uint32_t sw128_chunk(uint32_t row, uint32_t c)
+{
+    return row * 128u + (((c ^ (row & 7u)) & 7u) << 4);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle. `lbo` and `sbo` are byte offsets: for a
+// K-major operand sbo is the stride between 8-row groups and lbo is unused (encoded 16 B); for
+// an MN-major operand lbo is the stride between 64-element atom columns and sbo the stride
+// between groups of 8 contraction rows.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;   // descriptor version of this architecture
+    d |= (uint64_t)2u << 61;   // 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: bf16 A and B, fp32 accumulator, dense, M x N tile.
+// a_mn / b_mn select the MN-major layout of A / B (else K-major).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn)
+{
+    return (1u << 4)                      // D format: f32
+           | (1u << 7)                    // A format: bf16
+           | (1u << 10)                   // B format: bf16
+           | ((uint32_t)a_mn << 15)       // A major
+           | ((uint32_t)b_mn << 16)       // B major
+           | ((uint32_t)(N >> 3) << 17)   // N / 8
+           | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+// D[tmem] (+)= A[smem] * B[smem]; issued by one thread.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// The mbarrier receives one arrival when every MMA this thread issued before has completed.
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Generic-proxy shared-memory writes become visible to the tensor core (async proxy).
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Warp-wide: allocate `ncols` Tensor Memory columns, base address written to shared memory.
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Warp-wide: 32 consecutive fp32 columns of this thread's lane (lane quarter of the warp).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Split x into three bf16 terms h + m + l that carry its 24 significand bits.
+__device__ __forceinline__ void split3(float x, __nv_bfloat16 &h, __nv_bfloat16 &m, __nv_bfloat16 &l)
+{
+    h = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(h);
+    m = __float2bfloat16_rn(r1);
+    l = __float2bfloat16_rn(r1 - __bfloat162float(m));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(__nv_bfloat16 a, __nv_bfloat16 b)
+{
+    return (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+}
+
+#endif  // __CUDACC__
+
+}  // namespace umma
+}  // namespace stq
