@@ -17,7 +17,7 @@
 // Unrolling the per-token recurrence gives exactly these sums; inside a chunk nothing is rounded
 // to the state's codes.
 //
-// Design (B200, one persistent CTA of 256 threads per SM, 512 Tensor Memory columns):
+// Design (B200, one persistent CTA of 512 threads per SM, 512 Tensor Memory columns):
 //  * bf16 inputs are exact bf16 MMA operands. fp32 quantities that enter a contraction (K r, Q r,
 //    T, R', U, decayed U) are split into three bf16 terms carrying all 24 significand bits; the
 //    products keep the terms whose order is at most 2^-24 of the result (P U, which only feeds the
@@ -39,7 +39,7 @@ using umma::sw128_chunk;
 
 constexpr int D = 128;
 constexpr int C = 64;   // chunk length
-constexpr int NT = 256;
+constexpr int NT = 512;
 constexpr int LDL = 68; // row stride (floats) of the fp32 L and T work matrices
 
 // Shared-memory map (bytes from a 1024-aligned base).
@@ -74,8 +74,8 @@ constexpr uint32_t BIG_P0 = 49152, BIG_P1 = 57344;                        // P t
 constexpr uint32_t BIG_U0 = 0, BIG_U1 = 16384;                            // U terms
 constexpr uint32_t BIG_Y0 = 32768, BIG_Y1 = 65536, BIG_Y2 = 81920;        // decayed U terms
 // requantization scratch in BIG (after the last MMA of the chunk has completed)
-constexpr uint32_t BIG_RED = 0;      // [4][128] f32 column-energy partials
-constexpr uint32_t BIG_RMAX = 2048;  // [2][128] f32 row-max partials
+constexpr uint32_t BIG_RED = 0;      // [4][128] f32 column-energy partials (per lane quarter)
+constexpr uint32_t BIG_RMAX = 2048;  // [4][128] f32 row-max partials (per column quarter)
 // T-inverse scratch in the RT area (before the T terms are written)
 constexpr uint32_t RT_G = 0;         // [3][16][17] f32
 
@@ -111,9 +111,9 @@ __device__ __forceinline__ void load_chunk_async(uint8_t *sm, uint32_t kq_off, i
                                                  int Lc)
 {
     const int tid = threadIdx.x;
-    // 2 tensors x 64 rows x 16 chunks of 16 B = 2048 copies, 8 per thread
+    // 2 tensors x 64 rows x 16 chunks of 16 B = 2048 copies, 4 per thread
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < 4; ++k) {
         const int e = tid + NT * k;
         const int tensor = e >> 10, row = (e >> 4) & 63, ch = e & 15;
         const __nv_bfloat16 *src = (tensor ? qbase : kbase) + (size_t)(row < Lc ? row : 0) * D + ch * 8;
@@ -137,36 +137,32 @@ __device__ __forceinline__ void load_chunk_async(uint8_t *sm, uint32_t kq_off, i
 
 
 // ---------------------------------------------------------------------------------------------
-// State load / store (packed little-endian offset-binary bitstream, row-major)
+// State load / store (packed little-endian offset-binary bitstream, row-major). Thread (row i,
+// quarter part) owns codes i, 32 part .. 32 part + 31: BITS 32-bit words at an 8-byte boundary.
 // ---------------------------------------------------------------------------------------------
-
-// Thread (row i, half h) unpacks codes i, 64h .. 64h+63 of the tile and writes them as bf16 into
-// the B-operand tile (contraction row i, atom column h).
 template <int BITS>
-__device__ __forceinline__ void load_codes_row(const uint8_t *gblock, uint8_t *qc, int i, int h)
+__device__ __forceinline__ void load_codes_row(const uint8_t *gblock, uint8_t *qc, int i, int part)
 {
     using P = PCfg<BITS>;
-    constexpr int NW = 2 * BITS;  // 32-bit words holding 64 codes
-    uint32_t wv[NW + 1];
-    const uint4 *src = reinterpret_cast<const uint4 *>(gblock + (size_t)i * P::ROWB + h * (P::ROWB / 2));
+    uint32_t wv[BITS + 1];
+    const uint2 *src = reinterpret_cast<const uint2 *>(gblock + (size_t)i * P::ROWB + part * (4 * BITS));
 #pragma unroll
-    for (int k = 0; k < NW / 4; ++k) {
-        const uint4 x = src[k];
-        wv[4 * k] = x.x;
-        wv[4 * k + 1] = x.y;
-        wv[4 * k + 2] = x.z;
-        wv[4 * k + 3] = x.w;
+    for (int k = 0; k < BITS / 2; ++k) {
+        const uint2 x = src[k];
+        wv[2 * k] = x.x;
+        wv[2 * k + 1] = x.y;
     }
-    wv[NW] = 0u;
+    wv[BITS] = 0u;
+    uint8_t *atom = qc + (part >> 1) * 16384;
 #pragma unroll
-    for (int c8 = 0; c8 < 8; ++c8) {
+    for (int k = 0; k < 4; ++k) {
         uint32_t packed[4];
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
             float f[2];
 #pragma unroll
             for (int z = 0; z < 2; ++z) {
-                const int col = 8 * c8 + e + z, bit = BITS * col, wi = bit >> 5, sh = bit & 31;
+                const int col = 8 * k + e + z, bit = BITS * col, wi = bit >> 5, sh = bit & 31;
                 uint32_t u = wv[wi] >> sh;
                 if (sh + BITS > 32) u |= wv[wi + 1] << (32 - sh);
                 u &= (1u << BITS) - 1u;
@@ -174,121 +170,62 @@ __device__ __forceinline__ void load_codes_row(const uint8_t *gblock, uint8_t *q
             }
             packed[e >> 1] = umma::pack_bf16(__float2bfloat16_rn(f[0]), __float2bfloat16_rn(f[1]));
         }
-        *reinterpret_cast<uint4 *>(qc + h * 16384 + sw128_chunk(i, c8)) =
+        *reinterpret_cast<uint4 *>(atom + sw128_chunk(i, 4 * (part & 1) + k)) =
             make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }
 }
 
-// Pack 64 integer codes (values in [-qmax, qmax]) of row i, half h into the tile in HBM.
 template <int BITS>
-__device__ __forceinline__ void store_codes_row(uint8_t *gblock, int i, int h, const int (&q)[64])
+__device__ __forceinline__ void store_codes_row(uint8_t *gblock, int i, int part, const int (&q)[32])
 {
     using P = PCfg<BITS>;
-    constexpr int NW = 2 * BITS;
-    uint32_t wv[NW];
+    uint32_t wv[BITS];
 #pragma unroll
-    for (int k = 0; k < NW; ++k) wv[k] = 0u;
+    for (int k = 0; k < BITS; ++k) wv[k] = 0u;
 #pragma unroll
-    for (int col = 0; col < 64; ++col) {
+    for (int col = 0; col < 32; ++col) {
         const uint32_t u = (uint32_t)(q[col] + P::OFFS);
         const int bit = BITS * col, wi = bit >> 5, sh = bit & 31;
         wv[wi] |= u << sh;
         if (sh + BITS > 32) wv[wi + 1] |= u >> (32 - sh);
     }
-    uint4 *dst = reinterpret_cast<uint4 *>(gblock + (size_t)i * P::ROWB + h * (P::ROWB / 2));
+    uint2 *dst = reinterpret_cast<uint2 *>(gblock + (size_t)i * P::ROWB + part * (4 * BITS));
 #pragma unroll
-    for (int k = 0; k < NW / 4; ++k) dst[k] = make_uint4(wv[4 * k], wv[4 * k + 1], wv[4 * k + 2], wv[4 * k + 3]);
+    for (int k = 0; k < BITS / 2; ++k) dst[k] = make_uint2(wv[2 * k], wv[2 * k + 1]);
 }
 
 // ---------------------------------------------------------------------------------------------
-// T = (I + L)^-1 for a strictly lower triangular 64 x 64 L (fp32, row stride LDL), by 16 x 16
-// blocks: the four diagonal blocks by forward substitution (one warp each), then the off-diagonal
-// blocks T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj in order of distance i - j. G: [3][16][17] scratch.
-// All 256 threads call it; it ends with a barrier.
+// bf16 term splitting, two values at a time (packed conversions, f32x2 residuals).
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ void invert_unit_lower(const float *L, float *T, float *G)
+__device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 h) { return *reinterpret_cast<uint32_t *>(&h); }
+
+// x = h + m + l exactly (three bf16 terms carry the 24 significand bits of each value).
+__device__ __forceinline__ void split3_pair(float2 x, uint32_t &h, uint32_t &m, uint32_t &l)
 {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (warp < 4 && lane < 16) {
-        const int b0 = 16 * warp, c = lane;
-        float x[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) x[t] = (t == c) ? 1.f : 0.f;
-#pragma unroll
-        for (int s = 0; s < 16; ++s) {
-            const float xs = x[s];
-#pragma unroll
-            for (int t = s + 1; t < 16; ++t) x[t] = fmaf(-L[(b0 + t) * LDL + b0 + s], xs, x[t]);
-        }
-#pragma unroll
-        for (int t = 0; t < 16; ++t) T[(b0 + t) * LDL + b0 + c] = x[t];
-    }
-    // zero the strictly upper blocks (never read by the products below, but T is an MMA operand)
-    for (int e = tid; e < 64 * 64; e += NT) {
-        const int t = e >> 6, s = e & 63;
-        if ((s >> 4) > (t >> 4)) T[t * LDL + s] = 0.f;
-    }
-    __syncthreads();
-    const int r = tid >> 4, c = tid & 15;
-#pragma unroll
-    for (int d = 1; d < 4; ++d) {
-        // G_ij = sum_{k=j}^{i-1} L_ik T_kj for the blocks at distance d
-        for (int j = 0; j + d < 4; ++j) {
-            const int i = j + d;
-            float acc = 0.f;
-            for (int k = j; k < i; ++k) {
-                const float *Lr = L + (16 * i + r) * LDL + 16 * k;
-                const float *Tc = T + (16 * k) * LDL + 16 * j + c;
-#pragma unroll
-                for (int u = 0; u < 16; ++u) acc = fmaf(Lr[u], Tc[u * LDL], acc);
-            }
-            G[j * 272 + r * 17 + c] = acc;
-        }
-        __syncthreads();
-        for (int j = 0; j + d < 4; ++j) {
-            const int i = j + d;
-            const float *Tr = T + (16 * i + r) * LDL + 16 * i;
-            float acc = 0.f;
-#pragma unroll
-            for (int u = 0; u < 16; ++u) acc = fmaf(Tr[u], G[j * 272 + u * 17 + c], acc);
-            T[(16 * i + r) * LDL + 16 * j + c] = -acc;
-        }
-        __syncthreads();
-    }
+    const float2 neg = make_float2(-1.f, -1.f);
+    const __nv_bfloat162 hb = __floats2bfloat162_rn(x.x, x.y);
+    const float2 r1 = __ffma2_rn(__bfloat1622float2(hb), neg, x);
+    const __nv_bfloat162 mb = __floats2bfloat162_rn(r1.x, r1.y);
+    const float2 r2 = __ffma2_rn(__bfloat1622float2(mb), neg, r1);
+    h = bf2_bits(hb);
+    m = bf2_bits(mb);
+    l = bf2_bits(__floats2bfloat162_rn(r2.x, r2.y));
 }
 
-// Warp reduce-scatter of 64 per-lane values: afterwards lane l holds the warp sums of entries
-// 2l and 2l+1 in v[0], v[1].
-__device__ __forceinline__ void warp_reduce_scatter64(float (&v)[64])
+__device__ __forceinline__ void split2_pair(float2 x, uint32_t &h, uint32_t &l)
 {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int step = 0; step < 5; ++step) {
-        const int o = 16 >> step, n = 64 >> step, hn = n >> 1;
-        const bool up = (lane & o) != 0;
-#pragma unroll
-        for (int k = 0; k < hn; ++k) {
-            const float keep = up ? v[k + hn] : v[k];
-            const float send = up ? v[k] : v[k + hn];
-            v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-    }
+    const __nv_bfloat162 hb = __floats2bfloat162_rn(x.x, x.y);
+    const float2 r1 = __ffma2_rn(__bfloat1622float2(hb), make_float2(-1.f, -1.f), x);
+    h = bf2_bits(hb);
+    l = bf2_bits(__floats2bfloat162_rn(r1.x, r1.y));
 }
 
-
-// Split helpers writing 8 consecutive values as one 16-byte chunk per term.
+// Eight values -> one 16-byte chunk per term.
 __device__ __forceinline__ void store_split3(uint8_t *t0, uint8_t *t1, uint8_t *t2, uint32_t off, const float (&x)[8])
 {
     uint32_t a[4], b[4], c[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        __nv_bfloat16 h0, m0, l0, h1, m1, l1;
-        umma::split3(x[2 * e], h0, m0, l0);
-        umma::split3(x[2 * e + 1], h1, m1, l1);
-        a[e] = umma::pack_bf16(h0, h1);
-        b[e] = umma::pack_bf16(m0, m1);
-        c[e] = umma::pack_bf16(l0, l1);
-    }
+    for (int e = 0; e < 4; ++e) split3_pair(make_float2(x[2 * e], x[2 * e + 1]), a[e], b[e], c[e]);
     *reinterpret_cast<uint4 *>(t0 + off) = make_uint4(a[0], a[1], a[2], a[3]);
     *reinterpret_cast<uint4 *>(t1 + off) = make_uint4(b[0], b[1], b[2], b[3]);
     *reinterpret_cast<uint4 *>(t2 + off) = make_uint4(c[0], c[1], c[2], c[3]);
@@ -298,13 +235,7 @@ __device__ __forceinline__ void store_split2(uint8_t *t0, uint8_t *t1, uint32_t 
 {
     uint32_t a[4], b[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * e]), h1 = __float2bfloat16_rn(x[2 * e + 1]);
-        const __nv_bfloat16 l0 = __float2bfloat16_rn(x[2 * e] - __bfloat162float(h0));
-        const __nv_bfloat16 l1 = __float2bfloat16_rn(x[2 * e + 1] - __bfloat162float(h1));
-        a[e] = umma::pack_bf16(h0, h1);
-        b[e] = umma::pack_bf16(l0, l1);
-    }
+    for (int e = 0; e < 4; ++e) split2_pair(make_float2(x[2 * e], x[2 * e + 1]), a[e], b[e]);
     *reinterpret_cast<uint4 *>(t0 + off) = make_uint4(a[0], a[1], a[2], a[3]);
     *reinterpret_cast<uint4 *>(t1 + off) = make_uint4(b[0], b[1], b[2], b[3]);
 }
@@ -319,6 +250,94 @@ __device__ __forceinline__ void bf16x8_to_f32(uint4 raw, float (&x)[8])
     }
 }
 
+// ---------------------------------------------------------------------------------------------
+// T = (I + L)^-1 for a strictly lower triangular 64 x 64 L (fp32, row stride LDL), by 16 x 16
+// blocks: the four diagonal blocks by forward substitution (one warp each), then the off-diagonal
+// blocks T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj in order of distance i - j. G: [3][16][17]
+// scratch. All threads call it; it ends with a barrier.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void invert_unit_lower(const float *L, float *T, float *G)
+{
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (warp < 4 && lane < 16) {
+        const int b0 = 16 * warp, c = lane;
+        float x[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) x[t] = (t == c) ? 1.f : 0.f;
+#pragma unroll
+        for (int s = 0; s < 15; ++s) {
+            const float xs = x[s];
+#pragma unroll
+            for (int t = s + 1; t < 16; ++t) x[t] = fmaf(-L[(b0 + t) * LDL + b0 + s], xs, x[t]);
+        }
+#pragma unroll
+        for (int t = 0; t < 16; ++t) T[(b0 + t) * LDL + b0 + c] = x[t];
+    } else if (warp >= 4) {
+        // zero the strictly upper blocks (T is an MMA operand in full)
+        for (int e = tid - 128; e < 64 * 64; e += NT - 128) {
+            const int t = e >> 6, s = e & 63;
+            if ((s >> 4) > (t >> 4)) T[t * LDL + s] = 0.f;
+        }
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int d = 1; d < 4; ++d) {
+        const int nblk = 4 - d;
+        // G_j = sum_{k=j}^{j+d-1} L_{j+d,k} T_kj, one element per thread and block
+        for (int e = tid; e < 256 * nblk; e += NT) {
+            const int j = e >> 8, r = (e >> 4) & 15, c = e & 15, i = j + d;
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            for (int k = j; k < i; ++k) {
+                const float *Lr = L + (16 * i + r) * LDL + 16 * k;
+                const float *Tc = T + (16 * k) * LDL + 16 * j + c;
+#pragma unroll
+                for (int u = 0; u < 16; u += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4 *>(Lr + u);
+                    a0 = fmaf(l4.x, Tc[u * LDL], a0);
+                    a1 = fmaf(l4.y, Tc[(u + 1) * LDL], a1);
+                    a2 = fmaf(l4.z, Tc[(u + 2) * LDL], a2);
+                    a3 = fmaf(l4.w, Tc[(u + 3) * LDL], a3);
+                }
+            }
+            G[j * 272 + r * 17 + c] = (a0 + a1) + (a2 + a3);
+        }
+        __syncthreads();
+        for (int e = tid; e < 256 * nblk; e += NT) {
+            const int j = e >> 8, r = (e >> 4) & 15, c = e & 15, i = j + d;
+            const float *Tr = T + (16 * i + r) * LDL + 16 * i;
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+            for (int u = 0; u < 16; u += 4) {
+                const float4 t4 = *reinterpret_cast<const float4 *>(Tr + u);
+                a0 = fmaf(t4.x, G[j * 272 + u * 17 + c], a0);
+                a1 = fmaf(t4.y, G[j * 272 + (u + 1) * 17 + c], a1);
+                a2 = fmaf(t4.z, G[j * 272 + (u + 2) * 17 + c], a2);
+                a3 = fmaf(t4.w, G[j * 272 + (u + 3) * 17 + c], a3);
+            }
+            T[(16 * i + r) * LDL + 16 * j + c] = -((a0 + a1) + (a2 + a3));
+        }
+        __syncthreads();
+    }
+}
+
+// Warp reduce-scatter of 32 per-lane values: afterwards v[0] of lane l is the warp sum of entry l.
+__device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32])
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int step = 0; step < 5; ++step) {
+        const int o = 16 >> step, hn = 16 >> step;
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int k = 0; k < hn; ++k) {
+            const float keep = up ? v[k + hn] : v[k];
+            const float send = up ? v[k] : v[k + hn];
+            v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    return v[0];
+}
+
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int32_t *status)
 {
     const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
@@ -326,10 +345,23 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int32_t 
     return ok;
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
 
 // ---------------------------------------------------------------------------------------------
 // The kernel: persistent CTAs over (request, head) tiles of one code width; the chunks of a tile
-// run in order.
+// run in order. Warp w reads Tensor Memory lane quarter q4 = w % 4 and column quarter cq = w / 4.
 // ---------------------------------------------------------------------------------------------
 template <int BITS>
 __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant__ TileParams p, const int T_tok)
@@ -337,7 +369,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
     using P = PCfg<BITS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, ch = warp >> 2;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, cq = warp >> 2;
     float *sR = smf(sm, OFF_SMALL + S_R), *sC = smf(sm, OFF_SMALL + S_C), *sW = smf(sm, OFF_SMALL + S_W);
     double *sLG = smd(sm, OFF_SMALL + S_LG), *sG = smd(sm, OFF_SMALL + S_G);
     float *sGam = smf(sm, OFF_SMALL + S_GAM), *sDC = smf(sm, OFF_SMALL + S_DC);
@@ -379,7 +411,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
 
         // ---- the tile's state onto the chip ----------------------------------------------
         __syncthreads();  // the previous tile is completely done with shared memory
-        load_codes_row<BITS>(gblock, sm + OFF_QC, tid >> 1, tid & 1);
+        load_codes_row<BITS>(gblock, sm + OFF_QC, tid >> 2, tid & 3);
         if (tid < D) {
             const float *sc = reinterpret_cast<const float *>(gblock + P::SOFF);
             sR[tid] = sc[tid];
@@ -395,6 +427,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
             if (lane == 0) miscf[0] = s;
         }
 
+#pragma unroll 1
         for (int c = 0; c < nch && ok; ++c, parity ^= 1u) {
             const int t0 = c * C, Lc = (T_tok - t0) < C ? (T_tok - t0) : C;
             const uint32_t kq = (c & 1) ? OFF_XY1 : OFF_XY0;  // this chunk's K / Q
@@ -404,13 +437,13 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
             const float *sAlpha = smf(sm, OFF_SMALL + S_ALPHA) + buf * C;
             float *Lm = smf(sm, lt), *Tm = smf(sm, lt + 64 * LDL * 4);
 
-            // v rows for R' (lane quarters 0, 1: row t, columns 64 ch .. +63), in flight early
-            uint4 vraw[8];
+            // v rows for R' (lane quarters 0, 1: row t, columns 32 cq .. +31), in flight early
+            uint4 vraw[4];
             if (q4 < 2) {
                 const int t = 32 * q4 + lane;
-                const uint4 *vs = reinterpret_cast<const uint4 *>(vg + (size_t)(t0 + (t < Lc ? t : 0)) * D + 64 * ch);
+                const uint4 *vs = reinterpret_cast<const uint4 *>(vg + (size_t)(t0 + (t < Lc ? t : 0)) * D + 32 * cq);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) vraw[k] = t < Lc ? vs[k] : make_uint4(0u, 0u, 0u, 0u);
+                for (int k = 0; k < 4; ++k) vraw[k] = t < Lc ? vs[k] : make_uint4(0u, 0u, 0u, 0u);
             }
             cp_async_wait_all();
             umma::fence_proxy_async();
@@ -430,7 +463,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                 }
                 umma::mma_commit(smem_u32(&bars[0]));
             }
-            // ---- cumulative log decay of the chunk (fp64) ------------------------------
+            // ---- cumulative log decay of the chunk (fp64), warps 0 and 1 -------------------
             if (tid < C) {
                 double g = tid < Lc ? log((double)sAlpha[tid]) : 0.0;
 #pragma unroll
@@ -440,17 +473,19 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                 }
                 sLG[tid] = g;  // within-warp inclusive prefix
             }
-            // ---- A operand of D2: three bf16 terms of [K r; Q r] ------------------------
+            // ---- A operand of D2: three bf16 terms of [K r; Q r] (row m, columns 32 part ..) -
             {
-                const int m = tid >> 1, h = tid & 1, row = m & 63;
-                const uint8_t *xb = sm + kq + (m < 64 ? (h ? KQ_K1 : KQ_K0) : (h ? KQ_Q1 : KQ_Q0));
-                uint8_t *a0 = big + h * 16384, *a1 = a0 + 32768, *a2 = a0 + 65536;
+                const int m = tid >> 2, part = tid & 3, row = m & 63, hb = part >> 1;
+                const uint8_t *xb = sm + kq + (m < 64 ? (hb ? KQ_K1 : KQ_K0) : (hb ? KQ_Q1 : KQ_Q0));
+                uint8_t *a0 = big + hb * 16384, *a1 = a0 + 32768, *a2 = a0 + 65536;
+                const float *rr = sR + 32 * part;
 #pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
+                for (int k = 0; k < 4; ++k) {
+                    const int c8 = 4 * (part & 1) + k;
                     float x[8];
                     bf16x8_to_f32(*reinterpret_cast<const uint4 *>(xb + sw128_chunk(row, c8)), x);
-                    const float4 ra = *reinterpret_cast<const float4 *>(sR + 64 * h + 8 * c8);
-                    const float4 rb = *reinterpret_cast<const float4 *>(sR + 64 * h + 8 * c8 + 4);
+                    const float4 ra = *reinterpret_cast<const float4 *>(rr + 8 * k);
+                    const float4 rb = *reinterpret_cast<const float4 *>(rr + 8 * k + 4);
                     x[0] *= ra.x; x[1] *= ra.y; x[2] *= ra.z; x[3] *= ra.w;
                     x[4] *= rb.x; x[5] *= rb.y; x[6] *= rb.z; x[7] *= rb.w;
                     store_split3(a0, a1, a2, sw128_chunk(m, c8), x);
@@ -461,7 +496,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
             if (tid == 0) {
                 const uint32_t abase = smem_u32(big), bbase = smem_u32(sm + OFF_QC);
                 const uint32_t id = umma::idesc_bf16(128, 128, 0, 1);
-#pragma unroll
+#pragma unroll 1
                 for (int term = 0; term < 3; ++term)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
@@ -484,52 +519,49 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                 if (tid == 0) miscf[1] = (float)exp(gl);
             }
 
-            // ---- L (lane quarters 0, 1) and P (quarters 2, 3) from D1 ---------------------
+            // ---- L (lane quarters 0, 1) and P (quarters 2, 3) from D1, columns 16 cq .. ---
             ok = wait_bar(smem_u32(&bars[0]), parity, p.status);
             if (!__syncthreads_and(ok)) break;
             umma::fence_after_sync();
-            float pv[32];
+            float pv[16];
             {
-                float v[32];
-                umma::tmem_ld32(tl + TM_D1 + 32 * ch, v);
+                float v[16];
+                tmem_ld16(tl + TM_D1 + 16 * cq, v);
                 const int t = 32 * (q4 & 1) + lane;
                 const double gt = sG[t];
                 if (q4 < 2) {
                     const float bt = sBeta[t];
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) {
-                        const int s = 32 * ch + u;
+                    for (int u = 0; u < 16; ++u) {
+                        const int s = 16 * cq + u;
                         Lm[t * LDL + s] = s < t ? bt * expf((float)(gt - sG[s])) * v[u] : 0.f;
                     }
                 } else {
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) {
-                        const int s = 32 * ch + u;
+                    for (int u = 0; u < 16; ++u) {
+                        const int s = 16 * cq + u;
                         pv[u] = s <= t ? expf((float)(gt - sG[s])) * v[u] : 0.f;
                     }
                 }
             }
             __syncthreads();
             invert_unit_lower(Lm, Tm, smf(sm, OFF_RT + RT_G));
-            // T in three bf16 terms (K-major, rows t, contraction s)
+            // T in three bf16 terms (K-major, rows t, contraction s), one chunk per thread
             {
-                const int t = tid >> 2, part = tid & 3;
-                uint8_t *r0 = sm + OFF_RT, *r1 = r0 + 8192, *r2 = r0 + 16384;
-#pragma unroll
-                for (int hc = 0; hc < 2; ++hc) {
-                    const int c8 = 2 * part + hc;
-                    float x[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] = Tm[t * LDL + 8 * c8 + e];
-                    store_split3(r0, r1, r2, sw128_chunk(t, c8), x);
-                }
+                const int t = tid >> 3, c8 = tid & 7;
+                uint8_t *r0 = sm + OFF_RT;
+                float x[8];
+                const float4 xa = *reinterpret_cast<const float4 *>(Tm + t * LDL + 8 * c8);
+                const float4 xb4 = *reinterpret_cast<const float4 *>(Tm + t * LDL + 8 * c8 + 4);
+                x[0] = xa.x; x[1] = xa.y; x[2] = xa.z; x[3] = xa.w;
+                x[4] = xb4.x; x[5] = xb4.y; x[6] = xb4.z; x[7] = xb4.w;
+                store_split3(r0, r0 + 8192, r0 + 16384, sw128_chunk(t, c8), x);
             }
             __syncthreads();  // L / T are dead: the area takes the next chunk's K / Q
             if (c + 1 < nch) {
                 const int t1 = t0 + C, L1 = (T_tok - t1) < C ? (T_tok - t1) : C;
                 load_chunk_async(sm, lt, buf ^ 1, kg + (size_t)t1 * D, qg + (size_t)t1 * D, bg + t1, ag + t1, L1);
             }
-
 
             // ---- R' (quarters 0, 1) and P terms (quarters 2, 3) once D2 is complete -------
             ok = wait_bar(smem_u32(&bars[1]), parity, p.status);
@@ -538,32 +570,25 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
             if (q4 < 2) {
                 const int t = 32 * q4 + lane;
                 const float bt = sBeta[t], gt = sGam[t];
-                uint8_t *r0 = big + BIG_R0 + ch * 8192, *r1 = big + BIG_R1 + ch * 8192, *r2 = big + BIG_R2 + ch * 8192;
+                const uint32_t aoff = (cq >> 1) * 8192;
+                float v[32];
+                umma::tmem_ld32(tl + TM_D2 + 32 * cq, v);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float v[32];
-                    umma::tmem_ld32(tl + TM_D2 + 64 * ch + 32 * hh, v);
+                for (int k = 0; k < 4; ++k) {
+                    float vv[8], x[8];
+                    bf16x8_to_f32(vraw[k], vv);
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        const int c8 = 4 * hh + c4;
-                        float vv[8], x[8];
-                        bf16x8_to_f32(vraw[c8], vv);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int j = 64 * ch + 8 * c8 + e;
-                            x[e] = bt * (vv[e] - gt * (sC[j] * v[8 * c4 + e]));
-                        }
-                        store_split3(r0, r1, r2, sw128_chunk(t, c8), x);
-                    }
+                    for (int e = 0; e < 8; ++e) x[e] = bt * (vv[e] - gt * (sC[32 * cq + 8 * k + e] * v[8 * k + e]));
+                    store_split3(big + BIG_R0, big + BIG_R1, big + BIG_R2, aoff + sw128_chunk(t, 4 * (cq & 1) + k), x);
                 }
             } else {
                 const int t = 32 * (q4 - 2) + lane;
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
+                for (int k = 0; k < 2; ++k) {
                     float x[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] = pv[8 * c4 + e];
-                    store_split2(big + BIG_P0, big + BIG_P1, sw128_chunk(t, 4 * ch + c4), x);
+                    for (int e = 0; e < 8; ++e) x[e] = pv[8 * k + e];
+                    store_split2(big + BIG_P0, big + BIG_P1, sw128_chunk(t, 2 * cq + k), x);
                 }
             }
             umma::fence_proxy_async();
@@ -589,23 +614,20 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
             if (q4 >= 2) {
                 const int t = 32 * (q4 - 2) + lane;
                 const float dc = sDC[t];
+                const uint32_t aoff = (cq >> 1) * 8192;
+                float v[32];
+                umma::tmem_ld32(tl + TM_DU + 32 * cq, v);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float v[32];
-                    umma::tmem_ld32(tl + TM_DU + 64 * ch + 32 * hh, v);
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t off = aoff + sw128_chunk(t, 4 * (cq & 1) + k);
+                    float x[8], y[8];
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        const int c8 = 4 * hh + c4;
-                        const uint32_t off = ch * 8192 + sw128_chunk(t, c8);
-                        float x[8], y[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            x[e] = v[8 * c4 + e];
-                            y[e] = dc * x[e];
-                        }
-                        store_split2(big + BIG_U0, big + BIG_U1, off, x);
-                        store_split3(big + BIG_Y0, big + BIG_Y1, big + BIG_Y2, off, y);
+                    for (int e = 0; e < 8; ++e) {
+                        x[e] = v[8 * k + e];
+                        y[e] = dc * x[e];
                     }
+                    store_split2(big + BIG_U0, big + BIG_U1, off, x);
+                    store_split3(big + BIG_Y0, big + BIG_Y1, big + BIG_Y2, off, y);
                 }
             }
             umma::fence_proxy_async();
@@ -643,63 +665,52 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
             if (q4 >= 2) {
                 const int t = 32 * (q4 - 2) + lane;
                 const float gt = sGam[t];
+                float a[32], d[32];
+                umma::tmem_ld32(tl + TM_D2 + 32 * cq, a);
+                umma::tmem_ld32(tl + TM_DP + 32 * cq, d);
+                if (t < Lc) {
+                    float4 *dst = reinterpret_cast<float4 *>(og + (size_t)(t0 + t) * D + 32 * cq);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float a[32], d[32];
-                    umma::tmem_ld32(tl + TM_D2 + 64 * ch + 32 * hh, a);
-                    umma::tmem_ld32(tl + TM_DP + 64 * ch + 32 * hh, d);
-                    if (t < Lc) {
-                        float4 *dst = reinterpret_cast<float4 *>(og + (size_t)(t0 + t) * D + 64 * ch + 32 * hh);
-#pragma unroll
-                        for (int u = 0; u < 32; u += 4) {
-                            float4 o4;
-                            const int j = 64 * ch + 32 * hh + u;
-                            o4.x = gt * (sC[j] * a[u]) + d[u];
-                            o4.y = gt * (sC[j + 1] * a[u + 1]) + d[u + 1];
-                            o4.z = gt * (sC[j + 2] * a[u + 2]) + d[u + 2];
-                            o4.w = gt * (sC[j + 3] * a[u + 3]) + d[u + 3];
-                            bad |= !isfinite(o4.x) || !isfinite(o4.y) || !isfinite(o4.z) || !isfinite(o4.w);
-                            dst[u >> 2] = o4;
-                        }
+                    for (int u = 0; u < 32; u += 4) {
+                        const float4 c4 = *reinterpret_cast<const float4 *>(sC + 32 * cq + u);
+                        float4 o4;
+                        o4.x = gt * (c4.x * a[u]) + d[u];
+                        o4.y = gt * (c4.y * a[u + 1]) + d[u + 1];
+                        o4.z = gt * (c4.z * a[u + 2]) + d[u + 2];
+                        o4.w = gt * (c4.w * a[u + 3]) + d[u + 3];
+                        bad |= !isfinite(o4.x) || !isfinite(o4.y) || !isfinite(o4.z) || !isfinite(o4.w);
+                        dst[u >> 2] = o4;
                     }
                 }
             }
-            // ---- chunk-end state S_C = gamma_C S0 + D3 (row i, columns 64 ch .. +63) --------
+            // ---- chunk-end state S_C = gamma_C S0 + D3 (row i, columns 32 cq .. +31) -------
             const int i = 32 * q4 + lane;
-            float S[64];
+            float S[32];
             {
                 const float gC = miscf[1], ri = sR[i];
-                const uint8_t *qrow = sm + OFF_QC + ch * 16384;
+                const uint8_t *qrow = sm + OFF_QC + (cq >> 1) * 16384;
+                float v[32];
+                umma::tmem_ld32(tl + TM_D3 + 32 * cq, v);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float v[32];
-                    umma::tmem_ld32(tl + TM_D3 + 64 * ch + 32 * hh, v);
+                for (int k = 0; k < 4; ++k) {
+                    float qv[8];
+                    bf16x8_to_f32(*reinterpret_cast<const uint4 *>(qrow + sw128_chunk(i, 4 * (cq & 1) + k)), qv);
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        const int c8 = 4 * hh + c4;
-                        float qv[8];
-                        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(qrow + sw128_chunk(i, c8)), qv);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int j = 64 * ch + 8 * c8 + e;
-                            S[8 * c8 + e] = gC * ((ri * sC[j]) * qv[e]) + v[8 * c4 + e];
-                        }
-                    }
+                    for (int e = 0; e < 8; ++e)
+                        S[8 * k + e] = gC * ((ri * sC[32 * cq + 8 * k + e]) * qv[e]) + v[8 * k + e];
                 }
             }
             umma::fence_before_sync();
             __syncthreads();  // every use of the chunk-start scales is done
 
-
             // ---- requantize: column scales (impact-weighted RMS), row scales, codes -----------
             {
                 float *red = smf(big, BIG_RED), *rmax = smf(big, BIG_RMAX);
                 const float wi = sW[i];
-                float e[64];
+                float e2[32];
 #pragma unroll
-                for (int j = 0; j < 64; ++j) e[j] = wi * S[j] * S[j];
-                warp_reduce_scatter64(e);
-                *reinterpret_cast<float2 *>(red + q4 * D + 64 * ch + 2 * lane) = make_float2(e[0], e[1]);
+                for (int j = 0; j < 32; ++j) e2[j] = wi * S[j] * S[j];
+                red[q4 * D + 32 * cq + lane] = warp_reduce_scatter32(e2);
                 __syncthreads();
                 if (tid < D) {
                     const float E = (red[tid] + red[D + tid]) + (red[2 * D + tid] + red[3 * D + tid]);
@@ -712,40 +723,40 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                 __syncthreads();
                 float m = 0.f;
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    S[j] = S[j] * red[64 * ch + j];
+                for (int j = 0; j < 32; ++j) {
+                    S[j] = S[j] * red[32 * cq + j];
                     m = fmaxf(m, fabsf(S[j]));
                 }
-                rmax[ch * D + i] = m;
+                rmax[cq * D + i] = m;
                 __syncthreads();
-                m = fmaxf(rmax[i], rmax[D + i]);
+                m = fmaxf(fmaxf(rmax[i], rmax[D + i]), fmaxf(rmax[2 * D + i], rmax[3 * D + i]));
                 float ri = m / (float)P::QMAX;
                 if (ri == 0.f) ri = 1.f;
                 bad |= !isfinite(ri);
                 const float rri = __frcp_rn(ri);
-                int qc[64];
+                int qc[32];
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
+                for (int j = 0; j < 32; ++j) {
                     float x = rintf(S[j] * rri);
                     x = fminf(fmaxf(x, -(float)P::QMAX), (float)P::QMAX);
                     qc[j] = (int)x;
                 }
-                // next chunk's B operand (row i, atom column ch) and scales
-                uint8_t *qrow = sm + OFF_QC + ch * 16384;
+                // next chunk's B operand (row i, columns 32 cq ..) and scales
+                uint8_t *qrow = sm + OFF_QC + (cq >> 1) * 16384;
 #pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
+                for (int k = 0; k < 4; ++k) {
                     uint32_t w4[4];
 #pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2)
-                        w4[e2] = umma::pack_bf16(__float2bfloat16_rn((float)qc[8 * c8 + 2 * e2]),
-                                                 __float2bfloat16_rn((float)qc[8 * c8 + 2 * e2 + 1]));
-                    *reinterpret_cast<uint4 *>(qrow + sw128_chunk(i, c8)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    for (int e = 0; e < 4; ++e)
+                        w4[e] = bf2_bits(__floats2bfloat162_rn((float)qc[8 * k + 2 * e], (float)qc[8 * k + 2 * e + 1]));
+                    *reinterpret_cast<uint4 *>(qrow + sw128_chunk(i, 4 * (cq & 1) + k)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
-                if (ch == 0) sR[i] = ri;
+                if (cq == 0) sR[i] = ri;
                 if (c + 1 == nch) {  // the last chunk of the call: the state goes back to HBM
-                    store_codes_row<BITS>(gblock, i, ch, qc);
+                    store_codes_row<BITS>(gblock, i, cq, qc);
                     float *gsc = reinterpret_cast<float *>(gblock + P::SOFF);
-                    if (ch == 0) gsc[i] = ri;
+                    if (cq == 0) gsc[i] = ri;
                     if (tid < D) gsc[D + tid] = sC[tid];
                 }
             }
