@@ -240,6 +240,59 @@ def oracle_workers():
 # GPU arm
 # ------------------------------------------------------------------------------------------------
 
+def prefill_leg(dev, steps: int = 3, warmup: int = 1) -> dict:
+    """The chunked-prefill workload (16 requests x 16 heads, 6-bit, an 8192-token prompt in 64-token
+    chunks, bf16 inputs) timed as whole stq_prefill_chunk calls, inputs resident in HBM."""
+    import torch
+
+    import quantized_linear_attention_stq_b200 as stq
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl = wlm.WORKLOADS["prefill16_b16_6bit"]
+    B, H, d, T, C = wl.batch, wl.heads, wl.d, 8192, 64
+    bits = wlm.head_bits(wl)
+    lay = stq.Layout(bits, d, gate=wl.gate, in_dtype=wl.in_dtype)
+    pool = lay.alloc_pool(B, dev)
+    slots = torch.arange(B, dtype=torch.int32, device=dev)
+    w = wlm.impact_weights(wl, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stq.init_state(lay, pool, slots, torch.stack([wlm.initial_state(wl, r, dev) for r in range(B)]), w,
+                   status=status)
+    inp = wlm.prefill_inputs(wl, 0, T, dev)
+    o = torch.empty(B, H, T, d, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, stq.prefill_workspace_bytes(lay, B, T, C)), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call():
+        stq.prefill_chunk(lay, pool, slots, inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], w, o, chunk=C,
+                          workspace=ws, status=status, stream=stream)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for k in range(steps):
+        call()
+        ev[k + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    if status.item() != 0:
+        raise RuntimeError(f"device status after prefill: {stq.status_flags(status)}")
+    ms = ev[0].elapsed_time(ev[-1]) / steps
+    in_bytes = B * H * T * (3 * d * 2 + 8)  # q, k, v bf16 + beta, alpha
+    out_bytes = B * H * T * d * 4             # o fp32
+    state_bytes = 2 * B * sum(lay.head_bytes(h) for h in range(H))  # read at the start, written at the end
+    nbytes = in_bytes + out_bytes + state_bytes
+    peak, kind = measured_peaks()
+    achieved = nbytes / (ms / 1e3) / 1e9
+    del inp, o, pool
+    return {"workload": "prefill16_b16_6bit", "prompt_tokens": T, "chunk": C, "requests": B, "heads": H,
+            "ms_per_call": ms, "head_tokens_per_s": B * H * T / (ms / 1e3), "tokens_per_s": B * T / (ms / 1e3),
+            "calls": steps, "kernel": "prefill_wy_kernel<6> (tcgen05, one launch)",
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "peak_kind": kind, "bytes_per_call": nbytes}}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -384,6 +437,8 @@ def run_ours(args):
         "clocks": clocks.summary(t_wall0, t_wall1),
         "gpu": torch.cuda.get_device_name(dev),
     }
+    if world == 1 and not args.no_prefill:
+        result["prefill"] = prefill_leg(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, sample = time_oracle(args.workload, oracle_workers(), 16, 20)
         result["cpu_baseline"] = {"value": rate, "unit": "head-steps/s", "cores": cores, "kind": "oracle",
@@ -434,6 +489,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the chunked-prefill leg")
     ap.add_argument("--batch", type=int, default=0, help="requests per GPU (default: the workload's)")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -115,3 +115,88 @@ def test_multi_chunk_equals_single_chunk_calls(stq, orc):
     torch.cuda.synchronize()
     assert torch.equal(p_full, p_seq)
     assert torch.equal(o_full, torch.cat(outs, dim=2))
+
+
+def test_full_geometry_chunk_chain_and_sampled_first_chunk(stq, orc):
+    """The 16-request x 16-head, 6-bit prefill workload in its bench launch shape (all tiles in
+    one launch, more tiles than SMs), over 4 chunks: the multi-chunk call equals the chain of
+    single-chunk calls bit for bit, and sampled tiles match the oracle on the first chunk."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl = wlm.WORKLOADS["prefill16_b16_6bit"]
+    B, H, d, T, C = wl.batch, wl.heads, wl.d, 256, 64
+    bits = wlm.head_bits(wl)
+    lay = stq.Layout(bits, d, in_dtype=wl.in_dtype)
+    w = wlm.impact_weights(wl)
+    blocks = []
+    for r in range(B):
+        S0 = wlm.initial_state(wl, r)
+        blocks.append([orc.quantize(bits[h], as_f64(S0[h]), as_f64(w[h]))[0] for h in range(H)])
+    opool = oracle_pool(orc, bits, d, blocks)
+    inp = {n: x.to(DEV) for n, x in wlm.prefill_inputs(wl, 0, T).items()}
+    slots = torch.arange(B, dtype=torch.int32, device=DEV)
+    wd = w.to(DEV)
+    ws = torch.empty(1, dtype=torch.uint8, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    p_full = torch.from_numpy(opool.copy()).to(DEV)
+    o_full = torch.zeros(B, H, T, d, device=DEV)
+    stq.prefill_chunk(lay, p_full, slots, inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], wd, o_full,
+                      chunk=C, workspace=ws, status=status)
+    p_seq = torch.from_numpy(opool.copy()).to(DEV)
+    outs = []
+    first_pool = None
+    for c0 in range(0, T, C):
+        part = {n: x[:, :, c0:c0 + C].contiguous() for n, x in inp.items()}
+        o_part = torch.zeros(B, H, C, d, device=DEV)
+        stq.prefill_chunk(lay, p_seq, slots, part["q"], part["k"], part["v"], part["beta"], part["alpha"], wd,
+                          o_part, chunk=C, workspace=ws, status=status)
+        outs.append(o_part)
+        if first_pool is None:
+            torch.cuda.synchronize()
+            first_pool = p_seq.cpu().numpy()
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.equal(p_full, p_seq)
+    assert torch.equal(o_full, torch.cat(outs, dim=2))
+    # teacher-forced first chunk of sampled tiles
+    cpu_inp = {n: x[:, :, :C].cpu() for n, x in inp.items()}
+    o0 = outs[0].cpu().numpy()
+    tally = Tally(updates_per_check=C)
+    rng = np.random.default_rng(5)
+    for r, h in zip(rng.integers(0, B, 6), rng.integers(0, H, 6)):
+        res = _oracle_chunk(orc, opool, bits, d, int(r), int(h), cpu_inp, 0, C, w, C)
+        assert res["status"] == orc.OK
+        compare_block(orc, bits[h], d, tile_bytes(orc, first_pool, bits, d, int(r), int(h)), res["block"],
+                      res["tie"], tally, f"req {r} head {h}")
+        for t in range(C):
+            compare_o(o0[r, h, t], res["o"][t], tally, f"token {t} req {r} head {h}")
+    tally.check_budget()
+
+
+def test_fp32_inputs_sequential_form(stq, orc):
+    """fp32 inputs (the sequential kernel) on a short single chunk, teacher forced."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    bits = [6, 4]
+    B, d, T = 2, 128, 23
+    wl_, w, opool = _setup(orc, B, bits, dtype=torch.float32)
+    lay = stq.Layout(bits, d, in_dtype=torch.float32)
+    inp = wlm.prefill_inputs(wl_, 0, T)
+    gpool = torch.from_numpy(opool.copy()).to(DEV)
+    slots = torch.arange(B, dtype=torch.int32, device=DEV)
+    o = torch.zeros(B, len(bits), T, d, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stq.prefill_chunk(lay, gpool, slots, *(inp[n].to(DEV) for n in ("q", "k", "v", "beta", "alpha")), w.to(DEV), o,
+                      chunk=64, workspace=torch.empty(1, dtype=torch.uint8, device=DEV), status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    gp, og = gpool.cpu().numpy(), o.cpu().numpy()
+    tally = Tally(updates_per_check=T)
+    for r in range(B):
+        for h in range(len(bits)):
+            res = _oracle_chunk(orc, opool, bits, d, r, h, inp, 0, T, w, 64)
+            compare_block(orc, bits[h], d, tile_bytes(orc, gp, bits, d, r, h), res["block"], res["tie"], tally,
+                          f"req {r} head {h}")
+            for t in range(T):
+                compare_o(og[r, h, t], res["o"][t], tally, f"token {t} req {r} head {h}")
+    tally.check_budget()
