@@ -240,7 +240,7 @@ def oracle_workers():
 # GPU arm
 # ------------------------------------------------------------------------------------------------
 
-def prefill_leg(dev, steps: int = 3, warmup: int = 1) -> dict:
+def prefill_leg(dev, steps: int = 3, warmup: int = 1, T: int = 8192) -> dict:
     """The chunked-prefill workload (16 requests x 16 heads, 6-bit, an 8192-token prompt in 64-token
     chunks, bf16 inputs) timed as whole stq_prefill_chunk calls, inputs resident in HBM."""
     import torch
@@ -249,7 +249,7 @@ def prefill_leg(dev, steps: int = 3, warmup: int = 1) -> dict:
     from quantized_linear_attention_stq_b200 import workloads as wlm
 
     wl = wlm.WORKLOADS["prefill16_b16_6bit"]
-    B, H, d, T, C = wl.batch, wl.heads, wl.d, 8192, 64
+    B, H, d, C = wl.batch, wl.heads, wl.d, 64
     bits = wlm.head_bits(wl)
     lay = stq.Layout(bits, d, gate=wl.gate, in_dtype=wl.in_dtype)
     pool = lay.alloc_pool(B, dev)
@@ -438,7 +438,7 @@ def run_ours(args):
         "gpu": torch.cuda.get_device_name(dev),
     }
     if world == 1 and not args.no_prefill:
-        result["prefill"] = prefill_leg(dev)
+        result["prefill"] = prefill_leg(dev, T=args.prefill_tokens)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, sample = time_oracle(args.workload, oracle_workers(), 16, 20)
         result["cpu_baseline"] = {"value": rate, "unit": "head-steps/s", "cores": cores, "kind": "oracle",
@@ -490,12 +490,20 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the chunked-prefill leg")
+    ap.add_argument("--prefill-only", action="store_true", help="run only the chunked-prefill leg (profiling)")
+    ap.add_argument("--prefill-tokens", type=int, default=8192, help="prompt length of the prefill leg")
     ap.add_argument("--batch", type=int, default=0, help="requests per GPU (default: the workload's)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.prefill_only:
+        import torch
+
+        dev = torch.device("cuda", torch.cuda.current_device())
+        print(json.dumps({"prefill": prefill_leg(dev, steps=args.steps, warmup=args.warmup, T=args.prefill_tokens)}),
+              flush=True)
     else:
         run_ours(args)
 
