@@ -74,10 +74,10 @@ constexpr uint32_t BIG_P0 = 49152, BIG_P1 = 57344;                        // P t
 constexpr uint32_t BIG_U0 = 0, BIG_U1 = 16384;                            // U terms
 constexpr uint32_t BIG_Y0 = 32768, BIG_Y1 = 65536, BIG_Y2 = 81920;        // decayed U terms
 // requantization scratch in BIG (after the last MMA of the chunk has completed)
-constexpr uint32_t BIG_RED = 0;      // [4][128] f32 column-energy partials (per lane quarter)
-constexpr uint32_t BIG_RMAX = 2048;  // [4][128] f32 row-max partials (per column quarter)
-// T-inverse scratch in the RT area (before the T terms are written)
-constexpr uint32_t RT_G = 0;         // [3][16][17] f32
+constexpr int LDSQ = 132;                     // row stride (floats) of the weighted squares
+constexpr uint32_t BIG_SQ = 0;                // [128][LDSQ] f32 w_i S_ij^2
+constexpr uint32_t BIG_RED = 128 * LDSQ * 4;  // [4][128] f32 column-energy partials (per row quarter)
+constexpr uint32_t BIG_RMAX = BIG_RED + 2048; // [4][128] f32 row-max partials (per column quarter)
 
 // Tensor Memory columns
 constexpr uint32_t TM_D1 = 0, TM_D3 = 0, TM_D2 = 128, TM_DU = 256, TM_DP = 384;
@@ -250,92 +250,61 @@ __device__ __forceinline__ void bf16x8_to_f32(uint4 raw, float (&x)[8])
     }
 }
 
-// ---------------------------------------------------------------------------------------------
-// T = (I + L)^-1 for a strictly lower triangular 64 x 64 L (fp32, row stride LDL), by 16 x 16
-// blocks: the four diagonal blocks by forward substitution (one warp each), then the off-diagonal
-// blocks T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj in order of distance i - j. G: [3][16][17]
-// scratch. All threads call it; it ends with a barrier.
-// ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ void invert_unit_lower(const float *L, float *T, float *G)
+constexpr int INV_WARP0 = 12;  // warps 12..15 form T while warps 0..11 build the D2 operand
+constexpr int MMA_TID = 64;    // issues every MMA group (lane quarter 2: it loads no v rows)
+
+__device__ __forceinline__ void named_bar(int id, int count)
 {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (warp < 4 && lane < 16) {
-        const int b0 = 16 * warp, c = lane;
-        float x[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) x[t] = (t == c) ? 1.f : 0.f;
-#pragma unroll
-        for (int s = 0; s < 15; ++s) {
-            const float xs = x[s];
-#pragma unroll
-            for (int t = s + 1; t < 16; ++t) x[t] = fmaf(-L[(b0 + t) * LDL + b0 + s], xs, x[t]);
-        }
-#pragma unroll
-        for (int t = 0; t < 16; ++t) T[(b0 + t) * LDL + b0 + c] = x[t];
-    } else if (warp >= 4) {
-        // zero the strictly upper blocks (T is an MMA operand in full)
-        for (int e = tid - 128; e < 64 * 64; e += NT - 128) {
-            const int t = e >> 6, s = e & 63;
-            if ((s >> 4) > (t >> 4)) T[t * LDL + s] = 0.f;
-        }
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int d = 1; d < 4; ++d) {
-        const int nblk = 4 - d;
-        // G_j = sum_{k=j}^{j+d-1} L_{j+d,k} T_kj, one element per thread and block
-        for (int e = tid; e < 256 * nblk; e += NT) {
-            const int j = e >> 8, r = (e >> 4) & 15, c = e & 15, i = j + d;
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-            for (int k = j; k < i; ++k) {
-                const float *Lr = L + (16 * i + r) * LDL + 16 * k;
-                const float *Tc = T + (16 * k) * LDL + 16 * j + c;
-#pragma unroll
-                for (int u = 0; u < 16; u += 4) {
-                    const float4 l4 = *reinterpret_cast<const float4 *>(Lr + u);
-                    a0 = fmaf(l4.x, Tc[u * LDL], a0);
-                    a1 = fmaf(l4.y, Tc[(u + 1) * LDL], a1);
-                    a2 = fmaf(l4.z, Tc[(u + 2) * LDL], a2);
-                    a3 = fmaf(l4.w, Tc[(u + 3) * LDL], a3);
-                }
-            }
-            G[j * 272 + r * 17 + c] = (a0 + a1) + (a2 + a3);
-        }
-        __syncthreads();
-        for (int e = tid; e < 256 * nblk; e += NT) {
-            const int j = e >> 8, r = (e >> 4) & 15, c = e & 15, i = j + d;
-            const float *Tr = T + (16 * i + r) * LDL + 16 * i;
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-            for (int u = 0; u < 16; u += 4) {
-                const float4 t4 = *reinterpret_cast<const float4 *>(Tr + u);
-                a0 = fmaf(t4.x, G[j * 272 + u * 17 + c], a0);
-                a1 = fmaf(t4.y, G[j * 272 + (u + 1) * 17 + c], a1);
-                a2 = fmaf(t4.z, G[j * 272 + (u + 2) * 17 + c], a2);
-                a3 = fmaf(t4.w, G[j * 272 + (u + 3) * 17 + c], a3);
-            }
-            T[(16 * i + r) * LDL + 16 * j + c] = -((a0 + a1) + (a2 + a3));
-        }
-        __syncthreads();
-    }
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// Warp reduce-scatter of 32 per-lane values: afterwards v[0] of lane l is the warp sum of entry l.
-__device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32])
+// ---------------------------------------------------------------------------------------------
+// T = (I + L)^-1 for a strictly lower triangular 64 x 64 L given transposed (Lt[s][t] = L_ts, row
+// stride LDL), by right-looking forward substitution on the 64 columns of the identity, run by the
+// 128 threads of warps 12..15. Thread (warp wi, lane: column group g = lane / 8, row group q = lane
+// % 8) keeps rows 8q .. 8q+7 of columns c0 .. c0+3, c0 = 16 wi + 4 g; step s takes the final x_s of
+// each column from its owner by a shuffle and updates every row below it. The result goes to T.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void invert_unit_lower(const float *Lt, float *T)
 {
-    const int lane = threadIdx.x & 31;
+    const int wi = (threadIdx.x >> 5) - INV_WARP0, lane = threadIdx.x & 31;
+    const int g = lane >> 3, q = lane & 7, base = lane & ~7, c0 = 16 * wi + 4 * g;
+    float2 x[4][4];  // [column][row pair]
 #pragma unroll
-    for (int step = 0; step < 5; ++step) {
-        const int o = 16 >> step, hn = 16 >> step;
-        const bool up = (lane & o) != 0;
+    for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
-        for (int k = 0; k < hn; ++k) {
-            const float keep = up ? v[k + hn] : v[k];
-            const float send = up ? v[k] : v[k + hn];
-            v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        for (int k = 0; k < 4; ++k)
+            x[cc][k] = make_float2((8 * q + 2 * k == c0 + cc) ? 1.f : 0.f, (8 * q + 2 * k + 1 == c0 + cc) ? 1.f : 0.f);
+    // x_s = 0 for s < c0: the steps before the warp's first column change nothing
+#pragma unroll 1
+    for (int sb = 2 * wi; sb < 8; ++sb) {
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int s = 8 * sb + m;
+            const float4 l0 = *reinterpret_cast<const float4 *>(Lt + s * LDL + 8 * q);
+            const float4 l1 = *reinterpret_cast<const float4 *>(Lt + s * LDL + 8 * q + 4);
+            const float2 la = make_float2(l0.x, l0.y), lb = make_float2(l0.z, l0.w);
+            const float2 lc = make_float2(l1.x, l1.y), ld = make_float2(l1.z, l1.w);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                const float own = (m & 1) ? x[cc][m >> 1].y : x[cc][m >> 1].x;
+                const float xs = -__shfl_sync(0xffffffffu, own, base | sb);
+                const float2 nx = make_float2(xs, xs);
+                x[cc][0] = __ffma2_rn(la, nx, x[cc][0]);
+                x[cc][1] = __ffma2_rn(lb, nx, x[cc][1]);
+                x[cc][2] = __ffma2_rn(lc, nx, x[cc][2]);
+                x[cc][3] = __ffma2_rn(ld, nx, x[cc][3]);
+            }
         }
     }
-    return v[0];
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            T[(8 * q + 2 * k) * LDL + c0 + cc] = x[cc][k].x;
+            T[(8 * q + 2 * k + 1) * LDL + c0 + cc] = x[cc][k].y;
+        }
+    named_bar(2, 128);
 }
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int32_t *status)
@@ -368,7 +337,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
 {
     using P = PCfg<BITS>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base, derived from the shared array so that accesses stay shared-space
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, cq = warp >> 2;
     float *sR = smf(sm, OFF_SMALL + S_R), *sC = smf(sm, OFF_SMALL + S_C), *sW = smf(sm, OFF_SMALL + S_W);
     double *sLG = smd(sm, OFF_SMALL + S_LG), *sG = smd(sm, OFF_SMALL + S_G);
@@ -451,7 +421,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
             __syncthreads();
 
             // ---- D1 = [K;Q] K^T (M 128, N 64) ------------------------------------------
-            if (tid == 0) {
+            if (tid == MMA_TID) {
                 umma::fence_after_sync();
                 const uint32_t base = smem_u32(sm + kq);
                 const uint32_t id = umma::idesc_bf16(128, 64, 0, 0);
@@ -473,44 +443,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                 }
                 sLG[tid] = g;  // within-warp inclusive prefix
             }
-            // ---- A operand of D2: three bf16 terms of [K r; Q r] (row m, columns 32 part ..) -
-            {
-                const int m = tid >> 2, part = tid & 3, row = m & 63, hb = part >> 1;
-                const uint8_t *xb = sm + kq + (m < 64 ? (hb ? KQ_K1 : KQ_K0) : (hb ? KQ_Q1 : KQ_Q0));
-                uint8_t *a0 = big + hb * 16384, *a1 = a0 + 32768, *a2 = a0 + 65536;
-                const float *rr = sR + 32 * part;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int c8 = 4 * (part & 1) + k;
-                    float x[8];
-                    bf16x8_to_f32(*reinterpret_cast<const uint4 *>(xb + sw128_chunk(row, c8)), x);
-                    const float4 ra = *reinterpret_cast<const float4 *>(rr + 8 * k);
-                    const float4 rb = *reinterpret_cast<const float4 *>(rr + 8 * k + 4);
-                    x[0] *= ra.x; x[1] *= ra.y; x[2] *= ra.z; x[3] *= ra.w;
-                    x[4] *= rb.x; x[5] *= rb.y; x[6] *= rb.z; x[7] *= rb.w;
-                    store_split3(a0, a1, a2, sw128_chunk(m, c8), x);
-                }
-            }
-            umma::fence_proxy_async();
             __syncthreads();
-            if (tid == 0) {
-                const uint32_t abase = smem_u32(big), bbase = smem_u32(sm + OFF_QC);
-                const uint32_t id = umma::idesc_bf16(128, 128, 0, 1);
-#pragma unroll 1
-                for (int term = 0; term < 3; ++term)
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma::mma_bf16(tmem + TM_D2,
-                                       umma::smem_desc(abase + term * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                       umma::smem_desc(bbase + kk * 2048, 16384, 1024), id, (term | kk) != 0);
-                umma::mma_commit(smem_u32(&bars[1]));
-            }
-            // finish the prefix across the two warps, then the decay factors
-            if (tid < C) {
-                double g = sLG[tid];
-                if (tid >= 32) g += sLG[31];
-                sG[tid] = g;
-            }
+            if (tid < C) sG[tid] = sLG[tid] + (tid >= 32 ? sLG[31] : 0.0);
             __syncthreads();
             if (tid < C) {
                 const double gl = sG[C - 1], g = sG[tid];
@@ -519,7 +453,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                 if (tid == 0) miscf[1] = (float)exp(gl);
             }
 
-            // ---- L (lane quarters 0, 1) and P (quarters 2, 3) from D1, columns 16 cq .. ---
+            // ---- L (lane quarters 0, 1; stored transposed) and P (quarters 2, 3) from D1 ----
             ok = wait_bar(smem_u32(&bars[0]), parity, p.status);
             if (!__syncthreads_and(ok)) break;
             umma::fence_after_sync();
@@ -534,7 +468,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
 #pragma unroll
                     for (int u = 0; u < 16; ++u) {
                         const int s = 16 * cq + u;
-                        Lm[t * LDL + s] = s < t ? bt * expf((float)(gt - sG[s])) * v[u] : 0.f;
+                        Lm[s * LDL + t] = s < t ? bt * expf((float)(gt - sG[s])) * v[u] : 0.f;
                     }
                 } else {
 #pragma unroll
@@ -544,18 +478,58 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                     }
                 }
             }
+            umma::fence_before_sync();
             __syncthreads();
-            invert_unit_lower(Lm, Tm, smf(sm, OFF_RT + RT_G));
-            // T in three bf16 terms (K-major, rows t, contraction s), one chunk per thread
-            {
-                const int t = tid >> 3, c8 = tid & 7;
+
+            if (warp < INV_WARP0) {
+                // ---- warps 0..11: A operand of D2, three bf16 terms of [K r; Q r] ------------
+                for (int unit = tid; unit < 4 * D; unit += 32 * INV_WARP0) {
+                    const int m = unit >> 2, part = unit & 3, row = m & 63, hb = part >> 1;
+                    const uint8_t *xb = sm + kq + (m < 64 ? (hb ? KQ_K1 : KQ_K0) : (hb ? KQ_Q1 : KQ_Q0));
+                    uint8_t *a0 = big + hb * 16384, *a1 = a0 + 32768, *a2 = a0 + 65536;
+                    const float *rr = sR + 32 * part;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int c8 = 4 * (part & 1) + k;
+                        float x[8];
+                        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(xb + sw128_chunk(row, c8)), x);
+                        const float4 ra = *reinterpret_cast<const float4 *>(rr + 8 * k);
+                        const float4 rb = *reinterpret_cast<const float4 *>(rr + 8 * k + 4);
+                        x[0] *= ra.x; x[1] *= ra.y; x[2] *= ra.z; x[3] *= ra.w;
+                        x[4] *= rb.x; x[5] *= rb.y; x[6] *= rb.z; x[7] *= rb.w;
+                        store_split3(a0, a1, a2, sw128_chunk(m, c8), x);
+                    }
+                }
+                umma::fence_proxy_async();
+                named_bar(1, 32 * INV_WARP0);
+                if (tid == MMA_TID) {
+                    umma::fence_after_sync();
+                    const uint32_t abase = smem_u32(big), bbase = smem_u32(sm + OFF_QC);
+                    const uint32_t id = umma::idesc_bf16(128, 128, 0, 1);
+#pragma unroll 1
+                    for (int term = 0; term < 3; ++term)
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            umma::mma_bf16(tmem + TM_D2,
+                                           umma::smem_desc(abase + term * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16,
+                                                           1024),
+                                           umma::smem_desc(bbase + kk * 2048, 16384, 1024), id, (term | kk) != 0);
+                    umma::mma_commit(smem_u32(&bars[1]));
+                }
+            } else {
+                // ---- warps 12..15: T = (I + L)^-1, then its three bf16 terms -----------------
+                invert_unit_lower(Lm, Tm);
                 uint8_t *r0 = sm + OFF_RT;
-                float x[8];
-                const float4 xa = *reinterpret_cast<const float4 *>(Tm + t * LDL + 8 * c8);
-                const float4 xb4 = *reinterpret_cast<const float4 *>(Tm + t * LDL + 8 * c8 + 4);
-                x[0] = xa.x; x[1] = xa.y; x[2] = xa.z; x[3] = xa.w;
-                x[4] = xb4.x; x[5] = xb4.y; x[6] = xb4.z; x[7] = xb4.w;
-                store_split3(r0, r0 + 8192, r0 + 16384, sw128_chunk(t, c8), x);
+                for (int unit = tid - 32 * INV_WARP0; unit < 64 * 8; unit += 128) {
+                    const int t = unit >> 3, c8 = unit & 7;
+                    float x[8];
+                    const float4 xa = *reinterpret_cast<const float4 *>(Tm + t * LDL + 8 * c8);
+                    const float4 xb4 = *reinterpret_cast<const float4 *>(Tm + t * LDL + 8 * c8 + 4);
+                    x[0] = xa.x; x[1] = xa.y; x[2] = xa.z; x[3] = xa.w;
+                    x[4] = xb4.x; x[5] = xb4.y; x[6] = xb4.z; x[7] = xb4.w;
+                    store_split3(r0, r0 + 8192, r0 + 16384, sw128_chunk(t, c8), x);
+                }
+                umma::fence_proxy_async();
             }
             __syncthreads();  // L / T are dead: the area takes the next chunk's K / Q
             if (c + 1 < nch) {
@@ -594,7 +568,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
             umma::fence_proxy_async();
             __syncthreads();
             // ---- DU = T R' (rows 64..127 of an M 128 instruction) ---------------------------
-            if (tid == 0) {
+            if (tid == MMA_TID) {
+                umma::fence_after_sync();
                 const uint32_t ta = smem_u32(sm + OFF_RT) - 8192, rb = smem_u32(big);
                 const uint32_t id = umma::idesc_bf16(128, 128, 0, 1);
                 constexpr int A_T[6] = {0, 0, 1, 0, 1, 2}, B_T[6] = {0, 1, 0, 2, 1, 0};
@@ -634,7 +609,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
             umma::fence_before_sync();
             __syncthreads();
             // ---- DP = P U (rows 64..127) and D3 = K^T (decayed U) ----------------------------
-            if (tid == 0) {
+            if (tid == MMA_TID) {
                 umma::fence_after_sync();
                 const uint32_t bb = smem_u32(big);
                 const uint32_t id = umma::idesc_bf16(128, 128, 0, 1);
@@ -705,12 +680,31 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
 
             // ---- requantize: column scales (impact-weighted RMS), row scales, codes -----------
             {
-                float *red = smf(big, BIG_RED), *rmax = smf(big, BIG_RMAX);
+                float *red = smf(big, BIG_RED), *rmax = smf(big, BIG_RMAX), *sq = smf(big, BIG_SQ);
                 const float wi = sW[i];
-                float e2[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) e2[j] = wi * S[j] * S[j];
-                red[q4 * D + 32 * cq + lane] = warp_reduce_scatter32(e2);
+                for (int k = 0; k < 8; ++k) {
+                    float4 e4;
+                    e4.x = wi * S[4 * k] * S[4 * k];
+                    e4.y = wi * S[4 * k + 1] * S[4 * k + 1];
+                    e4.z = wi * S[4 * k + 2] * S[4 * k + 2];
+                    e4.w = wi * S[4 * k + 3] * S[4 * k + 3];
+                    *reinterpret_cast<float4 *>(sq + i * LDSQ + 32 * cq + 4 * k) = e4;
+                }
+                __syncthreads();
+                {
+                    // column j = tid % 128 summed over the 32 rows of quarter tid / 128
+                    const int j = tid & (D - 1), r0 = 32 * (tid >> 7);
+                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+                    for (int r = 0; r < 32; r += 4) {
+                        a0 += sq[(r0 + r) * LDSQ + j];
+                        a1 += sq[(r0 + r + 1) * LDSQ + j];
+                        a2 += sq[(r0 + r + 2) * LDSQ + j];
+                        a3 += sq[(r0 + r + 3) * LDSQ + j];
+                    }
+                    red[(tid >> 7) * D + j] = (a0 + a1) + (a2 + a3);
+                }
                 __syncthreads();
                 if (tid < D) {
                     const float E = (red[tid] + red[D + tid]) + (red[2 * D + tid] + red[3 * D + tid]);
