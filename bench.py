@@ -110,6 +110,28 @@ def profiled_traffic():
         return None
 
 
+# fp32 lane operations on the FMA pipe that one state element needs in this formulation of the
+# decode step: code unpack 1, the k and q column sums 2, the update 2, the column energy 1, the
+# column rescale 1, the rounding 1 (FP16 pivots: column sums 2, update 2)
+FMA_OPS_PER_ELEMENT = {4: 8, 6: 8, 8: 8, 16: 4}
+FP32_LANES_PER_SM = 128
+
+
+def clocks_sm_mhz(summary) -> float:
+    v = summary.get("sm_mhz") if isinstance(summary, dict) else None
+    return float(v) if v else 1965.0
+
+
+def alu_roofline(bits, B: int, step_s: float, sm_mhz: float) -> dict:
+    """The FMA-pipe co-bound of the decode step: algorithmic fp32 lane operations per step over
+    the step time, against 148 SMs x 128 fp32 lanes x the SM clock sampled during the run."""
+    ops = sum(FMA_OPS_PER_ELEMENT[b] for b in bits) * 128 * 128 * B
+    peak = 148 * FP32_LANES_PER_SM * sm_mhz * 1e6 / 1e12
+    achieved = ops / step_s / 1e12
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tlane-op/s", "frac": achieved / peak,
+            "ops_per_step": ops, "note": "fp32 lane operations on the FMA pipe; peak = 148 SMs x 128 lanes x clock"}
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle sampling around the timed region."""
 
@@ -240,6 +262,47 @@ def oracle_workers():
 # GPU arm
 # ------------------------------------------------------------------------------------------------
 
+def per_layer_graph_leg(stq, lay, pool, slots, toks, w, status, dev, steps: int, warmup: int, heads_per_layer: int = 48):
+    """The serving shape of a decode token: one stq_decode_step per layer (48 heads each), all
+    layers of a token captured in one CUDA graph and replayed; inputs resident in HBM."""
+    import torch
+
+    B, H, d = toks[0]["q"].shape
+    L = H // heads_per_layer
+
+    def part(x, lo):
+        return x[:, lo:lo + heads_per_layer].contiguous()
+
+    per_tok = [[{n: part(x[n], heads_per_layer * l) for n in x} for l in range(L)] for x in toks]
+    w_l = [w[heads_per_layer * l:heads_per_layer * (l + 1)].contiguous() for l in range(L)]
+    o_l = [torch.empty(B, heads_per_layer, d, dtype=torch.float32, device=dev) for _ in range(L)]
+    graphs = []
+    cap = torch.cuda.Stream(dev)
+    for t in range(len(toks)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            for l in range(L):
+                x = per_tok[t][l]
+                stq.decode_step(lay, pool, slots, x["q"], x["k"], x["v"], x["beta"], x["alpha"], w_l[l], o_l[l],
+                                head_begin=heads_per_layer * l, status=status)
+        graphs.append(g)
+    stream = torch.cuda.current_stream(dev)
+    for t in range(warmup):
+        graphs[t % len(graphs)].replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for t in range(steps):
+        graphs[t % len(graphs)].replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    del graphs, per_tok
+    return {"layers": L, "heads_per_layer": heads_per_layer, "ms_per_token": ms,
+            "head_steps_per_s": B * H / (ms / 1e3), "steps": steps,
+            "note": "one stq_decode_step per layer, a token's layers captured in one CUDA graph"}
+
+
 def prefill_leg(dev, steps: int = 3, warmup: int = 1, T: int = 8192) -> dict:
     """The chunked-prefill workload (16 requests x 16 heads, 6-bit, an 8192-token prompt in 64-token
     chunks, bf16 inputs) timed as whole stq_prefill_chunk calls, inputs resident in HBM."""
@@ -334,6 +397,10 @@ def run_ours(args):
     toks = [wlm.decode_inputs(wl, 1000 * rank + t, dev) for t in range(TOKENS_CYCLED)]
     o = torch.empty(B, H, d, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    # the workload is a generation of wl.steps tokens; longer runs restart it from the initial
+    # pool (a device copy between generations, outside the per-step timings)
+    pristine = pool.clone()
+    gen = max(1, wl.steps)
     torch.cuda.synchronize(dev)
 
     def step(t):
@@ -346,31 +413,43 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     if status.item() != 0:
         raise RuntimeError(f"device status after warm-up: {stq.status_flags(status)}")
+    pool.copy_(pristine)
 
     clocks = ClockSampler(dev.index)
     clocks.start()
     time.sleep(0.3)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier(dev)
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
-    ev[0].record(stream)
     for t in range(args.steps):
-        step(args.warmup + t)
-        ev[t + 1].record(stream)
+        if t > 0 and t % gen == 0:
+            pool.copy_(pristine, non_blocking=True)
+        ev0[t].record(stream)
+        step(t)
+        ev1[t].record(stream)
     torch.cuda.synchronize(dev)
     t_wall1 = time.time()
     barrier(dev)
     time.sleep(0.3)
     clocks.stop()
-    total_ms = ev[0].elapsed_time(ev[-1])
-    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    per_step = [ev0[i].elapsed_time(ev1[i]) for i in range(args.steps)]
+    total_ms = sum(per_step)
     total_ms_max = reduce_max(total_ms, dev)
     if status.item() != 0:
         raise RuntimeError(f"device status after timing: {stq.status_flags(status)}")
 
+    graph_leg = None
+    if world == 1 and H % 48 == 0 and args.workload == DEFAULT_WORKLOAD:
+        pool.copy_(pristine)
+        graph_leg = per_layer_graph_leg(stq, lay, pool, slots, toks, w, status, dev, min(args.steps, gen), 5)
+        if status.item() != 0:
+            raise RuntimeError(f"device status after the per-layer graph leg: {stq.status_flags(status)}")
+    pool.copy_(pristine)
+
     # end to end through the public API with host buffers: H2D inputs, step, D2H readout
-    e2e_steps = max(1, min(args.steps, 50))
+    e2e_steps = max(1, min(args.steps, 50, gen))
     host_in = [{n: x.cpu().pin_memory() for n, x in toks[t].items()} for t in range(min(TOKENS_CYCLED, e2e_steps))]
     dev_in = {n: torch.empty_like(x) for n, x in toks[0].items()}
     host_o = torch.empty(B, H, d, dtype=torch.float32).pin_memory()
@@ -392,6 +471,7 @@ def run_ours(args):
     e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
 
     # figures
+    clocks_summary = clocks.summary(t_wall0, t_wall1)
     state_bytes = 2 * sum(lay.head_bytes(h) for h in range(H)) * B  # read + write, one launch
     io_bytes = B * H * (3 * d * (2 if wl.in_dtype == torch.bfloat16 else 4) + 4 * d + 8)
     # the d = 128 decode launches one kernel per width present (largest blocks first), for every
@@ -419,6 +499,9 @@ def run_ours(args):
                    "widths": {str(b): bits.count(b) for b in sorted(set(bits))}, "in_dtype": str(wl.in_dtype),
                    "gate": "scalar" if wl.gate == 0 else "channel", "tokens_cycled": TOKENS_CYCLED,
                    "l2": "no flush: the 2.0 GB state pool read+written per step exceeds the 126 MB L2",
+                   "generation_tokens": gen,
+                   "timing": "CUDA events around each step; the pool restarts from its initial state every "
+                             "generation_tokens steps, between steps and outside the timings",
                    "parallelism": f"dp{world} (independent requests per GPU)",
                    "s0_row_max_to_median": round(row_ratio, 2), "s0_col_max_to_median": round(col_ratio, 2)},
         "tokens_per_s": B * world / step_s,
@@ -433,10 +516,13 @@ def run_ours(args):
                      "kernel_source_sha256": decode_source_hash()},
         "e2e": {"value": head_steps / (e2e_ms / 1e3 / e2e_steps), "unit": "head-steps/s",
                 "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes, "steps": e2e_steps},
+        "alu_roofline": alu_roofline(bits, B, step_s_local, clocks_sm_mhz(clocks_summary)),
         "gpu_launches": args.steps * launches_per_step,
-        "clocks": clocks.summary(t_wall0, t_wall1),
+        "clocks": clocks_summary,
         "gpu": torch.cuda.get_device_name(dev),
     }
+    if graph_leg is not None:
+        result["per_layer_graph"] = graph_leg
     if world == 1 and not args.no_prefill:
         result["prefill"] = prefill_leg(dev, T=args.prefill_tokens)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -484,7 +570,7 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=512)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)

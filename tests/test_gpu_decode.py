@@ -427,3 +427,52 @@ def test_full_batch70_launch_sampled(stq, orc):
         compare_block(orc, bits[h], d, got, res["block"], res["tie"], tally, f"req {r} head {h}", err_scale=M)
         compare_o(o[r, h].cpu().numpy(), res["o"], tally, f"o req {r} head {h}")
     tally.check_budget()
+
+
+def test_per_layer_calls_equal_one_call_and_graph_replay(stq):
+    """A token issued as one stq_decode_step per layer of 48 heads (the serving shape) gives the
+    same bytes and readout as one call over all heads, eagerly and replayed from a CUDA graph."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl_ = wlm.scaled(wlm.WORKLOADS["full2304_b70_mixed"], batch=3)
+    B, H, d = wl_.batch, wl_.heads, wl_.d
+    bits = wlm.head_bits(wl_)
+    lay = stq.Layout(bits, d)
+    w = wlm.impact_weights(wl_, DEV)
+    slots = torch.arange(B, dtype=torch.int32, device=DEV)
+    pool0 = lay.alloc_pool(B)
+    stq.init_state(lay, pool0, slots, torch.stack([wlm.initial_state(wl_, r, DEV) for r in range(B)]), w)
+    inp = wlm.decode_inputs(wl_, 0, DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pool_a = pool0.clone()
+    o_a = torch.zeros(B, H, d, device=DEV)
+    stq.decode_step(lay, pool_a, slots, inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], w, o_a,
+                    status=status)
+    per = 48
+    parts = [{n: x[:, l * per:(l + 1) * per].contiguous() for n, x in inp.items()} for l in range(H // per)]
+    w_l = [w[l * per:(l + 1) * per].contiguous() for l in range(H // per)]
+    o_l = [torch.zeros(B, per, d, device=DEV) for _ in range(H // per)]
+
+    def token(pool):
+        for l, x in enumerate(parts):
+            stq.decode_step(lay, pool, slots, x["q"], x["k"], x["v"], x["beta"], x["alpha"], w_l[l], o_l[l],
+                            head_begin=l * per, status=status)
+
+    pool_b = pool0.clone()
+    token(pool_b)
+    torch.cuda.synchronize()
+    assert status.item() == 0, stq.status_flags(status)
+    assert torch.equal(pool_a, pool_b)
+    assert torch.equal(o_a, torch.cat(o_l, dim=1))
+    pool_c = pool0.clone()
+    for t in o_l:
+        t.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        token(pool_c)
+    pool_c.copy_(pool0)
+    g.replay()
+    torch.cuda.synchronize()
+    assert status.item() == 0, stq.status_flags(status)
+    assert torch.equal(pool_a, pool_c)
+    assert torch.equal(o_a, torch.cat(o_l, dim=1))
