@@ -30,6 +30,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "quantized-state head-steps/sec and achieved HBM GB/s (% roofline) at batch 70"
 DEFAULT_WORKLOAD = "full2304_b70_mixed"
+LIFETIME_WORKLOAD = "full2304_b70_lifetime"  # same workload, lifetime-aware widths
 TOKENS_CYCLED = 8
 FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ("quantized_linear_attention_stq_b200/csrc/decode_d128.cu",
@@ -370,11 +371,24 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(dev)
-    wl = wlm.WORKLOADS[args.workload]
+    lifetime = args.workload == LIFETIME_WORKLOAD
+    wl = wlm.WORKLOADS[DEFAULT_WORKLOAD if lifetime else args.workload]
     if args.batch:
         wl = wlm.scaled(wl, batch=args.batch)
     B, H, d = wl.batch, wl.heads, wl.d
     bits = wlm.head_bits(wl)
+    if lifetime:
+        # the same requests, inputs and byte budget, with widths from the lifetime-aware allocation
+        # calibrated on four other requests' states
+        import numpy as np
+
+        from quantized_linear_attention_stq_b200 import calibrate
+
+        w_cal = wlm.impact_weights(wl, dev)
+        S_cal = torch.stack([wlm.initial_state(wl, 100 + r, dev) for r in range(4)])
+        bits = calibrate.lifetime_widths(S_cal, w_cal, np.log(wlm.gate_values(wl).double().numpy()),
+                                         stq.Layout(bits, d).bytes_per_request, bits.count(16))
+        del S_cal
     lay = stq.Layout(bits, d, gate=wl.gate, in_dtype=wl.in_dtype)
     pool = lay.alloc_pool(B, dev)
     slots = torch.arange(B, dtype=torch.int32, device=dev)
@@ -441,7 +455,7 @@ def run_ours(args):
         raise RuntimeError(f"device status after timing: {stq.status_flags(status)}")
 
     graph_leg = None
-    if world == 1 and H % 48 == 0 and args.workload == DEFAULT_WORKLOAD:
+    if world == 1 and H % 48 == 0 and args.workload in (DEFAULT_WORKLOAD, LIFETIME_WORKLOAD):
         pool.copy_(pristine)
         graph_leg = per_layer_graph_leg(stq, lay, pool, slots, toks, w, status, dev, min(args.steps, gen), 5)
         if status.item() != 0:
@@ -551,9 +565,11 @@ def run_ours(args):
     }
     if graph_leg is not None:
         result["per_layer_graph"] = graph_leg
+    if lifetime:
+        result["config"]["widths_from"] = "lifetime-aware allocation (stq_allocate_widths), same byte budget"
     if world == 1 and not args.no_prefill:
         result["prefill"] = prefill_leg(dev, T=args.prefill_tokens)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not lifetime:
         rate, cores, sample = time_oracle(args.workload, oracle_workers(), 16, 20)
         result["cpu_baseline"] = {"value": rate, "unit": "head-steps/s", "cores": cores, "kind": "oracle",
                                   "sample": sample}

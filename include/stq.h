@@ -145,8 +145,9 @@ size_t stq_prefill_workspace_bytes(const stq_layout *layout, int32_t B, int32_t 
 /* Chunked prefill of T tokens for all H heads of B requests, in place. Tokens are cut into
  * chunks [0,chunk), [chunk,2chunk), ... of this call (the last may be short); inside a chunk
  * the state is carried unquantized, o_t = S_t^T q_t is emitted for every token, and the state is
- * requantized into the pool at the end of every chunk. chunk == 1 is the decode step token by
- * token.
+ * requantized at the end of every chunk exactly as a decode step requantizes it; the pool holds
+ * the requantized state after the last chunk (a multi-chunk call equals the same chunks issued one
+ * call each). chunk == 1 is the decode step token by token.
  *   q, k        device [B][H][T][d_k] of in_dtype;  v device [B][H][T][d_v] of in_dtype
  *   beta, alpha device fp32 [B][H][T] (scalar gate)
  *   w           device fp32 [H][d_k]
@@ -164,6 +165,27 @@ stq_status stq_prefill_chunk(const stq_layout *layout, void *pool, int32_t pool_
 stq_status stq_dequantize(const stq_layout *layout, const void *pool, int32_t pool_slots,
                           const int32_t *slots, int32_t B, float *S_out, int32_t *dev_status,
                           void *stream);
+
+/* Lifetime-aware width allocation (host only; no device work). The time dimension of the method
+ * ("线性注意力状态量化难题" (aitest123.com/news/n1kj09), section 时间维度; "K1 論文詳解", section
+ * 方法): a state unit's quantization error lives as long as its memory, so under a fixed budget
+ * the heads with large error and long lifetime get the higher precision, and the few
+ * highest-risk heads stay FP16 pivots. The pages fix no formula; this library uses, per head h:
+ *   lifetime weight  lam_h = 1 / max(1 - exp(l_h), 1e-12),  l_h = mean log-retention of the gate
+ *   risk             R_h(b) = lam_h * D_h(b),  D_h(b) = calibration distortion at width b
+ *   pivots           the num_pivots heads of largest R_h(8) (ties: lower head index)
+ *   the rest start at 4 bits; repeatedly the step 4 -> 6 or 6 -> 8 of largest risk reduction per
+ *   extra byte (ties: lower head index) is taken if the request's head-block bytes stay within
+ *   budget_bytes, otherwise that head keeps its width; until no step fits.
+ *   distortion          host double [H][3]: D_h at widths 4, 6, 8 (finite, >= 0)
+ *   mean_log_retention  host double [H] (finite, <= 0)
+ *   d                   d_k = d_v of the heads (16, 32, 64 or 128), sets the head-block bytes
+ *   widths_out          host uint8 [H], written: 4, 6, 8 or 16
+ * Returns STQ_ERR_INVALID_ARG for bad arguments or a budget below the smallest allocation (pivots
+ * at 16 bits, every other head at 4 bits). Deterministic; thread-safe. */
+stq_status stq_allocate_widths(int32_t num_heads, int32_t d, const double *distortion,
+                               const double *mean_log_retention, int32_t num_pivots,
+                               uint64_t budget_bytes, uint8_t *widths_out);
 
 #ifdef __cplusplus
 }

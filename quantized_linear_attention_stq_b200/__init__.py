@@ -6,5 +6,5 @@ All computation is in ``libstq.so`` (hand-written CUDA for sm_100a, C ABI in inc
 ``api`` marshals torch tensors into it and ``workloads`` draws seeded synthetic inputs.
 """
 from .api import (GATE_CHANNEL, GATE_CHANNEL_DECAY_FIRST, GATE_SCALAR, Layout, StqError,  # noqa: F401
-                  decode_step, dequantize, init_state, lib, prefill_chunk, prefill_workspace_bytes,
+                  allocate_widths, decode_step, dequantize, init_state, lib, prefill_chunk, prefill_workspace_bytes,
                   status_flags, status_string)

@@ -27,7 +27,7 @@ EXPORTS = (
     "stq_abi_version", "stq_status_string", "stq_layout_create", "stq_layout_destroy",
     "stq_layout_bytes_per_request", "stq_layout_head_offset", "stq_layout_head_bytes",
     "stq_layout_head_bits", "stq_init_state", "stq_decode_step", "stq_prefill_workspace_bytes",
-    "stq_prefill_chunk", "stq_dequantize",
+    "stq_prefill_chunk", "stq_dequantize", "stq_allocate_widths",
 )
 
 
@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
             L.stq_prefill_chunk.restype = i32
             L.stq_dequantize.argtypes = [P, P, i32, P, i32, P, P, P]
             L.stq_dequantize.restype = i32
+            L.stq_allocate_widths.argtypes = [i32, i32, P, P, i32, ctypes.c_uint64, P]
+            L.stq_allocate_widths.restype = i32
             _lib_handle = L
     return _lib_handle
 
@@ -230,3 +232,20 @@ def status_flags(status: torch.Tensor) -> list:
     """Names of the conditions OR-ed into a device status word (synchronizes)."""
     v = int(status.item())
     return [status_string(c) for c in (STQ_ERR_NONFINITE, STQ_ERR_TIMEOUT, STQ_ERR_BOUNDS) if v & (1 << c)]
+
+
+def allocate_widths(distortion, mean_log_retention, d: int, num_pivots: int, budget_bytes: int) -> list:
+    """Lifetime-aware widths per head (host only): distortion [H][3] at widths 4, 6, 8 and the mean
+    log-retention [H] of each head's gate; see stq_allocate_widths in include/stq.h."""
+    import numpy as np
+
+    D = np.ascontiguousarray(np.asarray(distortion, dtype=np.float64))
+    lr = np.ascontiguousarray(np.asarray(mean_log_retention, dtype=np.float64))
+    H = lr.shape[0]
+    if D.shape != (H, 3):
+        raise ValueError("distortion must be [H][3]")
+    out = np.zeros(H, dtype=np.uint8)
+    _check(lib().stq_allocate_widths(H, int(d), D.ctypes.data_as(ctypes.c_void_p), lr.ctypes.data_as(ctypes.c_void_p),
+                                     int(num_pivots), int(budget_bytes), out.ctypes.data_as(ctypes.c_void_p)),
+           "stq_allocate_widths")
+    return [int(x) for x in out]
