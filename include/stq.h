@@ -187,6 +187,20 @@ stq_status stq_allocate_widths(int32_t num_heads, int32_t d, const double *disto
                                const double *mean_log_retention, int32_t num_pivots,
                                uint64_t budget_bytes, uint8_t *widths_out);
 
+/* Key-row impact scores from calibration tokens ("线性注意力状态量化难题", section 空间维度): the
+ * readout error is a sum over key rows of the row's state error times a weight set by the current
+ * key, query and gate; the score is that weight's mean square, the w the quantizer takes. With
+ * one update E -> E' of a state error, the next readout error is E'^T q = E^T g, where
+ *   STQ_GATE_SCALAR               g = a (q - b (k.q) k)
+ *   STQ_GATE_CHANNEL              g = a*q - b (k.(a*q)) k
+ *   STQ_GATE_CHANNEL_DECAY_FIRST  g = a * (q - b (k.q) k)
+ *   q, k    device [T][H][d] of in_dtype (calibration tokens of H heads)
+ *   beta    device fp32 [T][H];  alpha device fp32 [T][H] (scalar gate) or [T][H][d]
+ *   w_out   device fp32 [H][d], written: w_i = mean over the T tokens of g_i^2
+ * d in {16, 32, 64, 128}. Enqueued on `stream`; allocates nothing. */
+stq_status stq_row_impact(int32_t T, int32_t H, int32_t d, int32_t gate, int32_t in_dtype, const void *q,
+                          const void *k, const float *beta, const float *alpha, float *w_out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -86,3 +86,33 @@ def allocate(distortion, mean_log_retention, d: int, num_pivots: int, budget_byt
         else:
             blocked.add(h)
     return [16 if level[h] is None else WIDTHS[level[h]] for h in range(H)]
+
+
+def row_impact(q, k, beta, alpha, gate: int = 0):
+    """Key-row impact scores of one head over calibration tokens ("线性注意力状态量化难题",
+    section 空间维度: the output error is the sum over key rows of each row's accumulated error
+    times a weight set by the current key, query and gate; the row impact score is that weight's
+    mean square). One update S' = A(S) carries a state error E to E' and the next readout error
+    is E'^T q = E^T g, so row i's weight is g_i:
+      scalar gate            g = a (q - b (k.q) k)
+      channel gate (literal) g = a*q - b (k.(a*q)) k          (S' = diag(a)(S - b k k^T S) + ...)
+      channel, decay first   g = a * (q - b (k.q) k)          (S' = diag(a) S - b k k^T diag(a) S + ...)
+    q, k: [T][d]; beta: [T]; alpha: [T] (scalar gate) or [T][d]. Returns w[d] = mean_t g_t^2."""
+    T = len(q)
+    d = len(q[0])
+    acc = [0.0] * d
+    for t in range(T):
+        qt = [float(x) for x in q[t]]
+        kt = [float(x) for x in k[t]]
+        b = float(beta[t])
+        a = [float(alpha[t])] * d if gate == 0 else [float(x) for x in alpha[t]]
+        if gate == 1:
+            aq = [a[i] * qt[i] for i in range(d)]
+            kaq = sum(kt[i] * aq[i] for i in range(d))
+            g = [aq[i] - b * kaq * kt[i] for i in range(d)]
+        else:
+            kq = sum(kt[i] * qt[i] for i in range(d))
+            g = [a[i] * (qt[i] - b * kq * kt[i]) for i in range(d)]
+        for i in range(d):
+            acc[i] += g[i] * g[i]
+    return [x / T for x in acc]

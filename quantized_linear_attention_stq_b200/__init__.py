@@ -7,4 +7,4 @@ All computation is in ``libstq.so`` (hand-written CUDA for sm_100a, C ABI in inc
 """
 from .api import (GATE_CHANNEL, GATE_CHANNEL_DECAY_FIRST, GATE_SCALAR, Layout, StqError,  # noqa: F401
                   allocate_widths, decode_step, dequantize, init_state, lib, prefill_chunk, prefill_workspace_bytes,
-                  status_flags, status_string)
+                  row_impact, status_flags, status_string)

@@ -27,7 +27,7 @@ EXPORTS = (
     "stq_abi_version", "stq_status_string", "stq_layout_create", "stq_layout_destroy",
     "stq_layout_bytes_per_request", "stq_layout_head_offset", "stq_layout_head_bytes",
     "stq_layout_head_bits", "stq_init_state", "stq_decode_step", "stq_prefill_workspace_bytes",
-    "stq_prefill_chunk", "stq_dequantize", "stq_allocate_widths",
+    "stq_prefill_chunk", "stq_dequantize", "stq_allocate_widths", "stq_row_impact",
 )
 
 
@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
             L.stq_dequantize.restype = i32
             L.stq_allocate_widths.argtypes = [i32, i32, P, P, i32, ctypes.c_uint64, P]
             L.stq_allocate_widths.restype = i32
+            L.stq_row_impact.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P]
+            L.stq_row_impact.restype = i32
             _lib_handle = L
     return _lib_handle
 
@@ -249,3 +251,20 @@ def allocate_widths(distortion, mean_log_retention, d: int, num_pivots: int, bud
                                      int(num_pivots), int(budget_bytes), out.ctypes.data_as(ctypes.c_void_p)),
            "stq_allocate_widths")
     return [int(x) for x in out]
+
+
+def row_impact(q, k, beta, alpha, gate: int = GATE_SCALAR, stream=None) -> torch.Tensor:
+    """Key-row impact scores w [H][d] from calibration tokens q, k [T][H][d], beta [T][H] and
+    alpha [T][H] (scalar gate) or [T][H][d]; see stq_row_impact in include/stq.h."""
+    T, H, d = q.shape
+    dev = q.device
+    if q.dtype not in _DTYPES:
+        raise TypeError("q must be float32 or bfloat16")
+    _need(k, "k", q.dtype, (T, H, d), dev)
+    _need(beta, "beta", torch.float32, (T, H), dev)
+    _need(alpha, "alpha", torch.float32, (T, H) if gate == GATE_SCALAR else (T, H, d), dev)
+    _need(q, "q", q.dtype, (T, H, d), dev)
+    w = torch.empty(H, d, dtype=torch.float32, device=dev)
+    _check(lib().stq_row_impact(T, H, d, int(gate), _DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(beta), _ptr(alpha),
+                                _ptr(w), _stream(stream)), "stq_row_impact")
+    return w

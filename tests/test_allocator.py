@@ -115,3 +115,41 @@ def test_library_rejects_bad_arguments():
         stq.allocate_widths(dist, lr, 100, 0, 10 ** 9)
     with pytest.raises(stq.StqError):
         stq.allocate_widths(dist, lr, D, 5, 10 ** 9)
+
+
+@pytest.mark.parametrize("gate", [0, 1, 2])
+def test_row_impact_is_the_readout_sensitivity_of_a_row_error(orc, gate):
+    """The impact weight g_i of key row i is what a unit error in row i does to the next readout:
+    perturb row i of the state by x, run the oracle's decode update and readout, compare."""
+    rng = np.random.default_rng(11 + gate)
+    d = 8
+    S = rng.normal(size=(d, d))
+    q, k, v = rng.normal(size=d), rng.normal(size=d), rng.normal(size=d)
+    k /= np.linalg.norm(k)
+    beta = 0.7
+    alpha = 0.93 if gate == 0 else rng.uniform(0.5, 1.0, size=d)
+    w = alo.row_impact([q], [k], [beta], [alpha] if gate == 0 else [alpha], gate)
+    _, base = orc.update(gate, S, q, k, v, beta, alpha)
+    for i in range(d):
+        x = rng.normal(size=d)
+        Sp = S.copy()
+        Sp[i] += x
+        _, o = orc.update(gate, Sp, q, k, v, beta, alpha)
+        ratio = (o - base) / x
+        # the readout moves by g_i * x: one common factor, whose square is w_i
+        assert np.allclose(ratio, ratio[0], rtol=1e-9, atol=1e-12)
+        assert ratio[0] ** 2 == pytest.approx(w[i], rel=1e-9, abs=1e-15)
+
+
+def test_row_impact_special_cases():
+    rng = np.random.default_rng(3)
+    d, T = 6, 5
+    q = rng.normal(size=(T, d))
+    k = rng.normal(size=(T, d))
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    # beta = 0: the weight is the decayed query
+    w = alo.row_impact(q, k, np.zeros(T), np.full(T, 0.8))
+    assert np.allclose(w, (0.64 * q ** 2).mean(axis=0), rtol=1e-12)
+    # q = k (unit) and beta = 1: the delta rule erases what the query would read
+    w = alo.row_impact(k, k, np.ones(T), np.ones(T))
+    assert np.allclose(w, 0.0, atol=1e-24)

@@ -57,3 +57,23 @@ def test_lifetime_widths_budget_order_and_error_growth(stq):
         assert st.item() == 0, stq.status_flags(st)
         peak[name] = o.abs().max().item()
     assert peak["lifetime"] * 100 < peak["random"], peak
+
+
+@pytest.mark.parametrize("d,gate,dtype", [(128, 0, torch.bfloat16), (128, 1, torch.float32), (64, 2, torch.bfloat16),
+                                          (16, 0, torch.float32)])
+def test_row_impact_matches_oracle(stq, d, gate, dtype):
+    from oracle import allocate as alo
+
+    g = torch.Generator().manual_seed(d + gate)
+    T, H = 37, 5
+    q = torch.randn(T, H, d, generator=g).to(dtype)
+    k = torch.nn.functional.normalize(torch.randn(T, H, d, generator=g), dim=-1).to(dtype)
+    beta = torch.sigmoid(torch.randn(T, H, generator=g))
+    alpha = torch.rand(T, H, generator=g) * 0.5 + 0.5 if gate == 0 else torch.rand(T, H, d, generator=g) * 0.5 + 0.5
+    w = stq.row_impact(q.to(DEV), k.to(DEV), beta.to(DEV), alpha.to(DEV), gate=gate)
+    torch.cuda.synchronize()
+    got = w.cpu().double().numpy()
+    for h in range(H):
+        ref = alo.row_impact(q[:, h].double().numpy(), k[:, h].double().numpy(), beta[:, h].double().numpy(),
+                             alpha[:, h].double().numpy(), gate)
+        np.testing.assert_allclose(got[h], ref, rtol=2e-5, atol=1e-12)
