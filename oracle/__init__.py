@@ -78,6 +78,12 @@ def lib():
             L.orc_prefill_seq.restype = i32
             L.orc_chunk_wy.argtypes = [i32, i32, i32, P, P, P, P, P, P, P, P]
             L.orc_chunk_wy.restype = i32
+            L.orc_uniform_block_bytes.argtypes, L.orc_uniform_block_bytes.restype = [i32, i32, i32], sz
+            L.orc_quantize_uniform.argtypes = [i32, i32, i32, P, P, P, P, f64]
+            L.orc_quantize_uniform.restype = i32
+            L.orc_dequantize_uniform.argtypes, L.orc_dequantize_uniform.restype = [i32, i32, i32, P, P], i32
+            L.orc_decode_step_uniform.argtypes = [i32, i32, i32, i32, P, P, P, P, f64, P, P, P, P, f64]
+            L.orc_decode_step_uniform.restype = i32
             _lib = L
     return _lib
 
@@ -250,3 +256,47 @@ def request_layout(head_bits, dk: int, dv: int):
         pos += block_bytes(int(b), dk, dv)
     total = (pos + 127) // 128 * 128
     return np.array(offs, dtype=np.int64), total
+
+
+# ---------------------------------------------------------------------------------------------
+# Uniform baseline quantizer (one scale per head; see stq_oracle.c)
+# ---------------------------------------------------------------------------------------------
+
+def uniform_block_bytes(bits: int, dk: int, dv: int) -> int:
+    return int(lib().orc_uniform_block_bytes(bits, dk, dv))
+
+
+def quantize_uniform(bits: int, S, delta: float = TIE_DELTA):
+    """Uniform per-head quantization into a fresh block. Returns (block, x, tie, status)."""
+    S = _f64(S)
+    dk, dv = S.shape
+    block = np.zeros(uniform_block_bytes(bits, dk, dv), dtype=np.uint8)
+    x = np.zeros((dk, dv))
+    tie = np.zeros((dk, dv), dtype=np.uint8)
+    st = lib().orc_quantize_uniform(bits, dk, dv, _p(S), _p(block), _p(x), _p(tie), float(delta))
+    return block, x, tie.astype(bool), st
+
+
+def dequantize_uniform(bits: int, dk: int, dv: int, block) -> np.ndarray:
+    block = np.ascontiguousarray(np.asarray(block, dtype=np.uint8))
+    S = np.zeros((dk, dv))
+    lib().orc_dequantize_uniform(bits, dk, dv, _p(block), _p(S))
+    return S
+
+
+def uniform_scale(bits: int, dk: int, dv: int, block) -> float:
+    off = scale_offset(bits, dk, dv)
+    return float(np.asarray(block, dtype=np.uint8)[off:off + 4].view(np.float32)[0])
+
+
+def decode_step_uniform(bits: int, gate: int, block, q, k, v, beta: float, alpha, dk: int, dv: int,
+                        delta: float = TIE_DELTA):
+    """One decode step of a uniformly quantized head on a copy of ``block``."""
+    blk = np.ascontiguousarray(np.asarray(block, dtype=np.uint8)).copy()
+    o = np.zeros(dv, dtype=np.float32)
+    x = np.zeros((dk, dv))
+    tie = np.zeros((dk, dv), dtype=np.uint8)
+    a = _f64(np.atleast_1d(alpha))
+    st = lib().orc_decode_step_uniform(bits, dk, dv, gate, _p(blk), _p(_f64(q)), _p(_f64(k)), _p(_f64(v)),
+                                       float(beta), _p(a), _p(o), _p(x), _p(tie), float(delta))
+    return dict(block=blk, o=o, x=x, tie=tie.astype(bool), status=st)

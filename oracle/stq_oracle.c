@@ -528,3 +528,92 @@ int orc_chunk_wy(int dk, int dv, int C, const double *S0, const double *q, const
     free(P);
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Uniform baseline quantizer: one scale per head                                             */
+/*                                                                                            */
+/* [P5 直接量化为什么会翻车 / 数据说话] and [P1 實驗結果]: the pages compare the method with     */
+/* uniform INT quantization of the state ("统一INT8"), the direct approach whose errors        */
+/* accumulate. Reading: symmetric per-head (per-tensor) INT quantization with the method's     */
+/* code range and rounding, fp32 scale:                                                        */
+/*   s = max_ij |S_ij| / qmax,  s := 1 if it is 0,  s~ = fp32(s)                               */
+/*   x_ij = S_ij / s~,  Q_ij = clamp(round_half_even(x_ij), -qmax, qmax)                       */
+/* Block: the codes bitstream as for the method, zero padding to 16 bytes, s~ (fp32), zero    */
+/* padding to 128 bytes.                                                                       */
+/* ------------------------------------------------------------------------------------------ */
+
+size_t orc_uniform_block_bytes(int bits, int dk, int dv)
+{
+    return round_up(orc_scale_offset(bits, dk, dv) + 4, 128);
+}
+
+int orc_quantize_uniform(int bits, int dk, int dv, const double *S, uint8_t *block, double *x_out,
+                         uint8_t *tie_out, double delta)
+{
+    if (!(bits == 4 || bits == 6 || bits == 8) || dk < 1 || dv < 1) return ORC_EINVAL;
+    size_t n = (size_t)dk * dv;
+    int nonfinite = 0;
+    double m = 0.0;
+    for (size_t e = 0; e < n; ++e) {
+        if (!isfinite(S[e])) nonfinite = 1;
+        if (fabs(S[e]) > m) m = fabs(S[e]);
+    }
+    memset(block, 0, orc_uniform_block_bytes(bits, dk, dv));
+    int qmax = orc_qmax(bits);
+    double s = m / (double)qmax;
+    if (s == 0.0) s = 1.0;
+    float sf = (float)s;
+    if (!isfinite(sf) || sf == 0.0f) nonfinite = 1;
+    int32_t *u = (int32_t *)malloc(sizeof(int32_t) * n);
+    for (size_t e = 0; e < n; ++e) {
+        double x = S[e] / (double)sf;
+        double qv = orc_round_half_even(x);
+        if (qv > qmax) qv = qmax;
+        if (qv < -qmax) qv = -qmax;
+        if (!isfinite(x)) qv = 0.0;
+        u[e] = (int32_t)qv + (1 << (bits - 1));
+        if (x_out) x_out[e] = x;
+        if (tie_out) tie_out[e] = isfinite(x) ? (tie_distance(x) <= delta) : 0;
+    }
+    orc_pack(bits, n, u, block);
+    store_f32(block + orc_scale_offset(bits, dk, dv), sf);
+    free(u);
+    return nonfinite ? ORC_ENONFINITE : ORC_OK;
+}
+
+int orc_dequantize_uniform(int bits, int dk, int dv, const uint8_t *block, double *S)
+{
+    if (!(bits == 4 || bits == 6 || bits == 8) || dk < 1 || dv < 1) return ORC_EINVAL;
+    size_t n = (size_t)dk * dv;
+    int32_t *u = (int32_t *)malloc(sizeof(int32_t) * n);
+    orc_unpack(bits, n, block, u);
+    double s = (double)load_f32(block + orc_scale_offset(bits, dk, dv));
+    for (size_t e = 0; e < n; ++e) S[e] = s * (double)(u[e] - (1 << (bits - 1)));
+    free(u);
+    return ORC_OK;
+}
+
+/* One decode step of a uniformly quantized head: dequantize -> update -> readout -> requantize. */
+int orc_decode_step_uniform(int bits, int dk, int dv, int gate, uint8_t *block, const double *q,
+                            const double *k, const double *v, double beta, const double *alpha,
+                            float *o, double *x_out, uint8_t *tie_out, double delta)
+{
+    if (!(bits == 4 || bits == 6 || bits == 8) || dk < 1 || dv < 1) return ORC_EINVAL;
+    if (gate != ORC_GATE_SCALAR && gate != ORC_GATE_CHANNEL && gate != ORC_GATE_CHANNEL_DECAY_FIRST)
+        return ORC_EINVAL;
+    size_t n = (size_t)dk * dv;
+    double *S = (double *)malloc(sizeof(double) * n);
+    double *od = (double *)malloc(sizeof(double) * dv);
+    orc_dequantize_uniform(bits, dk, dv, block, S);
+    orc_update(dk, dv, gate, S, q, k, v, beta, alpha, od);
+    int nonfinite = 0;
+    for (int j = 0; j < dv; ++j) {
+        o[j] = (float)od[j];
+        if (!isfinite(o[j])) nonfinite = 1;
+    }
+    int st = orc_quantize_uniform(bits, dk, dv, S, block, x_out, tie_out, delta);
+    free(S);
+    free(od);
+    if (st != ORC_OK) return st;
+    return nonfinite ? ORC_ENONFINITE : ORC_OK;
+}

@@ -47,4 +47,12 @@ int orc_chunk_wy(int dk, int dv, int C, const double *S0, const double *q, const
                  const double *v, const double *beta, const double *alpha, double *S_end,
                  double *O);
 
+size_t orc_uniform_block_bytes(int bits, int dk, int dv);
+int orc_quantize_uniform(int bits, int dk, int dv, const double *S, uint8_t *block, double *x_out,
+                         uint8_t *tie_out, double delta);
+int orc_dequantize_uniform(int bits, int dk, int dv, const uint8_t *block, double *S);
+int orc_decode_step_uniform(int bits, int dk, int dv, int gate, uint8_t *block, const double *q,
+                            const double *k, const double *v, double beta, const double *alpha,
+                            float *o, double *x_out, uint8_t *tie_out, double delta);
+
 #endif

@@ -532,3 +532,68 @@ def test_prefill_empty_call_is_identity(orc):
     e = np.zeros((0, 16))
     res = orc.prefill_seq(4, 0, block, e, e, e, np.zeros(0), np.zeros(0), w, 64, 16, 16)
     assert np.array_equal(res["block"], block)
+
+
+# ---------------------------------------------------------------------------------------------
+# Uniform baseline quantizer (one scale per head)
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [4, 6, 8])
+def test_uniform_integer_multiples_round_trip_exactly(orc, bits):
+    # S = s * G with integer G, max |G| = qmax: the scale is s and the codes are G exactly
+    rng = np.random.default_rng(bits)
+    qm = orc.qmax(bits)
+    G = rng.integers(-qm, qm + 1, size=(9, 7)).astype(float)
+    G[3, 2] = -qm
+    s = 2.0 ** -5 * 3
+    blk, x, tie, st = orc.quantize_uniform(bits, s * G)
+    assert st == orc.OK
+    assert orc.uniform_scale(bits, 9, 7, blk) == s
+    assert np.array_equal(orc.unpack(bits, 63, blk).reshape(9, 7) - (1 << (bits - 1)), G.astype(int))
+    assert np.array_equal(orc.dequantize_uniform(bits, 9, 7, blk), s * G)
+
+
+@pytest.mark.parametrize("bits", [4, 6])
+def test_uniform_rounds_half_to_even_and_bounds_the_error(orc, bits):
+    qm = orc.qmax(bits)
+    # a planted tie: max entry qmax*s, another entry at exactly 2.5*s
+    S = np.zeros((3, 4))
+    S[0, 0] = qm * 0.25
+    S[1, 1] = 2.5 * 0.25
+    S[2, 3] = -1.5 * 0.25
+    blk, x, tie, st = orc.quantize_uniform(bits, S)
+    codes = orc.unpack(bits, 12, blk).reshape(3, 4) - (1 << (bits - 1))
+    assert codes[1, 1] == 2 and codes[2, 3] == -2 and tie[1, 1] and tie[2, 3]
+    # random states: |S - s Q| <= s/2 everywhere, and the largest entry maps to +-qmax
+    rng = np.random.default_rng(5)
+    S = rng.normal(size=(16, 16)) * np.exp(rng.normal(size=(16, 1)))
+    blk, x, tie, st = orc.quantize_uniform(bits, S)
+    s = orc.uniform_scale(bits, 16, 16, blk)
+    Sh = orc.dequantize_uniform(bits, 16, 16, blk)
+    assert np.max(np.abs(S - Sh)) <= s / 2 * (1 + 1e-12)
+    assert np.max(np.abs(orc.unpack(bits, 256, blk) - (1 << (bits - 1)))) == qm
+
+
+def test_uniform_block_layout_and_zero_state(orc):
+    # codes padded to 16 bytes, one fp32 scale, padding to 128 bytes
+    assert orc.uniform_block_bytes(4, 128, 128) == 8320
+    assert orc.uniform_block_bytes(6, 128, 128) == 12416
+    assert orc.uniform_block_bytes(8, 16, 16) == 384
+    blk, _, _, st = orc.quantize_uniform(6, np.zeros((4, 4)))
+    assert st == orc.OK and orc.uniform_scale(6, 4, 4, blk) == 1.0
+    assert np.all(orc.dequantize_uniform(6, 4, 4, blk) == 0.0)
+
+
+def test_uniform_decode_step_is_update_then_uniform_requantization(orc):
+    rng = np.random.default_rng(9)
+    d = 8
+    S = rng.normal(size=(d, d))
+    blk, _, _, _ = orc.quantize_uniform(8, S)
+    q, k, v = rng.normal(size=d), rng.normal(size=d), rng.normal(size=d)
+    k /= np.linalg.norm(k)
+    res = orc.decode_step_uniform(8, 0, blk, q, k, v, 0.6, 0.97, d, d)
+    S_deq = orc.dequantize_uniform(8, d, d, blk)
+    S_new, o = orc.update(0, S_deq, q, k, v, 0.6, 0.97)
+    assert np.array_equal(res["o"], o.astype(np.float32))
+    ref_blk, _, _, _ = orc.quantize_uniform(8, S_new)
+    assert np.array_equal(res["block"], ref_blk)
