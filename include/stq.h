@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define STQ_ABI_VERSION 1
+#define STQ_ABI_VERSION 2
 
 typedef enum {
     STQ_OK = 0,
@@ -80,6 +80,13 @@ typedef enum {
     STQ_GATE_CHANNEL_DECAY_FIRST = 2 /* alpha [B][H][d_k]   */
 } stq_gate;
 
+/* How the 4/6/8-bit heads of a layout are scaled. STQ_SCALES_UNIFORM is the baseline the pages
+ * compare the method with ("线性注意力状态量化难题", sections 直接量化为什么会翻车 / 数据说话): one
+ * symmetric scale per head, s = max_ij |S_ij| / qmax (0 -> 1), stored fp32, codes
+ * Q_ij = round_half_even(S_ij / s); its head block is the codes bitstream, zero padding to 16
+ * bytes, s, zero padding to 128 bytes. Uniform layouts run on the plain (untuned) kernels. */
+typedef enum { STQ_SCALES_ROW_COLUMN = 0, STQ_SCALES_UNIFORM = 1 } stq_scale_mode;
+
 /* Static description of one model's state: fixed across requests and steps. */
 typedef struct {
     int32_t num_heads;         /* H >= 1 (all layers' heads of one request, in pool order)   */
@@ -88,6 +95,7 @@ typedef struct {
     const uint8_t *head_bits;  /* host [H]: 4, 6, 8, or 16 (FP16 pivot head); copied         */
     int32_t gate;              /* stq_gate                                                   */
     int32_t in_dtype;          /* stq_dtype of q, k, v                                       */
+    int32_t scale_mode;        /* stq_scale_mode (0: the method's row x column scales)       */
 } stq_layout_desc;
 
 typedef struct stq_layout stq_layout; /* opaque, host-only, immutable after creation */

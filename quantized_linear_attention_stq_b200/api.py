@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libstq.so")
 STQ_OK, STQ_ERR_INVALID_ARG, STQ_ERR_UNSUPPORTED, STQ_ERR_CUDA = 0, 1, 2, 3
 STQ_ERR_NONFINITE, STQ_ERR_TIMEOUT, STQ_ERR_BOUNDS = 4, 5, 6
 GATE_SCALAR, GATE_CHANNEL, GATE_CHANNEL_DECAY_FIRST = 0, 1, 2
+SCALES_ROW_COLUMN, SCALES_UNIFORM = 0, 1  # stq_scale_mode
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 
 # Every function the public header declares (checked against include/stq.h by the tests).
@@ -40,7 +41,7 @@ class StqError(RuntimeError):
 class _Desc(ctypes.Structure):
     _fields_ = [("num_heads", ctypes.c_int32), ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32),
                 ("head_bits", ctypes.POINTER(ctypes.c_uint8)), ("gate", ctypes.c_int32),
-                ("in_dtype", ctypes.c_int32)]
+                ("in_dtype", ctypes.c_int32), ("scale_mode", ctypes.c_int32)]
 
 
 _lock = threading.Lock()
@@ -120,14 +121,15 @@ class Layout:
     """Host-side description of one model's quantized state (see stq_layout_desc)."""
 
     def __init__(self, head_bits: Sequence[int], d: int, gate: int = GATE_SCALAR,
-                 in_dtype: torch.dtype = torch.bfloat16):
+                 in_dtype: torch.dtype = torch.bfloat16, scale_mode: int = SCALES_ROW_COLUMN):
         self.head_bits = [int(b) for b in head_bits]
         self.H, self.d, self.gate, self.in_dtype = len(self.head_bits), int(d), int(gate), in_dtype
+        self.scale_mode = int(scale_mode)
         if in_dtype not in _DTYPES:
             raise TypeError(f"unsupported input dtype {in_dtype}")
         arr = (ctypes.c_uint8 * self.H)(*self.head_bits)
         desc = _Desc(self.H, self.d, self.d, ctypes.cast(arr, ctypes.POINTER(ctypes.c_uint8)),
-                     self.gate, _DTYPES[in_dtype])
+                     self.gate, _DTYPES[in_dtype], self.scale_mode)
         handle = ctypes.c_void_p()
         _check(lib().stq_layout_create(ctypes.byref(desc), ctypes.byref(handle)), "stq_layout_create")
         self._h = handle

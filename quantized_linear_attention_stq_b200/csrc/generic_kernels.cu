@@ -16,6 +16,7 @@ constexpr int kThreads = 256;
 
 struct TileRef {
     bool ok;
+    bool uniform;  // one scale for the whole head (the baseline quantizer)
     int b, head, bits;
     uint8_t *block;
 };
@@ -27,6 +28,7 @@ __device__ __forceinline__ TileRef tile_ref(const TileParams &p, int b, int pos)
     t.b = b;
     t.head = entry_head(e);
     t.bits = entry_bits(e);
+    t.uniform = entry_uniform(e);
     const int slot = p.slots[b];
     t.ok = slot >= 0 && slot < p.pool_slots;
     t.block = t.ok ? p.pool + (uint64_t)slot * p.req_bytes + e.off : nullptr;
@@ -43,13 +45,21 @@ __device__ __forceinline__ int read_code(const uint8_t *codes, int bits, int n)
     return (int)(((lo | (hi << 8)) >> (bit & 7)) & ((1u << bits) - 1u));
 }
 
-// Dequantize a tile from global memory into S (row stride ld): S_ij = fp32(r_i c_j) * Q_ij.
-__device__ void dequant_to_smem(const uint8_t *block, int bits, int dk, int dv, float *S, int ld)
+// Dequantize a tile from global memory into S (row stride ld): S_ij = fp32(r_i c_j) * Q_ij, or
+// S_ij = s * Q_ij for a uniformly scaled head.
+__device__ void dequant_to_smem(const uint8_t *block, int bits, bool uniform, int dk, int dv, float *S, int ld)
 {
     const int n = dk * dv;
     if (bits == 16) {
         const __half *h = reinterpret_cast<const __half *>(block);
         for (int e = threadIdx.x; e < n; e += blockDim.x) S[(e / dv) * ld + e % dv] = __half2float(h[e]);
+        return;
+    }
+    if (uniform) {
+        const float su = *reinterpret_cast<const float *>(block + scale_offset(bits, dk, dv));
+        const int off = 1 << (bits - 1);
+        for (int e = threadIdx.x; e < n; e += blockDim.x)
+            S[(e / dv) * ld + e % dv] = su * (float)(read_code(block, bits, e) - off);
         return;
     }
     const float *r = reinterpret_cast<const float *>(block + scale_offset(bits, dk, dv));
@@ -65,10 +75,11 @@ __device__ void dequant_to_smem(const uint8_t *block, int bits, int dk, int dv, 
 // Fit scales to the fp32 state in S and write codes + scales into `block` (or fp16 values for a
 // pivot head). `wv` holds the impact weights of the head in shared memory. Needs a CTA-wide
 // barrier before (S complete) and provides one after.
-__device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, int dk, int dv,
+__device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, bool uniform, int dk, int dv,
                                    uint8_t *block, float *cs, float *rs, int32_t *status)
 {
     const int n = dk * dv;
+    __shared__ uint32_t smax;
     if (bits == 16) {
         __half *h = reinterpret_cast<__half *>(block);
         bool bad = false;
@@ -81,6 +92,42 @@ __device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, 
         return;
     }
     const float qmax = (float)((1 << (bits - 1)) - 1);
+    if (uniform) {
+        // one symmetric scale per head: s = max |S_ij| / qmax (1 when the head is all zero). The
+        // magnitudes are non-negative, so their fp32 bit patterns order like their values and an
+        // integer max reduces them; a NaN is skipped by fmaxf and caught by the finiteness flag.
+        if (threadIdx.x == 0) smax = 0u;
+        __syncthreads();
+        float m = 0.f;
+        bool bad = false;
+        for (int e = threadIdx.x; e < n; e += blockDim.x) {
+            const float x = S[(e / dv) * ld + e % dv];
+            m = fmaxf(m, fabsf(x));
+            bad |= !isfinite(x);
+        }
+        for (int sh = 16; sh > 0; sh >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, sh));
+        if ((threadIdx.x & 31) == 0) atomicMax(&smax, __float_as_uint(m));
+        __syncthreads();
+        float su = __uint_as_float(smax) / qmax;
+        if (su == 0.f) su = 1.f;
+        bad |= !isfinite(su);
+        if (threadIdx.x == 0) *reinterpret_cast<float *>(block + scale_offset(bits, dk, dv)) = su;
+        const int cpg = bits == 4 ? 2 : (bits == 6 ? 4 : 1);
+        const int bpg = bits == 6 ? 3 : 1;
+        const int off = 1 << (bits - 1);
+        for (int g = threadIdx.x; g < n / cpg; g += blockDim.x) {
+            uint32_t word = 0;
+            for (int t = 0; t < cpg; ++t) {
+                const int e = g * cpg + t;
+                const float xr = S[(e / dv) * ld + e % dv] / su;
+                const float x = isfinite(xr) ? fminf(fmaxf(rintf(xr), -qmax), qmax) : 0.f;  // rintf: half to even
+                word |= (uint32_t)((int)x + off) << (bits * t);
+            }
+            for (int t = 0; t < bpg; ++t) block[g * bpg + t] = (uint8_t)(word >> (8 * t));
+        }
+        if (__syncthreads_or(bad) && threadIdx.x == 0) flag(status, kFlagNonfinite);
+        return;
+    }
     // column scales: impact-weighted RMS over the key rows
     for (int j = threadIdx.x; j < dv; j += blockDim.x) {
         float W = 0.f, E = 0.f;
@@ -123,9 +170,8 @@ __device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, 
         for (int t = 0; t < cpg; ++t) {
             const int e = g * cpg + t;
             const int i = e / dv, j = e % dv;
-            float x = (S[i * ld + j] / cs[j]) / rs[i];
-            x = fminf(fmaxf(rintf(x), -qmax), qmax);  // rintf rounds half to even
-            if (!isfinite(x)) x = 0.f;
+            const float xr = (S[i * ld + j] / cs[j]) / rs[i];
+            const float x = isfinite(xr) ? fminf(fmaxf(rintf(xr), -qmax), qmax) : 0.f;  // rintf: half to even
             word |= (uint32_t)((int)x + off) << (bits * t);
         }
         for (int t = 0; t < bpg; ++t) block[g * bpg + t] = (uint8_t)(word >> (8 * t));
@@ -154,7 +200,7 @@ __global__ void __launch_bounds__(kThreads) init_kernel(const __grid_constant__ 
     for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) S[(e / dv) * ld + e % dv] = src[e];
     for (int i = threadIdx.x; i < dk; i += blockDim.x) wv[i] = p.w[(uint64_t)t.head * dk + i];
     __syncthreads();
-    quantize_from_smem(S, ld, wv, t.bits, dk, dv, t.block, cs, rs, p.status);
+    quantize_from_smem(S, ld, wv, t.bits, t.uniform, dk, dv, t.block, cs, rs, p.status);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -170,7 +216,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const __grid_constant
     }
     const int dk = p.dk, dv = p.dv;
     float *dst = p.S_out + ((uint64_t)b * p.head_count + t.head) * dk * dv;
-    dequant_to_smem(t.block, t.bits, dk, dv, dst, dv);  // writes straight to global, row stride dv
+    dequant_to_smem(t.block, t.bits, t.uniform, dk, dv, dst, dv);  // writes straight to global, row stride dv
 }
 
 // ------------------------------------------------------------------------------------------
@@ -205,7 +251,7 @@ __global__ void __launch_bounds__(kThreads) decode_generic_kernel(const __grid_c
         wv[i] = p.w[(uint64_t)t.head * dk + i];
     }
     for (int j = threadIdx.x; j < dv; j += blockDim.x) vv[j] = load_in<IN_BF16>(p.v, tile * dv + j);
-    dequant_to_smem(t.block, t.bits, dk, dv, S, ld);
+    dequant_to_smem(t.block, t.bits, t.uniform, dk, dv, S, ld);
     __syncthreads();
     const float beta = p.beta[tile];
     const bool decay_first = p.gate == 2;
@@ -233,7 +279,7 @@ __global__ void __launch_bounds__(kThreads) decode_generic_kernel(const __grid_c
         bad |= !isfinite(acc);
     }
     if (bad) flag(p.status, kFlagNonfinite);
-    quantize_from_smem(S, ld, wv, t.bits, dk, dv, t.block, cs, rs, p.status);
+    quantize_from_smem(S, ld, wv, t.bits, t.uniform, dk, dv, t.block, cs, rs, p.status);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -264,7 +310,7 @@ __global__ void __launch_bounds__(kThreads) prefill_seq_kernel(const __grid_cons
     const uint64_t tile = (uint64_t)b * p.head_count + t.head;
     const bool channel = p.gate != 0, decay_first = p.gate == 2;
     for (int i = threadIdx.x; i < dk; i += blockDim.x) wv[i] = p.w[(uint64_t)t.head * dk + i];
-    dequant_to_smem(t.block, t.bits, dk, dv, S, ld);
+    dequant_to_smem(t.block, t.bits, t.uniform, dk, dv, S, ld);
     bool bad = false;
     for (int tok = 0; tok < T; ++tok) {
         const uint64_t row = tile * T + tok;
@@ -297,10 +343,10 @@ __global__ void __launch_bounds__(kThreads) prefill_seq_kernel(const __grid_cons
         }
         if ((tok + 1) % chunk == 0 || tok == T - 1) {
             __syncthreads();
-            quantize_from_smem(S, ld, wv, t.bits, dk, dv, t.block, cs, rs, p.status);
+            quantize_from_smem(S, ld, wv, t.bits, t.uniform, dk, dv, t.block, cs, rs, p.status);
             if (tok != T - 1) {
                 __syncthreads();
-                dequant_to_smem(t.block, t.bits, dk, dv, S, ld);
+                dequant_to_smem(t.block, t.bits, t.uniform, dk, dv, S, ld);
             }
         }
         __syncthreads();

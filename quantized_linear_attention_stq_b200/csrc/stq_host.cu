@@ -13,6 +13,7 @@
 
 struct stq_layout {
     int32_t H, dk, dv, gate, in_dtype;
+    bool uniform;  // STQ_SCALES_UNIFORM
     std::vector<uint8_t> bits;
     std::vector<uint64_t> offset;
     std::vector<uint64_t> bytes;
@@ -40,7 +41,8 @@ void fill_table(stq::TileParams &p, const stq_layout *L, const std::vector<int> 
     for (int e = 0; e < n; ++e) {
         const int h = ord[first + e];
         p.table[e].off = (uint32_t)L->offset[h];
-        p.table[e].info = (uint32_t)(h - h0) | ((uint32_t)L->bits[h] << 16);
+        p.table[e].info = (uint32_t)(h - h0) | ((uint32_t)L->bits[h] << 16) |
+                          ((L->uniform && L->bits[h] != 16) ? (1u << 24) : 0u);
     }
 }
 
@@ -81,6 +83,7 @@ stq_status stq_layout_create(const stq_layout_desc *desc, stq_layout **out)
     if (desc->num_heads < 1 || desc->d_k < 1 || desc->d_v < 1) return STQ_ERR_INVALID_ARG;
     if (desc->gate < STQ_GATE_SCALAR || desc->gate > STQ_GATE_CHANNEL_DECAY_FIRST) return STQ_ERR_INVALID_ARG;
     if (desc->in_dtype != STQ_F32 && desc->in_dtype != STQ_BF16) return STQ_ERR_INVALID_ARG;
+    if (desc->scale_mode != STQ_SCALES_ROW_COLUMN && desc->scale_mode != STQ_SCALES_UNIFORM) return STQ_ERR_INVALID_ARG;
     const int d = desc->d_k;
     if (desc->d_v != d || !(d == 16 || d == 32 || d == 64 || d == 128)) return STQ_ERR_UNSUPPORTED;
     if (desc->num_heads > 65535) return STQ_ERR_UNSUPPORTED;
@@ -91,13 +94,15 @@ stq_status stq_layout_create(const stq_layout_desc *desc, stq_layout **out)
     L->dv = desc->d_v;
     L->gate = desc->gate;
     L->in_dtype = desc->in_dtype;
+    L->uniform = desc->scale_mode == STQ_SCALES_UNIFORM;
     uint64_t pos = 0;
     for (int h = 0; h < L->H; ++h) {
         const int b = desc->head_bits[h];
         if (b != 4 && b != 6 && b != 8 && b != 16) return STQ_ERR_UNSUPPORTED;
         L->bits.push_back((uint8_t)b);
         L->offset.push_back(pos);
-        const uint64_t nb = stq::head_block_bytes(b, L->dk, L->dv);
+        const uint64_t nb = (L->uniform && b != 16) ? stq::uniform_block_bytes(b, L->dk, L->dv)
+                                                    : stq::head_block_bytes(b, L->dk, L->dv);
         L->bytes.push_back(nb);
         pos += nb;
     }
@@ -211,7 +216,7 @@ stq_status stq_decode_step(const stq_layout *L, void *pool, int32_t pool_slots, 
     p->gate = L->gate;
     p->w = w;
     const int in_bf16 = L->in_dtype == STQ_BF16;
-    const bool tuned = L->dk == 128;
+    const bool tuned = L->dk == 128 && !L->uniform;
     const int maxb = tuned ? stq::decode_d128_max_requests() : 65535;
     const std::vector<int> ord = order_by_size(L, head_begin, head_count);
     const size_t in_sz = in_bf16 ? 2 : 4;
@@ -290,7 +295,8 @@ stq_status stq_prefill_chunk(const stq_layout *L, void *pool, int32_t pool_slots
     // 128 x 128 heads with bf16 inputs, the scalar gate and 64-token chunks take the tensor-core
     // WY path, one launch per code width; FP16 pivot heads and every other configuration take the
     // sequential kernel.
-    const bool wy = L->dk == 128 && L->gate == STQ_GATE_SCALAR && L->in_dtype == STQ_BF16 && chunk == 64;
+    const bool wy = L->dk == 128 && L->gate == STQ_GATE_SCALAR && L->in_dtype == STQ_BF16 && chunk == 64 &&
+                    !L->uniform;
     if (!wy) {
         std::vector<int> ord(L->H);
         for (int h = 0; h < L->H; ++h) ord[h] = h;

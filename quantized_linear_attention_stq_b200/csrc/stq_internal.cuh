@@ -46,6 +46,12 @@ struct TileEntry {
 };
 __host__ __device__ inline int entry_head(const TileEntry &e) { return (int)(e.info & 0xffffu); }
 __host__ __device__ inline int entry_bits(const TileEntry &e) { return (int)((e.info >> 16) & 0xffu); }
+// bit 24: the head uses one uniform scale (the baseline quantizer) instead of row x column scales
+__host__ __device__ inline bool entry_uniform(const TileEntry &e) { return ((e.info >> 24) & 1u) != 0; }
+__host__ __device__ constexpr uint32_t uniform_block_bytes(int bits, int dk, int dv)
+{
+    return round_up_u32(scale_offset(bits, dk, dv) + 4u, 128);
+}
 
 // Head table capacity of one launch; larger head ranges are split into several launches.
 constexpr int kMaxTable = 3072;

@@ -114,6 +114,41 @@ def compare_block(orc, bits, d, got, ref_block, ref_tie, tally: Tally, what="", 
     assert not got[n_used:].any()
 
 
+def uniform_request_layout(orc, head_bits, d):
+    """Offsets and request bytes of a uniformly scaled layout: 4/6/8-bit heads take the
+    single-scale block, FP16 pivot heads their usual block, the request padded to 128 bytes."""
+    offs, pos = [], 0
+    for b in head_bits:
+        offs.append(pos)
+        pos += orc.block_bytes(16, d, d) if int(b) == 16 else orc.uniform_block_bytes(int(b), d, d)
+    return offs, (pos + 127) // 128 * 128
+
+
+def compare_uniform_block(orc, bits, d, got, ref_block, ref_tie, tally: Tally, what=""):
+    """Codes and the one scale of a uniformly scaled head (the rule above, with the single scale
+    in place of the row and column scales); padding stays zero."""
+    got = np.asarray(got, dtype=np.uint8)
+    ref_block = np.asarray(ref_block, dtype=np.uint8)
+    Qg = orc.codes(bits, d, d, got)
+    Qr = orc.codes(bits, d, d, ref_block)
+    diff = np.abs(Qg - Qr)
+    bad = (diff > 1) | ((diff == 1) & ~ref_tie)
+    if bad.any():
+        i, j = np.argwhere(bad)[0]
+        raise AssertionError(f"{what}: {int(bad.sum())} codes differ off a tie, first at ({i},{j}): "
+                             f"gpu {Qg[i, j]} oracle {Qr[i, j]}")
+    tally.codes += Qg.size
+    tally.tie_flips += int((diff == 1).sum())
+    sg = orc.uniform_scale(bits, d, d, got)
+    sr = orc.uniform_scale(bits, d, d, ref_block)
+    rel = abs(sg - sr) / abs(sr)
+    assert rel <= SCALE_RTOL, f"{what}: scale rel error {rel}"
+    tally.max_scale_rel = max(tally.max_scale_rel, float(rel))
+    so = orc.scale_offset(bits, d, d)
+    assert not got[orc.codes_bytes(bits, d, d): so].any()
+    assert not got[so + 4:].any()
+
+
 def compare_o(got, ref, tally: Tally, what=""):
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)

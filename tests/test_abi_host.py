@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol(stq):
         assert hasattr(L, name), name
         assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
     assert sorted(stq.api.EXPORTS) == declared_functions()
-    assert L.stq_abi_version() == 1
+    assert L.stq_abi_version() == 2
 
 
 def test_status_strings(stq):
@@ -61,6 +61,26 @@ def test_layout_matches_oracle_layout(stq, orc, d):
         assert lay.head_bytes(h) == orc.block_bytes(b, d, d)
         assert lay.head_bits_of(h) == b
     assert lay.bytes_per_request % 128 == 0
+
+
+@pytest.mark.parametrize("d", [16, 128])
+def test_uniform_layout_matches_oracle_layout(stq, orc, d):
+    """Uniformly scaled heads hold the codes, padding, one fp32 scale and padding to 128 bytes;
+    FP16 pivot heads keep their block."""
+    bits = [4, 6, 8, 16, 6]
+    lay = stq.Layout(bits, d, scale_mode=stq.SCALES_UNIFORM)
+    pos = 0
+    for h, b in enumerate(bits):
+        nb = orc.block_bytes(16, d, d) if b == 16 else orc.uniform_block_bytes(b, d, d)
+        assert lay.head_offset(h) == pos and lay.head_bytes(h) == nb
+        pos += nb
+    assert lay.bytes_per_request == pos
+    # 6-bit 128 x 128: 12,288 code bytes + 4 scale bytes -> 12,416 (vs 13,312 with row x column scales)
+    if d == 128:
+        assert lay.head_bytes(1) == 12416
+    with pytest.raises(stq.StqError) as e:
+        stq.Layout([4], d, scale_mode=2)
+    assert e.value.status == stq.api.STQ_ERR_INVALID_ARG
 
 
 def test_mixed_workload_bytes_per_token(stq):

@@ -26,8 +26,14 @@ MUTANTS = {
     "row_scale_ignores_column": ("double t = fabs(S[(size_t)i * dv + j] / (double)cf[j]);",
                                  "double t = fabs(S[(size_t)i * dv + j]);"),
     "round_half_up": ("n = (fmod(f, 2.0) == 0.0) ? f : f + 1.0;", "n = f + 1.0;"),
-    "offset_binary_off_by_one": ("u[e] = (int32_t)qv + (1 << (bits - 1));",
-                                 "u[e] = (int32_t)qv + (1 << (bits - 1)) - 1;"),
+    "offset_binary_off_by_one": ("            u[e] = (int32_t)qv + (1 << (bits - 1));",
+                                 "            u[e] = (int32_t)qv + (1 << (bits - 1)) - 1;"),
+    "uniform_offset_off_by_one": ("\n        u[e] = (int32_t)qv + (1 << (bits - 1));",
+                                  "\n        u[e] = (int32_t)qv + (1 << (bits - 1)) - 1;"),
+    "uniform_scale_without_qmax": ("double s = m / (double)qmax;", "double s = m;"),
+    "uniform_scale_never_one": ("    if (s == 0.0) s = 1.0;\n    float sf", "    float sf"),
+    "uniform_dequant_offset": ("S[e] = s * (double)(u[e] - (1 << (bits - 1)));",
+                               "S[e] = s * (double)(u[e] - (1 << (bits - 1)) + 1);"),
     "pack_msb_first": ("out[bit / 8] |= (uint8_t)(1u << (bit % 8));",
                        "out[bit / 8] |= (uint8_t)(1u << (7 - bit % 8));"),
     "half_truncates": ("double r = orc_round_half_even(ldexp(a, 10 - e));",
