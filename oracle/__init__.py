@@ -30,6 +30,7 @@ _LIB_PATH = os.path.join(_OUT_DIR, "libstq_oracle.so")
 
 OK, EINVAL, ENONFINITE = 0, 1, 4
 GATE_SCALAR, GATE_CHANNEL, GATE_CHANNEL_DECAY_FIRST = 0, 1, 2
+SCALE_F32, SCALE_BF16 = 0, 1  # storage format of the row and column scales
 TIE_DELTA = 1e-3
 
 _lock = threading.Lock()
@@ -84,6 +85,16 @@ def lib():
             L.orc_dequantize_uniform.argtypes, L.orc_dequantize_uniform.restype = [i32, i32, i32, P, P], i32
             L.orc_decode_step_uniform.argtypes = [i32, i32, i32, i32, P, P, P, P, f64, P, P, P, P, f64]
             L.orc_decode_step_uniform.restype = i32
+            L.orc_block_bytes_s.argtypes, L.orc_block_bytes_s.restype = [i32, i32, i32, i32], sz
+            L.orc_bf16_to_double.argtypes, L.orc_bf16_to_double.restype = [ctypes.c_uint16], f64
+            L.orc_double_to_bf16.argtypes, L.orc_double_to_bf16.restype = [f64], ctypes.c_uint16
+            L.orc_quantize_s.argtypes = [i32, i32, i32, i32, P, P, P, P, P, P, P, P, f64]
+            L.orc_quantize_s.restype = i32
+            L.orc_dequantize_s.argtypes, L.orc_dequantize_s.restype = [i32, i32, i32, i32, P, P], i32
+            L.orc_decode_step_s.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, f64, P, P, P, P, P, P, P, f64]
+            L.orc_decode_step_s.restype = i32
+            L.orc_prefill_seq_s.argtypes = [i32, i32, i32, i32, i32, P, i32, i32, P, P, P, P, P, P, P, P, P, P, f64]
+            L.orc_prefill_seq_s.restype = i32
             _lib = L
     return _lib
 
@@ -133,6 +144,14 @@ def unpack(bits: int, n: int, data) -> np.ndarray:
     u = np.zeros(n, dtype=np.int32)
     lib().orc_unpack(bits, n, _p(data), _p(u))
     return u
+
+
+def bf16_to_double(h: int) -> float:
+    return lib().orc_bf16_to_double(int(h))
+
+
+def double_to_bf16(x: float) -> int:
+    return lib().orc_double_to_bf16(float(x))
 
 
 def half_to_double(h: int) -> float:
@@ -300,3 +319,83 @@ def decode_step_uniform(bits: int, gate: int, block, q, k, v, beta: float, alpha
     st = lib().orc_decode_step_uniform(bits, dk, dv, gate, _p(blk), _p(_f64(q)), _p(_f64(k)), _p(_f64(v)),
                                        float(beta), _p(a), _p(o), _p(x), _p(tie), float(delta))
     return dict(block=blk, o=o, x=x, tie=tie.astype(bool), status=st)
+
+
+# ---------------------------------------------------------------------------------------------
+# Scale storage formats (fp32, or bf16 for 16-bit scales; see stq_oracle.c)
+# ---------------------------------------------------------------------------------------------
+
+def block_bytes_s(bits: int, sfmt: int, dk: int, dv: int) -> int:
+    return int(lib().orc_block_bytes_s(bits, sfmt, dk, dv))
+
+
+def quantize_s(bits: int, sfmt: int, S, w=None, c_given=None, r_given=None, delta: float = TIE_DELTA):
+    """Quantize with scales stored in format sfmt; c_given / r_given replace the fitted stored
+    scales. Returns (block, x, tie, scale_tie, status); scale_tie holds dk row flags, then dv
+    column flags."""
+    S = _f64(S)
+    dk, dv = S.shape
+    w = _f64(np.ones(dk) if w is None else w)
+    block = np.zeros(block_bytes_s(bits, sfmt, dk, dv), dtype=np.uint8)
+    x = np.zeros((dk, dv))
+    tie = np.zeros((dk, dv), dtype=np.uint8)
+    stie = np.zeros(dk + dv, dtype=np.uint8)
+    cg = None if c_given is None else _f64(c_given)
+    rg = None if r_given is None else _f64(r_given)
+    st = lib().orc_quantize_s(bits, sfmt, dk, dv, _p(S), _p(w), _p(cg), _p(rg), _p(block), _p(x), _p(tie),
+                              _p(stie), float(delta))
+    return block, x, tie.astype(bool), stie.astype(bool), st
+
+
+def dequantize_s(bits: int, sfmt: int, dk: int, dv: int, block) -> np.ndarray:
+    block = np.ascontiguousarray(np.asarray(block, dtype=np.uint8))
+    assert block.size >= block_bytes_s(bits, sfmt, dk, dv)
+    S = np.zeros((dk, dv))
+    st = lib().orc_dequantize_s(bits, sfmt, dk, dv, _p(block), _p(S))
+    assert st == OK
+    return S
+
+
+def scales_s(bits: int, sfmt: int, dk: int, dv: int, block):
+    """(r, c) stored scales of a head block as fp64 values."""
+    if sfmt == SCALE_F32:
+        r, c = scales(bits, dk, dv, block)
+        return r.astype(np.float64), c.astype(np.float64)
+    off = scale_offset(bits, dk, dv)
+    raw = np.asarray(block, dtype=np.uint8)[off: off + 2 * (dk + dv)].view(np.uint16)
+    vals = np.array([bf16_to_double(int(h)) for h in raw])
+    return vals[:dk], vals[dk:]
+
+
+def decode_step_s(bits: int, sfmt: int, gate: int, block, q, k, v, beta: float, alpha, w, dk: int, dv: int,
+                  delta: float = TIE_DELTA):
+    """One decode step on a copy of ``block`` with scales in format sfmt. Returns dict(block, o,
+    S_new (fp64 before requantization), x, tie, scale_tie, status)."""
+    blk = np.ascontiguousarray(np.asarray(block, dtype=np.uint8)).copy()
+    o = np.zeros(dv, dtype=np.float32)
+    S_new = np.zeros((dk, dv))
+    x = np.zeros((dk, dv))
+    tie = np.zeros((dk, dv), dtype=np.uint8)
+    stie = np.zeros(dk + dv, dtype=np.uint8)
+    a = _f64(np.atleast_1d(alpha))
+    wv = _f64(np.ones(dk) if w is None else w)
+    st = lib().orc_decode_step_s(bits, sfmt, dk, dv, gate, _p(blk), _p(_f64(q)), _p(_f64(k)), _p(_f64(v)),
+                                 float(beta), _p(a), _p(wv), _p(o), _p(S_new), _p(x), _p(tie), _p(stie),
+                                 float(delta))
+    return dict(block=blk, o=o, S_new=S_new, x=x, tie=tie.astype(bool), scale_tie=stie.astype(bool), status=st)
+
+
+def prefill_seq_s(bits: int, sfmt: int, gate: int, block, q, k, v, beta, alpha, w, chunk: int, dk: int, dv: int,
+                  delta: float = TIE_DELTA):
+    """Sequential chunked prefill on a copy of ``block`` with scales in format sfmt."""
+    blk = np.ascontiguousarray(np.asarray(block, dtype=np.uint8)).copy()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T = q.shape[0]
+    o = np.zeros((T, dv), dtype=np.float32)
+    x = np.zeros((dk, dv))
+    tie = np.zeros((dk, dv), dtype=np.uint8)
+    stie = np.zeros(dk + dv, dtype=np.uint8)
+    st = lib().orc_prefill_seq_s(bits, sfmt, dk, dv, gate, _p(blk), T, chunk, _p(q), _p(k), _p(v),
+                                 _p(_f64(beta)), _p(_f64(alpha)), _p(_f64(w)), _p(o), _p(x), _p(tie), _p(stie),
+                                 float(delta))
+    return dict(block=blk, o=o, x=x, tie=tie.astype(bool), scale_tie=stie.astype(bool), status=st)

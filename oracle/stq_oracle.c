@@ -24,7 +24,8 @@
  *   bits in {4,6,8}: packed codes, code (i,j) occupies bits [b*n, b*n+b) of a little-endian
  *     bitstream, n = i*dv + j, bit k of the stream is bit (k mod 8) of byte k/8; each code is
  *     stored offset-binary u = Q + 2^(b-1); then zero padding to a 16-byte boundary; then
- *     r[dk] fp32, then c[dv] fp32; then zero padding to a 128-byte boundary.
+ *     r[dk], then c[dv], each fp32 (or bf16 in the 16-bit scale format); then zero padding to
+ *     a 128-byte boundary.
  *   bits == 16 (pivot): S as fp16 row-major, padded to 128 bytes.
  */
 #include <math.h>
@@ -83,12 +84,17 @@ size_t orc_scale_offset(int bits, int dk, int dv)
     return round_up(orc_codes_bytes(bits, dk, dv), 16);
 }
 
-size_t orc_block_bytes(int bits, int dk, int dv)
+static int valid_sfmt(int sfmt) { return sfmt == ORC_SCALE_F32 || sfmt == ORC_SCALE_BF16; }
+static size_t scale_bytes(int sfmt) { return sfmt == ORC_SCALE_BF16 ? 2 : 4; }
+
+size_t orc_block_bytes_s(int bits, int sfmt, int dk, int dv)
 {
-    if (!valid_bits(bits) || dk < 1 || dv < 1) return 0;
+    if (!valid_bits(bits) || !valid_sfmt(sfmt) || dk < 1 || dv < 1) return 0;
     if (bits == 16) return round_up((size_t)2 * dk * dv, 128);
-    return round_up(orc_scale_offset(bits, dk, dv) + (size_t)4 * dk + (size_t)4 * dv, 128);
+    return round_up(orc_scale_offset(bits, dk, dv) + scale_bytes(sfmt) * ((size_t)dk + (size_t)dv), 128);
 }
+
+size_t orc_block_bytes(int bits, int dk, int dv) { return orc_block_bytes_s(bits, ORC_SCALE_F32, dk, dv); }
 
 /* ------------------------------------------------------------------------------------------ */
 /* Packing: offset-binary codes into a little-endian bitstream                                */
@@ -173,6 +179,61 @@ static double half_units(double a)
 }
 
 /* ------------------------------------------------------------------------------------------ */
+/* bfloat16, from the format's definition (1 sign, 8 exponent bits biased by 127, 7 fraction  */
+/* bits; exponent 0 = subnormal with quantum 2^-133; exponent 255 = inf/NaN): the upper half  */
+/* of an IEEE binary32 pattern.                                                               */
+/* ------------------------------------------------------------------------------------------ */
+
+double orc_bf16_to_double(uint16_t h)
+{
+    int s = (h >> 15) & 1;
+    int e = (h >> 7) & 0xff;
+    int m = h & 0x7f;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -133);
+    else if (e == 255)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(128 + m), e - 134); /* (1 + m/128) * 2^(e-127) */
+    return s ? -v : v;
+}
+
+uint16_t orc_double_to_bf16(double x)
+{
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double a = fabs(x);
+    if (isnan(x)) return 0x7fc0;
+    /* the largest finite value is (2 - 2^-7) 2^127; half an ulp above it rounds to inf */
+    if (a >= ldexp(255.0 + 0.5, 120)) return sign | 0x7f80;
+    if (a < ldexp(1.0, -126)) {
+        double r = orc_round_half_even(ldexp(a, 133)); /* subnormal: multiple of 2^-133 */
+        return sign | (uint16_t)r;
+    }
+    int E;
+    frexp(a, &E);  /* a = f * 2^E, f in [0.5, 1) */
+    int e = E - 1; /* a in [2^e, 2^(e+1)) */
+    double r = orc_round_half_even(ldexp(a, 7 - e)); /* significand in [128, 256] */
+    if (r == 256.0) {
+        r = 128.0;
+        e += 1;
+    }
+    if (e > 127) return sign | 0x7f80;
+    return sign | (uint16_t)(((e + 127) << 7) | ((int)r - 128));
+}
+
+/* Position of a positive value on the bf16 grid in units of the quantum at that magnitude:
+ * used only to flag scale rounding near-ties. */
+static double bf16_units(double a)
+{
+    a = fabs(a);
+    if (a < ldexp(1.0, -126)) return ldexp(a, 133);
+    int E;
+    frexp(a, &E);
+    return ldexp(a, 7 - (E - 1));
+}
+
+/* ------------------------------------------------------------------------------------------ */
 /* Little-endian fp32 / u16 storage                                                           */
 /* ------------------------------------------------------------------------------------------ */
 
@@ -191,6 +252,32 @@ static uint16_t load_u16(const uint8_t *p)
     return h;
 }
 
+/* The value a scale takes once stored in format sfmt (fp32 or bf16, round half to even). */
+static double stored_scale(int sfmt, double v)
+{
+    if (sfmt == ORC_SCALE_BF16) return orc_bf16_to_double(orc_double_to_bf16(v));
+    return (double)(float)v;
+}
+/* Distance of v from the nearest rounding tie of format sfmt, in quanta of that format. */
+static double scale_tie_distance(int sfmt, double v)
+{
+    if (sfmt == ORC_SCALE_BF16) return tie_distance(bf16_units(v));
+    int E;
+    frexp(fabs(v), &E);
+    return tie_distance(ldexp(fabs(v), 23 - (E - 1)));
+}
+static void store_scale(int sfmt, uint8_t *p, double v)
+{
+    if (sfmt == ORC_SCALE_BF16)
+        store_u16(p, orc_double_to_bf16(v));
+    else
+        store_f32(p, (float)v);
+}
+static double load_scale(int sfmt, const uint8_t *p)
+{
+    return sfmt == ORC_SCALE_BF16 ? orc_bf16_to_double(load_u16(p)) : (double)load_f32(p);
+}
+
 /* ------------------------------------------------------------------------------------------ */
 /* Quantizer: impact-weighted column scale, row scale from the column-normalised max,         */
 /* round-half-to-even codes.                                                                  */
@@ -199,12 +286,14 @@ static uint16_t load_u16(const uint8_t *p)
 /* sets the quantization step; the column scale is fitted by weighted least squares in which  */
 /* high-impact rows weigh more; the two are fitted jointly.                                   */
 /* Specification (READING c5/c6/c8: column first, then the row from the stored column scale,  */
-/* one pass; fp32 storage):                                                                   */
+/* one pass; fp32 storage, or bf16 in the 16-bit scale format):                               */
 /*   W     = sum_i w_i                                                                        */
-/*   c_j   = sqrt( sum_i w_i S_ij^2 / W ),   c_j := 1 if it is 0,   c~_j = fp32(c_j)           */
+/*   c_j   = sqrt( sum_i w_i S_ij^2 / W ),   c_j := 1 if it is 0,   c~_j = stored(c_j)         */
 /*   t_ij  = S_ij / c~_j                                                                      */
-/*   r_i   = max_j |t_ij| / qmax,            r_i := 1 if it is 0,   r~_i = fp32(r_i)           */
+/*   r_i   = max_j |t_ij| / qmax,            r_i := 1 if it is 0,   r~_i = stored(r_i)         */
 /*   x_ij  = t_ij / r~_i,  Q_ij = clamp(round_half_even(x_ij), -qmax, qmax)                   */
+/* stored() rounds half to even to the format. With bf16 scales r~_i may sit just below r_i,  */
+/* so |x| may pass qmax by a fraction of a step: the clamp takes it back.                     */
 /* Pivot heads ([P1 方法], [P5 时间维度]: the highest-risk heads stay FP16): S -> fp16, RNE.    */
 /* ------------------------------------------------------------------------------------------ */
 
@@ -215,15 +304,22 @@ static int check_weights(int dk, const double *w)
     return ORC_OK;
 }
 
-int orc_quantize(int bits, int dk, int dv, const double *S, const double *w, uint8_t *block,
-                 double *x_out, uint8_t *tie_out, double delta)
+/* Quantize one head. sfmt: ORC_SCALE_F32 or ORC_SCALE_BF16. c_given / r_given (optional):
+ * stored column / row scale values to use instead of fitting them (used by the tests to
+ * requantize with the scales another implementation chose at a scale rounding near-tie).
+ * stie_out (optional, dk + dv flags: rows, then columns): the fitted scale lay within `delta`
+ * quanta of a rounding tie of the storage format. */
+int orc_quantize_s(int bits, int sfmt, int dk, int dv, const double *S, const double *w,
+                   const double *c_given, const double *r_given, uint8_t *block, double *x_out,
+                   uint8_t *tie_out, uint8_t *stie_out, double delta)
 {
-    if (!valid_bits(bits) || dk < 1 || dv < 1) return ORC_EINVAL;
+    if (!valid_bits(bits) || !valid_sfmt(sfmt) || dk < 1 || dv < 1) return ORC_EINVAL;
     size_t n = (size_t)dk * dv;
     int nonfinite = 0;
     for (size_t e = 0; e < n; ++e)
         if (!isfinite(S[e])) nonfinite = 1;
-    memset(block, 0, orc_block_bytes(bits, dk, dv));
+    memset(block, 0, orc_block_bytes_s(bits, sfmt, dk, dv));
+    if (stie_out) memset(stie_out, 0, (size_t)dk + (size_t)dv);
 
     if (bits == 16) {
         for (size_t e = 0; e < n; ++e) {
@@ -239,36 +335,47 @@ int orc_quantize(int bits, int dk, int dv, const double *S, const double *w, uin
     if (check_weights(dk, w) != ORC_OK) return ORC_EINVAL;
     int qmax = orc_qmax(bits);
     size_t soff = orc_scale_offset(bits, dk, dv);
-    float *cf = (float *)malloc(sizeof(float) * dv);
-    float *rf = (float *)malloc(sizeof(float) * dk);
+    size_t sb = scale_bytes(sfmt);
+    double *cs = (double *)malloc(sizeof(double) * dv);
+    double *rs = (double *)malloc(sizeof(double) * dk);
     int32_t *u = (int32_t *)malloc(sizeof(int32_t) * n);
 
     double W = 0.0;
     for (int i = 0; i < dk; ++i) W += w[i];
 
     for (int j = 0; j < dv; ++j) {
-        double acc = 0.0;
-        for (int i = 0; i < dk; ++i) acc += w[i] * S[(size_t)i * dv + j] * S[(size_t)i * dv + j];
-        double c = sqrt(acc / W);
-        if (c == 0.0) c = 1.0;
-        cf[j] = (float)c;
-        if (!isfinite(cf[j])) nonfinite = 1;
+        if (c_given) {
+            cs[j] = c_given[j];
+        } else {
+            double acc = 0.0;
+            for (int i = 0; i < dk; ++i) acc += w[i] * S[(size_t)i * dv + j] * S[(size_t)i * dv + j];
+            double c = sqrt(acc / W);
+            if (c == 0.0) c = 1.0;
+            cs[j] = stored_scale(sfmt, c);
+            if (stie_out) stie_out[dk + j] = isfinite(c) && scale_tie_distance(sfmt, c) <= delta;
+        }
+        if (!isfinite(cs[j])) nonfinite = 1;
     }
     for (int i = 0; i < dk; ++i) {
-        double m = 0.0;
-        for (int j = 0; j < dv; ++j) {
-            double t = fabs(S[(size_t)i * dv + j] / (double)cf[j]);
-            if (t > m) m = t;
+        if (r_given) {
+            rs[i] = r_given[i];
+        } else {
+            double m = 0.0;
+            for (int j = 0; j < dv; ++j) {
+                double t = fabs(S[(size_t)i * dv + j] / cs[j]);
+                if (t > m) m = t;
+            }
+            double r = m / (double)qmax;
+            if (r == 0.0) r = 1.0;
+            rs[i] = stored_scale(sfmt, r);
+            if (stie_out) stie_out[i] = isfinite(r) && scale_tie_distance(sfmt, r) <= delta;
         }
-        double r = m / (double)qmax;
-        if (r == 0.0) r = 1.0;
-        rf[i] = (float)r;
-        if (!isfinite(rf[i]) || rf[i] == 0.0f) nonfinite = 1;
+        if (!isfinite(rs[i]) || rs[i] == 0.0) nonfinite = 1;
     }
     for (int i = 0; i < dk; ++i) {
         for (int j = 0; j < dv; ++j) {
             size_t e = (size_t)i * dv + j;
-            double x = (S[e] / (double)cf[j]) / (double)rf[i];
+            double x = (S[e] / cs[j]) / rs[i];
             double qv = orc_round_half_even(x);
             if (qv > qmax) qv = qmax;
             if (qv < -qmax) qv = -qmax;
@@ -279,18 +386,24 @@ int orc_quantize(int bits, int dk, int dv, const double *S, const double *w, uin
         }
     }
     orc_pack(bits, n, u, block);
-    for (int i = 0; i < dk; ++i) store_f32(block + soff + 4 * (size_t)i, rf[i]);
-    for (int j = 0; j < dv; ++j) store_f32(block + soff + 4 * (size_t)dk + 4 * (size_t)j, cf[j]);
-    free(cf);
-    free(rf);
+    for (int i = 0; i < dk; ++i) store_scale(sfmt, block + soff + sb * (size_t)i, rs[i]);
+    for (int j = 0; j < dv; ++j) store_scale(sfmt, block + soff + sb * ((size_t)dk + (size_t)j), cs[j]);
+    free(cs);
+    free(rs);
     free(u);
     return nonfinite ? ORC_ENONFINITE : ORC_OK;
 }
 
-/* Dequantize: S_ij = r~_i * c~_j * Q_ij (fp64), or the fp16 value of a pivot head. */
-int orc_dequantize(int bits, int dk, int dv, const uint8_t *block, double *S)
+int orc_quantize(int bits, int dk, int dv, const double *S, const double *w, uint8_t *block,
+                 double *x_out, uint8_t *tie_out, double delta)
 {
-    if (!valid_bits(bits) || dk < 1 || dv < 1) return ORC_EINVAL;
+    return orc_quantize_s(bits, ORC_SCALE_F32, dk, dv, S, w, NULL, NULL, block, x_out, tie_out, NULL, delta);
+}
+
+/* Dequantize: S_ij = r~_i * c~_j * Q_ij (fp64), or the fp16 value of a pivot head. */
+int orc_dequantize_s(int bits, int sfmt, int dk, int dv, const uint8_t *block, double *S)
+{
+    if (!valid_bits(bits) || !valid_sfmt(sfmt) || dk < 1 || dv < 1) return ORC_EINVAL;
     size_t n = (size_t)dk * dv;
     if (bits == 16) {
         for (size_t e = 0; e < n; ++e) S[e] = orc_half_to_double(load_u16(block + 2 * e));
@@ -299,10 +412,11 @@ int orc_dequantize(int bits, int dk, int dv, const uint8_t *block, double *S)
     size_t soff = orc_scale_offset(bits, dk, dv);
     int32_t *u = (int32_t *)malloc(sizeof(int32_t) * n);
     orc_unpack(bits, n, block, u);
+    size_t sb = scale_bytes(sfmt);
     for (int i = 0; i < dk; ++i) {
-        double r = (double)load_f32(block + soff + 4 * (size_t)i);
+        double r = load_scale(sfmt, block + soff + sb * (size_t)i);
         for (int j = 0; j < dv; ++j) {
-            double c = (double)load_f32(block + soff + 4 * (size_t)dk + 4 * (size_t)j);
+            double c = load_scale(sfmt, block + soff + sb * ((size_t)dk + (size_t)j));
             size_t e = (size_t)i * dv + j;
             double qv = (double)(u[e] - (1 << (bits - 1)));
             S[e] = r * c * qv;
@@ -310,6 +424,11 @@ int orc_dequantize(int bits, int dk, int dv, const uint8_t *block, double *S)
     }
     free(u);
     return ORC_OK;
+}
+
+int orc_dequantize(int bits, int dk, int dv, const uint8_t *block, double *S)
+{
+    return orc_dequantize_s(bits, ORC_SCALE_F32, dk, dv, block, S);
 }
 
 /* ------------------------------------------------------------------------------------------ */
@@ -363,19 +482,19 @@ void orc_update(int dk, int dv, int gate, double *S, const double *q, const doub
  * o is emitted as fp32 (RNE of the fp64 value). S_new_out (optional) receives the fp64
  * updated state before requantization. x_out / tie_out (optional) receive the requantizer's
  * real-valued codes and near-tie flags. */
-int orc_decode_step(int bits, int dk, int dv, int gate, uint8_t *block, const double *q,
-                    const double *k, const double *v, double beta, const double *alpha,
-                    const double *w, float *o, double *S_new_out, double *x_out,
-                    uint8_t *tie_out, double delta)
+int orc_decode_step_s(int bits, int sfmt, int dk, int dv, int gate, uint8_t *block, const double *q,
+                      const double *k, const double *v, double beta, const double *alpha,
+                      const double *w, float *o, double *S_new_out, double *x_out,
+                      uint8_t *tie_out, uint8_t *stie_out, double delta)
 {
-    if (!valid_bits(bits) || dk < 1 || dv < 1) return ORC_EINVAL;
+    if (!valid_bits(bits) || !valid_sfmt(sfmt) || dk < 1 || dv < 1) return ORC_EINVAL;
     if (gate != ORC_GATE_SCALAR && gate != ORC_GATE_CHANNEL && gate != ORC_GATE_CHANNEL_DECAY_FIRST)
         return ORC_EINVAL;
     if (bits != 16 && check_weights(dk, w) != ORC_OK) return ORC_EINVAL;
     size_t n = (size_t)dk * dv;
     double *S = (double *)malloc(sizeof(double) * n);
     double *od = (double *)malloc(sizeof(double) * dv);
-    orc_dequantize(bits, dk, dv, block, S);
+    orc_dequantize_s(bits, sfmt, dk, dv, block, S);
     orc_update(dk, dv, gate, S, q, k, v, beta, alpha, od);
     int nonfinite = 0;
     for (int j = 0; j < dv; ++j) {
@@ -383,11 +502,20 @@ int orc_decode_step(int bits, int dk, int dv, int gate, uint8_t *block, const do
         if (!isfinite(o[j])) nonfinite = 1;
     }
     if (S_new_out) memcpy(S_new_out, S, sizeof(double) * n);
-    int st = orc_quantize(bits, dk, dv, S, w, block, x_out, tie_out, delta);
+    int st = orc_quantize_s(bits, sfmt, dk, dv, S, w, NULL, NULL, block, x_out, tie_out, stie_out, delta);
     free(S);
     free(od);
     if (st != ORC_OK) return st;
     return nonfinite ? ORC_ENONFINITE : ORC_OK;
+}
+
+int orc_decode_step(int bits, int dk, int dv, int gate, uint8_t *block, const double *q,
+                    const double *k, const double *v, double beta, const double *alpha,
+                    const double *w, float *o, double *S_new_out, double *x_out,
+                    uint8_t *tie_out, double delta)
+{
+    return orc_decode_step_s(bits, ORC_SCALE_F32, dk, dv, gate, block, q, k, v, beta, alpha, w, o, S_new_out,
+                             x_out, tie_out, NULL, delta);
 }
 
 /* ------------------------------------------------------------------------------------------ */
@@ -400,12 +528,12 @@ int orc_decode_step(int bits, int dk, int dv, int gate, uint8_t *block, const do
 /* Layouts: q,k [T][dk], v [T][dv], beta [T], alpha [T] (scalar gate) or [T][dk], o [T][dv].  */
 /* ------------------------------------------------------------------------------------------ */
 
-int orc_prefill_seq(int bits, int dk, int dv, int gate, uint8_t *block, int T, int chunk,
-                    const double *q, const double *k, const double *v, const double *beta,
-                    const double *alpha, const double *w, float *o, double *x_out,
-                    uint8_t *tie_out, double delta)
+int orc_prefill_seq_s(int bits, int sfmt, int dk, int dv, int gate, uint8_t *block, int T, int chunk,
+                      const double *q, const double *k, const double *v, const double *beta,
+                      const double *alpha, const double *w, float *o, double *x_out,
+                      uint8_t *tie_out, uint8_t *stie_out, double delta)
 {
-    if (!valid_bits(bits) || dk < 1 || dv < 1 || T < 0 || chunk < 1) return ORC_EINVAL;
+    if (!valid_bits(bits) || !valid_sfmt(sfmt) || dk < 1 || dv < 1 || T < 0 || chunk < 1) return ORC_EINVAL;
     if (bits != 16 && check_weights(dk, w) != ORC_OK) return ORC_EINVAL;
     size_t n = (size_t)dk * dv;
     int na = (gate == ORC_GATE_SCALAR) ? 1 : dk;
@@ -414,7 +542,7 @@ int orc_prefill_seq(int bits, int dk, int dv, int gate, uint8_t *block, int T, i
     int status = ORC_OK;
     for (int c0 = 0; c0 < T; c0 += chunk) {
         int c1 = c0 + chunk < T ? c0 + chunk : T;
-        orc_dequantize(bits, dk, dv, block, S);
+        orc_dequantize_s(bits, sfmt, dk, dv, block, S);
         for (int t = c0; t < c1; ++t) {
             orc_update(dk, dv, gate, S, q + (size_t)t * dk, k + (size_t)t * dk,
                        v + (size_t)t * dv, beta[t], alpha + (size_t)t * na, od);
@@ -423,13 +551,22 @@ int orc_prefill_seq(int bits, int dk, int dv, int gate, uint8_t *block, int T, i
                 if (!isfinite(o[(size_t)t * dv + j])) status = ORC_ENONFINITE;
             }
         }
-        int st = orc_quantize(bits, dk, dv, S, w, block, x_out, tie_out, delta);
+        int st = orc_quantize_s(bits, sfmt, dk, dv, S, w, NULL, NULL, block, x_out, tie_out, stie_out, delta);
         if (st == ORC_EINVAL) status = st;
         if (st == ORC_ENONFINITE && status == ORC_OK) status = st;
     }
     free(S);
     free(od);
     return status;
+}
+
+int orc_prefill_seq(int bits, int dk, int dv, int gate, uint8_t *block, int T, int chunk,
+                    const double *q, const double *k, const double *v, const double *beta,
+                    const double *alpha, const double *w, float *o, double *x_out,
+                    uint8_t *tie_out, double delta)
+{
+    return orc_prefill_seq_s(bits, ORC_SCALE_F32, dk, dv, gate, block, T, chunk, q, k, v, beta, alpha, w, o,
+                             x_out, tie_out, NULL, delta);
 }
 
 /* ------------------------------------------------------------------------------------------ */

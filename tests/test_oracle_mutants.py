@@ -22,8 +22,12 @@ MUTANTS = {
                                  "double a = 1.0;"),
     "column_weight_index": ("acc += w[i] * S[(size_t)i * dv + j] * S[(size_t)i * dv + j];",
                             "acc += w[j % dk] * S[(size_t)i * dv + j] * S[(size_t)i * dv + j];"),
+    "bf16_truncates": ("double r = orc_round_half_even(ldexp(a, 7 - e));", "double r = floor(ldexp(a, 7 - e));"),
+    "bf16_scale_stored_as_fp32": ("if (sfmt == ORC_SCALE_BF16) return orc_bf16_to_double(orc_double_to_bf16(v));",
+                                  "if (sfmt == ORC_SCALE_BF16) return (double)(float)v;"),
+    "row_scale_from_unrounded_column": ("cs[j] = stored_scale(sfmt, c);\n", "cs[j] = c;\n"),
     "column_scale_no_sqrt": ("double c = sqrt(acc / W);", "double c = acc / W;"),
-    "row_scale_ignores_column": ("double t = fabs(S[(size_t)i * dv + j] / (double)cf[j]);",
+    "row_scale_ignores_column": ("double t = fabs(S[(size_t)i * dv + j] / cs[j]);",
                                  "double t = fabs(S[(size_t)i * dv + j]);"),
     "round_half_up": ("n = (fmod(f, 2.0) == 0.0) ? f : f + 1.0;", "n = f + 1.0;"),
     "offset_binary_off_by_one": ("            u[e] = (int32_t)qv + (1 << (bits - 1));",

@@ -597,3 +597,178 @@ def test_uniform_decode_step_is_update_then_uniform_requantization(orc):
     assert np.array_equal(res["o"], o.astype(np.float32))
     ref_blk, _, _, _ = orc.quantize_uniform(8, S_new)
     assert np.array_equal(res["block"], ref_blk)
+
+
+# ----------------------------------------------------------------------------------------------
+# 16-bit (bf16) scale storage
+# ----------------------------------------------------------------------------------------------
+
+def _fp32_rne_to_bf16(x32):
+    """Textbook round-to-nearest-even of binary32 patterns to their upper 16 bits (add 0x7fff
+    plus the lowest kept bit, then truncate): correct for every finite input."""
+    u = np.asarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def test_bf16_decode_all_patterns_are_fp32_upper_halves(orc):
+    pats = np.arange(65536, dtype=np.uint32)
+    with np.errstate(invalid="ignore"):
+        ref = (pats << 16).astype(np.uint32).view(np.float32).astype(np.float64)
+    got = np.array([orc.bf16_to_double(int(h)) for h in pats])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def test_bf16_encode_matches_fp32_rne_on_fp32_values(orc):
+    """For values exactly representable in fp32, rounding to bf16 is the textbook bit rounding;
+    exact ties go to the even pattern, and 255.5 * 2^120 (half an ulp above the largest finite
+    value) overflows to infinity."""
+    rng = np.random.default_rng(21)
+    vals = [0.0, 1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8), 2.0 ** -133, 2.0 ** -134,
+            3 * 2.0 ** -134, 2.0 ** -126, 255.0 * 2.0 ** 120, 255.5 * 2.0 ** 120 - 2.0 ** 104, 255.5 * 2.0 ** 120]
+    for e in (-130, -126, -20, -1, 0, 7, 100, 126):
+        for m in (0, 1, 2, 126, 127):
+            vals.append((128 + m + 0.5) * 2.0 ** (e - 7))  # exact ties
+    vals += list((rng.standard_normal(3000) * 10.0 ** rng.uniform(-30, 30, 3000)).astype(np.float32))
+    x32 = np.array(vals, dtype=np.float32)
+    assert np.array_equal(x32.astype(np.float64), np.array(vals, dtype=np.float64))  # all fp32-exact
+    ref = _fp32_rne_to_bf16(x32)
+    for x, h in zip(vals, ref):
+        assert orc.double_to_bf16(float(x)) == int(h), x
+    assert orc.double_to_bf16(255.5 * 2.0 ** 120) == 0x7F80
+    assert orc.double_to_bf16(1.0 + 2.0 ** -8) == 0x3F80 and orc.double_to_bf16(1.0 + 3 * 2.0 ** -8) == 0x3F82
+
+
+def test_bf16_encode_rounds_the_exact_value_once(orc):
+    """READING: a scale is rounded to bf16 from its exact value in one step, not through fp32: just
+    above a bf16 tie by less than an fp32 half-ulp rounds up."""
+    assert orc.double_to_bf16(1.0 + 2.0 ** -8 + 2.0 ** -40) == 0x3F81
+    assert orc.double_to_bf16(1.0 + 2.0 ** -8 - 2.0 ** -40) == 0x3F80
+
+
+def test_bf16_scale_block_layout(orc):
+    """Codes, padding to 16 bytes, r[dk] and c[dv] in bf16, padding to 128 bytes: at 128 x 128 a
+    6-bit head is 12,800 bytes, 5.12x smaller than fp32, and with 1.4% FP16 pivot heads the state
+    is 5.01x smaller (the pages report 5.03x / 5.08x at 6 bits)."""
+    for bits, want in ((4, 8704), (6, 12800), (8, 16896)):
+        assert orc.block_bytes_s(bits, orc.SCALE_BF16, 128, 128) == want
+        assert orc.block_bytes_s(bits, orc.SCALE_F32, 128, 128) == orc.block_bytes(bits, 128, 128)
+    assert orc.block_bytes_s(16, orc.SCALE_BF16, 128, 128) == 32768
+    assert abs(65536 / 12800 - 5.12) < 1e-12
+    mixed = 0.986 * 12800 + 0.014 * 32768
+    assert abs(65536 / mixed - 5.01) < 0.01
+    assert orc.block_bytes_s(6, 2, 128, 128) == 0  # unknown format
+
+
+# rows g with max |g| = qmax and sum g^2 = 8 * 4^k: a circulant of g has column RMS exactly 2^k
+EXACT_ROWS = {4: ([7, 5, 5, 3, 3, 3, 1, 1], 2), 6: ([31, 23, 17, 13, 9, 3, 3, 1], 4),
+              8: ([127, 121, 44, 7, 3, 2, 0, 0], 6)}
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("sfmt", [0, 1])
+def test_scales_exact_round_trip(orc, bits, sfmt):
+    """S = circ(+-g) diag(c) with bf16-exact c and equal weights: the fitted column scale is
+    2^k c_j, the row scale 2^-k, both exact in either format, the codes are the integers and
+    dequantization gives S back exactly."""
+    g, k = EXACT_ROWS[bits]
+    assert sum(x * x for x in g) == 8 * 4 ** k and max(g) == orc.qmax(bits)
+    d = 8
+    rng = np.random.default_rng(bits * 10 + sfmt)
+    G = np.array([[g[(j - i) % d] for j in range(d)] for i in range(d)], dtype=np.float64)
+    G *= np.where(rng.random((d, d)) < 0.5, -1.0, 1.0)
+    c = (128 + rng.integers(0, 128, d)) / 128.0 * 2.0 ** rng.integers(-6, 6, d)
+    S = G * c[None, :]
+    block, x, tie, stie, st = orc.quantize_s(bits, sfmt, S, np.full(d, 0.7))
+    assert st == orc.OK
+    r_s, c_s = orc.scales_s(bits, sfmt, d, d, block)
+    assert np.array_equal(c_s, c * 2.0 ** k) and np.array_equal(r_s, np.full(d, 2.0 ** -k))
+    assert np.array_equal(orc.codes(bits, d, d, block), G.astype(int))
+    assert np.array_equal(orc.dequantize_s(bits, sfmt, d, d, block), S)
+    assert not stie.any()
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_bf16_scales_bounds(orc, bits):
+    """On an outlier state: every stored scale is a bf16 value within half a bf16 ulp of its
+    defining quantity (the column's impact-weighted RMS; the row's largest magnitude over the
+    stored column scales, over qmax), and every code is within half a step of the stored step."""
+    rng = np.random.default_rng(60 + bits)
+    dk, dv = 128, 96
+    S = _outlier_state(rng, 128)[:, :dv]
+    w = np.exp(rng.normal(0, 1, dk))
+    block, x, tie, stie, st = orc.quantize_s(bits, orc.SCALE_BF16, S, w)
+    assert st == orc.OK
+    r, c = orc.scales_s(bits, orc.SCALE_BF16, dk, dv, block)
+    rc = np.concatenate([r, c])
+    assert np.array_equal(rc.astype(np.float32).astype(np.float64), rc)
+    assert not (rc.astype(np.float32).view(np.uint32) & 0xFFFF).any()  # bf16 values: low half zero
+    def half_ulp(v):  # half the bf16 quantum of the binade [2^e, 2^(e+1)) holding v
+        return 2.0 ** (np.floor(np.log2(v)) - 8)
+
+    rms = np.sqrt((w[:, None] * S ** 2).sum(axis=0) / w.sum())
+    assert np.all(np.abs(c - rms) <= half_ulp(rms) * (1 + 1e-9))
+    t = np.abs(S / c[None, :]).max(axis=1) / orc.qmax(bits)
+    assert np.all(np.abs(r - t) <= half_ulp(t) * (1 + 1e-9))
+    Q = orc.codes(bits, dk, dv, block)
+    step = r[:, None] * c[None, :]
+    assert np.all(np.abs(S - step * Q) <= 0.5 * step * (1 + 1e-9))
+    assert np.all(np.abs(Q).max(axis=1) >= orc.qmax(bits) - 1)
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_bf16_sign_pattern_gives_full_scale(orc, bits):
+    """S = diag(a) Sigma diag(b): with bf16 scales every code has Sigma's sign and magnitude within
+    qmax (1 - 2^-7) of qmax (the stored column scales carry up to 2^-8 relative rounding each way),
+    so qmax at 4 and 6 bits and 126 or 127 at 8 bits; every row reaches qmax."""
+    d = 64
+    rng = np.random.default_rng(70 + bits)
+    a = np.exp(rng.normal(0, 0.8, d))
+    b = np.exp(rng.normal(0, 0.8, d))
+    sig = np.where(rng.random((d, d)) < 0.5, -1.0, 1.0)
+    block, _, _, _, st = orc.quantize_s(bits, orc.SCALE_BF16, a[:, None] * sig * b[None, :], np.exp(rng.normal(0, 1, d)))
+    assert st == orc.OK
+    Q = orc.codes(bits, d, d, block)
+    qm = orc.qmax(bits)
+    assert np.array_equal(np.sign(Q), sig.astype(int))
+    assert np.all(np.abs(Q) >= np.ceil(qm * (1 - 2.0 ** -7) - 0.5)) and np.all(np.abs(Q).max(axis=1) == qm)
+    if bits < 8:
+        assert np.all(np.abs(Q) == qm)
+
+
+def test_bf16_given_scales_are_used_as_stored(orc):
+    """Scales passed in replace the fitted ones: with the fitted scales given back the block is
+    identical, and with another column scale the codes follow it."""
+    rng = np.random.default_rng(77)
+    S = _outlier_state(rng, 32)
+    w = np.exp(rng.normal(0, 1, 32))
+    blk, _, _, _, _ = orc.quantize_s(6, orc.SCALE_BF16, S, w)
+    r, c = orc.scales_s(6, orc.SCALE_BF16, 32, 32, blk)
+    again, _, _, _, _ = orc.quantize_s(6, orc.SCALE_BF16, S, w, c_given=c, r_given=r)
+    assert np.array_equal(again, blk)
+    c2 = c.copy()
+    c2[5] = orc.bf16_to_double(orc.double_to_bf16(c[5]) + 1)  # one bf16 ulp up
+    other, _, _, _, _ = orc.quantize_s(6, orc.SCALE_BF16, S, w, c_given=c2)
+    r3, c3 = orc.scales_s(6, orc.SCALE_BF16, 32, 32, other)
+    assert np.array_equal(c3, c2)
+    Q = orc.codes(6, 32, 32, other)
+    step = r3[:, None] * c3[None, :]
+    assert np.all(np.abs(S - step * Q) <= 0.5 * step * (1 + 1e-9))
+
+
+def test_bf16_decode_step_is_update_then_requantization(orc):
+    rng = np.random.default_rng(78)
+    d = 16
+    S0 = _outlier_state(rng, d)
+    w = np.exp(rng.normal(0, 1, d))
+    blk = orc.quantize_s(4, orc.SCALE_BF16, S0, w)[0]
+    q, k = rng.standard_normal(d), rng.standard_normal(d)
+    q, k = q / np.linalg.norm(q), k / np.linalg.norm(k)
+    v = rng.standard_normal(d)
+    res = orc.decode_step_s(4, orc.SCALE_BF16, 0, blk, q, k, v, 0.6, 0.97, w, d, d)
+    assert res["status"] == orc.OK
+    S1, o = orc.update(0, orc.dequantize_s(4, orc.SCALE_BF16, d, d, blk), q, k, v, 0.6, 0.97)
+    assert np.array_equal(res["o"], o.astype(np.float32))
+    assert np.array_equal(res["block"], orc.quantize_s(4, orc.SCALE_BF16, S1, w)[0])
+    assert res["block"].size == orc.block_bytes_s(4, orc.SCALE_BF16, d, d)
