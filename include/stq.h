@@ -18,7 +18,10 @@
  *   column scale c'_j = sqrt( sum_i w_i S'_ij^2 / sum_i w_i )   (w: per-head key-row impact)
  *   row scale    r'_i = max_j |S'_ij / c'_j| / qmax
  *   requantize   Q'_ij = round_half_even(S'_ij / (r'_i c'_j)); a zero scale is replaced by 1
- * Scales are stored as fp32 and codes are computed from the stored scales; a pivot head (b = 16)
+ * Scales are stored as fp32 (or, with scale_dtype = STQ_BF16, as bf16 rounded half to even: the
+ * 16-bit scales that bring a 6-bit 128 x 128 head to 5.12x compression, the figure the k1 page's
+ * section 實驗結果 reports as ~5.03x with pivots) and codes are computed from the stored scales,
+ * column scales first, then the row scales from the stored column scales; a pivot head (b = 16)
  * stores S' as fp16 (round to nearest even) and has no scales. With the channel gate alpha is a
  * vector over key rows: STQ_GATE_CHANNEL substitutes it literally,
  * S'_ij = alpha_i (S_ij - beta k_i u_j) + beta k_i v_j; STQ_GATE_CHANNEL_DECAY_FIRST decays first,
@@ -28,7 +31,8 @@
  * order) padded to 128 bytes; request `slot` starts at pool + slot * bytes_per_request. A quantized
  * head block holds the codes as a little-endian bitstream (code (i,j) at bit b*(i*d_v + j), bit k
  * of the stream = bit k%8 of byte k/8, stored offset-binary Q + 2^(b-1)), zero padding to 16 bytes,
- * r[d_k] fp32, c[d_v] fp32, zero padding to 128 bytes. A pivot head block is S as fp16 row-major,
+ * r[d_k], c[d_v] (fp32, or bf16 in the 16-bit scale format), zero padding to 128 bytes. A pivot
+ * head block is S as fp16 row-major,
  * padded to 128 bytes. The pool is its own checkpoint: its bytes plus the layout descriptor.
  *
  * Conventions for every call below.
@@ -60,7 +64,7 @@
 extern "C" {
 #endif
 
-#define STQ_ABI_VERSION 2
+#define STQ_ABI_VERSION 3
 
 typedef enum {
     STQ_OK = 0,
@@ -96,6 +100,8 @@ typedef struct {
     int32_t gate;              /* stq_gate                                                   */
     int32_t in_dtype;          /* stq_dtype of q, k, v                                       */
     int32_t scale_mode;        /* stq_scale_mode (0: the method's row x column scales)       */
+    int32_t scale_dtype;       /* stq_dtype of the stored row and column scales: STQ_F32 (0) */
+                               /* or STQ_BF16 (16-bit scales; row x column mode only)        */
 } stq_layout_desc;
 
 typedef struct stq_layout stq_layout; /* opaque, host-only, immutable after creation */

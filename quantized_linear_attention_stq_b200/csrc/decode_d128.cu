@@ -98,7 +98,9 @@ template <int BITS, int GATE, int IN_BF16>
 struct Cfg {
     static constexpr int RB = BITS == 16 ? 256 : 16 * BITS;    // bytes of one 128-wide row
     static constexpr uint32_t SOFF = scale_offset(BITS, D, D);  // byte offset of r[]
-    static constexpr uint32_t BLK = head_block_bytes(BITS, D, D);
+    static constexpr uint32_t BLK = head_block_bytes(BITS, D, D);  // ring room (fp32 scales)
+    // bytes of the block with 16-bit scales: the copy is shorter, the ring layout the same
+    static constexpr uint32_t BLK16 = head_block_bytes_bf16s(BITS, D, D);
     static constexpr uint32_t ROW_IN = D * (IN_BF16 ? 2u : 4u);
     static constexpr uint32_t K_OFF = BLK, Q_OFF = BLK + ROW_IN, V_OFF = BLK + 2 * ROW_IN;
     static constexpr uint32_t W_OFF = BLK + 3 * ROW_IN, A_OFF = W_OFF + 4 * D;
@@ -314,8 +316,9 @@ __device__ __forceinline__ void issue_next(const TileParams &p, SmemFixed &sm, u
     if (GATE == 0) cp_async4(smem_u32(&sm.scal[slot_i][1]), p.alpha + row);
     cp_async_arrive(bar);
     const uint32_t dst = smem_u32(ring_slot<BITS, GATE, IN_BF16>(smem, slot_i));
-    mbar_arrive_expect_tx(bar, C::LEN);
-    bulk_g2s(dst, src, C::BLK, bar);
+    const uint32_t blk = p.scale_bf16 ? C::BLK16 : C::BLK;
+    mbar_arrive_expect_tx(bar, C::LEN - (C::BLK - blk));
+    bulk_g2s(dst, src, blk, bar);
     bulk_g2s(dst + C::K_OFF, (const uint8_t *)p.k + (size_t)row * C::ROW_IN, C::ROW_IN, bar);
     bulk_g2s(dst + C::Q_OFF, (const uint8_t *)p.q + (size_t)row * C::ROW_IN, C::ROW_IN, bar);
     bulk_g2s(dst + C::V_OFF, (const uint8_t *)p.v + (size_t)row * C::ROW_IN, C::ROW_IN, bar);
@@ -326,7 +329,7 @@ __device__ __forceinline__ void issue_next(const TileParams &p, SmemFixed &sm, u
 // Wait for tile n (ring slot n % NS) and compute its row factors, row i = threadIdx.x, with
 // per-warp sums of w, q.k and q.(alpha k). Returns false on a timeout.
 template <int BITS, int GATE, int IN_BF16>
-__device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, int n, int my_count)
+__device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, int n, int my_count, int sb16)
 {
     using C = Cfg<BITS, GATE, IN_BF16>;
     if (n >= my_count) return true;
@@ -339,7 +342,7 @@ __device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, in
     const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16>(smem, slot_i);
     const int i = threadIdx.x;
     constexpr bool pivot = BITS == 16;
-    const float r = pivot ? 1.f : reinterpret_cast<const float *>(tile + C::SOFF)[i];
+    const float r = pivot ? 1.f : load_scale(tile + C::SOFF, i, sb16);
     const float k = load_in<IN_BF16>(tile + C::K_OFF, i);
     const float q = load_in<IN_BF16>(tile + C::Q_OFF, i);
     const float w = reinterpret_cast<const float *>(tile + C::W_OFF)[i];
@@ -422,7 +425,8 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
 
     // ---- Column finals (column j = tid): update coefficients and the readout ---------------
     const int j = tid;
-    const float cj = pivot ? 1.f : reinterpret_cast<const float *>(tile + C::SOFF)[D + j];
+    const int sb16 = p.scale_bf16;
+    const float cj = pivot ? 1.f : load_scale(tile + C::SOFF, D + j, sb16);
     const float inv_sig = (j & 1) ? 1.f / C::SIG1 : 1.f;  // powers of two: exact
     {
         // k~Q partials in the half-0 regions (0, 2, 4, 6), q~Q partials in the half-1 regions
@@ -534,12 +538,15 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
         if (x == 0.f) {  // zero column: scale 1 (a NaN stays NaN)
             c = 1.f;
             b = 0.f;
+        } else if (sb16) {  // the codes follow the stored (rounded) scale
+            c = round_scale(c, 1);
+            b = (cj * inv_sig) * fast_rcp(c);
         }
-        reinterpret_cast<float *>(sm.meta[n & 3].gblock + C::SOFF)[D + j] = c;
+        store_scale(reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + C::SOFF), D + j, c, sb16);
         if (!isfinite(c) || c == 0.f) flag(p.status, kFlagNonfinite);
         sm.colB[j] = b;
     }
-    const bool ok = precompute_rows<BITS, GATE, IN_BF16>(sm, smem, n + 1, my_count);
+    const bool ok = precompute_rows<BITS, GATE, IN_BF16>(sm, smem, n + 1, my_count, sb16);
     if (__syncthreads_or(!ok)) return false;  // B4: new column scales and next row factors ready
     if constexpr (pivot) return true;
 
@@ -585,9 +592,12 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
         if (v == 0.f) {  // zero row: scale 1
             r = 1.f;
             s = 0.f;
+        } else if (sb16) {  // the codes follow the stored (rounded) scale: s = 1 / (sqrt(w_i) r~_i)
+            r = round_scale(r, 1);
+            s = (sm.rowRq[pb][i] * C::QMAX) * fast_rcp(r);
         }
         sm.rowS[i] = make_float2(s, s);
-        reinterpret_cast<float *>(sm.meta[n & 3].gblock + C::SOFF)[i] = r;
+        store_scale(reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + C::SOFF), i, r, sb16);
         if (!isfinite(r) || r == 0.f) flag(p.status, kFlagNonfinite);
     }
     __syncwarp();
@@ -657,7 +667,7 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
         it.rG = G - it.qG * p.B;
         for (int k = 0; k < C::NS; ++k) issue_next<BITS, GATE, IN_BF16>(p, sm, smem, it, my_count);
     }
-    bool failed = __syncthreads_or(!precompute_rows<BITS, GATE, IN_BF16>(sm, smem, 0, my_count));
+    bool failed = __syncthreads_or(!precompute_rows<BITS, GATE, IN_BF16>(sm, smem, 0, my_count, p.scale_bf16));
 
     int n = 0;
     for (; n < my_count && !failed; ++n) {
@@ -666,7 +676,7 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
         if (sm.meta[n & 3].skip) {  // out-of-range slot: nothing loaded, nothing to do
             __syncthreads();
             if (tid == 0) issue_next<BITS, GATE, IN_BF16>(p, sm, smem, sm.iss, my_count);
-            const bool ok = precompute_rows<BITS, GATE, IN_BF16>(sm, smem, n + 1, my_count);
+            const bool ok = precompute_rows<BITS, GATE, IN_BF16>(sm, smem, n + 1, my_count, p.scale_bf16);
             failed = __syncthreads_or(!ok || !got);
         } else {
             failed = !process_tile<BITS, GATE, IN_BF16>(p, sm, smem, n, my_count, tcol);

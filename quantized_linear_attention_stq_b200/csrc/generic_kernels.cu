@@ -17,6 +17,7 @@ constexpr int kThreads = 256;
 struct TileRef {
     bool ok;
     bool uniform;  // one scale for the whole head (the baseline quantizer)
+    int sb16;      // row and column scales stored as bf16
     int b, head, bits;
     uint8_t *block;
 };
@@ -29,6 +30,7 @@ __device__ __forceinline__ TileRef tile_ref(const TileParams &p, int b, int pos)
     t.head = entry_head(e);
     t.bits = entry_bits(e);
     t.uniform = entry_uniform(e);
+    t.sb16 = p.scale_bf16;
     const int slot = p.slots[b];
     t.ok = slot >= 0 && slot < p.pool_slots;
     t.block = t.ok ? p.pool + (uint64_t)slot * p.req_bytes + e.off : nullptr;
@@ -47,7 +49,8 @@ __device__ __forceinline__ int read_code(const uint8_t *codes, int bits, int n)
 
 // Dequantize a tile from global memory into S (row stride ld): S_ij = fp32(r_i c_j) * Q_ij, or
 // S_ij = s * Q_ij for a uniformly scaled head.
-__device__ void dequant_to_smem(const uint8_t *block, int bits, bool uniform, int dk, int dv, float *S, int ld)
+__device__ void dequant_to_smem(const uint8_t *block, int bits, bool uniform, int sb16, int dk, int dv, float *S,
+                                int ld)
 {
     const int n = dk * dv;
     if (bits == 16) {
@@ -62,12 +65,11 @@ __device__ void dequant_to_smem(const uint8_t *block, int bits, bool uniform, in
             S[(e / dv) * ld + e % dv] = su * (float)(read_code(block, bits, e) - off);
         return;
     }
-    const float *r = reinterpret_cast<const float *>(block + scale_offset(bits, dk, dv));
-    const float *c = r + dk;
+    const uint8_t *sc = block + scale_offset(bits, dk, dv);
     const int off = 1 << (bits - 1);
     for (int e = threadIdx.x; e < n; e += blockDim.x) {
         const int i = e / dv, j = e % dv;
-        const float rc = r[i] * c[j];
+        const float rc = load_scale(sc, i, sb16) * load_scale(sc, dk + j, sb16);
         S[i * ld + j] = rc * (float)(read_code(block, bits, e) - off);
     }
 }
@@ -75,8 +77,8 @@ __device__ void dequant_to_smem(const uint8_t *block, int bits, bool uniform, in
 // Fit scales to the fp32 state in S and write codes + scales into `block` (or fp16 values for a
 // pivot head). `wv` holds the impact weights of the head in shared memory. Needs a CTA-wide
 // barrier before (S complete) and provides one after.
-__device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, bool uniform, int dk, int dv,
-                                   uint8_t *block, float *cs, float *rs, int32_t *status)
+__device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, bool uniform, int sb16, int dk,
+                                   int dv, uint8_t *block, float *cs, float *rs, int32_t *status)
 {
     const int n = dk * dv;
     __shared__ uint32_t smax;
@@ -138,7 +140,7 @@ __device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, 
         }
         float c = sqrtf(E / W);
         if (c == 0.f) c = 1.f;
-        cs[j] = c;
+        cs[j] = round_scale(c, sb16);  // the codes use the stored value
     }
     __syncthreads();
     // row scales: largest column-normalised magnitude over qmax
@@ -147,17 +149,17 @@ __device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, 
         for (int j = 0; j < dv; ++j) m = fmaxf(m, fabsf(S[i * ld + j] / cs[j]));
         float r = m / qmax;
         if (r == 0.f) r = 1.f;
-        rs[i] = r;
+        rs[i] = round_scale(r, sb16);
     }
     __syncthreads();
     bool bad = false;
-    float *rg = reinterpret_cast<float *>(block + scale_offset(bits, dk, dv));
+    uint8_t *sg = block + scale_offset(bits, dk, dv);
     for (int i = threadIdx.x; i < dk; i += blockDim.x) {
-        rg[i] = rs[i];
+        store_scale(sg, i, rs[i], sb16);
         bad |= !isfinite(rs[i]) || rs[i] == 0.f;
     }
     for (int j = threadIdx.x; j < dv; j += blockDim.x) {
-        rg[dk + j] = cs[j];
+        store_scale(sg, dk + j, cs[j], sb16);
         bad |= !isfinite(cs[j]);
     }
     // codes, packed by groups of whole bytes: 2 codes/byte (4-bit), 4 codes/3 bytes (6-bit),
@@ -200,7 +202,7 @@ __global__ void __launch_bounds__(kThreads) init_kernel(const __grid_constant__ 
     for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) S[(e / dv) * ld + e % dv] = src[e];
     for (int i = threadIdx.x; i < dk; i += blockDim.x) wv[i] = p.w[(uint64_t)t.head * dk + i];
     __syncthreads();
-    quantize_from_smem(S, ld, wv, t.bits, t.uniform, dk, dv, t.block, cs, rs, p.status);
+    quantize_from_smem(S, ld, wv, t.bits, t.uniform, t.sb16, dk, dv, t.block, cs, rs, p.status);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -216,7 +218,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const __grid_constant
     }
     const int dk = p.dk, dv = p.dv;
     float *dst = p.S_out + ((uint64_t)b * p.head_count + t.head) * dk * dv;
-    dequant_to_smem(t.block, t.bits, t.uniform, dk, dv, dst, dv);  // writes straight to global, row stride dv
+    dequant_to_smem(t.block, t.bits, t.uniform, t.sb16, dk, dv, dst, dv);  // writes straight to global, row stride dv
 }
 
 // ------------------------------------------------------------------------------------------
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(kThreads) decode_generic_kernel(const __grid_c
         wv[i] = p.w[(uint64_t)t.head * dk + i];
     }
     for (int j = threadIdx.x; j < dv; j += blockDim.x) vv[j] = load_in<IN_BF16>(p.v, tile * dv + j);
-    dequant_to_smem(t.block, t.bits, t.uniform, dk, dv, S, ld);
+    dequant_to_smem(t.block, t.bits, t.uniform, t.sb16, dk, dv, S, ld);
     __syncthreads();
     const float beta = p.beta[tile];
     const bool decay_first = p.gate == 2;
@@ -279,7 +281,7 @@ __global__ void __launch_bounds__(kThreads) decode_generic_kernel(const __grid_c
         bad |= !isfinite(acc);
     }
     if (bad) flag(p.status, kFlagNonfinite);
-    quantize_from_smem(S, ld, wv, t.bits, t.uniform, dk, dv, t.block, cs, rs, p.status);
+    quantize_from_smem(S, ld, wv, t.bits, t.uniform, t.sb16, dk, dv, t.block, cs, rs, p.status);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -310,7 +312,7 @@ __global__ void __launch_bounds__(kThreads) prefill_seq_kernel(const __grid_cons
     const uint64_t tile = (uint64_t)b * p.head_count + t.head;
     const bool channel = p.gate != 0, decay_first = p.gate == 2;
     for (int i = threadIdx.x; i < dk; i += blockDim.x) wv[i] = p.w[(uint64_t)t.head * dk + i];
-    dequant_to_smem(t.block, t.bits, t.uniform, dk, dv, S, ld);
+    dequant_to_smem(t.block, t.bits, t.uniform, t.sb16, dk, dv, S, ld);
     bool bad = false;
     for (int tok = 0; tok < T; ++tok) {
         const uint64_t row = tile * T + tok;
@@ -343,10 +345,10 @@ __global__ void __launch_bounds__(kThreads) prefill_seq_kernel(const __grid_cons
         }
         if ((tok + 1) % chunk == 0 || tok == T - 1) {
             __syncthreads();
-            quantize_from_smem(S, ld, wv, t.bits, t.uniform, dk, dv, t.block, cs, rs, p.status);
+            quantize_from_smem(S, ld, wv, t.bits, t.uniform, t.sb16, dk, dv, t.block, cs, rs, p.status);
             if (tok != T - 1) {
                 __syncthreads();
-                dequant_to_smem(t.block, t.bits, t.uniform, dk, dv, S, ld);
+                dequant_to_smem(t.block, t.bits, t.uniform, t.sb16, dk, dv, S, ld);
             }
         }
         __syncthreads();

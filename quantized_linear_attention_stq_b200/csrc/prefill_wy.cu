@@ -383,9 +383,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
         __syncthreads();  // the previous tile is completely done with shared memory
         load_codes_row<BITS>(gblock, sm + OFF_QC, tid >> 2, tid & 3);
         if (tid < D) {
-            const float *sc = reinterpret_cast<const float *>(gblock + P::SOFF);
-            sR[tid] = sc[tid];
-            sC[tid] = sc[D + tid];
+            sR[tid] = load_scale(gblock + P::SOFF, tid, p.scale_bf16);
+            sC[tid] = load_scale(gblock + P::SOFF, D + tid, p.scale_bf16);
             sW[tid] = p.w[(size_t)head * D + tid];
         }
         load_chunk_async(sm, OFF_XY0, 0, kg, qg, bg, ag, T_tok < C ? T_tok : C);
@@ -710,6 +709,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                     const float E = (red[tid] + red[D + tid]) + (red[2 * D + tid] + red[3 * D + tid]);
                     float cj = sqrtf(E / miscf[0]);
                     if (cj == 0.f) cj = 1.f;
+                    cj = round_scale(cj, p.scale_bf16);  // the codes follow the stored scale
                     bad |= !isfinite(cj);
                     sC[tid] = cj;
                     red[tid] = __frcp_rn(cj);  // this column's partials have been read
@@ -726,6 +726,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                 m = fmaxf(fmaxf(rmax[i], rmax[D + i]), fmaxf(rmax[2 * D + i], rmax[3 * D + i]));
                 float ri = m / (float)P::QMAX;
                 if (ri == 0.f) ri = 1.f;
+                ri = round_scale(ri, p.scale_bf16);
                 bad |= !isfinite(ri);
                 const float rri = __frcp_rn(ri);
                 int qc[32];
@@ -749,9 +750,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                 if (cq == 0) sR[i] = ri;
                 if (c + 1 == nch) {  // the last chunk of the call: the state goes back to HBM
                     store_codes_row<BITS>(gblock, i, cq, qc);
-                    float *gsc = reinterpret_cast<float *>(gblock + P::SOFF);
-                    if (cq == 0) gsc[i] = ri;
-                    if (tid < D) gsc[D + tid] = sC[tid];
+                    if (cq == 0) store_scale(gblock + P::SOFF, i, ri, p.scale_bf16);
+                    if (tid < D) store_scale(gblock + P::SOFF, D + tid, sC[tid], p.scale_bf16);
                 }
             }
             if (bad) flag(p.status, kFlagNonfinite);

@@ -14,6 +14,7 @@
 struct stq_layout {
     int32_t H, dk, dv, gate, in_dtype;
     bool uniform;  // STQ_SCALES_UNIFORM
+    bool sb16;     // row and column scales stored as bf16
     std::vector<uint8_t> bits;
     std::vector<uint64_t> offset;
     std::vector<uint64_t> bytes;
@@ -38,6 +39,7 @@ std::vector<int> order_by_size(const stq_layout *L, int h0, int count)
 void fill_table(stq::TileParams &p, const stq_layout *L, const std::vector<int> &ord, int first, int n, int h0)
 {
     p.npos = n;
+    p.scale_bf16 = L->sb16 ? 1 : 0;
     for (int e = 0; e < n; ++e) {
         const int h = ord[first + e];
         p.table[e].off = (uint32_t)L->offset[h];
@@ -84,6 +86,8 @@ stq_status stq_layout_create(const stq_layout_desc *desc, stq_layout **out)
     if (desc->gate < STQ_GATE_SCALAR || desc->gate > STQ_GATE_CHANNEL_DECAY_FIRST) return STQ_ERR_INVALID_ARG;
     if (desc->in_dtype != STQ_F32 && desc->in_dtype != STQ_BF16) return STQ_ERR_INVALID_ARG;
     if (desc->scale_mode != STQ_SCALES_ROW_COLUMN && desc->scale_mode != STQ_SCALES_UNIFORM) return STQ_ERR_INVALID_ARG;
+    if (desc->scale_dtype != STQ_F32 && desc->scale_dtype != STQ_BF16) return STQ_ERR_INVALID_ARG;
+    if (desc->scale_dtype == STQ_BF16 && desc->scale_mode == STQ_SCALES_UNIFORM) return STQ_ERR_UNSUPPORTED;
     const int d = desc->d_k;
     if (desc->d_v != d || !(d == 16 || d == 32 || d == 64 || d == 128)) return STQ_ERR_UNSUPPORTED;
     if (desc->num_heads > 65535) return STQ_ERR_UNSUPPORTED;
@@ -95,6 +99,7 @@ stq_status stq_layout_create(const stq_layout_desc *desc, stq_layout **out)
     L->gate = desc->gate;
     L->in_dtype = desc->in_dtype;
     L->uniform = desc->scale_mode == STQ_SCALES_UNIFORM;
+    L->sb16 = desc->scale_dtype == STQ_BF16;
     uint64_t pos = 0;
     for (int h = 0; h < L->H; ++h) {
         const int b = desc->head_bits[h];
@@ -102,6 +107,7 @@ stq_status stq_layout_create(const stq_layout_desc *desc, stq_layout **out)
         L->bits.push_back((uint8_t)b);
         L->offset.push_back(pos);
         const uint64_t nb = (L->uniform && b != 16) ? stq::uniform_block_bytes(b, L->dk, L->dv)
+                            : L->sb16               ? stq::head_block_bytes_bf16s(b, L->dk, L->dv)
                                                     : stq::head_block_bytes(b, L->dk, L->dv);
         L->bytes.push_back(nb);
         pos += nb;

@@ -38,6 +38,12 @@ __host__ __device__ constexpr uint32_t head_block_bytes(int bits, int dk, int dv
     return bits == 16 ? round_up_u32(2u * dk * dv, 128)
                       : round_up_u32(scale_offset(bits, dk, dv) + 4u * dk + 4u * dv, 128);
 }
+// The same block with its row and column scales stored as bf16 (the 16-bit scale format).
+__host__ __device__ constexpr uint32_t head_block_bytes_bf16s(int bits, int dk, int dv)
+{
+    return bits == 16 ? round_up_u32(2u * dk * dv, 128)
+                      : round_up_u32(scale_offset(bits, dk, dv) + 2u * dk + 2u * dv, 128);
+}
 
 // One entry of the per-launch head table, in processing order (largest blocks first).
 struct TileEntry {
@@ -68,6 +74,7 @@ struct TileParams {
     int32_t head_count;  // heads of the call (row stride of the per-head input arrays)
     int32_t dk, dv;
     int32_t gate;
+    int32_t scale_bf16;  // 1: row and column scales stored as bf16 (else fp32)
     // decode / prefill inputs (indexed by request and call-relative head)
     const void *q, *k, *v;
     const float *beta, *alpha, *w;
@@ -101,6 +108,25 @@ __device__ __forceinline__ float load_in(const void *base, size_t idx)
         return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base)[idx]);
     else
         return reinterpret_cast<const float *>(base)[idx];
+}
+
+// Scale n of a head block's scale array (r[0..dk) then c[0..dv)) in the layout's storage format;
+// a stored bf16 scale is rounded half to even from the fp32 value.
+__device__ __forceinline__ float load_scale(const uint8_t *scales, int n, int bf16)
+{
+    return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(scales)[n])
+                : reinterpret_cast<const float *>(scales)[n];
+}
+__device__ __forceinline__ float round_scale(float v, int bf16)
+{
+    return bf16 ? __bfloat162float(__float2bfloat16_rn(v)) : v;
+}
+__device__ __forceinline__ void store_scale(uint8_t *scales, int n, float v, int bf16)
+{
+    if (bf16)
+        reinterpret_cast<__nv_bfloat16 *>(scales)[n] = __float2bfloat16_rn(v);
+    else
+        reinterpret_cast<float *>(scales)[n] = v;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)

@@ -37,12 +37,16 @@ class Tally:
     pivot_values: int = 0
     pivot_diffs: int = 0
     updates_per_check: int = 1   # fp32 updates a pivot state carried since the oracle's bytes
+    scales: int = 0              # bf16 scales checked
+    scale_flips: int = 0         # of which one bf16 step off the oracle's, at a flagged near-tie
 
     def check_budget(self):
         assert self.codes + self.pivot_values > 0
         assert self.tie_flips <= CODE_TIE_BUDGET * self.codes, f"{self.tie_flips} tie flips in {self.codes} codes"
         assert self.pivot_diffs <= PIVOT_DIFF_BUDGET * self.updates_per_check * self.pivot_values, \
             f"{self.pivot_diffs} of {self.pivot_values} fp16 pivot values differ"
+        assert self.scale_flips <= SCALE_FLIP_BUDGET * self.scales + 2, \
+            f"{self.scale_flips} of {self.scales} bf16 scales one step off"
 
 
 def oracle_pool(orc, head_bits, d, blocks_per_request):
@@ -147,6 +151,58 @@ def compare_uniform_block(orc, bits, d, got, ref_block, ref_tie, tally: Tally, w
     so = orc.scale_offset(bits, d, d)
     assert not got[orc.codes_bytes(bits, d, d): so].any()
     assert not got[so + 4:].any()
+
+
+SCALE_FLIP_BUDGET = 2e-3
+
+
+def _bf16_neighbours(orc, a, b):
+    """a and b are adjacent bf16 values (patterns one apart, same sign)."""
+    ha, hb = orc.double_to_bf16(float(a)), orc.double_to_bf16(float(b))
+    return (ha & 0x8000) == (hb & 0x8000) and abs(ha - hb) == 1
+
+
+def compare_block_bf16s(orc, bits, d, got, S_new, w, tally: Tally, what=""):
+    """A head block with bf16 row and column scales against the oracle's requantization of the
+    same updated state S_new (fp64). A stored bf16 scale may differ from the oracle's by one bf16
+    step only where the oracle flags the exact scale as a rounding near-tie; the oracle then
+    continues with the GPU's stored scales (column scales first, then rows: codes follow the
+    stored scales), and the codes are compared with the code rule above. Flipped scales stay
+    below SCALE_FLIP_BUDGET of the scales checked (counted in tally.scale_flips)."""
+    got = np.asarray(got, dtype=np.uint8)
+    sf = orc.SCALE_BF16
+    rg, cg = orc.scales_s(bits, sf, d, d, got)
+    blk, x, tie, stie, st = orc.quantize_s(bits, sf, S_new, w)
+    assert st == orc.OK
+    ro, co = orc.scales_s(bits, sf, d, d, blk)
+    for name, gv, ov, flags in (("column", cg, co, stie[d:]), ):
+        diff = gv != ov
+        bad = diff & ~(flags & np.array([_bf16_neighbours(orc, a, b) for a, b in zip(gv, ov)]))
+        assert not bad.any(), f"{what}: {name} scale {int(np.argmax(bad))} gpu {gv[bad][0]!r} oracle {ov[bad][0]!r}"
+        tally.scale_flips += int(diff.sum())
+    if (cg != co).any():
+        blk, x, tie, stie, st = orc.quantize_s(bits, sf, S_new, w, c_given=cg)
+        ro = orc.scales_s(bits, sf, d, d, blk)[0]
+    diff = rg != ro
+    bad = diff & ~(stie[:d] & np.array([_bf16_neighbours(orc, a, b) for a, b in zip(rg, ro)]))
+    assert not bad.any(), f"{what}: row scale {int(np.argmax(bad))} gpu {rg[bad][0]!r} oracle {ro[bad][0]!r}"
+    tally.scale_flips += int(diff.sum())
+    tally.scales += 2 * d
+    if diff.any():
+        blk, x, tie, _, st = orc.quantize_s(bits, sf, S_new, w, c_given=cg, r_given=rg)
+    Qg = orc.codes(bits, d, d, got)
+    Qr = orc.codes(bits, d, d, blk)
+    cdiff = np.abs(Qg - Qr)
+    badc = (cdiff > 1) | ((cdiff == 1) & ~tie)
+    if badc.any():
+        i, j = np.argwhere(badc)[0]
+        raise AssertionError(f"{what}: {int(badc.sum())} codes differ off a tie, first at ({i},{j}): "
+                             f"gpu {Qg[i, j]} oracle {Qr[i, j]} x {x[i, j]!r}")
+    tally.codes += Qg.size
+    tally.tie_flips += int((cdiff == 1).sum())
+    so = orc.scale_offset(bits, d, d)
+    assert not got[orc.codes_bytes(bits, d, d): so].any()
+    assert not got[so + 4 * d:].any()
 
 
 def compare_o(got, ref, tally: Tally, what=""):

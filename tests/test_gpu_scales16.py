@@ -1,0 +1,236 @@
+"""GPU parity of the 16-bit (bf16) scale format against the oracle (needs a B200).
+
+With scale_dtype = bf16 a head block stores its row and column scales as bf16, which brings a
+6-bit 128 x 128 head to 5.12x compression against fp32 (the k1 page's section 實驗結果 reports
+~5.03x with pivots). The codes follow the stored scales. Teacher-forced protocol as in
+test_gpu_decode.py; blocks are compared with the bf16-scale rule of tests/_parity.py (a stored
+scale may sit one bf16 step off the oracle's only at a flagged scale near-tie, and the codes are
+then checked against the oracle's requantization with the GPU's stored scales).
+"""
+import numpy as np
+import pytest
+import torch
+
+from _parity import Tally, as_f64, compare_block, compare_block_bf16s, compare_o, update_magnitude
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def stq():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for the gpu tests")
+    import quantized_linear_attention_stq_b200 as m
+
+    m.lib()  # fails loudly if libstq.so is missing
+    return m
+
+
+def _wl(name, **changes):
+    from quantized_linear_attention_stq_b200 import workloads as wl
+
+    return wl.scaled(wl.WORKLOADS[name], **changes)
+
+
+def _layout(orc, bits, d):
+    offs, pos = [], 0
+    for b in bits:
+        offs.append(pos)
+        pos += orc.block_bytes_s(int(b), orc.SCALE_BF16, d, d)
+    return offs, (pos + 127) // 128 * 128
+
+
+def _tile(orc, pool, bits, d, slot, h):
+    offs, total = _layout(orc, bits, d)
+    n = orc.block_bytes_s(int(bits[h]), orc.SCALE_BF16, d, d)
+    return np.asarray(pool[slot * total + offs[h]: slot * total + offs[h] + n])
+
+
+def _oracle_pool(orc, bits, d, S0, w):
+    offs, total = _layout(orc, bits, d)
+    B, H = S0.shape[0], S0.shape[1]
+    pool = np.zeros(B * total, dtype=np.uint8)
+    for r in range(B):
+        for h in range(H):
+            blk, _, _, _, st = orc.quantize_s(bits[h], orc.SCALE_BF16, as_f64(S0[r, h]), as_f64(w[h]))
+            assert st == orc.OK
+            pool[r * total + offs[h]: r * total + offs[h] + blk.size] = blk
+    return pool
+
+
+def test_layout_sizes(stq, orc):
+    bits = [4, 6, 8, 16, 6]
+    lay = stq.Layout(bits, 128, scale_dtype=torch.bfloat16)
+    offs, total = _layout(orc, bits, 128)
+    assert lay.bytes_per_request == total
+    assert [lay.head_offset(h) for h in range(5)] == offs
+    assert [lay.head_bytes(h) for h in range(5)] == [8704, 12800, 16896, 32768, 12800]
+    with pytest.raises(stq.StqError) as e:
+        stq.Layout([4], 128, scale_mode=stq.SCALES_UNIFORM, scale_dtype=torch.bfloat16)
+    assert e.value.status == stq.api.STQ_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("d", [16, 128])
+def test_init_and_dequantize(stq, orc, d):
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl_ = _wl("full2304_b70_mixed", batch=3, heads=6, d=d)
+    bits = [4, 6, 8, 16, 8, 6]
+    lay = stq.Layout(bits, d, scale_dtype=torch.bfloat16)
+    w = wlm.impact_weights(wl_)
+    S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(3)])
+    pool = lay.alloc_pool(3)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stq.init_state(lay, pool, torch.arange(3, dtype=torch.int32, device=DEV), S0.to(DEV), w.to(DEV), status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    gp = pool.cpu().numpy()
+    ref = _oracle_pool(orc, bits, d, S0, w)
+    tally = Tally()
+    for r in range(3):
+        for h in range(6):
+            got = _tile(orc, gp, bits, d, r, h)
+            if bits[h] == 16:
+                blk, _, tie, _ = orc.quantize(16, as_f64(S0[r, h]), as_f64(w[h]))
+                compare_block(orc, 16, d, got, blk, tie, tally, f"init req {r} head {h}")
+            else:
+                compare_block_bf16s(orc, bits[h], d, got, as_f64(S0[r, h]), as_f64(w[h]), tally,
+                                    f"init req {r} head {h}")
+    tally.check_budget()
+    # dequantize the oracle's bytes: fp32(r~ c~) * Q against the fp64 product
+    out = torch.zeros(3, 6, d, d, device=DEV)
+    stq.dequantize(lay, torch.from_numpy(ref).to(DEV), torch.tensor([2, 0, 1], dtype=torch.int32, device=DEV), out,
+                   status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    got = out.cpu().double().numpy()
+    for r, slot in enumerate((2, 0, 1)):
+        for h in range(6):
+            blk = _tile(orc, ref, bits, d, slot, h)
+            want = orc.dequantize_s(bits[h], orc.SCALE_BF16, d, d, blk)
+            assert np.all(np.abs(got[r, h] - want) <= 2.0 ** -23 * np.abs(want)), f"req {r} head {h}"
+
+
+def _decode_teacher_forced(stq, orc, wl_, bits, steps):
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    B, H, d = wl_.batch, wl_.heads, wl_.d
+    lay = stq.Layout(bits, d, gate=wl_.gate, in_dtype=wl_.in_dtype, scale_dtype=torch.bfloat16)
+    w = wlm.impact_weights(wl_)
+    S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(B)])
+    opool = _oracle_pool(orc, bits, d, S0, w)
+    offs, total = _layout(orc, bits, d)
+    slot_of = np.random.default_rng(13).permutation(B + 2)[:B].astype(np.int32)
+    gpool = torch.zeros((B + 2) * total, dtype=torch.uint8, device=DEV)
+    slots = torch.from_numpy(slot_of).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    tally = Tally()
+    for t in range(steps):
+        inp = wlm.decode_inputs(wl_, t)
+        host = np.zeros((B + 2) * total, dtype=np.uint8)
+        for r in range(B):
+            host[slot_of[r] * total:(slot_of[r] + 1) * total] = opool[r * total:(r + 1) * total]
+        gpool.copy_(torch.from_numpy(host).to(DEV))
+        o = torch.zeros(B, H, d, device=DEV)
+        g = {n: x.to(DEV) for n, x in inp.items()}
+        stq.decode_step(lay, gpool, slots, g["q"], g["k"], g["v"], g["beta"], g["alpha"], w.to(DEV), o,
+                        status=status)
+        torch.cuda.synchronize()
+        assert status.item() == 0, stq.status_flags(status)
+        gp, og = gpool.cpu().numpy(), o.cpu().numpy()
+        for r in range(B):
+            for h in range(H):
+                ref_blk = _tile(orc, opool, bits, d, r, h)
+                q, k, v = as_f64(inp["q"][r, h]), as_f64(inp["k"][r, h]), as_f64(inp["v"][r, h])
+                beta, alpha = float(inp["beta"][r, h]), inp["alpha"][r, h].double().numpy()
+                res = orc.decode_step_s(bits[h], orc.SCALE_BF16, wl_.gate, ref_blk, q, k, v, beta, alpha,
+                                        as_f64(w[h]), d, d)
+                assert res["status"] == orc.OK
+                got = _tile(orc, gp, bits, d, int(slot_of[r]), h)
+                what = f"step {t} req {r} head {h}"
+                if bits[h] == 16:
+                    M = update_magnitude(orc.dequantize(16, d, d, ref_blk), k, v, beta, alpha)
+                    compare_block(orc, 16, d, got, res["block"], res["tie"], tally, what, err_scale=M)
+                else:
+                    compare_block_bf16s(orc, bits[h], d, got, res["S_new"], as_f64(w[h]), tally, what)
+                compare_o(og[r, h], res["o"], tally, "o " + what)
+                opool[r * total + offs[h]: r * total + offs[h] + res["block"].size] = res["block"]
+    tally.check_budget()
+    return tally
+
+
+@pytest.mark.parametrize("bits", [4, 6, 8])
+def test_decode_d128(stq, orc, bits):
+    """The tuned 128 x 128 kernel with bf16 scales: 5 requests x 8 heads, 3 steps."""
+    wl_ = _wl("layer48_b8_4bit", batch=5, heads=8, bits=bits)
+    _decode_teacher_forced(stq, orc, wl_, [bits] * 8, 3)
+
+
+def test_decode_d128_mixed_with_pivots(stq, orc):
+    wl_ = _wl("full2304_b70_mixed", batch=4, heads=9)
+    _decode_teacher_forced(stq, orc, wl_, [4, 16, 6, 8, 4, 6, 16, 8, 6], 2)
+
+
+@pytest.mark.parametrize("gate", [1, 2])
+def test_decode_d128_channel_gates(stq, orc, gate):
+    wl_ = _wl("channel32_b128_4bit", batch=3, heads=4, gate=gate)
+    _decode_teacher_forced(stq, orc, wl_, [4, 6, 8, 6], 2)
+
+
+@pytest.mark.parametrize("d", [16, 32, 64])
+def test_decode_small_heads(stq, orc, d):
+    wl_ = _wl("layer48_b8_4bit", batch=3, heads=5, d=d, in_dtype=torch.float32)
+    _decode_teacher_forced(stq, orc, wl_, [4, 6, 8, 16, 6], 3)
+
+
+@pytest.mark.parametrize("d,in_dtype,T", [(128, torch.bfloat16, 64), (32, torch.float32, 64),
+                                          (128, torch.bfloat16, 40)])
+def test_prefill_chunk(stq, orc, d, in_dtype, T):
+    """One chunk per call, twice in a row, teacher-forced: 128 x 128 heads with bf16 inputs and
+    64-token chunks take the tensor-core path, the others the sequential kernel; a 40-token call
+    is a short last chunk."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    bits = [4, 6, 8, 16]
+    wl_ = _wl("prefill16_b16_6bit", batch=2, heads=4, d=d, in_dtype=in_dtype)
+    lay = stq.Layout(bits, d, in_dtype=in_dtype, scale_dtype=torch.bfloat16)
+    w = wlm.impact_weights(wl_)
+    S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(2)])
+    opool = _oracle_pool(orc, bits, d, S0, w)
+    offs, total = _layout(orc, bits, d)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    tally = Tally()
+    tally.updates_per_check = T
+    for call in range(2):
+        inp = wlm.prefill_inputs(wl_, call * T, T)
+        pool = torch.from_numpy(opool.copy()).to(DEV)
+        o = torch.zeros(2, 4, T, d, device=DEV)
+        stq.prefill_chunk(lay, pool, torch.arange(2, dtype=torch.int32, device=DEV),
+                          *(inp[n].to(DEV) for n in ("q", "k", "v", "beta", "alpha")), w.to(DEV), o, chunk=64,
+                          status=status)
+        torch.cuda.synchronize()
+        assert status.item() == 0, stq.status_flags(status)
+        gp, og = pool.cpu().numpy(), o.cpu().numpy()
+        for r in range(2):
+            for h, b in enumerate(bits):
+                blk = _tile(orc, opool, bits, d, r, h)
+                args = [as_f64(inp[n][r, h]) for n in ("q", "k", "v", "beta", "alpha")]
+                what = f"call {call} req {r} head {h}"
+                got = _tile(orc, gp, bits, d, r, h)
+                if b == 16:
+                    res = orc.prefill_seq_s(16, orc.SCALE_BF16, 0, blk, *args, as_f64(w[h]), 64, d, d)
+                    # a pivot carries T fp32 updates inside the chunk: the per-step bound times T
+                    M = T * np.max(np.abs(orc.dequantize(16, d, d, blk))) * np.ones((d, d)) * 4.0
+                    compare_block(orc, 16, d, got, res["block"], res["tie"], tally, what, err_scale=M)
+                else:
+                    S = orc.dequantize_s(b, orc.SCALE_BF16, d, d, blk)
+                    for t in range(T):
+                        S, _ = orc.update(0, S, args[0][t], args[1][t], args[2][t], args[3][t], args[4][t])
+                    res = orc.prefill_seq_s(b, orc.SCALE_BF16, 0, blk, *args, as_f64(w[h]), 64, d, d)
+                    compare_block_bf16s(orc, b, d, got, S, as_f64(w[h]), tally, what)
+                for t in range(T):
+                    compare_o(og[r, h, t], res["o"][t], tally, f"o token {t} " + what)
+                opool[r * total + offs[h]: r * total + offs[h] + res["block"].size] = res["block"]
+    tally.check_budget()
