@@ -91,9 +91,12 @@ def lib():
             L.orc_quantize_s.argtypes = [i32, i32, i32, i32, P, P, P, P, P, P, P, P, f64]
             L.orc_quantize_s.restype = i32
             L.orc_dequantize_s.argtypes, L.orc_dequantize_s.restype = [i32, i32, i32, i32, P, P], i32
-            L.orc_decode_step_s.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, f64, P, P, P, P, P, P, P, f64]
+            L.orc_decode_step_s.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, P, f64, P, P, P, P, P, P, P, f64]
             L.orc_decode_step_s.restype = i32
-            L.orc_prefill_seq_s.argtypes = [i32, i32, i32, i32, i32, P, i32, i32, P, P, P, P, P, P, P, P, P, P, f64]
+            L.orc_prefill_seq_s.argtypes = [i32, i32, i32, i32, i32, i32, P, i32, i32, P, P, P, P, P, P, P, P, P, P,
+                                            f64]
+            L.orc_quantize_fit.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P, f64]
+            L.orc_quantize_fit.restype = i32
             L.orc_prefill_seq_s.restype = i32
             _lib = L
     return _lib
@@ -368,7 +371,7 @@ def scales_s(bits: int, sfmt: int, dk: int, dv: int, block):
 
 
 def decode_step_s(bits: int, sfmt: int, gate: int, block, q, k, v, beta: float, alpha, w, dk: int, dv: int,
-                  delta: float = TIE_DELTA):
+                  delta: float = TIE_DELTA, rounds: int = 0):
     """One decode step on a copy of ``block`` with scales in format sfmt. Returns dict(block, o,
     S_new (fp64 before requantization), x, tie, scale_tie, status)."""
     blk = np.ascontiguousarray(np.asarray(block, dtype=np.uint8)).copy()
@@ -379,14 +382,14 @@ def decode_step_s(bits: int, sfmt: int, gate: int, block, q, k, v, beta: float, 
     stie = np.zeros(dk + dv, dtype=np.uint8)
     a = _f64(np.atleast_1d(alpha))
     wv = _f64(np.ones(dk) if w is None else w)
-    st = lib().orc_decode_step_s(bits, sfmt, dk, dv, gate, _p(blk), _p(_f64(q)), _p(_f64(k)), _p(_f64(v)),
+    st = lib().orc_decode_step_s(bits, sfmt, rounds, dk, dv, gate, _p(blk), _p(_f64(q)), _p(_f64(k)), _p(_f64(v)),
                                  float(beta), _p(a), _p(wv), _p(o), _p(S_new), _p(x), _p(tie), _p(stie),
                                  float(delta))
     return dict(block=blk, o=o, S_new=S_new, x=x, tie=tie.astype(bool), scale_tie=stie.astype(bool), status=st)
 
 
 def prefill_seq_s(bits: int, sfmt: int, gate: int, block, q, k, v, beta, alpha, w, chunk: int, dk: int, dv: int,
-                  delta: float = TIE_DELTA):
+                  delta: float = TIE_DELTA, rounds: int = 0):
     """Sequential chunked prefill on a copy of ``block`` with scales in format sfmt."""
     blk = np.ascontiguousarray(np.asarray(block, dtype=np.uint8)).copy()
     q, k, v = _f64(q), _f64(k), _f64(v)
@@ -395,7 +398,21 @@ def prefill_seq_s(bits: int, sfmt: int, gate: int, block, q, k, v, beta, alpha, 
     x = np.zeros((dk, dv))
     tie = np.zeros((dk, dv), dtype=np.uint8)
     stie = np.zeros(dk + dv, dtype=np.uint8)
-    st = lib().orc_prefill_seq_s(bits, sfmt, dk, dv, gate, _p(blk), T, chunk, _p(q), _p(k), _p(v),
+    st = lib().orc_prefill_seq_s(bits, sfmt, rounds, dk, dv, gate, _p(blk), T, chunk, _p(q), _p(k), _p(v),
                                  _p(_f64(beta)), _p(_f64(alpha)), _p(_f64(w)), _p(o), _p(x), _p(tie), _p(stie),
                                  float(delta))
     return dict(block=blk, o=o, x=x, tie=tie.astype(bool), scale_tie=stie.astype(bool), status=st)
+
+
+def quantize_fit(bits: int, sfmt: int, rounds: int, S, w=None, delta: float = TIE_DELTA):
+    """One-pass fit plus `rounds` rounds of the impact-weighted joint refinement (stq_oracle.c).
+    Returns (block, x, tie, status)."""
+    S = _f64(S)
+    dk, dv = S.shape
+    w = _f64(np.ones(dk) if w is None else w)
+    block = np.zeros(block_bytes_s(bits, sfmt, dk, dv), dtype=np.uint8)
+    x = np.zeros((dk, dv))
+    tie = np.zeros((dk, dv), dtype=np.uint8)
+    st = lib().orc_quantize_fit(bits, sfmt, rounds, dk, dv, _p(S), _p(w), _p(block), _p(x), _p(tie), None,
+                                float(delta))
+    return block, x, tie.astype(bool), st

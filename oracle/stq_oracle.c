@@ -394,6 +394,92 @@ int orc_quantize_s(int bits, int sfmt, int dk, int dv, const double *S, const do
     return nonfinite ? ORC_ENONFINITE : ORC_OK;
 }
 
+/* ------------------------------------------------------------------------------------------ */
+/* Impact-aware joint refinement of the two scales                                            */
+/*                                                                                            */
+/* [P5 空间维度]: the output error is the sum over key rows of each row's error weighted by a   */
+/* coefficient whose mean square is the row impact score; the column scale is fitted by       */
+/* weighted least squares in which high-impact rows weigh more; the row scale reflects the     */
+/* row's magnitude and its impact; [P1 方法]: the two scales are fitted jointly.               */
+/* READING c23: after the one-pass fit above, `rounds` rounds of alternating least squares on  */
+/* the impact-weighted reconstruction error  E = sum_i w_i sum_j (S_ij - r_i c_j Q_ij)^2:      */
+/*   c_j <- sum_i w_i r~_i Q_ij S_ij / sum_i w_i (r~_i Q_ij)^2        (codes Q of the last round) */
+/*   r_i <- sum_j c~_j Q_ij S_ij / sum_j (c~_j Q_ij)^2                (new stored c~, same Q)    */
+/*   Q_ij <- clamp(round_half_even((S_ij / c~_j) / r~_i), -qmax, qmax)                         */
+/* each new scale stored (fp32 or bf16) before it is used; a scale whose denominator is 0, or  */
+/* whose new value is not finite and positive, keeps its previous value. The weight of a row   */
+/* multiplies all of that row's terms, so the row step does not depend on w_i: impact reaches */
+/* the row scales through the jointly fitted column scales. With rounds = 0 this is the       */
+/* one-pass quantizer.                                                                        */
+/* ------------------------------------------------------------------------------------------ */
+
+static void codes_with(int bits, int dk, int dv, const double *S, const double *cs, const double *rs, int32_t *Q)
+{
+    int qmax = orc_qmax(bits);
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j) {
+            size_t e = (size_t)i * dv + j;
+            double x = (S[e] / cs[j]) / rs[i];
+            double qv = orc_round_half_even(x);
+            if (qv > qmax) qv = qmax;
+            if (qv < -qmax) qv = -qmax;
+            if (!isfinite(x)) qv = 0.0;
+            Q[e] = (int32_t)qv;
+        }
+}
+
+int orc_quantize_fit(int bits, int sfmt, int rounds, int dk, int dv, const double *S, const double *w,
+                     uint8_t *block, double *x_out, uint8_t *tie_out, uint8_t *stie_out, double delta)
+{
+    if (rounds < 0) return ORC_EINVAL;
+    int st = orc_quantize_s(bits, sfmt, dk, dv, S, w, NULL, NULL, block, x_out, tie_out, stie_out, delta);
+    if (bits == 16 || rounds == 0 || st == ORC_EINVAL) return st;
+    size_t n = (size_t)dk * dv;
+    size_t soff = orc_scale_offset(bits, dk, dv);
+    size_t sb = scale_bytes(sfmt);
+    double *cs = (double *)malloc(sizeof(double) * dv);
+    double *rs = (double *)malloc(sizeof(double) * dk);
+    int32_t *Q = (int32_t *)malloc(sizeof(int32_t) * n);
+    for (int i = 0; i < dk; ++i) rs[i] = load_scale(sfmt, block + soff + sb * (size_t)i);
+    for (int j = 0; j < dv; ++j) cs[j] = load_scale(sfmt, block + soff + sb * ((size_t)dk + (size_t)j));
+    if (stie_out) memset(stie_out, 0, (size_t)dk + (size_t)dv);
+    for (int round = 0; round < rounds; ++round) {
+        int last = round == rounds - 1;
+        codes_with(bits, dk, dv, S, cs, rs, Q);
+        for (int j = 0; j < dv; ++j) {
+            double num = 0.0, den = 0.0;
+            for (int i = 0; i < dk; ++i) {
+                double a = rs[i] * (double)Q[(size_t)i * dv + j];
+                num += w[i] * a * S[(size_t)i * dv + j];
+                den += w[i] * a * a;
+            }
+            if (den > 0.0) {
+                double c = stored_scale(sfmt, num / den);
+                if (isfinite(c) && c > 0.0) cs[j] = c;
+                if (last && stie_out) stie_out[dk + j] = scale_tie_distance(sfmt, num / den) <= delta;
+            }
+        }
+        for (int i = 0; i < dk; ++i) {
+            double num = 0.0, den = 0.0;
+            for (int j = 0; j < dv; ++j) {
+                double a = cs[j] * (double)Q[(size_t)i * dv + j];
+                num += a * S[(size_t)i * dv + j];
+                den += a * a;
+            }
+            if (den > 0.0) {
+                double r = stored_scale(sfmt, num / den);
+                if (isfinite(r) && r > 0.0) rs[i] = r;
+                if (last && stie_out) stie_out[i] = scale_tie_distance(sfmt, num / den) <= delta;
+            }
+        }
+    }
+    st = orc_quantize_s(bits, sfmt, dk, dv, S, w, cs, rs, block, x_out, tie_out, NULL, delta);
+    free(cs);
+    free(rs);
+    free(Q);
+    return st;
+}
+
 int orc_quantize(int bits, int dk, int dv, const double *S, const double *w, uint8_t *block,
                  double *x_out, uint8_t *tie_out, double delta)
 {
@@ -482,7 +568,7 @@ void orc_update(int dk, int dv, int gate, double *S, const double *q, const doub
  * o is emitted as fp32 (RNE of the fp64 value). S_new_out (optional) receives the fp64
  * updated state before requantization. x_out / tie_out (optional) receive the requantizer's
  * real-valued codes and near-tie flags. */
-int orc_decode_step_s(int bits, int sfmt, int dk, int dv, int gate, uint8_t *block, const double *q,
+int orc_decode_step_s(int bits, int sfmt, int rounds, int dk, int dv, int gate, uint8_t *block, const double *q,
                       const double *k, const double *v, double beta, const double *alpha,
                       const double *w, float *o, double *S_new_out, double *x_out,
                       uint8_t *tie_out, uint8_t *stie_out, double delta)
@@ -502,7 +588,7 @@ int orc_decode_step_s(int bits, int sfmt, int dk, int dv, int gate, uint8_t *blo
         if (!isfinite(o[j])) nonfinite = 1;
     }
     if (S_new_out) memcpy(S_new_out, S, sizeof(double) * n);
-    int st = orc_quantize_s(bits, sfmt, dk, dv, S, w, NULL, NULL, block, x_out, tie_out, stie_out, delta);
+    int st = orc_quantize_fit(bits, sfmt, rounds, dk, dv, S, w, block, x_out, tie_out, stie_out, delta);
     free(S);
     free(od);
     if (st != ORC_OK) return st;
@@ -514,7 +600,7 @@ int orc_decode_step(int bits, int dk, int dv, int gate, uint8_t *block, const do
                     const double *w, float *o, double *S_new_out, double *x_out,
                     uint8_t *tie_out, double delta)
 {
-    return orc_decode_step_s(bits, ORC_SCALE_F32, dk, dv, gate, block, q, k, v, beta, alpha, w, o, S_new_out,
+    return orc_decode_step_s(bits, ORC_SCALE_F32, 0, dk, dv, gate, block, q, k, v, beta, alpha, w, o, S_new_out,
                              x_out, tie_out, NULL, delta);
 }
 
@@ -528,7 +614,7 @@ int orc_decode_step(int bits, int dk, int dv, int gate, uint8_t *block, const do
 /* Layouts: q,k [T][dk], v [T][dv], beta [T], alpha [T] (scalar gate) or [T][dk], o [T][dv].  */
 /* ------------------------------------------------------------------------------------------ */
 
-int orc_prefill_seq_s(int bits, int sfmt, int dk, int dv, int gate, uint8_t *block, int T, int chunk,
+int orc_prefill_seq_s(int bits, int sfmt, int rounds, int dk, int dv, int gate, uint8_t *block, int T, int chunk,
                       const double *q, const double *k, const double *v, const double *beta,
                       const double *alpha, const double *w, float *o, double *x_out,
                       uint8_t *tie_out, uint8_t *stie_out, double delta)
@@ -551,7 +637,7 @@ int orc_prefill_seq_s(int bits, int sfmt, int dk, int dv, int gate, uint8_t *blo
                 if (!isfinite(o[(size_t)t * dv + j])) status = ORC_ENONFINITE;
             }
         }
-        int st = orc_quantize_s(bits, sfmt, dk, dv, S, w, NULL, NULL, block, x_out, tie_out, stie_out, delta);
+        int st = orc_quantize_fit(bits, sfmt, rounds, dk, dv, S, w, block, x_out, tie_out, stie_out, delta);
         if (st == ORC_EINVAL) status = st;
         if (st == ORC_ENONFINITE && status == ORC_OK) status = st;
     }
@@ -565,7 +651,7 @@ int orc_prefill_seq(int bits, int dk, int dv, int gate, uint8_t *block, int T, i
                     const double *alpha, const double *w, float *o, double *x_out,
                     uint8_t *tie_out, double delta)
 {
-    return orc_prefill_seq_s(bits, ORC_SCALE_F32, dk, dv, gate, block, T, chunk, q, k, v, beta, alpha, w, o,
+    return orc_prefill_seq_s(bits, ORC_SCALE_F32, 0, dk, dv, gate, block, T, chunk, q, k, v, beta, alpha, w, o,
                              x_out, tie_out, NULL, delta);
 }
 

@@ -43,6 +43,8 @@ int orc_quantize_s(int bits, int sfmt, int dk, int dv, const double *S, const do
                    const double *c_given, const double *r_given, uint8_t *block, double *x_out,
                    uint8_t *tie_out, uint8_t *stie_out, double delta);
 int orc_dequantize_s(int bits, int sfmt, int dk, int dv, const uint8_t *block, double *S);
+int orc_quantize_fit(int bits, int sfmt, int rounds, int dk, int dv, const double *S, const double *w,
+                     uint8_t *block, double *x_out, uint8_t *tie_out, uint8_t *stie_out, double delta);
 
 void orc_update(int dk, int dv, int gate, double *S, const double *q, const double *k,
                 const double *v, double beta, const double *alpha, double *o);
@@ -50,7 +52,7 @@ int orc_decode_step(int bits, int dk, int dv, int gate, uint8_t *block, const do
                     const double *k, const double *v, double beta, const double *alpha,
                     const double *w, float *o, double *S_new_out, double *x_out,
                     uint8_t *tie_out, double delta);
-int orc_decode_step_s(int bits, int sfmt, int dk, int dv, int gate, uint8_t *block, const double *q,
+int orc_decode_step_s(int bits, int sfmt, int rounds, int dk, int dv, int gate, uint8_t *block, const double *q,
                       const double *k, const double *v, double beta, const double *alpha,
                       const double *w, float *o, double *S_new_out, double *x_out,
                       uint8_t *tie_out, uint8_t *stie_out, double delta);
@@ -58,7 +60,7 @@ int orc_prefill_seq(int bits, int dk, int dv, int gate, uint8_t *block, int T, i
                     const double *q, const double *k, const double *v, const double *beta,
                     const double *alpha, const double *w, float *o, double *x_out,
                     uint8_t *tie_out, double delta);
-int orc_prefill_seq_s(int bits, int sfmt, int dk, int dv, int gate, uint8_t *block, int T, int chunk,
+int orc_prefill_seq_s(int bits, int sfmt, int rounds, int dk, int dv, int gate, uint8_t *block, int T, int chunk,
                       const double *q, const double *k, const double *v, const double *beta,
                       const double *alpha, const double *w, float *o, double *x_out,
                       uint8_t *tie_out, uint8_t *stie_out, double delta);

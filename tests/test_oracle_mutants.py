@@ -25,6 +25,9 @@ MUTANTS = {
     "bf16_truncates": ("double r = orc_round_half_even(ldexp(a, 7 - e));", "double r = floor(ldexp(a, 7 - e));"),
     "bf16_scale_stored_as_fp32": ("if (sfmt == ORC_SCALE_BF16) return orc_bf16_to_double(orc_double_to_bf16(v));",
                                   "if (sfmt == ORC_SCALE_BF16) return (double)(float)v;"),
+    "fit_column_unweighted": ("num += w[i] * a * S[(size_t)i * dv + j];", "num += a * S[(size_t)i * dv + j];"),
+    "fit_row_without_column_scale": ("double a = cs[j] * (double)Q[(size_t)i * dv + j];",
+                                     "double a = (double)Q[(size_t)i * dv + j];"),
     "row_scale_from_unrounded_column": ("cs[j] = stored_scale(sfmt, c);\n", "cs[j] = c;\n"),
     "column_scale_no_sqrt": ("double c = sqrt(acc / W);", "double c = acc / W;"),
     "row_scale_ignores_column": ("double t = fabs(S[(size_t)i * dv + j] / cs[j]);",

@@ -772,3 +772,65 @@ def test_bf16_decode_step_is_update_then_requantization(orc):
     assert np.array_equal(res["o"], o.astype(np.float32))
     assert np.array_equal(res["block"], orc.quantize_s(4, orc.SCALE_BF16, S1, w)[0])
     assert res["block"].size == orc.block_bytes_s(4, orc.SCALE_BF16, d, d)
+
+
+
+# ----------------------------------------------------------------------------------------------
+# Impact-aware joint refinement of the scales (alternating weighted least squares)
+# ----------------------------------------------------------------------------------------------
+
+def _weighted_error(orc, bits, sfmt, S, w, block):
+    d_k, d_v = S.shape
+    r, c = orc.scales_s(bits, sfmt, d_k, d_v, block)
+    Q = orc.codes(bits, d_k, d_v, block)
+    return float((w[:, None] * (S - r[:, None] * c[None, :] * Q) ** 2).sum())
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("sfmt", [0, 1])
+def test_fit_rounds_never_raise_the_weighted_error(orc, bits, sfmt):
+    """Each least-squares step minimises the impact-weighted error for fixed codes and each code
+    step picks the nearest codes for fixed scales, so the error cannot rise from round to round
+    (up to the rounding of the stored scales); on an outlier state it falls."""
+    rng = np.random.default_rng(90 + bits + 10 * sfmt)
+    S = _outlier_state(rng, 64)
+    w = np.exp(rng.normal(0, 1, 64))
+    E = [_weighted_error(orc, bits, sfmt, S, w, orc.quantize_fit(bits, sfmt, k, S, w)[0]) for k in range(4)]
+    slack = 1e-6 if sfmt == 0 else 3e-2
+    for a, b in zip(E, E[1:]):
+        assert b <= a * (1 + slack), E
+    assert E[3] < E[0], E
+    assert np.array_equal(orc.quantize_fit(bits, sfmt, 0, S, w)[0], orc.quantize_s(bits, sfmt, S, w)[0])
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_fit_rounds_keep_an_exact_fit(orc, bits):
+    """An exactly representable state (the exact round-trip fixture) is a fixed point."""
+    g, k = EXACT_ROWS[bits]
+    d = 8
+    rng = np.random.default_rng(bits)
+    G = np.array([[g[(j - i) % d] for j in range(d)] for i in range(d)], dtype=np.float64)
+    G *= np.where(rng.random((d, d)) < 0.5, -1.0, 1.0)
+    c = (128 + rng.integers(0, 128, d)) / 128.0 * 2.0 ** rng.integers(-6, 6, d)
+    S = G * c[None, :]
+    w = np.full(d, 0.7)
+    for sfmt in (0, 1):
+        blk = orc.quantize_fit(bits, sfmt, 3, S, w)[0]
+        assert np.array_equal(blk, orc.quantize_fit(bits, sfmt, 0, S, w)[0])
+        assert np.array_equal(orc.dequantize_s(bits, sfmt, d, d, blk), S)
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_fit_follows_the_impact_weights(orc, bits):
+    """The weight on two key rows: two rounds of the joint fit cut those rows' error to a small
+    fraction of the one-pass error, and of the error left by the same fit run with equal weights
+    (a dropped weight, or a transposed index in the column step, would not)."""
+    rng = np.random.default_rng(95 + bits)
+    d = 24
+    S = _outlier_state(rng, d)
+    w = np.full(d, 1e-9)
+    w[[3, 11]] = 1.0
+    e_one = _weighted_error(orc, bits, 0, S, w, orc.quantize_fit(bits, 0, 0, S, w)[0])
+    e_fit = _weighted_error(orc, bits, 0, S, w, orc.quantize_fit(bits, 0, 2, S, w)[0])
+    e_eq = _weighted_error(orc, bits, 0, S, w, orc.quantize_fit(bits, 0, 2, S, np.ones(d))[0])
+    assert e_fit < 0.2 * e_one and e_fit < 0.2 * e_eq, (e_one, e_fit, e_eq)
