@@ -390,7 +390,8 @@ def run_ours(args):
                                          stq.Layout(bits, d).bytes_per_request, bits.count(16))
         del S_cal
     scale_dtype = torch.bfloat16 if args.scale_dtype == "bf16" else torch.float32
-    lay = stq.Layout(bits, d, gate=wl.gate, in_dtype=wl.in_dtype, scale_dtype=scale_dtype)
+    lay = stq.Layout(bits, d, gate=wl.gate, in_dtype=wl.in_dtype, scale_dtype=scale_dtype,
+                     fit_rounds=args.fit_rounds)
     pool = lay.alloc_pool(B, dev)
     slots = torch.arange(B, dtype=torch.int32, device=dev)
     w = wlm.impact_weights(wl, dev)
@@ -540,7 +541,7 @@ def run_ours(args):
         "config": {"workload": args.workload, "batch_per_gpu": B, "heads": H, "d_k": d, "d_v": d,
                    "widths": {str(b): bits.count(b) for b in sorted(set(bits))}, "in_dtype": str(wl.in_dtype),
                    "gate": "scalar" if wl.gate == 0 else "channel", "tokens_cycled": TOKENS_CYCLED,
-                   "scale_dtype": args.scale_dtype,
+                   "scale_dtype": args.scale_dtype, "fit_rounds": args.fit_rounds,
                    "l2": "no flush: the 2.0 GB state pool read+written per step exceeds the 126 MB L2",
                    "generation_tokens": gen,
                    "timing": "CUDA events around each step; the pool restarts from its initial state every "
@@ -627,6 +628,8 @@ def main(argv=None):
     ap.add_argument("--batch", type=int, default=0, help="requests per GPU (default: the workload's)")
     ap.add_argument("--scale-dtype", choices=("f32", "bf16"), default="f32",
                     help="storage of the row and column scales (bf16: the 16-bit scale format)")
+    ap.add_argument("--fit-rounds", type=int, default=0,
+                    help="rounds of the impact-weighted joint scale refinement (runs on the plain kernels)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -21,7 +21,13 @@
  * Scales are stored as fp32 (or, with scale_dtype = STQ_BF16, as bf16 rounded half to even: the
  * 16-bit scales that bring a 6-bit 128 x 128 head to 5.12x compression, the figure the k1 page's
  * section 實驗結果 reports as ~5.03x with pivots) and codes are computed from the stored scales,
- * column scales first, then the row scales from the stored column scales; a pivot head (b = 16)
+ * column scales first, then the row scales from the stored column scales. A layout may ask for
+ * scale_fit_rounds rounds of joint refinement after that fit (the pages fit the two scales jointly,
+ * weighting high-impact rows more: "线性注意力状态量化难题", section 空间维度): each round refits
+ * every column scale by impact-weighted least squares, c_j = sum_i w_i a_ij S_ij / sum_i w_i a_ij^2
+ * with a_ij = r_i Q_ij, then every row scale by least squares, r_i = sum_j b_ij S_ij / sum_j b_ij^2
+ * with b_ij = c_j Q_ij (new c, same Q), then recomputes the codes; a refit value that is not finite
+ * and positive keeps the old one. A pivot head (b = 16)
  * stores S' as fp16 (round to nearest even) and has no scales. With the channel gate alpha is a
  * vector over key rows: STQ_GATE_CHANNEL substitutes it literally,
  * S'_ij = alpha_i (S_ij - beta k_i u_j) + beta k_i v_j; STQ_GATE_CHANNEL_DECAY_FIRST decays first,
@@ -64,7 +70,7 @@
 extern "C" {
 #endif
 
-#define STQ_ABI_VERSION 3
+#define STQ_ABI_VERSION 4
 
 typedef enum {
     STQ_OK = 0,
@@ -102,6 +108,8 @@ typedef struct {
     int32_t scale_mode;        /* stq_scale_mode (0: the method's row x column scales)       */
     int32_t scale_dtype;       /* stq_dtype of the stored row and column scales: STQ_F32 (0) */
                                /* or STQ_BF16 (16-bit scales; row x column mode only)        */
+    int32_t scale_fit_rounds;  /* 0: the one-pass fit above. 1..8: that many rounds of the    */
+                               /* impact-weighted joint refinement (row x column mode only)  */
 } stq_layout_desc;
 
 typedef struct stq_layout stq_layout; /* opaque, host-only, immutable after creation */

@@ -41,7 +41,8 @@ class StqError(RuntimeError):
 class _Desc(ctypes.Structure):
     _fields_ = [("num_heads", ctypes.c_int32), ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32),
                 ("head_bits", ctypes.POINTER(ctypes.c_uint8)), ("gate", ctypes.c_int32),
-                ("in_dtype", ctypes.c_int32), ("scale_mode", ctypes.c_int32), ("scale_dtype", ctypes.c_int32)]
+                ("in_dtype", ctypes.c_int32), ("scale_mode", ctypes.c_int32), ("scale_dtype", ctypes.c_int32),
+                ("scale_fit_rounds", ctypes.c_int32)]
 
 
 _lock = threading.Lock()
@@ -122,18 +123,19 @@ class Layout:
 
     def __init__(self, head_bits: Sequence[int], d: int, gate: int = GATE_SCALAR,
                  in_dtype: torch.dtype = torch.bfloat16, scale_mode: int = SCALES_ROW_COLUMN,
-                 scale_dtype: torch.dtype = torch.float32):
+                 scale_dtype: torch.dtype = torch.float32, fit_rounds: int = 0):
         self.head_bits = [int(b) for b in head_bits]
         self.H, self.d, self.gate, self.in_dtype = len(self.head_bits), int(d), int(gate), in_dtype
         self.scale_mode = int(scale_mode)
         self.scale_dtype = scale_dtype
+        self.fit_rounds = int(fit_rounds)
         if in_dtype not in _DTYPES:
             raise TypeError(f"unsupported input dtype {in_dtype}")
         if scale_dtype not in _DTYPES:
             raise TypeError(f"unsupported scale dtype {scale_dtype}")
         arr = (ctypes.c_uint8 * self.H)(*self.head_bits)
         desc = _Desc(self.H, self.d, self.d, ctypes.cast(arr, ctypes.POINTER(ctypes.c_uint8)),
-                     self.gate, _DTYPES[in_dtype], self.scale_mode, _DTYPES[scale_dtype])
+                     self.gate, _DTYPES[in_dtype], self.scale_mode, _DTYPES[scale_dtype], self.fit_rounds)
         handle = ctypes.c_void_p()
         _check(lib().stq_layout_create(ctypes.byref(desc), ctypes.byref(handle)), "stq_layout_create")
         self._h = handle

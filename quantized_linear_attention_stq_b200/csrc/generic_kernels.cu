@@ -18,6 +18,7 @@ struct TileRef {
     bool ok;
     bool uniform;  // one scale for the whole head (the baseline quantizer)
     int sb16;      // row and column scales stored as bf16
+    int rounds;    // rounds of the impact-weighted joint refinement of the scales
     int b, head, bits;
     uint8_t *block;
 };
@@ -31,6 +32,7 @@ __device__ __forceinline__ TileRef tile_ref(const TileParams &p, int b, int pos)
     t.bits = entry_bits(e);
     t.uniform = entry_uniform(e);
     t.sb16 = p.scale_bf16;
+    t.rounds = p.fit_rounds;
     const int slot = p.slots[b];
     t.ok = slot >= 0 && slot < p.pool_slots;
     t.block = t.ok ? p.pool + (uint64_t)slot * p.req_bytes + e.off : nullptr;
@@ -77,8 +79,56 @@ __device__ void dequant_to_smem(const uint8_t *block, int bits, bool uniform, in
 // Fit scales to the fp32 state in S and write codes + scales into `block` (or fp16 values for a
 // pivot head). `wv` holds the impact weights of the head in shared memory. Needs a CTA-wide
 // barrier before (S complete) and provides one after.
-__device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, bool uniform, int sb16, int dk,
-                                   int dv, uint8_t *block, float *cs, float *rs, int32_t *status)
+// Signed code of x = (s / c) / r, rounded half to even and clamped (0 for a non-finite x).
+__device__ __forceinline__ float code_of(float s, float c, float r, float qmax)
+{
+    const float x = (s / c) / r;
+    return isfinite(x) ? fminf(fmaxf(rintf(x), -qmax), qmax) : 0.f;
+}
+
+// Rounds of alternating impact-weighted least squares on the stored scales cs[dv], rs[dk] (the
+// one-pass fit on entry): each round refits every column scale c_j = sum_i w_i a_i S_ij /
+// sum_i w_i a_i^2 with a_i = r_i Q_ij, then every row scale r_i = sum_j b_j S_ij / sum_j b_j^2
+// with b_j = c~_j Q_ij, both with the codes Q of the round's starting scales; each new value is
+// rounded to the storage format and kept only if finite and positive (else the old one stays).
+// Needs a CTA-wide barrier before and provides one after.
+__device__ void refine_scales(const float *S, int ld, const float *wv, float qmax, int sb16, int rounds, int dk,
+                              int dv, float *cs, float *rs)
+{
+    __shared__ float cn[128], rn[128];
+    for (int round = 0; round < rounds; ++round) {
+        for (int j = threadIdx.x; j < dv; j += blockDim.x) {
+            float num = 0.f, den = 0.f;
+            for (int i = 0; i < dk; ++i) {
+                const float s = S[i * ld + j];
+                const float a = rs[i] * code_of(s, cs[j], rs[i], qmax);
+                num += wv[i] * a * s;
+                den += wv[i] * a * a;
+            }
+            const float c = den > 0.f ? round_scale(num / den, sb16) : 0.f;
+            cn[j] = (isfinite(c) && c > 0.f) ? c : cs[j];
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < dk; i += blockDim.x) {
+            float num = 0.f, den = 0.f;
+            for (int j = 0; j < dv; ++j) {
+                const float s = S[i * ld + j];
+                const float b = cn[j] * code_of(s, cs[j], rs[i], qmax);
+                num += b * s;
+                den += b * b;
+            }
+            const float r = den > 0.f ? round_scale(num / den, sb16) : 0.f;
+            rn[i] = (isfinite(r) && r > 0.f) ? r : rs[i];
+        }
+        __syncthreads();
+        for (int j = threadIdx.x; j < dv; j += blockDim.x) cs[j] = cn[j];
+        for (int i = threadIdx.x; i < dk; i += blockDim.x) rs[i] = rn[i];
+        __syncthreads();
+    }
+}
+
+__device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, bool uniform, int sb16, int rounds,
+                                   int dk, int dv, uint8_t *block, float *cs, float *rs, int32_t *status)
 {
     const int n = dk * dv;
     __shared__ uint32_t smax;
@@ -152,6 +202,7 @@ __device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, 
         rs[i] = round_scale(r, sb16);
     }
     __syncthreads();
+    if (rounds > 0) refine_scales(S, ld, wv, qmax, sb16, rounds, dk, dv, cs, rs);
     bool bad = false;
     uint8_t *sg = block + scale_offset(bits, dk, dv);
     for (int i = threadIdx.x; i < dk; i += blockDim.x) {
@@ -202,7 +253,7 @@ __global__ void __launch_bounds__(kThreads) init_kernel(const __grid_constant__ 
     for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) S[(e / dv) * ld + e % dv] = src[e];
     for (int i = threadIdx.x; i < dk; i += blockDim.x) wv[i] = p.w[(uint64_t)t.head * dk + i];
     __syncthreads();
-    quantize_from_smem(S, ld, wv, t.bits, t.uniform, t.sb16, dk, dv, t.block, cs, rs, p.status);
+    quantize_from_smem(S, ld, wv, t.bits, t.uniform, t.sb16, t.rounds, dk, dv, t.block, cs, rs, p.status);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -281,7 +332,7 @@ __global__ void __launch_bounds__(kThreads) decode_generic_kernel(const __grid_c
         bad |= !isfinite(acc);
     }
     if (bad) flag(p.status, kFlagNonfinite);
-    quantize_from_smem(S, ld, wv, t.bits, t.uniform, t.sb16, dk, dv, t.block, cs, rs, p.status);
+    quantize_from_smem(S, ld, wv, t.bits, t.uniform, t.sb16, t.rounds, dk, dv, t.block, cs, rs, p.status);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -345,7 +396,7 @@ __global__ void __launch_bounds__(kThreads) prefill_seq_kernel(const __grid_cons
         }
         if ((tok + 1) % chunk == 0 || tok == T - 1) {
             __syncthreads();
-            quantize_from_smem(S, ld, wv, t.bits, t.uniform, t.sb16, dk, dv, t.block, cs, rs, p.status);
+            quantize_from_smem(S, ld, wv, t.bits, t.uniform, t.sb16, t.rounds, dk, dv, t.block, cs, rs, p.status);
             if (tok != T - 1) {
                 __syncthreads();
                 dequant_to_smem(t.block, t.bits, t.uniform, t.sb16, dk, dv, S, ld);

@@ -15,6 +15,7 @@ struct stq_layout {
     int32_t H, dk, dv, gate, in_dtype;
     bool uniform;  // STQ_SCALES_UNIFORM
     bool sb16;     // row and column scales stored as bf16
+    int fit_rounds;  // rounds of the impact-weighted joint refinement of the scales
     std::vector<uint8_t> bits;
     std::vector<uint64_t> offset;
     std::vector<uint64_t> bytes;
@@ -40,6 +41,7 @@ void fill_table(stq::TileParams &p, const stq_layout *L, const std::vector<int> 
 {
     p.npos = n;
     p.scale_bf16 = L->sb16 ? 1 : 0;
+    p.fit_rounds = L->fit_rounds;
     for (int e = 0; e < n; ++e) {
         const int h = ord[first + e];
         p.table[e].off = (uint32_t)L->offset[h];
@@ -88,6 +90,8 @@ stq_status stq_layout_create(const stq_layout_desc *desc, stq_layout **out)
     if (desc->scale_mode != STQ_SCALES_ROW_COLUMN && desc->scale_mode != STQ_SCALES_UNIFORM) return STQ_ERR_INVALID_ARG;
     if (desc->scale_dtype != STQ_F32 && desc->scale_dtype != STQ_BF16) return STQ_ERR_INVALID_ARG;
     if (desc->scale_dtype == STQ_BF16 && desc->scale_mode == STQ_SCALES_UNIFORM) return STQ_ERR_UNSUPPORTED;
+    if (desc->scale_fit_rounds < 0 || desc->scale_fit_rounds > 8) return STQ_ERR_INVALID_ARG;
+    if (desc->scale_fit_rounds > 0 && desc->scale_mode == STQ_SCALES_UNIFORM) return STQ_ERR_UNSUPPORTED;
     const int d = desc->d_k;
     if (desc->d_v != d || !(d == 16 || d == 32 || d == 64 || d == 128)) return STQ_ERR_UNSUPPORTED;
     if (desc->num_heads > 65535) return STQ_ERR_UNSUPPORTED;
@@ -100,6 +104,7 @@ stq_status stq_layout_create(const stq_layout_desc *desc, stq_layout **out)
     L->in_dtype = desc->in_dtype;
     L->uniform = desc->scale_mode == STQ_SCALES_UNIFORM;
     L->sb16 = desc->scale_dtype == STQ_BF16;
+    L->fit_rounds = desc->scale_fit_rounds;
     uint64_t pos = 0;
     for (int h = 0; h < L->H; ++h) {
         const int b = desc->head_bits[h];
@@ -222,7 +227,7 @@ stq_status stq_decode_step(const stq_layout *L, void *pool, int32_t pool_slots, 
     p->gate = L->gate;
     p->w = w;
     const int in_bf16 = L->in_dtype == STQ_BF16;
-    const bool tuned = L->dk == 128 && !L->uniform;
+    const bool tuned = L->dk == 128 && !L->uniform && L->fit_rounds == 0;
     const int maxb = tuned ? stq::decode_d128_max_requests() : 65535;
     const std::vector<int> ord = order_by_size(L, head_begin, head_count);
     const size_t in_sz = in_bf16 ? 2 : 4;
@@ -302,7 +307,7 @@ stq_status stq_prefill_chunk(const stq_layout *L, void *pool, int32_t pool_slots
     // WY path, one launch per code width; FP16 pivot heads and every other configuration take the
     // sequential kernel.
     const bool wy = L->dk == 128 && L->gate == STQ_GATE_SCALAR && L->in_dtype == STQ_BF16 && chunk == 64 &&
-                    !L->uniform;
+                    !L->uniform && L->fit_rounds == 0;
     if (!wy) {
         std::vector<int> ord(L->H);
         for (int h = 0; h < L->H; ++h) ord[h] = h;

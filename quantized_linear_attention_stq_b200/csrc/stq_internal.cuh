@@ -75,6 +75,7 @@ struct TileParams {
     int32_t dk, dv;
     int32_t gate;
     int32_t scale_bf16;  // 1: row and column scales stored as bf16 (else fp32)
+    int32_t fit_rounds;  // rounds of the impact-weighted joint refinement of the scales
     // decode / prefill inputs (indexed by request and call-relative head)
     const void *q, *k, *v;
     const float *beta, *alpha, *w;

@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol(stq):
         assert hasattr(L, name), name
         assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
     assert sorted(stq.api.EXPORTS) == declared_functions()
-    assert L.stq_abi_version() == 3
+    assert L.stq_abi_version() == 4
 
 
 def test_status_strings(stq):

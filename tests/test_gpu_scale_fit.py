@@ -1,0 +1,243 @@
+"""GPU parity of the impact-aware joint refinement of the scales against the oracle (needs a B200).
+
+A layout with fit_rounds = n refits, after the one-pass fit, every column scale by impact-weighted
+least squares and every row scale by least squares, n times, recomputing the codes in between
+(the pages fit the two scales jointly and weight high-impact rows more: "线性注意力状态量化难题"
+(aitest123.com/news/n1kj09), section 空间维度; "K1 論文詳解" (k1-news.pages.dev/paper/2026-10-09),
+section 方法). Such layouts run on the plain kernels. Teacher-forced protocol as in
+test_gpu_decode.py; blocks are compared with the joint-fit rule of tests/_parity.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+from _parity import (Tally, as_f64, compare_block, compare_block_fit, compare_o, oracle_pool, tile_bytes,
+                     update_magnitude)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+ROUNDS = 2
+
+
+@pytest.fixture(scope="module")
+def stq():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for the gpu tests")
+    import quantized_linear_attention_stq_b200 as m
+
+    m.lib()  # fails loudly if libstq.so is missing
+    return m
+
+
+def _wl(name, **changes):
+    from quantized_linear_attention_stq_b200 import workloads as wl
+
+    return wl.scaled(wl.WORKLOADS[name], **changes)
+
+
+def _oracle_pool(orc, bits, d, S0, w, rounds):
+    B, H = S0.shape[0], S0.shape[1]
+    blocks = []
+    for r in range(B):
+        row = []
+        for h in range(H):
+            blk, _, _, st = orc.quantize_fit(bits[h], orc.SCALE_F32, 0 if bits[h] == 16 else rounds,
+                                             as_f64(S0[r, h]), as_f64(w[h]))
+            assert st == orc.OK
+            row.append(blk)
+        blocks.append(row)
+    return oracle_pool(orc, bits, d, blocks)
+
+
+@pytest.mark.parametrize("d", [16, 128])
+def test_init(stq, orc, d):
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl_ = _wl("full2304_b70_mixed", batch=3, heads=6, d=d)
+    bits = [4, 6, 8, 16, 8, 6]
+    lay = stq.Layout(bits, d, fit_rounds=ROUNDS)
+    assert lay.bytes_per_request == stq.Layout(bits, d).bytes_per_request
+    w = wlm.impact_weights(wl_)
+    S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(3)])
+    pool = lay.alloc_pool(3)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stq.init_state(lay, pool, torch.arange(3, dtype=torch.int32, device=DEV), S0.to(DEV), w.to(DEV), status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    gp = pool.cpu().numpy()
+    tally = Tally()
+    for r in range(3):
+        for h in range(6):
+            got = tile_bytes(orc, gp, bits, d, r, h)
+            if bits[h] == 16:
+                blk, _, tie, _ = orc.quantize(16, as_f64(S0[r, h]), as_f64(w[h]))
+                compare_block(orc, 16, d, got, blk, tie, tally, f"init req {r} head {h}")
+            else:
+                compare_block_fit(orc, bits[h], d, got, as_f64(S0[r, h]), as_f64(w[h]), ROUNDS, tally,
+                                  f"init req {r} head {h}")
+    tally.check_budget()
+
+
+def _decode_teacher_forced(stq, orc, wl_, bits, steps):
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    B, H, d = wl_.batch, wl_.heads, wl_.d
+    lay = stq.Layout(bits, d, gate=wl_.gate, in_dtype=wl_.in_dtype, fit_rounds=ROUNDS)
+    w = wlm.impact_weights(wl_)
+    S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(B)])
+    opool = _oracle_pool(orc, bits, d, S0, w, ROUNDS)
+    offs, total = orc.request_layout(bits, d, d)
+    gpool = torch.zeros(B * total, dtype=torch.uint8, device=DEV)
+    slots = torch.arange(B, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    tally = Tally()
+    for t in range(steps):
+        inp = wlm.decode_inputs(wl_, t)
+        gpool.copy_(torch.from_numpy(opool.copy()).to(DEV))
+        o = torch.zeros(B, H, d, device=DEV)
+        g = {n: x.to(DEV) for n, x in inp.items()}
+        stq.decode_step(lay, gpool, slots, g["q"], g["k"], g["v"], g["beta"], g["alpha"], w.to(DEV), o,
+                        status=status)
+        torch.cuda.synchronize()
+        assert status.item() == 0, stq.status_flags(status)
+        gp, og = gpool.cpu().numpy(), o.cpu().numpy()
+        for r in range(B):
+            for h in range(H):
+                ref_blk = tile_bytes(orc, opool, bits, d, r, h)
+                q, k, v = as_f64(inp["q"][r, h]), as_f64(inp["k"][r, h]), as_f64(inp["v"][r, h])
+                beta, alpha = float(inp["beta"][r, h]), inp["alpha"][r, h].double().numpy()
+                rounds = 0 if bits[h] == 16 else ROUNDS
+                res = orc.decode_step_s(bits[h], orc.SCALE_F32, wl_.gate, ref_blk, q, k, v, beta, alpha,
+                                        as_f64(w[h]), d, d, rounds=rounds)
+                assert res["status"] == orc.OK
+                got = tile_bytes(orc, gp, bits, d, r, h)
+                what = f"step {t} req {r} head {h}"
+                if bits[h] == 16:
+                    M = update_magnitude(orc.dequantize(16, d, d, ref_blk), k, v, beta, alpha)
+                    compare_block(orc, 16, d, got, res["block"], res["tie"], tally, what, err_scale=M)
+                else:
+                    compare_block_fit(orc, bits[h], d, got, res["S_new"], as_f64(w[h]), ROUNDS, tally, what)
+                compare_o(og[r, h], res["o"], tally, "o " + what)
+                opool[r * total + offs[h]: r * total + offs[h] + res["block"].size] = res["block"]
+    tally.check_budget()
+
+
+def test_decode_d128_mixed_with_pivots(stq, orc):
+    wl_ = _wl("full2304_b70_mixed", batch=3, heads=8)
+    _decode_teacher_forced(stq, orc, wl_, [4, 16, 6, 8, 4, 6, 8, 6], 2)
+
+
+@pytest.mark.parametrize("gate", [1, 2])
+def test_decode_channel_gates(stq, orc, gate):
+    wl_ = _wl("channel32_b128_4bit", batch=2, heads=3, gate=gate, d=32, in_dtype=torch.float32)
+    _decode_teacher_forced(stq, orc, wl_, [4, 6, 8], 3)
+
+
+def test_prefill_chunk(stq, orc):
+    """A 64-token chunk and a 30-token chunk in one call (routed to the sequential kernel), one
+    request x three heads at d = 128, bf16 inputs: the first chunk's end state is checked through
+    the oracle's chunk, then the call's final block from the oracle's bytes after that chunk."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    bits, d, T = [4, 6, 8], 128, 94
+    wl_ = _wl("prefill16_b16_6bit", batch=1, heads=3)
+    lay = stq.Layout(bits, d, in_dtype=torch.bfloat16, fit_rounds=ROUNDS)
+    w = wlm.impact_weights(wl_)
+    S0 = wlm.initial_state(wl_, 0)[None]
+    opool = _oracle_pool(orc, bits, d, S0, w, ROUNDS)
+    inp = wlm.prefill_inputs(wl_, 0, T)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    tally = Tally()
+    # the 64-token chunk alone
+    pool = torch.from_numpy(opool.copy()).to(DEV)
+    o = torch.zeros(1, 3, 64, d, device=DEV)
+    stq.prefill_chunk(lay, pool, torch.zeros(1, dtype=torch.int32, device=DEV),
+                      *(inp[n][:, :, :64].contiguous().to(DEV) for n in ("q", "k", "v", "beta", "alpha")), w.to(DEV),
+                      o, chunk=64, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0, stq.status_flags(status)
+    gp, og = pool.cpu().numpy(), o.cpu().numpy()
+    offs, total = orc.request_layout(bits, d, d)
+    for h, b in enumerate(bits):
+        blk = tile_bytes(orc, opool, bits, d, 0, h)
+        args = [as_f64(inp[n][0, h, :64]) for n in ("q", "k", "v", "beta", "alpha")]
+        S = orc.dequantize(b, d, d, blk)
+        for t in range(64):
+            S, _ = orc.update(0, S, args[0][t], args[1][t], args[2][t], args[3][t], args[4][t])
+        res = orc.prefill_seq_s(b, orc.SCALE_F32, 0, blk, *args, as_f64(w[h]), 64, d, d, rounds=ROUNDS)
+        compare_block_fit(orc, b, d, tile_bytes(orc, gp, bits, d, 0, h), S, as_f64(w[h]), ROUNDS, tally,
+                          f"chunk 0 head {h}")
+        for t in range(64):
+            compare_o(og[0, h, t], res["o"][t], tally, f"o token {t} head {h}")
+        opool[offs[h]: offs[h] + res["block"].size] = res["block"]
+    # the 30-token rest from the oracle's bytes
+    pool = torch.from_numpy(opool.copy()).to(DEV)
+    o = torch.zeros(1, 3, T - 64, d, device=DEV)
+    stq.prefill_chunk(lay, pool, torch.zeros(1, dtype=torch.int32, device=DEV),
+                      *(inp[n][:, :, 64:].contiguous().to(DEV) for n in ("q", "k", "v", "beta", "alpha")), w.to(DEV),
+                      o, chunk=64, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0, stq.status_flags(status)
+    gp = pool.cpu().numpy()
+    for h, b in enumerate(bits):
+        blk = tile_bytes(orc, opool, bits, d, 0, h)
+        args = [as_f64(inp[n][0, h, 64:]) for n in ("q", "k", "v", "beta", "alpha")]
+        S = orc.dequantize(b, d, d, blk)
+        for t in range(T - 64):
+            S, _ = orc.update(0, S, args[0][t], args[1][t], args[2][t], args[3][t], args[4][t])
+        compare_block_fit(orc, b, d, tile_bytes(orc, gp, bits, d, 0, h), S, as_f64(w[h]), ROUNDS, tally,
+                          f"chunk 1 head {h}")
+    tally.check_budget()
+
+
+def test_study_joint_fit_error_accumulation(stq):
+    """The joint refinement against the one-pass scales over 256 decode tokens of all 2304 heads
+    of one request of the mixed workload, beside the exact fp64 recurrence (as the uniform
+    baseline study in test_gpu_uniform.py): per head the relative state error at the end and the
+    impact-weighted one, sum_i w_i |E_i|^2 / sum_i w_i |S_i|^2, the quantity the refinement fits."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl_ = _wl("full2304_b70_mixed", batch=1)
+    H, d, steps = wl_.heads, wl_.d, 256
+    w = wlm.impact_weights(wl_).to(DEV)
+    S0 = wlm.initial_state(wl_, 0).to(DEV)
+    slots = torch.zeros(1, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    runs = {}
+    for rounds in (0, ROUNDS):
+        for b in (4, 6, 8):
+            lay = stq.Layout([b] * H, d, fit_rounds=rounds)
+            pool = lay.alloc_pool(1, DEV)
+            stq.init_state(lay, pool, slots, S0[None].contiguous(), w, status=status)
+            runs[rounds, b] = dict(lay=lay, pool=pool)
+    S = S0.double()
+    for t in range(steps):
+        inp = {n: x.to(DEV) for n, x in wlm.decode_inputs(wl_, t).items()}
+        k, v = inp["k"][0].double(), inp["v"][0].double()
+        beta, alpha = inp["beta"][0].double()[:, None, None], inp["alpha"][0].double()[:, None, None]
+        u = torch.einsum("hi,hij->hj", k, S)
+        S = alpha * (S - beta * k[:, :, None] * u[:, None, :]) + beta * k[:, :, None] * v[:, None, :]
+        for run in runs.values():
+            o = torch.zeros(1, H, d, device=DEV)
+            stq.decode_step(run["lay"], run["pool"], slots, inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"],
+                            w, o, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0, stq.status_flags(status)
+    wd = w.double()[:, :, None]
+    print()
+    print("| width | fit rounds | median state err | p90 state err | median weighted err | p90 weighted err |")
+    print("|---|---|---|---|---|---|")
+    med = {}
+    for (rounds, b), run in sorted(runs.items(), key=lambda kv: (kv[0][1], kv[0][0])):
+        Sq = torch.zeros(1, H, d, d, device=DEV)
+        stq.dequantize(run["lay"], run["pool"], slots, Sq)
+        E = Sq[0].double() - S
+        err = (E.norm(dim=(1, 2)) / S.norm(dim=(1, 2))).cpu().numpy()
+        werr = ((wd * E ** 2).sum(dim=(1, 2)) / (wd * S ** 2).sum(dim=(1, 2))).sqrt().cpu().numpy()
+        med[rounds, b] = float(np.median(werr))
+        print(f"| {b} | {rounds} | {np.median(err):.3e} | {np.quantile(err, 0.9):.3e} | {np.median(werr):.3e} | "
+              f"{np.quantile(werr, 0.9):.3e} |")
+        assert np.isfinite(err).all()
+    for b in (6, 8):
+        assert med[ROUNDS, b] < med[0, b]
