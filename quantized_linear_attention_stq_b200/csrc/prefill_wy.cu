@@ -260,50 +260,122 @@ __device__ __forceinline__ void named_bar(int id, int count)
 
 // ---------------------------------------------------------------------------------------------
 // T = (I + L)^-1 for a strictly lower triangular 64 x 64 L given transposed (Lt[s][t] = L_ts, row
-// stride LDL), by right-looking forward substitution on the 64 columns of the identity, run by the
-// 128 threads of warps 12..15. Thread (warp wi, lane: column group g = lane / 8, row group q = lane
-// % 8) keeps rows 8q .. 8q+7 of columns c0 .. c0+3, c0 = 16 wi + 4 g; step s takes the final x_s of
-// each column from its owner by a shuffle and updates every row below it. The result goes to T.
+// stride LDL; its entries on and above the diagonal are zero), by 16 x 16 blocks, run by the 128
+// threads of warps 12..15 with the work split evenly:
+//   1. warp w inverts the diagonal block D_w = (I + L_ww)^-1 by forward substitution;
+//   2-4. the blocks at distance 1, 2, 3 below the diagonal, T_ij = -D_i sum_{k=j}^{i-1} L_ik T_kj:
+//        three blocks of 16 columns (one per warp), then two blocks as four jobs of 8 columns, then
+//        one block as four jobs of 4 columns; a job forms M = sum_k L_ik T_kj, parks it in a
+//        scratch block above the diagonal and multiplies by -D_i;
+//   5. the six blocks above the diagonal are zeroed.
+// In a job, lane (r = lane % 16, h = lane / 16) computes row r of the block, columns h nc/2 ..
+// (h + 1) nc/2 - 1 of the job's nc. The result goes to T (row-major, stride LDL).
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ void invert_unit_lower(const float *Lt, float *T)
+// NH consecutive floats from shared memory, 8-byte aligned (16-byte aligned for NH >= 4)
+template <int NH>
+__device__ __forceinline__ void load_row(const float *src, float (&v)[NH])
 {
-    const int wi = (threadIdx.x >> 5) - INV_WARP0, lane = threadIdx.x & 31;
-    const int g = lane >> 3, q = lane & 7, base = lane & ~7, c0 = 16 * wi + 4 * g;
-    float2 x[4][4];  // [column][row pair]
+    if constexpr (NH >= 4) {
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc)
+        for (int e = 0; e < NH; e += 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(src + e);
+            v[e] = a.x;
+            v[e + 1] = a.y;
+            v[e + 2] = a.z;
+            v[e + 3] = a.w;
+        }
+    } else {
+        const float2 a = *reinterpret_cast<const float2 *>(src);
+        v[0] = a.x;
+        v[1] = a.y;
+    }
+}
+
+template <int NC>
+__device__ __forceinline__ void inverse_block_job(const float *Lt, float *T, float *scr, int i, int j, int c_lo)
+{
+    constexpr int NH = NC / 2;
+    const int lane = threadIdx.x & 31, r = lane & 15, h = lane >> 4;
+    const int col = 16 * j + c_lo + h * NH;  // first absolute column of this lane
+    float m[NH];
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-            x[cc][k] = make_float2((8 * q + 2 * k == c0 + cc) ? 1.f : 0.f, (8 * q + 2 * k + 1 == c0 + cc) ? 1.f : 0.f);
-    // x_s = 0 for s < c0: the steps before the warp's first column change nothing
-#pragma unroll 1
-    for (int sb = 2 * wi; sb < 8; ++sb) {
+    for (int e = 0; e < NH; ++e) m[e] = 0.f;
+    for (int kb = j; kb < i; ++kb) {
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int s = 8 * sb + m;
-            const float4 l0 = *reinterpret_cast<const float4 *>(Lt + s * LDL + 8 * q);
-            const float4 l1 = *reinterpret_cast<const float4 *>(Lt + s * LDL + 8 * q + 4);
-            const float2 la = make_float2(l0.x, l0.y), lb = make_float2(l0.z, l0.w);
-            const float2 lc = make_float2(l1.x, l1.y), ld = make_float2(l1.z, l1.w);
+        for (int k = 0; k < 16; ++k) {
+            const float l = Lt[(16 * kb + k) * LDL + 16 * i + r];  // L(16i + r, 16kb + k)
+            float tr[NH];
+            load_row<NH>(T + (16 * kb + k) * LDL + col, tr);
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                const float own = (m & 1) ? x[cc][m >> 1].y : x[cc][m >> 1].x;
-                const float xs = -__shfl_sync(0xffffffffu, own, base | sb);
-                const float2 nx = make_float2(xs, xs);
-                x[cc][0] = __ffma2_rn(la, nx, x[cc][0]);
-                x[cc][1] = __ffma2_rn(lb, nx, x[cc][1]);
-                x[cc][2] = __ffma2_rn(lc, nx, x[cc][2]);
-                x[cc][3] = __ffma2_rn(ld, nx, x[cc][3]);
-            }
+            for (int e = 0; e < NH; ++e) m[e] = fmaf(l, tr[e], m[e]);
         }
     }
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc)
+    for (int e = 0; e < NH; ++e) scr[r * LDL + h * NH + e] = m[e];
+    __syncwarp();
+    float dr[16];  // row r of D_i
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            T[(8 * q + 2 * k) * LDL + c0 + cc] = x[cc][k].x;
-            T[(8 * q + 2 * k + 1) * LDL + c0 + cc] = x[cc][k].y;
+    for (int k4 = 0; k4 < 4; ++k4) {
+        const float4 v = *reinterpret_cast<const float4 *>(T + (16 * i + r) * LDL + 16 * i + 4 * k4);
+        dr[4 * k4] = v.x;
+        dr[4 * k4 + 1] = v.y;
+        dr[4 * k4 + 2] = v.z;
+        dr[4 * k4 + 3] = v.w;
+    }
+    float out[NH];
+#pragma unroll
+    for (int e = 0; e < NH; ++e) out[e] = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        float mk[NH];
+        load_row<NH>(scr + k * LDL + h * NH, mk);
+#pragma unroll
+        for (int e = 0; e < NH; ++e) out[e] = fmaf(dr[k], mk[e], out[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < NH; ++e) T[(16 * i + r) * LDL + col + e] = -out[e];
+    __syncwarp();  // the scratch block is read by every lane before the next job writes it
+}
+
+__device__ __forceinline__ void invert_unit_lower(const float *Lt, float *T)
+{
+    const int wi = (threadIdx.x >> 5) - INV_WARP0, lane = threadIdx.x & 31;
+    // scratch: a 16 x 16 block above the diagonal, (0, 1 + wi) for warps 0..2 and (1, 3) for warp 3
+    float *scr = wi < 3 ? T + 16 * (1 + wi) : T + 16 * LDL + 48;
+    if (lane < 16) {
+        // 1. D_wi by forward substitution, lane c < 16 keeping all of column c in registers (the
+        //    chain of steps needs no data from other lanes; the L rows are the same for every lane)
+        const int b = 16 * wi, c = lane;
+        float x[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[e] = (e == c) ? 1.f : 0.f;
+#pragma unroll
+        for (int sidx = 0; sidx < 15; ++sidx) {
+            float l[16];  // L(b + e, b + sidx), zero for e <= sidx
+            load_row<16>(Lt + (b + sidx) * LDL + b, l);
+#pragma unroll
+            for (int e = sidx + 1; e < 16; ++e) x[e] = fmaf(l[e], -x[sidx], x[e]);
         }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) T[(b + e) * LDL + b + c] = x[e];
+    }
+    named_bar(2, 128);
+    // 2. distance 1: blocks (1,0), (2,1), (3,2)
+    if (wi < 3) inverse_block_job<16>(Lt, T, scr, wi + 1, wi, 0);
+    named_bar(2, 128);
+    // 3. distance 2: blocks (2,0) and (3,1), 8 columns per warp
+    inverse_block_job<8>(Lt, T, scr, 2 + (wi >> 1), wi >> 1, 8 * (wi & 1));
+    named_bar(2, 128);
+    // 4. distance 3: block (3,0), 4 columns per warp
+    inverse_block_job<4>(Lt, T, scr, 3, 0, 4 * wi);
+    named_bar(2, 128);
+    // 5. zeros above the diagonal: blocks (0,1..3), (1,2..3), (2,3)
+    for (int e = threadIdx.x - 32 * INV_WARP0; e < 6 * 256; e += 128) {
+        const int blk = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+        const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+        const int bj = blk < 3 ? 1 + blk : (blk < 5 ? blk - 1 : 3);
+        T[(16 * bi + rr) * LDL + 16 * bj + cc] = 0.f;
+    }
     named_bar(2, 128);
 }
 
