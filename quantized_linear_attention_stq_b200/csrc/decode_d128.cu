@@ -91,10 +91,20 @@ struct __align__(16) SmemChannel {
     float colG2[D];
 };
 
+// Only the joint scale refinement (FIT) needs these; they follow SmemFixed (and SmemChannel).
+// In the coordinates z_ij = sqrt(w_i) S'_ij / c'_j of the one-pass fit (c' its stored column
+// scale), the impact-weighted error is sum_ij c'_j^2 (z_ij - rho_i K_j Q_ij)^2 with rho_i =
+// sqrt(w_i) r_i and c_j = K_j c'_j.
+// The refit's column factors reuse SmemFixed arrays that are dead by then: colB holds K~_j (the
+// refitted stored column scale over c'_j) and colG1 holds c'_j^2 K~_j.
+struct __align__(16) SmemFit {
+    float rowRho[D];         // rho_i of the one-pass stored row scale
+};
+
 // ---------------------------------------------------------------------------------------------
 // Static per-width facts
 // ---------------------------------------------------------------------------------------------
-template <int BITS, int GATE, int IN_BF16>
+template <int BITS, int GATE, int IN_BF16, int FIT>
 struct Cfg {
     static constexpr int RB = BITS == 16 ? 256 : 16 * BITS;    // bytes of one 128-wide row
     static constexpr uint32_t SOFF = scale_offset(BITS, D, D);  // byte offset of r[]
@@ -105,7 +115,8 @@ struct Cfg {
     static constexpr uint32_t K_OFF = BLK, Q_OFF = BLK + ROW_IN, V_OFF = BLK + 2 * ROW_IN;
     static constexpr uint32_t W_OFF = BLK + 3 * ROW_IN, A_OFF = W_OFF + 4 * D;
     static constexpr uint32_t LEN = A_OFF + (GATE != 0 ? 4u * D : 0u);  // a multiple of 256
-    static constexpr uint32_t RING = (uint32_t)sizeof(SmemFixed) + (GATE == 1 ? (uint32_t)sizeof(SmemChannel) : 0u);
+    static constexpr uint32_t FIT_OFF = (uint32_t)sizeof(SmemFixed) + (GATE == 1 ? (uint32_t)sizeof(SmemChannel) : 0u);
+    static constexpr uint32_t RING = FIT_OFF + (FIT ? (uint32_t)sizeof(SmemFit) : 0u);
     // slots so that four CTAs fit an SM's 228 KB where they can
     static constexpr int NS = BITS == 4 ? 3 : 2;
     static constexpr size_t SMEM = RING + (size_t)NS * LEN;
@@ -267,10 +278,10 @@ __device__ __forceinline__ float sum4(const float *src, int stride)
     return (src[0] + src[stride]) + (src[2 * stride] + src[3 * stride]);
 }
 
-template <int BITS, int GATE, int IN_BF16>
+template <int BITS, int GATE, int IN_BF16, int FIT>
 __device__ __forceinline__ uint8_t *ring_slot(uint8_t *smem, int slot_i)
 {
-    return smem + Cfg<BITS, GATE, IN_BF16>::RING + (size_t)slot_i * Cfg<BITS, GATE, IN_BF16>::LEN;
+    return smem + Cfg<BITS, GATE, IN_BF16, FIT>::RING + (size_t)slot_i * Cfg<BITS, GATE, IN_BF16, FIT>::LEN;
 }
 
 __device__ __forceinline__ SmemChannel &channel(uint8_t *smem)
@@ -278,13 +289,19 @@ __device__ __forceinline__ SmemChannel &channel(uint8_t *smem)
     return *reinterpret_cast<SmemChannel *>(smem + sizeof(SmemFixed));
 }
 
+template <int BITS, int GATE, int IN_BF16, int FIT>
+__device__ __forceinline__ SmemFit &fitmem(uint8_t *smem)
+{
+    return *reinterpret_cast<SmemFit *>(smem + Cfg<BITS, GATE, IN_BF16, FIT>::FIT_OFF);
+}
+
 // Thread 0: stream this CTA's next tile into ring slot n % NS (codes + scales and the input rows
 // by bulk copy, the per-tile scalars by 4-byte cp.async), completing on the slot's mbarrier (two
 // arrivals: expect_tx + cp.async), and record where the tile lives and which row it reads.
-template <int BITS, int GATE, int IN_BF16>
+template <int BITS, int GATE, int IN_BF16, int FIT>
 __device__ __forceinline__ void issue_next(const TileParams &p, SmemFixed &sm, uint8_t *smem, Issuer &it, int my_count)
 {
-    using C = Cfg<BITS, GATE, IN_BF16>;
+    using C = Cfg<BITS, GATE, IN_BF16, FIT>;
     if (it.n >= my_count) return;
     const int n = it.n, slot_i = n % C::NS;
     const TileEntry e = p.table[it.pos];
@@ -315,7 +332,7 @@ __device__ __forceinline__ void issue_next(const TileParams &p, SmemFixed &sm, u
     cp_async4(smem_u32(&sm.scal[slot_i][0]), p.beta + row);
     if (GATE == 0) cp_async4(smem_u32(&sm.scal[slot_i][1]), p.alpha + row);
     cp_async_arrive(bar);
-    const uint32_t dst = smem_u32(ring_slot<BITS, GATE, IN_BF16>(smem, slot_i));
+    const uint32_t dst = smem_u32(ring_slot<BITS, GATE, IN_BF16, FIT>(smem, slot_i));
     const uint32_t blk = p.scale_bf16 ? C::BLK16 : C::BLK;
     mbar_arrive_expect_tx(bar, C::LEN - (C::BLK - blk));
     bulk_g2s(dst, src, blk, bar);
@@ -328,10 +345,10 @@ __device__ __forceinline__ void issue_next(const TileParams &p, SmemFixed &sm, u
 
 // Wait for tile n (ring slot n % NS) and compute its row factors, row i = threadIdx.x, with
 // per-warp sums of w, q.k and q.(alpha k). Returns false on a timeout.
-template <int BITS, int GATE, int IN_BF16>
+template <int BITS, int GATE, int IN_BF16, int FIT>
 __device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, int n, int my_count, int sb16)
 {
-    using C = Cfg<BITS, GATE, IN_BF16>;
+    using C = Cfg<BITS, GATE, IN_BF16, FIT>;
     if (n >= my_count) return true;
     const int slot_i = n % C::NS;
     const uint32_t phase = (uint32_t)(n / C::NS) & 1u;
@@ -339,7 +356,7 @@ __device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, in
     if (!__all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&sm.bars[slot_i]), phase))) return false;
     if (sm.meta[n & 3].skip) return true;  // skipped tile: nothing was loaded
     const int pb = n & 1;
-    const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16>(smem, slot_i);
+    const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16, FIT>(smem, slot_i);
     const int i = threadIdx.x;
     constexpr bool pivot = BITS == 16;
     const float r = pivot ? 1.f : load_scale(tile + C::SOFF, i, sb16);
@@ -374,17 +391,165 @@ __device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, in
     return true;
 }
 
+// One round of the impact-weighted joint refinement of the scales (the refit), on the tile's
+// z_ij = sqrt(w_i) S'_ij / c'_j in Tensor Memory. With the one-pass codes Q_ij = round(z_ij s_i):
+//   column step  K_j = sum_i rho_i Q_ij z_ij / sum_i (rho_i Q_ij)^2, c_j = K_j c'_j, stored as c~_j;
+//   row step     rho_i = sum_j c'_j^2 K~_j Q_ij z_ij / sum_j c'_j^2 K~_j^2 Q_ij^2, r_i = rho_i /
+//                sqrt(w_i), stored as r~_i,
+// each kept only if finite and positive. Writes the stored scales, K~_j into colB, c'_j^2 K~_j into
+// colG1 and the new s_i = 1 / (sqrt(w_i) r~_i) into rowS. Two CTA barriers; the row sums stay in
+// each half-warp. c_one is this thread's column c'_j (j = threadIdx.x); r_one / s_one are the
+// one-pass r and s of this lane's row i = 8 cg + rb.
+template <int BITS, int GATE, int IN_BF16, int FIT>
+__device__ __forceinline__ bool refit_scales(const TileParams &p, SmemFixed &sm, uint8_t *smem, int n, uint32_t tcol,
+                                             float c_one, float r_one, float s_one)
+{
+    using C = Cfg<BITS, GATE, IN_BF16, FIT>;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, cg = lane & 15, sub = lane >> 4;
+    const int rb = 2 * warp + sub, pb = n & 1, sb16 = p.scale_bf16;
+    const float *rho = fitmem<BITS, GATE, IN_BF16, FIT>(smem).rowRho;
+    const float2 rnd = make_float2(C::ROUND, C::ROUND), nrnd = make_float2(-C::ROUND, -C::ROUND);
+    uint8_t *gsc = reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + C::SOFF);
+    tmem_wait_st();
+    // ---- column sums over this thread's 16 rows --------------------------------------------
+    {
+        float2 aN[4], aD[4];
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) aN[pp] = aD[pp] = make_float2(0.f, 0.f);
+        float2 cha[8], chb[8];
+        tmem_ld16_async(tcol, cha);
+        tmem_wait_ld(cha);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            float2 (&ch)[8] = (k & 1) ? chb : cha;
+            float2 (&nx)[8] = (k & 1) ? cha : chb;
+            if (k + 1 < 8) tmem_ld16_async(tcol + 16 * (k + 1), nx);
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int i = 8 * (2 * k + r) + rb;
+                const float2 s2 = sm.rowS[i];
+                const float2 rr = make_float2(rho[i], rho[i]);
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) {
+                    const float2 z = ch[4 * r + pp];
+                    const float2 q = __fadd2_rn(__ffma2_rn(z, s2, rnd), nrnd);  // the one-pass code
+                    const float2 t = __fmul2_rn(q, rr);
+                    aN[pp] = __ffma2_rn(t, z, aN[pp]);
+                    aD[pp] = __ffma2_rn(t, t, aD[pp]);
+                }
+            }
+            if (k + 1 < 8) tmem_wait_ld(nx);
+        }
+        // halves 0/1 hold the same columns: half 0 keeps the numerators, half 1 the denominators
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+            const float2 send = sub ? aN[pp] : aD[pp];
+            const float2 keep = sub ? aD[pp] : aN[pp];
+            const float2 got = make_float2(__shfl_xor_sync(0xffffffffu, send.x, 16),
+                                           __shfl_xor_sync(0xffffffffu, send.y, 16));
+            aN[pp] = __fadd2_rn(keep, got);
+        }
+        float *dst = sm.red + rb * RS + 8 * cg;
+        *reinterpret_cast<float4 *>(dst) = f4_of(aN[0], aN[1]);
+        *reinterpret_cast<float4 *>(dst + 4) = f4_of(aN[2], aN[3]);
+    }
+    __syncthreads();
+    // ---- column j = tid: refitted stored scale --------------------------------------------
+    {
+        const int j = tid;
+        const float N = sum4(sm.red + j, 2 * RS), Dn = sum4(sm.red + RS + j, 2 * RS);
+        float cf = c_one;
+        if (Dn > 0.f) {
+            const float cn = round_scale(c_one * (N / Dn), sb16);
+            if (isfinite(cn) && cn > 0.f) cf = cn;
+        }
+        store_scale(gsc, D + j, cf, sb16);
+        const float K = cf / c_one;
+        sm.colB[j] = K;
+        sm.colG1[j] = c_one * c_one * K;
+    }
+    __syncthreads();
+    // ---- row sums over this thread's 8 columns, then across the half-warp ---------------------
+    float pn[16], pd[16];
+    {
+        float2 g[4], h[4];
+        load_pairs(sm.colG1 + 8 * cg, g);
+        load_pairs(sm.colB + 8 * cg, h);
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) h[pp] = __fmul2_rn(g[pp], h[pp]);  // c'^2 K~^2
+        float2 cha[8], chb[8];
+        tmem_ld16_async(tcol, cha);
+        tmem_wait_ld(cha);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            float2 (&ch)[8] = (k & 1) ? chb : cha;
+            float2 (&nx)[8] = (k & 1) ? cha : chb;
+            if (k + 1 < 8) tmem_ld16_async(tcol + 16 * (k + 1), nx);
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int m = 2 * k + r;
+                const float2 s2 = sm.rowS[8 * m + rb];
+                float2 n2 = make_float2(0.f, 0.f), d2 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) {
+                    const float2 z = ch[4 * r + pp];
+                    const float2 q = __fadd2_rn(__ffma2_rn(z, s2, rnd), nrnd);
+                    n2 = __ffma2_rn(__fmul2_rn(q, g[pp]), z, n2);
+                    d2 = __ffma2_rn(__fmul2_rn(q, h[pp]), q, d2);
+                }
+                pn[m] = n2.x + n2.y;
+                pd[m] = d2.x + d2.y;
+            }
+            if (k + 1 < 8) tmem_wait_ld(nx);
+        }
+    }
+    float *rm = sm.red + rb * RS + cg;
+    const float4 *src = reinterpret_cast<const float4 *>(sm.red + rb * RS + cg * RM);
+#pragma unroll
+    for (int m = 0; m < 16; ++m) rm[m * RM] = pn[m];
+    __syncwarp();
+    float num;
+    {
+        const float4 a = src[0], b = src[1], c = src[2], d = src[3];
+        num = ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + (b.z + b.w)) + ((c.x + c.y) + (c.z + c.w)) +
+              ((d.x + d.y) + (d.z + d.w));
+    }
+    __syncwarp();
+#pragma unroll
+    for (int m = 0; m < 16; ++m) rm[m * RM] = pd[m];
+    __syncwarp();
+    {
+        const float4 a = src[0], b = src[1], c = src[2], d = src[3];
+        const float den = ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + (b.z + b.w)) + ((c.x + c.y) + (c.z + c.w)) +
+                          ((d.x + d.y) + (d.z + d.w));
+        const int i = 8 * cg + rb;
+        float rf = r_one, sf = s_one;
+        if (den > 0.f) {
+            const float rq = sm.rowRq[pb][i] * C::QMAX;  // 1 / sqrt(w_i)
+            const float rn = round_scale((num / den) * rq, sb16);
+            if (isfinite(rn) && rn > 0.f) {
+                rf = rn;
+                sf = rq * fast_rcp(rn);
+            }
+        }
+        store_scale(gsc, i, rf, sb16);
+        sm.rowS[i] = make_float2(sf, sf);
+    }
+    __syncwarp();
+    return true;
+}
+
 // Tile n (ring slot n % NS). Returns false if the wait for the next tile timed out.
-template <int BITS, int GATE, int IN_BF16>
+template <int BITS, int GATE, int IN_BF16, int FIT>
 __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm, uint8_t *smem, int n, int my_count,
                                              uint32_t tcol)
 {
-    using C = Cfg<BITS, GATE, IN_BF16>;
+    using C = Cfg<BITS, GATE, IN_BF16, FIT>;
     constexpr bool pivot = BITS == 16;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, cg = lane & 15, sub = lane >> 4;
     const int pb = n & 1, slot_i = n % C::NS;
     const int rb = 2 * warp + sub;  // this thread's rows: rb + 8m, m < 16
-    const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16>(smem, slot_i);
+    const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16, FIT>(smem, slot_i);
     // the tile's record (sm.meta[n & 3]) stays valid until the issue after the next tile's B2
 
     // ---- Sweep A: unpack to TMEM, column sums of k~Q and q~Q -------------------------------
@@ -453,7 +618,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
         if (!isfinite(o)) flag(p.status, kFlagNonfinite);
     }
     __syncthreads();  // B2: coefficients ready; this tile's ring bytes are no longer read
-    if (tid == 0) issue_next<BITS, GATE, IN_BF16>(p, sm, smem, sm.iss, my_count);
+    if (tid == 0) issue_next<BITS, GATE, IN_BF16, FIT>(p, sm, smem, sm.iss, my_count);
 
     // ---- Sweep B: y = rho Q + kappa g1 (+ mu g2), column energy ---------------------------
     tmem_wait_st();
@@ -527,6 +692,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
     __syncthreads();  // B3: column energies complete
 
     // ---- New column scale of column j, then the next tile's row factors -------------------
+    float c_one = 1.f;  // the one-pass stored column scale c'_j (kept for the refit)
     if (!pivot) {
         // x = sum_i w_i S'_ij^2 / (sum_i w_i c_j^2) (times sigma_j^2), so c'_j = c_j sqrt(x) / sigma_j
         // and the factor taking y to S'_ij / c'_j is 1 / sqrt(x)
@@ -542,11 +708,12 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
             c = round_scale(c, 1);
             b = (cj * inv_sig) * fast_rcp(c);
         }
-        store_scale(reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + C::SOFF), D + j, c, sb16);
+        c_one = c;
+        if (!FIT) store_scale(reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + C::SOFF), D + j, c, sb16);
         if (!isfinite(c) || c == 0.f) flag(p.status, kFlagNonfinite);
         sm.colB[j] = b;
     }
-    const bool ok = precompute_rows<BITS, GATE, IN_BF16>(sm, smem, n + 1, my_count, sb16);
+    const bool ok = precompute_rows<BITS, GATE, IN_BF16, FIT>(sm, smem, n + 1, my_count, sb16);
     if (__syncthreads_or(!ok)) return false;  // B4: new column scales and next row factors ready
     if constexpr (pivot) return true;
 
@@ -578,6 +745,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
         }
     }
     __syncwarp();
+    float r_one = 1.f, s_one = 0.f;  // this lane's row (i = 8 cg + rb): one-pass stored r_i and its factor
     {
         // lane cg of this half finishes its row m = cg (i = 8 cg + rb) from the 16 partials
         const float4 *src = reinterpret_cast<const float4 *>(sm.red + rb * RS + cg * RM);
@@ -597,16 +765,31 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
             s = (sm.rowRq[pb][i] * C::QMAX) * fast_rcp(r);
         }
         sm.rowS[i] = make_float2(s, s);
-        store_scale(reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + C::SOFF), i, r, sb16);
+        if constexpr (FIT) {
+            r_one = r;
+            s_one = s;
+            fitmem<BITS, GATE, IN_BF16, FIT>(smem).rowRho[i] = r * fast_rcp(sm.rowRq[pb][i] * C::QMAX);  // sqrt(w_i) r_i
+        } else {
+            store_scale(reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + C::SOFF), i, r, sb16);
+        }
         if (!isfinite(r) || r == 0.f) flag(p.status, kFlagNonfinite);
     }
     __syncwarp();
+    if constexpr (FIT) {
+        if (!refit_scales<BITS, GATE, IN_BF16, FIT>(p, sm, smem, n, tcol, c_one, r_one, s_one)) return false;
+    }
 
     // ---- Sweep D: x = z s rounded half to even by the 2^23 + offset FFMA, packed, stored ----
     tmem_wait_st();
     {
         const float2 rnd = make_float2(C::ROUND, C::ROUND);
         uint8_t *dstrow = reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock) + rb * C::RB + cg * BITS;
+        float2 ik[4];  // 1 / K~_j of this thread's columns (refit only)
+        if constexpr (FIT) {
+            load_pairs(sm.colB + 8 * cg, ik);
+#pragma unroll
+            for (int pp = 0; pp < 4; ++pp) ik[pp] = make_float2(fast_rcp(ik[pp].x), fast_rcp(ik[pp].y));
+        }
         float2 cha[8], chb[8];
         tmem_ld16_async(tcol, cha);
         tmem_wait_ld(cha);
@@ -620,7 +803,17 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
                 const int m = 2 * k + r;
                 const float2 s2 = sm.rowS[8 * m + rb];
 #pragma unroll
-                for (int pp = 0; pp < 4; ++pp) ch[4 * r + pp] = __ffma2_rn(ch[4 * r + pp], s2, rnd);
+                for (int pp = 0; pp < 4; ++pp) {
+                    if constexpr (FIT) {
+                        // x = z / (K~_j rho~_i), clamped (refitted scales may clip), rounded by the add
+                        float2 v = __fmul2_rn(__fmul2_rn(ch[4 * r + pp], ik[pp]), s2);
+                        v.x = fminf(fmaxf(v.x, -C::QMAX), C::QMAX);
+                        v.y = fminf(fmaxf(v.y, -C::QMAX), C::QMAX);
+                        ch[4 * r + pp] = __fadd2_rn(v, rnd);
+                    } else {
+                        ch[4 * r + pp] = __ffma2_rn(ch[4 * r + pp], s2, rnd);
+                    }
+                }
                 pack_store_row<BITS>(dstrow + 8 * m * C::RB, cg, ch + 4 * r);
             }
             if (k + 1 < 8) tmem_wait_ld(nx);
@@ -629,10 +822,10 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
     return true;
 }
 
-template <int BITS, int GATE, int IN_BF16>
+template <int BITS, int GATE, int IN_BF16, int FIT>
 __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constant__ TileParams p)
 {
-    using C = Cfg<BITS, GATE, IN_BF16>;
+    using C = Cfg<BITS, GATE, IN_BF16, FIT>;
     extern __shared__ __align__(128) uint8_t smem[];
     SmemFixed &sm = *reinterpret_cast<SmemFixed *>(smem);
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -665,9 +858,9 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
         it.b = (int)blockIdx.x - it.pos * p.B;
         it.qG = G / p.B;
         it.rG = G - it.qG * p.B;
-        for (int k = 0; k < C::NS; ++k) issue_next<BITS, GATE, IN_BF16>(p, sm, smem, it, my_count);
+        for (int k = 0; k < C::NS; ++k) issue_next<BITS, GATE, IN_BF16, FIT>(p, sm, smem, it, my_count);
     }
-    bool failed = __syncthreads_or(!precompute_rows<BITS, GATE, IN_BF16>(sm, smem, 0, my_count, p.scale_bf16));
+    bool failed = __syncthreads_or(!precompute_rows<BITS, GATE, IN_BF16, FIT>(sm, smem, 0, my_count, p.scale_bf16));
 
     int n = 0;
     for (; n < my_count && !failed; ++n) {
@@ -675,11 +868,11 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
         const bool got = mbar_wait_bounded(smem_u32(&sm.bars[n % C::NS]), (uint32_t)(n / C::NS) & 1u);
         if (sm.meta[n & 3].skip) {  // out-of-range slot: nothing loaded, nothing to do
             __syncthreads();
-            if (tid == 0) issue_next<BITS, GATE, IN_BF16>(p, sm, smem, sm.iss, my_count);
-            const bool ok = precompute_rows<BITS, GATE, IN_BF16>(sm, smem, n + 1, my_count, p.scale_bf16);
+            if (tid == 0) issue_next<BITS, GATE, IN_BF16, FIT>(p, sm, smem, sm.iss, my_count);
+            const bool ok = precompute_rows<BITS, GATE, IN_BF16, FIT>(sm, smem, n + 1, my_count, p.scale_bf16);
             failed = __syncthreads_or(!ok || !got);
         } else {
-            failed = !process_tile<BITS, GATE, IN_BF16>(p, sm, smem, n, my_count, tcol);
+            failed = !process_tile<BITS, GATE, IN_BF16, FIT>(p, sm, smem, n, my_count, tcol);
         }
     }
     if (failed && tid == 0) {
@@ -698,11 +891,11 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
     }
 }
 
-template <int BITS, int GATE, int IN_BF16>
+template <int BITS, int GATE, int IN_BF16, int FIT>
 cudaError_t launch_t(const TileParams &p, cudaStream_t s)
 {
-    using C = Cfg<BITS, GATE, IN_BF16>;
-    auto kernel = decode_d128_kernel<BITS, GATE, IN_BF16>;
+    using C = Cfg<BITS, GATE, IN_BF16, FIT>;
+    auto kernel = decode_d128_kernel<BITS, GATE, IN_BF16, FIT>;
     const int smem = (int)C::SMEM;
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -730,16 +923,16 @@ cudaError_t launch_t(const TileParams &p, cudaStream_t s)
     return cudaGetLastError();
 }
 
-template <int BITS>
+template <int BITS, int FIT>
 cudaError_t launch_bits(const TileParams &p, int in_bf16, cudaStream_t s)
 {
     switch (p.gate * 2 + (in_bf16 ? 1 : 0)) {
-    case 0: return launch_t<BITS, 0, 0>(p, s);
-    case 1: return launch_t<BITS, 0, 1>(p, s);
-    case 2: return launch_t<BITS, 1, 0>(p, s);
-    case 3: return launch_t<BITS, 1, 1>(p, s);
-    case 4: return launch_t<BITS, 2, 0>(p, s);
-    default: return launch_t<BITS, 2, 1>(p, s);
+    case 0: return launch_t<BITS, 0, 0, FIT>(p, s);
+    case 1: return launch_t<BITS, 0, 1, FIT>(p, s);
+    case 2: return launch_t<BITS, 1, 0, FIT>(p, s);
+    case 3: return launch_t<BITS, 1, 1, FIT>(p, s);
+    case 4: return launch_t<BITS, 2, 0, FIT>(p, s);
+    default: return launch_t<BITS, 2, 1, FIT>(p, s);
     }
 }
 
@@ -747,14 +940,16 @@ cudaError_t launch_bits(const TileParams &p, int in_bf16, cudaStream_t s)
 
 int decode_d128_max_requests() { return MAXB; }
 
-// All entries of p.table have the width `bits`.
+// All entries of p.table have the width `bits`. p.fit_rounds is 0 or 1 (one round of the joint
+// scale refinement; FP16 pivot heads have no scales and ignore it).
 cudaError_t launch_decode_d128(const TileParams &p, int bits, int in_bf16, cudaStream_t s)
 {
+    const bool fit = p.fit_rounds > 0;
     switch (bits) {
-    case 4: return launch_bits<4>(p, in_bf16, s);
-    case 6: return launch_bits<6>(p, in_bf16, s);
-    case 8: return launch_bits<8>(p, in_bf16, s);
-    default: return launch_bits<16>(p, in_bf16, s);
+    case 4: return fit ? launch_bits<4, 1>(p, in_bf16, s) : launch_bits<4, 0>(p, in_bf16, s);
+    case 6: return fit ? launch_bits<6, 1>(p, in_bf16, s) : launch_bits<6, 0>(p, in_bf16, s);
+    case 8: return fit ? launch_bits<8, 1>(p, in_bf16, s) : launch_bits<8, 0>(p, in_bf16, s);
+    default: return launch_bits<16, 0>(p, in_bf16, s);
     }
 }
 

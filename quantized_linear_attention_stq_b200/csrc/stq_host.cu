@@ -227,7 +227,7 @@ stq_status stq_decode_step(const stq_layout *L, void *pool, int32_t pool_slots, 
     p->gate = L->gate;
     p->w = w;
     const int in_bf16 = L->in_dtype == STQ_BF16;
-    const bool tuned = L->dk == 128 && !L->uniform && L->fit_rounds == 0;
+    const bool tuned = L->dk == 128 && !L->uniform && L->fit_rounds <= 1;  // one refit round runs tuned
     const int maxb = tuned ? stq::decode_d128_max_requests() : 65535;
     const std::vector<int> ord = order_by_size(L, head_begin, head_count);
     const size_t in_sz = in_bf16 ? 2 : 4;

@@ -4,8 +4,9 @@ A layout with fit_rounds = n refits, after the one-pass fit, every column scale 
 least squares and every row scale by least squares, n times, recomputing the codes in between
 (the pages fit the two scales jointly and weight high-impact rows more: "线性注意力状态量化难题"
 (aitest123.com/news/n1kj09), section 空间维度; "K1 論文詳解" (k1-news.pages.dev/paper/2026-10-09),
-section 方法). Such layouts run on the plain kernels. Teacher-forced protocol as in
-test_gpu_decode.py; blocks are compared with the joint-fit rule of tests/_parity.py.
+section 方法). A layout with one round decodes 128 x 128 heads on the tuned kernel; other layouts
+with refinement run on the plain kernels. Teacher-forced protocol as in test_gpu_decode.py; blocks
+are compared with the joint-fit rule of tests/_parity.py.
 """
 import numpy as np
 import pytest
@@ -18,6 +19,7 @@ pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
 ROUNDS = 2
+STUDY_ROUNDS = (0, 1, 2)
 
 
 @pytest.fixture(scope="module")
@@ -79,14 +81,14 @@ def test_init(stq, orc, d):
     tally.check_budget()
 
 
-def _decode_teacher_forced(stq, orc, wl_, bits, steps):
+def _decode_teacher_forced(stq, orc, wl_, bits, steps, rounds=ROUNDS):
     from quantized_linear_attention_stq_b200 import workloads as wlm
 
     B, H, d = wl_.batch, wl_.heads, wl_.d
-    lay = stq.Layout(bits, d, gate=wl_.gate, in_dtype=wl_.in_dtype, fit_rounds=ROUNDS)
+    lay = stq.Layout(bits, d, gate=wl_.gate, in_dtype=wl_.in_dtype, fit_rounds=rounds)
     w = wlm.impact_weights(wl_)
     S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(B)])
-    opool = _oracle_pool(orc, bits, d, S0, w, ROUNDS)
+    opool = _oracle_pool(orc, bits, d, S0, w, rounds)
     offs, total = orc.request_layout(bits, d, d)
     gpool = torch.zeros(B * total, dtype=torch.uint8, device=DEV)
     slots = torch.arange(B, dtype=torch.int32, device=DEV)
@@ -107,9 +109,9 @@ def _decode_teacher_forced(stq, orc, wl_, bits, steps):
                 ref_blk = tile_bytes(orc, opool, bits, d, r, h)
                 q, k, v = as_f64(inp["q"][r, h]), as_f64(inp["k"][r, h]), as_f64(inp["v"][r, h])
                 beta, alpha = float(inp["beta"][r, h]), inp["alpha"][r, h].double().numpy()
-                rounds = 0 if bits[h] == 16 else ROUNDS
+                hr = 0 if bits[h] == 16 else rounds
                 res = orc.decode_step_s(bits[h], orc.SCALE_F32, wl_.gate, ref_blk, q, k, v, beta, alpha,
-                                        as_f64(w[h]), d, d, rounds=rounds)
+                                        as_f64(w[h]), d, d, rounds=hr)
                 assert res["status"] == orc.OK
                 got = tile_bytes(orc, gp, bits, d, r, h)
                 what = f"step {t} req {r} head {h}"
@@ -117,15 +119,30 @@ def _decode_teacher_forced(stq, orc, wl_, bits, steps):
                     M = update_magnitude(orc.dequantize(16, d, d, ref_blk), k, v, beta, alpha)
                     compare_block(orc, 16, d, got, res["block"], res["tie"], tally, what, err_scale=M)
                 else:
-                    compare_block_fit(orc, bits[h], d, got, res["S_new"], as_f64(w[h]), ROUNDS, tally, what)
+                    compare_block_fit(orc, bits[h], d, got, res["S_new"], as_f64(w[h]), rounds, tally, what)
                 compare_o(og[r, h], res["o"], tally, "o " + what)
                 opool[r * total + offs[h]: r * total + offs[h] + res["block"].size] = res["block"]
     tally.check_budget()
 
 
-def test_decode_d128_mixed_with_pivots(stq, orc):
+@pytest.mark.parametrize("rounds", [1, 2])
+def test_decode_d128_mixed_with_pivots(stq, orc, rounds):
+    """One round runs on the tuned 128 x 128 kernel, two on the plain kernel."""
     wl_ = _wl("full2304_b70_mixed", batch=3, heads=8)
-    _decode_teacher_forced(stq, orc, wl_, [4, 16, 6, 8, 4, 6, 8, 6], 2)
+    _decode_teacher_forced(stq, orc, wl_, [4, 16, 6, 8, 4, 6, 8, 6], 2, rounds)
+
+
+@pytest.mark.parametrize("bits", [4, 6, 8])
+def test_decode_d128_tuned_one_round(stq, orc, bits):
+    """The tuned kernel's refit at each width: 5 requests x 6 heads, 3 steps."""
+    wl_ = _wl("layer48_b8_4bit", batch=5, heads=6, bits=bits)
+    _decode_teacher_forced(stq, orc, wl_, [bits] * 6, 3, 1)
+
+
+@pytest.mark.parametrize("gate", [1, 2])
+def test_decode_d128_tuned_channel_gates(stq, orc, gate):
+    wl_ = _wl("channel32_b128_4bit", batch=2, heads=4, gate=gate)
+    _decode_teacher_forced(stq, orc, wl_, [4, 6, 8, 6], 2, 1)
 
 
 @pytest.mark.parametrize("gate", [1, 2])
@@ -205,7 +222,7 @@ def test_study_joint_fit_error_accumulation(stq):
     slots = torch.zeros(1, dtype=torch.int32, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     runs = {}
-    for rounds in (0, ROUNDS):
+    for rounds in STUDY_ROUNDS:
         for b in (4, 6, 8):
             lay = stq.Layout([b] * H, d, fit_rounds=rounds)
             pool = lay.alloc_pool(1, DEV)
