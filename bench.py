@@ -218,10 +218,13 @@ def oracle_sample_tiles(workload_name: str, n_tiles: int, seed_offset: int = 0):
     bits_all = wlm.head_bits(wl)
     rng = np.random.default_rng(1234 + seed_offset)
     heads = rng.choice(len(bits_all), size=n_tiles, replace=False)
-    # make sure every width of the workload appears
-    for b in sorted(set(bits_all)):
-        if not any(bits_all[h] == b for h in heads):
-            heads[rng.integers(n_tiles)] = bits_all.index(b)
+    # with room for it, make sure every width of the workload appears (a single-tile sample keeps
+    # its random draw, so that samples over many processes follow the workload's width mix)
+    widths = sorted(set(bits_all))
+    if n_tiles >= len(widths):
+        for slot, b in enumerate(widths):
+            if not any(bits_all[h] == b for h in heads):
+                heads[slot] = bits_all.index(b)
     small = wlm.scaled(wl, batch=1, heads=len(heads), outliers=wl.outliers)
     S0 = wlm.initial_state(small, 0).double().numpy()
     w_all = wlm.impact_weights(wl).double().numpy()
