@@ -209,7 +209,7 @@ def compare_block_bf16s(orc, bits, d, got, S_new, w, tally: Tally, what=""):
     assert not got[so + 4 * d:].any()
 
 
-def compare_block_fit(orc, bits, d, got, S_new, w, rounds, tally: Tally, what=""):
+def compare_block_fit(orc, bits, d, got, S_new, w, rounds, tally: Tally, what="", sfmt=0):
     """A head block whose fp32 scales went through `rounds` rounds of the joint refinement,
     against the oracle's refinement of the same updated state S_new (fp64). The refinement
     recomputes codes between its least-squares steps, so a code that flips at a near-tie in an
@@ -221,16 +221,18 @@ def compare_block_fit(orc, bits, d, got, S_new, w, rounds, tally: Tally, what=""
     above); and the impact-weighted reconstruction error of the GPU's block, the quantity the
     refinement minimises, may exceed the oracle's by at most 1e-3 relative."""
     got = np.asarray(got, dtype=np.uint8)
-    blk, _, _, st = orc.quantize_fit(bits, orc.SCALE_F32, rounds, S_new, w)
+    blk, _, _, st = orc.quantize_fit(bits, sfmt, rounds, S_new, w)
     assert st == orc.OK
-    rg, cg = orc.scales_s(bits, orc.SCALE_F32, d, d, got)
-    ro, co = orc.scales_s(bits, orc.SCALE_F32, d, d, blk)
+    rg, cg = orc.scales_s(bits, sfmt, d, d, got)
+    ro, co = orc.scales_s(bits, sfmt, d, d, blk)
     rels = np.concatenate([np.abs(rg - ro) / ro, np.abs(cg - co) / co])
-    assert rels.max() <= 10 * SCALE_RTOL, f"{what}: scale rel error {rels.max()}"
+    # with bf16 storage a refitted scale may also land one bf16 step (<= 2^-7 relative) away
+    tol = SCALE_RTOL if sfmt == orc.SCALE_F32 else SCALE_RTOL + 2.0 ** -7
+    assert rels.max() <= 10 * tol, f"{what}: scale rel error {rels.max()}"
     tally.scales += rels.size
-    tally.fit_scale_outliers += int((rels > SCALE_RTOL).sum())
+    tally.fit_scale_outliers += int((rels > tol).sum())
     tally.max_scale_rel = max(tally.max_scale_rel, float(rels.max()))
-    req, x, tie, _, st = orc.quantize_s(bits, orc.SCALE_F32, S_new, w, c_given=cg, r_given=rg)
+    req, x, tie, _, st = orc.quantize_s(bits, sfmt, S_new, w, c_given=cg, r_given=rg)
     Qg = orc.codes(bits, d, d, got)
     Qr = orc.codes(bits, d, d, req)
     cdiff = np.abs(Qg - Qr)
@@ -249,7 +251,7 @@ def compare_block_fit(orc, bits, d, got, S_new, w, rounds, tally: Tally, what=""
     assert e_gpu <= e_orc * (1 + 1e-3) + 1e-300, f"{what}: weighted error {e_gpu} against the oracle's {e_orc}"
     so = orc.scale_offset(bits, d, d)
     assert not got[orc.codes_bytes(bits, d, d): so].any()
-    assert not got[so + 8 * d:].any()
+    assert not got[so + (8 if sfmt == orc.SCALE_F32 else 4) * d:].any()
 
 
 def compare_o(got, ref, tally: Tally, what=""):

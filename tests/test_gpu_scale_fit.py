@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 import torch
 
-from _parity import (Tally, as_f64, compare_block, compare_block_fit, compare_o, oracle_pool, tile_bytes,
+from _parity import (Tally, as_f64, compare_block, compare_block_fit, compare_o, tile_bytes,
                      update_magnitude)
 
 pytestmark = pytest.mark.gpu
@@ -38,18 +38,25 @@ def _wl(name, **changes):
     return wl.scaled(wl.WORKLOADS[name], **changes)
 
 
-def _oracle_pool(orc, bits, d, S0, w, rounds):
+def _layout_s(orc, bits, d, sfmt):
+    offs, pos = [], 0
+    for b in bits:
+        offs.append(pos)
+        pos += orc.block_bytes_s(int(b), sfmt, d, d)
+    return offs, (pos + 127) // 128 * 128
+
+
+def _oracle_pool(orc, bits, d, S0, w, rounds, sfmt=0):
     B, H = S0.shape[0], S0.shape[1]
-    blocks = []
+    offs, total = _layout_s(orc, bits, d, sfmt)
+    pool = np.zeros(B * total, dtype=np.uint8)
     for r in range(B):
-        row = []
         for h in range(H):
-            blk, _, _, st = orc.quantize_fit(bits[h], orc.SCALE_F32, 0 if bits[h] == 16 else rounds,
+            blk, _, _, st = orc.quantize_fit(bits[h], sfmt, 0 if bits[h] == 16 else rounds,
                                              as_f64(S0[r, h]), as_f64(w[h]))
             assert st == orc.OK
-            row.append(blk)
-        blocks.append(row)
-    return oracle_pool(orc, bits, d, blocks)
+            pool[r * total + offs[h]: r * total + offs[h] + blk.size] = blk
+    return pool
 
 
 @pytest.mark.parametrize("d", [16, 128])
@@ -81,15 +88,17 @@ def test_init(stq, orc, d):
     tally.check_budget()
 
 
-def _decode_teacher_forced(stq, orc, wl_, bits, steps, rounds=ROUNDS):
+def _decode_teacher_forced(stq, orc, wl_, bits, steps, rounds=ROUNDS, sfmt=0):
     from quantized_linear_attention_stq_b200 import workloads as wlm
 
     B, H, d = wl_.batch, wl_.heads, wl_.d
-    lay = stq.Layout(bits, d, gate=wl_.gate, in_dtype=wl_.in_dtype, fit_rounds=rounds)
+    lay = stq.Layout(bits, d, gate=wl_.gate, in_dtype=wl_.in_dtype, fit_rounds=rounds,
+                     scale_dtype=torch.bfloat16 if sfmt == orc.SCALE_BF16 else torch.float32)
     w = wlm.impact_weights(wl_)
     S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(B)])
-    opool = _oracle_pool(orc, bits, d, S0, w, rounds)
-    offs, total = orc.request_layout(bits, d, d)
+    opool = _oracle_pool(orc, bits, d, S0, w, rounds, sfmt)
+    offs, total = _layout_s(orc, bits, d, sfmt)
+    assert lay.bytes_per_request == total
     gpool = torch.zeros(B * total, dtype=torch.uint8, device=DEV)
     slots = torch.arange(B, dtype=torch.int32, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
@@ -106,20 +115,21 @@ def _decode_teacher_forced(stq, orc, wl_, bits, steps, rounds=ROUNDS):
         gp, og = gpool.cpu().numpy(), o.cpu().numpy()
         for r in range(B):
             for h in range(H):
-                ref_blk = tile_bytes(orc, opool, bits, d, r, h)
+                n_b = orc.block_bytes_s(bits[h], sfmt, d, d)
+                ref_blk = opool[r * total + offs[h]: r * total + offs[h] + n_b]
                 q, k, v = as_f64(inp["q"][r, h]), as_f64(inp["k"][r, h]), as_f64(inp["v"][r, h])
                 beta, alpha = float(inp["beta"][r, h]), inp["alpha"][r, h].double().numpy()
                 hr = 0 if bits[h] == 16 else rounds
-                res = orc.decode_step_s(bits[h], orc.SCALE_F32, wl_.gate, ref_blk, q, k, v, beta, alpha,
+                res = orc.decode_step_s(bits[h], sfmt, wl_.gate, ref_blk, q, k, v, beta, alpha,
                                         as_f64(w[h]), d, d, rounds=hr)
                 assert res["status"] == orc.OK
-                got = tile_bytes(orc, gp, bits, d, r, h)
+                got = gp[r * total + offs[h]: r * total + offs[h] + n_b]
                 what = f"step {t} req {r} head {h}"
                 if bits[h] == 16:
                     M = update_magnitude(orc.dequantize(16, d, d, ref_blk), k, v, beta, alpha)
                     compare_block(orc, 16, d, got, res["block"], res["tie"], tally, what, err_scale=M)
                 else:
-                    compare_block_fit(orc, bits[h], d, got, res["S_new"], as_f64(w[h]), rounds, tally, what)
+                    compare_block_fit(orc, bits[h], d, got, res["S_new"], as_f64(w[h]), rounds, tally, what, sfmt)
                 compare_o(og[r, h], res["o"], tally, "o " + what)
                 opool[r * total + offs[h]: r * total + offs[h] + res["block"].size] = res["block"]
     tally.check_budget()
@@ -143,6 +153,43 @@ def test_decode_d128_tuned_one_round(stq, orc, bits):
 def test_decode_d128_tuned_channel_gates(stq, orc, gate):
     wl_ = _wl("channel32_b128_4bit", batch=2, heads=4, gate=gate)
     _decode_teacher_forced(stq, orc, wl_, [4, 6, 8, 6], 2, 1)
+
+
+@pytest.mark.parametrize("rounds", [1, 2])
+def test_decode_d128_bf16_scales(stq, orc, rounds):
+    """The refit with 16-bit scales: every refitted value is rounded to bf16 before it is used
+    (one round on the tuned kernel, two on the plain kernel)."""
+    wl_ = _wl("full2304_b70_mixed", batch=3, heads=6)
+    _decode_teacher_forced(stq, orc, wl_, [4, 6, 8, 16, 6, 4], 2, rounds, orc.SCALE_BF16)
+
+
+def test_zero_heads_keep_unit_scales(stq, orc):
+    """An all-zero state stays all-zero through a step with v = 0: every refit denominator is 0,
+    so the scales stay 1 and the codes 0, without a non-finite flag."""
+    bits, d = [4, 6, 8], 128
+    lay = stq.Layout(bits, d, fit_rounds=1)
+    pool = lay.alloc_pool(2)
+    slots = torch.arange(2, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    w = torch.ones(3, d, device=DEV)
+    stq.init_state(lay, pool, slots, torch.zeros(2, 3, d, d, device=DEV), w, status=status)
+    q = torch.randn(2, 3, d, device=DEV).bfloat16()
+    k = torch.nn.functional.normalize(torch.randn(2, 3, d, device=DEV), dim=-1).bfloat16()
+    v = torch.zeros(2, 3, d, device=DEV).bfloat16()
+    beta = torch.full((2, 3), 0.5, device=DEV)
+    alpha = torch.full((2, 3), 0.9, device=DEV)
+    o = torch.full((2, 3, d), 7.0, device=DEV)
+    stq.decode_step(lay, pool, slots, q, k, v, beta, alpha, w, o, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0, stq.status_flags(status)
+    assert torch.all(o == 0)
+    gp = pool.cpu().numpy()
+    for r in range(2):
+        for h, b in enumerate(bits):
+            blk = tile_bytes(orc, gp, bits, d, r, h)
+            assert np.all(orc.codes(b, d, d, blk) == 0)
+            rs, cs = orc.scales(b, d, d, blk)
+            assert np.all(rs == 1.0) and np.all(cs == 1.0)
 
 
 @pytest.mark.parametrize("gate", [1, 2])
