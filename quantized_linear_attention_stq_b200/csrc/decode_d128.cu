@@ -831,6 +831,9 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
     const int tid = threadIdx.x, warp = tid >> 5;
     const int G = (int)gridDim.x;
     const int my_count = (p.ntiles - (int)blockIdx.x + G - 1) / G;
+    // A launch that follows this one in the same call (another width or request group: disjoint
+    // tiles) may start as its CTAs find room; see launch_t.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     for (int b = tid; b < p.B; b += NT) sm.slots[b] = p.slots[b];
     if (warp == 0) {  // Tensor Memory for this CTA's tile (released below on every path)
@@ -891,8 +894,12 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
     }
 }
 
+// pdl: this launch follows another launch of the same stq_decode_step call. Those touch disjoint
+// tiles, so it may start while the earlier one drains (programmatic dependent launch); the first
+// launch of a call is ordered normally after all earlier work on the stream, so every launch of a
+// call starts after the previous call has finished.
 template <int BITS, int GATE, int IN_BF16, int FIT>
-cudaError_t launch_t(const TileParams &p, cudaStream_t s)
+cudaError_t launch_t(const TileParams &p, cudaStream_t s, bool pdl)
 {
     using C = Cfg<BITS, GATE, IN_BF16, FIT>;
     auto kernel = decode_d128_kernel<BITS, GATE, IN_BF16, FIT>;
@@ -919,20 +926,33 @@ cudaError_t launch_t(const TileParams &p, cudaStream_t s)
     if (per_sm > (int)(512 / TMEM_COLS)) per_sm = (int)(512 / TMEM_COLS);
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int grid = p.ntiles < sms * per_sm ? p.ntiles : sms * per_sm;
-    kernel<<<grid, NT, smem, s>>>(p);
-    return cudaGetLastError();
+    if (!pdl) {
+        kernel<<<grid, NT, smem, s>>>(p);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
 template <int BITS, int FIT>
-cudaError_t launch_bits(const TileParams &p, int in_bf16, cudaStream_t s)
+cudaError_t launch_bits(const TileParams &p, int in_bf16, cudaStream_t s, bool pdl)
 {
     switch (p.gate * 2 + (in_bf16 ? 1 : 0)) {
-    case 0: return launch_t<BITS, 0, 0, FIT>(p, s);
-    case 1: return launch_t<BITS, 0, 1, FIT>(p, s);
-    case 2: return launch_t<BITS, 1, 0, FIT>(p, s);
-    case 3: return launch_t<BITS, 1, 1, FIT>(p, s);
-    case 4: return launch_t<BITS, 2, 0, FIT>(p, s);
-    default: return launch_t<BITS, 2, 1, FIT>(p, s);
+    case 0: return launch_t<BITS, 0, 0, FIT>(p, s, pdl);
+    case 1: return launch_t<BITS, 0, 1, FIT>(p, s, pdl);
+    case 2: return launch_t<BITS, 1, 0, FIT>(p, s, pdl);
+    case 3: return launch_t<BITS, 1, 1, FIT>(p, s, pdl);
+    case 4: return launch_t<BITS, 2, 0, FIT>(p, s, pdl);
+    default: return launch_t<BITS, 2, 1, FIT>(p, s, pdl);
     }
 }
 
@@ -942,14 +962,14 @@ int decode_d128_max_requests() { return MAXB; }
 
 // All entries of p.table have the width `bits`. p.fit_rounds is 0 or 1 (one round of the joint
 // scale refinement; FP16 pivot heads have no scales and ignore it).
-cudaError_t launch_decode_d128(const TileParams &p, int bits, int in_bf16, cudaStream_t s)
+cudaError_t launch_decode_d128(const TileParams &p, int bits, int in_bf16, cudaStream_t s, bool pdl)
 {
     const bool fit = p.fit_rounds > 0;
     switch (bits) {
-    case 4: return fit ? launch_bits<4, 1>(p, in_bf16, s) : launch_bits<4, 0>(p, in_bf16, s);
-    case 6: return fit ? launch_bits<6, 1>(p, in_bf16, s) : launch_bits<6, 0>(p, in_bf16, s);
-    case 8: return fit ? launch_bits<8, 1>(p, in_bf16, s) : launch_bits<8, 0>(p, in_bf16, s);
-    default: return launch_bits<16, 0>(p, in_bf16, s);
+    case 4: return fit ? launch_bits<4, 1>(p, in_bf16, s, pdl) : launch_bits<4, 0>(p, in_bf16, s, pdl);
+    case 6: return fit ? launch_bits<6, 1>(p, in_bf16, s, pdl) : launch_bits<6, 0>(p, in_bf16, s, pdl);
+    case 8: return fit ? launch_bits<8, 1>(p, in_bf16, s, pdl) : launch_bits<8, 0>(p, in_bf16, s, pdl);
+    default: return launch_bits<16, 0>(p, in_bf16, s, pdl);
     }
 }
 

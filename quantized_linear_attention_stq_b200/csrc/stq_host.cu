@@ -232,6 +232,7 @@ stq_status stq_decode_step(const stq_layout *L, void *pool, int32_t pool_slots, 
     const std::vector<int> ord = order_by_size(L, head_begin, head_count);
     const size_t in_sz = in_bf16 ? 2 : 4;
     const int na = L->gate == STQ_GATE_SCALAR ? 1 : L->dk;
+    bool later = false;  // a tuned launch of this call already went out: the next ones may overlap it
     for (int b0 = 0; b0 < B; b0 += maxb) {
         const int nb = std::min(maxb, B - b0);
         // requests [b0, b0+nb): shift every per-request array
@@ -254,9 +255,11 @@ stq_status stq_decode_step(const stq_layout *L, void *pool, int32_t pool_slots, 
             }
             fill_table(*p, L, ord, first, n, head_begin);
             p->ntiles = nb * n;
-            const cudaError_t e = tuned ? stq::launch_decode_d128(*p, L->bits[ord[first]], in_bf16, (cudaStream_t)stream)
+            const cudaError_t e = tuned ? stq::launch_decode_d128(*p, L->bits[ord[first]], in_bf16,
+                                                                  (cudaStream_t)stream, later)
                                         : stq::launch_decode_generic(*p, in_bf16, (cudaStream_t)stream);
             if (e != cudaSuccess) return STQ_ERR_CUDA;
+            later = tuned;
             first += n;
         }
     }
