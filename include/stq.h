@@ -121,8 +121,9 @@ int32_t stq_abi_version(void);
 const char *stq_status_string(int32_t status);
 
 /* Build a layout from `desc` (host only; no CUDA call). Returns STQ_ERR_INVALID_ARG for NULL
- * pointers or non-positive sizes, STQ_ERR_UNSUPPORTED for widths other than {4,6,8,16} or
- * shapes the device path does not support. On success *out owns a new layout, released with
+ * pointers, non-positive sizes, an unknown gate, input dtype, scale mode or scale dtype, or
+ * scale_fit_rounds outside 0..8; STQ_ERR_UNSUPPORTED for widths other than {4,6,8,16}, shapes the
+ * device path does not support, or bf16 scales / refinement rounds with the uniform mode. On success *out owns a new layout, released with
  * stq_layout_destroy. The layout may be shared between threads. */
 stq_status stq_layout_create(const stq_layout_desc *desc, stq_layout **out);
 void stq_layout_destroy(stq_layout *layout);

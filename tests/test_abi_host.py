@@ -117,6 +117,20 @@ def test_layout_rejects_bad_descriptors(stq):
     assert e.value.status == stq.api.STQ_ERR_INVALID_ARG
     with pytest.raises(stq.StqError):
         stq.Layout([4], 128, gate=7)
+    with pytest.raises(stq.StqError) as e:
+        stq.Layout([4], 128, fit_rounds=9)
+    assert e.value.status == stq.api.STQ_ERR_INVALID_ARG
+    with pytest.raises(stq.StqError) as e:
+        stq.Layout([4], 128, fit_rounds=-1)
+    assert e.value.status == stq.api.STQ_ERR_INVALID_ARG
+    with pytest.raises(stq.StqError) as e:
+        stq.Layout([4], 128, scale_mode=stq.SCALES_UNIFORM, fit_rounds=1)
+    assert e.value.status == stq.api.STQ_ERR_UNSUPPORTED
+    with pytest.raises(TypeError):
+        stq.Layout([4], 128, scale_dtype=torch.float16)
+    # the scale format and the refinement leave the pool layout of row x column heads as specified
+    assert stq.Layout([6], 128, fit_rounds=3).head_bytes(0) == 13312
+    assert stq.Layout([6], 128, scale_dtype=torch.bfloat16).head_bytes(0) == 12800
 
 
 def test_calls_reject_bad_arguments_before_enqueueing(stq):
