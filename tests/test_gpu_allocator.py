@@ -77,3 +77,68 @@ def test_row_impact_matches_oracle(stq, d, gate, dtype):
         ref = alo.row_impact(q[:, h].double().numpy(), k[:, h].double().numpy(), beta[:, h].double().numpy(),
                              alpha[:, h].double().numpy(), gate)
         np.testing.assert_allclose(got[h], ref, rtol=2e-5, atol=1e-12)
+
+
+def test_study_time_and_space_dimensions_over_2048_tokens(stq):
+    """The method's two dimensions together, over 2048 decode tokens of all 2304 heads of one
+    request (the pages follow their states for 2048 decode steps: "线性注意力状态量化难题", section
+    空间维度): random widths (the workload as specified) or lifetime-aware widths within the same
+    bytes (time dimension), each with the one-pass scales or one round of the impact-weighted joint
+    refit (space dimension), beside the exact fp64 recurrence. Per configuration and checkpoint:
+    the median and p90 over heads of the relative state error, and the heads no longer finite."""
+    from quantized_linear_attention_stq_b200 import calibrate
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl = wlm.WORKLOADS["full2304_b70_mixed"]
+    H, d = wl.heads, wl.d
+    rand_bits = wlm.head_bits(wl)
+    w = wlm.impact_weights(wl, DEV)
+    log_ret = np.log(wlm.gate_values(wl).double().numpy())
+    budget = stq.Layout(rand_bits, d).bytes_per_request
+    S_cal = torch.stack([wlm.initial_state(wl, 100 + r, DEV) for r in range(4)])
+    life_bits = calibrate.lifetime_widths(S_cal, w, log_ret, budget, 32)
+    del S_cal
+    S0 = wlm.initial_state(wl, 0, DEV)
+    slots = torch.zeros(1, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    runs = {}
+    for wname, bits in (("random", rand_bits), ("lifetime", life_bits)):
+        for rounds in (0, 1):
+            lay = stq.Layout(bits, d, fit_rounds=rounds)
+            pool = lay.alloc_pool(1, DEV)
+            stq.init_state(lay, pool, slots, S0[None].contiguous(), w, status=status)
+            runs[wname, rounds] = (lay, pool)
+    S = S0.double()
+    checkpoints = (256, 1024, 2048)
+    rows = []
+    for t in range(checkpoints[-1]):
+        inp = wlm.decode_inputs(wl, t, DEV, batch=1)
+        k, v = inp["k"][0].double(), inp["v"][0].double()
+        beta, alpha = inp["beta"][0].double()[:, None, None], inp["alpha"][0].double()[:, None, None]
+        u = torch.einsum("hi,hij->hj", k, S)
+        S = alpha * (S - beta * k[:, :, None] * u[:, None, :]) + beta * k[:, :, None] * v[:, None, :]
+        o = torch.empty(1, H, d, device=DEV)
+        for lay, pool in runs.values():
+            stq.decode_step(lay, pool, slots, inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], w, o,
+                            status=status)
+        if t + 1 in checkpoints:
+            for (wname, rounds), (lay, pool) in runs.items():
+                Sq = torch.zeros(1, H, d, d, device=DEV)
+                stq.dequantize(lay, pool, slots, Sq)
+                err = ((Sq[0].double() - S).norm(dim=(1, 2)) / S.norm(dim=(1, 2))).cpu().numpy()
+                fin = np.isfinite(err)
+                rows.append((t + 1, wname, rounds, float(np.median(err[fin])) if fin.any() else float("nan"),
+                             float(np.quantile(err[fin], 0.9)) if fin.any() else float("nan"), int((~fin).sum())))
+    torch.cuda.synchronize()
+    print()
+    print("| tokens | widths | refit rounds | median state err | p90 state err | heads not finite |")
+    print("|---|---|---|---|---|---|")
+    for r in rows:
+        print(f"| {r[0]} | {r[1]} | {r[2]} | {r[3]:.3e} | {r[4]:.3e} | {r[5]} |")
+    final = {(r[1], r[2]): r for r in rows if r[0] == checkpoints[-1]}
+    # the specified widths with one-pass scales blow up; either dimension alone keeps the tail
+    # bounded; both together do best
+    assert all(r[5] == 0 for r in final.values())
+    assert final["random", 0][4] > 100.0
+    assert final["random", 1][4] < 1.0 and final["lifetime", 0][4] < 1.0
+    assert final["lifetime", 1][4] < min(final["random", 1][4], final["lifetime", 0][4])
