@@ -307,7 +307,7 @@ def per_layer_graph_leg(stq, lay, pool, slots, toks, w, status, dev, steps: int,
             "note": "one stq_decode_step per layer, a token's layers captured in one CUDA graph"}
 
 
-def prefill_leg(dev, steps: int = 3, warmup: int = 1, T: int = 8192) -> dict:
+def prefill_leg(dev, steps: int = 3, warmup: int = 1, T: int = 8192, fit_rounds: int = 0) -> dict:
     """The chunked-prefill workload (16 requests x 16 heads, 6-bit, an 8192-token prompt in 64-token
     chunks, bf16 inputs) timed as whole stq_prefill_chunk calls, inputs resident in HBM."""
     import torch
@@ -318,7 +318,7 @@ def prefill_leg(dev, steps: int = 3, warmup: int = 1, T: int = 8192) -> dict:
     wl = wlm.WORKLOADS["prefill16_b16_6bit"]
     B, H, d, C = wl.batch, wl.heads, wl.d, 64
     bits = wlm.head_bits(wl)
-    lay = stq.Layout(bits, d, gate=wl.gate, in_dtype=wl.in_dtype)
+    lay = stq.Layout(bits, d, gate=wl.gate, in_dtype=wl.in_dtype, fit_rounds=fit_rounds)
     pool = lay.alloc_pool(B, dev)
     slots = torch.arange(B, dtype=torch.int32, device=dev)
     w = wlm.impact_weights(wl, dev)
@@ -355,7 +355,8 @@ def prefill_leg(dev, steps: int = 3, warmup: int = 1, T: int = 8192) -> dict:
     del inp, o, pool
     return {"workload": "prefill16_b16_6bit", "prompt_tokens": T, "chunk": C, "requests": B, "heads": H,
             "ms_per_call": ms, "head_tokens_per_s": B * H * T / (ms / 1e3), "tokens_per_s": B * T / (ms / 1e3),
-            "calls": steps, "kernel": "prefill_wy_kernel<6> (tcgen05, one launch)",
+            "calls": steps, "fit_rounds": fit_rounds,
+            "kernel": "prefill_wy_kernel<6> (tcgen05, one launch)" if fit_rounds <= 1 else "prefill_seq_kernel",
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "peak_kind": kind, "bytes_per_call": nbytes}}
 
@@ -574,7 +575,7 @@ def run_ours(args):
     if lifetime:
         result["config"]["widths_from"] = "lifetime-aware allocation (stq_allocate_widths), same byte budget"
     if world == 1 and not args.no_prefill:
-        result["prefill"] = prefill_leg(dev, T=args.prefill_tokens)
+        result["prefill"] = prefill_leg(dev, T=args.prefill_tokens, fit_rounds=args.fit_rounds)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not lifetime:
         rate, cores, sample = time_oracle(args.workload, oracle_workers(), 16, 20)
         result["cpu_baseline"] = {"value": rate, "unit": "head-steps/s", "cores": cores, "kind": "oracle",
@@ -642,7 +643,8 @@ def main(argv=None):
         import torch
 
         dev = torch.device("cuda", torch.cuda.current_device())
-        print(json.dumps({"prefill": prefill_leg(dev, steps=args.steps, warmup=args.warmup, T=args.prefill_tokens)}),
+        print(json.dumps({"prefill": prefill_leg(dev, steps=args.steps, warmup=args.warmup, T=args.prefill_tokens,
+                                                 fit_rounds=args.fit_rounds)}),
               flush=True)
     else:
         run_ours(args)

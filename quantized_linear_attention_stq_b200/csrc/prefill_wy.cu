@@ -404,7 +404,9 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
 // The kernel: persistent CTAs over (request, head) tiles of one code width; the chunks of a tile
 // run in order. Warp w reads Tensor Memory lane quarter q4 = w % 4 and column quarter cq = w / 4.
 // ---------------------------------------------------------------------------------------------
-template <int BITS>
+// FIT: one round of the impact-weighted joint refit at every chunk end (a separate instance, so
+// that the plain requantization keeps its registers).
+template <int BITS, int FIT>
 __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant__ TileParams p, const int T_tok)
 {
     using P = PCfg<BITS>;
@@ -808,6 +810,79 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                     x = fminf(fmaxf(x, -(float)P::QMAX), (float)P::QMAX);
                     qc[j] = (int)x;
                 }
+                if constexpr (FIT) {
+                    // One round of the impact-weighted joint refit (the same round as the decode
+                    // kernel's): S[j] holds t_ij = S'_ij / c~_j, qc the one-pass codes.
+                    //   c_j <- c~_j sum_i w_i r~_i Q_ij t_ij / sum_i w_i (r~_i Q_ij)^2
+                    //   r_i <- sum_j c~new_j c~_j Q_ij t_ij / sum_j (c~new_j Q_ij)^2
+                    // each stored (rounded) and kept only if finite and positive.
+                    float *red2 = rmax;  // free once the row scales are formed
+                    const float wr = wi * ri;
+#pragma unroll 1
+                    for (int pass = 0; pass < 2; ++pass) {
+                        __syncthreads();  // the previous readers of sq / red are done
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            float e[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const float qv = (float)qc[4 * k + u];
+                                e[u] = pass == 0 ? wr * qv * S[4 * k + u] : (wr * ri) * (qv * qv);
+                            }
+                            *reinterpret_cast<float4 *>(sq + i * LDSQ + 32 * cq + 4 * k) = make_float4(e[0], e[1], e[2], e[3]);
+                        }
+                        __syncthreads();
+                        const int j = tid & (D - 1), r0 = 32 * (tid >> 7);
+                        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+                        for (int r = 0; r < 32; r += 4) {
+                            a0 += sq[(r0 + r) * LDSQ + j];
+                            a1 += sq[(r0 + r + 1) * LDSQ + j];
+                            a2 += sq[(r0 + r + 2) * LDSQ + j];
+                            a3 += sq[(r0 + r + 3) * LDSQ + j];
+                        }
+                        (pass == 0 ? red : red2)[(tid >> 7) * D + j] = (a0 + a1) + (a2 + a3);
+                    }
+                    __syncthreads();
+                    if (tid < D) {
+                        const float N = (red[tid] + red[D + tid]) + (red[2 * D + tid] + red[3 * D + tid]);
+                        const float Dn = (red2[tid] + red2[D + tid]) + (red2[2 * D + tid] + red2[3 * D + tid]);
+                        const float co = sC[tid];
+                        float cn = co;
+                        if (Dn > 0.f) {
+                            const float cr = round_scale(co * (N / Dn), p.scale_bf16);
+                            if (isfinite(cr) && cr > 0.f) cn = cr;
+                        }
+                        red[tid] = cn * co;             // row-step factor of the numerator
+                        red2[tid] = cn * cn;            // and of the denominator
+                        red[2 * D + tid] = co / cn;     // t -> S' / c~new
+                        sC[tid] = cn;
+                    }
+                    __syncthreads();
+                    float pn = 0.f, pd = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float qv = (float)qc[j];
+                        pn += red[32 * cq + j] * qv * S[j];
+                        pd += red2[32 * cq + j] * (qv * qv);
+                    }
+                    sq[cq * D + i] = pn;
+                    sq[4 * D + cq * D + i] = pd;
+                    __syncthreads();
+                    const float num = (sq[i] + sq[D + i]) + (sq[2 * D + i] + sq[3 * D + i]);
+                    const float den = (sq[4 * D + i] + sq[5 * D + i]) + (sq[6 * D + i] + sq[7 * D + i]);
+                    if (den > 0.f) {
+                        const float rn = round_scale(num / den, p.scale_bf16);
+                        if (isfinite(rn) && rn > 0.f) ri = rn;
+                    }
+                    const float rrn = __frcp_rn(ri);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        float x = rintf(S[j] * red[2 * D + 32 * cq + j] * rrn);
+                        x = fminf(fmaxf(x, -(float)P::QMAX), (float)P::QMAX);
+                        qc[j] = (int)x;
+                    }
+                }
                 // next chunk's B operand (row i, columns 32 cq ..) and scales
                 uint8_t *qrow = sm + OFF_QC + (cq >> 1) * 16384;
 #pragma unroll
@@ -840,10 +915,10 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
     }
 }
 
-template <int BITS>
+template <int BITS, int FIT>
 cudaError_t launch_w(const TileParams &p, int T, cudaStream_t s)
 {
-    auto kernel = prefill_wy_kernel<BITS>;
+    auto kernel = prefill_wy_kernel<BITS, FIT>;
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
     int dev = 0, sms = 0;
@@ -861,10 +936,11 @@ cudaError_t launch_w(const TileParams &p, int T, cudaStream_t s)
 // p.table has width `bits` (4, 6 or 8).
 cudaError_t launch_prefill_wy(const TileParams &p, int bits, int T, cudaStream_t s)
 {
+    const bool fit = p.fit_rounds > 0;  // 0 or 1 here
     switch (bits) {
-    case 4: return launch_w<4>(p, T, s);
-    case 6: return launch_w<6>(p, T, s);
-    case 8: return launch_w<8>(p, T, s);
+    case 4: return fit ? launch_w<4, 1>(p, T, s) : launch_w<4, 0>(p, T, s);
+    case 6: return fit ? launch_w<6, 1>(p, T, s) : launch_w<6, 0>(p, T, s);
+    case 8: return fit ? launch_w<8, 1>(p, T, s) : launch_w<8, 0>(p, T, s);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -310,7 +310,7 @@ stq_status stq_prefill_chunk(const stq_layout *L, void *pool, int32_t pool_slots
     // WY path, one launch per code width; FP16 pivot heads and every other configuration take the
     // sequential kernel.
     const bool wy = L->dk == 128 && L->gate == STQ_GATE_SCALAR && L->in_dtype == STQ_BF16 && chunk == 64 &&
-                    !L->uniform && L->fit_rounds == 0;
+                    !L->uniform && L->fit_rounds <= 1;
     if (!wy) {
         std::vector<int> ord(L->H);
         for (int h = 0; h < L->H; ++h) ord[h] = h;

@@ -198,18 +198,19 @@ def test_decode_channel_gates(stq, orc, gate):
     _decode_teacher_forced(stq, orc, wl_, [4, 6, 8], 3)
 
 
-def test_prefill_chunk(stq, orc):
-    """A 64-token chunk and a 30-token chunk in one call (routed to the sequential kernel), one
-    request x three heads at d = 128, bf16 inputs: the first chunk's end state is checked through
-    the oracle's chunk, then the call's final block from the oracle's bytes after that chunk."""
+@pytest.mark.parametrize("rounds", [1, 2])
+def test_prefill_chunk(stq, orc, rounds):
+    """A 64-token chunk, then a 30-token chunk from the oracle's bytes, one request x three heads at
+    d = 128, bf16 inputs: one round runs in the tensor-core prefill's chunk-end requantization, two
+    on the sequential kernel."""
     from quantized_linear_attention_stq_b200 import workloads as wlm
 
     bits, d, T = [4, 6, 8], 128, 94
     wl_ = _wl("prefill16_b16_6bit", batch=1, heads=3)
-    lay = stq.Layout(bits, d, in_dtype=torch.bfloat16, fit_rounds=ROUNDS)
+    lay = stq.Layout(bits, d, in_dtype=torch.bfloat16, fit_rounds=rounds)
     w = wlm.impact_weights(wl_)
     S0 = wlm.initial_state(wl_, 0)[None]
-    opool = _oracle_pool(orc, bits, d, S0, w, ROUNDS)
+    opool = _oracle_pool(orc, bits, d, S0, w, rounds)
     inp = wlm.prefill_inputs(wl_, 0, T)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     tally = Tally()
@@ -229,8 +230,8 @@ def test_prefill_chunk(stq, orc):
         S = orc.dequantize(b, d, d, blk)
         for t in range(64):
             S, _ = orc.update(0, S, args[0][t], args[1][t], args[2][t], args[3][t], args[4][t])
-        res = orc.prefill_seq_s(b, orc.SCALE_F32, 0, blk, *args, as_f64(w[h]), 64, d, d, rounds=ROUNDS)
-        compare_block_fit(orc, b, d, tile_bytes(orc, gp, bits, d, 0, h), S, as_f64(w[h]), ROUNDS, tally,
+        res = orc.prefill_seq_s(b, orc.SCALE_F32, 0, blk, *args, as_f64(w[h]), 64, d, d, rounds=rounds)
+        compare_block_fit(orc, b, d, tile_bytes(orc, gp, bits, d, 0, h), S, as_f64(w[h]), rounds, tally,
                           f"chunk 0 head {h}")
         for t in range(64):
             compare_o(og[0, h, t], res["o"][t], tally, f"o token {t} head {h}")
@@ -250,7 +251,7 @@ def test_prefill_chunk(stq, orc):
         S = orc.dequantize(b, d, d, blk)
         for t in range(T - 64):
             S, _ = orc.update(0, S, args[0][t], args[1][t], args[2][t], args[3][t], args[4][t])
-        compare_block_fit(orc, b, d, tile_bytes(orc, gp, bits, d, 0, h), S, as_f64(w[h]), ROUNDS, tally,
+        compare_block_fit(orc, b, d, tile_bytes(orc, gp, bits, d, 0, h), S, as_f64(w[h]), rounds, tally,
                           f"chunk 1 head {h}")
     tally.check_budget()
 
