@@ -200,15 +200,14 @@ __device__ __forceinline__ void unpack_row(const uint8_t *src, int cg, float2 of
         Q[2] = __fadd2_rn(code_pair<4>(wd >> 16, magic), off);
         Q[3] = __fadd2_rn(code_pair<4>(wd >> 24, magic), off);
     } else if constexpr (BITS == 6) {
-        uint32_t lo, hi;
-        if ((cg & 1) == 0) {
-            lo = *reinterpret_cast<const uint32_t *>(src);
-            hi = *reinterpret_cast<const uint16_t *>(src + 4);
-        } else {
-            const uint32_t w1 = *reinterpret_cast<const uint32_t *>(src + 2);
-            lo = (uint32_t)(*reinterpret_cast<const uint16_t *>(src)) | (w1 << 16);
-            hi = w1 >> 16;
-        }
+        // the 6-byte segment starts 4-byte aligned for even cg and 2 bytes past it for odd cg: load
+        // the two aligned words around it and shift (no branch on the lane's parity; the bits of
+        // hi above 15 belong to the next lane and are never used)
+        const int odd = cg & 1;
+        const uint32_t *a = reinterpret_cast<const uint32_t *>(src - 2 * odd);
+        const uint32_t w0 = a[0], w1 = a[1];
+        const uint32_t lo = __funnelshift_r(w0, w1, 16 * odd);
+        const uint32_t hi = w1 >> (16 * odd);
         Q[0] = __fadd2_rn(code_pair<6>(lo, magic), off);
         Q[1] = __fadd2_rn(code_pair<6>(lo >> 12, magic), off);
         Q[2] = __fadd2_rn(code_pair<6>(__funnelshift_r(lo, hi, 24), magic), off);
@@ -244,14 +243,12 @@ __device__ __forceinline__ void pack_store_row(uint8_t *dst, int cg, const float
                                           ((uint64_t)MAGIC << 18) + ((uint64_t)MAGIC << 24) + ((uint64_t)MAGIC << 30));
         const uint32_t lo = f0 + (f1 << 6) + (f2 << 12) + (f3 << 18) + (f4 << 24) + (f5 << 30) - C;
         // bits 32..47: the top 4 bits of code 5, codes 6 and 7 (garbage above bit 15 is dropped)
-        const uint32_t hi = ((f5 >> 2) + (f6 << 4) + (f7 << 10)) & 0xFFFFu;
-        if ((cg & 1) == 0) {
-            *reinterpret_cast<uint32_t *>(dst) = lo;
-            *reinterpret_cast<uint16_t *>(dst + 4) = (uint16_t)hi;
-        } else {
-            *reinterpret_cast<uint16_t *>(dst) = (uint16_t)(lo & 0xFFFFu);
-            *reinterpret_cast<uint32_t *>(dst + 2) = (lo >> 16) | (hi << 16);
-        }
+        const uint32_t hi = (f5 >> 2) + (f6 << 4) + (f7 << 10);
+        // three 2-byte stores fit every lane's alignment (no branch on the lane's parity)
+        uint16_t *d16 = reinterpret_cast<uint16_t *>(dst);
+        d16[0] = (uint16_t)lo;
+        d16[1] = (uint16_t)(lo >> 16);
+        d16[2] = (uint16_t)hi;
     } else {
         uint2 wd;
         wd.x = __byte_perm(__byte_perm(f0, f1, 0x0040), __byte_perm(f2, f3, 0x0040), 0x5410);
