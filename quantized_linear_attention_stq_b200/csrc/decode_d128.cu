@@ -104,7 +104,7 @@ struct __align__(16) SmemFit {
 // ---------------------------------------------------------------------------------------------
 // Static per-width facts
 // ---------------------------------------------------------------------------------------------
-template <int BITS, int GATE, int IN_BF16, int FIT>
+template <int BITS, int GATE, int IN_BF16, int FIT, int SB16>
 struct Cfg {
     static constexpr int RB = BITS == 16 ? 256 : 16 * BITS;    // bytes of one 128-wide row
     static constexpr uint32_t SOFF = scale_offset(BITS, D, D);  // byte offset of r[]
@@ -275,10 +275,10 @@ __device__ __forceinline__ float sum4(const float *src, int stride)
     return (src[0] + src[stride]) + (src[2 * stride] + src[3 * stride]);
 }
 
-template <int BITS, int GATE, int IN_BF16, int FIT>
+template <int BITS, int GATE, int IN_BF16, int FIT, int SB16>
 __device__ __forceinline__ uint8_t *ring_slot(uint8_t *smem, int slot_i)
 {
-    return smem + Cfg<BITS, GATE, IN_BF16, FIT>::RING + (size_t)slot_i * Cfg<BITS, GATE, IN_BF16, FIT>::LEN;
+    return smem + Cfg<BITS, GATE, IN_BF16, FIT, SB16>::RING + (size_t)slot_i * Cfg<BITS, GATE, IN_BF16, FIT, SB16>::LEN;
 }
 
 __device__ __forceinline__ SmemChannel &channel(uint8_t *smem)
@@ -286,19 +286,19 @@ __device__ __forceinline__ SmemChannel &channel(uint8_t *smem)
     return *reinterpret_cast<SmemChannel *>(smem + sizeof(SmemFixed));
 }
 
-template <int BITS, int GATE, int IN_BF16, int FIT>
+template <int BITS, int GATE, int IN_BF16, int FIT, int SB16>
 __device__ __forceinline__ SmemFit &fitmem(uint8_t *smem)
 {
-    return *reinterpret_cast<SmemFit *>(smem + Cfg<BITS, GATE, IN_BF16, FIT>::FIT_OFF);
+    return *reinterpret_cast<SmemFit *>(smem + Cfg<BITS, GATE, IN_BF16, FIT, SB16>::FIT_OFF);
 }
 
 // Thread 0: stream this CTA's next tile into ring slot n % NS (codes + scales and the input rows
 // by bulk copy, the per-tile scalars by 4-byte cp.async), completing on the slot's mbarrier (two
 // arrivals: expect_tx + cp.async), and record where the tile lives and which row it reads.
-template <int BITS, int GATE, int IN_BF16, int FIT>
+template <int BITS, int GATE, int IN_BF16, int FIT, int SB16>
 __device__ __forceinline__ void issue_next(const TileParams &p, SmemFixed &sm, uint8_t *smem, Issuer &it, int my_count)
 {
-    using C = Cfg<BITS, GATE, IN_BF16, FIT>;
+    using C = Cfg<BITS, GATE, IN_BF16, FIT, SB16>;
     if (it.n >= my_count) return;
     const int n = it.n, slot_i = n % C::NS;
     const TileEntry e = p.table[it.pos];
@@ -329,8 +329,8 @@ __device__ __forceinline__ void issue_next(const TileParams &p, SmemFixed &sm, u
     cp_async4(smem_u32(&sm.scal[slot_i][0]), p.beta + row);
     if (GATE == 0) cp_async4(smem_u32(&sm.scal[slot_i][1]), p.alpha + row);
     cp_async_arrive(bar);
-    const uint32_t dst = smem_u32(ring_slot<BITS, GATE, IN_BF16, FIT>(smem, slot_i));
-    const uint32_t blk = p.scale_bf16 ? C::BLK16 : C::BLK;
+    const uint32_t dst = smem_u32(ring_slot<BITS, GATE, IN_BF16, FIT, SB16>(smem, slot_i));
+    const uint32_t blk = SB16 ? C::BLK16 : C::BLK;
     mbar_arrive_expect_tx(bar, C::LEN - (C::BLK - blk));
     bulk_g2s(dst, src, blk, bar);
     bulk_g2s(dst + C::K_OFF, (const uint8_t *)p.k + (size_t)row * C::ROW_IN, C::ROW_IN, bar);
@@ -342,10 +342,10 @@ __device__ __forceinline__ void issue_next(const TileParams &p, SmemFixed &sm, u
 
 // Wait for tile n (ring slot n % NS) and compute its row factors, row i = threadIdx.x, with
 // per-warp sums of w, q.k and q.(alpha k). Returns false on a timeout.
-template <int BITS, int GATE, int IN_BF16, int FIT>
-__device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, int n, int my_count, int sb16)
+template <int BITS, int GATE, int IN_BF16, int FIT, int SB16>
+__device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, int n, int my_count)
 {
-    using C = Cfg<BITS, GATE, IN_BF16, FIT>;
+    using C = Cfg<BITS, GATE, IN_BF16, FIT, SB16>;
     if (n >= my_count) return true;
     const int slot_i = n % C::NS;
     const uint32_t phase = (uint32_t)(n / C::NS) & 1u;
@@ -353,10 +353,10 @@ __device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, in
     if (!__all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&sm.bars[slot_i]), phase))) return false;
     if (sm.meta[n & 3].skip) return true;  // skipped tile: nothing was loaded
     const int pb = n & 1;
-    const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16, FIT>(smem, slot_i);
+    const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16, FIT, SB16>(smem, slot_i);
     const int i = threadIdx.x;
     constexpr bool pivot = BITS == 16;
-    const float r = pivot ? 1.f : load_scale(tile + C::SOFF, i, sb16);
+    const float r = pivot ? 1.f : load_scale(tile + C::SOFF, i, SB16);
     const float k = load_in<IN_BF16>(tile + C::K_OFF, i);
     const float q = load_in<IN_BF16>(tile + C::Q_OFF, i);
     const float w = reinterpret_cast<const float *>(tile + C::W_OFF)[i];
@@ -397,14 +397,15 @@ __device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, in
 // colG1 and the new s_i = 1 / (sqrt(w_i) r~_i) into rowS. Two CTA barriers; the row sums stay in
 // each half-warp. c_one is this thread's column c'_j (j = threadIdx.x); r_one / s_one are the
 // one-pass r and s of this lane's row i = 8 cg + rb.
-template <int BITS, int GATE, int IN_BF16, int FIT>
+template <int BITS, int GATE, int IN_BF16, int FIT, int SB16>
 __device__ __forceinline__ bool refit_scales(const TileParams &p, SmemFixed &sm, uint8_t *smem, int n, uint32_t tcol,
                                              float c_one, float r_one, float s_one)
 {
-    using C = Cfg<BITS, GATE, IN_BF16, FIT>;
+    using C = Cfg<BITS, GATE, IN_BF16, FIT, SB16>;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, cg = lane & 15, sub = lane >> 4;
-    const int rb = 2 * warp + sub, pb = n & 1, sb16 = p.scale_bf16;
-    const float *rho = fitmem<BITS, GATE, IN_BF16, FIT>(smem).rowRho;
+    const int rb = 2 * warp + sub, pb = n & 1;
+    constexpr int sb16 = SB16;
+    const float *rho = fitmem<BITS, GATE, IN_BF16, FIT, SB16>(smem).rowRho;
     const float2 rnd = make_float2(C::ROUND, C::ROUND), nrnd = make_float2(-C::ROUND, -C::ROUND);
     uint8_t *gsc = reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + C::SOFF);
     tmem_wait_st();
@@ -537,16 +538,16 @@ __device__ __forceinline__ bool refit_scales(const TileParams &p, SmemFixed &sm,
 }
 
 // Tile n (ring slot n % NS). Returns false if the wait for the next tile timed out.
-template <int BITS, int GATE, int IN_BF16, int FIT>
+template <int BITS, int GATE, int IN_BF16, int FIT, int SB16>
 __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm, uint8_t *smem, int n, int my_count,
                                              uint32_t tcol)
 {
-    using C = Cfg<BITS, GATE, IN_BF16, FIT>;
+    using C = Cfg<BITS, GATE, IN_BF16, FIT, SB16>;
     constexpr bool pivot = BITS == 16;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, cg = lane & 15, sub = lane >> 4;
     const int pb = n & 1, slot_i = n % C::NS;
     const int rb = 2 * warp + sub;  // this thread's rows: rb + 8m, m < 16
-    const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16, FIT>(smem, slot_i);
+    const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16, FIT, SB16>(smem, slot_i);
     // the tile's record (sm.meta[n & 3]) stays valid until the issue after the next tile's B2
 
     // ---- Sweep A: unpack to TMEM, column sums of k~Q and q~Q -------------------------------
@@ -587,7 +588,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
 
     // ---- Column finals (column j = tid): update coefficients and the readout ---------------
     const int j = tid;
-    const int sb16 = p.scale_bf16;
+    constexpr int sb16 = SB16;
     const float cj = pivot ? 1.f : load_scale(tile + C::SOFF, D + j, sb16);
     const float inv_sig = (j & 1) ? 1.f / C::SIG1 : 1.f;  // powers of two: exact
     {
@@ -615,7 +616,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
         if (!isfinite(o)) flag(p.status, kFlagNonfinite);
     }
     __syncthreads();  // B2: coefficients ready; this tile's ring bytes are no longer read
-    if (tid == 0) issue_next<BITS, GATE, IN_BF16, FIT>(p, sm, smem, sm.iss, my_count);
+    if (tid == 0) issue_next<BITS, GATE, IN_BF16, FIT, SB16>(p, sm, smem, sm.iss, my_count);
 
     // ---- Sweep B: y = rho Q + kappa g1 (+ mu g2), column energy ---------------------------
     tmem_wait_st();
@@ -710,7 +711,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
         if (!isfinite(c) || c == 0.f) flag(p.status, kFlagNonfinite);
         sm.colB[j] = b;
     }
-    const bool ok = precompute_rows<BITS, GATE, IN_BF16, FIT>(sm, smem, n + 1, my_count, sb16);
+    const bool ok = precompute_rows<BITS, GATE, IN_BF16, FIT, SB16>(sm, smem, n + 1, my_count);
     if (__syncthreads_or(!ok)) return false;  // B4: new column scales and next row factors ready
     if constexpr (pivot) return true;
 
@@ -765,7 +766,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
         if constexpr (FIT) {
             r_one = r;
             s_one = s;
-            fitmem<BITS, GATE, IN_BF16, FIT>(smem).rowRho[i] = r * fast_rcp(sm.rowRq[pb][i] * C::QMAX);  // sqrt(w_i) r_i
+            fitmem<BITS, GATE, IN_BF16, FIT, SB16>(smem).rowRho[i] = r * fast_rcp(sm.rowRq[pb][i] * C::QMAX);  // sqrt(w_i) r_i
         } else {
             store_scale(reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + C::SOFF), i, r, sb16);
         }
@@ -773,7 +774,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
     }
     __syncwarp();
     if constexpr (FIT) {
-        if (!refit_scales<BITS, GATE, IN_BF16, FIT>(p, sm, smem, n, tcol, c_one, r_one, s_one)) return false;
+        if (!refit_scales<BITS, GATE, IN_BF16, FIT, SB16>(p, sm, smem, n, tcol, c_one, r_one, s_one)) return false;
     }
 
     // ---- Sweep D: x = z s rounded half to even by the 2^23 + offset FFMA, packed, stored ----
@@ -819,10 +820,10 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
     return true;
 }
 
-template <int BITS, int GATE, int IN_BF16, int FIT>
+template <int BITS, int GATE, int IN_BF16, int FIT, int SB16>
 __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constant__ TileParams p)
 {
-    using C = Cfg<BITS, GATE, IN_BF16, FIT>;
+    using C = Cfg<BITS, GATE, IN_BF16, FIT, SB16>;
     extern __shared__ __align__(128) uint8_t smem[];
     SmemFixed &sm = *reinterpret_cast<SmemFixed *>(smem);
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -858,9 +859,9 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
         it.b = (int)blockIdx.x - it.pos * p.B;
         it.qG = G / p.B;
         it.rG = G - it.qG * p.B;
-        for (int k = 0; k < C::NS; ++k) issue_next<BITS, GATE, IN_BF16, FIT>(p, sm, smem, it, my_count);
+        for (int k = 0; k < C::NS; ++k) issue_next<BITS, GATE, IN_BF16, FIT, SB16>(p, sm, smem, it, my_count);
     }
-    bool failed = __syncthreads_or(!precompute_rows<BITS, GATE, IN_BF16, FIT>(sm, smem, 0, my_count, p.scale_bf16));
+    bool failed = __syncthreads_or(!precompute_rows<BITS, GATE, IN_BF16, FIT, SB16>(sm, smem, 0, my_count));
 
     int n = 0;
     for (; n < my_count && !failed; ++n) {
@@ -868,11 +869,11 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
         const bool got = mbar_wait_bounded(smem_u32(&sm.bars[n % C::NS]), (uint32_t)(n / C::NS) & 1u);
         if (sm.meta[n & 3].skip) {  // out-of-range slot: nothing loaded, nothing to do
             __syncthreads();
-            if (tid == 0) issue_next<BITS, GATE, IN_BF16, FIT>(p, sm, smem, sm.iss, my_count);
-            const bool ok = precompute_rows<BITS, GATE, IN_BF16, FIT>(sm, smem, n + 1, my_count, p.scale_bf16);
+            if (tid == 0) issue_next<BITS, GATE, IN_BF16, FIT, SB16>(p, sm, smem, sm.iss, my_count);
+            const bool ok = precompute_rows<BITS, GATE, IN_BF16, FIT, SB16>(sm, smem, n + 1, my_count);
             failed = __syncthreads_or(!ok || !got);
         } else {
-            failed = !process_tile<BITS, GATE, IN_BF16, FIT>(p, sm, smem, n, my_count, tcol);
+            failed = !process_tile<BITS, GATE, IN_BF16, FIT, SB16>(p, sm, smem, n, my_count, tcol);
         }
     }
     if (failed && tid == 0) {
@@ -895,11 +896,11 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
 // tiles, so it may start while the earlier one drains (programmatic dependent launch); the first
 // launch of a call is ordered normally after all earlier work on the stream, so every launch of a
 // call starts after the previous call has finished.
-template <int BITS, int GATE, int IN_BF16, int FIT>
+template <int BITS, int GATE, int IN_BF16, int FIT, int SB16>
 cudaError_t launch_t(const TileParams &p, cudaStream_t s, bool pdl)
 {
-    using C = Cfg<BITS, GATE, IN_BF16, FIT>;
-    auto kernel = decode_d128_kernel<BITS, GATE, IN_BF16, FIT>;
+    using C = Cfg<BITS, GATE, IN_BF16, FIT, SB16>;
+    auto kernel = decode_d128_kernel<BITS, GATE, IN_BF16, FIT, SB16>;
     const int smem = (int)C::SMEM;
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -940,17 +941,26 @@ cudaError_t launch_t(const TileParams &p, cudaStream_t s, bool pdl)
     return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
-template <int BITS, int FIT>
+template <int BITS, int FIT, int SB16>
 cudaError_t launch_bits(const TileParams &p, int in_bf16, cudaStream_t s, bool pdl)
 {
     switch (p.gate * 2 + (in_bf16 ? 1 : 0)) {
-    case 0: return launch_t<BITS, 0, 0, FIT>(p, s, pdl);
-    case 1: return launch_t<BITS, 0, 1, FIT>(p, s, pdl);
-    case 2: return launch_t<BITS, 1, 0, FIT>(p, s, pdl);
-    case 3: return launch_t<BITS, 1, 1, FIT>(p, s, pdl);
-    case 4: return launch_t<BITS, 2, 0, FIT>(p, s, pdl);
-    default: return launch_t<BITS, 2, 1, FIT>(p, s, pdl);
+    case 0: return launch_t<BITS, 0, 0, FIT, SB16>(p, s, pdl);
+    case 1: return launch_t<BITS, 0, 1, FIT, SB16>(p, s, pdl);
+    case 2: return launch_t<BITS, 1, 0, FIT, SB16>(p, s, pdl);
+    case 3: return launch_t<BITS, 1, 1, FIT, SB16>(p, s, pdl);
+    case 4: return launch_t<BITS, 2, 0, FIT, SB16>(p, s, pdl);
+    default: return launch_t<BITS, 2, 1, FIT, SB16>(p, s, pdl);
     }
+}
+
+// the refit and the scale format as compile-time parameters of the tuned kernel
+template <int BITS>
+cudaError_t launch_modes(const TileParams &p, int in_bf16, cudaStream_t s, bool pdl)
+{
+    const bool fit = p.fit_rounds > 0, sb16 = p.scale_bf16 != 0;
+    if (fit) return sb16 ? launch_bits<BITS, 1, 1>(p, in_bf16, s, pdl) : launch_bits<BITS, 1, 0>(p, in_bf16, s, pdl);
+    return sb16 ? launch_bits<BITS, 0, 1>(p, in_bf16, s, pdl) : launch_bits<BITS, 0, 0>(p, in_bf16, s, pdl);
 }
 
 }  // namespace
@@ -961,12 +971,11 @@ int decode_d128_max_requests() { return MAXB; }
 // scale refinement; FP16 pivot heads have no scales and ignore it).
 cudaError_t launch_decode_d128(const TileParams &p, int bits, int in_bf16, cudaStream_t s, bool pdl)
 {
-    const bool fit = p.fit_rounds > 0;
     switch (bits) {
-    case 4: return fit ? launch_bits<4, 1>(p, in_bf16, s, pdl) : launch_bits<4, 0>(p, in_bf16, s, pdl);
-    case 6: return fit ? launch_bits<6, 1>(p, in_bf16, s, pdl) : launch_bits<6, 0>(p, in_bf16, s, pdl);
-    case 8: return fit ? launch_bits<8, 1>(p, in_bf16, s, pdl) : launch_bits<8, 0>(p, in_bf16, s, pdl);
-    default: return launch_bits<16, 0>(p, in_bf16, s, pdl);
+    case 4: return launch_modes<4>(p, in_bf16, s, pdl);
+    case 6: return launch_modes<6>(p, in_bf16, s, pdl);
+    case 8: return launch_modes<8>(p, in_bf16, s, pdl);
+    default: return launch_bits<16, 0, 0>(p, in_bf16, s, pdl);  // pivots: no scales
     }
 }
 
