@@ -590,18 +590,21 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                     umma::mma_commit(smem_u32(&bars[1]));
                 }
             } else {
-                // ---- warps 12..15: T = (I + L)^-1, then its three bf16 terms -----------------
+                // ---- warps 12..15: T = (I + L)^-1 ------------------------------------------
                 invert_unit_lower(Lm, Tm);
+            }
+            __syncthreads();  // T is complete
+            {
+                // its three bf16 terms, one 8-column unit of one row per thread (all 16 warps)
+                static_assert(NT == 64 * 8, "one T unit per thread");
                 uint8_t *r0 = sm + OFF_RT;
-                for (int unit = tid - 32 * INV_WARP0; unit < 64 * 8; unit += 128) {
-                    const int t = unit >> 3, c8 = unit & 7;
-                    float x[8];
-                    const float4 xa = *reinterpret_cast<const float4 *>(Tm + t * LDL + 8 * c8);
-                    const float4 xb4 = *reinterpret_cast<const float4 *>(Tm + t * LDL + 8 * c8 + 4);
-                    x[0] = xa.x; x[1] = xa.y; x[2] = xa.z; x[3] = xa.w;
-                    x[4] = xb4.x; x[5] = xb4.y; x[6] = xb4.z; x[7] = xb4.w;
-                    store_split3(r0, r0 + 8192, r0 + 16384, sw128_chunk(t, c8), x);
-                }
+                const int t = tid >> 3, c8 = tid & 7;
+                float x[8];
+                const float4 xa = *reinterpret_cast<const float4 *>(Tm + t * LDL + 8 * c8);
+                const float4 xb4 = *reinterpret_cast<const float4 *>(Tm + t * LDL + 8 * c8 + 4);
+                x[0] = xa.x; x[1] = xa.y; x[2] = xa.z; x[3] = xa.w;
+                x[4] = xb4.x; x[5] = xb4.y; x[6] = xb4.z; x[7] = xb4.w;
+                store_split3(r0, r0 + 8192, r0 + 16384, sw128_chunk(t, c8), x);
                 umma::fence_proxy_async();
             }
             __syncthreads();  // L / T are dead: the area takes the next chunk's K / Q
