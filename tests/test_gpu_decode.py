@@ -476,3 +476,48 @@ def test_per_layer_calls_equal_one_call_and_graph_replay(stq):
     assert status.item() == 0, stq.status_flags(status)
     assert torch.equal(pool_a, pool_c)
     assert torch.equal(o_a, torch.cat(o_l, dim=1))
+
+
+def test_more_heads_than_one_launch_table(stq, orc):
+    """3200 heads of one width in one call: the host splits the head table (3072 entries per
+    launch) for init, decode and dequantize. Sampled heads on both sides of the split match the
+    oracle, and every head stays finite."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    H, d, B = 3200, 128, 1
+    wl_ = _wl("layer48_b8_4bit", batch=B, heads=H, bits=4)
+    bits = [4] * H
+    lay = stq.Layout(bits, d)
+    w = wlm.impact_weights(wl_)
+    S0 = wlm.initial_state(wl_, 0)[None]
+    pool = lay.alloc_pool(B)
+    slots = torch.zeros(1, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stq.init_state(lay, pool, slots, S0.to(DEV), w.to(DEV), status=status)
+    sample = [0, 1, 3071, 3072, 3073, 3199]
+    offs, total = orc.request_layout(bits, d, d)
+    pre = {}
+    for h in sample:
+        blk = orc.quantize(4, as_f64(S0[0, h]), as_f64(w[h]))[0]
+        pre[h] = blk
+        pool[offs[h]: offs[h] + blk.size] = torch.from_numpy(blk).to(DEV)
+    inp = wlm.decode_inputs(wl_, 0)
+    o = torch.zeros(B, H, d, device=DEV)
+    g = {n: x.to(DEV) for n, x in inp.items()}
+    stq.decode_step(lay, pool, slots, g["q"], g["k"], g["v"], g["beta"], g["alpha"], w.to(DEV), o, status=status)
+    out = torch.zeros(B, H, d, d, device=DEV)
+    stq.dequantize(lay, pool, slots, out, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0, stq.status_flags(status)
+    assert torch.isfinite(o).all() and torch.isfinite(out).all()
+    gp = pool.cpu().numpy()
+    tally = Tally()
+    for h in sample:
+        res = orc.decode_step(4, 0, pre[h], as_f64(inp["q"][0, h]), as_f64(inp["k"][0, h]), as_f64(inp["v"][0, h]),
+                              float(inp["beta"][0, h]), float(inp["alpha"][0, h]), as_f64(w[h]), d, d)
+        got = gp[offs[h]: offs[h] + pre[h].size]
+        compare_block(orc, 4, d, got, res["block"], res["tie"], tally, f"head {h}")
+        compare_o(o[0, h].cpu().numpy(), res["o"], tally, f"o head {h}")
+        want = orc.dequantize(4, d, d, got)
+        assert np.all(np.abs(out[0, h].cpu().double().numpy() - want) <= 2.0 ** -23 * np.abs(want)), f"head {h}"
+    tally.check_budget()
