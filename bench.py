@@ -307,6 +307,45 @@ def per_layer_graph_leg(stq, lay, pool, slots, toks, w, status, dev, steps: int,
             "note": "one stq_decode_step per layer, a token's layers captured in one CUDA graph"}
 
 
+def init_dequant_leg(stq, wlm, wl, lay, w, dev, requests: int = 10, reps: int = 5) -> dict:
+    """stq_init_state and stq_dequantize over `requests` requests of the workload (all heads), timed
+    as whole calls with inputs resident in HBM. Algorithmic bytes: the fp32 states read (init) or
+    written (dequantize) plus the packed blocks written or read."""
+    import torch
+
+    H, d = wl.heads, wl.d
+    slots = torch.arange(requests, dtype=torch.int32, device=dev)
+    S0 = torch.stack([wlm.initial_state(wl, r, dev) for r in range(requests)])
+    out = torch.empty_like(S0)
+    pool = lay.alloc_pool(requests, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    packed = requests * sum(lay.head_bytes(h) for h in range(H))
+    dense = S0.numel() * 4
+    res = {}
+    for name, call in (("init", lambda: stq.init_state(lay, pool, slots, S0, w, status=status, stream=stream)),
+                       ("dequantize", lambda: stq.dequantize(lay, pool, slots, out, status=status, stream=stream))):
+        call()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / reps
+        gbs = (packed + dense) / (ms / 1e3) / 1e9
+        peak, kind = measured_peaks()
+        res[name] = {"ms_per_call": ms, "bytes_per_call": packed + dense, "achieved_gbs": gbs, "frac": gbs / peak,
+                     "peak_kind": kind}
+    if status.item() != 0:
+        raise RuntimeError(f"device status after the init/dequantize leg: {stq.status_flags(status)}")
+    del S0, out, pool
+    res["requests"] = requests
+    res["kernels"] = "init_kernel / dequant_kernel (one CTA per tile)"
+    return res
+
+
 def prefill_leg(dev, steps: int = 3, warmup: int = 1, T: int = 8192, fit_rounds: int = 0) -> dict:
     """The chunked-prefill workload (16 requests x 16 heads, 6-bit, an 8192-token prompt in 64-token
     chunks, bf16 inputs) timed as whole stq_prefill_chunk calls, inputs resident in HBM."""
@@ -467,6 +506,9 @@ def run_ours(args):
         if status.item() != 0:
             raise RuntimeError(f"device status after the per-layer graph leg: {stq.status_flags(status)}")
     pool.copy_(pristine)
+    init_leg = None
+    if world == 1:
+        init_leg = init_dequant_leg(stq, wlm, wl, lay, w, dev)
 
     # end to end through the public API with host buffers: every step copies its inputs from pinned
     # host memory and reads its readout back; copies run on their own streams (double-buffered
@@ -572,6 +614,8 @@ def run_ours(args):
     }
     if graph_leg is not None:
         result["per_layer_graph"] = graph_leg
+    if init_leg is not None:
+        result["init_dequantize"] = init_leg
     if lifetime:
         result["config"]["widths_from"] = "lifetime-aware allocation (stq_allocate_widths), same byte budget"
     if world == 1 and not args.no_prefill:

@@ -39,6 +39,10 @@ __device__ __forceinline__ TileRef tile_ref(const TileParams &p, int b, int pos)
     return t;
 }
 
+// (row, column) of flat element e of a dk x dv tile; dv is a power of two (16 .. 128)
+__device__ __forceinline__ int row_of(int e, int dv) { return e >> (__ffs(dv) - 1); }
+__device__ __forceinline__ int col_of(int e, int dv) { return e & (dv - 1); }
+
 // Code n (offset-binary) of a b-bit little-endian bitstream. Reads at most two bytes; the byte
 // after the last code is inside the block (scales follow the codes).
 __device__ __forceinline__ int read_code(const uint8_t *codes, int bits, int n)
@@ -57,20 +61,21 @@ __device__ void dequant_to_smem(const uint8_t *block, int bits, bool uniform, in
     const int n = dk * dv;
     if (bits == 16) {
         const __half *h = reinterpret_cast<const __half *>(block);
-        for (int e = threadIdx.x; e < n; e += blockDim.x) S[(e / dv) * ld + e % dv] = __half2float(h[e]);
+        for (int e = threadIdx.x; e < n; e += blockDim.x) S[row_of(e, dv) * ld + col_of(e, dv)] = __half2float(h[e]);
         return;
     }
     if (uniform) {
         const float su = *reinterpret_cast<const float *>(block + scale_offset(bits, dk, dv));
         const int off = 1 << (bits - 1);
         for (int e = threadIdx.x; e < n; e += blockDim.x)
-            S[(e / dv) * ld + e % dv] = su * (float)(read_code(block, bits, e) - off);
+            S[row_of(e, dv) * ld + col_of(e, dv)] = su * (float)(read_code(block, bits, e) - off);
         return;
     }
     const uint8_t *sc = block + scale_offset(bits, dk, dv);
     const int off = 1 << (bits - 1);
+    const int shv = __ffs(dv) - 1;  // dv is a power of two
     for (int e = threadIdx.x; e < n; e += blockDim.x) {
-        const int i = e / dv, j = e % dv;
+        const int i = e >> shv, j = e & (dv - 1);
         const float rc = load_scale(sc, i, sb16) * load_scale(sc, dk + j, sb16);
         S[i * ld + j] = rc * (float)(read_code(block, bits, e) - off);
     }
@@ -136,7 +141,7 @@ __device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, 
         __half *h = reinterpret_cast<__half *>(block);
         bool bad = false;
         for (int e = threadIdx.x; e < n; e += blockDim.x) {
-            const float x = S[(e / dv) * ld + e % dv];
+            const float x = S[row_of(e, dv) * ld + col_of(e, dv)];
             bad |= !(fabsf(x) < 65520.0f);  // overflows fp16 (or is NaN)
             h[e] = __float2half_rn(x);
         }
@@ -153,7 +158,7 @@ __device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, 
         float m = 0.f;
         bool bad = false;
         for (int e = threadIdx.x; e < n; e += blockDim.x) {
-            const float x = S[(e / dv) * ld + e % dv];
+            const float x = S[row_of(e, dv) * ld + col_of(e, dv)];
             m = fmaxf(m, fabsf(x));
             bad |= !isfinite(x);
         }
@@ -167,11 +172,13 @@ __device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, 
         const int cpg = bits == 4 ? 2 : (bits == 6 ? 4 : 1);
         const int bpg = bits == 6 ? 3 : 1;
         const int off = 1 << (bits - 1);
+        const float isu = __frcp_rn(su);
+        const int shv = __ffs(dv) - 1;
         for (int g = threadIdx.x; g < n / cpg; g += blockDim.x) {
             uint32_t word = 0;
             for (int t = 0; t < cpg; ++t) {
                 const int e = g * cpg + t;
-                const float xr = S[(e / dv) * ld + e % dv] / su;
+                const float xr = S[(e >> shv) * ld + (e & (dv - 1))] * isu;
                 const float x = isfinite(xr) ? fminf(fmaxf(rintf(xr), -qmax), qmax) : 0.f;  // rintf: half to even
                 word |= (uint32_t)((int)x + off) << (bits * t);
             }
@@ -194,9 +201,12 @@ __device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, 
     }
     __syncthreads();
     // row scales: largest column-normalised magnitude over qmax
+    __shared__ float ic1[128];
+    for (int j = threadIdx.x; j < dv; j += blockDim.x) ic1[j] = __frcp_rn(cs[j]);
+    __syncthreads();
     for (int i = threadIdx.x; i < dk; i += blockDim.x) {
         float m = 0.f;
-        for (int j = 0; j < dv; ++j) m = fmaxf(m, fabsf(S[i * ld + j] / cs[j]));
+        for (int j = 0; j < dv; ++j) m = fmaxf(m, fabsf(S[i * ld + j] * ic1[j]));
         float r = m / qmax;
         if (r == 0.f) r = 1.f;
         rs[i] = round_scale(r, sb16);
@@ -213,17 +223,24 @@ __device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, 
         store_scale(sg, dk + j, cs[j], sb16);
         bad |= !isfinite(cs[j]);
     }
+    // reciprocals of the stored scales (correctly rounded): x = S * (1/c) * (1/r) is within a few
+    // fp32 ulps of (S / c) / r, ~10^-4 of a code step at most, far inside the rounding-tie window
+    __shared__ float ics[128], irs[128];
+    for (int j = threadIdx.x; j < dv; j += blockDim.x) ics[j] = __frcp_rn(cs[j]);
+    for (int i = threadIdx.x; i < dk; i += blockDim.x) irs[i] = __frcp_rn(rs[i]);
+    __syncthreads();
     // codes, packed by groups of whole bytes: 2 codes/byte (4-bit), 4 codes/3 bytes (6-bit),
-    // 1 code/byte (8-bit)
+    // 1 code/byte (8-bit); dv is a power of two
     const int cpg = bits == 4 ? 2 : (bits == 6 ? 4 : 1);
     const int bpg = bits == 6 ? 3 : 1;
     const int off = 1 << (bits - 1);
+    const int shv = __ffs(dv) - 1;
     for (int g = threadIdx.x; g < n / cpg; g += blockDim.x) {
         uint32_t word = 0;
         for (int t = 0; t < cpg; ++t) {
             const int e = g * cpg + t;
-            const int i = e / dv, j = e % dv;
-            const float xr = (S[i * ld + j] / cs[j]) / rs[i];
+            const int i = e >> shv, j = e & (dv - 1);
+            const float xr = (S[i * ld + j] * ics[j]) * irs[i];
             const float x = isfinite(xr) ? fminf(fmaxf(rintf(xr), -qmax), qmax) : 0.f;  // rintf: half to even
             word |= (uint32_t)((int)x + off) << (bits * t);
         }
@@ -250,7 +267,8 @@ __global__ void __launch_bounds__(kThreads) init_kernel(const __grid_constant__ 
     float *cs = wv + dk;
     float *rs = cs + dv;
     const float *src = p.S0 + ((uint64_t)b * p.head_count + t.head) * dk * dv;
-    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) S[(e / dv) * ld + e % dv] = src[e];
+    const int shv = __ffs(dv) - 1;  // dv is a power of two
+    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) S[(e >> shv) * ld + (e & (dv - 1))] = src[e];
     for (int i = threadIdx.x; i < dk; i += blockDim.x) wv[i] = p.w[(uint64_t)t.head * dk + i];
     __syncthreads();
     quantize_from_smem(S, ld, wv, t.bits, t.uniform, t.sb16, t.rounds, dk, dv, t.block, cs, rs, p.status);
@@ -317,7 +335,7 @@ __global__ void __launch_bounds__(kThreads) decode_generic_kernel(const __grid_c
     __syncthreads();
     // S' = alpha (S - beta k u^T) + beta k v^T   (decay-first: alpha S - beta k u^T + beta k v^T)
     for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
-        const int i = e / dv, j = e % dv;
+        const int i = row_of(e, dv), j = col_of(e, dv);
         const float s = S[i * ld + j];
         S[i * ld + j] = decay_first ? av[i] * s - beta * kv[i] * uv[j] + beta * kv[i] * vv[j]
                                     : av[i] * (s - beta * kv[i] * uv[j]) + beta * kv[i] * vv[j];
@@ -382,7 +400,7 @@ __global__ void __launch_bounds__(kThreads) prefill_seq_kernel(const __grid_cons
         }
         __syncthreads();
         for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
-            const int i = e / dv, j = e % dv;
+            const int i = row_of(e, dv), j = col_of(e, dv);
             const float s = S[i * ld + j];
             S[i * ld + j] = decay_first ? av[i] * s - beta * kv[i] * uv[j] + beta * kv[i] * vv[j]
                                         : av[i] * (s - beta * kv[i] * uv[j]) + beta * kv[i] * vv[j];
