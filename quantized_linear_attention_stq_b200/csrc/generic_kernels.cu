@@ -53,6 +53,43 @@ __device__ __forceinline__ int read_code(const uint8_t *codes, int bits, int n)
     return (int)(((lo | (hi << 8)) >> (bit & 7)) & ((1u << bits) - 1u));
 }
 
+// Pack the offset-binary codes of a dk x dv tile into `block` with whole 32-bit stores: a thread
+// takes a group of codes that fills whole words (8 x 4-bit, 16 x 6-bit = 3 words, 4 x 8-bit), so
+// every group starts 4-byte aligned. code(e) returns the signed code of flat element e.
+template <int BITS, typename CodeOf>
+__device__ __forceinline__ void pack_codes_words(uint8_t *block, int n, CodeOf code)
+{
+    constexpr int CW = BITS == 6 ? 16 : 32 / BITS;  // codes per group
+    constexpr int WW = BITS == 6 ? 3 : 1;           // words per group
+    constexpr int OFF = 1 << (BITS - 1);
+    uint32_t *out = reinterpret_cast<uint32_t *>(block);
+    for (int g = threadIdx.x; g < n / CW; g += blockDim.x) {
+        uint32_t w[WW];
+#pragma unroll
+        for (int k = 0; k < WW; ++k) w[k] = 0u;
+#pragma unroll
+        for (int t = 0; t < CW; ++t) {
+            const uint32_t u = (uint32_t)(code(g * CW + t) + OFF);
+            const int bit = BITS * t;
+            w[bit >> 5] |= u << (bit & 31);
+            if ((bit & 31) + BITS > 32) w[(bit >> 5) + 1] |= u >> (32 - (bit & 31));
+        }
+#pragma unroll
+        for (int k = 0; k < WW; ++k) out[g * WW + k] = w[k];
+    }
+}
+
+template <typename CodeOf>
+__device__ __forceinline__ void pack_codes(uint8_t *block, int bits, int n, CodeOf code)
+{
+    if (bits == 4)
+        pack_codes_words<4>(block, n, code);
+    else if (bits == 6)
+        pack_codes_words<6>(block, n, code);
+    else
+        pack_codes_words<8>(block, n, code);
+}
+
 // Dequantize a tile from global memory into S (row stride ld): S_ij = fp32(r_i c_j) * Q_ij, or
 // S_ij = s * Q_ij for a uniformly scaled head.
 __device__ void dequant_to_smem(const uint8_t *block, int bits, bool uniform, int sb16, int dk, int dv, float *S,
@@ -169,21 +206,12 @@ __device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, 
         if (su == 0.f) su = 1.f;
         bad |= !isfinite(su);
         if (threadIdx.x == 0) *reinterpret_cast<float *>(block + scale_offset(bits, dk, dv)) = su;
-        const int cpg = bits == 4 ? 2 : (bits == 6 ? 4 : 1);
-        const int bpg = bits == 6 ? 3 : 1;
-        const int off = 1 << (bits - 1);
         const float isu = __frcp_rn(su);
         const int shv = __ffs(dv) - 1;
-        for (int g = threadIdx.x; g < n / cpg; g += blockDim.x) {
-            uint32_t word = 0;
-            for (int t = 0; t < cpg; ++t) {
-                const int e = g * cpg + t;
-                const float xr = S[(e >> shv) * ld + (e & (dv - 1))] * isu;
-                const float x = isfinite(xr) ? fminf(fmaxf(rintf(xr), -qmax), qmax) : 0.f;  // rintf: half to even
-                word |= (uint32_t)((int)x + off) << (bits * t);
-            }
-            for (int t = 0; t < bpg; ++t) block[g * bpg + t] = (uint8_t)(word >> (8 * t));
-        }
+        pack_codes(block, bits, n, [&](int e) {
+            const float xr = S[(e >> shv) * ld + (e & (dv - 1))] * isu;
+            return (int)(isfinite(xr) ? fminf(fmaxf(rintf(xr), -qmax), qmax) : 0.f);  // rintf: half to even
+        });
         if (__syncthreads_or(bad) && threadIdx.x == 0) flag(status, kFlagNonfinite);
         return;
     }
@@ -229,23 +257,13 @@ __device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, 
     for (int j = threadIdx.x; j < dv; j += blockDim.x) ics[j] = __frcp_rn(cs[j]);
     for (int i = threadIdx.x; i < dk; i += blockDim.x) irs[i] = __frcp_rn(rs[i]);
     __syncthreads();
-    // codes, packed by groups of whole bytes: 2 codes/byte (4-bit), 4 codes/3 bytes (6-bit),
-    // 1 code/byte (8-bit); dv is a power of two
-    const int cpg = bits == 4 ? 2 : (bits == 6 ? 4 : 1);
-    const int bpg = bits == 6 ? 3 : 1;
-    const int off = 1 << (bits - 1);
+    // codes: whole 32-bit words per thread (pack_codes)
     const int shv = __ffs(dv) - 1;
-    for (int g = threadIdx.x; g < n / cpg; g += blockDim.x) {
-        uint32_t word = 0;
-        for (int t = 0; t < cpg; ++t) {
-            const int e = g * cpg + t;
-            const int i = e >> shv, j = e & (dv - 1);
-            const float xr = (S[i * ld + j] * ics[j]) * irs[i];
-            const float x = isfinite(xr) ? fminf(fmaxf(rintf(xr), -qmax), qmax) : 0.f;  // rintf: half to even
-            word |= (uint32_t)((int)x + off) << (bits * t);
-        }
-        for (int t = 0; t < bpg; ++t) block[g * bpg + t] = (uint8_t)(word >> (8 * t));
-    }
+    pack_codes(block, bits, n, [&](int e) {
+        const int i = e >> shv, j = e & (dv - 1);
+        const float xr = (S[i * ld + j] * ics[j]) * irs[i];
+        return (int)(isfinite(xr) ? fminf(fmaxf(rintf(xr), -qmax), qmax) : 0.f);  // rintf: half to even
+    });
     if (__syncthreads_or(bad) && threadIdx.x == 0) flag(status, kFlagNonfinite);
 }
 
