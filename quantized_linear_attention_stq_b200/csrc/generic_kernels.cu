@@ -305,7 +305,43 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const __grid_constant
     }
     const int dk = p.dk, dv = p.dv;
     float *dst = p.S_out + ((uint64_t)b * p.head_count + t.head) * dk * dv;
-    dequant_to_smem(t.block, t.bits, t.uniform, t.sb16, dk, dv, dst, dv);  // writes straight to global, row stride dv
+    if (t.bits == 16 || t.uniform || (reinterpret_cast<uintptr_t>(dst) & 15u) != 0) {
+        dequant_to_smem(t.block, t.bits, t.uniform, t.sb16, dk, dv, dst, dv);  // straight to global, row stride dv
+        return;
+    }
+    // row x column codes, 8 consecutive elements of a row per thread: the group's bits * 8 code
+    // bits are `bits` bytes at byte offset bits * g, unpacked at once; S_ij = fp32(r_i c_j) Q_ij
+    const uint8_t *sc = t.block + scale_offset(t.bits, dk, dv);
+    const int shv = __ffs(dv) - 1, bits = t.bits, off = 1 << (bits - 1);
+    const uint32_t mask = (1u << bits) - 1u;
+    for (int g = threadIdx.x; g < dk * dv / 8; g += blockDim.x) {
+        const int e0 = 8 * g, i = e0 >> shv, j0 = e0 & (dv - 1);
+        uint32_t lo, hi;
+        if (bits == 8) {
+            const uint2 wd = *reinterpret_cast<const uint2 *>(t.block + 8 * g);
+            lo = wd.x;
+            hi = wd.y;
+        } else if (bits == 4) {
+            lo = *reinterpret_cast<const uint32_t *>(t.block + 4 * g);
+            hi = 0u;
+        } else {  // 6 bytes at 6g, 2-byte aligned
+            const uint16_t *h = reinterpret_cast<const uint16_t *>(t.block + 6 * g);
+            lo = (uint32_t)h[0] | ((uint32_t)h[1] << 16);
+            hi = h[2];
+        }
+        const float r = load_scale(sc, i, t.sb16);
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int bit = bits * k;  // position in the 64-bit (hi:lo) group
+            const uint32_t u = (bit < 32 ? (bit + bits <= 32 ? lo >> bit : __funnelshift_r(lo, hi, bit))
+                                         : hi >> (bit - 32)) & mask;
+            v[k] = (r * load_scale(sc, dk + j0 + k, t.sb16)) * (float)((int)u - off);
+        }
+        float4 *o4 = reinterpret_cast<float4 *>(dst + e0);
+        o4[0] = make_float4(v[0], v[1], v[2], v[3]);
+        o4[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
 }
 
 // ------------------------------------------------------------------------------------------
