@@ -33,6 +33,7 @@ DEFAULT_WORKLOAD = "full2304_b70_mixed"
 LIFETIME_WORKLOAD = "full2304_b70_lifetime"  # same workload, lifetime-aware widths
 TOKENS_CYCLED = 8
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 DECODE_SOURCES = ("quantized_linear_attention_stq_b200/csrc/decode_d128.cu",
                   "quantized_linear_attention_stq_b200/csrc/stq_internal.cuh")
 TRAFFIC_FILE = "profiles/decode_d128_full2304_b70.md"
@@ -82,6 +83,21 @@ def measured_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "of measured"
     return FALLBACK_HBM_GBS, "of fallback"
+
+
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s of a kernel timed alone (the burst figure)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "of measured"
+    return FALLBACK_BF16_TFLOPS, "of fallback"
+
+
+# Dense contractions of one 64-token chunk of one 128 x 128 head in the UT form, as multiply-adds
+# x 2: [K;Q]K^T (128 x 64 x 128), [K;Q] S0 (128 x 128 x 128), T R' and P U (64 x 128 x 64 each),
+# K^T U (128 x 128 x 64). The bf16 operand splits make the tensor cores issue about four times this.
+PREFILL_FLOPS_PER_CHUNK_HEAD = 2 * (128 * 64 * 128 + 128 * 128 * 128 + 2 * 64 * 128 * 64 + 128 * 128 * 64)
 
 
 def decode_source_hash() -> str:
@@ -391,13 +407,19 @@ def prefill_leg(dev, steps: int = 3, warmup: int = 1, T: int = 8192, fit_rounds:
     nbytes = in_bytes + out_bytes + state_bytes
     peak, kind = measured_peaks()
     achieved = nbytes / (ms / 1e3) / 1e9
+    flops = B * H * (T // C) * PREFILL_FLOPS_PER_CHUNK_HEAD
+    tpeak, tkind = measured_tensor_peak()
+    tflops = flops / (ms / 1e3) / 1e12
     del inp, o, pool
     return {"workload": "prefill16_b16_6bit", "prompt_tokens": T, "chunk": C, "requests": B, "heads": H,
             "ms_per_call": ms, "head_tokens_per_s": B * H * T / (ms / 1e3), "tokens_per_s": B * T / (ms / 1e3),
             "calls": steps, "fit_rounds": fit_rounds,
             "kernel": "prefill_wy_kernel<6> (tcgen05, one launch)" if fit_rounds <= 1 else "prefill_seq_kernel",
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                         "peak_kind": kind, "bytes_per_call": nbytes}}
+                         "peak_kind": kind, "bytes_per_call": nbytes},
+            "tensor_roofline": {"bound": "tensor", "achieved": tflops, "peak": tpeak, "unit": "TFLOP/s",
+                                "frac": tflops / tpeak, "peak_kind": tkind, "flops_per_call": flops,
+                                "note": "algorithmic FLOPs of the five dense contractions per chunk and head"}}
 
 
 def run_ours(args):

@@ -215,26 +215,61 @@ __device__ void quantize_from_smem(float *S, int ld, const float *wv, int bits, 
         if (__syncthreads_or(bad) && threadIdx.x == 0) flag(status, kFlagNonfinite);
         return;
     }
-    // column scales: impact-weighted RMS over the key rows
-    for (int j = threadIdx.x; j < dv; j += blockDim.x) {
-        float W = 0.f, E = 0.f;
-        for (int i = 0; i < dk; ++i) {
-            const float x = S[i * ld + j];
-            W += wv[i];
-            E += wv[i] * x * x;
+    // column scales: impact-weighted RMS over the key rows. Every thread takes one column and
+    // every P-th row of it (P = threads / dv row classes, two running sums each); the partials are
+    // added per column after a barrier. W = sum_i w_i is the same for every column.
+    __shared__ float part[kThreads], wsum;
+    {
+        const int P = (int)blockDim.x / dv, j = (int)threadIdx.x % dv, cls = (int)threadIdx.x / dv;
+        float E0 = 0.f, E1 = 0.f;
+        int i = cls;
+        for (; i + P < dk; i += 2 * P) {
+            const float x0 = S[i * ld + j], x1 = S[(i + P) * ld + j];
+            E0 += wv[i] * x0 * x0;
+            E1 += wv[i + P] * x1 * x1;
         }
-        float c = sqrtf(E / W);
-        if (c == 0.f) c = 1.f;
-        cs[j] = round_scale(c, sb16);  // the codes use the stored value
+        if (i < dk) {
+            const float x0 = S[i * ld + j];
+            E0 += wv[i] * x0 * x0;
+        }
+        part[threadIdx.x] = E0 + E1;
+        if (threadIdx.x < 32) {
+            float W = 0.f;
+            for (int r = (int)threadIdx.x; r < dk; r += 32) W += wv[r];
+            for (int sh = 16; sh > 0; sh >>= 1) W += __shfl_xor_sync(0xffffffffu, W, sh);
+            if (threadIdx.x == 0) wsum = W;
+        }
     }
     __syncthreads();
-    // row scales: largest column-normalised magnitude over qmax
     __shared__ float ic1[128];
-    for (int j = threadIdx.x; j < dv; j += blockDim.x) ic1[j] = __frcp_rn(cs[j]);
+    for (int j = threadIdx.x; j < dv; j += blockDim.x) {
+        const int P = (int)blockDim.x / dv;
+        float E = 0.f;
+        for (int c = 0; c < P; ++c) E += part[c * dv + j];
+        float c = sqrtf(E / wsum);
+        if (c == 0.f) c = 1.f;
+        cs[j] = round_scale(c, sb16);  // the codes use the stored value
+        ic1[j] = __frcp_rn(cs[j]);
+    }
+    __syncthreads();
+    // row scales: largest column-normalised magnitude over qmax. Every thread takes one row and
+    // every P-th column of it; the partial maxima meet after a barrier (max is exact in any order).
+    {
+        const int P = (int)blockDim.x / dk, i = (int)threadIdx.x % dk, cls = (int)threadIdx.x / dk;
+        float m0 = 0.f, m1 = 0.f;
+        int j = cls;
+        for (; j + P < dv; j += 2 * P) {
+            m0 = fmaxf(m0, fabsf(S[i * ld + j] * ic1[j]));
+            m1 = fmaxf(m1, fabsf(S[i * ld + j + P] * ic1[j + P]));
+        }
+        if (j < dv) m0 = fmaxf(m0, fabsf(S[i * ld + j] * ic1[j]));
+        part[threadIdx.x] = fmaxf(m0, m1);
+    }
     __syncthreads();
     for (int i = threadIdx.x; i < dk; i += blockDim.x) {
+        const int P = (int)blockDim.x / dk;
         float m = 0.f;
-        for (int j = 0; j < dv; ++j) m = fmaxf(m, fabsf(S[i * ld + j] * ic1[j]));
+        for (int c = 0; c < P; ++c) m = fmaxf(m, part[c * dk + i]);
         float r = m / qmax;
         if (r == 0.f) r = 1.f;
         rs[i] = round_scale(r, sb16);
@@ -285,9 +320,43 @@ __global__ void __launch_bounds__(kThreads) init_kernel(const __grid_constant__ 
     float *cs = wv + dk;
     float *rs = cs + dv;
     const float *src = p.S0 + ((uint64_t)b * p.head_count + t.head) * dk * dv;
-    const int shv = __ffs(dv) - 1;  // dv is a power of two
-    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) S[(e >> shv) * ld + (e & (dv - 1))] = src[e];
     for (int i = threadIdx.x; i < dk; i += blockDim.x) wv[i] = p.w[(uint64_t)t.head * dk + i];
+    if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0 && dv >= 32) {
+        // 16-byte loads, 8 in flight per thread. Lane l of a warp takes chunk (l % 8) of row (l / 8)
+        // of a 4-row x 8-chunk block: rows are read 128 contiguous bytes at a time, and the scalar
+        // stores into the (dv + 1)-float rows fall on 32 different banks.
+        constexpr int U = 8;
+        const int cpr = dv / 4, gpr = cpr / 8, n4 = dk * cpr;
+        const float4 *s4 = reinterpret_cast<const float4 *>(src);
+        for (int base = threadIdx.x; base < n4; base += U * blockDim.x) {
+            float4 v[U];
+            int at[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int g = base + u * (int)blockDim.x;
+                at[u] = -1;
+                if (g < n4) {
+                    const int wg = g >> 5, l = g & 31;
+                    const int i = 4 * (wg / gpr) + (l >> 3), q = 8 * (wg % gpr) + (l & 7);
+                    v[u] = s4[i * cpr + q];
+                    at[u] = i * ld + 4 * q;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (at[u] >= 0) {
+                    float *d = S + at[u];
+                    d[0] = v[u].x;
+                    d[1] = v[u].y;
+                    d[2] = v[u].z;
+                    d[3] = v[u].w;
+                }
+            }
+        }
+    } else {
+        const int shv = __ffs(dv) - 1;  // dv is a power of two
+        for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) S[(e >> shv) * ld + (e & (dv - 1))] = src[e];
+    }
     __syncthreads();
     quantize_from_smem(S, ld, wv, t.bits, t.uniform, t.sb16, t.rounds, dk, dv, t.block, cs, rs, p.status);
 }
