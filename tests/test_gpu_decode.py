@@ -158,8 +158,10 @@ def test_many_requests_split_launches(stq, orc):
 # init and dequantize
 # ------------------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("d", [16, 128])
-def test_init_matches_oracle(stq, orc, d):
+@pytest.mark.parametrize("d,aligned", [(16, True), (32, True), (64, True), (128, True), (128, False), (32, False)])
+def test_init_matches_oracle(stq, orc, d, aligned):
+    """Init at every head size. The states reach the kernel 16-byte aligned (staged by 16-byte
+    loads for d >= 32), or one float past a 16-byte boundary (staged element by element)."""
     from quantized_linear_attention_stq_b200 import workloads as wlm
 
     wl_ = _wl("full2304_b70_mixed", batch=3, heads=8, d=d)
@@ -171,7 +173,15 @@ def test_init_matches_oracle(stq, orc, d):
     pool = lay.alloc_pool(3)
     slots = torch.arange(3, dtype=torch.int32, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
-    stq.init_state(lay, pool, slots, S0.to(DEV), w.to(DEV), status=status)
+    if aligned:
+        S0_dev = S0.to(DEV)
+        assert S0_dev.data_ptr() % 16 == 0
+    else:
+        flat = torch.zeros(S0.numel() + 1, device=DEV)
+        S0_dev = flat[1:].view(S0.shape)
+        S0_dev.copy_(S0.to(DEV))
+        assert S0_dev.data_ptr() % 16 == 4
+    stq.init_state(lay, pool, slots, S0_dev, w.to(DEV), status=status)
     torch.cuda.synchronize()
     assert status.item() == 0
     gp = pool.cpu().numpy()
