@@ -11,6 +11,11 @@
 #include "../../include/stq.h"
 #include "stq_internal.cuh"
 
+namespace stq {
+// Persistent streaming init of 128 x 128 row x column heads (init_d128.cu).
+cudaError_t launch_init_d128(const TileParams &p, cudaStream_t s);
+}  // namespace stq
+
 struct stq_layout {
     int32_t H, dk, dv, gate, in_dtype;
     bool uniform;  // STQ_SCALES_UNIFORM
@@ -162,12 +167,24 @@ stq_status stq_init_state(const stq_layout *L, void *pool, int32_t pool_slots, c
     p->S0 = S0;
     p->w = w;
     const std::vector<int> ord = order_by_size(L, 0, L->H);
-    for (int first = 0; first < L->H; first += stq::kMaxTable) {
-        const int n = std::min(stq::kMaxTable, L->H - first);
-        fill_table(*p, L, ord, first, n, 0);
-        p->ntiles = B * n;
-        const stq_status st = from_cuda(stq::launch_init_generic(*p, (cudaStream_t)stream));
-        if (st != STQ_OK) return st;
+    // 128 x 128 row x column heads without refinement rounds go to the persistent streaming
+    // kernel when S0 and w allow 16-byte copies; FP16 pivots and everything else to the plain one
+    const bool streamed = L->dk == 128 && L->dv == 128 && !L->uniform && L->fit_rounds == 0 && aligned(S0, 16) &&
+                          aligned(w, 16);
+    std::vector<int> plain, tuned;
+    for (int h : ord) (streamed && L->bits[h] != 16 ? tuned : plain).push_back(h);
+    for (int pass = 0; pass < 2; ++pass) {
+        const std::vector<int> &heads = pass == 0 ? plain : tuned;
+        const int nh = (int)heads.size();
+        for (int first = 0; first < nh; first += stq::kMaxTable) {
+            const int n = std::min(stq::kMaxTable, nh - first);
+            fill_table(*p, L, heads, first, n, 0);
+            p->ntiles = B * n;
+            const cudaError_t e = pass == 0 ? stq::launch_init_generic(*p, (cudaStream_t)stream)
+                                            : stq::launch_init_d128(*p, (cudaStream_t)stream);
+            const stq_status st = from_cuda(e);
+            if (st != STQ_OK) return st;
+        }
     }
     return STQ_OK;
 }
