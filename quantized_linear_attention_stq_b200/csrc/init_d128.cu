@@ -1,9 +1,9 @@
 // init_d128.cu -- initial quantization (stq_init_state) of 128 x 128 heads with row x column
 // scales. A persistent kernel, one 512-thread CTA per SM, streams whole fp32 tiles through a
-// two-slot shared-memory ring, one bulk copy per tile. A tile is first moved into a work tile
-// whose rows are padded to 132 floats (every later pass reads it without bank conflicts), which
-// frees its ring slot for the tile after next: two tiles are in flight while the current one is
-// fitted, coded and stored.
+// two-slot shared-memory ring, one bulk copy per tile. The first pass over a tile (its column
+// energies) also moves it into a work tile whose rows are padded to 132 floats, where every later
+// pass reads it without bank conflicts; that frees its ring slot for the tile after next, so two
+// tiles are in flight while the current one is fitted, coded and stored.
 //
 // Method: the column scale is the impact-weighted RMS of the column over the key rows, the row
 // scale the largest column-normalised magnitude of the row over qmax, the codes S / (r c) rounded
@@ -25,7 +25,7 @@ constexpr int NSI = 2;                                 // ring slots
 constexpr uint32_t TILE_BYTES = DI * DI * 4;           // one fp32 tile of S0
 constexpr uint32_t SLOT_BYTES = TILE_BYTES + DI * 4;   // + the head's impact weights
 constexpr uint32_t TX_BYTES = SLOT_BYTES;              // bytes a slot's copies complete
-constexpr uint32_t WORK_BYTES = DI * LDI * 4 + DI * 4; // the padded work tile + weights
+constexpr uint32_t WORK_BYTES = DI * LDI * 4;          // the padded work tile
 
 // The float arrays are read as float4: each starts 16-byte aligned.
 struct InitFixed {
@@ -118,16 +118,16 @@ __device__ __forceinline__ void store_group(uint8_t *dst, int bits, const uint32
     }
 }
 
-// Fit, code and store one tile held in shared memory (rows of LDI floats; wv = the head's
-// weights). Returns whether a stored scale is non-finite (or a row scale zero).
-__device__ __forceinline__ bool quantize_tile(InitFixed &sm, const float *S, const float *wv, uint8_t *gblock,
-                                              int bits, int sb16)
+// Phase 1 of a tile: move it from its ring slot (raw: 128 x 128 floats, then the head's
+// weights) into the padded work tile S, and form the partial column energies and the weight sum.
+// The caller's barrier after it frees the ring slot.
+__device__ __forceinline__ void energies(InitFixed &sm, const float *raw, float *S)
 {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const float qmax = (float)((1 << (bits - 1)) - 1);
+    const float *wv = raw + DI * DI;
     if (tid == 0) sm.slow = 0;
-    // ---- column energies: columns 4 (tid % 32) .. +3 over rows 8 (tid / 32) .. +7, as w_i x x
-    // in packed pairs; the 16 partials of a column are added after a barrier
+    // columns 4 (tid % 32) .. +3 over rows 8 (tid / 32) .. +7, as w_i x x in packed pairs; the 16
+    // partials of a column are added after the barrier
     {
         const int jq = tid & 31, rb = tid >> 5;
         const float4 wa = *reinterpret_cast<const float4 *>(wv + 8 * rb);
@@ -136,7 +136,9 @@ __device__ __forceinline__ bool quantize_tile(InitFixed &sm, const float *S, con
         float2 e01 = make_float2(0.f, 0.f), e23 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
-            const float4 x = *reinterpret_cast<const float4 *>(S + (8 * rb + r) * LDI + 4 * jq);
+            const int i = 8 * rb + r;
+            const float4 x = *reinterpret_cast<const float4 *>(raw + i * DI + 4 * jq);
+            *reinterpret_cast<float4 *>(S + i * LDI + 4 * jq) = x;
             const float2 ww = make_float2(wr[r], wr[r]);
             const float2 x01 = make_float2(x.x, x.y), x23 = make_float2(x.z, x.w);
             e01 = __ffma2_rn(__fmul2_rn(ww, x01), x01, e01);
@@ -150,7 +152,14 @@ __device__ __forceinline__ bool quantize_tile(InitFixed &sm, const float *S, con
             if (lane == 0) sm.wsum = W;
         }
     }
-    __syncthreads();
+}
+
+// The rest of a tile (in the padded work tile S, after the energies and a barrier): scales,
+// codes and stores. Returns whether a stored scale is non-finite (or a row scale zero).
+__device__ __forceinline__ bool quantize_tile(InitFixed &sm, const float *S, uint8_t *gblock, int bits, int sb16)
+{
+    const int tid = threadIdx.x;
+    const float qmax = (float)((1 << (bits - 1)) - 1);
     bool nf = false;  // a non-finite stored scale (or a zero row scale) met by this thread
     if (tid < DI) {
         float a[8];
@@ -286,19 +295,11 @@ __global__ void __launch_bounds__(NTI, 1) init_d128_kernel(const __grid_constant
         }
         const unsigned long long gb = sm.gblock[si];
         const int bits = sm.bits[si];
-        if (gb != 0ull) {
-            // into the padded work tile: float4 f of the tile is chunk f % 32 of row f / 32 (the
-            // eight lanes of a store phase write eight consecutive chunks of one row)
-            const float4 *raw = reinterpret_cast<const float4 *>(smem + RING_OFF + (uint32_t)si * SLOT_BYTES);
-            float4 *w4 = reinterpret_cast<float4 *>(work);
-#pragma unroll
-            for (int f = tid; f < DI * DI / 4; f += NTI) w4[(f >> 5) * (LDI / 4) + (f & 31)] = raw[f];
-            if (tid < DI / 4) w4[DI * LDI / 4 + tid] = raw[DI * DI / 4 + tid];
-        }
+        if (gb != 0ull) energies(sm, reinterpret_cast<const float *>(smem + RING_OFF + (uint32_t)si * SLOT_BYTES), work);
         __syncthreads();  // the ring slot is free: it takes the tile after next
         if (tid == 0) issue_tile(p, sm, smem, k + NSI, my_count, next);
         bool bad = false;
-        if (gb != 0ull) bad = quantize_tile(sm, work, work + DI * LDI, reinterpret_cast<uint8_t *>(gb), bits, p.scale_bf16);
+        if (gb != 0ull) bad = quantize_tile(sm, work, reinterpret_cast<uint8_t *>(gb), bits, p.scale_bf16);
         if (bad && tid == 0) flag(p.status, kFlagNonfinite);
         __syncthreads();  // every thread is done with the work tile and the per-tile scratch
     }
