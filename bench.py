@@ -358,7 +358,8 @@ def init_dequant_leg(stq, wlm, wl, lay, w, dev, requests: int = 10, reps: int = 
         raise RuntimeError(f"device status after the init/dequantize leg: {stq.status_flags(status)}")
     del S0, out, pool
     res["requests"] = requests
-    res["kernels"] = "init_kernel / dequant_kernel (one CTA per tile)"
+    res["kernels"] = ("init_d128_kernel (persistent, streaming; pivot heads: init_kernel) / "
+                      "dequant_kernel (one CTA per tile)")
     return res
 
 
