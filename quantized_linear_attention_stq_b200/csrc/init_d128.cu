@@ -94,16 +94,17 @@ __device__ __forceinline__ void issue_tile(const TileParams &p, InitFixed &sm, u
 
 // Pack 16 offset-binary codes (u < 2^bits) into 2 * bits bytes at dst: code k at bits
 // bits * k .. of a little-endian bitstream.
-__device__ __forceinline__ void store_group(uint8_t *dst, int bits, const uint32_t (&u)[16])
+template <int BITS>
+__device__ __forceinline__ void store_group(uint8_t *dst, const uint32_t (&u)[16])
 {
-    if (bits == 4) {
+    if constexpr (BITS == 4) {
         uint2 w;
         w.x = u[0] | (u[1] << 4) | (u[2] << 8) | (u[3] << 12) | (u[4] << 16) | (u[5] << 20) | (u[6] << 24) |
               (u[7] << 28);
         w.y = u[8] | (u[9] << 4) | (u[10] << 8) | (u[11] << 12) | (u[12] << 16) | (u[13] << 20) | (u[14] << 24) |
               (u[15] << 28);
         *reinterpret_cast<uint2 *>(dst) = w;
-    } else if (bits == 6) {
+    } else if constexpr (BITS == 6) {
         uint32_t *d32 = reinterpret_cast<uint32_t *>(dst);
         d32[0] = u[0] | (u[1] << 6) | (u[2] << 12) | (u[3] << 18) | (u[4] << 24) | (u[5] << 30);
         d32[1] = (u[5] >> 2) | (u[6] << 4) | (u[7] << 10) | (u[8] << 16) | (u[9] << 22) | (u[10] << 28);
@@ -156,10 +157,12 @@ __device__ __forceinline__ void energies(InitFixed &sm, const float *raw, float 
 
 // The rest of a tile (in the padded work tile S, after the energies and a barrier): scales,
 // codes and stores. Returns whether a stored scale is non-finite (or a row scale zero).
-__device__ __forceinline__ bool quantize_tile(InitFixed &sm, const float *S, uint8_t *gblock, int bits, int sb16)
+template <int BITS, int SB16>
+__device__ __forceinline__ bool quantize_tile(InitFixed &sm, const float *S, uint8_t *gblock)
 {
+    constexpr int bits = BITS, sb16 = SB16;
     const int tid = threadIdx.x;
-    const float qmax = (float)((1 << (bits - 1)) - 1);
+    constexpr float qmax = (float)((1 << (BITS - 1)) - 1);
     bool nf = false;  // a non-finite stored scale (or a zero row scale) met by this thread
     if (tid < DI) {
         float a[8];
@@ -210,8 +213,8 @@ __device__ __forceinline__ bool quantize_tile(InitFixed &sm, const float *S, uin
     const bool fast = !bad && sm.slow == 0;
     // ---- codes: 16 consecutive elements of row i = g % 128 (columns 16 (g / 128) ..) per group g;
     // x = (S * (1/c)) * (1/r) with the correctly rounded reciprocals, rounded half to even
-    const int off = 1 << (bits - 1);
-    const uint32_t mask = (1u << bits) - 1u;
+    constexpr int off = 1 << (BITS - 1);
+    constexpr uint32_t mask = (1u << BITS) - 1u;
 #pragma unroll 1
     for (int g = tid; g < DI * DI / 16; g += NTI) {
         const int i = g & (DI - 1), cg = g >> 7;
@@ -230,7 +233,7 @@ __device__ __forceinline__ bool quantize_tile(InitFixed &sm, const float *S, uin
                 const float4 x = row[k], c = ic[k];
                 float2 y01 = __fmul2_rn(__fmul2_rn(make_float2(x.x, x.y), make_float2(c.x, c.y)), ir2);
                 float2 y23 = __fmul2_rn(__fmul2_rn(make_float2(x.z, x.w), make_float2(c.z, c.w)), ir2);
-                if (sb16) {
+                if constexpr (SB16 != 0) {
                     y01 = make_float2(fminf(fmaxf(y01.x, -qmax), qmax), fminf(fmaxf(y01.y, -qmax), qmax));
                     y23 = make_float2(fminf(fmaxf(y23.x, -qmax), qmax), fminf(fmaxf(y23.y, -qmax), qmax));
                 }
@@ -256,7 +259,7 @@ __device__ __forceinline__ bool quantize_tile(InitFixed &sm, const float *S, uin
             }
         }
         // the group's 16 codes are 2 * bits bytes at byte 2 * bits * (8 i + cg) of the bitstream
-        store_group(gblock + 2 * bits * (8 * i + cg), bits, u);
+        store_group<BITS>(gblock + 2 * BITS * (8 * i + cg), u);
     }
     if (tid < DI) {
         uint8_t *sg = gblock + scale_offset(bits, DI, DI);
@@ -299,7 +302,17 @@ __global__ void __launch_bounds__(NTI, 1) init_d128_kernel(const __grid_constant
         __syncthreads();  // the ring slot is free: it takes the tile after next
         if (tid == 0) issue_tile(p, sm, smem, k + NSI, my_count, next);
         bool bad = false;
-        if (gb != 0ull) bad = quantize_tile(sm, work, reinterpret_cast<uint8_t *>(gb), bits, p.scale_bf16);
+        if (gb != 0ull) {
+            uint8_t *g = reinterpret_cast<uint8_t *>(gb);
+            switch (2 * bits + (p.scale_bf16 ? 1 : 0)) {
+            case 8: bad = quantize_tile<4, 0>(sm, work, g); break;
+            case 9: bad = quantize_tile<4, 1>(sm, work, g); break;
+            case 12: bad = quantize_tile<6, 0>(sm, work, g); break;
+            case 13: bad = quantize_tile<6, 1>(sm, work, g); break;
+            case 16: bad = quantize_tile<8, 0>(sm, work, g); break;
+            default: bad = quantize_tile<8, 1>(sm, work, g); break;
+            }
+        }
         if (bad && tid == 0) flag(p.status, kFlagNonfinite);
         __syncthreads();  // every thread is done with the work tile and the per-tile scratch
     }
