@@ -194,6 +194,102 @@ def test_init_matches_oracle(stq, orc, d, aligned):
     tally.check_budget()
 
 
+def _init_two_ways(stq, lay, S0, w, nslots=None):
+    """Init the same states twice: 16-byte aligned (the streaming kernel takes the 128 x 128 row x
+    column heads) and one float off (every head takes the plain kernel)."""
+    B = S0.shape[0]
+    out = []
+    for aligned in (True, False):
+        pool = lay.alloc_pool(nslots or B)
+        status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        if aligned:
+            S_dev = S0.to(DEV).contiguous()
+        else:
+            flat = torch.zeros(S0.numel() + 1, device=DEV)
+            S_dev = flat[1:].view(S0.shape)
+            S_dev.copy_(S0.to(DEV))
+        stq.init_state(lay, pool, torch.arange(B, dtype=torch.int32, device=DEV), S_dev, w.to(DEV), status=status)
+        torch.cuda.synchronize()
+        out.append((pool.cpu(), status.item()))
+    return out
+
+
+@pytest.mark.parametrize("scale_dtype", [torch.float32, torch.bfloat16])
+def test_init_degenerate_tiles_same_bytes_both_kernels(stq, scale_dtype):
+    """All-zero tiles (unit scales, zero codes) and subnormal tiles: every column energy underflows
+    to 0 (column scale 1) and the row scale is subnormal, so its reciprocal overflows and the codes
+    take the element-by-element form. Both init kernels reach these bytes exactly."""
+    bits = [4, 6, 8, 16]
+    lay = stq.Layout(bits, 128, scale_dtype=scale_dtype)
+    g = torch.Generator().manual_seed(11)
+    S0 = torch.randn(2, 4, 128, 128, generator=g) * 1e-39
+    S0[0, 0] = 0.0
+    S0[1, 2] = 0.0
+    w = torch.rand(4, 128, generator=g) + 0.5
+    (pa, sa), (pb, sb) = _init_two_ways(stq, lay, S0, w)
+    # fp32 scales stay finite and non-zero; a bf16 row scale may round to zero and be flagged
+    assert sa == sb and (sa == 0 or scale_dtype == torch.bfloat16)
+    assert torch.equal(pa, pb)
+
+
+def test_init_out_of_range_slots_flagged_others_written(stq, orc):
+    """Requests with an out-of-range pool slot are flagged and skipped by init; the others are
+    written as the oracle quantizes them, by both init kernels."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl_ = _wl("full2304_b70_mixed", batch=3, heads=4)
+    bits = [4, 6, 8, 16]
+    lay = stq.Layout(bits, 128)
+    w = wlm.impact_weights(wl_)
+    S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(3)])
+    total = lay.bytes_per_request
+    for aligned in (True, False):
+        pool = lay.alloc_pool(2)
+        pool.fill_(7)
+        status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        slots = torch.tensor([1, 5, -1], dtype=torch.int32, device=DEV)
+        if aligned:
+            S_dev = S0.to(DEV)
+        else:
+            flat = torch.zeros(S0.numel() + 1, device=DEV)
+            S_dev = flat[1:].view(S0.shape)
+            S_dev.copy_(S0.to(DEV))
+        stq.init_state(lay, pool, slots, S_dev, w.to(DEV), status=status)
+        torch.cuda.synchronize()
+        assert status.item() & (1 << stq.api.STQ_ERR_BOUNDS)
+        gp = pool.cpu().numpy()
+        assert np.all(gp[:total] == 7), "slot 0 belongs to no request and stays untouched"
+        ref = _oracle_init(orc, wl_, bits, S0[:1], w)
+        tally = Tally()
+        for h in range(4):
+            _, _, tie, _ = orc.quantize(bits[h], as_f64(S0[0, h]), as_f64(w[h]))
+            compare_block(orc, bits[h], 128, tile_bytes(orc, gp, bits, 128, 1, h), tile_bytes(orc, ref, bits, 128, 0, h),
+                          tie, tally, f"init slot 1 head {h} aligned={aligned}")
+        tally.check_budget()
+
+
+def test_init_nonfinite_state_is_flagged(stq, orc):
+    """A state with an infinite entry raises the non-finite flag in either init kernel; the other
+    heads of the call still match the oracle."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl_ = _wl("full2304_b70_mixed", batch=1, heads=3)
+    bits = [6, 4, 8]
+    lay = stq.Layout(bits, 128)
+    w = wlm.impact_weights(wl_)
+    S0 = torch.stack([wlm.initial_state(wl_, 0)])
+    S0[0, 1, 5, 9] = float("inf")
+    ref = _oracle_init(orc, wl_, [bits[0]], S0[:, :1], w[:1])
+    for (pool, status) in _init_two_ways(stq, lay, S0, w):
+        assert status & (1 << stq.api.STQ_ERR_NONFINITE)
+        gp = pool.numpy()
+        tally = Tally()
+        _, _, tie, _ = orc.quantize(bits[0], as_f64(S0[0, 0]), as_f64(w[0]))
+        compare_block(orc, bits[0], 128, tile_bytes(orc, gp, bits, 128, 0, 0), tile_bytes(orc, ref, [bits[0]], 128, 0, 0),
+                      tie, tally, "init head 0 beside a non-finite head")
+        tally.check_budget()
+
+
 def test_dequantize_matches_oracle(stq, orc):
     from quantized_linear_attention_stq_b200 import workloads as wlm
 
