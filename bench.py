@@ -695,6 +695,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the chunked-prefill leg")
     ap.add_argument("--prefill-only", action="store_true", help="run only the chunked-prefill leg (profiling)")
+    ap.add_argument("--init-only", action="store_true",
+                    help="run only the init / dequantize leg, over --batch requests (default 10; profiling)")
     ap.add_argument("--prefill-tokens", type=int, default=8192, help="prompt length of the prefill leg")
     ap.add_argument("--batch", type=int, default=0, help="requests per GPU (default: the workload's)")
     ap.add_argument("--scale-dtype", choices=("f32", "bf16"), default="f32",
@@ -713,6 +715,20 @@ def main(argv=None):
         print(json.dumps({"prefill": prefill_leg(dev, steps=args.steps, warmup=args.warmup, T=args.prefill_tokens,
                                                  fit_rounds=args.fit_rounds)}),
               flush=True)
+    elif args.init_only:
+        import torch
+
+        import quantized_linear_attention_stq_b200 as stq
+        from quantized_linear_attention_stq_b200 import workloads as wlm
+
+        dev = torch.device("cuda", torch.cuda.current_device())
+        wl = wlm.WORKLOADS[args.workload]
+        lay = stq.Layout(wlm.head_bits(wl), wl.d, gate=wl.gate, in_dtype=wl.in_dtype,
+                         scale_dtype=torch.bfloat16 if args.scale_dtype == "bf16" else torch.float32,
+                         fit_rounds=args.fit_rounds)
+        leg = init_dequant_leg(stq, wlm, wl, lay, wlm.impact_weights(wl, dev), dev, requests=args.batch or 10,
+                               reps=args.steps)
+        print(json.dumps({"init_dequantize": leg}), flush=True)
     else:
         run_ours(args)
 
