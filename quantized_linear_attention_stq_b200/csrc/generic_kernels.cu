@@ -1,6 +1,9 @@
 // generic_kernels.cu -- one CTA per (request, head) tile, the state staged in shared memory as
-// fp32 and every step written out directly: initial quantization, dequantization, and the decode
-// step for the small head sizes (d < 128). The tuned d = 128 decode lives in decode_d128.cu.
+// fp32 and every step written out directly: dequantization, the decode step for the small head
+// sizes (d < 128), the sequential prefill, and the initial quantization of the heads the streaming
+// init kernel does not take (FP16 pivots, uniform and multi-round layouts, d < 128, states that
+// are not 16-byte aligned). The tuned d = 128 decode lives in decode_d128.cu, the streaming init
+// of 128 x 128 row x column heads in init_d128.cu.
 //
 // Method (formulas in include/stq.h): per-step read -> gated delta rule update -> readout ->
 // requantize -> store ("线性注意力状态量化难题" (aitest123.com/news/n1kj09), section
