@@ -176,7 +176,7 @@ __device__ __forceinline__ void load_codes_row(const uint8_t *gblock, uint8_t *q
 }
 
 template <int BITS>
-__device__ __forceinline__ void store_codes_row(uint8_t *gblock, int i, int part, const int (&q)[32])
+__device__ __forceinline__ void store_codes_row(uint8_t *gblock, int i, int part, const float (&q)[32])
 {
     using P = PCfg<BITS>;
     uint32_t wv[BITS];
@@ -184,7 +184,7 @@ __device__ __forceinline__ void store_codes_row(uint8_t *gblock, int i, int part
     for (int k = 0; k < BITS; ++k) wv[k] = 0u;
 #pragma unroll
     for (int col = 0; col < 32; ++col) {
-        const uint32_t u = (uint32_t)(q[col] + P::OFFS);
+        const uint32_t u = (uint32_t)((int)q[col] + P::OFFS);
         const int bit = BITS * col, wi = bit >> 5, sh = bit & 31;
         wv[wi] |= u << sh;
         if (sh + BITS > 32) wv[wi + 1] |= u >> (32 - sh);
@@ -806,12 +806,14 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                 ri = round_scale(ri, p.scale_bf16);
                 bad |= !isfinite(ri);
                 const float rri = __frcp_rn(ri);
-                int qc[32];
+                // the codes as exact small integers in fp32: clamped, then rounded half to even by
+                // adding and subtracting 1.5 * 2^23 (the same value as rounding, then clamping)
+                constexpr float RND = 12582912.0f;
+                float qc[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    float x = rintf(S[j] * rri);
-                    x = fminf(fmaxf(x, -(float)P::QMAX), (float)P::QMAX);
-                    qc[j] = (int)x;
+                    const float x = fminf(fmaxf(S[j] * rri, -(float)P::QMAX), (float)P::QMAX);
+                    qc[j] = __fadd_rn(__fadd_rn(x, RND), -RND);
                 }
                 if constexpr (FIT) {
                     // One round of the impact-weighted joint refit (the same round as the decode
@@ -829,7 +831,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                             float e[4];
 #pragma unroll
                             for (int u = 0; u < 4; ++u) {
-                                const float qv = (float)qc[4 * k + u];
+                                const float qv = qc[4 * k + u];
                                 e[u] = pass == 0 ? wr * qv * S[4 * k + u] : (wr * ri) * (qv * qv);
                             }
                             *reinterpret_cast<float4 *>(sq + i * LDSQ + 32 * cq + 4 * k) = make_float4(e[0], e[1], e[2], e[3]);
@@ -865,7 +867,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                     float pn = 0.f, pd = 0.f;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const float qv = (float)qc[j];
+                        const float qv = qc[j];
                         pn += red[32 * cq + j] * qv * S[j];
                         pd += red2[32 * cq + j] * (qv * qv);
                     }
@@ -881,9 +883,9 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                     const float rrn = __frcp_rn(ri);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        float x = rintf(S[j] * red[2 * D + 32 * cq + j] * rrn);
-                        x = fminf(fmaxf(x, -(float)P::QMAX), (float)P::QMAX);
-                        qc[j] = (int)x;
+                        const float x =
+                            fminf(fmaxf(S[j] * red[2 * D + 32 * cq + j] * rrn, -(float)P::QMAX), (float)P::QMAX);
+                        qc[j] = __fadd_rn(__fadd_rn(x, RND), -RND);
                     }
                 }
                 // next chunk's B operand (row i, columns 32 cq ..) and scales
@@ -893,7 +895,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                     uint32_t w4[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        w4[e] = bf2_bits(__floats2bfloat162_rn((float)qc[8 * k + 2 * e], (float)qc[8 * k + 2 * e + 1]));
+                        w4[e] = bf2_bits(__floats2bfloat162_rn(qc[8 * k + 2 * e], qc[8 * k + 2 * e + 1]));
                     *reinterpret_cast<uint4 *>(qrow + sw128_chunk(i, 4 * (cq & 1) + k)) =
                         make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
