@@ -721,14 +721,16 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                 umma::tmem_ld32(tl + TM_DP + 32 * cq, d);
                 if (t < Lc) {
                     float4 *dst = reinterpret_cast<float4 *>(og + (size_t)(t0 + t) * D + 32 * cq);
+                    const float2 gt2 = make_float2(gt, gt);
 #pragma unroll
                     for (int u = 0; u < 32; u += 4) {
                         const float4 c4 = *reinterpret_cast<const float4 *>(sC + 32 * cq + u);
-                        float4 o4;
-                        o4.x = gt * (c4.x * a[u]) + d[u];
-                        o4.y = gt * (c4.y * a[u + 1]) + d[u + 1];
-                        o4.z = gt * (c4.z * a[u + 2]) + d[u + 2];
-                        o4.w = gt * (c4.w * a[u + 3]) + d[u + 3];
+                        // gt (c a) + d per element, two at a time
+                        const float2 o01 = __ffma2_rn(gt2, __fmul2_rn(make_float2(c4.x, c4.y), make_float2(a[u], a[u + 1])),
+                                                      make_float2(d[u], d[u + 1]));
+                        const float2 o23 = __ffma2_rn(gt2, __fmul2_rn(make_float2(c4.z, c4.w), make_float2(a[u + 2], a[u + 3])),
+                                                      make_float2(d[u + 2], d[u + 3]));
+                        const float4 o4 = make_float4(o01.x, o01.y, o23.x, o23.y);
                         bad |= !isfinite(o4.x) || !isfinite(o4.y) || !isfinite(o4.z) || !isfinite(o4.w);
                         dst[u >> 2] = o4;
                     }
@@ -742,13 +744,20 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                 const uint8_t *qrow = sm + OFF_QC + (cq >> 1) * 16384;
                 float v[32];
                 umma::tmem_ld32(tl + TM_D3 + 32 * cq, v);
+                const float2 gC2 = make_float2(gC, gC), ri2 = make_float2(ri, ri);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     float qv[8];
                     bf16x8_to_f32(*reinterpret_cast<const uint4 *>(qrow + sw128_chunk(i, 4 * (cq & 1) + k)), qv);
+                    // gC ((ri c_j) Q_ij) + D3_ij per element, two at a time
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        S[8 * k + e] = gC * ((ri * sC[32 * cq + 8 * k + e]) * qv[e]) + v[8 * k + e];
+                    for (int e = 0; e < 8; e += 2) {
+                        const float2 c2 = make_float2(sC[32 * cq + 8 * k + e], sC[32 * cq + 8 * k + e + 1]);
+                        const float2 s2 = __ffma2_rn(gC2, __fmul2_rn(__fmul2_rn(ri2, c2), make_float2(qv[e], qv[e + 1])),
+                                                     make_float2(v[8 * k + e], v[8 * k + e + 1]));
+                        S[8 * k + e] = s2.x;
+                        S[8 * k + e + 1] = s2.y;
+                    }
                 }
             }
             umma::fence_before_sync();
@@ -758,14 +767,13 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
             {
                 float *red = smf(big, BIG_RED), *rmax = smf(big, BIG_RMAX), *sq = smf(big, BIG_SQ);
                 const float wi = sW[i];
+                const float2 wi2 = make_float2(wi, wi);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    float4 e4;
-                    e4.x = wi * S[4 * k] * S[4 * k];
-                    e4.y = wi * S[4 * k + 1] * S[4 * k + 1];
-                    e4.z = wi * S[4 * k + 2] * S[4 * k + 2];
-                    e4.w = wi * S[4 * k + 3] * S[4 * k + 3];
-                    *reinterpret_cast<float4 *>(sq + i * LDSQ + 32 * cq + 4 * k) = e4;
+                    // (w_i S) S per element, two at a time
+                    const float2 a01 = make_float2(S[4 * k], S[4 * k + 1]), a23 = make_float2(S[4 * k + 2], S[4 * k + 3]);
+                    const float2 e01 = __fmul2_rn(__fmul2_rn(wi2, a01), a01), e23 = __fmul2_rn(__fmul2_rn(wi2, a23), a23);
+                    *reinterpret_cast<float4 *>(sq + i * LDSQ + 32 * cq + 4 * k) = make_float4(e01.x, e01.y, e23.x, e23.y);
                 }
                 __syncthreads();
                 {
@@ -794,9 +802,11 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                 __syncthreads();
                 float m = 0.f;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    S[j] = S[j] * red[32 * cq + j];
-                    m = fmaxf(m, fabsf(S[j]));
+                for (int j = 0; j < 32; j += 2) {
+                    const float2 t = __fmul2_rn(make_float2(S[j], S[j + 1]), make_float2(red[32 * cq + j], red[32 * cq + j + 1]));
+                    S[j] = t.x;
+                    S[j + 1] = t.y;
+                    m = fmaxf(m, fmaxf(fabsf(t.x), fabsf(t.y)));
                 }
                 rmax[cq * D + i] = m;
                 __syncthreads();
@@ -809,11 +819,16 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                 // the codes as exact small integers in fp32: clamped, then rounded half to even by
                 // adding and subtracting 1.5 * 2^23 (the same value as rounding, then clamping)
                 constexpr float RND = 12582912.0f;
+                const float2 rri2 = make_float2(rri, rri), rnd2 = make_float2(RND, RND), nrnd2 = make_float2(-RND, -RND);
                 float qc[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float x = fminf(fmaxf(S[j] * rri, -(float)P::QMAX), (float)P::QMAX);
-                    qc[j] = __fadd_rn(__fadd_rn(x, RND), -RND);
+                for (int j = 0; j < 32; j += 2) {
+                    float2 x = __fmul2_rn(make_float2(S[j], S[j + 1]), rri2);
+                    x.x = fminf(fmaxf(x.x, -(float)P::QMAX), (float)P::QMAX);
+                    x.y = fminf(fmaxf(x.y, -(float)P::QMAX), (float)P::QMAX);
+                    const float2 q = __fadd2_rn(__fadd2_rn(x, rnd2), nrnd2);
+                    qc[j] = q.x;
+                    qc[j + 1] = q.y;
                 }
                 if constexpr (FIT) {
                     // One round of the impact-weighted joint refit (the same round as the decode
