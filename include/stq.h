@@ -225,6 +225,14 @@ stq_status stq_allocate_widths(int32_t num_heads, int32_t d, const double *disto
 stq_status stq_row_impact(int32_t T, int32_t H, int32_t d, int32_t gate, int32_t in_dtype, const void *q,
                           const void *k, const float *beta, const float *alpha, float *w_out, void *stream);
 
+/* Self-test of the bounded wait every kernel of this library uses on its copies: one CTA waits on
+ * a barrier that nothing completes, gives up after the library's cap (about 4e9 SM clock cycles,
+ * ~2 s), ORs the STQ_ERR_TIMEOUT bit into *dev_status and exits, leaving the context usable. It
+ * shows how a stalled copy is reported, without a fault or a hang.
+ *   dev_status  device int32 status word (required)
+ * Enqueued on `stream`; returns STQ_ERR_INVALID_ARG for a null status word. */
+stq_status stq_selftest_wait_timeout(int32_t *dev_status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

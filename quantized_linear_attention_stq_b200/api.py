@@ -28,7 +28,7 @@ EXPORTS = (
     "stq_abi_version", "stq_status_string", "stq_layout_create", "stq_layout_destroy",
     "stq_layout_bytes_per_request", "stq_layout_head_offset", "stq_layout_head_bytes",
     "stq_layout_head_bits", "stq_init_state", "stq_decode_step", "stq_prefill_workspace_bytes",
-    "stq_prefill_chunk", "stq_dequantize", "stq_allocate_widths", "stq_row_impact",
+    "stq_prefill_chunk", "stq_dequantize", "stq_allocate_widths", "stq_row_impact", "stq_selftest_wait_timeout",
 )
 
 
@@ -82,6 +82,7 @@ def lib() -> ctypes.CDLL:
             L.stq_allocate_widths.restype = i32
             L.stq_row_impact.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P]
             L.stq_row_impact.restype = i32
+            L.stq_selftest_wait_timeout.argtypes, L.stq_selftest_wait_timeout.restype = [P, P], i32
             _lib_handle = L
     return _lib_handle
 
@@ -236,6 +237,13 @@ def dequantize(layout: Layout, pool, slots, S_out, status=None, stream=None):
     _need(S_out, "S_out", torch.float32, (B, layout.H, layout.d, layout.d), dev)
     _check(lib().stq_dequantize(layout.handle, _ptr(pool), _pool_slots(layout, pool), _ptr(slots), B, _ptr(S_out),
                                 _ptr(status), _stream(stream)), "stq_dequantize")
+
+
+def selftest_wait_timeout(status, stream=None):
+    """Run the bounded-wait self-test: it ORs the timeout bit into `status` (device int32 [1])
+    after about two seconds of device time."""
+    _need(status, "status", torch.int32, (1,), status.device)
+    _check(lib().stq_selftest_wait_timeout(_ptr(status), _stream(stream)), "stq_selftest_wait_timeout")
 
 
 def status_flags(status: torch.Tensor) -> list:

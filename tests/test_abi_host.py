@@ -159,6 +159,8 @@ def test_calls_reject_bad_arguments_before_enqueueing(stq):
                                None) == 1
     assert L.stq_prefill_chunk(h, fake, 4, fake, 2, 0, 64, None, None, None, None, None, None, None, None, 0, None,
                                None) == 0
+    # the bounded-wait self-test needs a status word to report into
+    assert L.stq_selftest_wait_timeout(None, None) == 1
 
 
 def test_python_binding_checks_shapes(stq):

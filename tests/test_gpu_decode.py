@@ -369,6 +369,32 @@ def test_nonfinite_input_is_flagged(stq, orc):
     assert status.item() & (1 << stq.api.STQ_ERR_NONFINITE)
 
 
+def test_bounded_wait_gives_up_and_reports_timeout(stq):
+    """A wait that nothing completes gives up after the library's cap (~2 s of clock) and reports
+    STQ_ERR_TIMEOUT in the status word; the context stays usable for the next call."""
+    import time
+
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    t0 = time.perf_counter()
+    stq.selftest_wait_timeout(status)
+    torch.cuda.synchronize()
+    waited = time.perf_counter() - t0
+    assert status.item() == 1 << stq.api.STQ_ERR_TIMEOUT
+    assert 0.5 < waited < 30.0
+    # a normal call afterwards runs and reports nothing
+    lay = stq.Layout([4, 16], 128)
+    pool = lay.alloc_pool(1)
+    st2 = torch.zeros(1, dtype=torch.int32, device=DEV)
+    S0 = torch.randn(1, 2, 128, 128, device=DEV)
+    stq.init_state(lay, pool, torch.zeros(1, dtype=torch.int32, device=DEV), S0, torch.ones(2, 128, device=DEV),
+                   status=st2)
+    out = torch.zeros_like(S0)
+    stq.dequantize(lay, pool, torch.zeros(1, dtype=torch.int32, device=DEV), out, status=st2)
+    torch.cuda.synchronize()
+    assert st2.item() == 0
+    assert torch.equal(out[0, 1], S0[0, 1].half().float())  # the pivot head round-trips through fp16
+
+
 def test_empty_calls_are_noops(stq):
     lay = stq.Layout([4], 128)
     pool = lay.alloc_pool(1)
