@@ -53,12 +53,13 @@
  *     may be NULL) as the bit (1 << code): STQ_ERR_NONFINITE when an updated state, scale or output
  *     is not finite (or a pivot overflows fp16; the tile's bytes are then unspecified),
  *     STQ_ERR_BOUNDS when a slot is outside [0, pool_slots) (that tile is skipped),
- *     STQ_ERR_TIMEOUT when a bounded wait for a staged copy gave up (the call's remaining tiles
- *     are skipped). Kernels never trap.
+ *     STQ_ERR_TIMEOUT when a bounded wait for a staged copy gave up (the thread block that timed
+ *     out skips its remaining tiles, whose bytes are then unspecified; other thread blocks of the
+ *     call carry on). Kernels never trap.
  *   - Slots within one call must be distinct. Calls on different streams must not touch the same
  *     slots concurrently.
  *   - Supported on the device: d_k == d_v == d in {16, 32, 64, 128}; widths {4, 6, 8, 16};
- *     q/k/v in fp32 or bf16. The prefill path supports d == 128 and the scalar gate.
+ *     q/k/v in fp32 or bf16; all three gates, for decode and for prefill.
  */
 #ifndef STQ_H
 #define STQ_H
@@ -173,7 +174,11 @@ size_t stq_prefill_workspace_bytes(const stq_layout *layout, int32_t B, int32_t 
  * the requantized state after the last chunk (a multi-chunk call equals the same chunks issued one
  * call each). chunk == 1 is the decode step token by token.
  *   q, k        device [B][H][T][d_k] of in_dtype;  v device [B][H][T][d_v] of in_dtype
- *   beta, alpha device fp32 [B][H][T] (scalar gate)
+ *   beta        device fp32 [B][H][T]
+ *   alpha       device fp32 [B][H][T] (scalar gate) or [B][H][T][d_k] (channel gates)
+ * 128 x 128 heads with bf16 inputs, the scalar gate and chunk == 64 run the tensor-core chunk
+ * form; FP16 pivot heads and every other shape, gate or chunk run a token-by-token kernel with the
+ * same chunk-boundary requantization.
  *   w           device fp32 [H][d_k]
  *   o           device fp32 [B][H][T][d_v], written
  *   workspace   device scratch of >= stq_prefill_workspace_bytes(...) bytes, 256-byte aligned

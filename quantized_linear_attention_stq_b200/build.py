@@ -40,20 +40,45 @@ def stale() -> bool:
     return os.path.getmtime(LIB) < max(os.path.getmtime(f) for f in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    if not (force or stale()):
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *ARCH, *FLAGS, "-shared", "-o", tmp, *sources()]
+def _compile(src: str, obj: str, ptxas_info: bool):
+    cmd = [_nvcc(), *ARCH, *FLAGS, "-c", "-o", obj, src]
     if ptxas_info:
         cmd += ["-Xptxas", "-v"]
-    if verbose:
-        print(" ".join(cmd), flush=True)
     proc = subprocess.run(cmd, capture_output=True, text=True)
+    return cmd, proc
+
+
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
+    """Compile every source to an object (in parallel, under the package's _build folder), then
+    link libstq.so. Objects whose source and headers are older than them are reused."""
+    if not (force or stale()):
+        return LIB
+    from concurrent.futures import ThreadPoolExecutor
+
+    objdir = os.path.join(ROOT, "_build", "stq")
+    os.makedirs(objdir, exist_ok=True)
+    headers = glob.glob(os.path.join(CSRC, "*.cuh")) + [HEADER]
+    newest_header = max(os.path.getmtime(f) for f in headers)
+    jobs = []
+    for src in sources():
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        fresh = os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(src), newest_header)
+        jobs.append((src, obj, force or not fresh))
+    todo = [j for j in jobs if j[2]]
+    with ThreadPoolExecutor(max_workers=max(1, min(len(todo), os.cpu_count() or 1))) as ex:
+        results = list(ex.map(lambda j: _compile(j[0], j[1], ptxas_info), todo))
+    for (src, _, _), (cmd, proc) in zip(todo, results):
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        if proc.returncode != 0:
+            raise RuntimeError(f"nvcc failed on {src} ({proc.returncode}):\n{proc.stdout}\n{proc.stderr}")
+        if verbose or ptxas_info:
+            sys.stdout.write(proc.stdout + proc.stderr)
+    tmp = LIB + f".tmp{os.getpid()}"
+    link = [_nvcc(), *ARCH, "-shared", "-o", tmp, *[j[1] for j in jobs]]
+    proc = subprocess.run(link, capture_output=True, text=True)
     if proc.returncode != 0:
-        raise RuntimeError(f"nvcc failed ({proc.returncode}):\n{proc.stdout}\n{proc.stderr}")
-    if verbose or ptxas_info:
-        sys.stdout.write(proc.stdout + proc.stderr)
+        raise RuntimeError(f"nvcc link failed ({proc.returncode}):\n{proc.stdout}\n{proc.stderr}")
     os.replace(tmp, LIB)
     return LIB
 

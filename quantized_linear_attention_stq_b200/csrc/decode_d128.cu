@@ -890,6 +890,11 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(sm.tmem_base), "r"(TMEM_COLS));
     }
+    // A launch that went out with programmatic dependent launch may have started before the launch
+    // ahead of it finished; it completes only after that one has (a no-op for a launch in plain
+    // stream order). Completion of a call's last launch therefore implies completion of the whole
+    // call, which is what the work after it on the stream relies on.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // pdl: this launch follows another launch of the same stq_decode_step call. Those touch disjoint

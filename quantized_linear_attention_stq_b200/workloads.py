@@ -154,7 +154,9 @@ def decode_inputs(wl: Workload, token: int, device="cpu", batch: Optional[int] =
 
 
 def prefill_inputs(wl: Workload, t0: int, T: int, device="cpu", batch: Optional[int] = None) -> dict:
-    """Inputs of prompt tokens [t0, t0+T): q, k, v [B, H, T, d], beta, alpha [B, H, T] fp32."""
+    """Inputs of prompt tokens [t0, t0+T): q, k, v [B, H, T, d], beta [B, H, T] fp32, alpha
+    [B, H, T] fp32 (scalar gate) or [B, H, T, d] (channel gates: the per-key-row gate of the head,
+    constant over tokens)."""
     B = wl.batch if batch is None else batch
     H, d = wl.heads, wl.d
     idx = 2_000_000 + t0 * 7 + T
@@ -162,9 +164,11 @@ def prefill_inputs(wl: Workload, t0: int, T: int, device="cpu", batch: Optional[
     k = _unit(torch.randn((B, H, T, d), generator=_gen(wl, _S_K, idx, device), device=device))
     v = torch.randn((B, H, T, d), generator=_gen(wl, _S_V, idx, device), device=device)
     beta = torch.sigmoid(torch.randn((B, H, T), generator=_gen(wl, _S_BETA, idx, device), device=device))
-    a = gate_values(wl)
-    assert a.dim() == 1, "prefill inputs are drawn for the scalar gate"
-    alpha = a.to(device)[None, :, None].expand(B, H, T).contiguous()
+    a = gate_values(wl).to(device)
+    if a.dim() == 1:
+        alpha = a[None, :, None].expand(B, H, T).contiguous()
+    else:
+        alpha = a[None, :, None, :].expand(B, H, T, d).contiguous()
     return dict(q=q.to(wl.in_dtype), k=k.to(wl.in_dtype), v=v.to(wl.in_dtype),
                 beta=beta.float(), alpha=alpha)
 

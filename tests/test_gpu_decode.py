@@ -154,6 +154,68 @@ def test_many_requests_split_launches(stq, orc):
     _decode_teacher_forced(stq, orc, wl_, [4], 1, slots_perm=False)
 
 
+def test_back_to_back_calls_without_sync(stq, orc):
+    """Two stq_decode_step calls issued back to back on one stream with no synchronization between
+    them (mixed widths with pivots and more than 256 requests: several width and request-group
+    launches per call) give the same pool bytes and readouts as the same calls with a
+    synchronization between them, and the second step matches the oracle from the first step's
+    pool on sampled tiles."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    bits = [4, 6, 8, 16, 8, 6, 4, 16]
+    wl_ = _wl("full2304_b70_mixed", batch=300, heads=len(bits), outliers=False)
+    B, H, d = wl_.batch, wl_.heads, wl_.d
+    lay = stq.Layout(bits, d, gate=wl_.gate, in_dtype=wl_.in_dtype)
+    w = wlm.impact_weights(wl_).to(DEV)
+    S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(B)]).to(DEV)
+    slots = torch.arange(B, dtype=torch.int32, device=DEV).flip(0).contiguous()
+    pool0 = lay.alloc_pool(B)
+    stq.init_state(lay, pool0, slots, S0, w)
+    ins = [{n: x.to(DEV) for n, x in wlm.decode_inputs(wl_, t).items()} for t in range(2)]
+
+    def run(sync_between):
+        pool = pool0.clone()
+        outs = [torch.zeros(B, H, d, device=DEV) for _ in range(2)]
+        status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        mid = None
+        for t in range(2):
+            g = ins[t]
+            stq.decode_step(lay, pool, slots, g["q"], g["k"], g["v"], g["beta"], g["alpha"], w, outs[t],
+                            status=status)
+            if sync_between and t == 0:
+                torch.cuda.synchronize()
+                mid = pool.clone()
+        torch.cuda.synchronize()
+        assert status.item() == 0, stq.status_flags(status)
+        return pool, outs, mid
+
+    p_ref, o_ref, mid = run(True)
+    p_b2b, o_b2b, _ = run(False)
+    assert torch.equal(p_ref, p_b2b)
+    assert torch.equal(o_ref[0], o_b2b[0]) and torch.equal(o_ref[1], o_b2b[1])
+    # second step teacher forced from the first step's GPU pool, sampled tiles
+    midh, finh, o1 = mid.cpu().numpy(), p_ref.cpu().numpy(), o_ref[1].cpu().numpy()
+    inp = {n: x.cpu() for n, x in ins[1].items()}
+    wc = w.cpu()
+    tally = Tally()
+    rng = np.random.default_rng(11)
+    slot_of = slots.cpu().numpy()
+    for r, h in zip(rng.integers(0, B, 24), rng.integers(0, H, 24)):
+        r, h = int(r), int(h)
+        pre = tile_bytes(orc, midh, bits, d, int(slot_of[r]), h)
+        alpha = inp["alpha"][r, h].double().numpy()
+        res = orc.decode_step(bits[h], wl_.gate, pre, as_f64(inp["q"][r, h]), as_f64(inp["k"][r, h]),
+                              as_f64(inp["v"][r, h]), float(inp["beta"][r, h]), alpha, as_f64(wc[h]), d, d)
+        M = None
+        if bits[h] == 16:
+            M = update_magnitude(orc.dequantize(16, d, d, pre), as_f64(inp["k"][r, h]), as_f64(inp["v"][r, h]),
+                                 float(inp["beta"][r, h]), alpha)
+        compare_block(orc, bits[h], d, tile_bytes(orc, finh, bits, d, int(slot_of[r]), h), res["block"], res["tie"],
+                      tally, f"req {r} head {h}", err_scale=M)
+        compare_o(o1[r, h], res["o"], tally, f"o req {r} head {h}")
+    tally.check_budget()
+
+
 # ------------------------------------------------------------------------------------------------
 # init and dequantize
 # ------------------------------------------------------------------------------------------------

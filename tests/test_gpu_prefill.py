@@ -9,7 +9,8 @@ import numpy as np
 import pytest
 import torch
 
-from _parity import Tally, as_f64, compare_block, compare_o, oracle_pool, tile_bytes
+from _parity import (Tally, as_f64, compare_block, compare_o, compare_pivot_exact, oracle_pool, pivot_chunk_exact,
+                     tile_bytes)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -25,10 +26,11 @@ def stq():
     return m
 
 
-def _setup(orc, B, bits, d=128, dtype=torch.bfloat16):
+def _setup(orc, B, bits, d=128, dtype=torch.bfloat16, base="prefill16_b16_6bit", gate=None):
     from quantized_linear_attention_stq_b200 import workloads as wlm
 
-    wl_ = wlm.scaled(wlm.WORKLOADS["prefill16_b16_6bit"], batch=B, heads=len(bits), d=d, in_dtype=dtype)
+    extra = {} if gate is None else {"gate": gate}
+    wl_ = wlm.scaled(wlm.WORKLOADS[base], batch=B, heads=len(bits), d=d, in_dtype=dtype, **extra)
     w = wlm.impact_weights(wl_)
     blocks = []
     for r in range(B):
@@ -42,12 +44,32 @@ def _setup(orc, B, bits, d=128, dtype=torch.bfloat16):
     return wl_, w, oracle_pool(orc, bits, d, blocks)
 
 
-def _oracle_chunk(orc, pool, bits, d, r, h, inp, t0, T, w, chunk):
+def _oracle_chunk(orc, pool, bits, d, r, h, inp, t0, T, w, chunk, gate=0):
     blk = tile_bytes(orc, pool, bits, d, r, h)
     sl = slice(t0, t0 + T)
-    return orc.prefill_seq(bits[h], 0, blk, as_f64(inp["q"][r, h, sl]), as_f64(inp["k"][r, h, sl]),
+    return orc.prefill_seq(bits[h], gate, blk, as_f64(inp["q"][r, h, sl]), as_f64(inp["k"][r, h, sl]),
                            as_f64(inp["v"][r, h, sl]), as_f64(inp["beta"][r, h, sl]), as_f64(inp["alpha"][r, h, sl]),
                            as_f64(w[h]), chunk, d, d)
+
+
+def _check_chunk(orc, opool, gp, og, bits, d, B, inp, T, w, gate, tally):
+    """Teacher-forced check of one single-chunk call: codes and scales (or, for a pivot, the
+    per-value fp16 rule with the error bound carried through the chunk) and every readout."""
+    for r in range(B):
+        for h in range(len(bits)):
+            what = f"req {r} head {h}"
+            res = _oracle_chunk(orc, opool, bits, d, r, h, inp, 0, T, w, 64, gate)
+            assert res["status"] == orc.OK
+            got = tile_bytes(orc, gp, bits, d, r, h)
+            if bits[h] == 16:
+                S0 = orc.dequantize(16, d, d, tile_bytes(orc, opool, bits, d, r, h))
+                args = [as_f64(inp[n][r, h, :T]) for n in ("q", "k", "v", "beta", "alpha")]
+                S_ex, bound = pivot_chunk_exact(orc, gate, S0, *args)
+                compare_pivot_exact(orc, d, got, res["block"], S_ex, bound, tally, what)
+            else:
+                compare_block(orc, bits[h], d, got, res["block"], res["tie"], tally, what)
+            for t in range(T):
+                compare_o(og[r, h, t], res["o"][t], tally, f"token {t} " + what)
 
 
 @pytest.mark.parametrize("T", [64, 37, 1])
@@ -71,21 +93,67 @@ def test_single_chunk_teacher_forced(stq, orc, T):
     assert status.item() == 0
     gp = gpool.cpu().numpy()
     og = o.cpu().numpy()
-    tally = Tally(updates_per_check=T)
-    for r in range(B):
-        for h in range(len(bits)):
-            res = _oracle_chunk(orc, opool, bits, d, r, h, inp, 0, T, w, 64)
-            assert res["status"] == orc.OK
-            # a pivot carries T fp32 updates inside the chunk: scale the per-step error bound by T
-            M = None
-            if bits[h] == 16:
-                S = orc.dequantize(16, d, d, tile_bytes(orc, opool, bits, d, r, h))
-                M = T * np.max(np.abs(S)) * np.ones((d, d)) * 4.0
-            compare_block(orc, bits[h], d, tile_bytes(orc, gp, bits, d, r, h), res["block"], res["tie"], tally,
-                          f"req {r} head {h}", err_scale=M)
-            for t in range(T):
-                compare_o(og[r, h, t], res["o"][t], tally, f"token {t} req {r} head {h}")
+    tally = Tally()
+    _check_chunk(orc, opool, gp, og, bits, d, B, inp, T, w, 0, tally)
     tally.check_budget()
+
+
+@pytest.mark.parametrize("gate", [1, 2])
+@pytest.mark.parametrize("d,T", [(128, 64), (128, 23), (32, 64), (32, 37)])
+def test_channel_gate_single_chunk_teacher_forced(stq, orc, gate, d, T):
+    """Both channel gates (alpha per key row: [B][H][T][d_k]) through stq_prefill_chunk, full and
+    short chunks, mixed widths with an FP16 pivot, against the oracle's sequential prefill."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    bits = [6, 4, 8, 16]
+    B = 2
+    wl_, w, opool = _setup(orc, B, bits, d=d, base="channel32_b128_4bit", gate=gate)
+    lay = stq.Layout(bits, d, gate=gate, in_dtype=torch.bfloat16)
+    inp = wlm.prefill_inputs(wl_, 0, T)
+    assert inp["alpha"].shape == (B, len(bits), T, d)
+    # permuted slots: request 0 lives in slot 1 and request 1 in slot 0
+    offs, total = orc.request_layout(bits, d, d)
+    swap = lambda a: np.concatenate([a[total:2 * total], a[:total]])  # noqa: E731
+    gpool = torch.from_numpy(swap(opool)).to(DEV)
+    slots = torch.tensor([1, 0], dtype=torch.int32, device=DEV)
+    o = torch.zeros(B, len(bits), T, d, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    stq.prefill_chunk(lay, gpool, slots, *(inp[n].to(DEV) for n in ("q", "k", "v", "beta", "alpha")), w.to(DEV), o,
+                      chunk=64, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0, stq.status_flags(status)
+    gp, og = swap(gpool.cpu().numpy()), o.cpu().numpy()
+    tally = Tally()
+    _check_chunk(orc, opool, gp, og, bits, d, B, inp, T, w, gate, tally)
+    tally.check_budget()
+
+
+@pytest.mark.parametrize("gate", [1, 2])
+def test_channel_gate_multi_chunk_equals_single_chunk_calls(stq, orc, gate):
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    bits = [6, 16, 4]
+    B, d, T, C = 2, 64, 80, 32
+    wl_, w, opool = _setup(orc, B, bits, d=d, base="channel32_b128_4bit", gate=gate)
+    lay = stq.Layout(bits, d, gate=gate, in_dtype=torch.bfloat16)
+    inp = {n: x.to(DEV) for n, x in wlm.prefill_inputs(wl_, 0, T).items()}
+    slots = torch.arange(B, dtype=torch.int32, device=DEV)
+    wd = w.to(DEV)
+    p_full = torch.from_numpy(opool.copy()).to(DEV)
+    o_full = torch.zeros(B, 3, T, d, device=DEV)
+    stq.prefill_chunk(lay, p_full, slots, inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], wd, o_full, chunk=C)
+    p_seq = torch.from_numpy(opool.copy()).to(DEV)
+    outs = []
+    for c0 in range(0, T, C):
+        sl = slice(c0, min(c0 + C, T))
+        part = {n: x[:, :, sl].contiguous() for n, x in inp.items()}
+        o_part = torch.zeros(B, 3, sl.stop - sl.start, d, device=DEV)
+        stq.prefill_chunk(lay, p_seq, slots, part["q"], part["k"], part["v"], part["beta"], part["alpha"], wd, o_part,
+                          chunk=C)
+        outs.append(o_part)
+    torch.cuda.synchronize()
+    assert torch.equal(p_full, p_seq)
+    assert torch.equal(o_full, torch.cat(outs, dim=2))
 
 
 def test_multi_chunk_equals_single_chunk_calls(stq, orc):
@@ -161,7 +229,7 @@ def test_full_geometry_chunk_chain_and_sampled_first_chunk(stq, orc):
     # teacher-forced first chunk of sampled tiles
     cpu_inp = {n: x[:, :, :C].cpu() for n, x in inp.items()}
     o0 = outs[0].cpu().numpy()
-    tally = Tally(updates_per_check=C)
+    tally = Tally()
     rng = np.random.default_rng(5)
     for r, h in zip(rng.integers(0, B, 6), rng.integers(0, H, 6)):
         res = _oracle_chunk(orc, opool, bits, d, int(r), int(h), cpu_inp, 0, C, w, C)
@@ -191,12 +259,6 @@ def test_fp32_inputs_sequential_form(stq, orc):
     torch.cuda.synchronize()
     assert status.item() == 0
     gp, og = gpool.cpu().numpy(), o.cpu().numpy()
-    tally = Tally(updates_per_check=T)
-    for r in range(B):
-        for h in range(len(bits)):
-            res = _oracle_chunk(orc, opool, bits, d, r, h, inp, 0, T, w, 64)
-            compare_block(orc, bits[h], d, tile_bytes(orc, gp, bits, d, r, h), res["block"], res["tie"], tally,
-                          f"req {r} head {h}")
-            for t in range(T):
-                compare_o(og[r, h, t], res["o"][t], tally, f"token {t} req {r} head {h}")
+    tally = Tally()
+    _check_chunk(orc, opool, gp, og, bits, d, B, inp, T, w, 0, tally)
     tally.check_budget()

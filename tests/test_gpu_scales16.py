@@ -11,7 +11,8 @@ import numpy as np
 import pytest
 import torch
 
-from _parity import Tally, as_f64, compare_block, compare_block_bf16s, compare_o, update_magnitude
+from _parity import (Tally, as_f64, compare_block, compare_block_bf16s, compare_o, compare_pivot_exact,
+                     pivot_chunk_exact, update_magnitude)
 
 pytestmark = pytest.mark.gpu
 
@@ -202,7 +203,6 @@ def test_prefill_chunk(stq, orc, d, in_dtype, T):
     offs, total = _layout(orc, bits, d)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     tally = Tally()
-    tally.updates_per_check = T
     for call in range(2):
         inp = wlm.prefill_inputs(wl_, call * T, T)
         pool = torch.from_numpy(opool.copy()).to(DEV)
@@ -221,9 +221,10 @@ def test_prefill_chunk(stq, orc, d, in_dtype, T):
                 got = _tile(orc, gp, bits, d, r, h)
                 if b == 16:
                     res = orc.prefill_seq_s(16, orc.SCALE_BF16, 0, blk, *args, as_f64(w[h]), 64, d, d)
-                    # a pivot carries T fp32 updates inside the chunk: the per-step bound times T
-                    M = T * np.max(np.abs(orc.dequantize(16, d, d, blk))) * np.ones((d, d)) * 4.0
-                    compare_block(orc, 16, d, got, res["block"], res["tie"], tally, what, err_scale=M)
+                    # a pivot carries T fp32 updates inside the chunk: per-value rule with the
+                    # error bound carried through the chunk
+                    S_ex, bound = pivot_chunk_exact(orc, 0, orc.dequantize(16, d, d, blk), *args)
+                    compare_pivot_exact(orc, d, got, res["block"], S_ex, bound, tally, what)
                 else:
                     S = orc.dequantize_s(b, orc.SCALE_BF16, d, d, blk)
                     for t in range(T):
