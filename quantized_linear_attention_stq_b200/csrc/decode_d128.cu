@@ -42,7 +42,6 @@ namespace {
 constexpr int D = 128;
 constexpr int NT = 128;                // threads per CTA: one tile at a time
 constexpr int NSMAX = 4;               // slots (tiles in flight) per CTA
-constexpr int MAXB = 256;              // requests per launch whose slots are cached in smem
 constexpr uint32_t MAGIC = 0x4B000000u;  // bit pattern of 2^23
 constexpr uint32_t TMEM_COLS = 128;    // per CTA: 128 lanes x 128 columns of fp32 = one tile
 // red[]: one region of RS floats per (warp, half) k = 2w + h. [0, 128): the half's column
@@ -56,13 +55,15 @@ constexpr int RS = 336;                // region stride (= 16 mod 32 banks: the 
 // position, request) = (t / B, t % B) and advanced without a division.
 struct Issuer {
     int n, pos, b, qG, rG;
+    int next_slot;  // pool slot of the next tile's request, loaded one issue ahead
 };
 
 // Per tile, written by the issuing thread: where the tile lives and which input row it uses.
 struct SlotMeta {
     unsigned long long gblock;  // address of the tile's head block in the pool
     uint32_t orow;              // request * head_count + head: the row of q, k, v, beta, alpha, o
-    uint32_t skip;              // 1: out-of-range slot, nothing was loaded
+    uint16_t skip;              // 1: out-of-range slot, nothing was loaded
+    uint16_t bits;              // code width of the tile
 };
 
 struct __align__(16) SmemFixed {
@@ -77,9 +78,7 @@ struct __align__(16) SmemFixed {
     float scal[NSMAX][2];    // per slot: beta, alpha
     SlotMeta meta[4];        // per tile n, at n % 4 (NS + 1 <= 4 tiles are live at a time)
     Issuer iss;              // thread 0's tile cursor
-    int32_t slots[MAXB];
     unsigned long long bars[NSMAX];
-    float2 unpack_off;       // (-(2^23 + o), -(2^23 + o * SIG1)), o = 2^(b-1)
     uint32_t magic;          // 0x4B000000, read at run time so the unpack keeps it in a register
                              // and forms each value with one LOP3 ((s & mask) | magic)
     uint32_t tmem_base;
@@ -102,15 +101,35 @@ struct __align__(16) SmemFit {
 };
 
 // ---------------------------------------------------------------------------------------------
-// Static per-width facts
+// Per-width facts. A launch either has one compile-time width (BITS = 4, 6, 8 or 16: FP16 pivots)
+// or takes each tile's width from the head table (BITS = 0: any mix of 4, 6 and 8 bits; the ring
+// slots are then sized for 8-bit tiles and only the unpack and pack steps branch on the width).
 // ---------------------------------------------------------------------------------------------
+struct Width {
+    int bits;
+    uint32_t rb;    // bytes of one 128-wide row of codes
+    uint32_t soff;  // byte offset of r[] in the head block
+    float qmax;
+    float round;    // 2^23 + 2^(b-1): the FFMA against it rounds half to even into the code bits
+    float sig1;     // odd columns are unpacked scaled by sig1 (even columns by 1)
+};
+
+__device__ __forceinline__ Width width_of(int bits)
+{
+    Width w;
+    w.bits = bits;
+    w.rb = bits == 16 ? 256u : 16u * (uint32_t)bits;
+    w.soff = bits == 16 ? 0u : 2048u * (uint32_t)bits;  // the codes of 128 x 128, a multiple of 16
+    w.qmax = bits == 16 ? 0.f : (float)((1 << (bits - 1)) - 1);
+    w.round = 8388608.0f + (bits == 16 ? 0.f : (float)(1 << (bits - 1)));
+    w.sig1 = bits == 4 ? 16.f : bits == 6 ? 64.f : 1.f;
+    return w;
+}
+
 template <int BITS, int GATE, int IN_BF16, int FIT, int SB16>
 struct Cfg {
-    static constexpr int RB = BITS == 16 ? 256 : 16 * BITS;    // bytes of one 128-wide row
-    static constexpr uint32_t SOFF = scale_offset(BITS, D, D);  // byte offset of r[]
-    static constexpr uint32_t BLK = head_block_bytes(BITS, D, D);  // ring room (fp32 scales)
-    // bytes of the block with 16-bit scales: the copy is shorter, the ring layout the same
-    static constexpr uint32_t BLK16 = head_block_bytes_bf16s(BITS, D, D);
+    static constexpr int RBITS = BITS == 0 ? 8 : BITS;                // the ring's slots fit this width
+    static constexpr uint32_t BLK = head_block_bytes(RBITS, D, D);    // ring room (fp32 scales)
     static constexpr uint32_t ROW_IN = D * (IN_BF16 ? 2u : 4u);
     static constexpr uint32_t K_OFF = BLK, Q_OFF = BLK + ROW_IN, V_OFF = BLK + 2 * ROW_IN;
     static constexpr uint32_t W_OFF = BLK + 3 * ROW_IN, A_OFF = W_OFF + 4 * D;
@@ -120,10 +139,6 @@ struct Cfg {
     // slots so that four CTAs fit an SM's 228 KB where they can
     static constexpr int NS = BITS == 4 ? 3 : 2;
     static constexpr size_t SMEM = RING + (size_t)NS * LEN;
-    static constexpr float QMAX = BITS == 16 ? 0.f : (float)((1 << (BITS - 1)) - 1);
-    static constexpr float ROUND = 8388608.0f + (BITS == 16 ? 0.f : (float)(1 << (BITS - 1)));
-    // odd columns are unpacked scaled by SIG1 (even columns by 1)
-    static constexpr float SIG1 = BITS == 4 ? 16.f : BITS == 6 ? 64.f : 1.f;
 };
 
 __device__ __forceinline__ float f_of(uint32_t x) { return __uint_as_float(x); }
@@ -303,6 +318,7 @@ __device__ __forceinline__ void issue_next(const TileParams &p, SmemFixed &sm, u
     const int n = it.n, slot_i = n % C::NS;
     const TileEntry e = p.table[it.pos];
     const int hr = entry_head(e), b = it.b;
+    const int slot = it.next_slot;
     ++it.n;
     it.b += it.rG;
     it.pos += it.qG;
@@ -310,11 +326,13 @@ __device__ __forceinline__ void issue_next(const TileParams &p, SmemFixed &sm, u
         it.b -= p.B;
         ++it.pos;
     }
+    if (it.n < my_count) it.next_slot = p.slots[it.b];  // used at the next issue
     const uint32_t bar = smem_u32(&sm.bars[slot_i]);
     const uint32_t row = (uint32_t)b * (uint32_t)p.head_count + (uint32_t)hr;
+    const int bits = BITS == 0 ? entry_bits(e) : BITS;
     SlotMeta &m = sm.meta[n & 3];
     m.orow = row;
-    const int slot = sm.slots[b];
+    m.bits = (uint16_t)bits;
     if (slot < 0 || slot >= p.pool_slots) {
         flag(p.status, kFlagBounds);
         m.skip = 1u;
@@ -330,7 +348,7 @@ __device__ __forceinline__ void issue_next(const TileParams &p, SmemFixed &sm, u
     if (GATE == 0) cp_async4(smem_u32(&sm.scal[slot_i][1]), p.alpha + row);
     cp_async_arrive(bar);
     const uint32_t dst = smem_u32(ring_slot<BITS, GATE, IN_BF16, FIT, SB16>(smem, slot_i));
-    const uint32_t blk = SB16 ? C::BLK16 : C::BLK;
+    const uint32_t blk = SB16 ? head_block_bytes_bf16s(bits, D, D) : head_block_bytes(bits, D, D);
     mbar_arrive_expect_tx(bar, C::LEN - (C::BLK - blk));
     bulk_g2s(dst, src, blk, bar);
     bulk_g2s(dst + C::K_OFF, (const uint8_t *)p.k + (size_t)row * C::ROW_IN, C::ROW_IN, bar);
@@ -353,10 +371,11 @@ __device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, in
     if (!__all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&sm.bars[slot_i]), phase))) return false;
     if (sm.meta[n & 3].skip) return true;  // skipped tile: nothing was loaded
     const int pb = n & 1;
+    const Width W = width_of(BITS == 0 ? (int)sm.meta[n & 3].bits : BITS);
     const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16, FIT, SB16>(smem, slot_i);
     const int i = threadIdx.x;
     constexpr bool pivot = BITS == 16;
-    const float r = pivot ? 1.f : load_scale(tile + C::SOFF, i, SB16);
+    const float r = pivot ? 1.f : load_scale(tile + W.soff, i, SB16);
     const float k = load_in<IN_BF16>(tile + C::K_OFF, i);
     const float q = load_in<IN_BF16>(tile + C::Q_OFF, i);
     const float w = reinterpret_cast<const float *>(tile + C::W_OFF)[i];
@@ -372,7 +391,7 @@ __device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, in
         const float mu = -sw * a * k;
         channel(smem).rowMu[i] = make_float2(mu, mu);
     }
-    if (!pivot) sm.rowRq[pb][i] = fast_rcp(sw * C::QMAX);
+    if (!pivot) sm.rowRq[pb][i] = fast_rcp(sw * W.qmax);
     float s0 = w, s1 = q * k, s2 = q * a * k;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -399,15 +418,14 @@ __device__ __forceinline__ bool precompute_rows(SmemFixed &sm, uint8_t *smem, in
 // one-pass r and s of this lane's row i = 8 cg + rb.
 template <int BITS, int GATE, int IN_BF16, int FIT, int SB16>
 __device__ __forceinline__ bool refit_scales(const TileParams &p, SmemFixed &sm, uint8_t *smem, int n, uint32_t tcol,
-                                             float c_one, float r_one, float s_one)
+                                             const Width &W, float c_one, float r_one, float s_one)
 {
-    using C = Cfg<BITS, GATE, IN_BF16, FIT, SB16>;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, cg = lane & 15, sub = lane >> 4;
     const int rb = 2 * warp + sub, pb = n & 1;
     constexpr int sb16 = SB16;
     const float *rho = fitmem<BITS, GATE, IN_BF16, FIT, SB16>(smem).rowRho;
-    const float2 rnd = make_float2(C::ROUND, C::ROUND), nrnd = make_float2(-C::ROUND, -C::ROUND);
-    uint8_t *gsc = reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + C::SOFF);
+    const float2 rnd = make_float2(W.round, W.round), nrnd = make_float2(-W.round, -W.round);
+    uint8_t *gsc = reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + W.soff);
     tmem_wait_st();
     // ---- column sums over this thread's 16 rows --------------------------------------------
     {
@@ -523,7 +541,7 @@ __device__ __forceinline__ bool refit_scales(const TileParams &p, SmemFixed &sm,
         const int i = 8 * cg + rb;
         float rf = r_one, sf = s_one;
         if (den > 0.f) {
-            const float rq = sm.rowRq[pb][i] * C::QMAX;  // 1 / sqrt(w_i)
+            const float rq = sm.rowRq[pb][i] * W.qmax;  // 1 / sqrt(w_i)
             const float rn = round_scale((num / den) * rq, sb16);
             if (isfinite(rn) && rn > 0.f) {
                 rf = rn;
@@ -535,6 +553,77 @@ __device__ __forceinline__ bool refit_scales(const TileParams &p, SmemFixed &sm,
     }
     __syncwarp();
     return true;
+}
+
+// Sweep A of a tile of width WB: unpack this thread's 16 row segments into Tensor Memory, with
+// the column sums of k~Q and q~Q (accumulated into accU / accP).
+template <int WB>
+__device__ __forceinline__ void sweep_unpack(const uint8_t *tile, const SmemFixed &sm, uint32_t tcol, int rb, int cg,
+                                             uint32_t magic, float2 (&accU)[4], float2 (&accP)[4])
+{
+    constexpr uint32_t RB = WB == 16 ? 256u : 16u * WB;
+    constexpr float o = WB == 16 ? 0.f : (float)(1 << (WB - 1));
+    constexpr float SIG1 = WB == 4 ? 16.f : WB == 6 ? 64.f : 1.f;
+    const float2 off = make_float2(-(8388608.0f + o), -(8388608.0f + o * SIG1));
+    const uint8_t *rowsrc = tile + rb * RB + cg * (WB == 16 ? 16 : WB);
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+        float2 ch[4];
+        unpack_row<WB>(rowsrc + 8 * m * RB, cg, off, magic, ch);
+        const float4 kq = sm.rowKQ[8 * m + rb];
+        const float2 kk = make_float2(kq.x, kq.y), qq = make_float2(kq.z, kq.w);
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+            accU[pp] = __ffma2_rn(kk, ch[pp], accU[pp]);
+            accP[pp] = __ffma2_rn(qq, ch[pp], accP[pp]);
+        }
+        tmem_st8(tcol + 8 * m, ch);
+    }
+}
+
+// Sweep D of a tile of width WB: x = z s (z / K~_j first with the refit) rounded half to even by
+// the FFMA against 2^23 + 2^(b-1), packed, stored to the head block in HBM.
+template <int WB, int FIT>
+__device__ __forceinline__ void sweep_pack(uint8_t *gblock, const SmemFixed &sm, uint32_t tcol, int rb, int cg)
+{
+    constexpr uint32_t RB = 16u * WB;
+    constexpr float QMAX = (float)((1 << (WB - 1)) - 1);
+    const float2 rnd = make_float2(8388608.0f + (float)(1 << (WB - 1)), 8388608.0f + (float)(1 << (WB - 1)));
+    uint8_t *dstrow = gblock + rb * RB + cg * WB;
+    float2 ik[4];  // 1 / K~_j of this thread's columns (refit only)
+    if constexpr (FIT) {
+        load_pairs(sm.colB + 8 * cg, ik);
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) ik[pp] = make_float2(fast_rcp(ik[pp].x), fast_rcp(ik[pp].y));
+    }
+    float2 cha[8], chb[8];
+    tmem_ld16_async(tcol, cha);
+    tmem_wait_ld(cha);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        float2 (&ch)[8] = (k & 1) ? chb : cha;
+        float2 (&nx)[8] = (k & 1) ? cha : chb;
+        if (k + 1 < 8) tmem_ld16_async(tcol + 16 * (k + 1), nx);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int m = 2 * k + r;
+            const float2 s2 = sm.rowS[8 * m + rb];
+#pragma unroll
+            for (int pp = 0; pp < 4; ++pp) {
+                if constexpr (FIT) {
+                    // x = z / (K~_j rho~_i), clamped (refitted scales may clip), rounded by the add
+                    float2 v = __fmul2_rn(__fmul2_rn(ch[4 * r + pp], ik[pp]), s2);
+                    v.x = fminf(fmaxf(v.x, -QMAX), QMAX);
+                    v.y = fminf(fmaxf(v.y, -QMAX), QMAX);
+                    ch[4 * r + pp] = __fadd2_rn(v, rnd);
+                } else {
+                    ch[4 * r + pp] = __ffma2_rn(ch[4 * r + pp], s2, rnd);
+                }
+            }
+            pack_store_row<WB>(dstrow + 8 * m * RB, cg, ch + 4 * r);
+        }
+        if (k + 1 < 8) tmem_wait_ld(nx);
+    }
 }
 
 // Tile n (ring slot n % NS). Returns false if the wait for the next tile timed out.
@@ -549,27 +638,23 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
     const int rb = 2 * warp + sub;  // this thread's rows: rb + 8m, m < 16
     const uint8_t *tile = ring_slot<BITS, GATE, IN_BF16, FIT, SB16>(smem, slot_i);
     // the tile's record (sm.meta[n & 3]) stays valid until the issue after the next tile's B2
+    const int bits = BITS == 0 ? (int)sm.meta[n & 3].bits : BITS;
+    const Width W = width_of(bits);
 
     // ---- Sweep A: unpack to TMEM, column sums of k~Q and q~Q -------------------------------
     {
-        const uint8_t *rowsrc = tile + rb * C::RB + cg * (pivot ? 16 : BITS);
-        const float2 off = sm.unpack_off;
         const uint32_t magic = sm.magic;
         float2 accU[4], accP[4];
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp) accU[pp] = accP[pp] = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            float2 ch[4];
-            unpack_row<BITS>(rowsrc + 8 * m * C::RB, cg, off, magic, ch);
-            const float4 kq = sm.rowKQ[8 * m + rb];
-            const float2 kk = make_float2(kq.x, kq.y), qq = make_float2(kq.z, kq.w);
-#pragma unroll
-            for (int pp = 0; pp < 4; ++pp) {
-                accU[pp] = __ffma2_rn(kk, ch[pp], accU[pp]);
-                accP[pp] = __ffma2_rn(qq, ch[pp], accP[pp]);
-            }
-            tmem_st8(tcol + 8 * m, ch);
+        if constexpr (BITS != 0) {
+            sweep_unpack<BITS>(tile, sm, tcol, rb, cg, magic, accU, accP);
+        } else if (bits == 4) {
+            sweep_unpack<4>(tile, sm, tcol, rb, cg, magic, accU, accP);
+        } else if (bits == 6) {
+            sweep_unpack<6>(tile, sm, tcol, rb, cg, magic, accU, accP);
+        } else {
+            sweep_unpack<8>(tile, sm, tcol, rb, cg, magic, accU, accP);
         }
         // halves 0/1 of a warp hold the same columns: half 0 keeps U, half 1 keeps P
 #pragma unroll
@@ -589,13 +674,13 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
     // ---- Column finals (column j = tid): update coefficients and the readout ---------------
     const int j = tid;
     constexpr int sb16 = SB16;
-    const float cj = pivot ? 1.f : load_scale(tile + C::SOFF, D + j, sb16);
-    const float inv_sig = (j & 1) ? 1.f / C::SIG1 : 1.f;  // powers of two: exact
+    const float cj = pivot ? 1.f : load_scale(tile + W.soff, D + j, sb16);
+    const float inv_sig = (j & 1) ? 1.f / W.sig1 : 1.f;  // powers of two: exact
     {
         // k~Q partials in the half-0 regions (0, 2, 4, 6), q~Q partials in the half-1 regions
         const float U = sum4(sm.red + j, 2 * RS) * inv_sig;
         const float P = sum4(sm.red + RS + j, 2 * RS) * inv_sig;
-        const float sig = (j & 1) ? C::SIG1 : 1.f;
+        const float sig = (j & 1) ? W.sig1 : 1.f;
         const float beta = sm.scal[slot_i][0], alpha = sm.scal[slot_i][1];
         const float vj = load_in<IN_BF16>(tile + C::V_OFF, j);
         const float qk = sm.rsum[pb][0][1] + sm.rsum[pb][1][1] + sm.rsum[pb][2][1] + sm.rsum[pb][3][1];
@@ -695,8 +780,8 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
         // x = sum_i w_i S'_ij^2 / (sum_i w_i c_j^2) (times sigma_j^2), so c'_j = c_j sqrt(x) / sigma_j
         // and the factor taking y to S'_ij / c'_j is 1 / sqrt(x)
         const float E = sum4(sm.red + D + j, 2 * RS);
-        const float W = sm.rsum[pb][0][0] + sm.rsum[pb][1][0] + sm.rsum[pb][2][0] + sm.rsum[pb][3][0];
-        const float x = E * fast_rcp(W);
+        const float wsum = sm.rsum[pb][0][0] + sm.rsum[pb][1][0] + sm.rsum[pb][2][0] + sm.rsum[pb][3][0];
+        const float x = E * fast_rcp(wsum);
         float b = rsqrtf(x);
         float c = (cj * inv_sig) * (x * b);
         if (x == 0.f) {  // zero column: scale 1 (a NaN stays NaN)
@@ -707,7 +792,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
             b = (cj * inv_sig) * fast_rcp(c);
         }
         c_one = c;
-        if (!FIT) store_scale(reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + C::SOFF), D + j, c, sb16);
+        if (!FIT) store_scale(reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + W.soff), D + j, c, sb16);
         if (!isfinite(c) || c == 0.f) flag(p.status, kFlagNonfinite);
         sm.colB[j] = b;
     }
@@ -754,67 +839,41 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
         // v = max_j |sqrt(w_i) S'_ij / c'_j|: r'_i = v / (sqrt(w_i) qmax), and the factor taking
         // z to the code is 1 / (sqrt(w_i) r'_i) = qmax / v
         float r = v * sm.rowRq[pb][i];
-        float s = C::QMAX * fast_rcp(v);
+        float s = W.qmax * fast_rcp(v);
         if (v == 0.f) {  // zero row: scale 1
             r = 1.f;
             s = 0.f;
         } else if (sb16) {  // the codes follow the stored (rounded) scale: s = 1 / (sqrt(w_i) r~_i)
             r = round_scale(r, 1);
-            s = (sm.rowRq[pb][i] * C::QMAX) * fast_rcp(r);
+            s = (sm.rowRq[pb][i] * W.qmax) * fast_rcp(r);
         }
         sm.rowS[i] = make_float2(s, s);
         if constexpr (FIT) {
             r_one = r;
             s_one = s;
-            fitmem<BITS, GATE, IN_BF16, FIT, SB16>(smem).rowRho[i] = r * fast_rcp(sm.rowRq[pb][i] * C::QMAX);  // sqrt(w_i) r_i
+            fitmem<BITS, GATE, IN_BF16, FIT, SB16>(smem).rowRho[i] = r * fast_rcp(sm.rowRq[pb][i] * W.qmax);  // sqrt(w_i) r_i
         } else {
-            store_scale(reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + C::SOFF), i, r, sb16);
+            store_scale(reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + W.soff), i, r, sb16);
         }
         if (!isfinite(r) || r == 0.f) flag(p.status, kFlagNonfinite);
     }
     __syncwarp();
     if constexpr (FIT) {
-        if (!refit_scales<BITS, GATE, IN_BF16, FIT, SB16>(p, sm, smem, n, tcol, c_one, r_one, s_one)) return false;
+        if (!refit_scales<BITS, GATE, IN_BF16, FIT, SB16>(p, sm, smem, n, tcol, W, c_one, r_one, s_one)) return false;
     }
 
     // ---- Sweep D: x = z s rounded half to even by the 2^23 + offset FFMA, packed, stored ----
     tmem_wait_st();
     {
-        const float2 rnd = make_float2(C::ROUND, C::ROUND);
-        uint8_t *dstrow = reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock) + rb * C::RB + cg * BITS;
-        float2 ik[4];  // 1 / K~_j of this thread's columns (refit only)
-        if constexpr (FIT) {
-            load_pairs(sm.colB + 8 * cg, ik);
-#pragma unroll
-            for (int pp = 0; pp < 4; ++pp) ik[pp] = make_float2(fast_rcp(ik[pp].x), fast_rcp(ik[pp].y));
-        }
-        float2 cha[8], chb[8];
-        tmem_ld16_async(tcol, cha);
-        tmem_wait_ld(cha);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            float2 (&ch)[8] = (k & 1) ? chb : cha;
-            float2 (&nx)[8] = (k & 1) ? cha : chb;
-            if (k + 1 < 8) tmem_ld16_async(tcol + 16 * (k + 1), nx);
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int m = 2 * k + r;
-                const float2 s2 = sm.rowS[8 * m + rb];
-#pragma unroll
-                for (int pp = 0; pp < 4; ++pp) {
-                    if constexpr (FIT) {
-                        // x = z / (K~_j rho~_i), clamped (refitted scales may clip), rounded by the add
-                        float2 v = __fmul2_rn(__fmul2_rn(ch[4 * r + pp], ik[pp]), s2);
-                        v.x = fminf(fmaxf(v.x, -C::QMAX), C::QMAX);
-                        v.y = fminf(fmaxf(v.y, -C::QMAX), C::QMAX);
-                        ch[4 * r + pp] = __fadd2_rn(v, rnd);
-                    } else {
-                        ch[4 * r + pp] = __ffma2_rn(ch[4 * r + pp], s2, rnd);
-                    }
-                }
-                pack_store_row<BITS>(dstrow + 8 * m * C::RB, cg, ch + 4 * r);
-            }
-            if (k + 1 < 8) tmem_wait_ld(nx);
+        uint8_t *gblock = reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock);
+        if constexpr (BITS != 0) {
+            sweep_pack<BITS, FIT>(gblock, sm, tcol, rb, cg);
+        } else if (bits == 4) {
+            sweep_pack<4, FIT>(gblock, sm, tcol, rb, cg);
+        } else if (bits == 6) {
+            sweep_pack<6, FIT>(gblock, sm, tcol, rb, cg);
+        } else {
+            sweep_pack<8, FIT>(gblock, sm, tcol, rb, cg);
         }
     }
     return true;
@@ -833,7 +892,6 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
     // tiles) may start as its CTAs find room; see launch_t.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    for (int b = tid; b < p.B; b += NT) sm.slots[b] = p.slots[b];
     if (warp == 0) {  // Tensor Memory for this CTA's tile (released below on every path)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
                      "r"(TMEM_COLS));
@@ -842,8 +900,6 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
     if (tid == 0) {
         for (int i = 0; i < C::NS; ++i) mbar_init(smem_u32(&sm.bars[i]), 2);
         fence_mbar_init();
-        const float o = BITS == 16 ? 0.f : (float)(1 << (BITS - 1));
-        sm.unpack_off = make_float2(-(8388608.0f + o), -(8388608.0f + o * C::SIG1));
         sm.magic = MAGIC;
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -859,6 +915,7 @@ __global__ void __launch_bounds__(NT, 4) decode_d128_kernel(const __grid_constan
         it.b = (int)blockIdx.x - it.pos * p.B;
         it.qG = G / p.B;
         it.rG = G - it.qG * p.B;
+        it.next_slot = my_count > 0 ? p.slots[it.b] : 0;
         for (int k = 0; k < C::NS; ++k) issue_next<BITS, GATE, IN_BF16, FIT, SB16>(p, sm, smem, it, my_count);
     }
     bool failed = __syncthreads_or(!precompute_rows<BITS, GATE, IN_BF16, FIT, SB16>(sm, smem, 0, my_count));
@@ -970,13 +1027,13 @@ cudaError_t launch_modes(const TileParams &p, int in_bf16, cudaStream_t s, bool 
 
 }  // namespace
 
-int decode_d128_max_requests() { return MAXB; }
-
-// All entries of p.table have the width `bits`. p.fit_rounds is 0 or 1 (one round of the joint
-// scale refinement; FP16 pivot heads have no scales and ignore it).
+// bits = 4, 6, 8: every entry of p.table has that width; bits = 0: any mix of 4, 6 and 8 bits;
+// bits = 16: FP16 pivot heads. p.fit_rounds is 0 or 1 (one round of the joint scale refinement;
+// FP16 pivot heads have no scales and ignore it).
 cudaError_t launch_decode_d128(const TileParams &p, int bits, int in_bf16, cudaStream_t s, bool pdl)
 {
     switch (bits) {
+    case 0: return launch_modes<0>(p, in_bf16, s, pdl);
     case 4: return launch_modes<4>(p, in_bf16, s, pdl);
     case 6: return launch_modes<6>(p, in_bf16, s, pdl);
     case 8: return launch_modes<8>(p, in_bf16, s, pdl);

@@ -2,10 +2,14 @@
 // checks, per-launch head tables and kernel dispatch. No device memory is allocated here and no
 // call synchronizes; every launch goes to the caller's stream.
 #include <algorithm>
+#include <cstddef>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <memory>
+#include <mutex>
 #include <new>
+#include <utility>
 #include <vector>
 
 #include "../../include/stq.h"
@@ -16,6 +20,16 @@ namespace stq {
 cudaError_t launch_init_d128(const TileParams &p, cudaStream_t s);
 }  // namespace stq
 
+namespace {
+// The head tables of one decode call (a head range of a layout), built on its first call and
+// reused: the FP16 pivot heads, and the other heads grouped by width.
+struct CallPlan {
+    std::vector<stq::TileEntry> pivots;
+    std::vector<stq::TileEntry> coded;  // the 4/6/8-bit heads, 8-bit first, then 6, then 4
+    int start[3], count[3];             // the 8-, 6- and 4-bit runs of `coded`
+};
+}  // namespace
+
 struct stq_layout {
     int32_t H, dk, dv, gate, in_dtype;
     bool uniform;  // STQ_SCALES_UNIFORM
@@ -25,6 +39,10 @@ struct stq_layout {
     std::vector<uint64_t> offset;
     std::vector<uint64_t> bytes;
     uint64_t req_bytes;
+    // decode plans by (head_begin, head_count); the layout is otherwise immutable and may be
+    // shared between threads, so the cache has its own lock
+    mutable std::mutex plan_mu;
+    mutable std::map<std::pair<int, int>, std::shared_ptr<const CallPlan>> plans;
 };
 
 namespace {
@@ -63,6 +81,45 @@ std::unique_ptr<stq::TileParams> new_params()
     std::unique_ptr<stq::TileParams> p(new (std::nothrow) stq::TileParams);
     if (p) std::memset(p.get(), 0, sizeof(stq::TileParams));
     return p;
+}
+
+// The decode path's parameter block: one per host thread, reused across calls (a launch copies
+// its parameters when it is enqueued). Only the fields before the table are cleared.
+stq::TileParams &thread_params()
+{
+    static thread_local stq::TileParams tp;
+    std::memset(&tp, 0, offsetof(stq::TileParams, table));
+    return tp;
+}
+
+stq::TileEntry entry_of(const stq_layout *L, int h, int h0)
+{
+    stq::TileEntry e;
+    e.off = (uint32_t)L->offset[h];
+    e.info = (uint32_t)(h - h0) | ((uint32_t)L->bits[h] << 16);
+    return e;
+}
+
+// Tables of the tuned decode path for heads [h0, h0 + count): the pivots, and the other heads
+// sorted by width (largest blocks first, head order inside a width).
+std::shared_ptr<const CallPlan> call_plan(const stq_layout *L, int h0, int count)
+{
+    std::lock_guard<std::mutex> lock(L->plan_mu);
+    auto it = L->plans.find({h0, count});
+    if (it != L->plans.end()) return it->second;
+    auto plan = std::make_shared<CallPlan>();
+    static const int widths[3] = {8, 6, 4};
+    for (int h = h0; h < h0 + count; ++h)
+        if (L->bits[h] == 16) plan->pivots.push_back(entry_of(L, h, h0));
+    for (int c = 0; c < 3; ++c) {
+        plan->start[c] = (int)plan->coded.size();
+        for (int h = h0; h < h0 + count; ++h)
+            if (L->bits[h] == widths[c]) plan->coded.push_back(entry_of(L, h, h0));
+        plan->count[c] = (int)plan->coded.size() - plan->start[c];
+    }
+    if (L->plans.size() > 4096) L->plans.clear();  // bounded: head ranges of one model are few
+    L->plans[{h0, count}] = plan;
+    return plan;
 }
 
 }  // namespace
@@ -232,6 +289,71 @@ stq_status stq_decode_step(const stq_layout *L, void *pool, int32_t pool_slots, 
         !aligned(w, 16) || !aligned(beta, 4) || !aligned(o, 16))
         return STQ_ERR_INVALID_ARG;
     if (B > 2147483647 / head_count) return STQ_ERR_UNSUPPORTED;
+    const int in_bf16 = L->in_dtype == STQ_BF16;
+    const size_t in_sz = in_bf16 ? 2 : 4;
+    const int na = L->gate == STQ_GATE_SCALAR ? 1 : L->dk;
+    if (L->dk == 128 && !L->uniform && L->fit_rounds <= 1) {
+        // the tuned kernel (one refit round included): the call's FP16 pivot heads in one launch,
+        // then all its other heads, any mix of widths, in one more (tables of at most kMaxTable
+        // heads each); a launch after the first may overlap the ones before it (disjoint tiles)
+        const std::shared_ptr<const CallPlan> plan = call_plan(L, head_begin, head_count);
+        stq::TileParams &tp = thread_params();
+        tp.pool = static_cast<uint8_t *>(pool);
+        tp.slots = slots;
+        tp.status = dev_status;
+        tp.req_bytes = L->req_bytes;
+        tp.pool_slots = pool_slots;
+        tp.B = B;
+        tp.head_count = head_count;
+        tp.dk = L->dk;
+        tp.dv = L->dv;
+        tp.gate = L->gate;
+        tp.scale_bf16 = L->sb16 ? 1 : 0;
+        tp.fit_rounds = L->fit_rounds;
+        tp.q = q;
+        tp.k = k;
+        tp.v = v;
+        tp.beta = beta;
+        tp.alpha = alpha;
+        tp.w = w;
+        tp.o = o;
+        bool later = false;
+        // Launch the table entries [first, first + n) with width `bits` (0: any mix of 4/6/8).
+        auto launch = [&](const std::vector<stq::TileEntry> &tab, int first0, int n0, int bits) -> bool {
+            for (int first = first0; first < first0 + n0; first += stq::kMaxTable) {
+                const int n = std::min(stq::kMaxTable, first0 + n0 - first);
+                std::memcpy(tp.table, tab.data() + first, sizeof(stq::TileEntry) * (size_t)n);
+                tp.npos = n;
+                tp.ntiles = B * n;
+                if (stq::launch_decode_d128(tp, bits, in_bf16, (cudaStream_t)stream, later) != cudaSuccess)
+                    return false;
+                later = true;
+            }
+            return true;
+        };
+        if (!launch(plan->pivots, 0, (int)plan->pivots.size(), 16)) return STQ_ERR_CUDA;
+        // A launch per width keeps each width's compile-time ring (three slots for 4-bit tiles) but
+        // pays the ring's start and the tail per launch: worth it when every width present has
+        // enough tiles to fill the GPU several times over. Otherwise (the serving shape: one call
+        // per layer) one launch takes every width.
+        static const int widths[3] = {8, 6, 4};
+        constexpr long long kPerWidthTiles = 8192;
+        int present = 0;
+        bool big = true;
+        for (int c = 0; c < 3; ++c)
+            if (plan->count[c] > 0) {
+                ++present;
+                big = big && (long long)plan->count[c] * B >= kPerWidthTiles;
+            }
+        if (present == 1 || big) {
+            for (int c = 0; c < 3; ++c)
+                if (plan->count[c] > 0 && !launch(plan->coded, plan->start[c], plan->count[c], widths[c]))
+                    return STQ_ERR_CUDA;
+        } else if (!launch(plan->coded, 0, (int)plan->coded.size(), 0)) {
+            return STQ_ERR_CUDA;
+        }
+        return STQ_OK;
+    }
     auto p = new_params();
     if (!p) return STQ_ERR_INVALID_ARG;
     p->pool = static_cast<uint8_t *>(pool);
@@ -243,13 +365,9 @@ stq_status stq_decode_step(const stq_layout *L, void *pool, int32_t pool_slots, 
     p->dv = L->dv;
     p->gate = L->gate;
     p->w = w;
-    const int in_bf16 = L->in_dtype == STQ_BF16;
-    const bool tuned = L->dk == 128 && !L->uniform && L->fit_rounds <= 1;  // one refit round runs tuned
-    const int maxb = tuned ? stq::decode_d128_max_requests() : 65535;
+    // the plain kernel (uniform scales, d < 128, two or more refit rounds): any mix of widths
+    const int maxb = 65535;
     const std::vector<int> ord = order_by_size(L, head_begin, head_count);
-    const size_t in_sz = in_bf16 ? 2 : 4;
-    const int na = L->gate == STQ_GATE_SCALAR ? 1 : L->dk;
-    bool later = false;  // a tuned launch of this call already went out: the next ones may overlap it
     for (int b0 = 0; b0 < B; b0 += maxb) {
         const int nb = std::min(maxb, B - b0);
         // requests [b0, b0+nb): shift every per-request array
@@ -262,22 +380,11 @@ stq_status stq_decode_step(const stq_layout *L, void *pool, int32_t pool_slots, 
         p->beta = beta + rq;
         p->alpha = alpha + rq * na;
         p->o = o + rq * L->dv;
-        // the tuned kernel takes one width per launch (largest blocks first); the plain kernel any mix
-        for (int first = 0; first < head_count;) {
-            int n = std::min(stq::kMaxTable, head_count - first);
-            if (tuned) {
-                int same = 1;
-                while (same < n && L->bits[ord[first + same]] == L->bits[ord[first]]) ++same;
-                n = same;
-            }
+        for (int first = 0; first < head_count; first += stq::kMaxTable) {
+            const int n = std::min(stq::kMaxTable, head_count - first);
             fill_table(*p, L, ord, first, n, head_begin);
             p->ntiles = nb * n;
-            const cudaError_t e = tuned ? stq::launch_decode_d128(*p, L->bits[ord[first]], in_bf16,
-                                                                  (cudaStream_t)stream, later)
-                                        : stq::launch_decode_generic(*p, in_bf16, (cudaStream_t)stream);
-            if (e != cudaSuccess) return STQ_ERR_CUDA;
-            later = tuned;
-            first += n;
+            if (stq::launch_decode_generic(*p, in_bf16, (cudaStream_t)stream) != cudaSuccess) return STQ_ERR_CUDA;
         }
     }
     return STQ_OK;

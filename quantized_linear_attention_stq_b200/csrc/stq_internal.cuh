@@ -92,12 +92,11 @@ struct TileParams {
 cudaError_t launch_init_generic(const TileParams &p, cudaStream_t s);
 cudaError_t launch_dequant_generic(const TileParams &p, cudaStream_t s);
 cudaError_t launch_decode_generic(const TileParams &p, int in_bf16, cudaStream_t s);
-// one width per launch; pdl: a later launch of the same call (disjoint tiles) that may overlap the
-// earlier ones
+// bits: the width of every head of the table (4, 6, 8; 16 for FP16 pivots) or 0 for any mix of 4, 6
+// and 8; pdl: a later launch of the same call (disjoint tiles) that may overlap the earlier ones
 cudaError_t launch_decode_d128(const TileParams &p, int bits, int in_bf16, cudaStream_t s, bool pdl);
 cudaError_t launch_prefill_seq(const TileParams &p, int in_bf16, int T, int chunk, cudaStream_t s);
 cudaError_t launch_prefill_wy(const TileParams &p, int bits, int T, cudaStream_t s);  // one width per launch
-int decode_d128_max_requests();
 
 // ------------------------------------------------------------------------------------------
 // Device helpers
