@@ -217,8 +217,8 @@ def _oracle_worker(args):
     n = 0
     for _ in range(reps):
         for i, t in enumerate(tiles):
-            res = orc.decode_step(t["bits"], 0, blocks[i], t["q"], t["k"], t["v"], t["beta"], t["alpha"], t["w"],
-                                  128, 128)
+            res = orc.decode_step(t["bits"], t["gate"], blocks[i], t["q"], t["k"], t["v"], t["beta"], t["alpha"],
+                                  t["w"], t["d"], t["d"])
             blocks[i] = res["block"]
             n += 1
     return n, time.perf_counter() - t0
@@ -245,15 +245,19 @@ def oracle_sample_tiles(workload_name: str, n_tiles: int, seed_offset: int = 0):
     S0 = wlm.initial_state(small, 0).double().numpy()
     w_all = wlm.impact_weights(wl).double().numpy()
     inp = wlm.decode_inputs(small, 0)
-    alpha = wlm.gate_values(wl).double().numpy()
+    alpha = wlm.gate_values(wl).double().numpy()  # [H] or [H, d]
     tiles = []
     for i, h in enumerate(heads):
         b = int(bits_all[h])
         blk, _, _, _ = orc.quantize(b, S0[i], w_all[h])
-        tiles.append(dict(bits=b, block=blk, w=w_all[h], q=inp["q"][0, i].double().numpy(),
+        tiles.append(dict(bits=b, gate=wl.gate, d=wl.d, block=blk, w=w_all[h], q=inp["q"][0, i].double().numpy(),
                           k=inp["k"][0, i].double().numpy(), v=inp["v"][0, i].double().numpy(),
-                          beta=float(inp["beta"][0, i]), alpha=float(alpha[h])))
+                          beta=float(inp["beta"][0, i]), alpha=alpha[h]))
     return tiles
+
+
+# Tiles per oracle process: the bounded sample both the CPU baseline and the reference arm step.
+ORACLE_TILES_PER_WORKER = 16
 
 
 def time_oracle(workload_name: str, workers: int, tiles_per_worker: int, reps: int):
@@ -269,9 +273,20 @@ def time_oracle(workload_name: str, workers: int, tiles_per_worker: int, reps: i
         wall = time.perf_counter() - t0
     n = sum(r[0] for r in res)
     widths = sorted({t["bits"] for s in samples for t in s})
-    sample = (f"{n} head-steps: {workers} processes x {tiles_per_worker} sampled 128x128 tiles of "
+    d = samples[0][0]["d"]
+    sample = (f"{n} head-steps: {workers} processes x {tiles_per_worker} sampled {d}x{d} tiles of "
               f"{workload_name} (widths {widths}) x {reps} decode steps; fp64 C oracle")
     return n / wall, workers, sample
+
+
+def cpu_baseline(workload_name: str, reps: int) -> dict:
+    """The oracle's rate on one core (one process) and on all host cores (one process per core,
+    disjoint tile samples), over the same kind of sample."""
+    rate1, _, sample1 = time_oracle(workload_name, 1, ORACLE_TILES_PER_WORKER, reps)
+    workers = oracle_workers()
+    rate, cores, sample = time_oracle(workload_name, workers, ORACLE_TILES_PER_WORKER, reps)
+    return {"value": rate, "unit": "head-steps/s", "cores": cores, "kind": "oracle", "sample": sample,
+            "single_core": {"value": rate1, "unit": "head-steps/s", "cores": 1, "sample": sample1}}
 
 
 def oracle_workers():
@@ -421,6 +436,117 @@ def prefill_leg(dev, steps: int = 3, warmup: int = 1, T: int = 8192, fit_rounds:
             "tensor_roofline": {"bound": "tensor", "achieved": tflops, "peak": tpeak, "unit": "TFLOP/s",
                                 "frac": tflops / tpeak, "peak_kind": tkind, "flops_per_call": flops,
                                 "note": "algorithmic FLOPs of the five dense contractions per chunk and head"}}
+
+
+L2_BYTES = 126 * 2 ** 20
+
+
+def _decode_generation(stq, wlm, wl, lay, pool, slots, w, dev, steps: int, tok0: int = 0) -> dict:
+    """Time `steps` decode steps of one generation on `pool` (inputs of 8 tokens cycled, resident
+    in HBM): one CUDA event pair around the whole generation, launches included. Reports whether
+    the state stayed finite instead of failing on the device status."""
+    import torch
+
+    B, H, d = wl.batch, wl.heads, wl.d
+    toks = [wlm.decode_inputs(wl, tok0 + t, dev) for t in range(TOKENS_CYCLED)]
+    o = torch.empty(B, H, d, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for t in range(steps):
+        x = toks[t % TOKENS_CYCLED]
+        stq.decode_step(lay, pool, slots, x["q"], x["k"], x["v"], x["beta"], x["alpha"], w, o, status=status,
+                        stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    pool_bytes = B * sum(lay.head_bytes(h) for h in range(H))
+    state_bytes = 2 * pool_bytes
+    gbs = state_bytes / (ms / 1e3) / 1e9
+    flags = stq.status_flags(status)
+    return {"steps": steps, "ms_per_step": ms, "head_steps_per_s": B * H / (ms / 1e3),
+            "tokens_per_s": B / (ms / 1e3), "state_bytes_per_step": state_bytes, "state_gbs": gbs,
+            "gbs_kind": ("effective: the whole pool stays in the 126 MB L2" if pool_bytes <= L2_BYTES
+                         else "HBM: the pool exceeds the L2"),
+            "finite": "non-finite state, scale or output" not in flags, "status": flags}
+
+
+def config_leg(stq, wlm, name: str, dev, fit_rounds: int = 0, steps: int = 0, warmup: int = 3) -> dict:
+    """One of the workloads' own decode configurations: the workload's requests and heads, a full
+    generation of its stated length (or `steps`), after `warmup` untimed steps from the same
+    initial pool."""
+    import torch
+
+    wl = wlm.WORKLOADS[name]
+    B, H, d = wl.batch, wl.heads, wl.d
+    bits = wlm.head_bits(wl)
+    lay = stq.Layout(bits, d, gate=wl.gate, in_dtype=wl.in_dtype, fit_rounds=fit_rounds)
+    pool = lay.alloc_pool(B, dev)
+    slots = torch.arange(B, dtype=torch.int32, device=dev)
+    w = wlm.impact_weights(wl, dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    stq.init_state(lay, pool, slots, torch.stack([wlm.initial_state(wl, r, dev) for r in range(B)]), w, status=st)
+    pristine = pool.clone()
+    _decode_generation(stq, wlm, wl, lay, pool, slots, w, dev, warmup)
+    pool.copy_(pristine)
+    res = _decode_generation(stq, wlm, wl, lay, pool, slots, w, dev, steps or wl.steps)
+    res.update({"workload": name, "requests": B, "heads": H, "d_k": d, "d_v": d,
+                "widths": {str(b): bits.count(b) for b in sorted(set(bits))}, "in_dtype": str(wl.in_dtype),
+                "gate": ("scalar", "channel", "channel_decay_first")[wl.gate], "fit_rounds": fit_rounds})
+    del pool, pristine
+    return res
+
+
+def prefill_then_decode_leg(stq, wlm, dev, decode_steps: int = 0) -> dict:
+    """The prefill workload end to end: the 8192-token prompt in 64-token chunks (one
+    stq_prefill_chunk call), then its stated decode generation on the same pool."""
+    import torch
+
+    wl = wlm.WORKLOADS["prefill16_b16_6bit"]
+    B, H, d, T, C = wl.batch, wl.heads, wl.d, wl.prompt, wl.chunk
+    bits = wlm.head_bits(wl)
+    lay = stq.Layout(bits, d, gate=wl.gate, in_dtype=wl.in_dtype)
+    pool = lay.alloc_pool(B, dev)
+    slots = torch.arange(B, dtype=torch.int32, device=dev)
+    w = wlm.impact_weights(wl, dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    stq.init_state(lay, pool, slots, torch.stack([wlm.initial_state(wl, r, dev) for r in range(B)]), w, status=st)
+    inp = wlm.prefill_inputs(wl, 0, T, dev)
+    o = torch.empty(B, H, T, d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    stq.prefill_chunk(lay, pool, slots, inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], w, o, chunk=C,
+                      status=st, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    pre_ms = e0.elapsed_time(e1)
+    del inp, o
+    dec = _decode_generation(stq, wlm, wl, lay, pool, slots, w, dev, decode_steps or wl.steps, tok0=T)
+    return {"workload": "prefill16_b16_6bit", "requests": B, "heads": H, "d_k": d, "prompt_tokens": T, "chunk": C,
+            "prefill_ms": pre_ms, "prefill_tokens_per_s": B * T / (pre_ms / 1e3),
+            "prefill_finite": "non-finite state, scale or output" not in stq.status_flags(st),
+            "decode": dec}
+
+
+def config_legs(dev, steps: int = 0, warmup: int = 3) -> dict:
+    """Every configuration of the workload set besides the headline step (which the main line
+    measures): the small parity case, one 48-head layer at batch 8, the channel-gate workload over
+    its 2048-step generation (one-pass fit and one refit round), and prefill then decode."""
+    import quantized_linear_attention_stq_b200 as stq
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    out = {}
+    out["pr1_d16_6bit"] = config_leg(stq, wlm, "pr1_d16_6bit", dev, steps=steps, warmup=warmup)
+    out["layer48_b8_4bit"] = config_leg(stq, wlm, "layer48_b8_4bit", dev, steps=steps, warmup=warmup)
+    out["channel32_b128_4bit"] = config_leg(stq, wlm, "channel32_b128_4bit", dev, steps=steps, warmup=warmup)
+    out["channel32_b128_4bit_fit1"] = config_leg(stq, wlm, "channel32_b128_4bit", dev, fit_rounds=1, steps=steps,
+                                                 warmup=warmup)
+    out["prefill16_b16_6bit"] = prefill_then_decode_leg(stq, wlm, dev, decode_steps=steps)
+    return out
 
 
 def run_ours(args):
@@ -586,9 +712,11 @@ def run_ours(args):
     clocks_summary = clocks.summary(t_wall0, t_wall1)
     state_bytes = 2 * sum(lay.head_bytes(h) for h in range(H)) * B  # read + write, one launch
     io_bytes = B * H * (3 * d * (2 if wl.in_dtype == torch.bfloat16 else 4) + 4 * d + 8)
-    # the d = 128 decode launches one kernel per width present (largest blocks first), for every
-    # group of up to 1024 requests; its launches of one step together move `state_bytes`
-    launches_per_step = math.ceil(B / 1024) * sum(math.ceil(bits.count(b) / 3072) for b in set(bits))
+    # the d = 128 decode: one launch for the FP16 pivots, then one per width when every width has
+    # at least 8192 tiles, else one for all widths; together they move `state_bytes`
+    coded = [b for b in set(bits) if b != 16]
+    per_width = all(bits.count(b) * B >= 8192 for b in coded)
+    launches_per_step = (16 in bits) + (len(coded) if per_width else 1)
     step_s_local = total_ms / 1e3 / args.steps
     achieved = state_bytes / step_s_local / 1e9
     peak, peak_kind = measured_peaks()
@@ -625,7 +753,8 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_kind": peak_kind, "traffic": profiled_traffic(),
                      "bytes_per_step": state_bytes, "launches_per_step": launches_per_step,
-                     "kernel": "decode_d128_kernel<width> (one launch per width of the step)",
+                     "kernel": ("decode_d128_kernel<width> (pivots, then one launch per width)" if per_width
+                                else "decode_d128_kernel<width> (pivots, then one launch for all widths)"),
                      "kernel_source_sha256": decode_source_hash()},
         "e2e": {"value": head_steps / (e2e_ms / 1e3 / e2e_steps), "unit": "head-steps/s",
                 "copies": "uploads and readouts on their own streams, overlapping the neighbouring steps",
@@ -643,10 +772,10 @@ def run_ours(args):
         result["config"]["widths_from"] = "lifetime-aware allocation (stq_allocate_widths), same byte budget"
     if world == 1 and not args.no_prefill:
         result["prefill"] = prefill_leg(dev, T=args.prefill_tokens, fit_rounds=args.fit_rounds)
+    if world == 1 and not args.no_configs and args.workload == DEFAULT_WORKLOAD:
+        result["configs"] = config_legs(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not lifetime:
-        rate, cores, sample = time_oracle(args.workload, oracle_workers(), 16, 20)
-        result["cpu_baseline"] = {"value": rate, "unit": "head-steps/s", "cores": cores, "kind": "oracle",
-                                  "sample": sample}
+        result["cpu_baseline"] = cpu_baseline(args.workload, 20)
     elif rank == 0:
         result["cpu_baseline"] = None
     if world > 1:
@@ -661,8 +790,9 @@ def run_reference(args):
     if rank != 0:
         return
     workers = oracle_workers()
-    # one step = one sampled tile per worker; all steps run back to back inside the workers
-    rate, cores, sample = time_oracle(args.workload, workers, 1, max(1, args.steps))
+    # one step = one decode step of ORACLE_TILES_PER_WORKER sampled tiles per worker (the CPU
+    # baseline's sample); all steps run back to back inside the workers
+    rate, cores, sample = time_oracle(args.workload, workers, ORACLE_TILES_PER_WORKER, max(1, args.steps))
     result = {
         "metric": METRIC,
         "impl": "reference",
@@ -671,7 +801,7 @@ def run_reference(args):
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": workers / rate * 1e3,
+        "ms_per_step": workers * ORACLE_TILES_PER_WORKER / rate * 1e3,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -693,6 +823,10 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workload configurations")
+    ap.add_argument("--configs-only", action="store_true",
+                    help="run only the other workload configurations (each for --steps decode steps when "
+                         "given explicitly, else its own generation length; profiling)")
     ap.add_argument("--no-prefill", action="store_true", help="skip the chunked-prefill leg")
     ap.add_argument("--prefill-only", action="store_true", help="run only the chunked-prefill leg (profiling)")
     ap.add_argument("--init-only", action="store_true",
@@ -708,6 +842,12 @@ def main(argv=None):
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.configs_only:
+        import torch
+
+        dev = torch.device("cuda", torch.cuda.current_device())
+        steps = args.steps if any(a.startswith("--steps") for a in (argv if argv is not None else sys.argv[1:])) else 0
+        print(json.dumps({"configs": config_legs(dev, steps=steps, warmup=args.warmup)}), flush=True)
     elif args.prefill_only:
         import torch
 
