@@ -967,25 +967,31 @@ cudaError_t launch_t(const TileParams &p, cudaStream_t s, bool pdl)
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (err != cudaSuccess) return err;
-    int sms = 0, smem_sm = 0, regs_sm = 0;
-    err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
-    if (err != cudaSuccess) return err;
-    cudaFuncAttributes fa;
-    err = cudaFuncGetAttributes(&fa, kernel);
-    if (err != cudaSuccess) return err;
-    // resident CTAs per SM, from shared memory (+1 KB reserved per CTA), registers and the SM's
-    // 512 Tensor Memory columns (TMEM_COLS per CTA); the runtime's occupancy query does not
-    // model Tensor Memory and reports 1 for kernels that allocate it
-    int per_sm = smem_sm / (smem + 1024);
-    const int by_regs = regs_sm / (NT * (fa.numRegs > 0 ? fa.numRegs : 64));
-    if (by_regs < per_sm) per_sm = by_regs;
-    if (per_sm > (int)(512 / TMEM_COLS)) per_sm = (int)(512 / TMEM_COLS);
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    const int grid = p.ntiles < sms * per_sm ? p.ntiles : sms * per_sm;
+    // The launch geometry of this instance on this device, worked out on its first launch there
+    // (per host thread) and reused: resident CTAs per SM from shared memory (+1 KB reserved per
+    // CTA), registers and the SM's 512 Tensor Memory columns (TMEM_COLS per CTA). The runtime's
+    // occupancy query does not model Tensor Memory and reports 1 for kernels that allocate it.
+    static thread_local int cached_dev = -1, cached_cap = 0;
+    if (cached_dev != dev) {
+        err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (err != cudaSuccess) return err;
+        int sms = 0, smem_sm = 0, regs_sm = 0;
+        err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (err == cudaSuccess) err = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+        if (err == cudaSuccess) err = cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+        if (err != cudaSuccess) return err;
+        cudaFuncAttributes fa;
+        err = cudaFuncGetAttributes(&fa, kernel);
+        if (err != cudaSuccess) return err;
+        int per_sm = smem_sm / (smem + 1024);
+        const int by_regs = regs_sm / (NT * (fa.numRegs > 0 ? fa.numRegs : 64));
+        if (by_regs < per_sm) per_sm = by_regs;
+        if (per_sm > (int)(512 / TMEM_COLS)) per_sm = (int)(512 / TMEM_COLS);
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
+        cached_cap = sms * per_sm;
+        cached_dev = dev;
+    }
+    const int grid = p.ntiles < cached_cap ? p.ntiles : cached_cap;
     if (!pdl) {
         kernel<<<grid, NT, smem, s>>>(p);
         return cudaGetLastError();
