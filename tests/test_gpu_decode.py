@@ -154,6 +154,40 @@ def test_many_requests_split_launches(stq, orc):
     _decode_teacher_forced(stq, orc, wl_, [4], 1, slots_perm=False)
 
 
+def test_per_width_launches_equal_one_launch_for_all_widths(stq):
+    """A large call (every width has at least 8192 tiles: one launch per width) and the same
+    requests issued in calls of 2048 requests (one launch for all widths) give the same bytes and
+    readouts, for both scale formats."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    bits = [4, 6, 16, 8]
+    for scale_dtype in (torch.float32, torch.bfloat16):
+        wl_ = _wl("full2304_b70_mixed", batch=8192, heads=len(bits), outliers=False)
+        B, H, d = wl_.batch, wl_.heads, wl_.d
+        lay = stq.Layout(bits, d, gate=wl_.gate, in_dtype=wl_.in_dtype, scale_dtype=scale_dtype)
+        w = wlm.impact_weights(wl_).to(DEV)
+        slots = torch.arange(B, dtype=torch.int32, device=DEV)
+        pool0 = lay.alloc_pool(B)
+        for b0 in range(0, B, 1024):
+            S0 = torch.stack([wlm.initial_state(wl_, r, DEV) for r in range(b0, b0 + 1024)])
+            stq.init_state(lay, pool0, slots[b0:b0 + 1024].clone(), S0, w)
+        g = {n: x.to(DEV) for n, x in wlm.decode_inputs(wl_, 0).items()}
+        status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        pool_a, o_a = pool0.clone(), torch.zeros(B, H, d, device=DEV)
+        stq.decode_step(lay, pool_a, slots, g["q"], g["k"], g["v"], g["beta"], g["alpha"], w, o_a, status=status)
+        pool_b, o_b = pool0.clone(), torch.zeros(B, H, d, device=DEV)
+        for b0 in range(0, B, 2048):
+            sl = slice(b0, b0 + 2048)
+            stq.decode_step(lay, pool_b, slots[sl].contiguous(), g["q"][sl].contiguous(), g["k"][sl].contiguous(),
+                            g["v"][sl].contiguous(), g["beta"][sl].contiguous(), g["alpha"][sl].contiguous(), w,
+                            o_b[sl], status=status)
+        torch.cuda.synchronize()
+        assert status.item() == 0, stq.status_flags(status)
+        assert torch.equal(pool_a, pool_b)
+        assert torch.equal(o_a, o_b)
+        del pool0, pool_a, pool_b
+
+
 def test_back_to_back_calls_without_sync(stq, orc):
     """Two stq_decode_step calls issued back to back on one stream with no synchronization between
     them (mixed widths with pivots and more than 256 requests: several width and request-group
