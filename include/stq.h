@@ -164,7 +164,12 @@ stq_status stq_decode_step(const stq_layout *layout, void *pool, int32_t pool_sl
                            const float *alpha, const float *w, float *o, int32_t *dev_status,
                            void *stream);
 
-/* Workspace bytes stq_prefill_chunk needs for B requests and T tokens in chunks of `chunk`. */
+/* Workspace bytes stq_prefill_chunk can use for B requests and T tokens in chunks of `chunk`.
+ * Nonzero only for the shapes that take the tensor-core chunk form with one plain
+ * requantization per chunk end (128 x 128 heads, bf16 inputs, the scalar gate, chunk == 64, row x
+ * column scales, no refit round) and at least one coded (4/6/8-bit) head: one record of 116736
+ * bytes per request, coded head and chunk of a segment, where the call is cut into segments of at
+ * most 32 chunks, so at most B x coded heads x 32 records whatever T. Host only. */
 size_t stq_prefill_workspace_bytes(const stq_layout *layout, int32_t B, int32_t T, int32_t chunk);
 
 /* Chunked prefill of T tokens for all H heads of B requests, in place. Tokens are cut into
@@ -181,7 +186,15 @@ size_t stq_prefill_workspace_bytes(const stq_layout *layout, int32_t B, int32_t 
  * same chunk-boundary requantization.
  *   w           device fp32 [H][d_k]
  *   o           device fp32 [B][H][T][d_v], written
- *   workspace   device scratch of >= stq_prefill_workspace_bytes(...) bytes, 256-byte aligned
+ *   workspace   device scratch of >= stq_prefill_workspace_bytes(...) bytes, 256-byte aligned, or
+ *               NULL. With a workspace the chunk form runs as three kernels per segment: the
+ *               state-free parts of every chunk in parallel, the state recurrence chunk after
+ *               chunk, then every chunk's readout in parallel; without one it runs as a single
+ *               kernel that keeps everything on chip (slower). The two agree up to the rounding
+ *               order of fp32 sums. A workspace that is given but too small or misaligned is
+ *               STQ_ERR_INVALID_ARG. It is the caller's memory, used on `stream` only and free again
+ *               when the call's work on `stream` is done: calls in flight at the same time need
+ *               separate workspaces.
  * T == 0 or B == 0 is a no-op. */
 stq_status stq_prefill_chunk(const stq_layout *layout, void *pool, int32_t pool_slots,
                              const int32_t *slots, int32_t B, int32_t T, int32_t chunk,

@@ -218,15 +218,19 @@ def prefill_chunk(layout: Layout, pool, slots, q, k, v, beta, alpha, w, o, chunk
     _need(alpha, "alpha", torch.float32, (B, H, T) if layout.gate == GATE_SCALAR else (B, H, T, d), dev)
     _need(w, "w", torch.float32, (H, d), dev)
     _need(o, "o", torch.float32, (B, H, T, d), dev)
+    # with a workspace of prefill_workspace_bytes() the tensor-core chunk form runs as three
+    # kernels (chunk-parallel inputs and readout around the sequential state kernel); without one
+    # it runs as one kernel
     need = prefill_workspace_bytes(layout, B, T, chunk)
-    ws_bytes = 0
-    if need:
-        if workspace is None or workspace.numel() * workspace.element_size() < need:
-            raise ValueError(f"prefill needs a workspace of {need} bytes")
+    ws_ptr, ws_bytes = None, 0
+    if need and workspace is not None:
         ws_bytes = workspace.numel() * workspace.element_size()
+        if ws_bytes < need:
+            raise ValueError(f"prefill workspace of {ws_bytes} bytes is below the {need} bytes it needs")
+        ws_ptr = _ptr(workspace)
     _check(lib().stq_prefill_chunk(layout.handle, _ptr(pool), _pool_slots(layout, pool), _ptr(slots), B, T, chunk,
                                    _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(w), _ptr(o),
-                                   _ptr(workspace) if need else None, ws_bytes, _ptr(status), _stream(stream)),
+                                   ws_ptr, ws_bytes, _ptr(status), _stream(stream)),
            "stq_prefill_chunk")
 
 

@@ -59,6 +59,23 @@ std::vector<int> order_by_size(const stq_layout *L, int h0, int count)
     return ord;
 }
 
+// Prefill shapes that take the tensor-core chunk form: 128 x 128 heads, bf16 inputs, the scalar
+// gate and 64-token chunks (the FP16 pivot heads of such a layout take the token-by-token kernel).
+bool wy_form(const stq_layout *L, int chunk)
+{
+    return L->dk == 128 && L->gate == STQ_GATE_SCALAR && L->in_dtype == STQ_BF16 && chunk == 64 && !L->uniform &&
+           L->fit_rounds <= 1;
+}
+// ... of which those with one plain requantization per chunk end and at least one coded head can
+// run as the three workspace kernels.
+bool ut_form(const stq_layout *L, int chunk)
+{
+    if (!wy_form(L, chunk) || L->fit_rounds != 0) return false;
+    for (int h = 0; h < L->H; ++h)
+        if (L->bits[h] != 16) return true;
+    return false;
+}
+
 // Fill the common fields of a TileParams for heads ord[first .. first+n) of a call.
 void fill_table(stq::TileParams &p, const stq_layout *L, const std::vector<int> &ord, int first, int n, int h0)
 {
@@ -393,7 +410,13 @@ stq_status stq_decode_step(const stq_layout *L, void *pool, int32_t pool_slots, 
 size_t stq_prefill_workspace_bytes(const stq_layout *L, int32_t B, int32_t T, int32_t chunk)
 {
     if (!L || B < 0 || T < 0 || chunk < 1) return 0;
-    return 0;  // the sequential prefill carries its state in shared memory
+    if (!ut_form(L, chunk)) return 0;  // the other kernels carry everything on chip
+    // one record per (request, coded head, chunk of a segment); the widths run one after another
+    int coded = 0;
+    for (int h = 0; h < L->H; ++h) coded += L->bits[h] != 16;
+    const int64_t nch = ((int64_t)T + 63) / 64;
+    const int64_t seg = nch < stq::kUtSegmentChunks ? nch : stq::kUtSegmentChunks;
+    return (size_t)B * (size_t)coded * (size_t)seg * (size_t)stq::kUtRecordBytes;
 }
 
 stq_status stq_prefill_chunk(const stq_layout *L, void *pool, int32_t pool_slots, const int32_t *slots, int32_t B,
@@ -404,8 +427,11 @@ stq_status stq_prefill_chunk(const stq_layout *L, void *pool, int32_t pool_slots
     if (!L || B < 0 || T < 0 || chunk < 1 || pool_slots < 0) return STQ_ERR_INVALID_ARG;
     if (B == 0 || T == 0) return STQ_OK;
     if (!pool || !slots || !q || !k || !v || !beta || !alpha || !w || !o) return STQ_ERR_INVALID_ARG;
+    // a workspace, when given, must hold stq_prefill_workspace_bytes; without one the chunk form
+    // runs as a single kernel
     const size_t need = stq_prefill_workspace_bytes(L, B, T, chunk);
-    if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256))) return STQ_ERR_INVALID_ARG;
+    if (need > 0 && workspace && (workspace_bytes < need || !aligned(workspace, 256))) return STQ_ERR_INVALID_ARG;
+    const bool use_ws = need > 0 && workspace != nullptr;
     if (B > 2147483647 / L->H) return STQ_ERR_UNSUPPORTED;
     if (!aligned(pool, 128) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(w, 16) ||
         !aligned(o, 16) || !aligned(beta, 4) || !aligned(alpha, 4))
@@ -431,10 +457,9 @@ stq_status stq_prefill_chunk(const stq_layout *L, void *pool, int32_t pool_slots
     p->w = w;
     p->o = o;
     // 128 x 128 heads with bf16 inputs, the scalar gate and 64-token chunks take the tensor-core
-    // WY path, one launch per code width; FP16 pivot heads and every other configuration take the
-    // sequential kernel.
-    const bool wy = L->dk == 128 && L->gate == STQ_GATE_SCALAR && L->in_dtype == STQ_BF16 && chunk == 64 &&
-                    !L->uniform && L->fit_rounds <= 1;
+    // chunk form, one width at a time (three kernels around the workspace, or one kernel); FP16
+    // pivot heads and every other configuration take the sequential kernel.
+    const bool wy = wy_form(L, chunk);
     if (!wy) {
         std::vector<int> ord(L->H);
         for (int h = 0; h < L->H; ++h) ord[h] = h;
@@ -450,6 +475,7 @@ stq_status stq_prefill_chunk(const stq_layout *L, void *pool, int32_t pool_slots
         fill_table(*p, L, ord, first, n, 0);
         p->ntiles = B * n;
         const cudaError_t e = bits == 16 ? stq::launch_prefill_seq(*p, 1, T, chunk, (cudaStream_t)stream)
+                              : use_ws   ? stq::launch_prefill_ut(*p, bits, T, workspace, (cudaStream_t)stream)
                                          : stq::launch_prefill_wy(*p, bits, T, (cudaStream_t)stream);
         if (e != cudaSuccess) return STQ_ERR_CUDA;
         first += n;

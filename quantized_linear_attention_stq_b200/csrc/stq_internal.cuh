@@ -97,6 +97,11 @@ cudaError_t launch_decode_generic(const TileParams &p, int in_bf16, cudaStream_t
 cudaError_t launch_decode_d128(const TileParams &p, int bits, int in_bf16, cudaStream_t s, bool pdl);
 cudaError_t launch_prefill_seq(const TileParams &p, int in_bf16, int T, int chunk, cudaStream_t s);
 cudaError_t launch_prefill_wy(const TileParams &p, int bits, int T, cudaStream_t s);  // one width per launch
+// The same chunk form as three kernels around a workspace of ntiles * min(chunks, kUtSegmentChunks)
+// records of kUtRecordBytes (one plain requantization per chunk end; one width per launch).
+constexpr uint64_t kUtRecordBytes = 116736;
+constexpr int kUtSegmentChunks = 32;
+cudaError_t launch_prefill_ut(const TileParams &p, int bits, int T, void *ws, cudaStream_t s);
 
 // ------------------------------------------------------------------------------------------
 // Device helpers

@@ -163,6 +163,34 @@ def test_calls_reject_bad_arguments_before_enqueueing(stq):
     assert L.stq_selftest_wait_timeout(None, None) == 1
 
 
+def test_prefill_workspace_sizes(stq):
+    """The three-kernel prefill asks for one record per (request, coded head, chunk of a segment of
+    at most 32 chunks); the shapes that run as one kernel ask for none. A workspace that is given
+    must be large enough and 256-byte aligned (checked on the host, before any CUDA call)."""
+    SEG = 32
+    bf = torch.bfloat16
+    REC = stq.prefill_workspace_bytes(stq.Layout([6], 128, in_dtype=bf), 1, 64, 64)
+    assert REC > 0 and REC % 1024 == 0
+    lay = stq.Layout([6, 16, 4, 8], 128, in_dtype=bf)
+    assert stq.prefill_workspace_bytes(lay, 3, 64, 64) == 3 * 3 * 1 * REC
+    assert stq.prefill_workspace_bytes(lay, 3, 65, 64) == 3 * 3 * 2 * REC
+    assert stq.prefill_workspace_bytes(lay, 2, 8192, 64) == 2 * 3 * SEG * REC
+    assert stq.prefill_workspace_bytes(lay, 0, 64, 64) == 0
+    assert stq.prefill_workspace_bytes(lay, 3, 0, 64) == 0
+    assert stq.prefill_workspace_bytes(lay, 3, 64, 32) == 0
+    for other in (stq.Layout([6, 4], 128, in_dtype=torch.float32), stq.Layout([6, 4], 64, in_dtype=bf),
+                  stq.Layout([6, 4], 128, gate=1, in_dtype=bf), stq.Layout([6, 4], 128, in_dtype=bf, fit_rounds=1),
+                  stq.Layout([16, 16], 128, in_dtype=bf)):
+        assert stq.prefill_workspace_bytes(other, 3, 640, 64) == 0
+    L = stq.lib()
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    need = stq.prefill_workspace_bytes(lay, 3, 64, 64)
+    args = (lay.handle, fake, 4, fake, 3, 64, 64, fake, fake, fake, fake, fake, fake, fake)
+    assert L.stq_prefill_chunk(*args, P(0x1000000), need - 1, None, None) == 1
+    assert L.stq_prefill_chunk(*args, P(0x1000080), need, None, None) == 1
+
+
 def test_python_binding_checks_shapes(stq):
     lay = stq.Layout([4, 4], 128)
     pool = torch.zeros(lay.bytes_per_request, dtype=torch.uint8)

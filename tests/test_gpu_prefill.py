@@ -72,8 +72,18 @@ def _check_chunk(orc, opool, gp, og, bits, d, B, inp, T, w, gate, tally):
                 compare_o(og[r, h, t], res["o"][t], tally, f"token {t} " + what)
 
 
+def _workspace(stq, lay, B, T, C, form):
+    """The three-kernel form gets a workspace of the size the library asks for; the one-kernel form
+    gets none."""
+    if form == "one_kernel":
+        return None
+    n = stq.prefill_workspace_bytes(lay, B, T, C)
+    return torch.empty(max(n, 1), dtype=torch.uint8, device=DEV)
+
+
+@pytest.mark.parametrize("form", ["workspace", "one_kernel"])
 @pytest.mark.parametrize("T", [64, 37, 1])
-def test_single_chunk_teacher_forced(stq, orc, T):
+def test_single_chunk_teacher_forced(stq, orc, T, form):
     from quantized_linear_attention_stq_b200 import workloads as wlm
 
     bits = [6, 4, 8, 16]
@@ -85,8 +95,8 @@ def test_single_chunk_teacher_forced(stq, orc, T):
     slots = torch.arange(B, dtype=torch.int32, device=DEV)
     o = torch.zeros(B, len(bits), T, d, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
-    ws_n = stq.prefill_workspace_bytes(lay, B, T, 64)
-    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=DEV)
+    ws = _workspace(stq, lay, B, T, 64, form)
+    assert form == "one_kernel" or stq.prefill_workspace_bytes(lay, B, T, 64) > 0
     stq.prefill_chunk(lay, gpool, slots, *(inp[n].to(DEV) for n in ("q", "k", "v", "beta", "alpha")), w.to(DEV), o,
                       chunk=64, workspace=ws, status=status)
     torch.cuda.synchronize()
@@ -156,7 +166,8 @@ def test_channel_gate_multi_chunk_equals_single_chunk_calls(stq, orc, gate):
     assert torch.equal(o_full, torch.cat(outs, dim=2))
 
 
-def test_multi_chunk_equals_single_chunk_calls(stq, orc):
+@pytest.mark.parametrize("form", ["workspace", "one_kernel"])
+def test_multi_chunk_equals_single_chunk_calls(stq, orc, form):
     from quantized_linear_attention_stq_b200 import workloads as wlm
 
     bits = [6, 8, 4]
@@ -166,7 +177,7 @@ def test_multi_chunk_equals_single_chunk_calls(stq, orc):
     inp = {n: x.to(DEV) for n, x in wlm.prefill_inputs(wl_, 0, T).items()}
     slots = torch.tensor([1, 0], dtype=torch.int32, device=DEV)
     wd = w.to(DEV)
-    ws = torch.empty(max(stq.prefill_workspace_bytes(lay, B, T, C), 1), dtype=torch.uint8, device=DEV)
+    ws = _workspace(stq, lay, B, T, C, form)
     p_full = torch.from_numpy(opool.copy()).to(DEV)
     o_full = torch.zeros(B, 3, T, d, device=DEV)
     stq.prefill_chunk(lay, p_full, slots, inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], wd, o_full,
@@ -185,7 +196,45 @@ def test_multi_chunk_equals_single_chunk_calls(stq, orc):
     assert torch.equal(o_full, torch.cat(outs, dim=2))
 
 
-def test_full_geometry_chunk_chain_and_sampled_first_chunk(stq, orc):
+def test_segments_equal_single_chunk_calls(stq, orc):
+    """A three-kernel call over more than one segment of workspace records (34 chunks, the last one
+    short; mixed widths with an FP16 pivot) equals the same chunks issued one call each, bit for
+    bit, and its status stays clear."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    bits = [6, 16, 4, 8]
+    B, d, C = 2, 128, 64
+    T = 33 * C + 10
+    wl_, w, opool = _setup(orc, B, bits)
+    lay = stq.Layout(bits, d, in_dtype=torch.bfloat16)
+    inp = {n: x.to(DEV) for n, x in wlm.prefill_inputs(wl_, 0, T).items()}
+    slots = torch.tensor([1, 0], dtype=torch.int32, device=DEV)
+    wd = w.to(DEV)
+    rec = stq.prefill_workspace_bytes(stq.Layout([6], d, in_dtype=torch.bfloat16), 1, C, C)
+    assert stq.prefill_workspace_bytes(lay, B, T, C) == B * 3 * 32 * rec  # two segments: 32 + 2 chunks
+    ws = _workspace(stq, lay, B, T, C, "workspace")
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    p_full = torch.from_numpy(opool.copy()).to(DEV)
+    o_full = torch.zeros(B, len(bits), T, d, device=DEV)
+    stq.prefill_chunk(lay, p_full, slots, inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], wd, o_full,
+                      chunk=C, workspace=ws, status=status)
+    p_seq = torch.from_numpy(opool.copy()).to(DEV)
+    outs = []
+    for c0 in range(0, T, C):
+        sl = slice(c0, min(c0 + C, T))
+        part = {n: x[:, :, sl].contiguous() for n, x in inp.items()}
+        o_part = torch.zeros(B, len(bits), sl.stop - sl.start, d, device=DEV)
+        stq.prefill_chunk(lay, p_seq, slots, part["q"], part["k"], part["v"], part["beta"], part["alpha"], wd, o_part,
+                          chunk=C, workspace=ws, status=status)
+        outs.append(o_part)
+    torch.cuda.synchronize()
+    assert status.item() == 0, stq.status_flags(status)
+    assert torch.equal(p_full, p_seq)
+    assert torch.equal(o_full, torch.cat(outs, dim=2))
+
+
+@pytest.mark.parametrize("form", ["workspace", "one_kernel"])
+def test_full_geometry_chunk_chain_and_sampled_first_chunk(stq, orc, form):
     """The 16-request x 16-head, 6-bit prefill workload in its bench launch shape (all tiles in
     one launch, more tiles than SMs), over 4 chunks: the multi-chunk call equals the chain of
     single-chunk calls bit for bit, and sampled tiles match the oracle on the first chunk."""
@@ -204,7 +253,7 @@ def test_full_geometry_chunk_chain_and_sampled_first_chunk(stq, orc):
     inp = {n: x.to(DEV) for n, x in wlm.prefill_inputs(wl, 0, T).items()}
     slots = torch.arange(B, dtype=torch.int32, device=DEV)
     wd = w.to(DEV)
-    ws = torch.empty(1, dtype=torch.uint8, device=DEV)
+    ws = _workspace(stq, lay, B, T, C, form)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     p_full = torch.from_numpy(opool.copy()).to(DEV)
     o_full = torch.zeros(B, H, T, d, device=DEV)
