@@ -202,6 +202,33 @@ stq_status stq_prefill_chunk(const stq_layout *layout, void *pool, int32_t pool_
                              const float *alpha, const float *w, float *o, void *workspace,
                              size_t workspace_bytes, int32_t *dev_status, void *stream);
 
+/* stq_prefill_chunk for callers that cannot allocate device memory, with the workspace in memory
+ * the library owns. It has no counterpart in the paper: the method says nothing about where
+ * scratch memory comes from; this call only moves the workspace into the library.
+ * Who needs it: a caller that may not allocate on this path - a serving loop whose device memory
+ * is fixed at start-up and handed out by its own pool, a plug-in or embedding host that gives this
+ * library no allocator, or code that must not call cudaMalloc / cudaFree because they can block
+ * until the whole device is idle and so stall every other stream.
+ * The records live in one fixed device array of 33554432 bytes (32 MiB), defined in the library
+ * and created with it on each device; the call allocates nothing, on the device or the host. It
+ * fits the segments to the array: segments of min(32, 32 MiB / (B * m * 116736)) chunks, where m
+ * is the largest number of heads of one code width; if one chunk of one width does not fit
+ * (B * m * 116736 > 32 MiB, for example more than 287 requests of one 4-bit head) the call returns
+ * STQ_ERR_UNSUPPORTED before any device work (use stq_prefill_chunk with a workspace instead).
+ * Nothing in the array has to start at zero: every record a call reads is written earlier in the
+ * same call. All calls on a device share the one array, so calls whose device work overlaps (on
+ * different streams, or from different host threads) race on it and give wrong results; keep
+ * them on one stream or order them. The first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress) and keeps it for later calls. Shapes without a workspace form
+ * run exactly as stq_prefill_chunk with workspace == NULL. Arguments, results and errors are
+ * otherwise those of stq_prefill_chunk; results equal stq_prefill_chunk with a workspace bit for
+ * bit (segment length changes no arithmetic). */
+stq_status stq_prefill_chunk_noalloc(const stq_layout *layout, void *pool, int32_t pool_slots,
+                                     const int32_t *slots, int32_t B, int32_t T, int32_t chunk,
+                                     const void *q, const void *k, const void *v, const float *beta,
+                                     const float *alpha, const float *w, float *o, int32_t *dev_status,
+                                     void *stream);
+
 /* Dequantize the pool into fp32: S_out[b][h][i][j] = fp32(r_i c_j) * Q_ij (the fp16 value for a
  * pivot head).  S_out device fp32 [B][H][d_k][d_v]. */
 stq_status stq_dequantize(const stq_layout *layout, const void *pool, int32_t pool_slots,

@@ -7,5 +7,6 @@ All computation is in ``libstq.so`` (hand-written CUDA for sm_100a, C ABI in inc
 """
 from .api import (GATE_CHANNEL, GATE_CHANNEL_DECAY_FIRST, GATE_SCALAR, SCALES_ROW_COLUMN, SCALES_UNIFORM,  # noqa: F401
                   Layout, StqError,
-                  allocate_widths, decode_step, dequantize, init_state, lib, prefill_chunk, prefill_workspace_bytes,
+                  allocate_widths, decode_step, dequantize, init_state, lib, prefill_chunk, prefill_chunk_noalloc,
+                  prefill_workspace_bytes,
                   row_impact, selftest_wait_timeout, status_flags, status_string)

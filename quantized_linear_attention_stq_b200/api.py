@@ -28,7 +28,8 @@ EXPORTS = (
     "stq_abi_version", "stq_status_string", "stq_layout_create", "stq_layout_destroy",
     "stq_layout_bytes_per_request", "stq_layout_head_offset", "stq_layout_head_bytes",
     "stq_layout_head_bits", "stq_init_state", "stq_decode_step", "stq_prefill_workspace_bytes",
-    "stq_prefill_chunk", "stq_dequantize", "stq_allocate_widths", "stq_row_impact", "stq_selftest_wait_timeout",
+    "stq_prefill_chunk", "stq_prefill_chunk_noalloc", "stq_dequantize", "stq_allocate_widths", "stq_row_impact",
+    "stq_selftest_wait_timeout",
 )
 
 
@@ -76,6 +77,8 @@ def lib() -> ctypes.CDLL:
             L.stq_prefill_workspace_bytes.restype = sz
             L.stq_prefill_chunk.argtypes = [P, P, i32, P, i32, i32, i32, P, P, P, P, P, P, P, P, sz, P, P]
             L.stq_prefill_chunk.restype = i32
+            L.stq_prefill_chunk_noalloc.argtypes = [P, P, i32, P, i32, i32, i32, P, P, P, P, P, P, P, P, P]
+            L.stq_prefill_chunk_noalloc.restype = i32
             L.stq_dequantize.argtypes = [P, P, i32, P, i32, P, P, P]
             L.stq_dequantize.restype = i32
             L.stq_allocate_widths.argtypes = [i32, i32, P, P, i32, ctypes.c_uint64, P]
@@ -232,6 +235,26 @@ def prefill_chunk(layout: Layout, pool, slots, q, k, v, beta, alpha, w, o, chunk
                                    _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(w), _ptr(o),
                                    ws_ptr, ws_bytes, _ptr(status), _stream(stream)),
            "stq_prefill_chunk")
+
+
+def prefill_chunk_noalloc(layout: Layout, pool, slots, q, k, v, beta, alpha, w, o, chunk: int = 64, status=None,
+                          stream=None):
+    """prefill_chunk for callers that cannot allocate device memory: the workspace is a fixed
+    32 MiB array inside the library (see stq_prefill_chunk_noalloc in include/stq.h); calls whose
+    device work overlaps race on it."""
+    B, H, T, d = q.shape
+    dev = pool.device
+    _need(slots, "slots", torch.int32, (B,), dev)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, layout.in_dtype, (B, H, T, d), dev)
+    _need(beta, "beta", torch.float32, (B, H, T), dev)
+    _need(alpha, "alpha", torch.float32, (B, H, T) if layout.gate == GATE_SCALAR else (B, H, T, d), dev)
+    _need(w, "w", torch.float32, (H, d), dev)
+    _need(o, "o", torch.float32, (B, H, T, d), dev)
+    _check(lib().stq_prefill_chunk_noalloc(layout.handle, _ptr(pool), _pool_slots(layout, pool), _ptr(slots), B, T,
+                                           chunk, _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(w), _ptr(o),
+                                           _ptr(status), _stream(stream)),
+           "stq_prefill_chunk_noalloc")
 
 
 def dequantize(layout: Layout, pool, slots, S_out, status=None, stream=None):

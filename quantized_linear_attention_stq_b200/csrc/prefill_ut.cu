@@ -944,7 +944,39 @@ cudaError_t launch_ut(const TileParams &p, int T, uint8_t *ws, cudaStream_t s)
     return cudaSuccess;
 }
 
+// The same with segments of at most `seg` chunks (the workspace holds ntiles * seg records).
+template <int BITS>
+cudaError_t launch_ut_seg(const TileParams &p, int T, uint8_t *ws, int seg, cudaStream_t s)
+{
+    int dev = 0, sms = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+    const int nch = (T + C - 1) / C;
+    for (int c0 = 0; c0 < nch; c0 += seg) {
+        const int nsc = nch - c0 < seg ? nch - c0 : seg;
+        const UtArgs a{ws, T, c0, nsc};
+        if ((err = launch_one(ut_inputs_kernel, P1_SMEM, p.ntiles * nsc, sms, p, a, s)) != cudaSuccess) return err;
+        if ((err = launch_one(ut_state_kernel<BITS>, P2_SMEM, p.ntiles, sms, p, a, s)) != cudaSuccess) return err;
+        if ((err = launch_one(ut_readout_kernel<BITS>, P3_SMEM, p.ntiles * nsc, sms, p, a, s)) != cudaSuccess)
+            return err;
+    }
+    return cudaSuccess;
+}
+
 }  // namespace
+
+cudaError_t launch_prefill_ut_seg(const TileParams &p, int bits, int T, void *ws, int seg, cudaStream_t s)
+{
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    if (seg < 1) return cudaErrorInvalidValue;
+    switch (bits) {
+    case 4: return launch_ut_seg<4>(p, T, w, seg, s);
+    case 6: return launch_ut_seg<6>(p, T, w, seg, s);
+    case 8: return launch_ut_seg<8>(p, T, w, seg, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
 
 // Chunked prefill of 128 x 128 tiles (bf16 inputs, scalar gate, 64-token chunks, one plain
 // requantization per chunk end) through the workspace; every entry of p.table has width `bits`.

@@ -141,6 +141,29 @@ std::shared_ptr<const CallPlan> call_plan(const stq_layout *L, int h0, int count
 
 }  // namespace
 
+// The workspace of stq_prefill_chunk_noalloc: one fixed array per device, part of this library's
+// module. The host-side name is only a handle; its device address comes from cudaGetSymbolAddress.
+constexpr size_t kNoallocScratchBytes = (size_t)32 << 20;
+static __device__ __align__(256) uint8_t stq_noalloc_scratch[kNoallocScratchBytes];
+
+namespace {
+// The array's device address on the current device, looked up on the first call per device and
+// kept (no allocation: a fixed table for the first 64 device ordinals).
+void *noalloc_scratch()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    static std::mutex mu;
+    static void *addr[64] = {};
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < 64 && addr[dev]) return addr[dev];
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, stq_noalloc_scratch) != cudaSuccess) return nullptr;
+    if (dev >= 0 && dev < 64) addr[dev] = ptr;
+    return ptr;
+}
+}  // namespace
+
 extern "C" {
 
 int32_t stq_abi_version(void) { return STQ_ABI_VERSION; }
@@ -479,6 +502,72 @@ stq_status stq_prefill_chunk(const stq_layout *L, void *pool, int32_t pool_slots
                                          : stq::launch_prefill_wy(*p, bits, T, (cudaStream_t)stream);
         if (e != cudaSuccess) return STQ_ERR_CUDA;
         first += n;
+    }
+    return STQ_OK;
+}
+
+stq_status stq_prefill_chunk_noalloc(const stq_layout *L, void *pool, int32_t pool_slots, const int32_t *slots,
+                                     int32_t B, int32_t T, int32_t chunk, const void *q, const void *k,
+                                     const void *v, const float *beta, const float *alpha, const float *w, float *o,
+                                     int32_t *dev_status, void *stream)
+{
+    if (!L || B < 0 || T < 0 || chunk < 1 || pool_slots < 0) return STQ_ERR_INVALID_ARG;
+    if (B == 0 || T == 0) return STQ_OK;
+    if (!ut_form(L, chunk))  // these shapes keep everything on chip: nothing to stage
+        return stq_prefill_chunk(L, pool, pool_slots, slots, B, T, chunk, q, k, v, beta, alpha, w, o, nullptr, 0,
+                                 dev_status, stream);
+    if (!pool || !slots || !q || !k || !v || !beta || !alpha || !w || !o) return STQ_ERR_INVALID_ARG;
+    if (B > 2147483647 / L->H) return STQ_ERR_UNSUPPORTED;
+    if (!aligned(pool, 128) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(w, 16) ||
+        !aligned(o, 16) || !aligned(beta, 4) || !aligned(alpha, 4))
+        return STQ_ERR_INVALID_ARG;
+    if (L->H > stq::kMaxTable) return STQ_ERR_UNSUPPORTED;
+    // one width at a time: the widest class sets how many chunks a segment of records can hold
+    int count[3] = {0, 0, 0};
+    static const int widths[3] = {8, 6, 4};
+    for (int h = 0; h < L->H; ++h)
+        for (int c = 0; c < 3; ++c) count[c] += L->bits[h] == widths[c];
+    const uint64_t most = (uint64_t)std::max(count[0], std::max(count[1], count[2]));
+    const uint64_t per_chunk = (uint64_t)B * most * stq::kUtRecordBytes;
+    if (per_chunk > kNoallocScratchBytes) return STQ_ERR_UNSUPPORTED;
+    const uint64_t fit = kNoallocScratchBytes / per_chunk;
+    const int seg = fit < (uint64_t)stq::kUtSegmentChunks ? (int)fit : stq::kUtSegmentChunks;
+    void *scratch = noalloc_scratch();
+    if (!scratch) return STQ_ERR_CUDA;
+
+    stq::TileParams &tp = thread_params();
+    tp.pool = static_cast<uint8_t *>(pool);
+    tp.slots = slots;
+    tp.status = dev_status;
+    tp.req_bytes = L->req_bytes;
+    tp.pool_slots = pool_slots;
+    tp.B = B;
+    tp.head_count = L->H;
+    tp.dk = L->dk;
+    tp.dv = L->dv;
+    tp.gate = L->gate;
+    tp.scale_bf16 = L->sb16 ? 1 : 0;
+    tp.fit_rounds = L->fit_rounds;
+    tp.q = q;
+    tp.k = k;
+    tp.v = v;
+    tp.beta = beta;
+    tp.alpha = alpha;
+    tp.w = w;
+    tp.o = o;
+    // FP16 pivots first (token-by-token kernel), then the 8-, 6- and 4-bit heads, head index order
+    static const int order[4] = {16, 8, 6, 4};
+    for (int c = 0; c < 4; ++c) {
+        int n = 0;
+        for (int h = 0; h < L->H; ++h)
+            if (L->bits[h] == order[c]) tp.table[n++] = entry_of(L, h, 0);
+        if (n == 0) continue;
+        tp.npos = n;
+        tp.ntiles = B * n;
+        const cudaError_t e = order[c] == 16
+                                  ? stq::launch_prefill_seq(tp, 1, T, chunk, (cudaStream_t)stream)
+                                  : stq::launch_prefill_ut_seg(tp, order[c], T, scratch, seg, (cudaStream_t)stream);
+        if (e != cudaSuccess) return STQ_ERR_CUDA;
     }
     return STQ_OK;
 }

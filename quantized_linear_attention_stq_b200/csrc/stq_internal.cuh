@@ -102,6 +102,8 @@ cudaError_t launch_prefill_wy(const TileParams &p, int bits, int T, cudaStream_t
 constexpr uint64_t kUtRecordBytes = 116736;
 constexpr int kUtSegmentChunks = 32;
 cudaError_t launch_prefill_ut(const TileParams &p, int bits, int T, void *ws, cudaStream_t s);
+// ... with segments of at most `seg` chunks (a workspace of ntiles * seg records)
+cudaError_t launch_prefill_ut_seg(const TileParams &p, int bits, int T, void *ws, int seg, cudaStream_t s);
 
 // ------------------------------------------------------------------------------------------
 // Device helpers
