@@ -102,10 +102,10 @@ __device__ __forceinline__ uint8_t *p1_box(uint8_t *sm, int b)
     return b < 2 ? sm + P1_L + 8192 * b : sm + P1_SPL + 8192 * (b - 2);
 }
 
-__global__ void __launch_bounds__(NT3, 2) ut_inputs_kernel(const __grid_constant__ TileParams p, const UtArgs a)
+// The inputs work of one CTA: units first, first + stride, ... of the segment.
+__device__ __forceinline__ void inputs_run(const TileParams &p, const UtArgs &a, uint8_t *sm, const int first,
+                                           const int stride)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = aligned_smem(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, cq = warp >> 2;
     float *sBeta = smf(sm, P1_SMALL + P1S_BETA), *sAlpha = smf(sm, P1_SMALL + P1S_ALPHA);
     float *sGam = smf(sm, P1_SMALL + P1S_GAM), *sInv = smf(sm, P1_SMALL + P1S_INV);
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(NT3, 2) ut_inputs_kernel(const __grid_constant
     };
     int issued = -1;  // the unit whose inputs are in flight
 
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    for (int u = first; u < units && ok; u += stride) {
         const int n = u / a.nsc, cc = u - n * a.nsc;
         const int b = n % p.B, pos = n / p.B;
         const int slot = p.slots[b];
@@ -163,9 +163,9 @@ __global__ void __launch_bounds__(NT3, 2) ut_inputs_kernel(const __grid_constant
         const __nv_bfloat16 *vg = reinterpret_cast<const __nv_bfloat16 *>(p.v) + rowbase * D;
         uint8_t *rec = ut_record(a, n, cc);
 
-        if (tid == 0 && u + (int)gridDim.x < units) {
+        if (tid == 0 && u + stride < units) {
             // the next unit's V rows into L2 while this one computes
-            const int u1 = u + gridDim.x, n1 = u1 / a.nsc, cc1 = u1 - n1 * a.nsc;
+            const int u1 = u + stride, n1 = u1 / a.nsc, cc1 = u1 - n1 * a.nsc;
             const uint64_t tr1 = (uint64_t)(n1 % p.B) * (uint64_t)p.head_count + (uint64_t)entry_head(p.table[n1 / p.B]);
             const int t1 = (a.c0 + cc1) * C, L1 = (a.T - t1) < C ? (a.T - t1) : C;
             l2_prefetch(reinterpret_cast<const __nv_bfloat16 *>(p.v) + (tr1 * (uint64_t)a.T + (uint64_t)t1) * D,
@@ -304,9 +304,9 @@ __global__ void __launch_bounds__(NT3, 2) ut_inputs_kernel(const __grid_constant
         ok = wait_bar(smem_u32(&bars[1]), parity, p.status);
         if (!__syncthreads_and(ok)) break;
         umma::fence_after_sync();
-        if (u + (int)gridDim.x < units) {
-            issue_inputs(u + gridDim.x);  // K / Q and beta / alpha are free once the MMAs are done
-            issued = u + gridDim.x;
+        if (u + stride < units) {
+            issue_inputs(u + stride);  // K / Q and beta / alpha are free once the MMAs are done
+            issued = u + stride;
         }
         {
             const int li = 32 * q4 + lane;  // i for W, j for U_v
@@ -330,6 +330,12 @@ __global__ void __launch_bounds__(NT3, 2) ut_inputs_kernel(const __grid_constant
         umma::fence_after_sync();
         umma::tmem_dealloc(tmem, 256);
     }
+}
+
+__global__ void __launch_bounds__(NT3, 2) ut_inputs_kernel(const __grid_constant__ TileParams p, const UtArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    inputs_run(p, a, aligned_smem(smem_raw), blockIdx.x, gridDim.x);
 }
 
 // =============================================================================================
@@ -741,11 +747,10 @@ constexpr uint32_t P3_SMEM = P3_SMALL + 1312 + 1024;
 constexpr int OST = 132;  // row stride (floats) of the readout staged over the term area
 static_assert(64 * OST * 4 <= 49152, "readout rows fit the term area");
 
-template <int BITS>
-__global__ void __launch_bounds__(NT3, 2) ut_readout_kernel(const __grid_constant__ TileParams p, const UtArgs a)
+// The readout work of one CTA: units first, first + stride, ... of the segment.
+__device__ __forceinline__ void readout_run(const TileParams &p, const UtArgs &a, uint8_t *sm, const int first,
+                                            const int stride)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = aligned_smem(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, cq = warp >> 2;
     float *sR = smf(sm, P3_SMALL + P3S_R), *sC = smf(sm, P3_SMALL + P3S_C), *sGam = smf(sm, P3_SMALL + P3S_GAM);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + P3_SMALL + P3S_BAR);
@@ -767,7 +772,7 @@ __global__ void __launch_bounds__(NT3, 2) ut_readout_kernel(const __grid_constan
     bool ok = true;
     const int units = p.ntiles * a.nsc;
 
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    for (int u = first; u < units && ok; u += stride) {
         const int n = u / a.nsc, cc = u - n * a.nsc;
         const int b = n % p.B, pos = n / p.B;
         const int slot = p.slots[b];
@@ -804,9 +809,9 @@ __global__ void __launch_bounds__(NT3, 2) ut_readout_kernel(const __grid_constan
 #pragma unroll
             for (int k = 0; k < 4; ++k) qraw[k] = t < Lc ? qs[k] : make_uint4(0u, 0u, 0u, 0u);
         }
-        if (tid == 0 && u + (int)gridDim.x < units) {
+        if (tid == 0 && u + stride < units) {
             // the next unit's record and q rows into L2
-            const int u1 = u + gridDim.x, n1 = u1 / a.nsc, cc1 = u1 - n1 * a.nsc;
+            const int u1 = u + stride, n1 = u1 / a.nsc, cc1 = u1 - n1 * a.nsc;
             const uint64_t tr1 = (uint64_t)(n1 % p.B) * (uint64_t)p.head_count + (uint64_t)entry_head(p.table[n1 / p.B]);
             const int t1 = (a.c0 + cc1) * C, L1 = (a.T - t1) < C ? (a.T - t1) : C;
             const uint8_t *r1 = ut_record(a, n1, cc1);
@@ -910,6 +915,13 @@ __global__ void __launch_bounds__(NT3, 2) ut_readout_kernel(const __grid_constan
         umma::fence_after_sync();
         umma::tmem_dealloc(tmem, 128);
     }
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(NT3, 2) ut_readout_kernel(const __grid_constant__ TileParams p, const UtArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    readout_run(p, a, aligned_smem(smem_raw), blockIdx.x, gridDim.x);
 }
 
 template <typename K>
