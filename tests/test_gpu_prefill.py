@@ -290,6 +290,70 @@ def test_full_geometry_chunk_chain_and_sampled_first_chunk(stq, orc, form):
     tally.check_budget()
 
 
+def test_bench_size_call_equals_segment_calls_and_first_chunk_parity(stq, orc):
+    """The bench's prefill in its launch configuration: 16 requests x 16 heads, 6-bit, an
+    8192-token prompt through the workspace (four segments of 32 chunks, 256 tiles in every
+    launch). The whole call equals four 2048-token calls (one segment each) bit for bit, and
+    sampled tiles match the oracle on the call's first chunk."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    wl = wlm.WORKLOADS["prefill16_b16_6bit"]
+    B, H, d, C, T = wl.batch, wl.heads, wl.d, wl.chunk, wl.prompt
+    bits = wlm.head_bits(wl)
+    lay = stq.Layout(bits, d, in_dtype=wl.in_dtype)
+    w = wlm.impact_weights(wl)
+    blocks = []
+    for r in range(B):
+        S0 = wlm.initial_state(wl, r)
+        blocks.append([orc.quantize(bits[h], as_f64(S0[h]), as_f64(w[h]))[0] for h in range(H)])
+    opool = oracle_pool(orc, bits, d, blocks)
+    inp = {n: x.to(DEV) for n, x in wlm.prefill_inputs(wl, 0, T).items()}
+    slots = torch.arange(B, dtype=torch.int32, device=DEV)
+    wd = w.to(DEV)
+    ws = _workspace(stq, lay, B, T, C, "workspace")
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    p_full = torch.from_numpy(opool.copy()).to(DEV)
+    o_full = torch.empty(B, H, T, d, device=DEV)
+    stq.prefill_chunk(lay, p_full, slots, inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], wd, o_full,
+                      chunk=C, workspace=ws, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0, stq.status_flags(status)
+    o_first = o_full[:, :, :C].cpu().numpy()
+    p_seg = torch.from_numpy(opool.copy()).to(DEV)
+    seg = 32 * C
+    for t0 in range(0, T, seg):
+        part = {n: x[:, :, t0:t0 + seg].contiguous() for n, x in inp.items()}
+        o_part = torch.empty(B, H, seg, d, device=DEV)
+        stq.prefill_chunk(lay, p_seg, slots, part["q"], part["k"], part["v"], part["beta"], part["alpha"], wd,
+                          o_part, chunk=C, workspace=ws, status=status)
+        assert torch.equal(o_part, o_full[:, :, t0:t0 + seg]), f"readouts of tokens {t0}.. differ"
+        del o_part, part
+    torch.cuda.synchronize()
+    assert status.item() == 0, stq.status_flags(status)
+    assert torch.equal(p_full, p_seg)
+    # the first chunk of sampled tiles against the oracle, from a one-chunk call's pool
+    p_one = torch.from_numpy(opool.copy()).to(DEV)
+    part = {n: x[:, :, :C].contiguous() for n, x in inp.items()}
+    o_one = torch.empty(B, H, C, d, device=DEV)
+    stq.prefill_chunk(lay, p_one, slots, part["q"], part["k"], part["v"], part["beta"], part["alpha"], wd, o_one,
+                      chunk=C, workspace=ws, status=status)
+    torch.cuda.synchronize()
+    assert torch.equal(o_one.cpu(), torch.from_numpy(o_first))
+    first_pool = p_one.cpu().numpy()
+    cpu_inp = {n: x[:, :, :C].cpu() for n, x in inp.items()}
+    del inp, o_full, ws, p_seg
+    tally = Tally()
+    rng = np.random.default_rng(11)
+    for r, h in zip(rng.integers(0, B, 6), rng.integers(0, H, 6)):
+        res = _oracle_chunk(orc, opool, bits, d, int(r), int(h), cpu_inp, 0, C, w, C)
+        assert res["status"] == orc.OK
+        compare_block(orc, bits[h], d, tile_bytes(orc, first_pool, bits, d, int(r), int(h)), res["block"],
+                      res["tie"], tally, f"req {r} head {h}")
+        for t in range(C):
+            compare_o(o_first[r, h, t], res["o"][t], tally, f"token {t} req {r} head {h}")
+    tally.check_budget()
+
+
 def test_fp32_inputs_sequential_form(stq, orc):
     """fp32 inputs (the sequential kernel) on a short single chunk, teacher forced."""
     from quantized_linear_attention_stq_b200 import workloads as wlm
