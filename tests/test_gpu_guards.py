@@ -46,7 +46,10 @@ def _written_ranges(lay, bits, d, scale_bytes, uniform):
 
 CASES = [
     ("d128 mixed widths, pivots", [4, 6, 8, 16, 6, 4], 128, torch.bfloat16, {}),
+    ("d128 mixed widths, prefill with a workspace", [4, 6, 8, 16, 6, 4], 128, torch.bfloat16, {"ws": True}),
     ("d128 bf16 scales", [4, 6, 8, 16], 128, torch.bfloat16, {"scale_dtype": torch.bfloat16}),
+    ("d128 bf16 scales, prefill with a workspace", [4, 6, 8, 16], 128, torch.bfloat16,
+     {"scale_dtype": torch.bfloat16, "ws": True}),
     ("d128 uniform", [4, 6, 8, 16], 128, torch.bfloat16, {"scale_mode": 1}),
     ("d64 mixed widths", [4, 6, 8, 16], 64, torch.bfloat16, {}),
     ("d16 fp32 inputs", [6, 4, 16], 16, torch.float32, {}),
@@ -55,6 +58,8 @@ CASES = [
 
 @pytest.mark.parametrize("name,bits,d,in_dtype,kw", CASES, ids=[c[0] for c in CASES])
 def test_kernels_write_only_their_head_bytes(stq, name, bits, d, in_dtype, kw):
+    kw = dict(kw)
+    use_ws = kw.pop("ws", False)
     lay = stq.Layout(bits, d, in_dtype=in_dtype, **kw)
     H, B, nslots = len(bits), 3, 4
     R = lay.bytes_per_request
@@ -83,7 +88,11 @@ def test_kernels_write_only_their_head_bytes(stq, name, bits, d, in_dtype, kw):
     beta = torch.sigmoid(torch.randn(B, H, T, generator=g, device=DEV))
     alpha = torch.full((B, H, T), 0.95, device=DEV)
     o = torch.empty(B, H, T, d, device=DEV)
-    stq.prefill_chunk(lay, pool, slots, q, k, v, beta, alpha, w, o, chunk=64, status=status)
+    ws = None
+    if use_ws:  # the three-kernel form; its workspace lies outside the guarded buffer
+        assert stq.prefill_workspace_bytes(lay, B, T, 64) > 0
+        ws = torch.empty(stq.prefill_workspace_bytes(lay, B, T, 64), dtype=torch.uint8, device=DEV)
+    stq.prefill_chunk(lay, pool, slots, q, k, v, beta, alpha, w, o, chunk=64, workspace=ws, status=status)
     out = torch.empty(B, H, d, d, device=DEV)
     stq.dequantize(lay, pool, slots, out, status=status)
     torch.cuda.synchronize()

@@ -186,12 +186,13 @@ def test_decode_small_heads(stq, orc, d):
     _decode_teacher_forced(stq, orc, wl_, [4, 6, 8, 16, 6], 3)
 
 
-@pytest.mark.parametrize("d,in_dtype,T", [(128, torch.bfloat16, 64), (32, torch.float32, 64),
-                                          (128, torch.bfloat16, 40)])
-def test_prefill_chunk(stq, orc, d, in_dtype, T):
+@pytest.mark.parametrize("d,in_dtype,T,ws", [(128, torch.bfloat16, 64, False), (32, torch.float32, 64, False),
+                                             (128, torch.bfloat16, 40, False), (128, torch.bfloat16, 64, True),
+                                             (128, torch.bfloat16, 40, True)])
+def test_prefill_chunk(stq, orc, d, in_dtype, T, ws):
     """One chunk per call, twice in a row, teacher-forced: 128 x 128 heads with bf16 inputs and
-    64-token chunks take the tensor-core path, the others the sequential kernel; a 40-token call
-    is a short last chunk."""
+    64-token chunks take the tensor-core path (with a workspace: the three-kernel form; without:
+    one kernel), the others the sequential kernel; a 40-token call is a short last chunk."""
     from quantized_linear_attention_stq_b200 import workloads as wlm
 
     bits = [4, 6, 8, 16]
@@ -207,9 +208,11 @@ def test_prefill_chunk(stq, orc, d, in_dtype, T):
         inp = wlm.prefill_inputs(wl_, call * T, T)
         pool = torch.from_numpy(opool.copy()).to(DEV)
         o = torch.zeros(2, 4, T, d, device=DEV)
+        wsb = torch.empty(stq.prefill_workspace_bytes(lay, 2, T, 64), dtype=torch.uint8, device=DEV) if ws else None
+        assert not ws or wsb.numel() > 0
         stq.prefill_chunk(lay, pool, torch.arange(2, dtype=torch.int32, device=DEV),
                           *(inp[n].to(DEV) for n in ("q", "k", "v", "beta", "alpha")), w.to(DEV), o, chunk=64,
-                          status=status)
+                          workspace=wsb, status=status)
         torch.cuda.synchronize()
         assert status.item() == 0, stq.status_flags(status)
         gp, og = pool.cpu().numpy(), o.cpu().numpy()
