@@ -102,7 +102,28 @@ __device__ __forceinline__ uint8_t *p1_box(uint8_t *sm, int b)
     return b < 2 ? sm + P1_L + 8192 * b : sm + P1_SPL + 8192 * (b - 2);
 }
 
-// The inputs work of one CTA: units first, first + stride, ... of the segment.
+// W^T and U_v^T of a finished unit (Tensor Memory columns 64..191) to its record: lane li = i for
+// W and j for U_v, tokens [t0, t0 + 32 * nq) in nq blocks of 32. W leaves row-major [t][i] (a
+// warp writes whole 128-byte rows), U_v^T row-major [j][t].
+__device__ __forceinline__ void inputs_readback(uint8_t *rec, uint32_t tl, int li, int t0, int nq)
+{
+    float *wg = reinterpret_cast<float *>(rec + REC_W);
+    for (int b = 0; b < nq; ++b) {
+        const int tb = t0 + 32 * b;
+        float v[32];
+        umma::tmem_ld32(tl + 64 + tb, v);  // W^T[i][t = tb + e]
+#pragma unroll
+        for (int e = 0; e < 32; ++e) wg[(tb + e) * D + li] = v[e];
+        umma::tmem_ld32(tl + 128 + tb, v);  // U_v^T[j][t]
+        float4 *ug = reinterpret_cast<float4 *>(rec + REC_UV + (size_t)(li * C + tb) * 4);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ug[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+    }
+}
+
+// The inputs work of one CTA: units first, first + stride, ... of the segment. A unit's W and U_v
+// stay in Tensor Memory until the next unit's inverse, during which warps 0..3 (idle then) write
+// them out; the last unit's go out after the loop.
 __device__ __forceinline__ void inputs_run(const TileParams &p, const UtArgs &a, uint8_t *sm, const int first,
                                            const int stride)
 {
@@ -149,7 +170,8 @@ __device__ __forceinline__ void inputs_run(const TileParams &p, const UtArgs &a,
         }
         cp_async_commit();
     };
-    int issued = -1;  // the unit whose inputs are in flight
+    int issued = -1;           // the unit whose inputs are in flight
+    uint8_t *pending = nullptr;  // the record whose W / U_v still sit in Tensor Memory
 
     for (int u = first; u < units && ok; u += stride) {
         const int n = u / a.nsc, cc = u - n * a.nsc;
@@ -254,7 +276,13 @@ __device__ __forceinline__ void inputs_run(const TileParams &p, const UtArgs &a,
 
         load_rows_async(sm + P1_KQ + KQ_Q0, sm + P1_KQ + KQ_Q1, vg, Lc);
         cp_async_commit();
-        if (warp >= 4) invert_unit_lower<4>(Lm, Tm);
+        if (warp >= 4) {
+            invert_unit_lower<4>(Lm, Tm);
+        } else if (pending) {
+            inputs_readback(pending, tl, 32 * q4 + lane, 0, 2);  // the previous unit, all 64 tokens
+            umma::fence_before_sync();
+        }
+        pending = nullptr;
         cp_async_wait_all();
         umma::fence_proxy_async();
         __syncthreads();  // T is complete and V has landed
@@ -308,20 +336,12 @@ __device__ __forceinline__ void inputs_run(const TileParams &p, const UtArgs &a,
             issue_inputs(u + stride);  // K / Q and beta / alpha are free once the MMAs are done
             issued = u + stride;
         }
-        {
-            const int li = 32 * q4 + lane;  // i for W, j for U_v
-            float v[32];
-            umma::tmem_ld32(tl + 64 + 32 * cq, v);  // W^T[i][t = 32 cq + e]
-            float *wg = reinterpret_cast<float *>(rec + REC_W);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) wg[(32 * cq + e) * D + li] = v[e];
-            umma::tmem_ld32(tl + 128 + 32 * cq, v);  // U_v^T[j][t]
-            float4 *ug = reinterpret_cast<float4 *>(rec + REC_UV + (size_t)(li * C + 32 * cq) * 4);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) ug[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-        }
-        umma::fence_before_sync();
+        pending = rec;
         parity ^= 1u;
+    }
+    if (ok && pending) {  // the last unit's W / U_v, on all eight warps
+        inputs_readback(pending, tl, 32 * q4 + lane, 32 * cq, 1);
+        umma::fence_before_sync();
     }
     cp_async_wait_all();
     umma::fence_before_sync();
