@@ -630,13 +630,18 @@ __global__ void __launch_bounds__(NT3, 2) ut_state_kernel(const __grid_constant_
                 // w_i S_ij^2 summed over the warp's 32 rows by a butterfly that leaves lane l with
                 // columns 2l and 2l + 1 of this thread's 64
                 const float wi = sW[i];
+                const float2 wi2 = make_float2(wi, wi);
                 float a1[32];
                 {
                     const bool up = (lane & 16) != 0;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float lo = (wi * S[e]) * S[e], hi = (wi * S[e + 32]) * S[e + 32];
-                        a1[e] = (up ? hi : lo) + __shfl_xor_sync(0xffffffffu, up ? lo : hi, 16);
+                    for (int e = 0; e < 32; e += 2) {
+                        // (w_i S) S per element, two at a time
+                        const float2 s_lo = make_float2(S[e], S[e + 1]), s_hi = make_float2(S[e + 32], S[e + 33]);
+                        const float2 lo = __fmul2_rn(__fmul2_rn(wi2, s_lo), s_lo);
+                        const float2 hi = __fmul2_rn(__fmul2_rn(wi2, s_hi), s_hi);
+                        a1[e] = (up ? hi.x : lo.x) + __shfl_xor_sync(0xffffffffu, up ? lo.x : hi.x, 16);
+                        a1[e + 1] = (up ? hi.y : lo.y) + __shfl_xor_sync(0xffffffffu, up ? lo.y : hi.y, 16);
                     }
                 }
                 float a2[16];
@@ -698,18 +703,31 @@ __global__ void __launch_bounds__(NT3, 2) ut_state_kernel(const __grid_constant_
             bad |= !isfinite(ri);
             {
                 const float rri = __frcp_rn(ri);
-                // the codes as exact small integers in fp32: clamped, then rounded half to even by
-                // adding and subtracting 1.5 * 2^23 (the same value as rounding, then clamping)
+                // the codes as exact small integers in fp32, rounded half to even by adding and
+                // subtracting 1.5 * 2^23. With an fp32 r_i that is a normal number no clamp is needed:
+                // |S'_ij / c_j| <= m_i and r_i = m_i / qmax, so after the three fp32 roundings
+                // |x| <= qmax (1 + 3 * 2^-24) < qmax + 1/2. A bf16 r_i may be up to 2^-9 below
+                // m_i / qmax, and a subnormal r_i has an inexact reciprocal, so there the value is
+                // clamped first (the same as rounding, then clamping).
                 constexpr float RND = 12582912.0f;
                 const float2 rri2 = make_float2(rri, rri), rnd2 = make_float2(RND, RND), nrnd2 = make_float2(-RND, -RND);
+                if (p.scale_bf16 || !(ri >= 1.17549435e-38f)) {
 #pragma unroll
-                for (int e = 0; e < 64; e += 2) {
-                    float2 x = __fmul2_rn(make_float2(S[e], S[e + 1]), rri2);
-                    x.x = fminf(fmaxf(x.x, -(float)P::QMAX), (float)P::QMAX);
-                    x.y = fminf(fmaxf(x.y, -(float)P::QMAX), (float)P::QMAX);
-                    const float2 q = __fadd2_rn(__fadd2_rn(x, rnd2), nrnd2);
-                    S[e] = q.x;
-                    S[e + 1] = q.y;
+                    for (int e = 0; e < 64; e += 2) {
+                        float2 x = __fmul2_rn(make_float2(S[e], S[e + 1]), rri2);
+                        x.x = fminf(fmaxf(x.x, -(float)P::QMAX), (float)P::QMAX);
+                        x.y = fminf(fmaxf(x.y, -(float)P::QMAX), (float)P::QMAX);
+                        const float2 q = __fadd2_rn(__fadd2_rn(x, rnd2), nrnd2);
+                        S[e] = q.x;
+                        S[e + 1] = q.y;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 64; e += 2) {
+                        const float2 q = __fadd2_rn(__fadd2_rn(__fmul2_rn(make_float2(S[e], S[e + 1]), rri2), rnd2), nrnd2);
+                        S[e] = q.x;
+                        S[e + 1] = q.y;
+                    }
                 }
             }
             // next chunk's A operand (row i, columns 64 cq ..) and scales; the same bytes and the
