@@ -430,7 +430,7 @@ def prefill_leg(dev, steps: int = 3, warmup: int = 1, T: int = 8192, fit_rounds:
     return {"workload": "prefill16_b16_6bit", "prompt_tokens": T, "chunk": C, "requests": B, "heads": H,
             "ms_per_call": ms, "head_tokens_per_s": B * H * T / (ms / 1e3), "tokens_per_s": B * T / (ms / 1e3),
             "calls": steps, "fit_rounds": fit_rounds,
-            "kernel": (f"ut_inputs_kernel + ut_state_kernel<6> + ut_readout_kernel<6> per segment of up to 32 chunks "
+            "kernel": (f"ut_inputs_kernel + ut_state_kernel<6> + ut_readout_kernel per segment of up to 32 chunks "
                        f"(tcgen05, workspace of {ws.numel()} bytes)") if stq.prefill_workspace_bytes(lay, B, T, C)
                       else "prefill_wy_kernel<6> (tcgen05, one launch)" if fit_rounds <= 1 else "prefill_seq_kernel",
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,

@@ -955,7 +955,6 @@ __device__ __forceinline__ void readout_run(const TileParams &p, const UtArgs &a
     }
 }
 
-template <int BITS>
 __global__ void __launch_bounds__(NT3, 2) ut_readout_kernel(const __grid_constant__ TileParams p, const UtArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -975,26 +974,7 @@ cudaError_t launch_one(K kernel, uint32_t smem, int work, int sms, const TilePar
     return cudaGetLastError();
 }
 
-template <int BITS>
-cudaError_t launch_ut(const TileParams &p, int T, uint8_t *ws, cudaStream_t s)
-{
-    int dev = 0, sms = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (err != cudaSuccess) return err;
-    const int nch = (T + C - 1) / C;
-    for (int c0 = 0; c0 < nch; c0 += kUtSegmentChunks) {
-        const int nsc = nch - c0 < kUtSegmentChunks ? nch - c0 : kUtSegmentChunks;
-        const UtArgs a{ws, T, c0, nsc};
-        if ((err = launch_one(ut_inputs_kernel, P1_SMEM, p.ntiles * nsc, sms, p, a, s)) != cudaSuccess) return err;
-        if ((err = launch_one(ut_state_kernel<BITS>, P2_SMEM, p.ntiles, sms, p, a, s)) != cudaSuccess) return err;
-        if ((err = launch_one(ut_readout_kernel<BITS>, P3_SMEM, p.ntiles * nsc, sms, p, a, s)) != cudaSuccess)
-            return err;
-    }
-    return cudaSuccess;
-}
-
-// The same with segments of at most `seg` chunks (the workspace holds ntiles * seg records).
+// Segments of at most `seg` chunks: the workspace holds ntiles * seg records.
 template <int BITS>
 cudaError_t launch_ut_seg(const TileParams &p, int T, uint8_t *ws, int seg, cudaStream_t s)
 {
@@ -1008,10 +988,16 @@ cudaError_t launch_ut_seg(const TileParams &p, int T, uint8_t *ws, int seg, cuda
         const UtArgs a{ws, T, c0, nsc};
         if ((err = launch_one(ut_inputs_kernel, P1_SMEM, p.ntiles * nsc, sms, p, a, s)) != cudaSuccess) return err;
         if ((err = launch_one(ut_state_kernel<BITS>, P2_SMEM, p.ntiles, sms, p, a, s)) != cudaSuccess) return err;
-        if ((err = launch_one(ut_readout_kernel<BITS>, P3_SMEM, p.ntiles * nsc, sms, p, a, s)) != cudaSuccess)
+        if ((err = launch_one(ut_readout_kernel, P3_SMEM, p.ntiles * nsc, sms, p, a, s)) != cudaSuccess)
             return err;
     }
     return cudaSuccess;
+}
+
+template <int BITS>
+cudaError_t launch_ut(const TileParams &p, int T, uint8_t *ws, cudaStream_t s)
+{
+    return launch_ut_seg<BITS>(p, T, ws, kUtSegmentChunks, s);
 }
 
 }  // namespace
