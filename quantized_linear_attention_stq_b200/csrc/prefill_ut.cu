@@ -706,9 +706,10 @@ __global__ void __launch_bounds__(NT3, 2) ut_state_kernel(const __grid_constant_
                 // the codes as exact small integers in fp32, rounded half to even by adding and
                 // subtracting 1.5 * 2^23. With an fp32 r_i that is a normal number no clamp is needed:
                 // |S'_ij / c_j| <= m_i and r_i = m_i / qmax, so after the three fp32 roundings
-                // |x| <= qmax (1 + 3 * 2^-24) < qmax + 1/2. A bf16 r_i may be up to 2^-9 below
-                // m_i / qmax, and a subnormal r_i has an inexact reciprocal, so there the value is
-                // clamped first (the same as rounding, then clamping).
+                // |x| <= qmax (1 + 3 * 2^-24) < qmax + 1/2. A bf16 r_i may be up to 2^-8 (relative)
+                // below m_i / qmax, which leaves under 0.01 of margin at qmax = 127, and a subnormal
+                // r_i has an inexact reciprocal, so there the value is clamped first (the same as
+                // rounding, then clamping).
                 constexpr float RND = 12582912.0f;
                 const float2 rri2 = make_float2(rri, rri), rnd2 = make_float2(RND, RND), nrnd2 = make_float2(-RND, -RND);
                 if (p.scale_bf16 || !(ri >= 1.17549435e-38f)) {
