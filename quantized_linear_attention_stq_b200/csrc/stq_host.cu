@@ -371,7 +371,6 @@ stq_status stq_decode_step(const stq_layout *L, void *pool, int32_t pool_slots, 
             }
             return true;
         };
-        if (!launch(plan->pivots, 0, (int)plan->pivots.size(), 16)) return STQ_ERR_CUDA;
         // A launch per width keeps each width's compile-time ring (three slots for 4-bit tiles) but
         // pays the ring's start and the tail per launch: worth it when every width present has
         // enough tiles to fill the GPU several times over. Otherwise (the serving shape: one call
@@ -392,6 +391,9 @@ stq_status stq_decode_step(const stq_layout *L, void *pool, int32_t pool_slots, 
         } else if (!launch(plan->coded, 0, (int)plan->coded.size(), 0)) {
             return STQ_ERR_CUDA;
         }
+        // The FP16 pivots last: their few CTAs fill SMs as the coded launch drains, instead of
+        // holding SMs while it starts.
+        if (!launch(plan->pivots, 0, (int)plan->pivots.size(), 16)) return STQ_ERR_CUDA;
         return STQ_OK;
     }
     auto p = new_params();
