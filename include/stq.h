@@ -167,9 +167,9 @@ stq_status stq_decode_step(const stq_layout *layout, void *pool, int32_t pool_sl
 /* Workspace bytes stq_prefill_chunk can use for B requests and T tokens in chunks of `chunk`.
  * Nonzero only for the shapes that take the tensor-core chunk form with one plain
  * requantization per chunk end (128 x 128 heads, bf16 inputs, the scalar gate, chunk == 64, row x
- * column scales, no refit round) and at least one coded (4/6/8-bit) head: one record of 116736
- * bytes per request, coded head and chunk of a segment, where the call is cut into segments of at
- * most 32 chunks, so at most B x coded heads x 32 records whatever T. Host only. */
+ * column scales, no refit round): one record of 116736 bytes per request, head (FP16 pivot heads
+ * included) and chunk of a segment, where the call is cut into segments of at most 32 chunks, so
+ * at most B x H x 32 records whatever T. Host only. */
 size_t stq_prefill_workspace_bytes(const stq_layout *layout, int32_t B, int32_t T, int32_t chunk);
 
 /* Chunked prefill of T tokens for all H heads of B requests, in place. Tokens are cut into
@@ -182,8 +182,9 @@ size_t stq_prefill_workspace_bytes(const stq_layout *layout, int32_t B, int32_t 
  *   beta        device fp32 [B][H][T]
  *   alpha       device fp32 [B][H][T] (scalar gate) or [B][H][T][d_k] (channel gates)
  * 128 x 128 heads with bf16 inputs, the scalar gate and chunk == 64 run the tensor-core chunk
- * form; FP16 pivot heads and every other shape, gate or chunk run a token-by-token kernel with the
- * same chunk-boundary requantization.
+ * form (with a workspace for every head, FP16 pivots included; without one for the 4/6/8-bit
+ * heads); the other heads, shapes, gates and chunks run a token-by-token kernel with the same
+ * chunk-boundary requantization.
  *   w           device fp32 [H][d_k]
  *   o           device fp32 [B][H][T][d_v], written
  *   workspace   device scratch of >= stq_prefill_workspace_bytes(...) bytes, 256-byte aligned, or
@@ -212,7 +213,7 @@ stq_status stq_prefill_chunk(const stq_layout *layout, void *pool, int32_t pool_
  * The records live in one fixed device array of 33554432 bytes (32 MiB), defined in the library
  * and created with it on each device; the call allocates nothing, on the device or the host. It
  * fits the segments to the array: segments of min(32, 32 MiB / (B * m * 116736)) chunks, where m
- * is the largest number of heads of one code width; if one chunk of one width does not fit
+ * is the largest number of heads of one width (FP16 pivots are a width); if one chunk of one width does not fit
  * (B * m * 116736 > 32 MiB, for example more than 287 requests of one 4-bit head) the call returns
  * STQ_ERR_UNSUPPORTED before any device work (use stq_prefill_chunk with a workspace instead).
  * Nothing in the array has to start at zero: every record a call reads is written earlier in the

@@ -137,6 +137,41 @@ __device__ __forceinline__ void store_split2(uint8_t *t0, uint8_t *t1, uint32_t 
     *reinterpret_cast<uint4 *>(t1 + off) = make_uint4(b[0], b[1], b[2], b[3]);
 }
 
+// x = h + m + l with three fp16 terms (33 significand bits: exact for an fp32 value whose terms
+// stay normal; the caller keeps |x| below 2^15 so that none overflows).
+__device__ __forceinline__ void store_split3_h(uint8_t *t0, uint8_t *t1, uint8_t *t2, uint32_t off,
+                                               const float (&x)[8])
+{
+    uint32_t a[4], b[4], c[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 v = make_float2(x[2 * e], x[2 * e + 1]);
+        const __half2 h = __floats2half2_rn(v.x, v.y);
+        const float2 hf = __half22float2(h);
+        const float2 r1 = make_float2(v.x - hf.x, v.y - hf.y);
+        const __half2 m = __floats2half2_rn(r1.x, r1.y);
+        const float2 mf = __half22float2(m);
+        const __half2 l = __floats2half2_rn(r1.x - mf.x, r1.y - mf.y);
+        a[e] = *reinterpret_cast<const uint32_t *>(&h);
+        b[e] = *reinterpret_cast<const uint32_t *>(&m);
+        c[e] = *reinterpret_cast<const uint32_t *>(&l);
+    }
+    *reinterpret_cast<uint4 *>(t0 + off) = make_uint4(a[0], a[1], a[2], a[3]);
+    *reinterpret_cast<uint4 *>(t1 + off) = make_uint4(b[0], b[1], b[2], b[3]);
+    *reinterpret_cast<uint4 *>(t2 + off) = make_uint4(c[0], c[1], c[2], c[3]);
+}
+
+__device__ __forceinline__ void f16x8_to_f32(uint4 raw, float (&x)[8])
+{
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[e]));
+        x[2 * e] = f.x;
+        x[2 * e + 1] = f.y;
+    }
+}
+
 __device__ __forceinline__ void bf16x8_to_f32(uint4 raw, float (&x)[8])
 {
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};

@@ -775,6 +775,247 @@ __global__ void __launch_bounds__(NT3, 2) ut_state_kernel(const __grid_constant_
 }
 
 // =============================================================================================
+// State kernel of an FP16 pivot head: the state is fp16 (exact as an fp16 MMA operand), W goes in
+// as three fp16 terms after an exact power-of-two scaling that keeps its largest magnitude in
+// [2^14, 2^15), and the chunk end rounds the state to fp16 (no scales, no codes).
+// =============================================================================================
+template <int DUMMY = 0>
+__global__ void __launch_bounds__(NT3, 2) ut_state_pivot_kernel(const __grid_constant__ TileParams p, const UtArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = aligned_smem(smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, cq = warp >> 2;
+    float *red = smf(sm, P2_SMALL + P2S_RED);
+    const float *sDC = smf(sm, P2_SMALL + P2S_G) + C, *sGC = sDC + C;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + P2_SMALL + P2S_BAR);
+    uint32_t *misc = reinterpret_cast<uint32_t *>(sm + P2_SMALL + P2S_MISC);
+
+    if (warp == 0) umma::tmem_alloc(smem_u32(misc), 128);
+    if (tid == 0) {
+        mbar_init(smem_u32(&bars[0]), 1);
+        mbar_init(smem_u32(&bars[1]), 1);
+        fence_mbar_init();
+    }
+    umma::fence_before_sync();
+    __syncthreads();
+    umma::fence_after_sync();
+    const uint32_t tmem = misc[0];
+    const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
+    uint32_t parity = 0;
+    bool ok = true;
+
+    for (int n = blockIdx.x; n < p.ntiles && ok; n += gridDim.x) {
+        const int b = n % p.B, pos = n / p.B;
+        const TileEntry ent = p.table[pos];
+        const int head = entry_head(ent);
+        const int slot = p.slots[b];
+        if (slot < 0 || slot >= p.pool_slots) {
+            if (tid == 0) flag(p.status, kFlagBounds);
+            continue;
+        }
+        uint8_t *gblock = p.pool + (uint64_t)slot * p.req_bytes + ent.off;
+        const uint64_t trow = (uint64_t)b * (uint64_t)p.head_count + (uint64_t)head;
+        const __nv_bfloat16 *kg = reinterpret_cast<const __nv_bfloat16 *>(p.k) + trow * (uint64_t)a.T * D;
+        // thread (row i, columns 64 cq .. +63) owns 8 16-byte pieces of the state, in the pool
+        // (row-major fp16) and in the MMA image (atom column cq, row i, swizzled)
+        const int i = 32 * q4 + lane;
+
+        // ---- the tile's fp16 state into the A-operand image; it is the first chunk's start state --
+        __syncthreads();  // the previous tile is done with shared memory
+        {
+            const int t0 = a.c0 * C, Lc = (a.T - t0) < C ? (a.T - t0) : C;
+            p2_stage(sm, ut_record(a, n, 0), kg + (size_t)t0 * D, Lc);
+        }
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(gblock + (size_t)i * (2 * D) + 128 * cq);
+            uint8_t *st = ut_record(a, n, 0) + REC_ST;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint4 v4 = src[k];
+                const uint32_t off = cq * 16384 + sw128_chunk(i, k);
+                *reinterpret_cast<uint4 *>(sm + P2_QC + off) = v4;
+                *reinterpret_cast<uint4 *>(st + off) = v4;
+            }
+        }
+
+#pragma unroll 1
+        for (int cc = 0; cc < a.nsc && ok; ++cc, parity ^= 1u) {
+            uint8_t *rec = ut_record(a, n, cc);
+            cp_async_wait_all();  // this chunk's W, gamma and K
+            umma::fence_proxy_async();
+            __syncthreads();
+            const int j = 32 * q4 + lane;
+            float uv[32];
+            {
+                const float4 *ug = reinterpret_cast<const float4 *>(rec + REC_UV + (size_t)(j * C + 32 * cq) * 4);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const float4 x = ug[k];
+                    uv[4 * k] = x.x; uv[4 * k + 1] = x.y; uv[4 * k + 2] = x.z; uv[4 * k + 3] = x.w;
+                }
+            }
+            // ---- B operand of D2: W [t][i] times 2^-e, three fp16 terms ------------------------
+            int e2;
+            {
+                const int t = tid >> 2, part = tid & 3;
+                float x[4][8];
+                float mx = 0.f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float *src = smf(sm, P2_BY + t * (WST * 4) + 32 * (part + 4 * k));
+                    const float4 w0 = *reinterpret_cast<const float4 *>(src);
+                    const float4 w1 = *reinterpret_cast<const float4 *>(src + 4);
+                    x[k][0] = w0.x; x[k][1] = w0.y; x[k][2] = w0.z; x[k][3] = w0.w;
+                    x[k][4] = w1.x; x[k][5] = w1.y; x[k][6] = w1.z; x[k][7] = w1.w;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(x[k][e]));
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                if (lane == 0) red[warp] = mx;
+                __syncthreads();  // every staged row is read; the maxima are in
+                mx = red[0];
+#pragma unroll
+                for (int w = 1; w < NT3 / 32; ++w) mx = fmaxf(mx, red[w]);
+                // e with max |W| 2^-e in [2^14, 2^15) (0 for an all-zero W; a non-finite W gives a
+                // non-finite state below, which is flagged)
+                e2 = (mx > 0.f && isfinite(mx)) ? ilogbf(mx) - 14 : 0;
+                const float down = ldexpf(1.f, -e2);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int c8 = part + 4 * k;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[k][e] *= down;
+                    uint8_t *box = sm + P2_BY + (c8 >> 3) * 8192;
+                    store_split3_h(box, box + 16384, box + 32768, sw128_chunk(t, c8 & 7), x[k]);
+                }
+            }
+            umma::fence_proxy_async();
+            umma::fence_before_sync();
+            __syncthreads();
+            // ---- D2^T 2^-e = S0^T (W 2^-e)^T (fp16 operands, M 128 = j, N 64 = t) -> columns 0..63
+            if (tid == 0) {
+                umma::fence_after_sync();
+                const uint32_t qc = smem_u32(sm + P2_QC), by = smem_u32(sm + P2_BY);
+                const uint32_t id = umma::idesc_f16(128, 64, 1, 0);
+#pragma unroll
+                for (int x = 0; x < 3; ++x)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma::mma_bf16(tmem, umma::smem_desc(qc + kk * 2048, 16384, 1024),
+                                       umma::smem_desc(by + x * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                                       id, (x | kk) != 0);
+                umma::mma_commit(smem_u32(&bars[0]));
+            }
+            ok = wait_bar(smem_u32(&bars[0]), parity, p.status);
+            if (!__syncthreads_and(ok)) break;
+            umma::fence_after_sync();
+            // ---- U^T = U_v^T - D2^T: two bf16 terms to the record; decayed U in three bf16 terms -
+            {
+                float d[32];
+                umma::tmem_ld32(tl + 32 * cq, d);
+                const float up = -ldexpf(1.f, e2);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) uv[e] = fmaf(up, d[e], uv[e]);
+                uint8_t *by = sm + P2_BY;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    float x[8], y[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        x[e] = uv[8 * k + e];
+                        y[e] = sDC[32 * cq + 8 * k + e] * x[e];
+                    }
+                    const uint32_t off = sw128_chunk(j, 4 * cq + k);
+                    store_split2(rec + REC_W, rec + REC_W + 16384, off, x);
+                    store_split3(by, by + 16384, by + 32768, off, y);
+                }
+            }
+            umma::fence_proxy_async();
+            umma::fence_before_sync();
+            __syncthreads();
+            // ---- D3 = K^T (decayed U) -> columns 0..127 -----------------------------------------
+            if (tid == 0) {
+                umma::fence_after_sync();
+                const uint32_t kb = smem_u32(sm + P2_K), by = smem_u32(sm + P2_BY);
+                const uint32_t id = umma::idesc_bf16(128, 128, 1, 0);
+#pragma unroll
+                for (int x = 0; x < 3; ++x)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma::mma_bf16(tmem, umma::smem_desc(kb + kk * 2048, 8192, 1024),
+                                       umma::smem_desc(by + x * 16384 + kk * 32, 16, 1024), id, (x | kk) != 0);
+                umma::mma_commit(smem_u32(&bars[1]));
+            }
+            ok = wait_bar(smem_u32(&bars[1]), parity, p.status);
+            if (!__syncthreads_and(ok)) break;
+            umma::fence_after_sync();
+
+            // ---- chunk end: S_C = gamma_C S0 + D3, rounded to fp16 (row i, columns 64 cq .. +63) --
+            uint4 out[8];
+            bool bad = false;
+            {
+                const float gC = sGC[0];
+                const uint8_t *srow = sm + P2_QC + cq * 16384;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v[32];
+                    umma::tmem_ld32(tl + 64 * cq + 32 * hh, v);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        float s0[8];
+                        f16x8_to_f32(*reinterpret_cast<const uint4 *>(srow + sw128_chunk(i, 4 * hh + k)), s0);
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int e = 0; e < 8; e += 2) {
+                            const float x0 = fmaf(gC, s0[e], v[8 * k + e]);
+                            const float x1 = fmaf(gC, s0[e + 1], v[8 * k + e + 1]);
+                            bad |= !(fabsf(x0) < 65520.0f) || !(fabsf(x1) < 65520.0f);  // overflows fp16 (or NaN)
+                            const __half2 h = __floats2half2_rn(x0, x1);
+                            w4[e >> 1] = *reinterpret_cast<const uint32_t *>(&h);
+                        }
+                        out[4 * hh + k] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
+                }
+            }
+            umma::fence_before_sync();
+            __syncthreads();  // the chunk-start state, gamma, K and the term area are free
+            if (cc + 1 < a.nsc) {
+                const int t1 = (a.c0 + cc + 1) * C, L1 = (a.T - t1) < C ? (a.T - t1) : C;
+                const uint8_t *nrec = ut_record(a, n, cc + 1);
+                p2_stage(sm, nrec, kg + (size_t)t1 * D, L1);
+                if (tid == 0) l2_prefetch(nrec + REC_UV, 32768u);
+            }
+            {
+                // the next chunk's A operand; the same bytes are its start state in the workspace,
+                // and after the segment's last chunk the state goes to the pool (row-major fp16)
+                const bool last = cc + 1 == a.nsc;
+                uint8_t *st = last ? nullptr : ut_record(a, n, cc + 1) + REC_ST;
+                uint4 *prow = reinterpret_cast<uint4 *>(gblock + (size_t)i * (2 * D) + 128 * cq);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t off = cq * 16384 + sw128_chunk(i, k);
+                    *reinterpret_cast<uint4 *>(sm + P2_QC + off) = out[k];
+                    if (last) prow[k] = out[k];
+                    else *reinterpret_cast<uint4 *>(st + off) = out[k];
+                }
+            }
+            if (bad) flag(p.status, kFlagNonfinite);
+            umma::fence_proxy_async();
+            umma::fence_before_sync();
+            __syncthreads();
+        }
+    }
+    cp_async_wait_all();
+    umma::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        umma::fence_after_sync();
+        umma::tmem_dealloc(tmem, 128);
+    }
+}
+
+// =============================================================================================
 // Readout kernel: per (tile, chunk) unit, o_t = gamma_t c (Q^T (q r))_t + (P U)_t. The chunk-start
 // codes, the U and P terms and the scales arrive as images by asynchronous copies.
 // =============================================================================================
@@ -786,9 +1027,11 @@ constexpr uint32_t P3_SMEM = P3_SMALL + 1312 + 1024;
 constexpr int OST = 132;  // row stride (floats) of the readout staged over the term area
 static_assert(64 * OST * 4 <= 49152, "readout rows fit the term area");
 
-// The readout work of one CTA: units first, first + stride, ... of the segment.
+// The readout work of one CTA: units first, first + stride, ... of the segment. For FP16 pivot
+// heads (`pivot`) the chunk-start state image is fp16 and unscaled (r = c = 1): D_a takes q as one
+// fp16 term (q has |q_i| <= 1; below 2^-17 fp16 keeps it to 2^-25).
 __device__ __forceinline__ void readout_run(const TileParams &p, const UtArgs &a, uint8_t *sm, const int first,
-                                            const int stride)
+                                            const int stride, const bool pivot)
 {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, cq = warp >> 2;
     float *sR = smf(sm, P3_SMALL + P3S_R), *sC = smf(sm, P3_SMALL + P3S_C), *sGam = smf(sm, P3_SMALL + P3S_GAM);
@@ -837,8 +1080,11 @@ __device__ __forceinline__ void readout_run(const TileParams &p, const UtArgs &a
             const int e = tid + NT3 * k;
             cp_async16(smem_u32(X + 32768 + 16 * e), rec + REC_PT + 16 * e, 16u);
         }
-        if (tid < 64) cp_async16(smem_u32(reinterpret_cast<uint8_t *>(sR) + 16 * tid), rec + REC_SC + 16 * tid, 16u);
-        else if (tid < 80) cp_async16(smem_u32(reinterpret_cast<uint8_t *>(sGam) + 16 * (tid - 64)), rec + REC_G + 16 * (tid - 64), 16u);
+        if (tid < 64) {
+            if (!pivot) cp_async16(smem_u32(reinterpret_cast<uint8_t *>(sR) + 16 * tid), rec + REC_SC + 16 * tid, 16u);
+        } else if (tid < 80) {
+            cp_async16(smem_u32(reinterpret_cast<uint8_t *>(sGam) + 16 * (tid - 64)), rec + REC_G + 16 * (tid - 64), 16u);
+        }
         cp_async_commit();
         // q row t, columns 32 part .. +31, in registers for the (q r) terms
         const int t = tid >> 2, part = tid & 3;
@@ -880,8 +1126,23 @@ __device__ __forceinline__ void readout_run(const TileParams &p, const UtArgs &a
         }
         ok = wait_bar(smem_u32(&bars[0]), parity, p.status);
         if (!__syncthreads_and(ok)) break;
-        // ---- three bf16 terms of (q r) [t][i] over the same area (K-major B, rows t) -----------
-        {
+        // ---- three bf16 terms of (q r) [t][i] over the same area (K-major B, rows t); for a
+        //      pivot, q as one fp16 term -----------------------------------------------------------
+        if (pivot) {
+            uint8_t *box = X + (part >> 1) * 8192;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float x[8];
+                bf16x8_to_f32(qraw[k], x);
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __half2 h = __floats2half2_rn(x[2 * e], x[2 * e + 1]);
+                    w4[e] = *reinterpret_cast<const uint32_t *>(&h);
+                }
+                *reinterpret_cast<uint4 *>(box + sw128_chunk(t, 4 * (part & 1) + k)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+        } else {
             uint8_t *box = X + (part >> 1) * 8192;
             const float *rr = sR + 32 * part;
 #pragma unroll
@@ -900,9 +1161,9 @@ __device__ __forceinline__ void readout_run(const TileParams &p, const UtArgs &a
         if (tid == 0) {
             umma::fence_after_sync();
             const uint32_t qc = smem_u32(sm + P3_QC), x0 = smem_u32(X);
-            const uint32_t id = umma::idesc_bf16(128, 64, 1, 0);
-#pragma unroll
-            for (int x = 0; x < 3; ++x)
+            const uint32_t id = pivot ? umma::idesc_f16(128, 64, 1, 0) : umma::idesc_bf16(128, 64, 1, 0);
+            const int terms = pivot ? 1 : 3;
+            for (int x = 0; x < terms; ++x)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     umma::mma_bf16(tmem, umma::smem_desc(qc + kk * 2048, 16384, 1024),
@@ -920,7 +1181,7 @@ __device__ __forceinline__ void readout_run(const TileParams &p, const UtArgs &a
             float av[32], dv[32];
             umma::tmem_ld32(tl + 32 * cq, av);
             umma::tmem_ld32(tl + 64 + 32 * cq, dv);
-            const float cj = sC[j];
+            const float cj = pivot ? 1.f : sC[j];
             float *ob = reinterpret_cast<float *>(X);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
@@ -956,14 +1217,16 @@ __device__ __forceinline__ void readout_run(const TileParams &p, const UtArgs &a
     }
 }
 
-__global__ void __launch_bounds__(NT3, 2) ut_readout_kernel(const __grid_constant__ TileParams p, const UtArgs a)
+__global__ void __launch_bounds__(NT3, 2) ut_readout_kernel(const __grid_constant__ TileParams p, const UtArgs a,
+                                                            const int pivot)
 {
     extern __shared__ uint8_t smem_raw[];
-    readout_run(p, a, aligned_smem(smem_raw), blockIdx.x, gridDim.x);
+    readout_run(p, a, aligned_smem(smem_raw), blockIdx.x, gridDim.x, pivot != 0);
 }
 
-template <typename K>
-cudaError_t launch_one(K kernel, uint32_t smem, int work, int sms, const TileParams &p, const UtArgs &a, cudaStream_t s)
+template <typename K, typename... X>
+cudaError_t launch_one(K kernel, uint32_t smem, int work, int sms, const TileParams &p, const UtArgs &a, cudaStream_t s,
+                       X... extra)
 {
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     // the whole carveout as shared memory, so that two CTAs fit on an SM
@@ -971,7 +1234,7 @@ cudaError_t launch_one(K kernel, uint32_t smem, int work, int sms, const TilePar
         err = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
     if (err != cudaSuccess) return err;
     const int grid = work < 2 * sms ? work : 2 * sms;
-    kernel<<<grid, NT3, smem, s>>>(p, a);
+    kernel<<<grid, NT3, smem, s>>>(p, a, extra...);
     return cudaGetLastError();
 }
 
@@ -988,8 +1251,13 @@ cudaError_t launch_ut_seg(const TileParams &p, int T, uint8_t *ws, int seg, cuda
         const int nsc = nch - c0 < seg ? nch - c0 : seg;
         const UtArgs a{ws, T, c0, nsc};
         if ((err = launch_one(ut_inputs_kernel, P1_SMEM, p.ntiles * nsc, sms, p, a, s)) != cudaSuccess) return err;
-        if ((err = launch_one(ut_state_kernel<BITS>, P2_SMEM, p.ntiles, sms, p, a, s)) != cudaSuccess) return err;
-        if ((err = launch_one(ut_readout_kernel, P3_SMEM, p.ntiles * nsc, sms, p, a, s)) != cudaSuccess)
+        if constexpr (BITS == 16)
+            err = launch_one(ut_state_pivot_kernel<0>, P2_SMEM, p.ntiles, sms, p, a, s);
+        else
+            err = launch_one(ut_state_kernel<BITS>, P2_SMEM, p.ntiles, sms, p, a, s);
+        if (err != cudaSuccess) return err;
+        if ((err = launch_one(ut_readout_kernel, P3_SMEM, p.ntiles * nsc, sms, p, a, s, (int)(BITS == 16))) !=
+            cudaSuccess)
             return err;
     }
     return cudaSuccess;
@@ -1011,12 +1279,14 @@ cudaError_t launch_prefill_ut_seg(const TileParams &p, int bits, int T, void *ws
     case 4: return launch_ut_seg<4>(p, T, w, seg, s);
     case 6: return launch_ut_seg<6>(p, T, w, seg, s);
     case 8: return launch_ut_seg<8>(p, T, w, seg, s);
+    case 16: return launch_ut_seg<16>(p, T, w, seg, s);
     default: return cudaErrorInvalidValue;
     }
 }
 
 // Chunked prefill of 128 x 128 tiles (bf16 inputs, scalar gate, 64-token chunks, one plain
-// requantization per chunk end) through the workspace; every entry of p.table has width `bits`.
+// requantization per chunk end) through the workspace; every entry of p.table has width `bits`
+// (4, 6, 8, or 16 for FP16 pivot heads).
 cudaError_t launch_prefill_ut(const TileParams &p, int bits, int T, void *ws, cudaStream_t s)
 {
     uint8_t *w = static_cast<uint8_t *>(ws);
@@ -1024,6 +1294,7 @@ cudaError_t launch_prefill_ut(const TileParams &p, int bits, int T, void *ws, cu
     case 4: return launch_ut<4>(p, T, w, s);
     case 6: return launch_ut<6>(p, T, w, s);
     case 8: return launch_ut<8>(p, T, w, s);
+    case 16: return launch_ut<16>(p, T, w, s);
     default: return cudaErrorInvalidValue;
     }
 }

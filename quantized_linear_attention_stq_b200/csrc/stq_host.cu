@@ -66,15 +66,9 @@ bool wy_form(const stq_layout *L, int chunk)
     return L->dk == 128 && L->gate == STQ_GATE_SCALAR && L->in_dtype == STQ_BF16 && chunk == 64 && !L->uniform &&
            L->fit_rounds <= 1;
 }
-// ... of which those with one plain requantization per chunk end and at least one coded head can
-// run as the three workspace kernels.
-bool ut_form(const stq_layout *L, int chunk)
-{
-    if (!wy_form(L, chunk) || L->fit_rounds != 0) return false;
-    for (int h = 0; h < L->H; ++h)
-        if (L->bits[h] != 16) return true;
-    return false;
-}
+// ... of which those with one plain requantization per chunk end run as the three workspace
+// kernels, every head (FP16 pivots included) in the chunk form.
+bool ut_form(const stq_layout *L, int chunk) { return wy_form(L, chunk) && L->fit_rounds == 0; }
 
 // Fill the common fields of a TileParams for heads ord[first .. first+n) of a call.
 void fill_table(stq::TileParams &p, const stq_layout *L, const std::vector<int> &ord, int first, int n, int h0)
@@ -436,12 +430,10 @@ size_t stq_prefill_workspace_bytes(const stq_layout *L, int32_t B, int32_t T, in
 {
     if (!L || B < 0 || T < 0 || chunk < 1) return 0;
     if (!ut_form(L, chunk)) return 0;  // the other kernels carry everything on chip
-    // one record per (request, coded head, chunk of a segment); the widths run one after another
-    int coded = 0;
-    for (int h = 0; h < L->H; ++h) coded += L->bits[h] != 16;
+    // one record per (request, head, chunk of a segment); the widths run one after another
     const int64_t nch = ((int64_t)T + 63) / 64;
     const int64_t seg = nch < stq::kUtSegmentChunks ? nch : stq::kUtSegmentChunks;
-    return (size_t)B * (size_t)coded * (size_t)seg * (size_t)stq::kUtRecordBytes;
+    return (size_t)B * (size_t)L->H * (size_t)seg * (size_t)stq::kUtRecordBytes;
 }
 
 stq_status stq_prefill_chunk(const stq_layout *L, void *pool, int32_t pool_slots, const int32_t *slots, int32_t B,
@@ -499,9 +491,9 @@ stq_status stq_prefill_chunk(const stq_layout *L, void *pool, int32_t pool_slots
         while (first + n < L->H && L->bits[ord[first + n]] == bits) ++n;
         fill_table(*p, L, ord, first, n, 0);
         p->ntiles = B * n;
-        const cudaError_t e = bits == 16 ? stq::launch_prefill_seq(*p, 1, T, chunk, (cudaStream_t)stream)
-                              : use_ws   ? stq::launch_prefill_ut(*p, bits, T, workspace, (cudaStream_t)stream)
-                                         : stq::launch_prefill_wy(*p, bits, T, (cudaStream_t)stream);
+        const cudaError_t e = use_ws       ? stq::launch_prefill_ut(*p, bits, T, workspace, (cudaStream_t)stream)
+                              : bits == 16 ? stq::launch_prefill_seq(*p, 1, T, chunk, (cudaStream_t)stream)
+                                           : stq::launch_prefill_wy(*p, bits, T, (cudaStream_t)stream);
         if (e != cudaSuccess) return STQ_ERR_CUDA;
         first += n;
     }
@@ -524,12 +516,12 @@ stq_status stq_prefill_chunk_noalloc(const stq_layout *L, void *pool, int32_t po
         !aligned(o, 16) || !aligned(beta, 4) || !aligned(alpha, 4))
         return STQ_ERR_INVALID_ARG;
     if (L->H > stq::kMaxTable) return STQ_ERR_UNSUPPORTED;
-    // one width at a time: the widest class sets how many chunks a segment of records can hold
-    int count[3] = {0, 0, 0};
-    static const int widths[3] = {8, 6, 4};
+    // one width at a time: the largest class sets how many chunks a segment of records can hold
+    int count[4] = {0, 0, 0, 0};
+    static const int widths[4] = {16, 8, 6, 4};
     for (int h = 0; h < L->H; ++h)
-        for (int c = 0; c < 3; ++c) count[c] += L->bits[h] == widths[c];
-    const uint64_t most = (uint64_t)std::max(count[0], std::max(count[1], count[2]));
+        for (int c = 0; c < 4; ++c) count[c] += L->bits[h] == widths[c];
+    const uint64_t most = (uint64_t)std::max(std::max(count[0], count[1]), std::max(count[2], count[3]));
     const uint64_t per_chunk = (uint64_t)B * most * stq::kUtRecordBytes;
     if (per_chunk > kNoallocScratchBytes) return STQ_ERR_UNSUPPORTED;
     const uint64_t fit = kNoallocScratchBytes / per_chunk;
@@ -557,19 +549,16 @@ stq_status stq_prefill_chunk_noalloc(const stq_layout *L, void *pool, int32_t po
     tp.alpha = alpha;
     tp.w = w;
     tp.o = o;
-    // FP16 pivots first (token-by-token kernel), then the 8-, 6- and 4-bit heads, head index order
-    static const int order[4] = {16, 8, 6, 4};
+    // FP16 pivots first, then the 8-, 6- and 4-bit heads, head index order inside a width
     for (int c = 0; c < 4; ++c) {
         int n = 0;
         for (int h = 0; h < L->H; ++h)
-            if (L->bits[h] == order[c]) tp.table[n++] = entry_of(L, h, 0);
+            if (L->bits[h] == widths[c]) tp.table[n++] = entry_of(L, h, 0);
         if (n == 0) continue;
         tp.npos = n;
         tp.ntiles = B * n;
-        const cudaError_t e = order[c] == 16
-                                  ? stq::launch_prefill_seq(tp, 1, T, chunk, (cudaStream_t)stream)
-                                  : stq::launch_prefill_ut_seg(tp, order[c], T, scratch, seg, (cudaStream_t)stream);
-        if (e != cudaSuccess) return STQ_ERR_CUDA;
+        if (stq::launch_prefill_ut_seg(tp, widths[c], T, scratch, seg, (cudaStream_t)stream) != cudaSuccess)
+            return STQ_ERR_CUDA;
     }
     return STQ_OK;
 }

@@ -1,6 +1,6 @@
 // umma.cuh -- fifth-generation tensor core (tcgen05) building blocks for sm_100a: shared-memory
-// matrix descriptors for 128-byte-swizzled bf16 tiles, the instruction descriptor of a
-// bf16 x bf16 -> fp32 MMA, MMA issue / commit, Tensor Memory allocation and loads.
+// matrix descriptors for 128-byte-swizzled 16-bit tiles, the instruction descriptors of a
+// bf16 x bf16 or fp16 x fp16 -> fp32 MMA, MMA issue / commit, Tensor Memory allocation and loads.
 //
 // Tile layouts (all bf16, 128-byte swizzle; every swizzle atom of 8 rows x 128 B starts on a
 // 1024-byte boundary):
@@ -55,6 +55,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
     return (1u << 4)                      // D format: f32
            | (1u << 7)                    // A format: bf16
            | (1u << 10)                   // B format: bf16
+           | ((uint32_t)a_mn << 15)       // A major
+           | ((uint32_t)b_mn << 16)       // B major
+           | ((uint32_t)(N >> 3) << 17)   // N / 8
+           | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+// The same with fp16 A and B (format code 0): both operands of one MMA have the same type.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_mn)
+{
+    return (1u << 4)                      // D format: f32
            | ((uint32_t)a_mn << 15)       // A major
            | ((uint32_t)b_mn << 16)       // B major
            | ((uint32_t)(N >> 3) << 17)   // N / 8

@@ -164,23 +164,24 @@ def test_calls_reject_bad_arguments_before_enqueueing(stq):
 
 
 def test_prefill_workspace_sizes(stq):
-    """The three-kernel prefill asks for one record per (request, coded head, chunk of a segment of
-    at most 32 chunks); the shapes that run as one kernel ask for none. A workspace that is given
-    must be large enough and 256-byte aligned (checked on the host, before any CUDA call)."""
+    """The three-kernel prefill asks for one record per (request, head, chunk of a segment of at
+    most 32 chunks), FP16 pivot heads included; the shapes that run as one kernel ask for none. A
+    workspace that is given must be large enough and 256-byte aligned (checked on the host, before
+    any CUDA call)."""
     SEG = 32
     bf = torch.bfloat16
     REC = stq.prefill_workspace_bytes(stq.Layout([6], 128, in_dtype=bf), 1, 64, 64)
     assert REC > 0 and REC % 1024 == 0
     lay = stq.Layout([6, 16, 4, 8], 128, in_dtype=bf)
-    assert stq.prefill_workspace_bytes(lay, 3, 64, 64) == 3 * 3 * 1 * REC
-    assert stq.prefill_workspace_bytes(lay, 3, 65, 64) == 3 * 3 * 2 * REC
-    assert stq.prefill_workspace_bytes(lay, 2, 8192, 64) == 2 * 3 * SEG * REC
+    assert stq.prefill_workspace_bytes(lay, 3, 64, 64) == 3 * 4 * 1 * REC
+    assert stq.prefill_workspace_bytes(lay, 3, 65, 64) == 3 * 4 * 2 * REC
+    assert stq.prefill_workspace_bytes(lay, 2, 8192, 64) == 2 * 4 * SEG * REC
+    assert stq.prefill_workspace_bytes(stq.Layout([16, 16], 128, in_dtype=bf), 3, 640, 64) == 3 * 2 * 10 * REC
     assert stq.prefill_workspace_bytes(lay, 0, 64, 64) == 0
     assert stq.prefill_workspace_bytes(lay, 3, 0, 64) == 0
     assert stq.prefill_workspace_bytes(lay, 3, 64, 32) == 0
     for other in (stq.Layout([6, 4], 128, in_dtype=torch.float32), stq.Layout([6, 4], 64, in_dtype=bf),
-                  stq.Layout([6, 4], 128, gate=1, in_dtype=bf), stq.Layout([6, 4], 128, in_dtype=bf, fit_rounds=1),
-                  stq.Layout([16, 16], 128, in_dtype=bf)):
+                  stq.Layout([6, 4], 128, gate=1, in_dtype=bf), stq.Layout([6, 4], 128, in_dtype=bf, fit_rounds=1)):
         assert stq.prefill_workspace_bytes(other, 3, 640, 64) == 0
     L = stq.lib()
     P = ctypes.c_void_p

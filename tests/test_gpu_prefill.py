@@ -211,7 +211,7 @@ def test_segments_equal_single_chunk_calls(stq, orc):
     slots = torch.tensor([1, 0], dtype=torch.int32, device=DEV)
     wd = w.to(DEV)
     rec = stq.prefill_workspace_bytes(stq.Layout([6], d, in_dtype=torch.bfloat16), 1, C, C)
-    assert stq.prefill_workspace_bytes(lay, B, T, C) == B * 3 * 32 * rec  # two segments: 32 + 2 chunks
+    assert stq.prefill_workspace_bytes(lay, B, T, C) == B * 4 * 32 * rec  # two segments: 32 + 2 chunks
     ws = _workspace(stq, lay, B, T, C, "workspace")
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     p_full = torch.from_numpy(opool.copy()).to(DEV)
