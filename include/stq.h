@@ -183,8 +183,8 @@ size_t stq_prefill_workspace_bytes(const stq_layout *layout, int32_t B, int32_t 
  *   alpha       device fp32 [B][H][T] (scalar gate) or [B][H][T][d_k] (channel gates)
  * 128 x 128 heads with bf16 inputs, the scalar gate and chunk == 64 run the tensor-core chunk
  * form (with a workspace for every head, FP16 pivots included; without one for the 4/6/8-bit
- * heads); the other heads, shapes, gates and chunks run a token-by-token kernel with the same
- * chunk-boundary requantization.
+ * heads); the other heads, shapes, gates and chunks run token by token with the same
+ * chunk-boundary requantization (128 x 128 heads with the state held on chip).
  *   w           device fp32 [H][d_k]
  *   o           device fp32 [B][H][T][d_v], written
  *   workspace   device scratch of >= stq_prefill_workspace_bytes(...) bytes, 256-byte aligned, or

@@ -477,12 +477,17 @@ stq_status stq_prefill_chunk(const stq_layout *L, void *pool, int32_t pool_slots
     // chunk form, one width at a time (three kernels around the workspace, or one kernel); FP16
     // pivot heads and every other configuration take the sequential kernel.
     const bool wy = wy_form(L, chunk);
+    const int in_bf16 = L->in_dtype == STQ_BF16;
     if (!wy) {
         std::vector<int> ord(L->H);
         for (int h = 0; h < L->H; ++h) ord[h] = h;
         fill_table(*p, L, ord, 0, L->H, 0);
         p->ntiles = B * L->H;
-        return from_cuda(stq::launch_prefill_seq(*p, L->in_dtype == STQ_BF16, T, chunk, (cudaStream_t)stream));
+        // 128 x 128 heads with row x column scales and no refit round: the state in registers;
+        // the others (smaller heads, the uniform baseline, refit rounds): the general kernel
+        const bool serial = L->dk == 128 && !L->uniform && L->fit_rounds == 0;
+        return from_cuda(serial ? stq::launch_prefill_serial(*p, in_bf16, T, chunk, (cudaStream_t)stream)
+                                : stq::launch_prefill_seq(*p, in_bf16, T, chunk, (cudaStream_t)stream));
     }
     const std::vector<int> ord = order_by_size(L, 0, L->H);
     for (int first = 0; first < L->H;) {
@@ -492,7 +497,7 @@ stq_status stq_prefill_chunk(const stq_layout *L, void *pool, int32_t pool_slots
         fill_table(*p, L, ord, first, n, 0);
         p->ntiles = B * n;
         const cudaError_t e = use_ws       ? stq::launch_prefill_ut(*p, bits, T, workspace, (cudaStream_t)stream)
-                              : bits == 16 ? stq::launch_prefill_seq(*p, 1, T, chunk, (cudaStream_t)stream)
+                              : bits == 16 ? stq::launch_prefill_serial(*p, 1, T, chunk, (cudaStream_t)stream)
                                            : stq::launch_prefill_wy(*p, bits, T, (cudaStream_t)stream);
         if (e != cudaSuccess) return STQ_ERR_CUDA;
         first += n;

@@ -96,6 +96,9 @@ cudaError_t launch_decode_generic(const TileParams &p, int in_bf16, cudaStream_t
 // and 8; pdl: a later launch of the same call (disjoint tiles) that may overlap the earlier ones
 cudaError_t launch_decode_d128(const TileParams &p, int bits, int in_bf16, cudaStream_t s, bool pdl);
 cudaError_t launch_prefill_seq(const TileParams &p, int in_bf16, int T, int chunk, cudaStream_t s);
+// 128 x 128 heads token by token with the state in registers: any gate, chunk length and width of
+// p.table (4/6/8 with row x column scales and no refit round, or 16)
+cudaError_t launch_prefill_serial(const TileParams &p, int in_bf16, int T, int chunk, cudaStream_t s);
 cudaError_t launch_prefill_wy(const TileParams &p, int bits, int T, cudaStream_t s);  // one width per launch
 // The same chunk form as three kernels around a workspace of ntiles * min(chunks, kUtSegmentChunks)
 // records of kUtRecordBytes (one plain requantization per chunk end; one width per launch).
