@@ -759,7 +759,11 @@ def run_ours(args):
         "step_ms_median": statistics.median(per_step),
         "step_ms_min": min(per_step),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": peak_kind, "traffic": profiled_traffic(),
+                     "peak_kind": peak_kind,
+                     # the committed capture is of the default step (batch 70, fp32 scales, one pass)
+                     "traffic": profiled_traffic() if (args.workload == DEFAULT_WORKLOAD and not args.batch
+                                                        and args.scale_dtype == "f32" and args.fit_rounds == 0)
+                     else None,
                      "bytes_per_step": state_bytes, "launches_per_step": launches_per_step,
                      "kernel": ("decode_d128_kernel<width> (pivots, then one launch per width)" if per_width
                                 else "decode_d128_kernel<width> (pivots, then one launch for all widths)"),
