@@ -45,8 +45,8 @@ constexpr int NSMAX = 4;               // slots (tiles in flight) per CTA
 constexpr uint32_t MAGIC = 0x4B000000u;  // bit pattern of 2^23
 constexpr uint32_t TMEM_COLS = 128;    // per CTA: 128 lanes x 128 columns of fp32 = one tile
 // red[]: one region of RS floats per (warp, half) k = 2w + h. [0, 128): the half's column
-// partials (k~Q for h = 0, q~Q for h = 1); [128, 256) of the h = 0 region: the warp's column
-// energies; later the half's 16 row-max partial rows of RM floats. Only warp w writes its two
+// partials, column j at cpos(j) (k~Q for h = 0, q~Q for h = 1); [128, 256) of the h = 0 region:
+// the warp's column energies; later the half's 16 row-max partial rows of RM floats. Only warp w writes its two
 // regions while other warps may be reading, so a warp never overwrites data still in use.
 constexpr int RM = 20;                 // row stride of the row-max partials (bank-conflict free)
 constexpr int RS = 336;                // region stride (= 16 mod 32 banks: the halves do not collide)
@@ -71,8 +71,8 @@ struct __align__(16) SmemFixed {
     float4 rowKQ[D];         // (k~, k~, q~, q~)
     float4 rowRK[D];         // (rho, rho, kappa, kappa)
     float rowRq[2][D];       // per tile parity: 1 / (sqrt(w_i) qmax)
-    float2 rowS[D];          // (s_i, s_i), s_i = 1 / (sqrt(w_i) r'_i) = qmax / max_j |z_ij|
-    float colG1[D];
+    float2 rowS[D];          // (s_i, s_i), s_i = 1 / (sqrt(w_i) r'_i) = qmax / max_j |z_ij|, at rpos<FIT>(i)
+    float colG1[D];          // per column j at cpos(j), as colB and colG2
     float colB[D];           // c_j / (sigma_j c'_j) = 1 / sqrt(x_j)
     float rsum[2][4][4];     // per parity, per warp: sum w, q.k, q.(alpha*k)
     float scal[NSMAX][2];    // per slot: beta, alpha
@@ -272,16 +272,45 @@ __device__ __forceinline__ void pack_store_row(uint8_t *dst, int cg, const float
     }
 }
 
-__device__ __forceinline__ float4 f4_of(float2 a, float2 b) { return make_float4(a.x, a.y, b.x, b.y); }
-
-__device__ __forceinline__ void load_pairs(const float *src, float2 (&out)[4])
+// Column j's place in the per-column arrays (colG1, colB, colG2) and in the column-partial regions
+// of red[]: lane cg keeps its columns 8 cg + 4 h + t (h < 2, t < 4) as two float4 at 4 cslot(cg, h),
+// cslot(cg, h) = 8 (2 (cg / 8) + h) + (cg + 4 h) % 8. Then the float4 of 8 lanes with the same h
+// and the floats of 32 threads j (column j each) both fall on 32 distinct banks. LIN: column j at
+// j instead (two-way conflicts on the float4, two fewer live addresses; the refit kernels, which
+// are short of registers, keep it).
+template <int LIN>
+__device__ __forceinline__ int cslot(int cg, int h)
 {
-    const float4 a = *reinterpret_cast<const float4 *>(src);
-    const float4 b = *reinterpret_cast<const float4 *>(src + 4);
+    return LIN ? 2 * cg + h : 8 * (2 * (cg >> 3) + h) + ((cg + 4 * h) & 7);
+}
+template <int LIN>
+__device__ __forceinline__ int cpos(int j)
+{
+    return LIN ? j : 4 * cslot<0>(j >> 3, (j >> 2) & 1) + (j & 3);
+}
+
+// Row i's place in rowS: [i % 8][i / 8], so that the 16 rows 8 m + rb of a half-warp are
+// consecutive (lane m writes row 8 m + rb); LIN: row i at i.
+template <int LIN>
+__device__ __forceinline__ int rpos(int i) { return LIN ? i : (i & 7) * 16 + (i >> 3); }
+
+// Lane cg's 8 columns of a per-column array (layout of cpos) as four pairs.
+template <int LIN>
+__device__ __forceinline__ void load_cols(const float *base, int cg, float2 (&out)[4])
+{
+    const float4 a = *reinterpret_cast<const float4 *>(base + 4 * cslot<LIN>(cg, 0));
+    const float4 b = *reinterpret_cast<const float4 *>(base + 4 * cslot<LIN>(cg, 1));
     out[0] = make_float2(a.x, a.y);
     out[1] = make_float2(a.z, a.w);
     out[2] = make_float2(b.x, b.y);
     out[3] = make_float2(b.z, b.w);
+}
+
+template <int LIN>
+__device__ __forceinline__ void store_cols(float *base, int cg, const float2 (&v)[4])
+{
+    *reinterpret_cast<float4 *>(base + 4 * cslot<LIN>(cg, 0)) = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
+    *reinterpret_cast<float4 *>(base + 4 * cslot<LIN>(cg, 1)) = make_float4(v[2].x, v[2].y, v[3].x, v[3].y);
 }
 
 // Sum of the 4 per-warp partials at `stride` floats apart.
@@ -443,7 +472,7 @@ __device__ __forceinline__ bool refit_scales(const TileParams &p, SmemFixed &sm,
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const int i = 8 * (2 * k + r) + rb;
-                const float2 s2 = sm.rowS[i];
+                const float2 s2 = sm.rowS[rpos<FIT>(i)];
                 const float2 rr = make_float2(rho[i], rho[i]);
 #pragma unroll
                 for (int pp = 0; pp < 4; ++pp) {
@@ -465,15 +494,13 @@ __device__ __forceinline__ bool refit_scales(const TileParams &p, SmemFixed &sm,
                                            __shfl_xor_sync(0xffffffffu, send.y, 16));
             aN[pp] = __fadd2_rn(keep, got);
         }
-        float *dst = sm.red + rb * RS + 8 * cg;
-        *reinterpret_cast<float4 *>(dst) = f4_of(aN[0], aN[1]);
-        *reinterpret_cast<float4 *>(dst + 4) = f4_of(aN[2], aN[3]);
+        store_cols<FIT>(sm.red + rb * RS, cg, aN);
     }
     __syncthreads();
     // ---- column j = tid: refitted stored scale --------------------------------------------
     {
         const int j = tid;
-        const float N = sum4(sm.red + j, 2 * RS), Dn = sum4(sm.red + RS + j, 2 * RS);
+        const float N = sum4(sm.red + cpos<FIT>(j), 2 * RS), Dn = sum4(sm.red + RS + cpos<FIT>(j), 2 * RS);
         float cf = c_one;
         if (Dn > 0.f) {
             const float cn = round_scale(c_one * (N / Dn), sb16);
@@ -481,16 +508,16 @@ __device__ __forceinline__ bool refit_scales(const TileParams &p, SmemFixed &sm,
         }
         store_scale(gsc, D + j, cf, sb16);
         const float K = cf / c_one;
-        sm.colB[j] = K;
-        sm.colG1[j] = c_one * c_one * K;
+        sm.colB[cpos<FIT>(j)] = K;
+        sm.colG1[cpos<FIT>(j)] = c_one * c_one * K;
     }
     __syncthreads();
     // ---- row sums over this thread's 8 columns, then across the half-warp ---------------------
     float pn[16], pd[16];
     {
         float2 g[4], h[4];
-        load_pairs(sm.colG1 + 8 * cg, g);
-        load_pairs(sm.colB + 8 * cg, h);
+        load_cols<FIT>(sm.colG1, cg, g);
+        load_cols<FIT>(sm.colB, cg, h);
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp) h[pp] = __fmul2_rn(g[pp], h[pp]);  // c'^2 K~^2
         float2 cha[8], chb[8];
@@ -504,7 +531,7 @@ __device__ __forceinline__ bool refit_scales(const TileParams &p, SmemFixed &sm,
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const int m = 2 * k + r;
-                const float2 s2 = sm.rowS[8 * m + rb];
+                const float2 s2 = sm.rowS[rpos<FIT>(8 * m + rb)];
                 float2 n2 = make_float2(0.f, 0.f), d2 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int pp = 0; pp < 4; ++pp) {
@@ -549,7 +576,7 @@ __device__ __forceinline__ bool refit_scales(const TileParams &p, SmemFixed &sm,
             }
         }
         store_scale(gsc, i, rf, sb16);
-        sm.rowS[i] = make_float2(sf, sf);
+        sm.rowS[rpos<FIT>(i)] = make_float2(sf, sf);
     }
     __syncwarp();
     return true;
@@ -592,7 +619,7 @@ __device__ __forceinline__ void sweep_pack(uint8_t *gblock, const SmemFixed &sm,
     uint8_t *dstrow = gblock + rb * RB + cg * WB;
     float2 ik[4];  // 1 / K~_j of this thread's columns (refit only)
     if constexpr (FIT) {
-        load_pairs(sm.colB + 8 * cg, ik);
+        load_cols<FIT>(sm.colB, cg, ik);
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp) ik[pp] = make_float2(fast_rcp(ik[pp].x), fast_rcp(ik[pp].y));
     }
@@ -607,7 +634,7 @@ __device__ __forceinline__ void sweep_pack(uint8_t *gblock, const SmemFixed &sm,
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             const int m = 2 * k + r;
-            const float2 s2 = sm.rowS[8 * m + rb];
+            const float2 s2 = sm.rowS[rpos<FIT>(8 * m + rb)];
 #pragma unroll
             for (int pp = 0; pp < 4; ++pp) {
                 if constexpr (FIT) {
@@ -665,9 +692,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
                                            __shfl_xor_sync(0xffffffffu, send.y, 16));
             accU[pp] = __fadd2_rn(keep, got);
         }
-        float *dst = sm.red + rb * RS + 8 * cg;
-        *reinterpret_cast<float4 *>(dst) = f4_of(accU[0], accU[1]);
-        *reinterpret_cast<float4 *>(dst + 4) = f4_of(accU[2], accU[3]);
+        store_cols<FIT>(sm.red + rb * RS, cg, accU);
     }
     __syncthreads();  // B1: column partials complete
 
@@ -678,8 +703,8 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
     const float inv_sig = (j & 1) ? 1.f / W.sig1 : 1.f;  // powers of two: exact
     {
         // k~Q partials in the half-0 regions (0, 2, 4, 6), q~Q partials in the half-1 regions
-        const float U = sum4(sm.red + j, 2 * RS) * inv_sig;
-        const float P = sum4(sm.red + RS + j, 2 * RS) * inv_sig;
+        const float U = sum4(sm.red + cpos<FIT>(j), 2 * RS) * inv_sig;
+        const float P = sum4(sm.red + RS + cpos<FIT>(j), 2 * RS) * inv_sig;
         const float sig = (j & 1) ? W.sig1 : 1.f;
         const float beta = sm.scal[slot_i][0], alpha = sm.scal[slot_i][1];
         const float vj = load_in<IN_BF16>(tile + C::V_OFF, j);
@@ -689,12 +714,12 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
         float o;
         if (GATE == 1) {
             const float qak = sm.rsum[pb][0][2] + sm.rsum[pb][1][2] + sm.rsum[pb][2][2] + sm.rsum[pb][3][2];
-            sm.colG1[j] = sig * (beta * vj) * rc;
-            channel(smem).colG2[j] = sig * (beta * u) * rc;
+            sm.colG1[cpos<FIT>(j)] = sig * (beta * vj) * rc;
+            channel(smem).colG2[cpos<FIT>(j)] = sig * (beta * u) * rc;
             o = cj * P + (qk * beta * vj - qak * beta * u);
         } else {
             const float h = GATE == 0 ? beta * (vj - alpha * u) : beta * (vj - u);
-            sm.colG1[j] = sig * h * rc;
+            sm.colG1[cpos<FIT>(j)] = sig * h * rc;
             o = cj * P + qk * h;
         }
         p.o[(size_t)sm.meta[n & 3].orow * D + j] = o;
@@ -707,8 +732,8 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
     tmem_wait_st();
     {
         float2 g1[4], g2[4], accE[4];
-        load_pairs(sm.colG1 + 8 * cg, g1);
-        if (GATE == 1) load_pairs(channel(smem).colG2 + 8 * cg, g2);
+        load_cols<FIT>(sm.colG1, cg, g1);
+        if (GATE == 1) load_cols<FIT>(channel(smem).colG2, cg, g2);
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp) accE[pp] = make_float2(0.f, 0.f);
         bool bad = false;
@@ -765,11 +790,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
             for (int pp = 0; pp < 4; ++pp)
                 accE[pp] = __fadd2_rn(accE[pp], make_float2(__shfl_xor_sync(0xffffffffu, accE[pp].x, 16),
                                                             __shfl_xor_sync(0xffffffffu, accE[pp].y, 16)));
-            if (sub == 0) {
-                float *dst = sm.red + 2 * warp * RS + D + 8 * cg;
-                *reinterpret_cast<float4 *>(dst) = f4_of(accE[0], accE[1]);
-                *reinterpret_cast<float4 *>(dst + 4) = f4_of(accE[2], accE[3]);
-            }
+            if (sub == 0) store_cols<FIT>(sm.red + 2 * warp * RS + D, cg, accE);
         }
     }
     __syncthreads();  // B3: column energies complete
@@ -779,7 +800,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
     if (!pivot) {
         // x = sum_i w_i S'_ij^2 / (sum_i w_i c_j^2) (times sigma_j^2), so c'_j = c_j sqrt(x) / sigma_j
         // and the factor taking y to S'_ij / c'_j is 1 / sqrt(x)
-        const float E = sum4(sm.red + D + j, 2 * RS);
+        const float E = sum4(sm.red + D + cpos<FIT>(j), 2 * RS);
         const float wsum = sm.rsum[pb][0][0] + sm.rsum[pb][1][0] + sm.rsum[pb][2][0] + sm.rsum[pb][3][0];
         const float x = E * fast_rcp(wsum);
         float b = rsqrtf(x);
@@ -794,7 +815,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
         c_one = c;
         if (!FIT) store_scale(reinterpret_cast<uint8_t *>(sm.meta[n & 3].gblock + W.soff), D + j, c, sb16);
         if (!isfinite(c) || c == 0.f) flag(p.status, kFlagNonfinite);
-        sm.colB[j] = b;
+        sm.colB[cpos<FIT>(j)] = b;
     }
     const bool ok = precompute_rows<BITS, GATE, IN_BF16, FIT, SB16>(sm, smem, n + 1, my_count);
     if (__syncthreads_or(!ok)) return false;  // B4: new column scales and next row factors ready
@@ -804,7 +825,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
     tmem_wait_st();
     {
         float2 bb[4];
-        load_pairs(sm.colB + 8 * cg, bb);
+        load_cols<FIT>(sm.colB, cg, bb);
         float *rm = sm.red + rb * RS + cg;
         float2 cha[8], chb[8];
         tmem_ld16_async(tcol, cha);
@@ -847,7 +868,7 @@ __device__ __forceinline__ bool process_tile(const TileParams &p, SmemFixed &sm,
             r = round_scale(r, 1);
             s = (sm.rowRq[pb][i] * W.qmax) * fast_rcp(r);
         }
-        sm.rowS[i] = make_float2(s, s);
+        sm.rowS[rpos<FIT>(i)] = make_float2(s, s);
         if constexpr (FIT) {
             r_one = r;
             s_one = s;
