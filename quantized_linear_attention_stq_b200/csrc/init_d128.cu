@@ -426,20 +426,21 @@ cudaError_t launch_init_d128(const TileParams &p, cudaStream_t s)
     if (err != cudaSuccess) return err;
     const int grid = p.ntiles < sms ? p.ntiles : sms;
     if (grid <= 0) return cudaSuccess;
-    // S0 as rows of 128 floats, copied as boxes of 32 columns x 128 rows, 128-byte swizzle
+    // S0 as rows of 128 floats, copied as boxes of 32 columns x 128 rows, 128-byte swizzle. Where
+    // no tensor map can be made (no driver entry point, or more rows than 32-bit TMA coordinates
+    // reach) the plain kernel takes the tiles.
     const EncodeTiled enc = encode_tiled();
-    if (!enc) return cudaErrorNotSupported;
     const uint64_t rows = (uint64_t)p.B * (uint64_t)p.head_count * DI;
-    if (rows > 0x7fffffffull) return cudaErrorInvalidValue;  // TMA row coordinates are 32-bit
     CUtensorMap map;
     const cuuint64_t dims[2] = {(cuuint64_t)DI, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)DI * 4};
     const cuuint32_t box[2] = {32, (cuuint32_t)DI};
     const cuuint32_t estr[2] = {1, 1};
-    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(p.S0), dims, strides, box, estr,
+    if (!enc || rows > 0x7fffffffull ||
+        enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(p.S0), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
+        return launch_init_generic(p, s);
     init_d128_kernel<<<grid, NTI, SMEM_INIT, s>>>(p, map);
     return cudaGetLastError();
 }
