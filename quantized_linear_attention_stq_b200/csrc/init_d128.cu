@@ -4,8 +4,9 @@
 // named barrier, so that one group's barrier waits overlap the other group's work. Whole fp32
 // tiles stream through a three-slot shared-memory ring: the two groups' tiles and the next one in
 // flight. A tile arrives by four TMA tensor copies (32-column quarters, 128-byte swizzle: the
-// 16-byte chunk c of row i of a quarter sits at chunk c ^ (i % 8)) and is read in place: every pass
-// then reads 32 distinct banks per 8-lane phase without a padded copy.
+// 16-byte chunk c of row i of a quarter sits at chunk c ^ (i % 8)) and is read in place: each pass
+// maps its lanes so that the 8 lanes of a 16-byte load phase of the tile hit 8 bank quads, with
+// no padded copy.
 //
 // Method: the column scale is the impact-weighted RMS of the column over the key rows, the row
 // scale the largest column-normalised magnitude of the row over qmax, the codes S / (r c) rounded
