@@ -367,6 +367,61 @@ __global__ void __launch_bounds__(kThreads) init_kernel(const __grid_constant__ 
 // ------------------------------------------------------------------------------------------
 // Dequantization: pool -> S_out fp32 [B][H][dk][dv]
 // ------------------------------------------------------------------------------------------
+// Row x column codes of width BITS (scales bf16 if SB16), 8 consecutive elements of a row per
+// thread: the group's BITS * 8 code bits are BITS bytes at byte offset BITS * g, unpacked at once,
+// and the 8 column scales are one or two 16-byte loads (8 | d_v, and the scales start on a 16-byte
+// boundary); S_ij = fp32(r_i c_j) Q_ij.
+template <int BITS, int SB16>
+__device__ __forceinline__ void dequant_rc(const uint8_t *block, const uint8_t *sc, int dk, int dv, float *dst)
+{
+    constexpr int off = 1 << (BITS - 1);
+    constexpr uint32_t mask = (1u << BITS) - 1u;
+    const int shv = __ffs(dv) - 1;
+    for (int g = threadIdx.x; g < dk * dv / 8; g += blockDim.x) {
+        const int e0 = 8 * g, i = e0 >> shv, j0 = e0 & (dv - 1);
+        uint32_t lo, hi;
+        if constexpr (BITS == 8) {
+            const uint2 wd = *reinterpret_cast<const uint2 *>(block + 8 * g);
+            lo = wd.x;
+            hi = wd.y;
+        } else if constexpr (BITS == 4) {
+            lo = *reinterpret_cast<const uint32_t *>(block + 4 * g);
+            hi = 0u;
+        } else {  // 6 bytes at 6g, 2-byte aligned
+            const uint16_t *h = reinterpret_cast<const uint16_t *>(block + 6 * g);
+            lo = (uint32_t)h[0] | ((uint32_t)h[1] << 16);
+            hi = h[2];
+        }
+        const float r = load_scale(sc, i, SB16);
+        float c[8];
+        if constexpr (SB16) {
+            const uint4 cw = *reinterpret_cast<const uint4 *>(sc + 2 * (dk + j0));
+            const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                c[2 * k] = __uint_as_float(w4[k] << 16);              // bf16 -> fp32: the high half of the word
+                c[2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u);
+            }
+        } else {
+            const float4 a = *reinterpret_cast<const float4 *>(sc + 4 * (dk + j0));
+            const float4 b = *reinterpret_cast<const float4 *>(sc + 4 * (dk + j0) + 16);
+            c[0] = a.x; c[1] = a.y; c[2] = a.z; c[3] = a.w;
+            c[4] = b.x; c[5] = b.y; c[6] = b.z; c[7] = b.w;
+        }
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int bit = BITS * k;  // position in the 64-bit (hi:lo) group
+            const uint32_t u = (bit < 32 ? (bit + BITS <= 32 ? lo >> bit : __funnelshift_r(lo, hi, bit))
+                                         : hi >> (bit - 32)) & mask;
+            v[k] = (r * c[k]) * (float)((int)u - off);
+        }
+        float4 *o4 = reinterpret_cast<float4 *>(dst + e0);
+        o4[0] = make_float4(v[0], v[1], v[2], v[3]);
+        o4[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads) dequant_kernel(const __grid_constant__ TileParams p)
 {
     const int b = blockIdx.x, pos = blockIdx.y;
@@ -381,38 +436,14 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const __grid_constant
         dequant_to_smem(t.block, t.bits, t.uniform, t.sb16, dk, dv, dst, dv);  // straight to global, row stride dv
         return;
     }
-    // row x column codes, 8 consecutive elements of a row per thread: the group's bits * 8 code
-    // bits are `bits` bytes at byte offset bits * g, unpacked at once; S_ij = fp32(r_i c_j) Q_ij
     const uint8_t *sc = t.block + scale_offset(t.bits, dk, dv);
-    const int shv = __ffs(dv) - 1, bits = t.bits, off = 1 << (bits - 1);
-    const uint32_t mask = (1u << bits) - 1u;
-    for (int g = threadIdx.x; g < dk * dv / 8; g += blockDim.x) {
-        const int e0 = 8 * g, i = e0 >> shv, j0 = e0 & (dv - 1);
-        uint32_t lo, hi;
-        if (bits == 8) {
-            const uint2 wd = *reinterpret_cast<const uint2 *>(t.block + 8 * g);
-            lo = wd.x;
-            hi = wd.y;
-        } else if (bits == 4) {
-            lo = *reinterpret_cast<const uint32_t *>(t.block + 4 * g);
-            hi = 0u;
-        } else {  // 6 bytes at 6g, 2-byte aligned
-            const uint16_t *h = reinterpret_cast<const uint16_t *>(t.block + 6 * g);
-            lo = (uint32_t)h[0] | ((uint32_t)h[1] << 16);
-            hi = h[2];
-        }
-        const float r = load_scale(sc, i, t.sb16);
-        float v[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int bit = bits * k;  // position in the 64-bit (hi:lo) group
-            const uint32_t u = (bit < 32 ? (bit + bits <= 32 ? lo >> bit : __funnelshift_r(lo, hi, bit))
-                                         : hi >> (bit - 32)) & mask;
-            v[k] = (r * load_scale(sc, dk + j0 + k, t.sb16)) * (float)((int)u - off);
-        }
-        float4 *o4 = reinterpret_cast<float4 *>(dst + e0);
-        o4[0] = make_float4(v[0], v[1], v[2], v[3]);
-        o4[1] = make_float4(v[4], v[5], v[6], v[7]);
+    switch (2 * t.bits + t.sb16) {
+    case 8: dequant_rc<4, 0>(t.block, sc, dk, dv, dst); break;
+    case 9: dequant_rc<4, 1>(t.block, sc, dk, dv, dst); break;
+    case 12: dequant_rc<6, 0>(t.block, sc, dk, dv, dst); break;
+    case 13: dequant_rc<6, 1>(t.block, sc, dk, dv, dst); break;
+    case 16: dequant_rc<8, 0>(t.block, sc, dk, dv, dst); break;
+    default: dequant_rc<8, 1>(t.block, sc, dk, dv, dst); break;
     }
 }
 
