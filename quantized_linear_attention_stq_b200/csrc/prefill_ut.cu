@@ -1022,8 +1022,12 @@ __global__ void __launch_bounds__(NT3, 2) ut_state_pivot_kernel(const __grid_con
 constexpr uint32_t P3_QC = 0;       // chunk-start codes, bf16 (A operand of D_a, MN-major)
 constexpr uint32_t P3_X = 32768;    // U^T terms (2 x 16 KB) and P terms (2 x 8 KB); then (q r) terms (3 x 16 KB)
 constexpr uint32_t P3_SMALL = 81920;
-constexpr uint32_t P3S_R = 0, P3S_C = 512, P3S_GAM = 1024, P3S_BAR = 1280, P3S_MISC = 1296;
-constexpr uint32_t P3_SMEM = P3_SMALL + 1312 + 1024;
+// r is kept as four 32-float parts at a 36-float stride (RPS): the parts that a warp's lanes read
+// at once sit on different banks
+constexpr int RPS = 36;
+constexpr uint32_t P3S_R = 0, P3S_C = 4 * RPS * 4, P3S_GAM = P3S_C + 512, P3S_BAR = P3S_GAM + 256,
+                   P3S_MISC = P3S_BAR + 16;
+constexpr uint32_t P3_SMEM = P3_SMALL + P3S_MISC + 16 + 1024;
 constexpr int OST = 132;  // row stride (floats) of the readout staged over the term area
 static_assert(64 * OST * 4 <= 49152, "readout rows fit the term area");
 
@@ -1081,7 +1085,10 @@ __device__ __forceinline__ void readout_run(const TileParams &p, const UtArgs &a
             cp_async16(smem_u32(X + 32768 + 16 * e), rec + REC_PT + 16 * e, 16u);
         }
         if (tid < 64) {
-            if (!pivot) cp_async16(smem_u32(reinterpret_cast<uint8_t *>(sR) + 16 * tid), rec + REC_SC + 16 * tid, 16u);
+            // r (chunks 0..31: part tid / 8 of the padded parts) and c (chunks 32..63)
+            uint8_t *dst = tid < 32 ? reinterpret_cast<uint8_t *>(sR) + 4 * RPS * (tid >> 3) + 16 * (tid & 7)
+                                    : reinterpret_cast<uint8_t *>(sC) + 16 * (tid - 32);
+            if (!pivot) cp_async16(smem_u32(dst), rec + REC_SC + 16 * tid, 16u);
         } else if (tid < 80) {
             cp_async16(smem_u32(reinterpret_cast<uint8_t *>(sGam) + 16 * (tid - 64)), rec + REC_G + 16 * (tid - 64), 16u);
         }
@@ -1144,13 +1151,15 @@ __device__ __forceinline__ void readout_run(const TileParams &p, const UtArgs &a
             }
         } else {
             uint8_t *box = X + (part >> 1) * 8192;
-            const float *rr = sR + 32 * part;
+            const float *rr = sR + RPS * part;  // r_i, i = 32 part + m, at m
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 float x[8];
                 bf16x8_to_f32(qraw[k], x);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] *= rr[8 * k + e];
+                const float4 r0 = *reinterpret_cast<const float4 *>(rr + 8 * k);
+                const float4 r1 = *reinterpret_cast<const float4 *>(rr + 8 * k + 4);
+                x[0] *= r0.x; x[1] *= r0.y; x[2] *= r0.z; x[3] *= r0.w;
+                x[4] *= r1.x; x[5] *= r1.y; x[6] *= r1.z; x[7] *= r1.w;
                 store_split3(box, box + 16384, box + 32768, sw128_chunk(t, 4 * (part & 1) + k), x);
             }
         }
