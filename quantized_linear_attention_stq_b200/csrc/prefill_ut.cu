@@ -290,7 +290,9 @@ __device__ __forceinline__ void inputs_run(const TileParams &p, const UtArgs &a,
         // ---- T' = T diag(beta) and T'' = T diag(beta gamma), three bf16 terms each ----------
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
-            const int unit = tid + NT3 * k, t = unit >> 3, c8 = unit & 7;
+            // the 8 lanes of a load phase take one unit c8 of 8 rows: 8 bank quads on Tm (row
+            // stride 68 floats), one broadcast address on beta and gamma
+            const int unit = tid + NT3 * k, t = (unit & 7) + 8 * (unit >> 6), c8 = (unit >> 3) & 7;
             float x[8], y[8];
             const float4 xa = *reinterpret_cast<const float4 *>(Tm + t * LDL + 8 * c8);
             const float4 xb = *reinterpret_cast<const float4 *>(Tm + t * LDL + 8 * c8 + 4);
@@ -503,8 +505,9 @@ __global__ void __launch_bounds__(NT3, 2) ut_state_kernel(const __grid_constant_
             // ---- B operand of D2: three bf16 terms of (W r) [t][i] ----------------------------
             {
                 // thread (t, part): 8-float units c8 = part + 4 k of row t, read before any term is
-                // written over the staged rows
-                const int t = tid >> 2, part = tid & 3;
+                // written over the staged rows; the 8 lanes of a phase take one unit of 8 rows (8
+                // bank quads on the 132-float rows and in the swizzled boxes, one address of r)
+                const int t = (tid & 7) + 8 * (tid >> 5), part = (tid >> 3) & 3;
                 float x[4][8];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
@@ -857,7 +860,8 @@ __global__ void __launch_bounds__(NT3, 2) ut_state_pivot_kernel(const __grid_con
             // ---- B operand of D2: W [t][i] times 2^-e, three fp16 terms ------------------------
             int e2;
             {
-                const int t = tid >> 2, part = tid & 3;
+                // the 8 lanes of a phase take one unit of 8 rows, as in the coded kernel
+                const int t = (tid & 7) + 8 * (tid >> 5), part = (tid >> 3) & 3;
                 float x[4][8];
                 float mx = 0.f;
 #pragma unroll
@@ -1093,8 +1097,9 @@ __device__ __forceinline__ void readout_run(const TileParams &p, const UtArgs &a
             cp_async16(smem_u32(reinterpret_cast<uint8_t *>(sGam) + 16 * (tid - 64)), rec + REC_G + 16 * (tid - 64), 16u);
         }
         cp_async_commit();
-        // q row t, columns 32 part .. +31, in registers for the (q r) terms
-        const int t = tid >> 2, part = tid & 3;
+        // q row t, columns 32 part .. +31, in registers for the (q r) terms; the 8 lanes of a
+        // phase take one part of 8 rows, so that their term stores fall in 8 bank quads
+        const int t = (tid & 7) + 8 * (tid >> 5), part = (tid >> 3) & 3;
         uint4 qraw[4];
         {
             const uint4 *qs = reinterpret_cast<const uint4 *>(qg + (size_t)(t < Lc ? t : 0) * D + 32 * part);
