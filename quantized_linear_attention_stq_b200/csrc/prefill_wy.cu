@@ -275,7 +275,10 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
             if (warp < INV_WARP0) {
                 // ---- warps 0..11: A operand of D2, three bf16 terms of [K r; Q r] ------------
                 for (int unit = tid; unit < 4 * D; unit += 32 * INV_WARP0) {
-                    const int m = unit >> 2, part = unit & 3, row = m & 63, hb = part >> 1;
+                    // the 8 lanes of a load phase take one part of 8 rows: one address of r, and 8
+                    // bank quads in the swizzled K / Q boxes and term tiles
+                    const int m = (unit & 7) + 8 * (unit >> 5), part = (unit >> 3) & 3, row = m & 63,
+                              hb = part >> 1;
                     const uint8_t *xb = sm + kq + (m < 64 ? (hb ? KQ_K1 : KQ_K0) : (hb ? KQ_Q1 : KQ_Q0));
                     uint8_t *a0 = big + hb * 16384, *a1 = a0 + 32768, *a2 = a0 + 65536;
                     const float *rr = sR + 32 * part;
@@ -316,7 +319,9 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const __grid_constant
                 // its three bf16 terms, one 8-column unit of one row per thread (all 16 warps)
                 static_assert(NT == 64 * 8, "one T unit per thread");
                 uint8_t *r0 = sm + OFF_RT;
-                const int t = tid >> 3, c8 = tid & 7;
+                // the 8 lanes of a load phase take one unit of 8 rows: 8 bank quads on Tm (row
+                // stride 68 floats) and in the swizzled term tiles
+                const int t = (tid & 7) + 8 * (tid >> 6), c8 = (tid >> 3) & 7;
                 float x[8];
                 const float4 xa = *reinterpret_cast<const float4 *>(Tm + t * LDL + 8 * c8);
                 const float4 xb4 = *reinterpret_cast<const float4 *>(Tm + t * LDL + 8 * c8 + 4);
