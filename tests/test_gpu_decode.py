@@ -9,7 +9,8 @@ import numpy as np
 import pytest
 import torch
 
-from _parity import Tally, as_f64, compare_block, compare_o, oracle_pool, tile_bytes, update_magnitude
+from _parity import (Tally, as_f64, compare_block, compare_block_bf16s, compare_o, oracle_pool, tile_bytes,
+                     update_magnitude)
 
 pytestmark = pytest.mark.gpu
 
@@ -362,6 +363,56 @@ def test_init_out_of_range_slots_flagged_others_written(stq, orc):
             compare_block(orc, bits[h], 128, tile_bytes(orc, gp, bits, 128, 1, h), tile_bytes(orc, ref, bits, 128, 0, h),
                           tie, tally, f"init slot 1 head {h} aligned={aligned}")
         tally.check_budget()
+
+
+@pytest.mark.parametrize("scale_dtype", [torch.float32, torch.bfloat16])
+def test_init_several_tiles_per_cta_with_skipped_requests(stq, orc, scale_dtype):
+    """Init with several tiles per CTA of the streaming kernel (40 requests x 14 row x column heads
+    = 560 tiles over at most 148 CTAs: both groups of a CTA take tiles, and the three ring slots
+    are each reused), mixed widths, and every seventh request on an out-of-range slot. The skipped
+    requests are flagged and leave the pool untouched; every written tile matches the oracle."""
+    from quantized_linear_attention_stq_b200 import workloads as wlm
+
+    B = 40
+    bits = [4, 6, 8, 16, 8, 6, 4, 4, 6, 8, 6, 4, 8, 16, 6, 4]
+    wl_ = _wl("full2304_b70_mixed", batch=B, heads=len(bits), outliers=False)
+    H, d = len(bits), 128
+    lay = stq.Layout(bits, d, scale_dtype=scale_dtype)
+    w = wlm.impact_weights(wl_)
+    S0 = torch.stack([wlm.initial_state(wl_, r) for r in range(B)])
+    total = lay.bytes_per_request
+    pool = lay.alloc_pool(B + 1)
+    pool.fill_(7)
+    slot_of = [-1 if r % 7 == 3 else r + 1 for r in range(B)]  # slot 0 belongs to no request
+    slots = torch.tensor(slot_of, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    S_dev = S0.to(DEV)
+    assert S_dev.data_ptr() % 16 == 0
+    stq.init_state(lay, pool, slots, S_dev, w.to(DEV), status=status)
+    torch.cuda.synchronize()
+    assert status.item() & (1 << stq.api.STQ_ERR_BOUNDS)
+    assert status.item() & ~(1 << stq.api.STQ_ERR_BOUNDS) == 0, stq.status_flags(status)
+    gp = pool.cpu().numpy()
+    assert np.all(gp[:total] == 7), "slot 0 belongs to no request and stays untouched"
+    written = [r for r in range(B) if slot_of[r] >= 0]
+    assert sorted(slot_of[r] for r in written) == [r + 1 for r in written]
+    for r in range(B):
+        if slot_of[r] < 0:
+            assert np.all(gp[(r + 1) * total:(r + 2) * total] == 7), f"skipped request {r}'s slot was written"
+    sb16 = scale_dtype == torch.bfloat16
+    tally = Tally()
+    for r in written:
+        for h in range(H):
+            base = slot_of[r] * total + lay.head_offset(h)
+            got = gp[base: base + lay.head_bytes(h)]
+            if sb16 and bits[h] != 16:
+                compare_block_bf16s(orc, bits[h], d, got, as_f64(S0[r, h]), as_f64(w[h]), tally,
+                                    f"init req {r} head {h}")
+            else:
+                blk, _, tie, st = orc.quantize(bits[h], as_f64(S0[r, h]), as_f64(w[h]))
+                assert st == orc.OK
+                compare_block(orc, bits[h], d, got[:blk.size], blk, tie, tally, f"init req {r} head {h}")
+    tally.check_budget()
 
 
 def test_init_nonfinite_state_is_flagged(stq, orc):
