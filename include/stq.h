@@ -140,8 +140,9 @@ int32_t stq_layout_head_bits(const stq_layout *layout, int32_t head);
  * applied to S0 (or the fp16 conversion for pivot heads).
  *   pool        device, >= pool_slots * bytes_per_request bytes, 128-byte aligned
  *   slots       device int32 [B], the pool slot of each request
- *   S0          device fp32 [B][H][d_k][d_v], row-major, 4-byte aligned (a 16-byte aligned S0
- *               is read with 16-byte loads)
+ *   S0          device fp32 [B][H][d_k][d_v], row-major, 4-byte aligned (with a 16-byte aligned
+ *               S0 and w, 128 x 128 row x column heads stream through TMA tensor copies; else
+ *               4-byte loads)
  *   w           device fp32 [H][d_k], impact weights, finite and > 0
  * B == 0 is a no-op. */
 stq_status stq_init_state(const stq_layout *layout, void *pool, int32_t pool_slots,
