@@ -400,16 +400,15 @@ using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t,
 
 EncodeTiled encode_tiled()
 {
-    static EncodeTiled fn = nullptr;
-    static bool looked = false;
-    if (!looked) {
+    // a function-local static: initialised once, safely across host threads
+    static const EncodeTiled fn = []() -> EncodeTiled {
         void *f = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiled>(f);
-        looked = true;
-    }
+            return reinterpret_cast<EncodeTiled>(f);
+        return nullptr;
+    }();
     return fn;
 }
 
