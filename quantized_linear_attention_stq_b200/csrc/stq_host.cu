@@ -390,8 +390,8 @@ stq_status stq_decode_step(const stq_layout *L, void *pool, int32_t pool_slots, 
         if (!launch(plan->pivots, 0, (int)plan->pivots.size(), 16)) return STQ_ERR_CUDA;
         return STQ_OK;
     }
-    auto p = new_params();
-    if (!p) return STQ_ERR_INVALID_ARG;
+    // the plain kernel: the same per-thread parameter block (the table entries are filled below)
+    stq::TileParams *p = &thread_params();
     p->pool = static_cast<uint8_t *>(pool);
     p->status = dev_status;
     p->req_bytes = L->req_bytes;
