@@ -127,6 +127,15 @@ def profiled_traffic():
         return None
 
 
+def step_traffic(args):
+    """The committed capture's DRAM bytes per step, for the step it was taken on (the default
+    workload at its own batch, fp32 scales, the one-pass fit) and the current decode source; None
+    for any other configuration."""
+    if args.workload != DEFAULT_WORKLOAD or args.batch or args.scale_dtype != "f32" or args.fit_rounds != 0:
+        return None
+    return profiled_traffic()
+
+
 # fp32 lane operations on the FMA pipe that one state element needs in this formulation of the
 # decode step: code unpack 1, the k and q column sums 2, the update 2, the column energy 1, the
 # column rescale 1, the rounding 1 (FP16 pivots: column sums 2, update 2)
@@ -759,11 +768,7 @@ def run_ours(args):
         "step_ms_median": statistics.median(per_step),
         "step_ms_min": min(per_step),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": peak_kind,
-                     # the committed capture is of the default step (batch 70, fp32 scales, one pass)
-                     "traffic": profiled_traffic() if (args.workload == DEFAULT_WORKLOAD and not args.batch
-                                                        and args.scale_dtype == "f32" and args.fit_rounds == 0)
-                     else None,
+                     "peak_kind": peak_kind, "traffic": step_traffic(args),
                      "bytes_per_step": state_bytes, "launches_per_step": launches_per_step,
                      "kernel": ("decode_d128_kernel<width> (pivots, then one launch per width)" if per_width
                                 else "decode_d128_kernel<width> (pivots, then one launch for all widths)"),

@@ -81,3 +81,16 @@ def test_reference_arm_other_ranks_exit_without_output():
                           timeout=120)
     assert proc.returncode == 0, proc.stderr
     assert proc.stdout.strip() == ""
+
+
+def test_step_traffic_only_for_the_profiled_step():
+    """The bench line carries the committed DRAM capture only for the configuration it was taken
+    on (and only while the decode source is the captured one)."""
+    import argparse
+
+    import bench
+
+    base = dict(workload=bench.DEFAULT_WORKLOAD, batch=0, scale_dtype="f32", fit_rounds=0)
+    assert bench.step_traffic(argparse.Namespace(**base)) == bench.profiled_traffic()
+    for change in (dict(batch=32), dict(scale_dtype="bf16"), dict(fit_rounds=1), dict(workload="layer48_b8_4bit")):
+        assert bench.step_traffic(argparse.Namespace(**{**base, **change})) is None, change
